@@ -1,0 +1,199 @@
+"""fp64 CPU oracle for the Mamba selective-SSM scan and decode state update.
+
+TEST INFRASTRUCTURE. Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package. The product path
+(``selective_state_space_39_b200``) never imports it, and this package never
+imports the product: the two share no code. The only shared module is the
+seeded input generator ``ssm_inputs``, which holds none of the method's
+arithmetic.
+
+The arithmetic lives in ``ssm_oracle.c`` (plain sequential fp64 loops). This
+module compiles it with gcc on first use and marshals numpy arrays to it.
+What it computes follows the page "Mamba 논문 리뷰: Selective State Space
+Models로 Transformer를 넘어서" (youngju.dev): §2.2 discretised recurrence,
+§3.1 softplus step size, §3.3 simplified ``selective_scan``, §3.4 block gate
+and D skip. Every function here is pinned by ``tests/test_oracle_pins.py``
+against closed forms, brute force and invariants.
+
+bf16 arrays are passed as numpy ``uint16`` holding the raw bf16 bits with
+``io="bf16"``; fp32 arrays as ``float32`` with ``io="f32"``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+SOURCE = os.path.join(_HERE, "ssm_oracle.c")
+_BUILD_DIR = os.path.join(_HERE, "_build")
+LIB_PATH = os.path.join(_BUILD_DIR, "liboracle.so")
+_lock = threading.Lock()
+
+
+def compile_library(source: str = SOURCE, out_path: str = LIB_PATH) -> str:
+    """Compile the oracle C source into a shared library with gcc (-O2, no
+    fast-math, so fp64 semantics are IEEE)."""
+    os.makedirs(os.path.dirname(out_path), exist_ok=True)
+    tmp = out_path + ".tmp.%d" % os.getpid()
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math",
+           "-ffp-contract=off", "-o", tmp, source, "-lm", "-lpthread"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, out_path)
+    return out_path
+
+
+def _needs_build(src: str, lib: str) -> bool:
+    return not os.path.exists(lib) or os.path.getmtime(lib) < os.path.getmtime(src)
+
+
+_F32P = ctypes.POINTER(ctypes.c_float)
+_F64P = ctypes.POINTER(ctypes.c_double)
+_I64P = ctypes.POINTER(ctypes.c_int64)
+
+
+class Oracle:
+    """Handle on one compiled oracle library (the default one, or a test's
+    deliberately mutated copy)."""
+
+    def __init__(self, lib_path: str):
+        self.lib = ctypes.CDLL(lib_path)
+        f = self.lib.oracle_selective_scan
+        f.restype = ctypes.c_int
+        f.argtypes = [ctypes.c_int64] * 4 + [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+                      _F32P, ctypes.c_void_p, ctypes.c_void_p, _F32P, ctypes.c_void_p,
+                      _F32P, ctypes.c_int, _F32P, _I64P, ctypes.c_int64, _F64P, _F64P,
+                      ctypes.c_int]
+        g = self.lib.oracle_state_update
+        g.restype = ctypes.c_int
+        g.argtypes = [ctypes.c_int64] * 3 + [ctypes.c_int, _F64P, ctypes.c_void_p,
+                      ctypes.c_void_p, _F32P, ctypes.c_void_p, ctypes.c_void_p, _F32P,
+                      ctypes.c_void_p, _F32P, ctypes.c_int, _F64P]
+
+    # -- helpers -----------------------------------------------------------
+    @staticmethod
+    def _io_array(a, io, shape, name, optional=False):
+        if a is None:
+            if optional:
+                return None
+            raise ValueError(f"{name} is required")
+        want = np.uint16 if io == "bf16" else np.float32
+        a = np.ascontiguousarray(a)
+        if a.dtype != want:
+            raise TypeError(f"{name}: expected {want} for io={io}, got {a.dtype}")
+        if tuple(a.shape) != tuple(shape):
+            raise ValueError(f"{name}: expected shape {shape}, got {a.shape}")
+        return a
+
+    @staticmethod
+    def _f32_array(a, shape, name, optional=True):
+        if a is None:
+            if optional:
+                return None
+            raise ValueError(f"{name} is required")
+        a = np.ascontiguousarray(a, dtype=np.float32)
+        if tuple(a.shape) != tuple(shape):
+            raise ValueError(f"{name}: expected shape {shape}, got {a.shape}")
+        return a
+
+    @staticmethod
+    def _ptr(a, ctype=None):
+        if a is None:
+            return None
+        if ctype is None:
+            return ctypes.c_void_p(a.ctypes.data)
+        return a.ctypes.data_as(ctypes.POINTER(ctype))
+
+    # -- the scan ----------------------------------------------------------
+    def selective_scan(self, x, delta, A, B, C, D=None, z=None, delta_bias=None,
+                       softplus=True, h0=None, io="f32", channels=None, nthreads=1):
+        """Selective scan over all channels, or over ``channels`` (a list of
+        (b, d) pairs). Returns ``(y, h_last)`` in fp64: for all channels
+        y is (batch, L, dim) and h_last (batch, dim, N); for a channel list
+        y is (nchan, L) and h_last (nchan, N)."""
+        x = np.asarray(x)
+        batch, L, dim = x.shape
+        N = np.asarray(A).shape[1]
+        x = self._io_array(x, io, (batch, L, dim), "x")
+        delta = self._io_array(delta, io, (batch, L, dim), "delta")
+        B = self._io_array(B, io, (batch, L, N), "B")
+        C = self._io_array(C, io, (batch, L, N), "C")
+        z = self._io_array(z, io, (batch, L, dim), "z", optional=True)
+        A = self._f32_array(A, (dim, N), "A", optional=False)
+        D = self._f32_array(D, (dim,), "D")
+        delta_bias = self._f32_array(delta_bias, (dim,), "delta_bias")
+        h0 = self._f32_array(h0, (batch, dim, N), "h0")
+        full = channels is None
+        if full:
+            bb, dd = np.meshgrid(np.arange(batch), np.arange(dim), indexing="ij")
+            chans = np.stack([bb.ravel(), dd.ravel()], axis=1).astype(np.int64)
+        else:
+            chans = np.ascontiguousarray(np.asarray(channels, dtype=np.int64).reshape(-1, 2))
+        nchan = chans.shape[0]
+        y = np.empty((nchan, L), dtype=np.float64)
+        h_last = np.empty((nchan, N), dtype=np.float64)
+        rc = self.lib.oracle_selective_scan(
+            batch, L, dim, N, 1 if io == "bf16" else 0, self._ptr(x), self._ptr(delta),
+            self._ptr(A, ctypes.c_float), self._ptr(B), self._ptr(C),
+            self._ptr(D, ctypes.c_float), self._ptr(z), self._ptr(delta_bias, ctypes.c_float),
+            1 if softplus else 0, self._ptr(h0, ctypes.c_float),
+            self._ptr(chans, ctypes.c_int64), nchan, self._ptr(y, ctypes.c_double),
+            self._ptr(h_last, ctypes.c_double), int(nthreads))
+        if rc != 0:
+            raise ValueError("oracle_selective_scan rejected its arguments")
+        if full:
+            y = y.reshape(batch, dim, L).transpose(0, 2, 1).copy()
+            h_last = h_last.reshape(batch, dim, N)
+        return y, h_last
+
+    # -- decode ------------------------------------------------------------
+    def state_update(self, state, x, delta, A, B, C, D=None, z=None, delta_bias=None,
+                     softplus=True, io="f32"):
+        """One decode step on the fp64 ``state`` (batch, dim, N), in place.
+        Returns y (batch, dim) in fp64."""
+        if state.dtype != np.float64 or not state.flags.c_contiguous:
+            raise TypeError("state must be a C-contiguous float64 array")
+        batch, dim, N = state.shape
+        x = self._io_array(x, io, (batch, dim), "x")
+        delta = self._io_array(delta, io, (batch, dim), "delta")
+        B = self._io_array(B, io, (batch, N), "B")
+        C = self._io_array(C, io, (batch, N), "C")
+        z = self._io_array(z, io, (batch, dim), "z", optional=True)
+        A = self._f32_array(A, (dim, N), "A", optional=False)
+        D = self._f32_array(D, (dim,), "D")
+        delta_bias = self._f32_array(delta_bias, (dim,), "delta_bias")
+        y = np.empty((batch, dim), dtype=np.float64)
+        rc = self.lib.oracle_state_update(
+            batch, dim, N, 1 if io == "bf16" else 0, self._ptr(state, ctypes.c_double),
+            self._ptr(x), self._ptr(delta), self._ptr(A, ctypes.c_float), self._ptr(B),
+            self._ptr(C), self._ptr(D, ctypes.c_float), self._ptr(z),
+            self._ptr(delta_bias, ctypes.c_float), 1 if softplus else 0,
+            self._ptr(y, ctypes.c_double))
+        if rc != 0:
+            raise ValueError("oracle_state_update rejected its arguments")
+        return y
+
+
+_default = None
+
+
+def get() -> Oracle:
+    """The oracle built from ``ssm_oracle.c`` (compiled on first use)."""
+    global _default
+    with _lock:
+        if _default is None:
+            if _needs_build(SOURCE, LIB_PATH):
+                compile_library()
+            _default = Oracle(LIB_PATH)
+        return _default
+
+
+def selective_scan(*args, **kwargs):
+    return get().selective_scan(*args, **kwargs)
+
+
+def state_update(*args, **kwargs):
+    return get().state_update(*args, **kwargs)

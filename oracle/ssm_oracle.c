@@ -1,0 +1,206 @@
+/*
+ * ssm_oracle.c -- plain, slow, sequential fp64 CPU oracle for the Mamba
+ * selective state-space scan and its single-token state update.
+ *
+ * TEST INFRASTRUCTURE. Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg load this library. The product (the CUDA
+ * library and its Python binding) never calls it and shares no code with it.
+ *
+ * What it computes, per batch b and channel d, with state h[n], n < N:
+ *
+ *   v      = delta[b,t,d] + bias[d]                 (bias: the dt projection's
+ *                                                    bias, Mamba block, §3.4)
+ *   Delta  = softplus(v) if softplus else v          (selection mechanism,
+ *                                                    §3.1: Delta_t = softplus(.))
+ *   h[n]   = exp(Delta * A[d,n]) * h[n]
+ *            + Delta * B[b,t,n] * x[b,t,d]           (discretised recurrence,
+ *                                                    §2.2, with the simplified
+ *                                                    deltaB = Delta*B of the
+ *                                                    §3.3 selective_scan)
+ *   y      = sum_n C[b,t,n] * h[n] + D[d] * x[b,t,d] (readout, §2.2 y_t = C h_t,
+ *                                                    plus the block's D skip)
+ *   y     *= z / (1 + exp(-z))   if z is given       (block gate y * SiLU(z), §3.4)
+ *
+ * with h = h0[b,d,:] (or 0) before t = 0 and h_last[b,d,:] = h after t = L-1.
+ * Section numbers refer to the page "Mamba 논문 리뷰: Selective State Space
+ * Models로 Transformer를 넘어서" (youngju.dev): §2.2 Zero-Order Hold
+ * discretisation, §3.1 Selection Mechanism, §3.3 Hardware-Aware algorithm
+ * (the simplified selective_scan), §3.4 Mamba Block.
+ *
+ * Readings where the pages are silent or inconsistent (each also listed in
+ * the design notes):
+ *   - B-bar: the simplified Delta*B of the §3.3 scan, not the exact ZOH form
+ *     of §2.2.
+ *   - softplus(v) = log1p(exp(v)) for v <= 20 and v itself above 20.
+ *   - The skip term D*x is added before the gate: y = (C.h + D x) * SiLU(z).
+ *   - y_t reads the state after x_t has entered it.
+ *
+ * Inputs are read in their storage type (bf16 or fp32) and widened exactly
+ * to double; every operation after that is fp64.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_MAX_N 1024
+
+/* Widen element i of an input tensor to double. bf16 is the upper half of an
+ * IEEE binary32, so shifting it into place is exact. */
+static double widen(const void* p, int64_t i, int is_bf16) {
+  if (is_bf16) {
+    uint32_t w = (uint32_t)((const uint16_t*)p)[i] << 16;
+    float f;
+    memcpy(&f, &w, sizeof f);
+    return (double)f;
+  }
+  return (double)((const float*)p)[i];
+}
+
+/* softplus(v) = log(1 + e^v) (§3.1); the identity above 20, where the
+ * difference is below 2.1e-9 relative. */
+static double softplus(double v) { return v > 20.0 ? v : log1p(exp(v)); }
+
+/* SiLU(z) = z * sigmoid(z) (§3.4 gate). */
+static double silu(double z) { return z / (1.0 + exp(-z)); }
+
+typedef struct {
+  int64_t batch, seqlen, dim, dstate;
+  int is_bf16;
+  const void* x;       /* (batch, seqlen, dim)    io type */
+  const void* delta;   /* (batch, seqlen, dim)    io type */
+  const float* A;      /* (dim, dstate)           fp32    */
+  const void* B;       /* (batch, seqlen, dstate) io type */
+  const void* C;       /* (batch, seqlen, dstate) io type */
+  const float* D;      /* (dim) fp32 or NULL              */
+  const void* z;       /* (batch, seqlen, dim) io or NULL */
+  const float* bias;   /* (dim) fp32 or NULL              */
+  int softplus;
+  const float* h0;     /* (batch, dim, dstate) fp32 or NULL */
+  const int64_t* chans;/* nchan pairs (b, d)              */
+  int64_t nchan;
+  double* y;           /* (nchan, seqlen)                 */
+  double* h_last;      /* (nchan, dstate) or NULL         */
+} scan_job;
+
+/* One channel (b, d), sequentially in t: the loop of the §3.3 selective_scan
+ * for a single (b, d) row, without materialising deltaA / deltaB. */
+static void scan_one_channel(const scan_job* j, int64_t k) {
+  const int64_t b = j->chans[2 * k], d = j->chans[2 * k + 1];
+  const int64_t L = j->seqlen, Dm = j->dim, N = j->dstate;
+  double h[ORACLE_MAX_N];
+  for (int64_t n = 0; n < N; ++n)
+    h[n] = j->h0 ? (double)j->h0[(b * Dm + d) * N + n] : 0.0;
+  const double bias = j->bias ? (double)j->bias[d] : 0.0;
+  const double Dd = j->D ? (double)j->D[d] : 0.0;
+  for (int64_t t = 0; t < L; ++t) {
+    const int64_t i_bld = (b * L + t) * Dm + d;
+    const int64_t i_bln = (b * L + t) * N;
+    const double xv = widen(j->x, i_bld, j->is_bf16);
+    const double v = widen(j->delta, i_bld, j->is_bf16) + bias;
+    const double dt = j->softplus ? softplus(v) : v;
+    double y = 0.0;
+    for (int64_t n = 0; n < N; ++n) {
+      const double dA = exp(dt * (double)j->A[d * N + n]);
+      const double dB = dt * widen(j->B, i_bln + n, j->is_bf16);
+      h[n] = dA * h[n] + dB * xv;
+      y += widen(j->C, i_bln + n, j->is_bf16) * h[n];
+    }
+    y += Dd * xv;
+    if (j->z) y *= silu(widen(j->z, i_bld, j->is_bf16));
+    j->y[k * L + t] = y;
+  }
+  if (j->h_last)
+    for (int64_t n = 0; n < N; ++n) j->h_last[k * N + n] = h[n];
+}
+
+typedef struct {
+  const scan_job* job;
+  int64_t lo, hi;
+} scan_slice;
+
+static void* scan_worker(void* arg) {
+  const scan_slice* s = (const scan_slice*)arg;
+  for (int64_t k = s->lo; k < s->hi; ++k) scan_one_channel(s->job, k);
+  return NULL;
+}
+
+/*
+ * oracle_selective_scan -- run the scan for `nchan` channels given as
+ * (b, d) pairs in `chans`, splitting the channels over `nthreads` threads
+ * (each channel stays sequential in t). Returns 0, or -1 on bad arguments.
+ */
+int oracle_selective_scan(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
+                          int is_bf16, const void* x, const void* delta, const float* A,
+                          const void* B, const void* C, const float* D, const void* z,
+                          const float* bias, int softplus_on, const float* h0,
+                          const int64_t* chans, int64_t nchan, double* y, double* h_last,
+                          int nthreads) {
+  if (batch < 0 || seqlen < 0 || dim < 0 || dstate <= 0 || dstate > ORACLE_MAX_N) return -1;
+  if (!x || !delta || !A || !B || !C || !chans || !y) return -1;
+  for (int64_t k = 0; k < nchan; ++k)
+    if (chans[2 * k] < 0 || chans[2 * k] >= batch || chans[2 * k + 1] < 0 ||
+        chans[2 * k + 1] >= dim)
+      return -1;
+  scan_job job = {batch, seqlen, dim, dstate, is_bf16, x, delta, A, B, C, D, z,
+                  bias, softplus_on, h0, chans, nchan, y, h_last};
+  if (nthreads < 1) nthreads = 1;
+  if (nthreads > 256) nthreads = 256;
+  if (nthreads == 1 || nchan < 2) {
+    for (int64_t k = 0; k < nchan; ++k) scan_one_channel(&job, k);
+    return 0;
+  }
+  pthread_t tid[256];
+  scan_slice sl[256];
+  int started = 0;
+  for (int w = 0; w < nthreads; ++w) {
+    sl[w].job = &job;
+    sl[w].lo = nchan * w / nthreads;
+    sl[w].hi = nchan * (w + 1) / nthreads;
+    if (pthread_create(&tid[w], NULL, scan_worker, &sl[w]) == 0) {
+      ++started;
+    } else {
+      scan_worker(&sl[w]);
+      tid[w] = 0;
+    }
+  }
+  for (int w = 0; w < nthreads; ++w)
+    if (tid[w]) pthread_join(tid[w], NULL);
+  (void)started;
+  return 0;
+}
+
+/*
+ * oracle_state_update -- one decode step (the recurrent, O(1)-per-token form
+ * of the same recurrence: the scan's loop body with L = 1). `state` is the
+ * oracle's own fp64 (batch, dim, dstate) state, updated in place; y is
+ * (batch, dim). x, delta, z are (batch, dim); B, C are (batch, dstate).
+ */
+int oracle_state_update(int64_t batch, int64_t dim, int64_t dstate, int is_bf16,
+                        double* state, const void* x, const void* delta, const float* A,
+                        const void* B, const void* C, const float* D, const void* z,
+                        const float* bias, int softplus_on, double* y) {
+  if (batch < 0 || dim < 0 || dstate <= 0 || !state || !x || !delta || !A || !B || !C || !y)
+    return -1;
+  for (int64_t b = 0; b < batch; ++b) {
+    for (int64_t d = 0; d < dim; ++d) {
+      const int64_t i_bd = b * dim + d;
+      const double xv = widen(x, i_bd, is_bf16);
+      const double v = widen(delta, i_bd, is_bf16) + (bias ? (double)bias[d] : 0.0);
+      const double dt = softplus_on ? softplus(v) : v;
+      double* h = state + i_bd * dstate;
+      double acc = 0.0;
+      for (int64_t n = 0; n < dstate; ++n) {
+        const double dA = exp(dt * (double)A[d * dstate + n]);
+        const double dB = dt * widen(B, b * dstate + n, is_bf16);
+        h[n] = dA * h[n] + dB * xv;
+        acc += widen(C, b * dstate + n, is_bf16) * h[n];
+      }
+      acc += (D ? (double)D[d] : 0.0) * xv;
+      if (z) acc *= silu(widen(z, i_bd, is_bf16));
+      y[i_bd] = acc;
+    }
+  }
+  return 0;
+}

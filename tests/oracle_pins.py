@@ -1,0 +1,328 @@
+"""Pins of the fp64 oracle to things other than itself.
+
+Each pin takes an ``oracle.Oracle`` handle and raises AssertionError when
+the oracle disagrees with a closed form, a brute-force evaluation of a
+different formula, a library routine, an invariant of the recurrence or a
+hand-worked example. ``tests/test_oracle_pins.py`` runs them against the
+real oracle and against deliberately broken copies of it (every broken copy
+must fail at least one pin).
+
+Source of the definitions: page "Mamba 논문 리뷰: Selective State Space
+Models로 Transformer를 넘어서" (youngju.dev) -- §2.2 discretised recurrence,
+§3.1 softplus step, §3.3 selective_scan, §3.4 D skip and SiLU gate, §4.1 the
+SSM as a (semi-separable) matrix acting on the sequence -- and the linear
+attention recurrence s_t = s_{t-1} + phi(k_t)^T v_t of the page "[논문 리뷰]
+Attention to Mamba: A Recipe for Cross-Architecture Distillation"
+(suanlab.com, stage 2), which is the A = 0 special case.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+from scipy.special import expit
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _f32(a):
+    return np.asarray(a, dtype=np.float32)
+
+
+def _softplus_lib(v):
+    return np.logaddexp(0.0, v)  # library log(1 + e^v)
+
+
+def _close(a, b, rtol, atol=0.0, what=""):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    err = np.abs(a - b)
+    tol = atol + rtol * np.abs(b)
+    if not np.all(err <= tol):
+        i = np.unravel_index(np.argmax(err - tol), err.shape)
+        raise AssertionError(f"{what}: mismatch at {i}: got {a[i]!r}, want {b[i]!r}")
+
+
+def random_case(seed, batch=2, L=9, dim=3, N=4, gate=True, skip=True, h0=True, A=None,
+                softplus=True):
+    r = _rng(seed)
+    case = dict(
+        x=_f32(r.standard_normal((batch, L, dim))),
+        delta=_f32(0.5 * r.standard_normal((batch, L, dim))),
+        A=_f32(-r.uniform(0.2, 3.0, (dim, N))) if A is None else _f32(A),
+        B=_f32(r.standard_normal((batch, L, N))),
+        C=_f32(r.standard_normal((batch, L, N))),
+        D=_f32(r.uniform(-1, 1, dim)) if skip else None,
+        z=_f32(r.standard_normal((batch, L, dim))) if gate else None,
+        delta_bias=_f32(r.uniform(-2, 0.5, dim)),
+        h0=_f32(r.standard_normal((batch, dim, N))) if h0 else None,
+        softplus=softplus,
+    )
+    return case
+
+
+def _delta_f64(case):
+    v = case["delta"].astype(np.float64)
+    if case["delta_bias"] is not None:
+        v = v + case["delta_bias"].astype(np.float64)[None, None, :]
+    return _softplus_lib(v) if case["softplus"] else v
+
+
+def _gate(y, case):
+    if case["z"] is None:
+        return y
+    z = case["z"].astype(np.float64)
+    return y * z * expit(z)
+
+
+def _skip(case):
+    if case["D"] is None:
+        return 0.0
+    return case["D"].astype(np.float64)[None, None, :] * case["x"].astype(np.float64)
+
+
+# --------------------------------------------------------------------------
+# pins
+def pin_softplus_library(o):
+    """L = 1, A = 0, B = C = x = 1, no skip: y = Delta = softplus(delta)."""
+    v = _f32(np.concatenate([np.linspace(-30, 40, 141), [0.0, 19.99, 20.0, 20.01, 25.0]]))
+    n = v.size
+    one = np.ones((1, 1, n), np.float32)
+    y, _ = o.selective_scan(one, v.reshape(1, 1, n), np.zeros((n, 1), np.float32),
+                            np.ones((1, 1, 1), np.float32), np.ones((1, 1, 1), np.float32),
+                            softplus=True)
+    _close(y[0, 0], _softplus_lib(v.astype(np.float64)), 3e-9, what="softplus")
+
+
+def pin_silu_library(o):
+    """Delta = 1 (softplus off), A = 0, B = C = x = 1: y = SiLU(z) = z sigmoid(z)."""
+    z = _f32(np.linspace(-12, 12, 97))
+    n = z.size
+    one = np.ones((1, 1, n), np.float32)
+    y, _ = o.selective_scan(one, one, np.zeros((n, 1), np.float32),
+                            np.ones((1, 1, 1), np.float32), np.ones((1, 1, 1), np.float32),
+                            z=z.reshape(1, 1, n), softplus=False)
+    zz = z.astype(np.float64)
+    _close(y[0, 0], zz * expit(zz), 1e-13, 1e-300, what="silu")
+
+
+def pin_A_zero_is_cumulative_sum(o):
+    """A = 0 => deltaA = 1: h_t = h0 + cumsum_s(Delta_s x_s B_s) (linear
+    attention's s_t = s_{t-1} + k_t^T v_t); y from a library prefix sum."""
+    c = random_case(11, batch=2, L=17, dim=3, N=4, A=np.zeros((3, 4)))
+    y, hl = o.selective_scan(c["x"], c["delta"], c["A"], c["B"], c["C"], D=c["D"], z=c["z"],
+                             delta_bias=c["delta_bias"], softplus=True, h0=c["h0"])
+    dt = _delta_f64(c)  # (b, L, d)
+    inc = (dt * c["x"].astype(np.float64))[..., None] * c["B"].astype(np.float64)[:, :, None, :]
+    h = c["h0"].astype(np.float64)[:, None] + np.cumsum(inc, axis=1)  # (b, L, d, n)
+    yy = np.einsum("bln,bldn->bld", c["C"].astype(np.float64), h) + _skip(c)
+    _close(y, _gate(yy, c), 1e-12, 1e-12, what="cumsum y")
+    _close(hl, h[:, -1], 1e-12, 1e-12, what="cumsum h_last")
+
+
+def pin_geometric_series(o):
+    """Constant Delta, B, C, x in t: h_t = a^(t+1) h0 + Delta B x (1 - a^(t+1)) / (1 - a)."""
+    r = _rng(5)
+    batch, L, dim, N = 2, 40, 3, 4
+    x = np.repeat(_f32(r.standard_normal((batch, 1, dim))), L, axis=1)
+    delta = np.repeat(_f32(0.4 * r.standard_normal((batch, 1, dim))), L, axis=1)
+    B = np.repeat(_f32(r.standard_normal((batch, 1, N))), L, axis=1)
+    C = np.repeat(_f32(r.standard_normal((batch, 1, N))), L, axis=1)
+    A = _f32(-r.uniform(0.3, 2.0, (dim, N)))
+    D = _f32(r.uniform(-1, 1, dim))
+    bias = _f32(r.uniform(-1, 0.5, dim))
+    h0 = _f32(r.standard_normal((batch, dim, N)))
+    y, hl = o.selective_scan(x, delta, A, B, C, D=D, delta_bias=bias, softplus=True, h0=h0)
+    dt = _softplus_lib(delta[:, 0].astype(np.float64) + bias)  # (b, d)
+    a = np.exp(dt[..., None] * A.astype(np.float64)[None])  # (b, d, n)
+    u = dt[..., None] * B[:, 0].astype(np.float64)[:, None, :] * x[:, 0].astype(np.float64)[..., None]
+    t = np.arange(1, L + 1, dtype=np.float64)[None, :, None, None]
+    h = a[:, None] ** t * h0.astype(np.float64)[:, None] + u[:, None] * (1 - a[:, None] ** t) / (1 - a[:, None])
+    yy = np.einsum("bn,bldn->bld", C[:, 0].astype(np.float64), h) + D[None, None] * x.astype(np.float64)
+    _close(y, yy, 1e-12, 1e-12, what="geometric y")
+    _close(hl, h[:, -1], 1e-12, 1e-12, what="geometric h_last")
+
+
+def pin_single_step_by_hand(o):
+    """L = 1: y = (C . (exp(Delta A) h0 + Delta B x) + D x) SiLU(z), written out."""
+    c = random_case(3, batch=2, L=1, dim=3, N=4)
+    y, hl = o.selective_scan(c["x"], c["delta"], c["A"], c["B"], c["C"], D=c["D"], z=c["z"],
+                             delta_bias=c["delta_bias"], softplus=True, h0=c["h0"])
+    for b in range(2):
+        for d in range(3):
+            v = float(c["delta"][b, 0, d]) + float(c["delta_bias"][d])
+            dt = math.log1p(math.exp(v))
+            h = [math.exp(dt * float(c["A"][d, n])) * float(c["h0"][b, d, n])
+                 + dt * float(c["B"][b, 0, n]) * float(c["x"][b, 0, d]) for n in range(4)]
+            yy = sum(float(c["C"][b, 0, n]) * h[n] for n in range(4)) + float(c["D"][d]) * float(c["x"][b, 0, d])
+            zz = float(c["z"][b, 0, d])
+            yy *= zz / (1 + math.exp(-zz))
+            _close(y[b, 0, d], yy, 1e-13, 1e-15, what="one step y")
+            _close(hl[b, d], h, 1e-13, 1e-15, what="one step h")
+
+
+def pin_dual_matrix_form(o):
+    """Brute force the sequence-mixing matrix (the SSM as a matrix, §4.1):
+    y_t = sum_{s<=t} M_ts x_s + C_t.(prod_{r<=t} a_r) h0 + D x_t with
+    M_ts = sum_n C_tn [prod_{s<r<=t} exp(Delta_r A_n)] Delta_s B_sn."""
+    c = random_case(7, batch=2, L=12, dim=3, N=4)
+    y, hl = o.selective_scan(c["x"], c["delta"], c["A"], c["B"], c["C"], D=c["D"], z=c["z"],
+                             delta_bias=c["delta_bias"], softplus=True, h0=c["h0"])
+    dt = _delta_f64(c)
+    batch, L, dim = c["x"].shape
+    N = c["A"].shape[1]
+    yy = np.zeros((batch, L, dim))
+    for b in range(batch):
+        for d in range(dim):
+            A = c["A"][d].astype(np.float64)
+            for t in range(L):
+                acc = 0.0
+                for s in range(t + 1):
+                    for n in range(N):
+                        decay = 1.0
+                        for rr in range(s + 1, t + 1):
+                            decay *= math.exp(dt[b, rr, d] * A[n])
+                        acc += float(c["C"][b, t, n]) * decay * dt[b, s, d] * float(c["B"][b, s, n]) * float(c["x"][b, s, d])
+                for n in range(N):
+                    decay = 1.0
+                    for rr in range(0, t + 1):
+                        decay *= math.exp(dt[b, rr, d] * A[n])
+                    acc += float(c["C"][b, t, n]) * decay * float(c["h0"][b, d, n])
+                yy[b, t, d] = acc
+    yy = _gate(yy + _skip(c), c)
+    _close(y, yy, 1e-11, 1e-12, what="dual form")
+
+
+def pin_linear_in_x_and_h0(o):
+    """Without the gate, y is affine in (x, h0): y(x, h0) = y(x, 0) + y(0, h0),
+    and y(a x1 + b x2, 0) = a y(x1, 0) + b y(x2, 0)."""
+    c = random_case(13, gate=False)
+    x2 = _f32(_rng(14).standard_normal(c["x"].shape))
+    run = lambda x, h0: o.selective_scan(x, c["delta"], c["A"], c["B"], c["C"], D=c["D"],
+                                         delta_bias=c["delta_bias"], softplus=True, h0=h0)[0]
+    zero_x = np.zeros_like(c["x"])
+    _close(run(c["x"], c["h0"]), run(c["x"], None) + run(zero_x, c["h0"]), 1e-11, 1e-12,
+           what="affine in h0")
+    a, b = 0.75, -1.5
+    lhs = run(_f32(a * c["x"].astype(np.float64) + b * x2), None)
+    rhs = a * run(c["x"], None) + b * run(x2, None)
+    # a*x + b*x2 is rounded once to fp32 on the left: tolerance 1e-6
+    _close(lhs, rhs, 1e-6, 1e-6, what="linear in x")
+
+
+def pin_split_invariance(o):
+    """scan(L1) then scan(L2, h0 = h_last) equals scan(L1 + L2)."""
+    c = random_case(17, batch=2, L=23, dim=3, N=4)
+    y, hl = o.selective_scan(c["x"], c["delta"], c["A"], c["B"], c["C"], D=c["D"], z=c["z"],
+                             delta_bias=c["delta_bias"], softplus=True, h0=c["h0"])
+    k = 10
+    part = lambda sl, h0: o.selective_scan(c["x"][:, sl], c["delta"][:, sl], c["A"],
+                                           c["B"][:, sl], c["C"][:, sl], D=c["D"],
+                                           z=c["z"][:, sl], delta_bias=c["delta_bias"],
+                                           softplus=True, h0=h0)
+    y1, h1 = part(slice(0, k), c["h0"])
+    # h0 is fp32 at the boundary: compare against the full run in fp64 with tolerance
+    y2, h2 = part(slice(k, None), _f32(h1))
+    _close(y1, y[:, :k], 0, 0, what="prefix identical")
+    _close(y2, y[:, k:], 1e-6, 1e-7, what="suffix")
+    _close(h2, hl, 1e-6, 1e-7, what="h_last")
+
+
+def pin_zero_step_keeps_state(o):
+    """Delta = 0 (softplus off, delta = bias = 0): deltaA = 1, deltaB = 0, so
+    h_t = h0 and y_t = C_t . h0 + D x_t."""
+    c = random_case(19, gate=False, softplus=False)
+    zero = np.zeros_like(c["delta"])
+    y, hl = o.selective_scan(c["x"], zero, c["A"], c["B"], c["C"], D=c["D"], softplus=False,
+                             h0=c["h0"])
+    yy = np.einsum("bln,bdn->bld", c["C"].astype(np.float64), c["h0"].astype(np.float64)) + _skip(c)
+    _close(y, yy, 1e-13, 1e-13, what="zero step y")
+    _close(hl, c["h0"], 0, 0, what="zero step h")
+
+
+def pin_large_step_is_memoryless(o):
+    """Delta = 60 with A <= -1: exp(Delta A) < 1e-26, so h_t = Delta B_t x_t
+    (the page's forgetting role of Delta, by the equations)."""
+    c = random_case(23, gate=False, softplus=False, A=-np.ones((3, 4)) * np.arange(1, 5))
+    big = np.full_like(c["delta"], 60.0)
+    y, hl = o.selective_scan(c["x"], big, c["A"], c["B"], c["C"], D=c["D"], softplus=False,
+                             h0=c["h0"])
+    h = 60.0 * c["x"].astype(np.float64)[..., None] * c["B"].astype(np.float64)[:, :, None, :]
+    yy = np.einsum("bln,bldn->bld", c["C"].astype(np.float64), h) + _skip(c)
+    _close(y, yy, 1e-14, 1e-14, what="memoryless y")
+    _close(hl, h[:, -1], 1e-14, 1e-14, what="memoryless h")
+
+
+def pin_golden_hand_worked(o):
+    with open(os.path.join(GOLDEN, "hand_worked_scan.json")) as f:
+        spec = json.load(f)
+    env = {"exp": math.exp, "log": math.log}
+    for case in spec["cases"]:
+        dims = case["dims"]
+        batch, L, dim, N = dims["batch"], dims["seqlen"], dims["dim"], dims["dstate"]
+        arr = lambda v, shape: None if v is None else _f32(v).reshape(shape)
+        y, hl = o.selective_scan(
+            arr(case["x"], (batch, L, dim)), arr(case["delta"], (batch, L, dim)),
+            arr(case["A"], (dim, N)), arr(case["B"], (batch, L, N)), arr(case["C"], (batch, L, N)),
+            D=arr(case["D"], (dim,)), z=arr(case["z"], (batch, L, dim)),
+            delta_bias=arr(case["delta_bias"], (dim,)), softplus=case["softplus"],
+            h0=arr(case["h0"], (batch, dim, N)))
+        want_y = np.array([eval(e, {"__builtins__": {}}, env) for e in case["y"]])
+        want_h = np.array([eval(e, {"__builtins__": {}}, env) for e in case["h_last"]])
+        _close(y.reshape(-1), want_y, 1e-14, 1e-15, what=case["name"] + " y")
+        _close(hl.reshape(-1), want_h, 1e-14, 1e-15, what=case["name"] + " h_last")
+
+
+def pin_decode_steps_equal_scan(o):
+    """L decode steps on a carried fp64 state equal one scan over the same tokens."""
+    c = random_case(29, batch=2, L=15, dim=3, N=4)
+    y, hl = o.selective_scan(c["x"], c["delta"], c["A"], c["B"], c["C"], D=c["D"], z=c["z"],
+                             delta_bias=c["delta_bias"], softplus=True, h0=c["h0"])
+    state = np.ascontiguousarray(c["h0"].astype(np.float64))
+    for t in range(c["x"].shape[1]):
+        yt = o.state_update(state, c["x"][:, t], c["delta"][:, t], c["A"], c["B"][:, t],
+                            c["C"][:, t], D=c["D"], z=c["z"][:, t], delta_bias=c["delta_bias"],
+                            softplus=True)
+        _close(yt, y[:, t], 1e-14, 1e-14, what=f"decode step {t}")
+    _close(state, hl, 1e-14, 1e-14, what="decode state")
+
+
+def pin_decode_single_step_by_hand(o):
+    c = random_case(31, batch=2, L=1, dim=3, N=4)
+    state = np.ascontiguousarray(c["h0"].astype(np.float64))
+    yt = o.state_update(state, c["x"][:, 0], c["delta"][:, 0], c["A"], c["B"][:, 0],
+                        c["C"][:, 0], D=c["D"], z=c["z"][:, 0], delta_bias=c["delta_bias"],
+                        softplus=True)
+    for b in range(2):
+        for d in range(3):
+            dt = math.log1p(math.exp(float(c["delta"][b, 0, d]) + float(c["delta_bias"][d])))
+            h = [math.exp(dt * float(c["A"][d, n])) * float(c["h0"][b, d, n])
+                 + dt * float(c["B"][b, 0, n]) * float(c["x"][b, 0, d]) for n in range(4)]
+            yy = sum(float(c["C"][b, 0, n]) * h[n] for n in range(4)) + float(c["D"][d]) * float(c["x"][b, 0, d])
+            zz = float(c["z"][b, 0, d])
+            yy *= zz / (1 + math.exp(-zz))
+            _close(yt[b, d], yy, 1e-13, 1e-15, what="decode by hand y")
+            _close(state[b, d], h, 1e-13, 1e-15, what="decode by hand h")
+
+
+ALL_PINS = [
+    pin_softplus_library,
+    pin_silu_library,
+    pin_A_zero_is_cumulative_sum,
+    pin_geometric_series,
+    pin_single_step_by_hand,
+    pin_dual_matrix_form,
+    pin_linear_in_x_and_h0,
+    pin_split_invariance,
+    pin_zero_step_keeps_state,
+    pin_large_step_is_memoryless,
+    pin_golden_hand_worked,
+    pin_decode_steps_equal_scan,
+    pin_decode_single_step_by_hand,
+]

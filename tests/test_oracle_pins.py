@@ -1,0 +1,93 @@
+"""The oracle against its pins (CPU only), and mutation checks: copies of the
+oracle source with one plausible mistake planted each must fail a pin."""
+import os
+import shutil
+
+import numpy as np
+import pytest
+
+import oracle
+from tests import oracle_pins as pins
+
+
+@pytest.fixture(scope="module")
+def o():
+    return oracle.get()
+
+
+@pytest.mark.parametrize("pin", pins.ALL_PINS, ids=lambda f: f.__name__)
+def test_oracle_pin(o, pin):
+    pin(o)
+
+
+def test_bf16_inputs_widen_exactly(o):
+    """bf16 storage is read as the exact binary32 value it denotes."""
+    import ssm_inputs as gen
+    c = pins.random_case(41, batch=2, L=8, dim=3, N=4)
+    bits = {k: gen.f32_to_bf16_bits(c[k]) for k in ("x", "delta", "B", "C", "z")}
+    wide = {k: gen.bf16_bits_to_f32(v) for k, v in bits.items()}
+    y16, h16 = o.selective_scan(bits["x"], bits["delta"], c["A"], bits["B"], bits["C"], D=c["D"],
+                                z=bits["z"], delta_bias=c["delta_bias"], h0=c["h0"], io="bf16")
+    y32, h32 = o.selective_scan(wide["x"], wide["delta"], c["A"], wide["B"], wide["C"], D=c["D"],
+                                z=wide["z"], delta_bias=c["delta_bias"], h0=c["h0"], io="f32")
+    assert np.array_equal(y16, y32) and np.array_equal(h16, h32)
+
+
+def test_channel_subset_and_threads_agree(o):
+    c = pins.random_case(43, batch=3, L=20, dim=5, N=4)
+    kw = dict(D=c["D"], z=c["z"], delta_bias=c["delta_bias"], h0=c["h0"])
+    y, hl = o.selective_scan(c["x"], c["delta"], c["A"], c["B"], c["C"], **kw)
+    y4, hl4 = o.selective_scan(c["x"], c["delta"], c["A"], c["B"], c["C"], nthreads=4, **kw)
+    assert np.array_equal(y, y4) and np.array_equal(hl, hl4)
+    chans = [(2, 4), (0, 0), (1, 3)]
+    ys, hs = o.selective_scan(c["x"], c["delta"], c["A"], c["B"], c["C"], channels=chans, **kw)
+    for k, (b, d) in enumerate(chans):
+        assert np.array_equal(ys[k], y[b, :, d]) and np.array_equal(hs[k], hl[b, d])
+
+
+def test_oracle_rejects_bad_channels(o):
+    c = pins.random_case(47)
+    with pytest.raises(ValueError):
+        o.selective_scan(c["x"], c["delta"], c["A"], c["B"], c["C"], channels=[(5, 0)])
+
+
+# (original, mutated) snippets of ssm_oracle.c: each is a plausible mistake.
+MUTANTS = {
+    "drop_skip": ("    y += Dd * xv;\n    if (j->z)", "    if (j->z)"),
+    "sign_of_A": ("exp(dt * (double)j->A[d * N + n])", "exp(-dt * (double)j->A[d * N + n])"),
+    "readout_before_update": (
+        "      h[n] = dA * h[n] + dB * xv;\n      y += widen(j->C, i_bln + n, j->is_bf16) * h[n];",
+        "      y += widen(j->C, i_bln + n, j->is_bf16) * h[n];\n      h[n] = dA * h[n] + dB * xv;"),
+    "B_C_swapped": ("const double dB = dt * widen(j->B, i_bln + n, j->is_bf16);\n      h[n] = dA * h[n] + dB * xv;\n      y += widen(j->C,",
+                    "const double dB = dt * widen(j->C, i_bln + n, j->is_bf16);\n      h[n] = dA * h[n] + dB * xv;\n      y += widen(j->B,"),
+    "bias_dropped": ("widen(j->delta, i_bld, j->is_bf16) + bias;", "widen(j->delta, i_bld, j->is_bf16);"),
+    "softplus_as_exp": ("return v > 20.0 ? v : log1p(exp(v));", "return v > 20.0 ? v : exp(v);"),
+    "sigmoid_not_silu": ("return z / (1.0 + exp(-z));", "return 1.0 / (1.0 + exp(-z));"),
+    "h0_ignored": ("h[n] = j->h0 ? (double)j->h0[(b * Dm + d) * N + n] : 0.0;", "h[n] = 0.0;"),
+    "A_transposed": ("exp(dt * (double)j->A[d * N + n])", "exp(dt * (double)j->A[(n * Dm + d) % (Dm * N)])"),
+    "x_index_wrong": ("const double xv = widen(j->x, i_bld, j->is_bf16);",
+                      "const double xv = widen(j->x, (i_bld + 1) % (j->batch * L * Dm), j->is_bf16);"),
+    "dB_without_delta": ("const double dB = dt * widen(j->B, i_bln + n, j->is_bf16);",
+                         "const double dB = widen(j->B, i_bln + n, j->is_bf16);"),
+    "decode_drops_gate": ("      if (z) acc *= silu(widen(z, i_bd, is_bf16));\n", ""),
+    "decode_state_not_kept": ("        h[n] = dA * h[n] + dB * xv;\n        acc +=",
+                              "        const double hn = dA * h[n] + dB * xv;\n        acc += 0 * hn +"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(name, tmp_path):
+    src = open(oracle.SOURCE).read()
+    before, after = MUTANTS[name]
+    assert src.count(before) >= 1, f"mutation anchor for {name} not found in the oracle source"
+    mutated = tmp_path / "ssm_oracle_mutant.c"
+    mutated.write_text(src.replace(before, after, 1))
+    lib = oracle.compile_library(str(mutated), str(tmp_path / "libmutant.so"))
+    m = oracle.Oracle(lib)
+    failed = []
+    for pin in pins.ALL_PINS:
+        try:
+            pin(m)
+        except (AssertionError, ValueError, FloatingPointError):
+            failed.append(pin.__name__)
+    assert failed, f"no pin caught the planted mistake {name}"
