@@ -1,0 +1,327 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 selective scan (one JSON line on rank 0).
+
+A step is one ssm_scan_fwd call (carry pass + main pass) over one batch of the
+synthetic Mamba-shaped workload, inputs resident in HBM, L2 flushed (256 MB
+write) before every timed step, each step timed with CUDA events on the
+launching stream. With torchrun (N > 1) every rank scans its own batch shard
+of an N-times larger global batch (weak scaling, no data-path collective);
+the time is the max over ranks.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the fp64 CPU oracle on host cores
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import ssm_inputs as gen  # noqa: E402
+
+METRIC = "selective-scan elements/s (B·L·D) and achieved HBM GB/s as % of B200 peak"
+DEFAULT_WORKLOAD = "mamba130m_layer_b8_l2048_d1536"
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(gen.SCAN_WORKLOADS))
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="target CPU time of the oracle baseline sample")
+    return ap.parse_args()
+
+
+def algorithmic_bytes(w, batch):
+    """Bytes a scan must move at least: inputs read once, outputs written
+    once, no (B, L, D, N) intermediates."""
+    es = 2 if w.io == "bf16" else 4
+    bld, bln = batch * w.seqlen * w.dim, batch * w.seqlen * w.dstate
+    per_elem = (4 if w.gate else 3) * es  # x, delta, (z), y
+    state = batch * w.dim * w.dstate * 4 * (2 if w.with_h0 else 1)  # h_last (+ h0)
+    params = w.dim * w.dstate * 4 + w.dim * 4 * (2 if w.skip else 1)  # A, bias, (D)
+    return bld * per_elem + 2 * bln * es + state + params
+
+
+def measured_hbm_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons with NVML while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index, interval_s=0.002):
+        self.samples, self.reasons, self.max_mhz, self.error = [], 0, None, None
+        self.interval = interval_s
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            idx = device_index
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            if vis:
+                idx = int(vis.split(",")[device_index])
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # pragma: no cover - depends on the box
+            self.nvml, self.error = None, f"nvml unavailable: {e}"
+        self.t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        get_reasons = getattr(self.nvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            getattr(self.nvml, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nvml.nvmlDeviceGetClockInfo(self.h, self.nvml.NVML_CLOCK_SM))
+                self.reasons |= int(get_reasons(self.h))
+            except Exception as e:  # pragma: no cover
+                self.error = str(e)
+                return
+            time.sleep(self.interval)
+
+    def __enter__(self):
+        if self.nvml:
+            self.t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self.nvml:
+            self.t.join()
+
+    def summary(self):
+        if not self.nvml:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": self.error}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and bit != 0x1]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+def cpu_oracle_rate(w, inp, target_s, rng_seed=0):
+    """Oracle throughput (elements/s) on a bounded sample of the workload's
+    channels, all host threads. Returns (value, cores, sample text)."""
+    import oracle
+    threads = gen.default_threads()
+    batch = inp["x"].shape[0]
+    rng = np.random.default_rng(rng_seed)
+    all_ch = [(b, d) for b in range(batch) for d in range(w.dim)]
+
+    def run(n):
+        idx = rng.choice(len(all_ch), size=min(n, len(all_ch)), replace=False)
+        chans = [all_ch[i] for i in idx]
+        t0 = time.perf_counter()
+        oracle.selective_scan(inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], D=inp["D"],
+                              z=inp["z"], delta_bias=inp["delta_bias"], h0=inp["h0"], io=w.io,
+                              channels=chans, nthreads=threads)
+        return len(chans), time.perf_counter() - t0
+
+    n, dt = run(threads)  # calibration
+    per_chan = dt / max(n, 1) * threads
+    n2 = int(max(threads, min(len(all_ch), target_s / max(per_chan, 1e-9) * threads)))
+    n2 = max(threads, n2 // threads * threads)
+    n, dt = run(n2)
+    value = n * w.seqlen / dt
+    return value, threads, f"{n} of {len(all_ch)} channels x {w.seqlen} steps, {dt:.1f} s"
+
+
+def reference_arm(args):
+    """--impl reference: the fp64 oracle on the host cores, rank 0 only."""
+    rank = int(os.environ.get("RANK", 0))
+    if rank != 0:
+        return 0
+    import oracle
+    w = gen.SCAN_WORKLOADS[args.workload]
+    threads = gen.default_threads()
+    inp = gen.workload_inputs(w)
+    rng = np.random.default_rng(1)
+    per_step = threads  # channels per step: one per host thread
+    all_ch = [(b, d) for b in range(w.batch) for d in range(w.dim)]
+    times = []
+    for i in range(args.warmup + args.steps):
+        idx = rng.choice(len(all_ch), size=per_step, replace=False)
+        t0 = time.perf_counter()
+        oracle.selective_scan(inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], D=inp["D"],
+                              z=inp["z"], delta_bias=inp["delta_bias"], h0=inp["h0"], io=w.io,
+                              channels=[all_ch[j] for j in idx], nthreads=threads)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = args.steps * per_step * w.seqlen / total
+    sample = f"{per_step} random channels x {w.seqlen} steps per step"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "elements/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "dim": w.dim,
+                   "dstate": w.dstate, "io": w.io},
+        "cpu_baseline": {"value": value, "unit": "elements/s", "cores": threads,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "elements/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return reference_arm(args)
+
+    import torch
+
+    from selective_state_space_39_b200 import dist as sdist
+    from selective_state_space_39_b200 import scan_plan, scan_workspace_bytes, ssm_scan_fwd
+
+    rank, local_rank, world = sdist.env_world()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU (the scan has no CPU path)")
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    sdist.init("nccl")
+
+    w = gen.SCAN_WORKLOADS[args.workload]
+    # weak scaling: global batch = world * w.batch; this rank's shard
+    b0, nb = sdist.batch_shard(world * w.batch, world, rank)
+    inp = gen.workload_inputs(w, batch=nb, batch_offset=b0)
+    dtype = torch.bfloat16 if w.io == "bf16" else torch.float32
+
+    def to_dev(a):
+        if a is None:
+            return None
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+    d = {k: to_dev(v) for k, v in inp.items()}
+    y = torch.empty((nb, w.seqlen, w.dim), dtype=dtype, device=device)
+    h_last = torch.empty((nb, w.dim, w.dstate), dtype=torch.float32, device=device)
+    ws = torch.empty(max(1, scan_workspace_bytes(nb, w.seqlen, w.dim, w.dstate, dtype)),
+                     dtype=torch.uint8, device=device)
+    plan = scan_plan(nb, w.seqlen, w.dim, w.dstate, dtype)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    def step():
+        ssm_scan_fwd(d["x"], d["delta"], d["A"], d["B"], d["C"], D=d["D"], z=d["z"],
+                     delta_bias=d["delta_bias"], h0=d["h0"], y=y, h_last=h_last, workspace=ws)
+
+    for _ in range(max(3, args.warmup)):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+
+    K = args.steps
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    sampler = ClockSampler(device.index)
+    sdist.barrier(device)
+    torch.cuda.synchronize()
+    with sampler:
+        for i in range(K):
+            flush.fill_(i & 0xFF)
+            starts[i].record()
+            step()
+            ends[i].record()
+        torch.cuda.synchronize()
+    sdist.barrier(device)
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    local_ms = sum(step_ms)
+    total_ms = sdist.max_over_ranks(local_ms, device)
+    ms_per_step = total_ms / K
+    elements = world * w.batch * w.seqlen * w.dim
+    value = elements * K / (total_ms * 1e-3)
+
+    # roofline of the call: algorithmic bytes / device time, against HBM peak
+    peak, peak_kind = measured_hbm_peak()
+    algo = algorithmic_bytes(w, nb)
+    achieved = algo / (statistics.mean(step_ms) * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": None,
+                "kernel": "ssm_scan_fwd: carry pass + main pass (%d launches)" % plan.kernels,
+                "algorithmic_bytes_per_launch": algo, "peak_kind": peak_kind}
+
+    # end to end through the public call: pinned host inputs -> device -> scan -> host
+    pinned = {k: (torch.from_numpy(v.view(np.int16) if v.dtype == np.uint16 else v)
+                  .view(dtype if v.dtype == np.uint16 else torch.float32).pin_memory()
+                  if v is not None else None) for k, v in inp.items()}
+    y_host = torch.empty(y.shape, dtype=dtype).pin_memory()
+    h_host = torch.empty(h_last.shape, dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in pinned.values() if t is not None)
+    d2h = y_host.numel() * y_host.element_size() + h_host.numel() * h_host.element_size()
+    e_ms = []
+    for i in range(args.e2e_steps + 2):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for k, t in pinned.items():
+            if t is not None:
+                d[k].copy_(t, non_blocking=True)
+        step()
+        y_host.copy_(y, non_blocking=True)
+        h_host.copy_(h_last, non_blocking=True)
+        e1.record()
+        e1.synchronize()
+        if i >= 2:
+            e_ms.append(e0.elapsed_time(e1))
+    e2e_ms = sdist.max_over_ranks(statistics.mean(e_ms), device)
+    e2e = {"value": elements / (e2e_ms * 1e-3), "unit": "elements/s",
+           "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    cpu = None
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        v, cores, sample = cpu_oracle_rate(w, inp, args.cpu_seconds)
+        cpu = {"value": v, "unit": "elements/s", "cores": cores, "kind": "oracle",
+               "sample": sample}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "elements/s", "n_gpus": world,
+            "steps": K, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if w.io == "bf16" else "f32",
+            "data": "synthetic (seeded Philox4x32-10, Mamba-shaped recipe)",
+            "config": {"workload": w.name, "batch_per_gpu": w.batch, "global_batch": world * w.batch,
+                       "seqlen": w.seqlen, "dim": w.dim, "dstate": w.dstate, "io": w.io,
+                       "gate": w.gate, "skip": w.skip, "h0": w.with_h0,
+                       "segments": plan.segments, "segment_steps": plan.segment_steps,
+                       "l2": "flushed (256 MB write) before every timed step",
+                       "parallelism": f"dp{world} (batch shards, no data-path collective)"},
+            "hbm_gbs": round(achieved, 1), "hbm_frac_of_peak": round(achieved / peak, 4),
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": K * plan.kernels, "clocks": sampler.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    sdist.finish()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

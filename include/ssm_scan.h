@@ -1,0 +1,164 @@
+/*
+ * ssm_scan.h -- C ABI of the B200 (sm_100a) selective state-space scan.
+ *
+ * The operation is the selective scan of Mamba as stated on the page
+ * "Mamba 논문 리뷰: Selective State Space Models로 Transformer를 넘어서"
+ * (youngju.dev): the discretised recurrence of §2.2 (Zero-Order Hold),
+ * with the input-dependent step of §3.1 (Delta = softplus(.)), the
+ * simplified deltaA = exp(Delta*A), deltaB = Delta*B of the §3.3
+ * selective_scan, and the D skip and y * SiLU(z) gate of the §3.4 Mamba
+ * block. Per batch b, channel d and state n (state fp32):
+ *
+ *   Delta   = softplus(delta[b,t,d] + delta_bias[d])   (or no softplus)
+ *   h[n]    = exp(Delta * A[d,n]) * h[n] + Delta * B[b,t,n] * x[b,t,d]
+ *   y[b,t,d]= (sum_n C[b,t,n] * h[n] + D[d] * x[b,t,d]) * SiLU(z[b,t,d])
+ *
+ * starting from h0[b,d,:] (or zero) and ending in h_last[b,d,:].
+ * softplus(v) is log(1 + e^v) for v <= 20 and v above 20.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller, dense and
+ *     row-major (C order) in the layouts given below. The library never
+ *     allocates, frees or synchronises, and keeps no mutable global state.
+ *   - io_dtype selects the storage type of x, delta, z, B, C and y:
+ *     SSM_DTYPE_F32 (IEEE binary32) or SSM_DTYPE_BF16 (bfloat16). A, D,
+ *     delta_bias, h0, h_last and the decode state are always fp32.
+ *   - Optional pointers may be NULL: D (no skip), z (no gate), delta_bias
+ *     (zero bias), h0 (zero initial state), h_last (not written).
+ *   - stream is a cudaStream_t (NULL = legacy default stream). Work is
+ *     enqueued asynchronously; errors of the kernels themselves surface at
+ *     the caller's next synchronisation.
+ *   - Return value: SSM_OK, or a negative SSM_ERR_* code. Argument errors
+ *     are detected on the host before anything is enqueued.
+ *   - Pointers must be aligned to their element size (h0 / h_last to 8
+ *     bytes, the decode state to 16 bytes when dstate % 4 == 0). The fast
+ *     path also wants 16-byte aligned bases and rows (dim and dstate
+ *     multiples of 16 bytes) and otherwise takes a slower path with plain
+ *     loads (SSM_SCAN_DISABLE_TMA=1 in the environment forces that path).
+ */
+#ifndef SSM_SCAN_H
+#define SSM_SCAN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  SSM_DTYPE_F32 = 0,
+  SSM_DTYPE_BF16 = 1,
+};
+
+enum {
+  SSM_OK = 0,
+  SSM_ERR_INVALID_ARG = -1, /* null required pointer, bad size, misaligned, aliasing */
+  SSM_ERR_UNSUPPORTED = -2, /* dstate or io_dtype this build does not support       */
+  SSM_ERR_WORKSPACE = -3,   /* workspace missing or smaller than required           */
+  SSM_ERR_CUDA = -4,        /* a CUDA runtime call or kernel launch failed          */
+  SSM_ERR_TIMEOUT = -5,     /* a bounded wait inside a kernel gave up (ssm_scan_status) */
+};
+
+/* dstate (N) values this build supports: 2, 4, 8, 16, 32, 64. */
+#define SSM_MAX_DSTATE 64
+
+/*
+ * How ssm_scan_fwd splits a problem (see ssm_scan_plan). The sequence is cut
+ * into `segments` of `segment_steps` steps; with more than one segment a
+ * carry pass computes each segment's end state and the main pass composes
+ * them (the recurrence of §2.2 is an associative composition of affine
+ * maps h -> a*h + b, which the pages' parallel associative scan relies on).
+ */
+typedef struct {
+  int32_t segments;
+  int32_t segment_steps;
+  int32_t channel_tiles;    /* CTAs along dim                                */
+  int32_t channels_per_cta;
+  int32_t ctas_carry;       /* CTAs of the carry pass (0 with one segment)   */
+  int32_t ctas_main;        /* CTAs of the main pass                         */
+  int32_t kernels;          /* kernel launches per ssm_scan_fwd call         */
+  int64_t workspace_bytes;  /* = ssm_scan_workspace_bytes(...)               */
+} ssm_scan_plan_t;
+
+/*
+ * ssm_scan_workspace_bytes -- bytes of device workspace ssm_scan_fwd needs
+ * for these sizes on the current device (0 when it needs none). The
+ * workspace holds per-segment carries of the sequence split (§2.2
+ * recurrence composed across sequence segments). Returns 0 for invalid
+ * sizes too; ssm_scan_fwd then reports the size error.
+ */
+size_t ssm_scan_workspace_bytes(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
+                                int io_dtype);
+
+/*
+ * ssm_scan_plan -- fill *out with the split ssm_scan_fwd will use for these
+ * sizes on the current device. Host only; enqueues nothing. The split
+ * targets about SSM_SCAN_CTAS_PER_SM (environment, default 4) resident CTAs
+ * per SM; SSM_SCAN_SEGMENTS (environment, > 0) forces the segment count.
+ * Returns SSM_OK or SSM_ERR_INVALID_ARG / SSM_ERR_UNSUPPORTED.
+ */
+int ssm_scan_plan(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate, int io_dtype,
+                  ssm_scan_plan_t* out);
+
+/*
+ * ssm_scan_fwd -- the selective scan (prefill / training-shaped forward).
+ *
+ *   x, delta, z, y : (batch, seqlen, dim)     io_dtype
+ *   B, C           : (batch, seqlen, dstate)  io_dtype, shared by all channels
+ *   A              : (dim, dstate)            fp32 (Mamba uses A = -exp(A_log))
+ *   D, delta_bias  : (dim)                    fp32, nullable
+ *   h0, h_last     : (batch, dim, dstate)     fp32, nullable
+ *   softplus       : nonzero applies softplus to delta + delta_bias
+ *   workspace      : device buffer of at least ssm_scan_workspace_bytes(...)
+ *                    bytes (may be NULL when that is 0); contents on entry
+ *                    are ignored; it must not be used by concurrent calls.
+ *
+ * y must not overlap any input. h_last may alias h0 (in-place resume).
+ * seqlen == 0 writes only h_last (= h0 or zero). batch or dim == 0 is a
+ * no-op. Returns SSM_OK or SSM_ERR_*.
+ */
+int ssm_scan_fwd(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate, int io_dtype,
+                 const void* x, const void* delta, const float* A, const void* B,
+                 const void* C, const float* D, const void* z, const float* delta_bias,
+                 int softplus, const float* h0, void* y, float* h_last, void* workspace,
+                 size_t workspace_bytes, void* stream);
+
+/*
+ * ssm_state_update -- one decode step: the recurrent, O(1)-per-token form of
+ * the same recurrence (the §3.3 loop body for a single t), updating the
+ * carried state in place.
+ *
+ *   state          : (batch, dim, dstate) fp32, read and written
+ *   x, delta, z, y : (batch, dim)             io_dtype (z nullable)
+ *   B, C           : (batch, dstate)          io_dtype
+ *   A              : (dim, dstate) fp32;  D, delta_bias : (dim) fp32, nullable
+ *
+ * y must not overlap any input or the state. Returns SSM_OK or SSM_ERR_*.
+ */
+int ssm_state_update(int64_t batch, int64_t dim, int64_t dstate, int io_dtype, float* state,
+                     const void* x, const void* delta, const float* A, const void* B,
+                     const void* C, const float* D, const void* z, const float* delta_bias,
+                     int softplus, void* y, void* stream);
+
+/*
+ * ssm_scan_status -- synchronise `stream`, then report whether every CTA of
+ * the last ssm_scan_fwd call that used this workspace (with these sizes)
+ * finished normally: SSM_OK, or SSM_ERR_TIMEOUT if a bounded wait inside a
+ * kernel gave up (its outputs are then incomplete). The wait bound is 2 s,
+ * or SSM_SCAN_WAIT_LIMIT_NS nanoseconds from the environment.
+ */
+int ssm_scan_status(const void* workspace, size_t workspace_bytes, int64_t batch,
+                    int64_t seqlen, int64_t dim, int64_t dstate, int io_dtype, void* stream);
+
+/* ssm_status_string -- static, human-readable text for an SSM_* code. */
+const char* ssm_status_string(int status);
+
+/* ssm_scan_version -- library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int ssm_scan_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSM_SCAN_H */

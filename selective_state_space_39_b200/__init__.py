@@ -1,0 +1,21 @@
+"""B200-native (sm_100a) selective state-space scan of Mamba.
+
+The work runs in libssmscan.so (hand-written CUDA kernels behind a C ABI,
+declared in include/ssm_scan.h); this package is a thin ctypes binding with
+the same entry-point names. PyTorch supplies device memory and streams.
+"""
+from ._binding import (  # noqa: F401
+    SSM_DTYPE_BF16,
+    SSM_DTYPE_F32,
+    ScanPlan,
+    SsmError,
+    lib,
+    scan_plan,
+    scan_workspace_bytes,
+    ssm_scan_fwd,
+    ssm_scan_status,
+    ssm_state_update,
+)
+
+__all__ = ["ssm_scan_fwd", "ssm_state_update", "ssm_scan_status", "scan_plan",
+           "scan_workspace_bytes", "SsmError", "SSM_DTYPE_F32", "SSM_DTYPE_BF16", "lib"]

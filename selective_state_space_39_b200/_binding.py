@@ -1,0 +1,199 @@
+"""ctypes binding of libssmscan.so: argument marshalling only.
+
+Every step of the scan runs in the library's CUDA kernels; this module only
+checks tensor metadata, allocates outputs/workspace with torch when the
+caller does not pass them, and forwards raw device pointers and the current
+CUDA stream. There is no CPU fallback: without the built library (or without
+a GPU) calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+SSM_DTYPE_F32, SSM_DTYPE_BF16 = 0, 1
+_STATUS = {0: "ok", -1: "invalid argument", -2: "unsupported size or dtype",
+           -3: "workspace missing or too small", -4: "CUDA error",
+           -5: "a kernel wait timed out"}
+
+
+class SsmError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {_STATUS.get(code, 'unknown status')} ({code})")
+
+
+class ScanPlan(ctypes.Structure):
+    _fields_ = [("segments", ctypes.c_int32), ("segment_steps", ctypes.c_int32),
+                ("channel_tiles", ctypes.c_int32), ("channels_per_cta", ctypes.c_int32),
+                ("ctas_carry", ctypes.c_int32), ("ctas_main", ctypes.c_int32),
+                ("kernels", ctypes.c_int32), ("workspace_bytes", ctypes.c_int64)]
+
+
+_lib = None
+_VP = ctypes.c_void_p
+_I64 = ctypes.c_int64
+
+
+def lib() -> ctypes.CDLL:
+    """Load libssmscan.so from the package directory (raises if absent)."""
+    global _lib
+    if _lib is None:
+        path = _build.LIB_PATH
+        if not os.path.exists(path):
+            raise RuntimeError(
+                f"{path} is missing: build it with `python -m selective_state_space_39_b200.build`"
+                " (the CUDA library is required; there is no CPU fallback)")
+        L = ctypes.CDLL(path)
+        L.ssm_scan_version.restype = ctypes.c_int
+        L.ssm_status_string.restype = ctypes.c_char_p
+        L.ssm_status_string.argtypes = [ctypes.c_int]
+        L.ssm_scan_workspace_bytes.restype = ctypes.c_size_t
+        L.ssm_scan_workspace_bytes.argtypes = [_I64, _I64, _I64, _I64, ctypes.c_int]
+        L.ssm_scan_plan.restype = ctypes.c_int
+        L.ssm_scan_plan.argtypes = [_I64, _I64, _I64, _I64, ctypes.c_int, ctypes.POINTER(ScanPlan)]
+        L.ssm_scan_fwd.restype = ctypes.c_int
+        L.ssm_scan_fwd.argtypes = [_I64, _I64, _I64, _I64, ctypes.c_int, _VP, _VP, _VP, _VP, _VP,
+                                   _VP, _VP, _VP, ctypes.c_int, _VP, _VP, _VP, _VP,
+                                   ctypes.c_size_t, _VP]
+        L.ssm_scan_status.restype = ctypes.c_int
+        L.ssm_scan_status.argtypes = [_VP, ctypes.c_size_t, _I64, _I64, _I64, _I64, ctypes.c_int,
+                                      _VP]
+        L.ssm_state_update.restype = ctypes.c_int
+        L.ssm_state_update.argtypes = [_I64, _I64, _I64, ctypes.c_int, _VP, _VP, _VP, _VP, _VP,
+                                       _VP, _VP, _VP, _VP, ctypes.c_int, _VP, _VP]
+        _lib = L
+    return _lib
+
+
+def _io_code(dtype: torch.dtype) -> int:
+    if dtype == torch.float32:
+        return SSM_DTYPE_F32
+    if dtype == torch.bfloat16:
+        return SSM_DTYPE_BF16
+    raise TypeError(f"io tensors must be float32 or bfloat16, got {dtype}")
+
+
+def _ptr(t, name, dtype=None, shape=None, device=None):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (there is no CPU path)")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t.data_ptr()
+
+
+def _stream_ptr(stream, device):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return stream.cuda_stream
+
+
+def scan_plan(batch, seqlen, dim, dstate, dtype=torch.bfloat16) -> ScanPlan:
+    out = ScanPlan()
+    rc = lib().ssm_scan_plan(batch, seqlen, dim, dstate, _io_code(dtype), ctypes.byref(out))
+    if rc != 0:
+        raise SsmError(rc, "ssm_scan_plan")
+    return out
+
+
+def scan_workspace_bytes(batch, seqlen, dim, dstate, dtype=torch.bfloat16) -> int:
+    return int(lib().ssm_scan_workspace_bytes(batch, seqlen, dim, dstate, _io_code(dtype)))
+
+
+def ssm_scan_fwd(x, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True, h0=None,
+                 y=None, h_last=None, workspace=None, return_last_state=True, stream=None):
+    """Selective scan through ssm_scan_fwd of libssmscan.so.
+
+    x, delta, z: (batch, L, dim); B, C: (batch, L, N) -- all float32 or all
+    bfloat16. A: (dim, N), D and delta_bias: (dim,), h0: (batch, dim, N),
+    float32. Returns (y, h_last); h_last is None when not requested."""
+    if x.dim() != 3:
+        raise ValueError("x must be (batch, seqlen, dim)")
+    batch, L, dim = x.shape
+    if A.dim() != 2 or A.shape[0] != dim:
+        raise ValueError("A must be (dim, dstate)")
+    N = A.shape[1]
+    dev = x.device
+    io = _io_code(x.dtype)
+    bld, bln = (batch, L, dim), (batch, L, N)
+    args_io = [_ptr(x, "x", x.dtype, bld), _ptr(delta, "delta", x.dtype, bld, dev)]
+    pA = _ptr(A, "A", torch.float32, (dim, N), dev)
+    pB = _ptr(B, "B", x.dtype, bln, dev)
+    pC = _ptr(C, "C", x.dtype, bln, dev)
+    pD = _ptr(D, "D", torch.float32, (dim,), dev)
+    pz = _ptr(z, "z", x.dtype, bld, dev)
+    pbias = _ptr(delta_bias, "delta_bias", torch.float32, (dim,), dev)
+    ph0 = _ptr(h0, "h0", torch.float32, (batch, dim, N), dev)
+    if y is None:
+        y = torch.empty(bld, dtype=x.dtype, device=dev)
+    py = _ptr(y, "y", x.dtype, bld, dev)
+    if h_last is None and return_last_state:
+        h_last = torch.empty((batch, dim, N), dtype=torch.float32, device=dev)
+    ph = _ptr(h_last, "h_last", torch.float32, (batch, dim, N), dev)
+    with torch.cuda.device(dev):
+        need = scan_workspace_bytes(batch, L, dim, N, x.dtype)
+        if workspace is None:
+            workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+        pws = _ptr(workspace, "workspace", None, None, dev)
+        rc = lib().ssm_scan_fwd(batch, L, dim, N, io, args_io[0], args_io[1], pA, pB, pC, pD, pz,
+                                pbias, 1 if softplus else 0, ph0, py, ph, pws,
+                                workspace.numel() * workspace.element_size(),
+                                _stream_ptr(stream, dev))
+    if rc != 0:
+        raise SsmError(rc, "ssm_scan_fwd")
+    return y, h_last
+
+
+def ssm_scan_status(workspace, batch, seqlen, dim, dstate, dtype=torch.bfloat16, stream=None):
+    """Synchronise the stream and return the status code of the last scan that
+    used `workspace` (0 = every CTA finished; -5 = a bounded wait timed out)."""
+    dev = workspace.device
+    with torch.cuda.device(dev):
+        return int(lib().ssm_scan_status(workspace.data_ptr(),
+                                         workspace.numel() * workspace.element_size(), batch,
+                                         seqlen, dim, dstate, _io_code(dtype),
+                                         _stream_ptr(stream, dev)))
+
+
+def ssm_state_update(state, x, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
+                     y=None, stream=None):
+    """One decode step through ssm_state_update of libssmscan.so; updates the
+    float32 state (batch, dim, N) in place and returns y (batch, dim)."""
+    if state.dim() != 3:
+        raise ValueError("state must be (batch, dim, dstate)")
+    batch, dim, N = state.shape
+    dev = state.device
+    io = _io_code(x.dtype)
+    bd, bn = (batch, dim), (batch, N)
+    ps = _ptr(state, "state", torch.float32, (batch, dim, N))
+    px = _ptr(x, "x", x.dtype, bd, dev)
+    pdl = _ptr(delta, "delta", x.dtype, bd, dev)
+    pA = _ptr(A, "A", torch.float32, (dim, N), dev)
+    pB = _ptr(B, "B", x.dtype, bn, dev)
+    pC = _ptr(C, "C", x.dtype, bn, dev)
+    pD = _ptr(D, "D", torch.float32, (dim,), dev)
+    pz = _ptr(z, "z", x.dtype, bd, dev)
+    pbias = _ptr(delta_bias, "delta_bias", torch.float32, (dim,), dev)
+    if y is None:
+        y = torch.empty(bd, dtype=x.dtype, device=dev)
+    py = _ptr(y, "y", x.dtype, bd, dev)
+    with torch.cuda.device(dev):
+        rc = lib().ssm_state_update(batch, dim, N, io, ps, px, pdl, pA, pB, pC, pD, pz, pbias,
+                                    1 if softplus else 0, py, _stream_ptr(stream, dev))
+    if rc != 0:
+        raise SsmError(rc, "ssm_state_update")
+    return y

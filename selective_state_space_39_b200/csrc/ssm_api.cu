@@ -1,0 +1,323 @@
+// ssm_api.cu -- the extern "C" entry points declared in include/ssm_scan.h:
+// argument validation (on the host, before anything is enqueued), the
+// sequence-segment plan, TMA tensor-map encoding and kernel launch.
+#include <stdlib.h>
+#include <string.h>
+
+#include <algorithm>
+
+#include "../../include/ssm_scan.h"
+#include "ssm_internal.h"
+
+namespace ssm {
+
+int scan_channels_per_thread(int dstate);
+
+namespace {
+
+constexpr int kVersion = 10000;  // 1.0.0
+
+struct Dims {
+  int64_t batch, seqlen, dim, dstate;
+  int io;
+};
+
+size_t io_bytes(int io) { return io == SSM_DTYPE_BF16 ? 2 : 4; }
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+  if (!a || !b || na == 0 || nb == 0) return false;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + nb && b0 < a0 + na;
+}
+
+int dims_status(const Dims& d) {
+  if (d.io != SSM_DTYPE_F32 && d.io != SSM_DTYPE_BF16) return SSM_ERR_UNSUPPORTED;
+  if (d.batch < 0 || d.seqlen < 0 || d.dim < 0) return SSM_ERR_INVALID_ARG;
+  if (d.dstate <= 0) return SSM_ERR_INVALID_ARG;
+  if (!scan_dstate_supported((int)std::min<int64_t>(d.dstate, 1 << 20))) return SSM_ERR_UNSUPPORTED;
+  // grid and index limits of this build
+  if (d.batch > 65535 || d.dim > (1 << 24) || d.seqlen > (1 << 30)) return SSM_ERR_UNSUPPORTED;
+  return SSM_OK;
+}
+
+int device_sms() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      sms <= 0) {
+    cudaGetLastError();  // clear: no device is not an error for planning
+    return 148;          // B200
+  }
+  return sms;
+}
+
+long env_long(const char* name, long dflt) {
+  const char* v = getenv(name);
+  if (!v || !*v) return dflt;
+  char* end = nullptr;
+  const long r = strtol(v, &end, 10);
+  return (end && *end == '\0') ? r : dflt;
+}
+
+// Split of the sequence into segments: enough CTAs for about
+// `ctas_per_sm` resident CTAs on every SM, in whole tiles.
+ScanPlan make_plan(const Dims& d) {
+  ScanPlan pl{};
+  const int T = kScanTileSteps;
+  pl.channels_per_thread = scan_channels_per_thread((int)d.dstate);
+  pl.dtile = kScanThreads * pl.channels_per_thread;
+  pl.dtiles = (int)std::max<int64_t>(1, (d.dim + pl.dtile - 1) / pl.dtile);
+  const int64_t tiles = std::max<int64_t>(1, (d.seqlen + T - 1) / T);
+  const int64_t cols = std::max<int64_t>(1, d.batch * pl.dtiles);
+  const long per_sm = std::max(1L, env_long("SSM_SCAN_CTAS_PER_SM", 4));
+  int64_t nseg = std::max<int64_t>(1, (int64_t)device_sms() * per_sm / cols);
+  const long forced = env_long("SSM_SCAN_SEGMENTS", 0);
+  if (forced > 0) nseg = forced;
+  nseg = std::min<int64_t>(std::min<int64_t>(nseg, tiles), 65535);
+  const int64_t tiles_per_seg = (tiles + nseg - 1) / nseg;
+  pl.seg_steps = (int)(tiles_per_seg * T);
+  pl.nseg = (int)((tiles + tiles_per_seg - 1) / tiles_per_seg);
+  pl.ctas_agg = pl.nseg > 1 ? (int)(d.batch * (pl.nseg - 1) * pl.dtiles) : 0;
+  pl.ctas_main = (int)(d.batch * pl.nseg * pl.dtiles);
+  size_t off = 0;
+  pl.off_status = off;
+  off = align_up(off + sizeof(int) * (size_t)(pl.ctas_agg + pl.ctas_main), 256);
+  const size_t nagg = (size_t)(pl.nseg - 1);
+  pl.off_state = off;
+  off = align_up(off + sizeof(float) * (size_t)d.batch * nagg * d.dstate * d.dim, 256);
+  pl.off_sum = off;
+  off = align_up(off + sizeof(float) * (size_t)d.batch * nagg * d.dim, 256);
+  pl.off_h0 = off;
+  if (pl.nseg > 1) off = align_up(off + sizeof(float) * (size_t)d.batch * d.dim * d.dstate, 256);
+  pl.bytes = off;
+  return pl;
+}
+
+// --- TMA tensor maps --------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// 3-D map over a (batch, rows, cols) row-major tensor with a box of
+// (1, box_rows, box_cols); out-of-range elements read as zero.
+bool encode_3d(CUtensorMap* map, const void* base, int io, int64_t batch, int64_t rows,
+               int64_t cols, int box_rows, int box_cols) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const size_t es = io_bytes(io);
+  const cuuint64_t gdim[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)batch};
+  const cuuint64_t gstride[2] = {(cuuint64_t)(cols * es), (cuuint64_t)(rows * cols * es)};
+  const cuuint32_t box[3] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows, 1};
+  const cuuint32_t estride[3] = {1, 1, 1};
+  const CUtensorMapDataType dt =
+      io == SSM_DTYPE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  const CUresult r = fn(map, dt, 3, const_cast<void*>(base), gdim, gstride, box, estride,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// TMA needs 16-byte aligned bases and 16-byte multiples for row strides.
+bool tma_eligible(const Dims& d, const void* x, const void* delta, const void* z, const void* B,
+                  const void* C) {
+  if (env_long("SSM_SCAN_DISABLE_TMA", 0) != 0) return false;
+  const size_t es = io_bytes(d.io);
+  if ((d.dim * es) % 16 != 0 || (d.dstate * es) % 16 != 0) return false;
+  if (!aligned(x, 16) || !aligned(delta, 16) || !aligned(B, 16) || !aligned(C, 16)) return false;
+  if (z && !aligned(z, 16)) return false;
+  if (d.seqlen <= 0 || d.dim <= 0 || d.batch <= 0) return false;
+  return encode_fn() != nullptr;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? SSM_OK : SSM_ERR_CUDA; }
+
+}  // namespace
+}  // namespace ssm
+
+using namespace ssm;
+
+extern "C" {
+
+int ssm_scan_version(void) { return kVersion; }
+
+const char* ssm_status_string(int status) {
+  switch (status) {
+    case SSM_OK: return "ok";
+    case SSM_ERR_INVALID_ARG: return "invalid argument";
+    case SSM_ERR_UNSUPPORTED: return "unsupported size or dtype";
+    case SSM_ERR_WORKSPACE: return "workspace missing or too small";
+    case SSM_ERR_CUDA: return "CUDA error";
+    case SSM_ERR_TIMEOUT: return "a kernel wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int ssm_scan_plan(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate, int io_dtype,
+                  ssm_scan_plan_t* out) {
+  const Dims d{batch, seqlen, dim, dstate, io_dtype};
+  const int st = dims_status(d);
+  if (st != SSM_OK) return st;
+  if (!out) return SSM_ERR_INVALID_ARG;
+  const ScanPlan pl = make_plan(d);
+  out->segments = pl.nseg;
+  out->segment_steps = pl.seg_steps;
+  out->channel_tiles = pl.dtiles;
+  out->channels_per_cta = pl.dtile;
+  out->ctas_carry = pl.ctas_agg;
+  out->ctas_main = pl.ctas_main;
+  out->kernels = (batch > 0 && dim > 0) ? (pl.nseg > 1 ? 2 : 1) : 0;
+  out->workspace_bytes = (int64_t)pl.bytes;
+  return SSM_OK;
+}
+
+size_t ssm_scan_workspace_bytes(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
+                                int io_dtype) {
+  const Dims d{batch, seqlen, dim, dstate, io_dtype};
+  if (dims_status(d) != SSM_OK) return 0;
+  return make_plan(d).bytes;
+}
+
+int ssm_scan_fwd(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate, int io_dtype,
+                 const void* x, const void* delta, const float* A, const void* B,
+                 const void* C, const float* D, const void* z, const float* delta_bias,
+                 int softplus, const float* h0, void* y, float* h_last, void* workspace,
+                 size_t workspace_bytes, void* stream) {
+  const Dims d{batch, seqlen, dim, dstate, io_dtype};
+  int st = dims_status(d);
+  if (st != SSM_OK) return st;
+  if (batch == 0 || dim == 0) return SSM_OK;
+  const size_t es = io_bytes(io_dtype);
+  const size_t n_bld = (size_t)batch * seqlen * dim, n_bln = (size_t)batch * seqlen * dstate;
+  // required pointers and element alignment
+  if (!A) return SSM_ERR_INVALID_ARG;
+  if (seqlen > 0 && (!x || !delta || !B || !C || !y)) return SSM_ERR_INVALID_ARG;
+  const void* io_ptrs[] = {x, delta, B, C, z, y};
+  for (const void* p : io_ptrs)
+    if (p && !aligned(p, es)) return SSM_ERR_INVALID_ARG;
+  const void* f32_ptrs[] = {A, D, delta_bias};
+  for (const void* p : f32_ptrs)
+    if (p && !aligned(p, 4)) return SSM_ERR_INVALID_ARG;
+  if ((h0 && !aligned(h0, 8)) || (h_last && !aligned(h_last, 8))) return SSM_ERR_INVALID_ARG;
+  // y must not overlap an input
+  const size_t by = n_bld * es;
+  if (overlap(y, by, x, n_bld * es) || overlap(y, by, delta, n_bld * es) ||
+      overlap(y, by, z, n_bld * es) || overlap(y, by, B, n_bln * es) ||
+      overlap(y, by, C, n_bln * es))
+    return SSM_ERR_INVALID_ARG;
+  const ScanPlan pl = make_plan(d);
+  if (pl.bytes > 0 && (!workspace || workspace_bytes < pl.bytes || !aligned(workspace, 16)))
+    return SSM_ERR_WORKSPACE;
+
+  ScanParams p{};
+  p.batch = (int)batch;
+  p.seqlen = (int)seqlen;
+  p.dim = (int)dim;
+  p.nseg = pl.nseg;
+  p.seg_steps = pl.seg_steps;
+  p.softplus = softplus ? 1 : 0;
+  p.pair_store = (dim % 2) == 0;
+  p.x = x; p.delta = delta; p.z = z; p.B = B; p.C = C;
+  p.A = A; p.D = D; p.bias = delta_bias; p.h0 = h0;
+  p.y = y; p.h_last = h_last;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  p.status = reinterpret_cast<int*>(ws + pl.off_status);
+  p.ws_state = reinterpret_cast<float*>(ws + pl.off_state);
+  p.ws_sum = reinterpret_cast<float*>(ws + pl.off_sum);
+  p.ws_h0 = reinterpret_cast<float*>(ws + pl.off_h0);
+  p.wait_limit_ns = (uint64_t)std::max(1L, env_long("SSM_SCAN_WAIT_LIMIT_NS",
+                                                    (long)kDefaultWaitLimitNs));
+
+  const bool use_tma = tma_eligible(d, x, delta, z, B, C);
+  ScanMaps maps;
+  memset(&maps, 0, sizeof maps);
+  if (use_tma) {
+    const int T = kScanTileSteps, DT = pl.dtile;
+    bool ok = encode_3d(&maps.x, x, io_dtype, batch, seqlen, dim, T, DT) &&
+              encode_3d(&maps.delta, delta, io_dtype, batch, seqlen, dim, T, DT) &&
+              encode_3d(&maps.B, B, io_dtype, batch, seqlen, dstate, T, (int)dstate) &&
+              encode_3d(&maps.C, C, io_dtype, batch, seqlen, dstate, T, (int)dstate);
+    if (ok && z) ok = encode_3d(&maps.z, z, io_dtype, batch, seqlen, dim, T, DT);
+    if (!ok) return SSM_ERR_CUDA;
+  }
+  st = cuda_status(launch_scan(pl, p, use_tma ? &maps : nullptr, use_tma, (int)dstate,
+                               io_dtype == SSM_DTYPE_BF16, static_cast<cudaStream_t>(stream)));
+  return st;
+}
+
+int ssm_scan_status(const void* workspace, size_t workspace_bytes, int64_t batch,
+                    int64_t seqlen, int64_t dim, int64_t dstate, int io_dtype, void* stream) {
+  const Dims d{batch, seqlen, dim, dstate, io_dtype};
+  int st = dims_status(d);
+  if (st != SSM_OK) return st;
+  if (batch == 0 || dim == 0) return SSM_OK;
+  const ScanPlan pl = make_plan(d);
+  if (!workspace || workspace_bytes < pl.bytes) return SSM_ERR_WORKSPACE;
+  const int n = pl.ctas_agg + pl.ctas_main;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SSM_ERR_CUDA;
+  int buf[1024];
+  const unsigned char* ws = static_cast<const unsigned char*>(workspace) + pl.off_status;
+  for (int i = 0; i < n; i += 1024) {
+    const int m = std::min(1024, n - i);
+    if (cudaMemcpy(buf, ws + sizeof(int) * (size_t)i, sizeof(int) * (size_t)m,
+                   cudaMemcpyDeviceToHost) != cudaSuccess)
+      return SSM_ERR_CUDA;
+    for (int k = 0; k < m; ++k)
+      if (buf[k] != kCtaOk) return SSM_ERR_TIMEOUT;
+  }
+  return SSM_OK;
+}
+
+int ssm_state_update(int64_t batch, int64_t dim, int64_t dstate, int io_dtype, float* state,
+                     const void* x, const void* delta, const float* A, const void* B,
+                     const void* C, const float* D, const void* z, const float* delta_bias,
+                     int softplus, void* y, void* stream) {
+  const Dims d{batch, 1, dim, dstate, io_dtype};
+  int st = dims_status(d);
+  if (st != SSM_OK) return st;
+  if (batch == 0 || dim == 0) return SSM_OK;
+  if (!state || !x || !delta || !A || !B || !C || !y) return SSM_ERR_INVALID_ARG;
+  const size_t es = io_bytes(io_dtype);
+  const void* io_ptrs[] = {x, delta, B, C, z, y};
+  for (const void* p : io_ptrs)
+    if (p && !aligned(p, es)) return SSM_ERR_INVALID_ARG;
+  const void* f32_ptrs[] = {A, D, delta_bias};
+  for (const void* p : f32_ptrs)
+    if (p && !aligned(p, 4)) return SSM_ERR_INVALID_ARG;
+  if (!aligned(state, dstate % 4 == 0 ? 16 : 8)) return SSM_ERR_INVALID_ARG;
+  const size_t nbd = (size_t)batch * dim, nbn = (size_t)batch * dstate;
+  const size_t by = nbd * es;
+  if (overlap(y, by, x, nbd * es) || overlap(y, by, delta, nbd * es) ||
+      overlap(y, by, z, nbd * es) || overlap(y, by, B, nbn * es) || overlap(y, by, C, nbn * es) ||
+      overlap(y, by, state, nbd * dstate * sizeof(float)))
+    return SSM_ERR_INVALID_ARG;
+  DecodeParams p{};
+  p.batch = (int)batch;
+  p.dim = (int)dim;
+  p.softplus = softplus ? 1 : 0;
+  p.state = state;
+  p.x = x; p.delta = delta; p.z = z; p.B = B; p.C = C;
+  p.A = A; p.D = D; p.bias = delta_bias; p.y = y;
+  return cuda_status(launch_decode(p, (int)dstate, io_dtype == SSM_DTYPE_BF16,
+                                   static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

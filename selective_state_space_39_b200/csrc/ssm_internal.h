@@ -1,0 +1,84 @@
+// ssm_internal.h -- parameters shared by the C entry points (ssm_api.cu) and
+// the kernel launchers (ssm_scan_kernels.cu). Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace ssm {
+
+// Launch shape of the scan: threads per CTA and sequence steps per tile.
+constexpr int kScanThreads = 128;
+constexpr int kScanTileSteps = 16;
+constexpr int kScanStages = 2;
+// Per-CTA status codes written to the workspace status area.
+constexpr int kCtaOk = 0;
+constexpr int kCtaTimeout = 1;
+// Default bound on any wait inside a kernel (nanoseconds).
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;
+
+// How one call of the scan is split: the sequence is cut into `nseg`
+// segments of `seg_steps` steps (a multiple of kScanTileSteps); segment
+// carries live in the caller's workspace.
+struct ScanPlan {
+  int channels_per_thread;  // 2 for dstate <= 16, 1 above
+  int dtile;                // channels per CTA
+  int dtiles;               // CTAs along dim
+  int nseg;                 // sequence segments
+  int seg_steps;            // steps per segment
+  int ctas_agg;             // CTAs of the carry pass (0 when nseg == 1)
+  int ctas_main;            // CTAs of the main pass
+  size_t off_status, off_state, off_sum, off_h0, bytes;
+};
+
+struct ScanParams {
+  int batch, seqlen, dim;
+  int nseg, seg_steps;
+  int softplus;
+  int pair_store;  // dim even: two-channel vector stores are aligned
+  const void* x;
+  const void* delta;
+  const void* z;
+  const void* B;
+  const void* C;
+  const float* A;
+  const float* D;
+  const float* bias;
+  const float* h0;  // caller's h0 (read only when nseg == 1)
+  void* y;
+  float* h_last;
+  float* ws_state;  // [batch][nseg-1][N][dim]
+  float* ws_sum;    // [batch][nseg-1][dim]
+  float* ws_h0;     // [batch][dim][N] copy of h0 taken by the carry pass
+  int* status;      // one int per CTA: carry-pass CTAs first, then main pass
+  uint64_t wait_limit_ns;
+};
+
+struct alignas(64) ScanMaps {
+  CUtensorMap x, delta, z, B, C;
+};
+
+struct DecodeParams {
+  int batch, dim;
+  int softplus;
+  float* state;
+  const void* x;
+  const void* delta;
+  const void* z;
+  const void* B;
+  const void* C;
+  const float* A;
+  const float* D;
+  const float* bias;
+  void* y;
+};
+
+// Kernel launchers (ssm_scan_kernels.cu). Return a cudaError_t.
+cudaError_t launch_scan(const ScanPlan& plan, const ScanParams& p, const ScanMaps* maps,
+                        bool use_tma, int dstate, bool bf16, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeParams& p, int dstate, bool bf16, cudaStream_t stream);
+bool scan_dstate_supported(int dstate);
+
+}  // namespace ssm

@@ -1,0 +1,630 @@
+// ssm_scan_kernels.cu -- sm_100a kernels of the selective state-space scan.
+//
+// What is computed (page "Mamba 논문 리뷰: Selective State Space Models로
+// Transformer를 넘어서", youngju.dev; §2.2 discretised recurrence, §3.1
+// softplus step, §3.3 selective_scan, §3.4 D skip and SiLU(z) gate):
+//   Delta_t = softplus(delta_t + bias),  a_n(t) = exp(Delta_t A_n)
+//   h_n(t)  = a_n(t) h_n(t-1) + Delta_t x_t B_n(t)
+//   y_t     = (sum_n C_n(t) h_n(t) + D x_t) * SiLU(z_t)
+//
+// Design (B200): the path is bound by FP32 arithmetic, not by memory, at
+// dstate = 16 (about 60 FP32 operations per 8 bytes moved), so the kernels
+// are built to minimise FP32 pipe work per element:
+//
+//  * Each thread owns CPT (2) channels and their whole state in registers;
+//    state pairs are updated with packed FP32x2 FMAs.
+//  * Structured A (A[d,n] = (n+1) A[d,0], which Mamba's A = -exp(log(
+//    arange(1, N+1))) init gives) is detected per channel from A itself;
+//    then a_n = r^(n+1) with r = exp(Delta A_0): one exp and a multiply
+//    chain instead of N exps. Other A falls back to one exp per state.
+//  * Scaled recurrence. With s_t ~ Delta_t x_t (never zero, see below) the
+//    state is kept as g_n = h_n / s_t, so that
+//        g_n(t) = (a_n(t) s_{t-1}/s_t) g_n(t-1) + B_n(t),   y_t = s_t sum_n C_n g_n
+//    costs one multiply (the chain of alpha_n = s_{t-1}/s_t r^(n+1)) and two
+//    FMAs per state, instead of two multiplies and two FMAs. s_t is Delta_t x_t
+//    plus copysign(2^-64); the computed state therefore follows the exact
+//    recurrence with Delta_t x_t replaced by s_t, |s_t - Delta_t x_t| <= 2^-64.
+//  * B and C (shared by all channels of a step) are widened to fp32 once per
+//    CTA in shared memory and read as broadcasts.
+//  * x, delta, z, B, C tiles of 16 steps are staged in shared memory by TMA
+//    (cp.async.bulk.tensor, no multicast) through a 2-stage mbarrier
+//    pipeline; every wait is bounded by a time limit.
+//  * The sequence is split into segments so the whole GPU is busy: a carry
+//    pass computes each segment's end state from a zero start (and the sum
+//    of Delta, which gives the segment's decay exp(A_n sum Delta)), and the
+//    main pass composes those affine carries ((a1,b1) then (a2,b2) ->
+//    (a1 a2, a2 b1 + b2), the associative scan of the state update) in its
+//    prologue before running its own segment exactly from the true start.
+//
+// bf16 io uses MUFU approximations (ex2/lg2/rcp/tanh.approx); fp32 io uses
+// the accurate expf / log1pf / IEEE division.
+#include <type_traits>
+
+#include "ssm_device.cuh"
+#include "ssm_internal.h"
+
+namespace ssm {
+
+namespace {
+
+constexpr int round_up(int v, int m) { return (v + m - 1) / m * m; }
+
+template <typename IOT, int N, int CPT, int NT, int T>
+struct ScanLayout {
+  static constexpr int DT = NT * CPT;
+  static constexpr int kTileBytes = T * DT * (int)sizeof(IOT);
+  static constexpr int kBCBytes = T * N * (int)sizeof(IOT);
+  static constexpr int kOffX = 0;
+  static constexpr int kOffD = kTileBytes;
+  static constexpr int kOffZ = 2 * kTileBytes;
+  static constexpr int kOffB = 3 * kTileBytes;
+  static constexpr int kOffC = kOffB + round_up(kBCBytes, 128);
+  static constexpr int kStageBytes = kOffC + round_up(kBCBytes, 128);
+  // fp32 copies of B (pre-scaled) and C for the tile: [2 buffers][2][T][N]
+  static constexpr int kBCF32Bytes = 2 * 2 * T * N * 4;
+};
+
+template <typename IOT, int N, int CPT, int NT, int T, int STAGES>
+constexpr int scan_smem_bytes() {
+  using L = ScanLayout<IOT, N, CPT, NT, T>;
+  return STAGES * L::kStageBytes + L::kBCF32Bytes + 8 * STAGES;
+}
+
+// Per-channel constants.
+struct Chan {
+  float A0;     // A[d,0] (natural units)
+  float bias;   // fast path: bias * log2(e); precise path: bias
+  float Dd;     // skip weight
+  bool valid;   // d < dim
+};
+
+// -------------------------------------------------------------------------
+// The scan kernel. kAgg = carry pass (segments 0..nseg-2: end state and
+// sum of Delta, no output); !kAgg = main pass (all segments, y and h_last).
+// Grid: (dtiles, segments, batch). Block: NT threads, CPT channels each.
+template <typename IOT, int N, int CPT, int NT, int T, int STAGES, bool kAgg, bool kTma>
+__global__ void __launch_bounds__(NT) scan_kernel(const ScanParams p,
+                                                  const __grid_constant__ ScanMaps maps) {
+  using IO = Io<IOT>;
+  using L = ScanLayout<IOT, N, CPT, NT, T>;
+  constexpr bool kFast = std::is_same<IOT, uint16_t>::value;
+  constexpr int DT = L::DT;
+  constexpr int NP = N / 2;
+  static_assert(N % 2 == 0, "dstate must be even");
+
+  extern __shared__ __align__(128) unsigned char smem[];
+  float* bcf = reinterpret_cast<float*>(smem + STAGES * L::kStageBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * L::kStageBytes + L::kBCF32Bytes);
+
+  const int tid = threadIdx.x;
+  const int dtile = blockIdx.x, seg = blockIdx.y, b = blockIdx.z;
+  const int dim = p.dim, L_ = p.seqlen;
+  const int d_local = tid * CPT;
+  const int d_first = dtile * DT + d_local;
+  const bool has_z = !kAgg && p.z != nullptr;
+  const int t_begin = seg * p.seg_steps;
+  const int t_end = min(t_begin + p.seg_steps, L_);
+  const int ntiles = t_end > t_begin ? (t_end - t_begin + T - 1) / T : 0;
+
+  const uint32_t stage_tx = (uint32_t)((kAgg ? 2 : (has_z ? 3 : 2)) * L::kTileBytes +
+                                       (kAgg ? 1 : 2) * L::kBCBytes);
+
+  auto issue_tile = [&](int it) {
+    unsigned char* st = smem + (it % STAGES) * L::kStageBytes;
+    uint64_t* bar = &full[it % STAGES];
+    const int t0 = t_begin + it * T;
+    mbar_arrive_expect_tx(bar, stage_tx);
+    tma_load_3d(st + L::kOffX, &maps.x, bar, dtile * DT, t0, b);
+    tma_load_3d(st + L::kOffD, &maps.delta, bar, dtile * DT, t0, b);
+    if (has_z) tma_load_3d(st + L::kOffZ, &maps.z, bar, dtile * DT, t0, b);
+    tma_load_3d(st + L::kOffB, &maps.B, bar, 0, t0, b);
+    if (!kAgg) tma_load_3d(st + L::kOffC, &maps.C, bar, 0, t0, b);
+  };
+
+  int issued = 0;  // tiles whose loads were issued (thread 0 only)
+  bool aborted = false;
+  if (tid == 0) {
+    if constexpr (kTma) {
+      prefetch_tensormap(&maps.x);
+      prefetch_tensormap(&maps.delta);
+      prefetch_tensormap(&maps.B);
+      if (!kAgg) prefetch_tensormap(&maps.C);
+      if (has_z) prefetch_tensormap(&maps.z);
+      for (int s = 0; s < STAGES; ++s) mbar_init(&full[s], 1);
+      fence_mbar_init();
+    }
+  }
+  __syncthreads();
+  if constexpr (kTma) {
+    if (tid == 0)
+      for (; issued < STAGES - 1 && issued < ntiles; ++issued) issue_tile(issued);
+  }
+
+  // ---- per-channel constants and structure of A ------------------------
+  Chan ch[CPT];
+  bool structured = true;
+#pragma unroll
+  for (int c = 0; c < CPT; ++c) {
+    const int d = d_first + c;
+    ch[c].valid = d < dim;
+    if (ch[c].valid) {
+      const float* Ar = p.A + (size_t)d * N;
+      ch[c].A0 = Ar[0];
+#pragma unroll
+      for (int n = 1; n < N; ++n) structured = structured && (Ar[n] == (float)(n + 1) * Ar[0]);
+      const float bias = p.bias ? p.bias[d] : 0.f;
+      ch[c].bias = kFast ? bias * kLog2e : bias;
+      ch[c].Dd = p.D ? p.D[d] : 0.f;
+    } else {
+      ch[c].A0 = -1.f;
+      ch[c].bias = 0.f;
+      ch[c].Dd = 0.f;
+    }
+  }
+
+  // ---- initial state ----------------------------------------------------
+  float2 g[CPT][NP];  // scaled state g = h / s_prev
+  float s_prev[CPT];
+  float qsum[CPT];
+#pragma unroll
+  for (int c = 0; c < CPT; ++c) {
+    s_prev[c] = 1.f;
+    qsum[c] = 0.f;
+#pragma unroll
+    for (int k = 0; k < NP; ++k) g[c][k] = make_float2(0.f, 0.f);
+  }
+  {
+    const int nagg = p.nseg - 1;
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) {
+      if (!ch[c].valid) continue;
+      const int d = d_first + c;
+      if constexpr (kAgg) {
+        // Segment 0 starts from h0 and keeps a copy of it for the main pass
+        // (so that h_last may alias h0); later segments start from zero.
+        if (seg == 0 && p.h0) {
+          const float2* src = reinterpret_cast<const float2*>(p.h0 + ((size_t)b * dim + d) * N);
+          float2* cpy = reinterpret_cast<float2*>(p.ws_h0 + ((size_t)b * dim + d) * N);
+#pragma unroll
+          for (int k = 0; k < NP; ++k) {
+            g[c][k] = src[k];
+            cpy[k] = g[c][k];
+          }
+        }
+      } else {
+        const float* h0 = p.nseg > 1 ? (p.h0 ? p.ws_h0 : nullptr) : p.h0;
+        if (seg > 0) {
+          // inclusive end state of segment 0, then compose segments 1..seg-1
+          const float* st0 = p.ws_state + ((size_t)b * nagg) * N * dim + d;
+#pragma unroll
+          for (int k = 0; k < NP; ++k)
+            g[c][k] = make_float2(st0[(size_t)(2 * k) * dim], st0[(size_t)(2 * k + 1) * dim]);
+          for (int j = 1; j < seg; ++j) {
+            const float sd = p.ws_sum[((size_t)b * nagg + j) * dim + d];
+            const float* stj = p.ws_state + ((size_t)b * nagg + j) * N * dim + d;
+            if (structured) {
+              const float e = expf(ch[c].A0 * sd);
+              float en = e;
+#pragma unroll
+              for (int k = 0; k < NP; ++k) {
+                const float e0 = en, e1 = en * e;
+                en = e1 * e;
+                g[c][k].x = fmaf(e0, g[c][k].x, stj[(size_t)(2 * k) * dim]);
+                g[c][k].y = fmaf(e1, g[c][k].y, stj[(size_t)(2 * k + 1) * dim]);
+              }
+            } else {
+              const float* Ar = p.A + (size_t)d * N;
+#pragma unroll
+              for (int k = 0; k < NP; ++k) {
+                g[c][k].x = fmaf(expf(Ar[2 * k] * sd), g[c][k].x, stj[(size_t)(2 * k) * dim]);
+                g[c][k].y =
+                    fmaf(expf(Ar[2 * k + 1] * sd), g[c][k].y, stj[(size_t)(2 * k + 1) * dim]);
+              }
+            }
+          }
+        } else if (h0) {
+          const float2* src = reinterpret_cast<const float2*>(h0 + ((size_t)b * dim + d) * N);
+#pragma unroll
+          for (int k = 0; k < NP; ++k) g[c][k] = src[k];
+        }
+      }
+    }
+  }
+
+  // ---- tile loop ----------------------------------------------------------
+  const bool pair_store = CPT == 2 && p.pair_store;
+  for (int it = 0; it < ntiles; ++it) {
+    const int buf = it & 1;
+    unsigned char* st;
+    if constexpr (kTma) {
+      st = smem + (it % STAGES) * L::kStageBytes;
+      const bool ok = mbar_wait_bounded(&full[it % STAGES], (uint32_t)((it / STAGES) & 1),
+                                        p.wait_limit_ns);
+      if (__syncthreads_or(!ok)) {
+        aborted = true;  // uniform across the CTA
+        // Let the loads already issued land (bounded) before the CTA's
+        // shared memory is released.
+        if (tid == 0)
+          for (int j = it; j < issued; ++j)
+            (void)mbar_wait_bounded(&full[j % STAGES], (uint32_t)((j / STAGES) & 1), 1000000ull);
+        break;
+      }
+    } else {
+      st = smem;
+      __syncthreads();  // every thread is done with the previous tile
+      const int t0 = t_begin + it * T;
+      const IOT* gx = reinterpret_cast<const IOT*>(p.x);
+      const IOT* gd = reinterpret_cast<const IOT*>(p.delta);
+      const IOT* gz = reinterpret_cast<const IOT*>(p.z);
+      IOT* sx = reinterpret_cast<IOT*>(st + L::kOffX);
+      IOT* sd = reinterpret_cast<IOT*>(st + L::kOffD);
+      IOT* sz = reinterpret_cast<IOT*>(st + L::kOffZ);
+      for (int i = tid; i < T * DT; i += NT) {
+        const int tt = t0 + i / DT, dd = dtile * DT + i % DT;
+        const bool in = tt < L_ && dd < dim;
+        const size_t gi = ((size_t)b * L_ + tt) * dim + dd;
+        sx[i] = in ? gx[gi] : IOT(0);
+        sd[i] = in ? gd[gi] : IOT(0);
+        if (has_z) sz[i] = in ? gz[gi] : IOT(0);
+      }
+      const IOT* gb = reinterpret_cast<const IOT*>(p.B);
+      const IOT* gc = reinterpret_cast<const IOT*>(p.C);
+      IOT* sb = reinterpret_cast<IOT*>(st + L::kOffB);
+      IOT* sc = reinterpret_cast<IOT*>(st + L::kOffC);
+      for (int i = tid; i < T * N; i += NT) {
+        const int tt = t0 + i / N;
+        const size_t gi = ((size_t)b * L_ + tt) * N + i % N;
+        sb[i] = tt < L_ ? gb[gi] : IOT(0);
+        if (!kAgg) sc[i] = tt < L_ ? gc[gi] : IOT(0);
+      }
+      __syncthreads();
+    }
+
+    // widen B (times ln2 on the fast path, see below) and C to fp32
+    {
+      const IOT* sb = reinterpret_cast<const IOT*>(st + L::kOffB);
+      const IOT* sc = reinterpret_cast<const IOT*>(st + L::kOffC);
+      float* fb = bcf + (buf * 2 + 0) * T * N;
+      float* fc = bcf + (buf * 2 + 1) * T * N;
+      const float bscale = kFast ? kLn2 : 1.f;
+      for (int i = tid; i < T * N; i += NT) {
+        fb[i] = IO::load(sb + i) * bscale;
+        if (!kAgg) fc[i] = IO::load(sc + i);
+      }
+    }
+    __syncthreads();
+    if constexpr (kTma) {
+      // The stage consumed by the previous tile is free: refill it.
+      if (tid == 0 && issued < ntiles) issue_tile(issued++);
+    }
+
+    const IOT* sx = reinterpret_cast<const IOT*>(st + L::kOffX) + d_local;
+    const IOT* sdl = reinterpret_cast<const IOT*>(st + L::kOffD) + d_local;
+    const IOT* sz = reinterpret_cast<const IOT*>(st + L::kOffZ) + d_local;
+    const float* fb = bcf + (buf * 2 + 0) * T * N;
+    const float* fc = bcf + (buf * 2 + 1) * T * N;
+    const int t0 = t_begin + it * T;
+    const int steps = min(T, t_end - t0);
+
+    for (int ss = 0; ss < steps; ++ss) {
+      float xv[CPT], dv[CPT], zv[CPT];
+      if constexpr (CPT == 2) {
+        const float2 x2 = IO::load2(sx + ss * DT), d2 = IO::load2(sdl + ss * DT);
+        xv[0] = x2.x; xv[1] = x2.y; dv[0] = d2.x; dv[1] = d2.y;
+        if (has_z) {
+          const float2 z2 = IO::load2(sz + ss * DT);
+          zv[0] = z2.x; zv[1] = z2.y;
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) {
+          xv[c] = IO::load(sx + ss * DT + c);
+          dv[c] = IO::load(sdl + ss * DT + c);
+          if (has_z) zv[c] = IO::load(sz + ss * DT + c);
+        }
+      }
+      const float* Bt = fb + ss * N;
+      const float* Ct = fc + ss * N;
+      float yv[CPT];
+#pragma unroll
+      for (int c = 0; c < CPT; ++c) {
+        // Step size. Fast path works in log2 units: q = Delta * log2(e).
+        float q, r;
+        if constexpr (kFast) {
+          const float v = fmaf(dv[c], kLog2e, ch[c].bias);
+          q = p.softplus ? (v > kSoftplusCut * kLog2e ? v : lg2_approx(1.f + ex2_approx(v))) : v;
+          r = ex2_approx(q * ch[c].A0);  // exp(Delta A0)
+        } else {
+          const float v = dv[c] + ch[c].bias;
+          q = p.softplus ? (v > kSoftplusCut ? v : log1pf(expf(v))) : v;
+          r = expf(q * ch[c].A0);
+        }
+        // s = Delta x in the path's units (fast: times log2 e, matched by
+        // B pre-scaled by ln 2), kept away from zero.
+        float s = q * xv[c];
+        s = s + copysignf(kScaleFloor, s);
+        const float rho = kFast ? s_prev[c] * rcp_approx(s) : s_prev[c] / s;
+        s_prev[c] = s;
+        if constexpr (kAgg) qsum[c] += q;
+
+        float2 acc = make_float2(0.f, 0.f);
+        if (structured) {
+          const float a0 = rho * r;
+          const float r2 = r * r;
+          float2 a = make_float2(a0, a0 * r);
+          const float2 rr = make_float2(r2, r2);
+          if constexpr (N % 4 == 0) {
+            const float4* B4 = reinterpret_cast<const float4*>(Bt);
+            const float4* C4 = reinterpret_cast<const float4*>(Ct);
+#pragma unroll
+            for (int k = 0; k < N / 4; ++k) {
+              const float4 bq = B4[k];
+              g[c][2 * k] = fma2(a, g[c][2 * k], make_float2(bq.x, bq.y));
+              a = mul2(a, rr);
+              g[c][2 * k + 1] = fma2(a, g[c][2 * k + 1], make_float2(bq.z, bq.w));
+              a = mul2(a, rr);
+              if constexpr (!kAgg) {
+                const float4 cq = C4[k];
+                acc = fma2(make_float2(cq.x, cq.y), g[c][2 * k], acc);
+                acc = fma2(make_float2(cq.z, cq.w), g[c][2 * k + 1], acc);
+              }
+            }
+          } else {
+            const float2* B2 = reinterpret_cast<const float2*>(Bt);
+            const float2* C2 = reinterpret_cast<const float2*>(Ct);
+#pragma unroll
+            for (int k = 0; k < NP; ++k) {
+              g[c][k] = fma2(a, g[c][k], B2[k]);
+              a = mul2(a, rr);
+              if constexpr (!kAgg) acc = fma2(C2[k], g[c][k], acc);
+            }
+          }
+        } else {
+          const float* Ar = p.A + (size_t)(ch[c].valid ? d_first + c : 0) * N;
+          const float2* B2 = reinterpret_cast<const float2*>(Bt);
+          const float2* C2 = reinterpret_cast<const float2*>(Ct);
+#pragma unroll
+          for (int k = 0; k < NP; ++k) {
+            float2 a;
+            if constexpr (kFast) {
+              a = make_float2(rho * ex2_approx(q * __ldg(Ar + 2 * k)),
+                              rho * ex2_approx(q * __ldg(Ar + 2 * k + 1)));
+            } else {
+              a = make_float2(rho * expf(q * __ldg(Ar + 2 * k)),
+                              rho * expf(q * __ldg(Ar + 2 * k + 1)));
+            }
+            g[c][k] = fma2(a, g[c][k], B2[k]);
+            if constexpr (!kAgg) acc = fma2(C2[k], g[c][k], acc);
+          }
+        }
+        if constexpr (!kAgg) {
+          float yy = fmaf(s, acc.x + acc.y, ch[c].Dd * xv[c]);
+          if (has_z) {
+            if constexpr (kFast) {
+              const float hz = 0.5f * zv[c];
+              yy *= fmaf(hz, tanh_approx(hz), hz);  // z * sigmoid(z)
+            } else {
+              yy *= zv[c] / (1.f + expf(-zv[c]));
+            }
+          }
+          yv[c] = yy;
+        }
+      }
+      if constexpr (!kAgg) {
+        IOT* yrow = reinterpret_cast<IOT*>(p.y) + ((size_t)b * L_ + (t0 + ss)) * dim + d_first;
+        if (pair_store && ch[CPT - 1].valid) {
+          IO::store2(yrow, yv[0], yv[CPT - 1]);
+        } else {
+#pragma unroll
+          for (int c = 0; c < CPT; ++c)
+            if (ch[c].valid) IO::store(yrow + c, yv[c]);
+        }
+      }
+    }
+  }
+
+  // ---- outputs of the segment ------------------------------------------
+  if (!aborted) {
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) {
+      if (!ch[c].valid) continue;
+      const int d = d_first + c;
+      if constexpr (kAgg) {
+        const int nagg = p.nseg - 1;
+        p.ws_sum[((size_t)b * nagg + seg) * dim + d] = kFast ? qsum[c] * kLn2 : qsum[c];
+        float* dst = p.ws_state + ((size_t)b * nagg + seg) * N * dim + d;
+#pragma unroll
+        for (int k = 0; k < NP; ++k) {
+          dst[(size_t)(2 * k) * dim] = s_prev[c] * g[c][k].x;
+          dst[(size_t)(2 * k + 1) * dim] = s_prev[c] * g[c][k].y;
+        }
+      } else if (p.h_last && seg == p.nseg - 1) {
+        float2* dst = reinterpret_cast<float2*>(p.h_last + ((size_t)b * dim + d) * N);
+        const float2 sp = make_float2(s_prev[c], s_prev[c]);
+#pragma unroll
+        for (int k = 0; k < NP; ++k) dst[k] = mul2(sp, g[c][k]);
+      }
+    }
+  }
+  if (tid == 0 && p.status) {
+    const int ctas_agg = kAgg ? 0 : (p.nseg > 1 ? p.batch * (p.nseg - 1) * (int)gridDim.x : 0);
+    const int id = ctas_agg + (b * (int)gridDim.y + seg) * (int)gridDim.x + dtile;
+    p.status[id] = aborted ? kCtaTimeout : kCtaOk;
+  }
+}
+
+// -------------------------------------------------------------------------
+// Decode: one step of the recurrence per (batch, channel). LPC lanes share a
+// channel, SPT states each; y is reduced across the LPC lanes by shuffles.
+template <typename IOT, int N>
+__global__ void __launch_bounds__(256) decode_kernel(const DecodeParams p) {
+  using IO = Io<IOT>;
+  constexpr bool kFast = std::is_same<IOT, uint16_t>::value;
+  constexpr int SPT = (N % 4 == 0) ? 4 : 2;
+  constexpr int LPC = N / SPT;
+  static_assert(LPC <= 32 && (LPC & (LPC - 1)) == 0, "lanes per channel must divide a warp");
+  const size_t gtid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const size_t chan = gtid / LPC;  // b * dim + d
+  const int lane_in = (int)(gtid % LPC);
+  const size_t nchan = (size_t)p.batch * p.dim;
+  const bool valid = chan < nchan;
+  const size_t cc = valid ? chan : 0;
+  const int b = (int)(cc / p.dim), d = (int)(cc % p.dim);
+
+  const float xv = IO::load(reinterpret_cast<const IOT*>(p.x) + cc);
+  const float v = IO::load(reinterpret_cast<const IOT*>(p.delta) + cc) + (p.bias ? p.bias[d] : 0.f);
+  float dt;
+  if (!p.softplus) {
+    dt = v;
+  } else if constexpr (kFast) {
+    dt = v > kSoftplusCut ? v : kLn2 * lg2_approx(1.f + ex2_approx(v * kLog2e));
+  } else {
+    dt = v > kSoftplusCut ? v : log1pf(expf(v));
+  }
+  const float dx = dt * xv;
+  float* hp = p.state + cc * N + lane_in * SPT;
+  const float* Ar = p.A + (size_t)d * N + lane_in * SPT;
+  const IOT* Bp = reinterpret_cast<const IOT*>(p.B) + (size_t)b * N + lane_in * SPT;
+  const IOT* Cp = reinterpret_cast<const IOT*>(p.C) + (size_t)b * N + lane_in * SPT;
+  float h[SPT];
+  if constexpr (SPT == 4) {
+    const float4 t4 = *reinterpret_cast<const float4*>(hp);
+    h[0] = t4.x; h[1] = t4.y; h[2] = t4.z; h[3] = t4.w;
+  } else {
+    const float2 t2 = *reinterpret_cast<const float2*>(hp);
+    h[0] = t2.x; h[1] = t2.y;
+  }
+  float acc = 0.f;
+#pragma unroll
+  for (int k = 0; k < SPT; ++k) {
+    const float a = kFast ? ex2_approx(dt * Ar[k] * kLog2e) : expf(dt * Ar[k]);
+    h[k] = fmaf(a, h[k], dx * IO::load(Bp + k));
+    acc = fmaf(IO::load(Cp + k), h[k], acc);
+  }
+#pragma unroll
+  for (int off = LPC / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (!valid) return;
+  if constexpr (SPT == 4) {
+    *reinterpret_cast<float4*>(hp) = make_float4(h[0], h[1], h[2], h[3]);
+  } else {
+    *reinterpret_cast<float2*>(hp) = make_float2(h[0], h[1]);
+  }
+  if (lane_in == 0) {
+    float yy = acc + (p.D ? p.D[d] : 0.f) * xv;
+    if (p.z) {
+      const float zz = IO::load(reinterpret_cast<const IOT*>(p.z) + cc);
+      if constexpr (kFast) {
+        const float hz = 0.5f * zz;
+        yy *= fmaf(hz, tanh_approx(hz), hz);
+      } else {
+        yy *= zz / (1.f + expf(-zz));
+      }
+    }
+    IO::store(reinterpret_cast<IOT*>(p.y) + cc, yy);
+  }
+}
+
+// -------------------------------------------------------------------------
+// cudaFuncSetAttribute once per kernel and device (up to 64 devices).
+template <typename K>
+cudaError_t ensure_smem_attr(K kernel, int smem) {
+  static unsigned long long done = 0ull;  // bit per device, set after success
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = dev < 64 ? (1ull << dev) : 0ull;
+  if (bit && (__atomic_load_n(&done, __ATOMIC_ACQUIRE) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess && bit) __atomic_fetch_or(&done, bit, __ATOMIC_RELEASE);
+  return e;
+}
+
+template <typename IOT, int N, int CPT>
+cudaError_t launch_scan_t(const ScanPlan& plan, const ScanParams& p, const ScanMaps* maps,
+                          bool use_tma, cudaStream_t stream) {
+  constexpr int NT = kScanThreads, T = kScanTileSteps, S = kScanStages;
+  static const ScanMaps none{};
+  const ScanMaps& m = maps ? *maps : none;
+  const dim3 block(NT);
+  cudaError_t err = cudaSuccess;
+  auto run = [&](auto kernel, int smem, dim3 grid) -> cudaError_t {
+    cudaError_t e = ensure_smem_attr(kernel, smem);
+    if (e != cudaSuccess) return e;
+    kernel<<<grid, block, smem, stream>>>(p, m);
+    return cudaGetLastError();
+  };
+  if (use_tma) {
+    constexpr int smem = scan_smem_bytes<IOT, N, CPT, NT, T, S>();
+    if (plan.nseg > 1) {
+      err = run(scan_kernel<IOT, N, CPT, NT, T, S, true, true>, smem,
+                dim3(plan.dtiles, plan.nseg - 1, p.batch));
+      if (err != cudaSuccess) return err;
+    }
+    return run(scan_kernel<IOT, N, CPT, NT, T, S, false, true>, smem,
+               dim3(plan.dtiles, plan.nseg, p.batch));
+  }
+  constexpr int smem = scan_smem_bytes<IOT, N, CPT, NT, T, 1>();
+  if (plan.nseg > 1) {
+    err = run(scan_kernel<IOT, N, CPT, NT, T, 1, true, false>, smem,
+              dim3(plan.dtiles, plan.nseg - 1, p.batch));
+    if (err != cudaSuccess) return err;
+  }
+  return run(scan_kernel<IOT, N, CPT, NT, T, 1, false, false>, smem,
+             dim3(plan.dtiles, plan.nseg, p.batch));
+}
+
+template <typename IOT>
+cudaError_t launch_scan_io(const ScanPlan& plan, const ScanParams& p, const ScanMaps* maps,
+                           bool use_tma, int dstate, cudaStream_t stream) {
+  switch (dstate) {
+    case 2: return launch_scan_t<IOT, 2, 2>(plan, p, maps, use_tma, stream);
+    case 4: return launch_scan_t<IOT, 4, 2>(plan, p, maps, use_tma, stream);
+    case 8: return launch_scan_t<IOT, 8, 2>(plan, p, maps, use_tma, stream);
+    case 16: return launch_scan_t<IOT, 16, 2>(plan, p, maps, use_tma, stream);
+    case 32: return launch_scan_t<IOT, 32, 1>(plan, p, maps, use_tma, stream);
+    case 64: return launch_scan_t<IOT, 64, 1>(plan, p, maps, use_tma, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <typename IOT>
+cudaError_t launch_decode_io(const DecodeParams& p, int dstate, cudaStream_t stream) {
+  const size_t chans = (size_t)p.batch * p.dim;
+  auto go = [&](auto kernel, int lpc) -> cudaError_t {
+    const size_t threads = chans * lpc;
+    const unsigned blocks = (unsigned)((threads + 255) / 256);
+    kernel<<<blocks, 256, 0, stream>>>(p);
+    return cudaGetLastError();
+  };
+  switch (dstate) {
+    case 2: return go(decode_kernel<IOT, 2>, 1);
+    case 4: return go(decode_kernel<IOT, 4>, 1);
+    case 8: return go(decode_kernel<IOT, 8>, 2);
+    case 16: return go(decode_kernel<IOT, 16>, 4);
+    case 32: return go(decode_kernel<IOT, 32>, 8);
+    case 64: return go(decode_kernel<IOT, 64>, 16);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+bool scan_dstate_supported(int dstate) {
+  return dstate == 2 || dstate == 4 || dstate == 8 || dstate == 16 || dstate == 32 ||
+         dstate == 64;
+}
+
+int scan_channels_per_thread(int dstate) { return dstate <= 16 ? 2 : 1; }
+
+cudaError_t launch_scan(const ScanPlan& plan, const ScanParams& p, const ScanMaps* maps,
+                        bool use_tma, int dstate, bool bf16, cudaStream_t stream) {
+  return bf16 ? launch_scan_io<uint16_t>(plan, p, maps, use_tma, dstate, stream)
+              : launch_scan_io<float>(plan, p, maps, use_tma, dstate, stream);
+}
+
+cudaError_t launch_decode(const DecodeParams& p, int dstate, bool bf16, cudaStream_t stream) {
+  return bf16 ? launch_decode_io<uint16_t>(p, dstate, stream)
+              : launch_decode_io<float>(p, dstate, stream);
+}
+
+}  // namespace ssm

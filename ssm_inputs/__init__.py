@@ -208,28 +208,33 @@ def delta_bias(dim, seed, nthreads=None):
 
 
 def make_scan_inputs(batch, seqlen, dim, dstate, io, seed, *, gate=True, skip=True,
-                     with_h0=False, nthreads=None):
+                     with_h0=False, nthreads=None, batch_offset=0):
     """All inputs of one scan, as numpy arrays (io tensors as float32, or as
-    uint16 bf16 bits when io == "bf16")."""
+    uint16 bf16 bits when io == "bf16"). ``batch_offset`` selects rows
+    batch_offset .. batch_offset+batch of a larger global batch (the values
+    of a row do not depend on how the batch is split)."""
     bld, bln = (batch, seqlen, dim), (batch, seqlen, dstate)
+    o_ld, o_ln, o_dn = (batch_offset * seqlen * dim, batch_offset * seqlen * dstate,
+                        batch_offset * dim * dstate)
     out = {
-        "x": fill(bld, seed, STREAM_X, out=io, nthreads=nthreads),
-        "delta": fill(bld, seed, STREAM_DELTA, b=0.5, out=io, nthreads=nthreads),
-        "B": fill(bln, seed, STREAM_B, out=io, nthreads=nthreads),
-        "C": fill(bln, seed, STREAM_C, out=io, nthreads=nthreads),
-        "z": fill(bld, seed, STREAM_Z, out=io, nthreads=nthreads) if gate else None,
+        "x": fill(bld, seed, STREAM_X, out=io, offset=o_ld, nthreads=nthreads),
+        "delta": fill(bld, seed, STREAM_DELTA, b=0.5, out=io, offset=o_ld, nthreads=nthreads),
+        "B": fill(bln, seed, STREAM_B, out=io, offset=o_ln, nthreads=nthreads),
+        "C": fill(bln, seed, STREAM_C, out=io, offset=o_ln, nthreads=nthreads),
+        "z": fill(bld, seed, STREAM_Z, out=io, offset=o_ld, nthreads=nthreads) if gate else None,
         "A": a_matrix(dim, dstate),
         "D": np.ones(dim, dtype=np.float32) if skip else None,
         "delta_bias": delta_bias(dim, seed, nthreads),
-        "h0": (fill((batch, dim, dstate), seed, STREAM_H0, out="f32", nthreads=nthreads)
-               if with_h0 else None),
+        "h0": (fill((batch, dim, dstate), seed, STREAM_H0, out="f32", offset=o_dn,
+                    nthreads=nthreads) if with_h0 else None),
     }
     return out
 
 
-def workload_inputs(w: ScanWorkload, nthreads=None):
-    return make_scan_inputs(w.batch, w.seqlen, w.dim, w.dstate, w.io, w.seed, gate=w.gate,
-                            skip=w.skip, with_h0=w.with_h0, nthreads=nthreads)
+def workload_inputs(w: ScanWorkload, nthreads=None, batch=None, batch_offset=0):
+    return make_scan_inputs(w.batch if batch is None else batch, w.seqlen, w.dim, w.dstate,
+                            w.io, w.seed, gate=w.gate, skip=w.skip, with_h0=w.with_h0,
+                            nthreads=nthreads, batch_offset=batch_offset)
 
 
 def make_decode_inputs(batch, dim, dstate, io, seed, step, nthreads=None):

@@ -1,0 +1,153 @@
+"""The C-ABI library on the host (no GPU work): it loads, exports every entry
+point include/ssm_scan.h declares, and rejects bad arguments before anything
+is enqueued. Every call here with fake pointers is one the library must
+reject on the host; none of them can reach a kernel launch."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ssm_scan.h")
+
+from selective_state_space_39_b200 import _binding as bnd  # noqa: E402
+
+
+@pytest.fixture(scope="module")
+def L():
+    from selective_state_space_39_b200 import build
+    build.build()
+    return bnd.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ssm_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for want in ["ssm_scan_fwd", "ssm_state_update", "ssm_scan_workspace_bytes",
+                 "ssm_scan_plan", "ssm_scan_status", "ssm_status_string", "ssm_scan_version"]:
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), f"libssmscan.so does not export {name}"
+
+
+def test_version_and_status_strings(L):
+    assert L.ssm_scan_version() >= 10000
+    assert L.ssm_status_string(0) == b"ok"
+    assert L.ssm_status_string(-1) == b"invalid argument"
+    assert L.ssm_status_string(-5) == b"a kernel wait timed out"
+    assert L.ssm_status_string(12345) == b"unknown status"
+
+
+def test_plan_splits_long_sequences(L):
+    p = bnd.ScanPlan()
+    assert L.ssm_scan_plan(1, 262144, 1536, 16, 1, ctypes.byref(p)) == 0
+    assert p.segments > 1 and p.segment_steps % 16 == 0
+    assert (p.segments - 1) * p.segment_steps < 262144 <= p.segments * p.segment_steps
+    assert p.kernels == 2 and p.channels_per_cta == 256 and p.channel_tiles == 6
+    assert p.ctas_main == p.segments * 6 and p.ctas_carry == (p.segments - 1) * 6
+    assert p.workspace_bytes == L.ssm_scan_workspace_bytes(1, 262144, 1536, 16, 1)
+    q = bnd.ScanPlan()
+    assert L.ssm_scan_plan(1, 1, 64, 16, 0, ctypes.byref(q)) == 0
+    assert q.segments == 1 and q.kernels == 1
+
+
+def test_plan_respects_forced_segments(L, monkeypatch):
+    monkeypatch.setenv("SSM_SCAN_SEGMENTS", "3")
+    p = bnd.ScanPlan()
+    assert L.ssm_scan_plan(2, 100, 64, 16, 0, ctypes.byref(p)) == 0
+    assert p.segments == 3 and p.segment_steps == 48
+    monkeypatch.setenv("SSM_SCAN_SEGMENTS", "1000")
+    assert L.ssm_scan_plan(2, 100, 64, 16, 0, ctypes.byref(p)) == 0
+    assert p.segments == 7 and p.segment_steps == 16  # at most one segment per 16-step tile
+
+
+def test_unsupported_sizes(L):
+    p = bnd.ScanPlan()
+    assert L.ssm_scan_plan(1, 8, 8, 3, 0, ctypes.byref(p)) == -2   # odd dstate
+    assert L.ssm_scan_plan(1, 8, 8, 128, 0, ctypes.byref(p)) == -2  # above 64
+    assert L.ssm_scan_plan(1, 8, 8, 16, 7, ctypes.byref(p)) == -2   # io dtype
+    assert L.ssm_scan_plan(-1, 8, 8, 16, 0, ctypes.byref(p)) == -1
+    assert L.ssm_scan_plan(1, 8, 8, 0, 0, ctypes.byref(p)) == -1
+    assert L.ssm_scan_workspace_bytes(1, 8, 8, 3, 0) == 0
+
+
+FAKE = 1 << 20  # an aligned address that is never dereferenced: every call below is rejected first
+# Fake-pointer calls run only on machines without a GPU, so that a regression
+# in host-side validation can never turn one into a kernel launch.
+no_gpu_only = pytest.mark.skipif(torch.cuda.is_available(),
+                                 reason="fake-pointer validation tests run only without a GPU")
+
+
+def scan(L, **kw):
+    a = dict(batch=2, seqlen=32, dim=64, dstate=16, io=1, x=FAKE, delta=FAKE + 4096,
+             A=FAKE + 8192, B=FAKE + 12288, C=FAKE + 16384, D=None, z=None, bias=None, sp=1,
+             h0=None, y=FAKE + 65536 * 4, h_last=None, ws=None, ws_bytes=0, stream=None)
+    a.update(kw)
+    return L.ssm_scan_fwd(a["batch"], a["seqlen"], a["dim"], a["dstate"], a["io"], a["x"],
+                          a["delta"], a["A"], a["B"], a["C"], a["D"], a["z"], a["bias"], a["sp"],
+                          a["h0"], a["y"], a["h_last"], a["ws"], a["ws_bytes"], a["stream"])
+
+
+@no_gpu_only
+def test_scan_rejects_bad_arguments(L):
+    assert scan(L, x=None) == -1
+    assert scan(L, A=None) == -1
+    assert scan(L, y=None) == -1
+    assert scan(L, x=FAKE + 1) == -1            # misaligned bf16
+    assert scan(L, io=0, B=FAKE + 12290) == -1  # misaligned fp32
+    assert scan(L, h0=FAKE + 4) == -1           # h0 needs 8-byte alignment
+    assert scan(L, y=FAKE + 2) == -1            # y overlaps x
+    assert scan(L, dstate=5) == -2
+    assert scan(L, seqlen=-3) == -1
+    assert scan(L) == -3                        # no workspace
+    need = L.ssm_scan_workspace_bytes(2, 32, 64, 16, 1)
+    assert scan(L, ws=FAKE * 64, ws_bytes=need - 1) == -3
+    assert scan(L, ws=FAKE * 64 + 8, ws_bytes=need) == -3  # workspace not 16-byte aligned
+    assert scan(L, batch=0) == 0 and scan(L, dim=0) == 0   # empty problems do nothing
+
+
+@no_gpu_only
+def test_state_update_rejects_bad_arguments(L):
+    def upd(**kw):
+        a = dict(batch=4, dim=64, dstate=16, io=1, state=FAKE, x=FAKE + 65536, delta=FAKE + 69632,
+                 A=FAKE + 73728, B=FAKE + 81920, C=FAKE + 86016, D=None, z=None, bias=None, sp=1,
+                 y=FAKE + 131072, stream=None)
+        a.update(kw)
+        return L.ssm_state_update(a["batch"], a["dim"], a["dstate"], a["io"], a["state"], a["x"],
+                                  a["delta"], a["A"], a["B"], a["C"], a["D"], a["z"], a["bias"],
+                                  a["sp"], a["y"], a["stream"])
+    assert upd(state=None) == -1
+    assert upd(state=FAKE + 8) == -1   # state needs 16-byte alignment for dstate % 4 == 0
+    assert upd(y=FAKE + 65536) == -1   # y overlaps x
+    assert upd(y=FAKE + 64) == -1      # y overlaps the state
+    assert upd(dstate=7) == -2
+    assert upd(C=None) == -1
+    assert upd(batch=0) == 0
+
+
+def test_binding_has_no_cpu_path():
+    from selective_state_space_39_b200 import ssm_scan_fwd
+    x = torch.zeros(1, 4, 8)
+    A = torch.zeros(8, 16)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        ssm_scan_fwd(x, x, A, torch.zeros(1, 4, 16), torch.zeros(1, 4, 16))
+
+
+def test_product_never_imports_the_oracle():
+    pkg = os.path.join(ROOT, "selective_state_space_39_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"^\s*(import|from)\s+oracle\b", text, re.M), f
+                assert "ssm_oracle" not in text and "liboracle" not in text, f

@@ -1,0 +1,225 @@
+"""GPU parity: the CUDA scan (through the C ABI) against the fp64 oracle.
+
+Bound (max|y - y_ref| / max|y_ref|, same for h_last): 1e-5 for fp32 io,
+1e-2 for bf16 io with fp32 state. Full-size workloads are checked on sampled
+channels (every step of each sampled channel), plus properties that hold at
+any size (no NaN/Inf, TMA path == plain-load path bit for bit)."""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import ssm_inputs as gen
+from tests.gpu_util import TOL, dev, gpu_scan, host, oracle_scan, rel_err, sample_channels
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _clean_env(monkeypatch):
+    for k in ("SSM_SCAN_SEGMENTS", "SSM_SCAN_DISABLE_TMA", "SSM_SCAN_CTAS_PER_SM",
+              "SSM_SCAN_WAIT_LIMIT_NS"):
+        monkeypatch.delenv(k, raising=False)
+    yield
+
+
+def _check(y, hl, yr, hr, io, what):
+    ey, eh = rel_err(y, yr), rel_err(hl, hr)
+    print(f"{what}: rel err y {ey:.3e}  h_last {eh:.3e}")
+    assert np.all(np.isfinite(y)) and np.all(np.isfinite(hl)), what
+    assert ey <= TOL[io], f"{what}: y rel err {ey:.3e} > {TOL[io]}"
+    assert eh <= TOL[io], f"{what}: h_last rel err {eh:.3e} > {TOL[io]}"
+
+
+# ---------------------------------------------------------------- workloads
+@pytest.mark.parametrize("segments", [None, "1", "3", "16"])
+def test_tiny_f32_workload_full(monkeypatch, segments):
+    if segments:
+        monkeypatch.setenv("SSM_SCAN_SEGMENTS", segments)
+    w = gen.SCAN_WORKLOADS["tiny_f32_b1_l256_d64"]
+    inp = gen.workload_inputs(w)
+    y, hl = gpu_scan(inp)
+    yr, hr = oracle_scan(inp, "f32")
+    _check(host(y), host(hl), yr, hr, "f32", f"tiny f32 segments={segments}")
+
+
+def _sampled_workload(name, nchan_per_batch=12):
+    w = gen.SCAN_WORKLOADS[name]
+    inp = gen.workload_inputs(w)
+    y, hl = gpu_scan(inp)
+    torch.cuda.synchronize()
+    assert torch.isfinite(y).all() and torch.isfinite(hl).all()
+    chans = sample_channels(w.batch, w.dim, nchan_per_batch)
+    yr, hr = oracle_scan(inp, w.io, channels=chans)
+    yg = host(y)
+    hg = host(hl)
+    ys = np.stack([yg[b, :, d] for b, d in chans])
+    hs = np.stack([hg[b, d] for b, d in chans])
+    _check(ys, hs, yr, hr, w.io, f"{name} ({len(chans)} channels)")
+    return inp, y, hl
+
+
+def test_mamba130m_layer_sampled():
+    inp, y, hl = _sampled_workload("mamba130m_layer_b8_l2048_d1536")
+
+
+def test_pythia1b_layer_with_h0_sampled():
+    _sampled_workload("pythia1b_layer_b4_l4096_d4096_h0", 8)
+
+
+def test_long_256k_sampled():
+    _sampled_workload("long_b1_l262144_d1536", 10)
+
+
+def test_tma_and_plain_paths_bitwise_equal(monkeypatch):
+    """Both loading paths feed the same arithmetic: outputs are identical."""
+    inp = gen.make_scan_inputs(3, 700, 1024, 16, "bf16", 7, with_h0=True)
+    y1, h1 = gpu_scan(inp)
+    monkeypatch.setenv("SSM_SCAN_DISABLE_TMA", "1")
+    y2, h2 = gpu_scan(inp)
+    assert torch.equal(y1, y2) and torch.equal(h1, h2)
+
+
+# ----------------------------------------------------------------- edge cases
+CASES = [
+    # batch, L, dim, N, io
+    (1, 1, 64, 16, "f32"),
+    (2, 17, 40, 16, "bf16"),     # ragged L and a partial channel tile
+    (1, 100, 300, 16, "f32"),    # dim not a multiple of the 256-channel tile
+    (2, 50, 33, 16, "f32"),      # odd dim: plain-load path, scalar stores
+    (2, 45, 36, 16, "bf16"),     # dim*2 bytes not a multiple of 16: plain-load path
+    (1, 64, 64, 2, "f32"),
+    (1, 64, 64, 4, "bf16"),
+    (2, 64, 64, 8, "f32"),
+    (1, 80, 96, 32, "f32"),
+    (1, 48, 64, 64, "bf16"),
+    (1, 64, 64, 64, "f32"),
+]
+
+
+def _case_inputs(batch, L, dim, N, io, seed, *, h0=True, gate=True, skip=True, bias=True,
+                 generic_A=False):
+    inp = gen.make_scan_inputs(batch, L, dim, N, io, seed, gate=gate, skip=skip, with_h0=h0)
+    if generic_A:
+        rng = np.random.default_rng(seed)
+        inp["A"] = (-rng.uniform(0.1, 4.0, (dim, N))).astype(np.float32)
+    if not bias:
+        inp["delta_bias"] = None
+    return inp
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "b%d_l%d_d%d_n%d_%s" % c)
+@pytest.mark.parametrize("segments", ["1", "4"])
+def test_edge_shapes(monkeypatch, case, segments):
+    monkeypatch.setenv("SSM_SCAN_SEGMENTS", segments)
+    batch, L, dim, N, io = case
+    inp = _case_inputs(batch, L, dim, N, io, seed=batch * 1000 + L + dim + N)
+    y, hl = gpu_scan(inp)
+    yr, hr = oracle_scan(inp, io)
+    _check(host(y), host(hl), yr, hr, io, f"{case} seg={segments}")
+
+
+FLAGS = [
+    dict(h0=False),
+    dict(gate=False),
+    dict(skip=False),
+    dict(bias=False),
+    dict(softplus=False),
+    dict(generic_A=True),
+    dict(generic_A=True, h0=False, gate=False),
+]
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("flags", FLAGS, ids=lambda f: "-".join(f"{k}={v}" for k, v in f.items()))
+def test_optional_terms(monkeypatch, io, flags):
+    monkeypatch.setenv("SSM_SCAN_SEGMENTS", "3")
+    flags = dict(flags)
+    softplus = flags.pop("softplus", True)
+    inp = _case_inputs(2, 200, 512, 16, io, seed=5, **flags)
+    if not softplus:
+        # keep Delta positive without softplus: delta + bias in [0.01, 0.3]
+        rng = np.random.default_rng(9)
+        d = rng.uniform(0.01, 0.3, inp["x"].shape).astype(np.float32)
+        inp["delta"] = gen.f32_to_bf16_bits(d) if io == "bf16" else d
+        inp["delta_bias"] = None
+    y, hl = gpu_scan(inp, softplus=softplus)
+    yr, hr = oracle_scan(inp, io, softplus=softplus)
+    _check(host(y), host(hl), yr, hr, io, f"{io} {flags} softplus={softplus}")
+
+
+def test_seqlen_zero_returns_h0():
+    inp = gen.make_scan_inputs(2, 0, 64, 16, "f32", 3, with_h0=True)
+    y, hl = gpu_scan(inp)
+    assert y.numel() == 0
+    assert torch.equal(hl.cpu(), torch.from_numpy(inp["h0"]))
+    inp["h0"] = None
+    _, hl = gpu_scan(inp)
+    assert torch.count_nonzero(hl).item() == 0
+
+
+@pytest.mark.parametrize("segments", ["1", "5"])
+def test_h_last_may_alias_h0(monkeypatch, segments):
+    monkeypatch.setenv("SSM_SCAN_SEGMENTS", segments)
+    from selective_state_space_39_b200 import ssm_scan_fwd
+    inp = gen.make_scan_inputs(2, 300, 512, 16, "bf16", 11, with_h0=True)
+    h = dev(inp["h0"]).clone()
+    y, hl = ssm_scan_fwd(dev(inp["x"]), dev(inp["delta"]), dev(inp["A"]), dev(inp["B"]),
+                         dev(inp["C"]), D=dev(inp["D"]), z=dev(inp["z"]),
+                         delta_bias=dev(inp["delta_bias"]), h0=h, h_last=h)
+    assert hl.data_ptr() == h.data_ptr()
+    yr, hr = oracle_scan(inp, "bf16")
+    _check(host(y), host(hl), yr, hr, "bf16", "aliased h0/h_last")
+
+
+def test_split_invariance_on_gpu(monkeypatch):
+    """scan(L1) then scan(L2, h0 = h_last) matches scan(L1 + L2)."""
+    monkeypatch.setenv("SSM_SCAN_SEGMENTS", "4")
+    inp = gen.make_scan_inputs(2, 640, 512, 16, "f32", 13, with_h0=True)
+    y, hl = gpu_scan(inp)
+    k = 272
+    first = {key: (v[:, :k] if key in ("x", "delta", "z", "B", "C") else v) for key, v in inp.items()}
+    second = {key: (v[:, k:] if key in ("x", "delta", "z", "B", "C") else v) for key, v in inp.items()}
+    y1, h1 = gpu_scan(first)
+    second["h0"] = h1.cpu().numpy()
+    y2, h2 = gpu_scan(second)
+    assert rel_err(host(y1), host(y)[:, :k]) <= 1e-5
+    assert rel_err(host(y2), host(y)[:, k:]) <= 1e-5
+    assert rel_err(host(h2), host(hl)) <= 1e-5
+
+
+def test_outputs_stay_in_bounds():
+    """Guard bands around y and h_last keep their sentinel values."""
+    from selective_state_space_39_b200 import ssm_scan_fwd
+    inp = gen.make_scan_inputs(3, 77, 520, 16, "bf16", 17, with_h0=True)
+    pad = 4096
+    n_y = 3 * 77 * 520
+    ybuf = torch.full((n_y + 2 * pad,), 7.0, dtype=torch.bfloat16, device="cuda")
+    hbuf = torch.full((3 * 520 * 16 + 2 * pad,), 7.0, dtype=torch.float32, device="cuda")
+    y = ybuf[pad:pad + n_y].view(3, 77, 520)
+    hl = hbuf[pad:pad + 3 * 520 * 16].view(3, 520, 16)
+    ssm_scan_fwd(dev(inp["x"]), dev(inp["delta"]), dev(inp["A"]), dev(inp["B"]), dev(inp["C"]),
+                 D=dev(inp["D"]), z=dev(inp["z"]), delta_bias=dev(inp["delta_bias"]),
+                 h0=dev(inp["h0"]), y=y, h_last=hl)
+    torch.cuda.synchronize()
+    for buf in (ybuf, hbuf):
+        assert torch.all(buf[:pad] == 7.0) and torch.all(buf[-pad:] == 7.0)
+    yr, hr = oracle_scan(inp, "bf16")
+    _check(host(y), host(hl), yr, hr, "bf16", "guard bands")
+
+
+def test_status_reports_ok():
+    from selective_state_space_39_b200 import scan_workspace_bytes, ssm_scan_status
+    inp = gen.make_scan_inputs(2, 500, 768, 16, "bf16", 19)
+    ws = torch.empty(scan_workspace_bytes(2, 500, 768, 16, torch.bfloat16), dtype=torch.uint8,
+                     device="cuda")
+    gpu_scan(inp, workspace=ws)
+    assert ssm_scan_status(ws, 2, 500, 768, 16, torch.bfloat16) == 0
+
+
+def test_repeated_calls_are_deterministic():
+    inp = gen.make_scan_inputs(2, 300, 1024, 16, "bf16", 23, with_h0=True)
+    y1, h1 = gpu_scan(inp)
+    y2, h2 = gpu_scan(inp)
+    assert torch.equal(y1, y2) and torch.equal(h1, h2)
