@@ -154,6 +154,14 @@ int ssm_scan_status(const void* workspace, size_t workspace_bytes, int64_t batch
 /* ssm_status_string -- static, human-readable text for an SSM_* code. */
 const char* ssm_status_string(int status);
 
+/*
+ * ssm_last_error_detail -- text describing the last SSM_ERR_CUDA /
+ * SSM_ERR_TIMEOUT failure on the calling host thread (which CUDA call failed
+ * and its error name); "" if none. The pointer stays valid until the next
+ * failing call on this thread.
+ */
+const char* ssm_last_error_detail(void);
+
 /* ssm_scan_version -- library version as MAJOR*10000 + MINOR*100 + PATCH. */
 int ssm_scan_version(void);
 

@@ -24,7 +24,11 @@ _STATUS = {0: "ok", -1: "invalid argument", -2: "unsupported size or dtype",
 class SsmError(RuntimeError):
     def __init__(self, code: int, where: str):
         self.code = code
-        super().__init__(f"{where}: {_STATUS.get(code, 'unknown status')} ({code})")
+        detail = ""
+        if code in (-4, -5) and _lib is not None:
+            detail = _lib.ssm_last_error_detail().decode(errors="replace")
+        msg = f"{where}: {_STATUS.get(code, 'unknown status')} ({code})"
+        super().__init__(msg + (f": {detail}" if detail else ""))
 
 
 class ScanPlan(ctypes.Structure):
@@ -40,10 +44,12 @@ _I64 = ctypes.c_int64
 
 
 def lib() -> ctypes.CDLL:
-    """Load libssmscan.so from the package directory (raises if absent)."""
+    """Load libssmscan.so from the package directory, or the build named by
+    $SSM_SCAN_LIBRARY (raises if absent)."""
     global _lib
     if _lib is None:
-        path = _build.LIB_PATH
+        # SSM_SCAN_LIBRARY may point at another build of the same library
+        path = os.environ.get("SSM_SCAN_LIBRARY") or _build.LIB_PATH
         if not os.path.exists(path):
             raise RuntimeError(
                 f"{path} is missing: build it with `python -m selective_state_space_39_b200.build`"
@@ -52,6 +58,8 @@ def lib() -> ctypes.CDLL:
         L.ssm_scan_version.restype = ctypes.c_int
         L.ssm_status_string.restype = ctypes.c_char_p
         L.ssm_status_string.argtypes = [ctypes.c_int]
+        L.ssm_last_error_detail.restype = ctypes.c_char_p
+        L.ssm_last_error_detail.argtypes = []
         L.ssm_scan_workspace_bytes.restype = ctypes.c_size_t
         L.ssm_scan_workspace_bytes.argtypes = [_I64, _I64, _I64, _I64, ctypes.c_int]
         L.ssm_scan_plan.restype = ctypes.c_int

@@ -1,6 +1,7 @@
 // ssm_api.cu -- the extern "C" entry points declared in include/ssm_scan.h:
 // argument validation (on the host, before anything is enqueued), the
 // sequence-segment plan, TMA tensor-map encoding and kernel launch.
+#include <stdio.h>
 #include <stdlib.h>
 #include <string.h>
 
@@ -16,6 +17,9 @@ int scan_channels_per_thread(int dstate);
 namespace {
 
 constexpr int kVersion = 10000;  // 1.0.0
+
+// Detail of the last failure on this host thread (ssm_last_error_detail).
+thread_local char g_detail[256] = "";
 
 struct Dims {
   int64_t batch, seqlen, dim, dstate;
@@ -72,7 +76,8 @@ ScanPlan make_plan(const Dims& d) {
   pl.dtiles = (int)std::max<int64_t>(1, (d.dim + pl.dtile - 1) / pl.dtile);
   const int64_t tiles = std::max<int64_t>(1, (d.seqlen + T - 1) / T);
   const int64_t cols = std::max<int64_t>(1, d.batch * pl.dtiles);
-  const long per_sm = std::max(1L, env_long("SSM_SCAN_CTAS_PER_SM", 4));
+  long per_sm = env_long("SSM_SCAN_CTAS_PER_SM", 0);
+  if (per_sm <= 0) per_sm = std::max(1, scan_ctas_per_sm((int)d.dstate, d.io == SSM_DTYPE_BF16));
   int64_t nseg = std::max<int64_t>(1, (int64_t)device_sms() * per_sm / cols);
   const long forced = env_long("SSM_SCAN_SEGMENTS", 0);
   if (forced > 0) nseg = forced;
@@ -133,6 +138,10 @@ bool encode_3d(CUtensorMap* map, const void* base, int io, int64_t batch, int64_
   const CUresult r = fn(map, dt, 3, const_cast<void*>(base), gdim, gstride, box, estride,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    snprintf(g_detail, sizeof g_detail,
+             "cuTensorMapEncodeTiled failed (CUresult %d) for dims (%lld, %lld, %lld) box (%d, %d)",
+             (int)r, (long long)cols, (long long)rows, (long long)batch, box_cols, box_rows);
   return r == CUDA_SUCCESS;
 }
 
@@ -148,7 +157,19 @@ bool tma_eligible(const Dims& d, const void* x, const void* delta, const void* z
   return encode_fn() != nullptr;
 }
 
-int cuda_status(cudaError_t e) { return e == cudaSuccess ? SSM_OK : SSM_ERR_CUDA; }
+int fail(int code, const char* what, cudaError_t e = cudaSuccess) {
+  if (e != cudaSuccess)
+    snprintf(g_detail, sizeof g_detail, "%s: %s (%s)", what, cudaGetErrorString(e),
+             cudaGetErrorName(e));
+  else
+    snprintf(g_detail, sizeof g_detail, "%s", what);
+  return code;
+}
+
+int cuda_status(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return SSM_OK;
+  return fail(SSM_ERR_CUDA, what, e);
+}
 
 }  // namespace
 }  // namespace ssm
@@ -158,6 +179,8 @@ using namespace ssm;
 extern "C" {
 
 int ssm_scan_version(void) { return kVersion; }
+
+const char* ssm_last_error_detail(void) { return g_detail; }
 
 const char* ssm_status_string(int status) {
   switch (status) {
@@ -259,7 +282,8 @@ int ssm_scan_fwd(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate, int
     if (!ok) return SSM_ERR_CUDA;
   }
   st = cuda_status(launch_scan(pl, p, use_tma ? &maps : nullptr, use_tma, (int)dstate,
-                               io_dtype == SSM_DTYPE_BF16, static_cast<cudaStream_t>(stream)));
+                               io_dtype == SSM_DTYPE_BF16, static_cast<cudaStream_t>(stream)),
+                   use_tma ? "scan launch (TMA path)" : "scan launch (plain-load path)");
   return st;
 }
 
@@ -272,16 +296,17 @@ int ssm_scan_status(const void* workspace, size_t workspace_bytes, int64_t batch
   const ScanPlan pl = make_plan(d);
   if (!workspace || workspace_bytes < pl.bytes) return SSM_ERR_WORKSPACE;
   const int n = pl.ctas_agg + pl.ctas_main;
-  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SSM_ERR_CUDA;
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(SSM_ERR_CUDA, "ssm_scan_status: stream synchronize", e);
   int buf[1024];
   const unsigned char* ws = static_cast<const unsigned char*>(workspace) + pl.off_status;
   for (int i = 0; i < n; i += 1024) {
     const int m = std::min(1024, n - i);
-    if (cudaMemcpy(buf, ws + sizeof(int) * (size_t)i, sizeof(int) * (size_t)m,
-                   cudaMemcpyDeviceToHost) != cudaSuccess)
-      return SSM_ERR_CUDA;
+    e = cudaMemcpy(buf, ws + sizeof(int) * (size_t)i, sizeof(int) * (size_t)m,
+                   cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return fail(SSM_ERR_CUDA, "ssm_scan_status: read status", e);
     for (int k = 0; k < m; ++k)
-      if (buf[k] != kCtaOk) return SSM_ERR_TIMEOUT;
+      if (buf[k] != kCtaOk) return fail(SSM_ERR_TIMEOUT, "a CTA's bounded wait timed out");
   }
   return SSM_OK;
 }
@@ -317,7 +342,8 @@ int ssm_state_update(int64_t batch, int64_t dim, int64_t dstate, int io_dtype, f
   p.x = x; p.delta = delta; p.z = z; p.B = B; p.C = C;
   p.A = A; p.D = D; p.bias = delta_bias; p.y = y;
   return cuda_status(launch_decode(p, (int)dstate, io_dtype == SSM_DTYPE_BF16,
-                                   static_cast<cudaStream_t>(stream)));
+                                   static_cast<cudaStream_t>(stream)),
+                     "decode launch");
 }
 
 }  // extern "C"

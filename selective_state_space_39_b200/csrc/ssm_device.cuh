@@ -41,8 +41,25 @@ __device__ __forceinline__ float tanh_approx(float x) {
 }
 
 // ------------------------------------------------------------ packed fp32 --
-__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
-__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+// Pairs of fp32 lanes: packed FFMA2/FMUL2 (SSM_PACKED_FP32=1, default) or
+// two scalar operations.
+#ifndef SSM_PACKED_FP32
+#define SSM_PACKED_FP32 1
+#endif
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+#if SSM_PACKED_FP32
+  return __ffma2_rn(a, b, c);
+#else
+  return make_float2(fmaf(a.x, b.x, c.x), fmaf(a.y, b.y, c.y));
+#endif
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+#if SSM_PACKED_FP32
+  return __fmul2_rn(a, b);
+#else
+  return make_float2(a.x * b.x, a.y * b.y);
+#endif
+}
 
 // ------------------------------------------------------------------ bf16 ---
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }

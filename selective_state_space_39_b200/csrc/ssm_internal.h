@@ -10,9 +10,15 @@
 namespace ssm {
 
 // Launch shape of the scan: threads per CTA and sequence steps per tile.
+#ifndef SSM_TILE_STEPS
+#define SSM_TILE_STEPS 16
+#endif
+#ifndef SSM_STAGES
+#define SSM_STAGES 2
+#endif
 constexpr int kScanThreads = 128;
-constexpr int kScanTileSteps = 16;
-constexpr int kScanStages = 2;
+constexpr int kScanTileSteps = SSM_TILE_STEPS;
+constexpr int kScanStages = SSM_STAGES;
 // Per-CTA status codes written to the workspace status area.
 constexpr int kCtaOk = 0;
 constexpr int kCtaTimeout = 1;
@@ -80,5 +86,8 @@ cudaError_t launch_scan(const ScanPlan& plan, const ScanParams& p, const ScanMap
                         bool use_tma, int dstate, bool bf16, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeParams& p, int dstate, bool bf16, cudaStream_t stream);
 bool scan_dstate_supported(int dstate);
+// Resident CTAs per SM of the main-pass kernel on the current device (0 if
+// the query fails).
+int scan_ctas_per_sm(int dstate, bool bf16);
 
 }  // namespace ssm

@@ -38,14 +38,32 @@
 //
 // bf16 io uses MUFU approximations (ex2/lg2/rcp/tanh.approx); fp32 io uses
 // the accurate expf / log1pf / IEEE division.
+#include <mutex>
+#include <set>
 #include <type_traits>
+#include <utility>
 
 #include "ssm_device.cuh"
 #include "ssm_internal.h"
 
+// Steps unrolled together inside a full tile, and the minimum resident CTAs
+// per SM requested from the register allocator.
+#ifndef SSM_TILE_UNROLL
+#define SSM_TILE_UNROLL 4
+#endif
+// Channels per thread at dstate 16.
+#ifndef SSM_CPT16
+#define SSM_CPT16 2
+#endif
+#ifndef SSM_MIN_CTAS
+#define SSM_MIN_CTAS 1
+#endif
+
 namespace ssm {
 
 namespace {
+
+constexpr int kTileUnroll = SSM_TILE_UNROLL;
 
 constexpr int round_up(int v, int m) { return (v + m - 1) / m * m; }
 
@@ -78,12 +96,51 @@ struct Chan {
   bool valid;   // d < dim
 };
 
+// Per-step, per-channel quantities computed ahead of the state update.
+struct StepScalars {
+  float a0, a1;  // alpha for states 0 and 1: rho r, rho r^2 (structured A)
+  float rr;      // r^2, the step of the alpha chain over state pairs
+  float rho;     // s_{t-1} / s_t (generic A)
+  float q;       // Delta (precise) or Delta log2(e) (fast)
+  float s;       // the state scale s_t ~ Delta x
+};
+
+// Step size, decay base and state scale for one channel and step.
+template <bool kFast>
+__device__ __forceinline__ StepScalars step_scalars(float xv, float dv, const Chan& ch,
+                                                    int softplus, float& s_prev) {
+  StepScalars o;
+  float q, r;
+  if constexpr (kFast) {
+    const float v = fmaf(dv, kLog2e, ch.bias);
+    q = softplus ? (v > kSoftplusCut * kLog2e ? v : lg2_approx(1.f + ex2_approx(v))) : v;
+    r = ex2_approx(q * ch.A0);  // exp(Delta A0)
+  } else {
+    const float v = dv + ch.bias;
+    q = softplus ? (v > kSoftplusCut ? v : log1pf(expf(v))) : v;
+    r = expf(q * ch.A0);
+  }
+  // s = Delta x in the path's units (fast: times log2 e, matched by B
+  // pre-scaled by ln 2), kept away from zero.
+  float s = q * xv;
+  s = s + copysignf(kScaleFloor, s);
+  const float rho = kFast ? s_prev * rcp_approx(s) : s_prev / s;
+  s_prev = s;
+  o.q = q;
+  o.s = s;
+  o.rho = rho;
+  o.a0 = rho * r;
+  o.a1 = o.a0 * r;
+  o.rr = r * r;
+  return o;
+}
+
 // -------------------------------------------------------------------------
 // The scan kernel. kAgg = carry pass (segments 0..nseg-2: end state and
 // sum of Delta, no output); !kAgg = main pass (all segments, y and h_last).
 // Grid: (dtiles, segments, batch). Block: NT threads, CPT channels each.
 template <typename IOT, int N, int CPT, int NT, int T, int STAGES, bool kAgg, bool kTma>
-__global__ void __launch_bounds__(NT) scan_kernel(const ScanParams p,
+__global__ void __launch_bounds__(NT, SSM_MIN_CTAS) scan_kernel(const ScanParams p,
                                                   const __grid_constant__ ScanMaps maps) {
   using IO = Io<IOT>;
   using L = ScanLayout<IOT, N, CPT, NT, T>;
@@ -102,6 +159,7 @@ __global__ void __launch_bounds__(NT) scan_kernel(const ScanParams p,
   const int d_local = tid * CPT;
   const int d_first = dtile * DT + d_local;
   const bool has_z = !kAgg && p.z != nullptr;
+  const int softplus = p.softplus;
   const int t_begin = seg * p.seg_steps;
   const int t_end = min(t_begin + p.seg_steps, L_);
   const int ntiles = t_end > t_begin ? (t_end - t_begin + T - 1) / T : 0;
@@ -161,6 +219,9 @@ __global__ void __launch_bounds__(NT) scan_kernel(const ScanParams p,
       ch[c].Dd = 0.f;
     }
   }
+  // One code path per CTA: the multiply-chain path when every channel of the
+  // CTA has structured A, one exp per state otherwise.
+  const bool cta_structured = __syncthreads_and(structured) != 0;
 
   // ---- initial state ----------------------------------------------------
   float2 g[CPT][NP];  // scaled state g = h / s_prev
@@ -194,31 +255,35 @@ __global__ void __launch_bounds__(NT) scan_kernel(const ScanParams p,
       } else {
         const float* h0 = p.nseg > 1 ? (p.h0 ? p.ws_h0 : nullptr) : p.h0;
         if (seg > 0) {
-          // inclusive end state of segment 0, then compose segments 1..seg-1
+          // Inclusive end state of segment 0, then compose the carries
+          // (decay exp(A_n sum Delta), end state) of segments 1..seg-1.
           const float* st0 = p.ws_state + ((size_t)b * nagg) * N * dim + d;
 #pragma unroll
           for (int k = 0; k < NP; ++k)
-            g[c][k] = make_float2(st0[(size_t)(2 * k) * dim], st0[(size_t)(2 * k + 1) * dim]);
+            g[c][k] = make_float2(__ldcg(st0 + (size_t)(2 * k) * dim),
+                                  __ldcg(st0 + (size_t)(2 * k + 1) * dim));
+          const float* Ar = p.A + (size_t)d * N;
           for (int j = 1; j < seg; ++j) {
-            const float sd = p.ws_sum[((size_t)b * nagg + j) * dim + d];
+            const float sd = __ldcg(p.ws_sum + ((size_t)b * nagg + j) * dim + d);
             const float* stj = p.ws_state + ((size_t)b * nagg + j) * N * dim + d;
-            if (structured) {
+            float bj[N];
+#pragma unroll
+            for (int n = 0; n < N; ++n) bj[n] = __ldcg(stj + (size_t)n * dim);
+            if (cta_structured) {
               const float e = expf(ch[c].A0 * sd);
               float en = e;
 #pragma unroll
               for (int k = 0; k < NP; ++k) {
                 const float e0 = en, e1 = en * e;
                 en = e1 * e;
-                g[c][k].x = fmaf(e0, g[c][k].x, stj[(size_t)(2 * k) * dim]);
-                g[c][k].y = fmaf(e1, g[c][k].y, stj[(size_t)(2 * k + 1) * dim]);
+                g[c][k].x = fmaf(e0, g[c][k].x, bj[2 * k]);
+                g[c][k].y = fmaf(e1, g[c][k].y, bj[2 * k + 1]);
               }
             } else {
-              const float* Ar = p.A + (size_t)d * N;
 #pragma unroll
               for (int k = 0; k < NP; ++k) {
-                g[c][k].x = fmaf(expf(Ar[2 * k] * sd), g[c][k].x, stj[(size_t)(2 * k) * dim]);
-                g[c][k].y =
-                    fmaf(expf(Ar[2 * k + 1] * sd), g[c][k].y, stj[(size_t)(2 * k + 1) * dim]);
+                g[c][k].x = fmaf(expf(Ar[2 * k] * sd), g[c][k].x, bj[2 * k]);
+                g[c][k].y = fmaf(expf(Ar[2 * k + 1] * sd), g[c][k].y, bj[2 * k + 1]);
               }
             }
           }
@@ -231,197 +296,223 @@ __global__ void __launch_bounds__(NT) scan_kernel(const ScanParams p,
     }
   }
 
-  // ---- tile loop ----------------------------------------------------------
-  const bool pair_store = CPT == 2 && p.pair_store;
-  for (int it = 0; it < ntiles; ++it) {
-    const int buf = it & 1;
-    unsigned char* st;
-    if constexpr (kTma) {
-      st = smem + (it % STAGES) * L::kStageBytes;
-      const bool ok = mbar_wait_bounded(&full[it % STAGES], (uint32_t)((it / STAGES) & 1),
-                                        p.wait_limit_ns);
-      if (__syncthreads_or(!ok)) {
-        aborted = true;  // uniform across the CTA
-        // Let the loads already issued land (bounded) before the CTA's
-        // shared memory is released.
-        if (tid == 0)
-          for (int j = it; j < issued; ++j)
-            (void)mbar_wait_bounded(&full[j % STAGES], (uint32_t)((j / STAGES) & 1), 1000000ull);
-        break;
+  // ---- per-step pieces ----------------------------------------------------
+  const bool pair_store = CPT == 2 && p.pair_store && ch[CPT - 1].valid;
+  struct StepIn {
+    float x[CPT], d[CPT], z[CPT];
+  };
+  // x, delta, z of smem row `row` for this thread's channels
+  auto load_in = [&](const unsigned char* st, int row) {
+    StepIn in;
+    const IOT* sx = reinterpret_cast<const IOT*>(st + L::kOffX) + d_local + row * DT;
+    const IOT* sdl = reinterpret_cast<const IOT*>(st + L::kOffD) + d_local + row * DT;
+    const IOT* sz = reinterpret_cast<const IOT*>(st + L::kOffZ) + d_local + row * DT;
+    if constexpr (CPT == 2) {
+      const float2 x2 = IO::load2(sx), d2 = IO::load2(sdl);
+      in.x[0] = x2.x; in.x[1] = x2.y; in.d[0] = d2.x; in.d[1] = d2.y;
+      if (!kAgg && has_z) {
+        const float2 z2 = IO::load2(sz);
+        in.z[0] = z2.x; in.z[1] = z2.y;
       }
     } else {
-      st = smem;
-      __syncthreads();  // every thread is done with the previous tile
-      const int t0 = t_begin + it * T;
-      const IOT* gx = reinterpret_cast<const IOT*>(p.x);
-      const IOT* gd = reinterpret_cast<const IOT*>(p.delta);
-      const IOT* gz = reinterpret_cast<const IOT*>(p.z);
-      IOT* sx = reinterpret_cast<IOT*>(st + L::kOffX);
-      IOT* sd = reinterpret_cast<IOT*>(st + L::kOffD);
-      IOT* sz = reinterpret_cast<IOT*>(st + L::kOffZ);
-      for (int i = tid; i < T * DT; i += NT) {
-        const int tt = t0 + i / DT, dd = dtile * DT + i % DT;
-        const bool in = tt < L_ && dd < dim;
-        const size_t gi = ((size_t)b * L_ + tt) * dim + dd;
-        sx[i] = in ? gx[gi] : IOT(0);
-        sd[i] = in ? gd[gi] : IOT(0);
-        if (has_z) sz[i] = in ? gz[gi] : IOT(0);
-      }
-      const IOT* gb = reinterpret_cast<const IOT*>(p.B);
-      const IOT* gc = reinterpret_cast<const IOT*>(p.C);
-      IOT* sb = reinterpret_cast<IOT*>(st + L::kOffB);
-      IOT* sc = reinterpret_cast<IOT*>(st + L::kOffC);
-      for (int i = tid; i < T * N; i += NT) {
-        const int tt = t0 + i / N;
-        const size_t gi = ((size_t)b * L_ + tt) * N + i % N;
-        sb[i] = tt < L_ ? gb[gi] : IOT(0);
-        if (!kAgg) sc[i] = tt < L_ ? gc[gi] : IOT(0);
-      }
-      __syncthreads();
-    }
-
-    // widen B (times ln2 on the fast path, see below) and C to fp32
-    {
-      const IOT* sb = reinterpret_cast<const IOT*>(st + L::kOffB);
-      const IOT* sc = reinterpret_cast<const IOT*>(st + L::kOffC);
-      float* fb = bcf + (buf * 2 + 0) * T * N;
-      float* fc = bcf + (buf * 2 + 1) * T * N;
-      const float bscale = kFast ? kLn2 : 1.f;
-      for (int i = tid; i < T * N; i += NT) {
-        fb[i] = IO::load(sb + i) * bscale;
-        if (!kAgg) fc[i] = IO::load(sc + i);
-      }
-    }
-    __syncthreads();
-    if constexpr (kTma) {
-      // The stage consumed by the previous tile is free: refill it.
-      if (tid == 0 && issued < ntiles) issue_tile(issued++);
-    }
-
-    const IOT* sx = reinterpret_cast<const IOT*>(st + L::kOffX) + d_local;
-    const IOT* sdl = reinterpret_cast<const IOT*>(st + L::kOffD) + d_local;
-    const IOT* sz = reinterpret_cast<const IOT*>(st + L::kOffZ) + d_local;
-    const float* fb = bcf + (buf * 2 + 0) * T * N;
-    const float* fc = bcf + (buf * 2 + 1) * T * N;
-    const int t0 = t_begin + it * T;
-    const int steps = min(T, t_end - t0);
-
-    for (int ss = 0; ss < steps; ++ss) {
-      float xv[CPT], dv[CPT], zv[CPT];
-      if constexpr (CPT == 2) {
-        const float2 x2 = IO::load2(sx + ss * DT), d2 = IO::load2(sdl + ss * DT);
-        xv[0] = x2.x; xv[1] = x2.y; dv[0] = d2.x; dv[1] = d2.y;
-        if (has_z) {
-          const float2 z2 = IO::load2(sz + ss * DT);
-          zv[0] = z2.x; zv[1] = z2.y;
-        }
-      } else {
 #pragma unroll
-        for (int c = 0; c < CPT; ++c) {
-          xv[c] = IO::load(sx + ss * DT + c);
-          dv[c] = IO::load(sdl + ss * DT + c);
-          if (has_z) zv[c] = IO::load(sz + ss * DT + c);
+      for (int c = 0; c < CPT; ++c) {
+        in.x[c] = IO::load(sx + c);
+        in.d[c] = IO::load(sdl + c);
+        if (!kAgg && has_z) in.z[c] = IO::load(sz + c);
+      }
+    }
+    return in;
+  };
+
+  // State update (and readout) of one step, given its precomputed scalars.
+  auto state_step = [&](auto kStructTag, const StepIn& in, const StepScalars* sc, const float* Bt,
+                        const float* Ct, int t_abs) {
+    constexpr bool kS = decltype(kStructTag)::value;
+    float2 acc[CPT];
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) acc[c] = make_float2(0.f, 0.f);
+    if constexpr (kS) {
+      const float2* B2 = reinterpret_cast<const float2*>(Bt);
+      const float2* C2 = reinterpret_cast<const float2*>(Ct);
+      (void)C2;
+#pragma unroll
+      for (int c = 0; c < CPT; ++c) {
+        // alpha_n = rho r^(n+1), two states at a time: (a0, a1) * (r^2)^k
+        float2 a = make_float2(sc[c].a0, sc[c].a1);
+        const float2 rr = make_float2(sc[c].rr, sc[c].rr);
+#pragma unroll
+        for (int k = 0; k < NP; ++k) {
+          g[c][k] = fma2(a, g[c][k], B2[k]);
+          if (k + 1 < NP) a = mul2(a, rr);
+          if constexpr (!kAgg) acc[c] = fma2(C2[k], g[c][k], acc[c]);
         }
       }
-      const float* Bt = fb + ss * N;
-      const float* Ct = fc + ss * N;
+    } else {
+#pragma unroll
+      for (int c = 0; c < CPT; ++c) {
+        const float* Ar = p.A + (size_t)(ch[c].valid ? d_first + c : 0) * N;
+        const float2* B2 = reinterpret_cast<const float2*>(Bt);
+        const float2* C2 = reinterpret_cast<const float2*>(Ct);
+        (void)C2;
+        const float rho = sc[c].rho, q = sc[c].q;
+#pragma unroll
+        for (int k = 0; k < NP; ++k) {
+          float2 a;
+          if constexpr (kFast) {
+            a = make_float2(rho * ex2_approx(q * __ldg(Ar + 2 * k)),
+                            rho * ex2_approx(q * __ldg(Ar + 2 * k + 1)));
+          } else {
+            a = make_float2(rho * expf(q * __ldg(Ar + 2 * k)),
+                            rho * expf(q * __ldg(Ar + 2 * k + 1)));
+          }
+          g[c][k] = fma2(a, g[c][k], B2[k]);
+          if constexpr (!kAgg) acc[c] = fma2(C2[k], g[c][k], acc[c]);
+        }
+      }
+    }
+    if constexpr (!kAgg) {
       float yv[CPT];
 #pragma unroll
       for (int c = 0; c < CPT; ++c) {
-        // Step size. Fast path works in log2 units: q = Delta * log2(e).
-        float q, r;
-        if constexpr (kFast) {
-          const float v = fmaf(dv[c], kLog2e, ch[c].bias);
-          q = p.softplus ? (v > kSoftplusCut * kLog2e ? v : lg2_approx(1.f + ex2_approx(v))) : v;
-          r = ex2_approx(q * ch[c].A0);  // exp(Delta A0)
-        } else {
-          const float v = dv[c] + ch[c].bias;
-          q = p.softplus ? (v > kSoftplusCut ? v : log1pf(expf(v))) : v;
-          r = expf(q * ch[c].A0);
-        }
-        // s = Delta x in the path's units (fast: times log2 e, matched by
-        // B pre-scaled by ln 2), kept away from zero.
-        float s = q * xv[c];
-        s = s + copysignf(kScaleFloor, s);
-        const float rho = kFast ? s_prev[c] * rcp_approx(s) : s_prev[c] / s;
-        s_prev[c] = s;
-        if constexpr (kAgg) qsum[c] += q;
-
-        float2 acc = make_float2(0.f, 0.f);
-        if (structured) {
-          const float a0 = rho * r;
-          const float r2 = r * r;
-          float2 a = make_float2(a0, a0 * r);
-          const float2 rr = make_float2(r2, r2);
-          if constexpr (N % 4 == 0) {
-            const float4* B4 = reinterpret_cast<const float4*>(Bt);
-            const float4* C4 = reinterpret_cast<const float4*>(Ct);
-#pragma unroll
-            for (int k = 0; k < N / 4; ++k) {
-              const float4 bq = B4[k];
-              g[c][2 * k] = fma2(a, g[c][2 * k], make_float2(bq.x, bq.y));
-              a = mul2(a, rr);
-              g[c][2 * k + 1] = fma2(a, g[c][2 * k + 1], make_float2(bq.z, bq.w));
-              a = mul2(a, rr);
-              if constexpr (!kAgg) {
-                const float4 cq = C4[k];
-                acc = fma2(make_float2(cq.x, cq.y), g[c][2 * k], acc);
-                acc = fma2(make_float2(cq.z, cq.w), g[c][2 * k + 1], acc);
-              }
-            }
+        float yy = fmaf(sc[c].s, acc[c].x + acc[c].y, ch[c].Dd * in.x[c]);
+        if (has_z) {
+          if constexpr (kFast) {
+            const float hz = 0.5f * in.z[c];
+            yy *= fmaf(hz, tanh_approx(hz), hz);  // z * sigmoid(z)
           } else {
-            const float2* B2 = reinterpret_cast<const float2*>(Bt);
-            const float2* C2 = reinterpret_cast<const float2*>(Ct);
-#pragma unroll
-            for (int k = 0; k < NP; ++k) {
-              g[c][k] = fma2(a, g[c][k], B2[k]);
-              a = mul2(a, rr);
-              if constexpr (!kAgg) acc = fma2(C2[k], g[c][k], acc);
-            }
-          }
-        } else {
-          const float* Ar = p.A + (size_t)(ch[c].valid ? d_first + c : 0) * N;
-          const float2* B2 = reinterpret_cast<const float2*>(Bt);
-          const float2* C2 = reinterpret_cast<const float2*>(Ct);
-#pragma unroll
-          for (int k = 0; k < NP; ++k) {
-            float2 a;
-            if constexpr (kFast) {
-              a = make_float2(rho * ex2_approx(q * __ldg(Ar + 2 * k)),
-                              rho * ex2_approx(q * __ldg(Ar + 2 * k + 1)));
-            } else {
-              a = make_float2(rho * expf(q * __ldg(Ar + 2 * k)),
-                              rho * expf(q * __ldg(Ar + 2 * k + 1)));
-            }
-            g[c][k] = fma2(a, g[c][k], B2[k]);
-            if constexpr (!kAgg) acc = fma2(C2[k], g[c][k], acc);
+            yy *= in.z[c] / (1.f + expf(-in.z[c]));
           }
         }
-        if constexpr (!kAgg) {
-          float yy = fmaf(s, acc.x + acc.y, ch[c].Dd * xv[c]);
-          if (has_z) {
-            if constexpr (kFast) {
-              const float hz = 0.5f * zv[c];
-              yy *= fmaf(hz, tanh_approx(hz), hz);  // z * sigmoid(z)
-            } else {
-              yy *= zv[c] / (1.f + expf(-zv[c]));
-            }
-          }
-          yv[c] = yy;
-        }
+        yv[c] = yy;
       }
-      if constexpr (!kAgg) {
-        IOT* yrow = reinterpret_cast<IOT*>(p.y) + ((size_t)b * L_ + (t0 + ss)) * dim + d_first;
-        if (pair_store && ch[CPT - 1].valid) {
-          IO::store2(yrow, yv[0], yv[CPT - 1]);
-        } else {
+      IOT* yrow = reinterpret_cast<IOT*>(p.y) + ((size_t)b * L_ + t_abs) * dim + d_first;
+      if (pair_store) {
+        IO::store2(yrow, yv[0], yv[CPT - 1]);
+      } else {
 #pragma unroll
-          for (int c = 0; c < CPT; ++c)
-            if (ch[c].valid) IO::store(yrow + c, yv[c]);
-        }
+        for (int c = 0; c < CPT; ++c)
+          if (ch[c].valid) IO::store(yrow + c, yv[c]);
       }
     }
-  }
+  };
+
+  // ---- tile loop ----------------------------------------------------------
+  auto run_tiles = [&](auto kStructTag) {
+    for (int it = 0; it < ntiles; ++it) {
+      const int buf = it & 1;
+      unsigned char* st;
+      if constexpr (kTma) {
+        st = smem + (it % STAGES) * L::kStageBytes;
+        const bool ok = mbar_wait_bounded(&full[it % STAGES], (uint32_t)((it / STAGES) & 1),
+                                          p.wait_limit_ns);
+        if (__syncthreads_or(!ok)) {
+          aborted = true;  // uniform across the CTA
+          // Let the loads already issued land (bounded) before the CTA's
+          // shared memory is released.
+          if (tid == 0)
+            for (int j = it; j < issued; ++j)
+              (void)mbar_wait_bounded(&full[j % STAGES], (uint32_t)((j / STAGES) & 1), 1000000ull);
+          return;
+        }
+      } else {
+        st = smem;
+        __syncthreads();  // every thread is done with the previous tile
+        const int t0 = t_begin + it * T;
+        const IOT* gx = reinterpret_cast<const IOT*>(p.x);
+        const IOT* gd = reinterpret_cast<const IOT*>(p.delta);
+        const IOT* gz = reinterpret_cast<const IOT*>(p.z);
+        IOT* sx = reinterpret_cast<IOT*>(st + L::kOffX);
+        IOT* sd = reinterpret_cast<IOT*>(st + L::kOffD);
+        IOT* sz = reinterpret_cast<IOT*>(st + L::kOffZ);
+        for (int i = tid; i < T * DT; i += NT) {
+          const int tt = t0 + i / DT, dd = dtile * DT + i % DT;
+          const bool in = tt < L_ && dd < dim;
+          const size_t gi = ((size_t)b * L_ + tt) * dim + dd;
+          sx[i] = in ? gx[gi] : IOT(0);
+          sd[i] = in ? gd[gi] : IOT(0);
+          if (has_z) sz[i] = in ? gz[gi] : IOT(0);
+        }
+        const IOT* gb = reinterpret_cast<const IOT*>(p.B);
+        const IOT* gc = reinterpret_cast<const IOT*>(p.C);
+        IOT* sb = reinterpret_cast<IOT*>(st + L::kOffB);
+        IOT* sc = reinterpret_cast<IOT*>(st + L::kOffC);
+        for (int i = tid; i < T * N; i += NT) {
+          const int tt = t0 + i / N;
+          const size_t gi = ((size_t)b * L_ + tt) * N + i % N;
+          sb[i] = tt < L_ ? gb[gi] : IOT(0);
+          if (!kAgg) sc[i] = tt < L_ ? gc[gi] : IOT(0);
+        }
+        __syncthreads();
+      }
+
+      // widen B (times ln2 on the fast path) and C to fp32
+      {
+        const IOT* sb = reinterpret_cast<const IOT*>(st + L::kOffB);
+        const IOT* sc = reinterpret_cast<const IOT*>(st + L::kOffC);
+        float* fb = bcf + (buf * 2 + 0) * T * N;
+        float* fc = bcf + (buf * 2 + 1) * T * N;
+        const float bscale = kFast ? kLn2 : 1.f;
+        for (int i = tid; i < T * N; i += NT) {
+          fb[i] = IO::load(sb + i) * bscale;
+          if (!kAgg) fc[i] = IO::load(sc + i);
+        }
+      }
+      __syncthreads();
+      if constexpr (kTma) {
+        // The stage consumed by the previous tile is free: refill it.
+        if (tid == 0 && issued < ntiles) issue_tile(issued++);
+      }
+
+      const float* fb = bcf + (buf * 2 + 0) * T * N;
+      const float* fc = bcf + (buf * 2 + 1) * T * N;
+      const int t0 = t_begin + it * T;
+      const int steps = min(T, t_end - t0);
+      // Software pipeline: the scalar chain of step row+1 (which does not
+      // depend on the state) is computed in the same iteration as the state
+      // update of step row, so the two interleave. Full tiles are unrolled
+      // (all shared-memory offsets become constants); the look-ahead at the
+      // last row re-reads that row and its result is discarded.
+      auto step_loop = [&](auto kFullTag, int nsteps) {
+        constexpr bool kFull = decltype(kFullTag)::value;
+        const int nst = kFull ? T : nsteps;
+        StepIn in_next = load_in(st, 0);
+        StepScalars sc_next[CPT];
+#pragma unroll
+        for (int c = 0; c < CPT; ++c)
+          sc_next[c] = step_scalars<kFast>(in_next.x[c], in_next.d[c], ch[c], softplus, s_prev[c]);
+        float s_last[CPT];
+#pragma unroll(kFull ? kTileUnroll : 1)
+        for (int row = 0; row < nst; ++row) {
+          const StepIn in = in_next;
+          StepScalars sc[CPT];
+#pragma unroll
+          for (int c = 0; c < CPT; ++c) {
+            sc[c] = sc_next[c];
+            s_last[c] = sc[c].s;
+            if constexpr (kAgg) qsum[c] += sc[c].q;
+          }
+          in_next = load_in(st, min(row + 1, nst - 1));
+#pragma unroll
+          for (int c = 0; c < CPT; ++c) {
+            float sp = sc[c].s;
+            sc_next[c] = step_scalars<kFast>(in_next.x[c], in_next.d[c], ch[c], softplus, sp);
+          }
+          state_step(kStructTag, in, sc, fb + row * N, fc + row * N, t0 + row);
+        }
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) s_prev[c] = s_last[c];  // scale of the last step
+      };
+      if (steps == T)
+        step_loop(std::true_type{}, T);
+      else
+        step_loop(std::false_type{}, steps);
+    }
+  };
+  if (cta_structured)
+    run_tiles(std::true_type{});
+  else
+    run_tiles(std::false_type{});
 
   // ---- outputs of the segment ------------------------------------------
   if (!aborted) {
@@ -525,17 +616,17 @@ __global__ void __launch_bounds__(256) decode_kernel(const DecodeParams p) {
 }
 
 // -------------------------------------------------------------------------
-// cudaFuncSetAttribute once per kernel and device (up to 64 devices).
-template <typename K>
-cudaError_t ensure_smem_attr(K kernel, int smem) {
-  static unsigned long long done = 0ull;  // bit per device, set after success
+// cudaFuncSetAttribute once per (kernel, device).
+cudaError_t ensure_smem_attr(const void* kernel, int smem) {
+  static std::mutex mu;
+  static std::set<std::pair<const void*, int>> done;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  const unsigned long long bit = dev < 64 ? (1ull << dev) : 0ull;
-  if (bit && (__atomic_load_n(&done, __ATOMIC_ACQUIRE) & bit)) return cudaSuccess;
+  std::lock_guard<std::mutex> lock(mu);
+  if (done.count({kernel, dev})) return cudaSuccess;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e == cudaSuccess && bit) __atomic_fetch_or(&done, bit, __ATOMIC_RELEASE);
+  if (e == cudaSuccess) done.insert({kernel, dev});
   return e;
 }
 
@@ -548,7 +639,7 @@ cudaError_t launch_scan_t(const ScanPlan& plan, const ScanParams& p, const ScanM
   const dim3 block(NT);
   cudaError_t err = cudaSuccess;
   auto run = [&](auto kernel, int smem, dim3 grid) -> cudaError_t {
-    cudaError_t e = ensure_smem_attr(kernel, smem);
+    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kernel), smem);
     if (e != cudaSuccess) return e;
     kernel<<<grid, block, smem, stream>>>(p, m);
     return cudaGetLastError();
@@ -573,6 +664,33 @@ cudaError_t launch_scan_t(const ScanPlan& plan, const ScanParams& p, const ScanM
              dim3(plan.dtiles, plan.nseg, p.batch));
 }
 
+template <typename IOT, int N, int CPT>
+int ctas_per_sm_t() {
+  constexpr int NT = kScanThreads, T = kScanTileSteps, S = kScanStages;
+  int n = 0;
+  auto kernel = scan_kernel<IOT, N, CPT, NT, T, S, false, true>;
+  constexpr int smem = scan_smem_bytes<IOT, N, CPT, NT, T, S>();
+  if (ensure_smem_attr(reinterpret_cast<const void*>(kernel), smem) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, NT, smem) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
+template <typename IOT>
+int ctas_per_sm_io(int dstate) {
+  switch (dstate) {
+    case 2: return ctas_per_sm_t<IOT, 2, 2>();
+    case 4: return ctas_per_sm_t<IOT, 4, 2>();
+    case 8: return ctas_per_sm_t<IOT, 8, 2>();
+    case 16: return ctas_per_sm_t<IOT, 16, SSM_CPT16>();
+    case 32: return ctas_per_sm_t<IOT, 32, 1>();
+    case 64: return ctas_per_sm_t<IOT, 64, 1>();
+    default: return 0;
+  }
+}
+
 template <typename IOT>
 cudaError_t launch_scan_io(const ScanPlan& plan, const ScanParams& p, const ScanMaps* maps,
                            bool use_tma, int dstate, cudaStream_t stream) {
@@ -580,7 +698,7 @@ cudaError_t launch_scan_io(const ScanPlan& plan, const ScanParams& p, const Scan
     case 2: return launch_scan_t<IOT, 2, 2>(plan, p, maps, use_tma, stream);
     case 4: return launch_scan_t<IOT, 4, 2>(plan, p, maps, use_tma, stream);
     case 8: return launch_scan_t<IOT, 8, 2>(plan, p, maps, use_tma, stream);
-    case 16: return launch_scan_t<IOT, 16, 2>(plan, p, maps, use_tma, stream);
+    case 16: return launch_scan_t<IOT, 16, SSM_CPT16>(plan, p, maps, use_tma, stream);
     case 32: return launch_scan_t<IOT, 32, 1>(plan, p, maps, use_tma, stream);
     case 64: return launch_scan_t<IOT, 64, 1>(plan, p, maps, use_tma, stream);
     default: return cudaErrorInvalidValue;
@@ -614,7 +732,11 @@ bool scan_dstate_supported(int dstate) {
          dstate == 64;
 }
 
-int scan_channels_per_thread(int dstate) { return dstate <= 16 ? 2 : 1; }
+int scan_channels_per_thread(int dstate) { return dstate < 16 ? 2 : dstate == 16 ? SSM_CPT16 : 1; }
+
+int scan_ctas_per_sm(int dstate, bool bf16) {
+  return bf16 ? ctas_per_sm_io<uint16_t>(dstate) : ctas_per_sm_io<float>(dstate);
+}
 
 cudaError_t launch_scan(const ScanPlan& plan, const ScanParams& p, const ScanMaps* maps,
                         bool use_tma, int dstate, bool bf16, cudaStream_t stream) {
