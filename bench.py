@@ -33,6 +33,7 @@ METRIC = "selective-scan elements/s (B·L·D) and achieved HBM GB/s as % of B200
 DEFAULT_WORKLOAD = "mamba130m_layer_b8_l2048_d1536"
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
+B200_SMS, FP32_LANES_PER_SM, B200_MAX_SM_MHZ = 148, 128, 1965.0
 
 
 def parse_args():
@@ -58,6 +59,31 @@ def algorithmic_bytes(w, batch):
     state = batch * w.dim * w.dstate * 4 * (2 if w.with_h0 else 1)  # h_last (+ h0)
     params = w.dim * w.dstate * 4 + w.dim * 4 * (2 if w.skip else 1)  # A, bias, (D)
     return bld * per_elem + 2 * bln * es + state + params
+
+
+def alu_ops_per_element(w):
+    """FP32 operations the recurrence needs per element in its plain form:
+    per state one multiply for the decay power, one for Delta x B, one FMA for
+    the state and one for the readout (4N), as counted for the roofline."""
+    return 4 * w.dstate
+
+
+def measured_traffic(workload):
+    """DRAM bytes per call from the committed ncu capture, or None when the
+    kernel sources changed since that capture (or none was taken)."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            t = json.load(f)
+        h = hashlib.sha256()
+        for src in t["kernel_sources"]:
+            with open(os.path.join(ROOT, src), "rb") as f:
+                h.update(f.read())
+        if h.hexdigest() != t["kernel_sources_sha256"]:
+            return None
+        return t["workloads"].get(workload, {}).get("per_call")
+    except Exception:
+        return None
 
 
 def measured_hbm_peak():
@@ -260,40 +286,54 @@ def main():
     elements = world * w.batch * w.seqlen * w.dim
     value = elements * K / (total_ms * 1e-3)
 
-    # roofline of the call: algorithmic bytes / device time, against HBM peak
+    # Rooflines of the call (carry pass + main pass). The binding one is the
+    # FP32 ALU: the path does ~4N FP32 operations per 8 bytes moved.
+    clocks = sampler.summary()
+    sm_mhz = clocks.get("sm_mhz") or B200_MAX_SM_MHZ
+    alu_peak = B200_SMS * FP32_LANES_PER_SM * sm_mhz * 1e6 / 1e9  # Gop/s
+    mean_s = statistics.mean(step_ms) * 1e-3
+    alu_achieved = alu_ops_per_element(w) * nb * w.seqlen * w.dim / mean_s / 1e9
+    traffic = measured_traffic(w.name) if world == 1 or nb == w.batch else None
+    kernel = "ssm_scan_fwd: carry pass + main pass (%d launches)" % plan.kernels
+    roofline = {"bound": "alu", "achieved": round(alu_achieved, 1), "peak": round(alu_peak, 1),
+                "unit": "Gop/s", "frac": round(alu_achieved / alu_peak, 4), "traffic": traffic,
+                "kernel": kernel, "ops_per_element": alu_ops_per_element(w),
+                "peak_kind": f"derived: {B200_SMS} SMs x {FP32_LANES_PER_SM} FP32 lanes x "
+                             f"{sm_mhz:.0f} MHz sampled SM clock"}
     peak, peak_kind = measured_hbm_peak()
     algo = algorithmic_bytes(w, nb)
-    achieved = algo / (statistics.mean(step_ms) * 1e-3) / 1e9
-    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": None,
-                "kernel": "ssm_scan_fwd: carry pass + main pass (%d launches)" % plan.kernels,
-                "algorithmic_bytes_per_launch": algo, "peak_kind": peak_kind}
+    achieved = algo / mean_s / 1e9
+    hbm_roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                    "frac": round(achieved / peak, 4), "traffic": traffic, "kernel": kernel,
+                    "algorithmic_bytes_per_launch": algo, "peak_kind": peak_kind}
 
     # end to end through the public call: pinned host inputs -> device -> scan -> host
-    pinned = {k: (torch.from_numpy(v.view(np.int16) if v.dtype == np.uint16 else v)
-                  .view(dtype if v.dtype == np.uint16 else torch.float32).pin_memory()
-                  if v is not None else None) for k, v in inp.items()}
-    y_host = torch.empty(y.shape, dtype=dtype).pin_memory()
-    h_host = torch.empty(h_last.shape, dtype=torch.float32).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in pinned.values() if t is not None)
-    d2h = y_host.numel() * y_host.element_size() + h_host.numel() * h_host.element_size()
-    e_ms = []
-    for i in range(args.e2e_steps + 2):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for k, t in pinned.items():
-            if t is not None:
-                d[k].copy_(t, non_blocking=True)
-        step()
-        y_host.copy_(y, non_blocking=True)
-        h_host.copy_(h_last, non_blocking=True)
-        e1.record()
-        e1.synchronize()
-        if i >= 2:
-            e_ms.append(e0.elapsed_time(e1))
-    e2e_ms = sdist.max_over_ranks(statistics.mean(e_ms), device)
-    e2e = {"value": elements / (e2e_ms * 1e-3), "unit": "elements/s",
-           "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+    e2e = None
+    if args.e2e_steps > 0:
+        pinned = {k: (torch.from_numpy(v.view(np.int16) if v.dtype == np.uint16 else v)
+                      .view(dtype if v.dtype == np.uint16 else torch.float32).pin_memory()
+                      if v is not None else None) for k, v in inp.items()}
+        y_host = torch.empty(y.shape, dtype=dtype).pin_memory()
+        h_host = torch.empty(h_last.shape, dtype=torch.float32).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in pinned.values() if t is not None)
+        d2h = y_host.numel() * y_host.element_size() + h_host.numel() * h_host.element_size()
+        e_ms = []
+        for i in range(args.e2e_steps + 2):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for k, t in pinned.items():
+                if t is not None:
+                    d[k].copy_(t, non_blocking=True)
+            step()
+            y_host.copy_(y, non_blocking=True)
+            h_host.copy_(h_last, non_blocking=True)
+            e1.record()
+            e1.synchronize()
+            if i >= 2:
+                e_ms.append(e0.elapsed_time(e1))
+        e2e_ms = sdist.max_over_ranks(statistics.mean(e_ms), device)
+        e2e = {"value": elements / (e2e_ms * 1e-3), "unit": "elements/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
     cpu = None
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
@@ -315,8 +355,8 @@ def main():
                        "l2": "flushed (256 MB write) before every timed step",
                        "parallelism": f"dp{world} (batch shards, no data-path collective)"},
             "hbm_gbs": round(achieved, 1), "hbm_frac_of_peak": round(achieved / peak, 4),
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": K * plan.kernels, "clocks": sampler.summary(),
+            "roofline": roofline, "hbm_roofline": hbm_roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": K * plan.kernels, "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
     sdist.finish()
