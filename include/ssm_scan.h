@@ -125,6 +125,36 @@ int ssm_scan_fwd(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate, int
                  size_t workspace_bytes, void* stream);
 
 /*
+ * ssm_scan_fwd_noalloc -- ssm_scan_fwd for callers that cannot allocate
+ * device memory. The Mamba pages have no counterpart to this call; it exists
+ * for callers that only get their input and output buffers and may not call
+ * cudaMalloc themselves (code running inside a memory pool or arena it does
+ * not own, real-time paths that must not allocate after start-up, plugins of
+ * a host framework). Same arguments, layouts and results as ssm_scan_fwd,
+ * without the workspace.
+ *
+ * Scratch: a fixed 8 MiB array reserved in device memory by the library on
+ * every GPU that loads it, kept until the process exits. Problems whose
+ * ssm_scan_workspace_bytes(...) exceeds 8 MiB are rejected with
+ * SSM_ERR_WORKSPACE (ssm_last_error_detail says how much they need); use
+ * ssm_scan_fwd for those.
+ *   - The first call on each device looks up the scratch's device address
+ *     (with that device current); make that first call before any stream
+ *     capture on the device.
+ *   - Every call on a device shares the one array and finds the previous
+ *     call's leftovers in it; nothing in it needs to start at zero (each call
+ *     writes every scratch word it reads). Calls that can run at the same
+ *     time on the GPU (different streams or host threads, without ordering
+ *     between them) race on the scratch and must be serialised by the caller.
+ *   - Allocates and frees nothing. Returns SSM_OK or SSM_ERR_*.
+ */
+int ssm_scan_fwd_noalloc(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
+                         int io_dtype, const void* x, const void* delta, const float* A,
+                         const void* B, const void* C, const float* D, const void* z,
+                         const float* delta_bias, int softplus, const float* h0, void* y,
+                         float* h_last, void* stream);
+
+/*
  * ssm_state_update -- one decode step: the recurrent, O(1)-per-token form of
  * the same recurrence (the §3.3 loop body for a single t), updating the
  * carried state in place.

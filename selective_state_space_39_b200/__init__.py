@@ -13,9 +13,10 @@ from ._binding import (  # noqa: F401
     scan_plan,
     scan_workspace_bytes,
     ssm_scan_fwd,
+    ssm_scan_fwd_noalloc,
     ssm_scan_status,
     ssm_state_update,
 )
 
-__all__ = ["ssm_scan_fwd", "ssm_state_update", "ssm_scan_status", "scan_plan",
+__all__ = ["ssm_scan_fwd", "ssm_scan_fwd_noalloc", "ssm_state_update", "ssm_scan_status", "scan_plan",
            "scan_workspace_bytes", "SsmError", "SSM_DTYPE_F32", "SSM_DTYPE_BF16", "lib"]

@@ -22,10 +22,10 @@ _STATUS = {0: "ok", -1: "invalid argument", -2: "unsupported size or dtype",
 
 
 class SsmError(RuntimeError):
-    def __init__(self, code: int, where: str):
+    def __init__(self, code: int, where: str, with_detail: bool = False):
         self.code = code
         detail = ""
-        if code in (-4, -5) and _lib is not None:
+        if (with_detail or code in (-4, -5)) and _lib is not None:
             detail = _lib.ssm_last_error_detail().decode(errors="replace")
         msg = f"{where}: {_STATUS.get(code, 'unknown status')} ({code})"
         super().__init__(msg + (f": {detail}" if detail else ""))
@@ -68,6 +68,10 @@ def lib() -> ctypes.CDLL:
         L.ssm_scan_fwd.argtypes = [_I64, _I64, _I64, _I64, ctypes.c_int, _VP, _VP, _VP, _VP, _VP,
                                    _VP, _VP, _VP, ctypes.c_int, _VP, _VP, _VP, _VP,
                                    ctypes.c_size_t, _VP]
+        L.ssm_scan_fwd_noalloc.restype = ctypes.c_int
+        L.ssm_scan_fwd_noalloc.argtypes = [_I64, _I64, _I64, _I64, ctypes.c_int, _VP, _VP, _VP,
+                                           _VP, _VP, _VP, _VP, _VP, ctypes.c_int, _VP, _VP, _VP,
+                                           _VP]
         L.ssm_scan_status.restype = ctypes.c_int
         L.ssm_scan_status.argtypes = [_VP, ctypes.c_size_t, _I64, _I64, _I64, _I64, ctypes.c_int,
                                       _VP]
@@ -163,6 +167,48 @@ def ssm_scan_fwd(x, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=Tr
                                 _stream_ptr(stream, dev))
     if rc != 0:
         raise SsmError(rc, "ssm_scan_fwd")
+    return y, h_last
+
+
+def ssm_scan_fwd_noalloc(x, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
+                         h0=None, y=None, h_last=None, return_last_state=True, stream=None):
+    """The selective scan through ssm_scan_fwd_noalloc of libssmscan.so.
+
+    For callers that cannot allocate device memory around the call: the
+    library takes its scratch from an 8 MiB array it reserves on each GPU, so
+    apart from the outputs (allocated here only when not passed in) nothing
+    is allocated. Problems needing more scratch raise SsmError (-3). Calls
+    that may overlap on the GPU share that scratch and must be ordered by the
+    caller. Same arguments and results as ssm_scan_fwd."""
+    if x.dim() != 3:
+        raise ValueError("x must be (batch, seqlen, dim)")
+    batch, L, dim = x.shape
+    if A.dim() != 2 or A.shape[0] != dim:
+        raise ValueError("A must be (dim, dstate)")
+    N = A.shape[1]
+    dev = x.device
+    bld, bln = (batch, L, dim), (batch, L, N)
+    px = _ptr(x, "x", x.dtype, bld)
+    pdl = _ptr(delta, "delta", x.dtype, bld, dev)
+    pA = _ptr(A, "A", torch.float32, (dim, N), dev)
+    pB = _ptr(B, "B", x.dtype, bln, dev)
+    pC = _ptr(C, "C", x.dtype, bln, dev)
+    pD = _ptr(D, "D", torch.float32, (dim,), dev)
+    pz = _ptr(z, "z", x.dtype, bld, dev)
+    pbias = _ptr(delta_bias, "delta_bias", torch.float32, (dim,), dev)
+    ph0 = _ptr(h0, "h0", torch.float32, (batch, dim, N), dev)
+    if y is None:
+        y = torch.empty(bld, dtype=x.dtype, device=dev)
+    py = _ptr(y, "y", x.dtype, bld, dev)
+    if h_last is None and return_last_state:
+        h_last = torch.empty((batch, dim, N), dtype=torch.float32, device=dev)
+    ph = _ptr(h_last, "h_last", torch.float32, (batch, dim, N), dev)
+    with torch.cuda.device(dev):
+        rc = lib().ssm_scan_fwd_noalloc(batch, L, dim, N, _io_code(x.dtype), px, pdl, pA, pB, pC,
+                                        pD, pz, pbias, 1 if softplus else 0, ph0, py, ph,
+                                        _stream_ptr(stream, dev))
+    if rc != 0:
+        raise SsmError(rc, "ssm_scan_fwd_noalloc", with_detail=True)
     return y, h_last
 
 

@@ -6,6 +6,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <mutex>
 
 #include "../../include/ssm_scan.h"
 #include "ssm_internal.h"
@@ -347,3 +348,75 @@ int ssm_state_update(int64_t batch, int64_t dim, int64_t dstate, int io_dtype, f
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Entry point for callers that cannot allocate device memory.
+//
+// Some callers have no way to call cudaMalloc around this library: code that
+// runs inside a memory pool or arena it does not own, real-time or embedded
+// callers that must not allocate after start-up, and plugins whose host
+// framework hands them only the input and output tensors. For them,
+// ssm_scan_fwd_noalloc takes its scratch (the per-CTA status words and the
+// sequence-segment carries that ssm_scan_fwd keeps in the caller's
+// workspace) from one array the library reserves in device memory for
+// every GPU that loads it, and calls ssm_scan_fwd with that array as the
+// workspace. It allocates nothing.
+namespace {
+
+constexpr size_t kNoallocScratchBytes = size_t(8) << 20;  // 8 MiB per GPU
+constexpr int kNoallocMaxDevices = 64;
+
+// The reserved scratch. In host code this name is only a stand-in for the
+// symbol, not a device address: the address must be looked up with
+// cudaGetSymbolAddress on each device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kNoallocMaxDevices] = {};
+
+// Device address of the scratch on the current device, looked up the first
+// time this device is seen (with the device current).
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(SSM_ERR_CUDA, "ssm_scan_fwd_noalloc: cudaGetDevice", e);
+  if (dev < 0 || dev >= kNoallocMaxDevices)
+    return fail(SSM_ERR_UNSUPPORTED, "ssm_scan_fwd_noalloc: device index above 63");
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(SSM_ERR_CUDA, "ssm_scan_fwd_noalloc: cudaGetSymbolAddress of the scratch", e);
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return SSM_OK;
+}
+
+}  // namespace
+
+extern "C" int ssm_scan_fwd_noalloc(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
+                                    int io_dtype, const void* x, const void* delta,
+                                    const float* A, const void* B, const void* C,
+                                    const float* D, const void* z, const float* delta_bias,
+                                    int softplus, const float* h0, void* y, float* h_last,
+                                    void* stream) {
+  const Dims d{batch, seqlen, dim, dstate, io_dtype};
+  const int st = dims_status(d);
+  if (st != SSM_OK) return st;
+  if (batch == 0 || dim == 0) return SSM_OK;
+  const size_t need = make_plan(d).bytes;
+  if (need > kNoallocScratchBytes) {
+    snprintf(g_detail, sizeof g_detail,
+             "ssm_scan_fwd_noalloc: this problem needs %zu bytes of scratch but the built-in "
+             "scratch holds %zu; call ssm_scan_fwd with a workspace instead",
+             need, kNoallocScratchBytes);
+    return SSM_ERR_WORKSPACE;
+  }
+  void* scratch = nullptr;
+  const int rc = noalloc_scratch(&scratch);
+  if (rc != SSM_OK) return rc;
+  return ssm_scan_fwd(batch, seqlen, dim, dstate, io_dtype, x, delta, A, B, C, D, z, delta_bias,
+                      softplus, h0, y, h_last, scratch, kNoallocScratchBytes, stream);
+}
