@@ -73,7 +73,7 @@ ScanPlan make_plan(const Dims& d) {
   ScanPlan pl{};
   const int T = kScanTileSteps;
   pl.channels_per_thread = scan_channels_per_thread((int)d.dstate);
-  pl.dtile = kScanThreads * pl.channels_per_thread;
+  pl.dtile = scan_threads(pl.channels_per_thread) * pl.channels_per_thread;
   pl.dtiles = (int)std::max<int64_t>(1, (d.dim + pl.dtile - 1) / pl.dtile);
   const int64_t tiles = std::max<int64_t>(1, (d.seqlen + T - 1) / T);
   const int64_t cols = std::max<int64_t>(1, d.batch * pl.dtiles);
@@ -258,7 +258,6 @@ int ssm_scan_fwd(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate, int
   p.nseg = pl.nseg;
   p.seg_steps = pl.seg_steps;
   p.softplus = softplus ? 1 : 0;
-  p.pair_store = (dim % 2) == 0;
   p.x = x; p.delta = delta; p.z = z; p.B = B; p.C = C;
   p.A = A; p.D = D; p.bias = delta_bias; p.h0 = h0;
   p.y = y; p.h_last = h_last;

@@ -86,9 +86,15 @@ struct Io<float> {
   __device__ static __forceinline__ float2 load2(const float* p) {
     return *reinterpret_cast<const float2*>(p);
   }
+  __device__ static __forceinline__ float4 load4(const float* p) {
+    return *reinterpret_cast<const float4*>(p);
+  }
   __device__ static __forceinline__ void store(float* p, float v) { *p = v; }
   __device__ static __forceinline__ void store2(float* p, float a, float b) {
     *reinterpret_cast<float2*>(p) = make_float2(a, b);
+  }
+  __device__ static __forceinline__ void store4(float* p, float a, float b, float c, float d) {
+    *reinterpret_cast<float4*>(p) = make_float4(a, b, c, d);
   }
 };
 
@@ -101,9 +107,16 @@ struct Io<uint16_t> {  // bf16 bits
     const uint32_t w = *reinterpret_cast<const uint32_t*>(p);
     return make_float2(bf16_lo(w), bf16_hi(w));
   }
+  __device__ static __forceinline__ float4 load4(const uint16_t* p) {
+    const uint2 w = *reinterpret_cast<const uint2*>(p);
+    return make_float4(bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y));
+  }
   __device__ static __forceinline__ void store(uint16_t* p, float v) { *p = f32_to_bf16(v); }
   __device__ static __forceinline__ void store2(uint16_t* p, float a, float b) {
     *reinterpret_cast<uint32_t*>(p) = pack_bf16x2(a, b);
+  }
+  __device__ static __forceinline__ void store4(uint16_t* p, float a, float b, float c, float d) {
+    *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(a, b), pack_bf16x2(c, d));
   }
 };
 
@@ -150,6 +163,15 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     if (mbar_try_wait(bar, parity)) return true;
     if (global_timer_ns() - t0 > limit_ns) return false;
   }
+}
+
+// ------------------------------------------- programmatic dependent launch --
+// Wait until the grid this one depends on has completed (or triggered); a
+// no-op when the launch did not enable programmatic serialisation.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Let the dependent grid start launching.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // -------------------------------------------------------------------- TMA --

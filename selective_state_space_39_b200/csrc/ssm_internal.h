@@ -16,7 +16,13 @@ namespace ssm {
 #ifndef SSM_STAGES
 #define SSM_STAGES 2
 #endif
-constexpr int kScanThreads = 128;
+#ifndef SSM_CTA_THREADS
+#define SSM_CTA_THREADS 128
+#endif
+constexpr int kScanThreads = SSM_CTA_THREADS;  // threads per CTA with 1 or 2 channels per thread
+// Threads per CTA of the scan for a given number of channels per thread
+// (4 channels per thread use half as many threads).
+constexpr int scan_threads(int cpt) { return cpt == 4 ? kScanThreads / 2 : kScanThreads; }
 constexpr int kScanTileSteps = SSM_TILE_STEPS;
 constexpr int kScanStages = SSM_STAGES;
 // Per-CTA status codes written to the workspace status area.
@@ -43,7 +49,6 @@ struct ScanParams {
   int batch, seqlen, dim;
   int nseg, seg_steps;
   int softplus;
-  int pair_store;  // dim even: two-channel vector stores are aligned
   const void* x;
   const void* delta;
   const void* z;
