@@ -42,7 +42,8 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(gen.SCAN_WORKLOADS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    choices=sorted(gen.SCAN_WORKLOADS) + sorted(gen.DECODE_WORKLOADS))
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
@@ -218,10 +219,85 @@ def reference_arm(args):
     return 0
 
 
+def decode_bench(args):
+    """--workload decode_*: ssm_state_update calls on a resident fp32 state
+    (one step = one call over all batch rows and channels). Timed twice: L2
+    flushed before every call, and back to back (the state fits in L2)."""
+    import torch
+
+    from selective_state_space_39_b200 import ssm_state_update
+    w = gen.DECODE_WORKLOADS[args.workload]
+    device = torch.device("cuda", 0)
+    dtype = torch.bfloat16 if w.io == "bf16" else torch.float32
+    const = gen.decode_constants(w.dim, w.dstate, w.seed)
+
+    def to_dev(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16).copy()).view(torch.bfloat16).to(device)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+    steps_in = [{k: to_dev(v) for k, v in gen.make_decode_inputs(
+        w.batch, w.dim, w.dstate, w.io, w.seed, i).items()} for i in range(8)]
+    A, D, bias = (to_dev(const[k]) for k in ("A", "D", "delta_bias"))
+    state = torch.zeros((w.batch, w.dim, w.dstate), dtype=torch.float32, device=device)
+    y = torch.empty((w.batch, w.dim), dtype=dtype, device=device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    def call(i):
+        s = steps_in[i % len(steps_in)]
+        ssm_state_update(state, s["x"], s["delta"], A, s["B"], s["C"], D=D, z=s["z"],
+                         delta_bias=bias, y=y)
+
+    for i in range(max(3, args.warmup)):
+        call(i)
+    torch.cuda.synchronize()
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    for i in range(K):
+        flush.fill_(i & 0xFF)
+        ev[i][0].record()
+        call(i)
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    cold_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(K):
+        call(i)
+    e1.record()
+    torch.cuda.synchronize()
+    warm_ms = e0.elapsed_time(e1) / K
+    es = 2 if w.io == "bf16" else 4
+    nbd = w.batch * w.dim
+    algo = nbd * w.dstate * 4 * 2 + nbd * es * 4 + 2 * w.batch * w.dstate * es + \
+        w.dim * w.dstate * 4 + 2 * w.dim * 4
+    peak, peak_kind = measured_hbm_peak()
+    gbs = algo / (cold_ms * 1e-3) / 1e9
+    line = {
+        "metric": "decode state-update elements/s (B·D per step) and HBM GB/s",
+        "value": nbd / (cold_ms * 1e-3), "unit": "elements/s", "n_gpus": 1, "steps": K,
+        "warmup": args.warmup, "ms_per_step": cold_ms, "higher_is_better": True,
+        "dtype": w.io, "data": "synthetic (seeded Philox4x32-10, Mamba-shaped recipe)",
+        "config": {"workload": w.name, "batch": w.batch, "dim": w.dim, "dstate": w.dstate,
+                   "l2": "flushed (256 MB write) before every timed call"},
+        "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(gbs / peak, 4), "algorithmic_bytes_per_launch": algo,
+                     "peak_kind": peak_kind},
+        "warm_l2": {"ms_per_step": warm_ms, "value": nbd / (warm_ms * 1e-3),
+                    "algorithmic_gbs": round(algo / (warm_ms * 1e-3) / 1e9, 1)},
+        "gpu_launches": 2 * K,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return reference_arm(args)
+    if args.workload in gen.DECODE_WORKLOADS:
+        return decode_bench(args)
 
     import torch
 

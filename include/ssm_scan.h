@@ -176,7 +176,9 @@ int ssm_state_update(int64_t batch, int64_t dim, int64_t dstate, int io_dtype, f
  * the last ssm_scan_fwd call that used this workspace (with these sizes)
  * finished normally: SSM_OK, or SSM_ERR_TIMEOUT if a bounded wait inside a
  * kernel gave up (its outputs are then incomplete). The wait bound is 2 s,
- * or SSM_SCAN_WAIT_LIMIT_NS nanoseconds from the environment.
+ * or SSM_SCAN_WAIT_LIMIT_NS nanoseconds from the environment. For testing
+ * this path, SSM_SCAN_TEST_STALL=1 in the environment makes the first CTA of
+ * the main pass (TMA path) wait for data that never arrives.
  */
 int ssm_scan_status(const void* workspace, size_t workspace_bytes, int64_t batch,
                     int64_t seqlen, int64_t dim, int64_t dstate, int io_dtype, void* stream);

@@ -268,6 +268,7 @@ int ssm_scan_fwd(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate, int
   p.ws_h0 = reinterpret_cast<float*>(ws + pl.off_h0);
   p.wait_limit_ns = (uint64_t)std::max(1L, env_long("SSM_SCAN_WAIT_LIMIT_NS",
                                                     (long)kDefaultWaitLimitNs));
+  p.test_stall = env_long("SSM_SCAN_TEST_STALL", 0) != 0 ? 1 : 0;
 
   const bool use_tma = tma_eligible(d, x, delta, z, B, C);
   ScanMaps maps;

@@ -65,6 +65,7 @@ struct ScanParams {
   float* ws_h0;     // [batch][dim][N] copy of h0 taken by the carry pass
   int* status;      // one int per CTA: carry-pass CTAs first, then main pass
   uint64_t wait_limit_ns;
+  int test_stall;   // test hook: CTA 0 of the main pass waits for 16 bytes that never arrive
 };
 
 struct alignas(64) ScanMaps {

@@ -171,11 +171,15 @@ __global__ void __launch_bounds__(NT, SSM_MIN_CTAS) scan_kernel(const ScanParams
   const uint32_t stage_tx = (uint32_t)((kAgg ? 2 : (has_z ? 3 : 2)) * L::kTileBytes +
                                        (kAgg ? 1 : 2) * L::kBCBytes);
 
+  // Test hook (ssm_scan_fwd with SSM_SCAN_TEST_STALL=1): the first CTA of the
+  // main pass expects 16 bytes more than its first tile brings, so its
+  // bounded wait runs out and it reports a timeout.
+  const bool stall_here = !kAgg && p.test_stall && dtile == 0 && seg == 0 && b == 0;
   auto issue_tile = [&](int it) {
     unsigned char* st = smem + (it % STAGES) * L::kStageBytes;
     uint64_t* bar = &full[it % STAGES];
     const int t0 = t_begin + it * T;
-    mbar_arrive_expect_tx(bar, stage_tx);
+    mbar_arrive_expect_tx(bar, stage_tx + ((stall_here && it == 0) ? 16u : 0u));
     tma_load_3d(st + L::kOffX, &maps.x, bar, dtile * DT, t0, b);
     tma_load_3d(st + L::kOffD, &maps.delta, bar, dtile * DT, t0, b);
     if (has_z) tma_load_3d(st + L::kOffZ, &maps.z, bar, dtile * DT, t0, b);
