@@ -31,7 +31,9 @@
  *   - Return value: SSM_OK, or a negative SSM_ERR_* code. Argument errors
  *     are detected on the host before anything is enqueued.
  *   - Pointers must be aligned to their element size (h0 / h_last to 8
- *     bytes, the decode state to 16 bytes when dstate % 4 == 0). The fast
+ *     bytes; for ssm_state_update the state and A to 16 bytes when
+ *     dstate % 4 == 0, else 8, and B, C to four elements when dstate % 4 == 0,
+ *     else two). The fast
  *     path also wants 16-byte aligned bases and rows (dim and dstate
  *     multiples of 16 bytes) and otherwise takes a slower path with plain
  *     loads (SSM_SCAN_DISABLE_TMA=1 in the environment forces that path).

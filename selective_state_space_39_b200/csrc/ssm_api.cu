@@ -329,6 +329,10 @@ int ssm_state_update(int64_t batch, int64_t dim, int64_t dstate, int io_dtype, f
   for (const void* p : f32_ptrs)
     if (p && !aligned(p, 4)) return SSM_ERR_INVALID_ARG;
   if (!aligned(state, dstate % 4 == 0 ? 16 : 8)) return SSM_ERR_INVALID_ARG;
+  // the kernel reads B, C in pairs of elements and rows of A as vectors
+  const size_t bc_align = (dstate % 4 == 0 ? 4 : 2) * es;
+  if (!aligned(B, bc_align) || !aligned(C, bc_align)) return SSM_ERR_INVALID_ARG;
+  if (!aligned(A, dstate % 4 == 0 ? 16 : 8)) return SSM_ERR_INVALID_ARG;
   const size_t nbd = (size_t)batch * dim, nbn = (size_t)batch * dstate;
   const size_t by = nbd * es;
   if (overlap(y, by, x, nbd * es) || overlap(y, by, delta, nbd * es) ||

@@ -612,7 +612,11 @@ __global__ void __launch_bounds__(NT, SSM_MIN_CTAS) scan_kernel(const ScanParams
 
 // -------------------------------------------------------------------------
 // Decode: one step of the recurrence per (batch, channel). LPC lanes share a
-// channel, SPT states each; y is reduced across the LPC lanes by shuffles.
+// channel, SPT states each (one float4 of the state per lane, so a warp reads
+// and writes contiguous runs of the (batch, dim, dstate) state); y is reduced
+// across the LPC lanes by shuffles. Every load of a thread is issued before
+// any arithmetic, so each thread makes a single round trip to memory: the
+// kernel is otherwise bound by the latency of its waves, not by bandwidth.
 template <typename IOT, int N>
 __global__ void __launch_bounds__(256) decode_kernel(const DecodeParams p) {
   using IO = Io<IOT>;
@@ -628,8 +632,36 @@ __global__ void __launch_bounds__(256) decode_kernel(const DecodeParams p) {
   const size_t cc = valid ? chan : 0;
   const int b = (int)(cc / p.dim), d = (int)(cc % p.dim);
 
+  // ---- all loads first ----
+  float* hp = p.state + cc * N + lane_in * SPT;
+  const float* Ar = p.A + (size_t)d * N + lane_in * SPT;
+  const IOT* Bp = reinterpret_cast<const IOT*>(p.B) + (size_t)b * N + lane_in * SPT;
+  const IOT* Cp = reinterpret_cast<const IOT*>(p.C) + (size_t)b * N + lane_in * SPT;
+  float h[SPT], a[SPT], bb[SPT], cv[SPT];
+  if constexpr (SPT == 4) {
+    const float4 t4 = *reinterpret_cast<const float4*>(hp);
+    h[0] = t4.x; h[1] = t4.y; h[2] = t4.z; h[3] = t4.w;
+    const float4 a4 = __ldg(reinterpret_cast<const float4*>(Ar));
+    a[0] = a4.x; a[1] = a4.y; a[2] = a4.z; a[3] = a4.w;
+    const float4 b4 = IO::load4(Bp), c4 = IO::load4(Cp);
+    bb[0] = b4.x; bb[1] = b4.y; bb[2] = b4.z; bb[3] = b4.w;
+    cv[0] = c4.x; cv[1] = c4.y; cv[2] = c4.z; cv[3] = c4.w;
+  } else {
+    const float2 t2 = *reinterpret_cast<const float2*>(hp);
+    h[0] = t2.x; h[1] = t2.y;
+    const float2 a2 = __ldg(reinterpret_cast<const float2*>(Ar));
+    a[0] = a2.x; a[1] = a2.y;
+    const float2 b2 = IO::load2(Bp), c2 = IO::load2(Cp);
+    bb[0] = b2.x; bb[1] = b2.y; cv[0] = c2.x; cv[1] = c2.y;
+  }
   const float xv = IO::load(reinterpret_cast<const IOT*>(p.x) + cc);
-  const float v = IO::load(reinterpret_cast<const IOT*>(p.delta) + cc) + (p.bias ? p.bias[d] : 0.f);
+  const float draw = IO::load(reinterpret_cast<const IOT*>(p.delta) + cc);
+  const float bias = p.bias ? p.bias[d] : 0.f;
+  const float Dd = p.D ? p.D[d] : 0.f;
+  const float zz = p.z ? IO::load(reinterpret_cast<const IOT*>(p.z) + cc) : 0.f;
+
+  // ---- arithmetic ----
+  const float v = draw + bias;
   float dt;
   if (!p.softplus) {
     dt = v;
@@ -639,24 +671,13 @@ __global__ void __launch_bounds__(256) decode_kernel(const DecodeParams p) {
     dt = v > kSoftplusCut ? v : log1pf(expf(v));
   }
   const float dx = dt * xv;
-  float* hp = p.state + cc * N + lane_in * SPT;
-  const float* Ar = p.A + (size_t)d * N + lane_in * SPT;
-  const IOT* Bp = reinterpret_cast<const IOT*>(p.B) + (size_t)b * N + lane_in * SPT;
-  const IOT* Cp = reinterpret_cast<const IOT*>(p.C) + (size_t)b * N + lane_in * SPT;
-  float h[SPT];
-  if constexpr (SPT == 4) {
-    const float4 t4 = *reinterpret_cast<const float4*>(hp);
-    h[0] = t4.x; h[1] = t4.y; h[2] = t4.z; h[3] = t4.w;
-  } else {
-    const float2 t2 = *reinterpret_cast<const float2*>(hp);
-    h[0] = t2.x; h[1] = t2.y;
-  }
+  const float dtl = kFast ? dt * kLog2e : dt;
   float acc = 0.f;
 #pragma unroll
   for (int k = 0; k < SPT; ++k) {
-    const float a = kFast ? ex2_approx(dt * Ar[k] * kLog2e) : expf(dt * Ar[k]);
-    h[k] = fmaf(a, h[k], dx * IO::load(Bp + k));
-    acc = fmaf(IO::load(Cp + k), h[k], acc);
+    const float e = kFast ? ex2_approx(dtl * a[k]) : expf(dtl * a[k]);
+    h[k] = fmaf(e, h[k], dx * bb[k]);
+    acc = fmaf(cv[k], h[k], acc);
   }
 #pragma unroll
   for (int off = LPC / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
@@ -667,9 +688,8 @@ __global__ void __launch_bounds__(256) decode_kernel(const DecodeParams p) {
     *reinterpret_cast<float2*>(hp) = make_float2(h[0], h[1]);
   }
   if (lane_in == 0) {
-    float yy = acc + (p.D ? p.D[d] : 0.f) * xv;
+    float yy = fmaf(Dd, xv, acc);
     if (p.z) {
-      const float zz = IO::load(reinterpret_cast<const IOT*>(p.z) + cc);
       if constexpr (kFast) {
         const float hz = 0.5f * zz;
         yy *= fmaf(hz, tanh_approx(hz), hz);

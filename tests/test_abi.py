@@ -128,6 +128,8 @@ def test_state_update_rejects_bad_arguments(L):
                                   a["sp"], a["y"], a["stream"])
     assert upd(state=None) == -1
     assert upd(state=FAKE + 8) == -1   # state needs 16-byte alignment for dstate % 4 == 0
+    assert upd(A=FAKE + 73728 + 8) == -1  # A rows are read as 16-byte vectors
+    assert upd(B=FAKE + 81922) == -1   # B is read four bf16 elements at a time
     assert upd(y=FAKE + 65536) == -1   # y overlaps x
     assert upd(y=FAKE + 64) == -1      # y overlaps the state
     assert upd(dstate=7) == -2
