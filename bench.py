@@ -277,6 +277,27 @@ def decode_bench(args):
     e1.record()
     torch.cuda.synchronize()
     warm_ms = e0.elapsed_time(e1) / K
+    # (4) the workload's whole decode run (w.steps consecutive calls) captured
+    #     in one CUDA graph and replayed: no per-call launch overhead.
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        call(0)  # first call outside capture (library state, attributes)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g):
+        for i in range(w.steps):
+            call(i)
+    g.replay()  # warm the graph
+    torch.cuda.synchronize()
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g0.record()
+    g.replay()
+    g1.record()
+    torch.cuda.synchronize()
+    graph_ms = g0.elapsed_time(g1) / w.steps
+    del g
     es = 2 if w.io == "bf16" else 4
     nbd = w.batch * w.dim
     algo = nbd * w.dstate * 4 * 2 + nbd * es * 4 + 2 * w.batch * w.dstate * es + \
@@ -298,6 +319,9 @@ def decode_bench(args):
                             "frac": round(algo / (read_ms * 1e-3) / 1e9 / peak, 4)},
         "warm_l2": {"ms_per_step": warm_ms, "value": nbd / (warm_ms * 1e-3),
                     "algorithmic_gbs": round(algo / (warm_ms * 1e-3) / 1e9, 1)},
+        "cuda_graph": {"calls": w.steps, "ms_per_step": graph_ms,
+                       "value": nbd / (graph_ms * 1e-3),
+                       "algorithmic_gbs": round(algo / (graph_ms * 1e-3) / 1e9, 1)},
         "gpu_launches": 2 * K,
     }
     print(json.dumps(line), flush=True)

@@ -9,8 +9,10 @@ arithmetic.
 
 The arithmetic lives in ``ssm_oracle.c`` (plain sequential fp64 loops). This
 module compiles it with gcc on first use and marshals numpy arrays to it.
-What it computes follows the page "Mamba 논문 리뷰: Selective State Space
-Models로 Transformer를 넘어서" (youngju.dev): §2.2 discretised recurrence,
+The backward pass (``selective_scan_bwd``) is the reverse-mode derivative
+of the same loop, written out in ``ssm_oracle.c``. What it computes follows
+the page "Mamba 논문 리뷰: Selective State Space Models로 Transformer를
+넘어서" (youngju.dev): §2.2 discretised recurrence,
 §3.1 softplus step size, §3.3 simplified ``selective_scan``, §3.4 block gate
 and D skip. Every function here is pinned by ``tests/test_oracle_pins.py``
 against closed forms, brute force and invariants.
@@ -67,6 +69,12 @@ class Oracle:
                       _F32P, ctypes.c_void_p, ctypes.c_void_p, _F32P, ctypes.c_void_p,
                       _F32P, ctypes.c_int, _F32P, _I64P, ctypes.c_int64, _F64P, _F64P,
                       ctypes.c_int]
+        fb = self.lib.oracle_selective_scan_bwd
+        fb.restype = ctypes.c_int
+        fb.argtypes = [ctypes.c_int64] * 4 + [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+                       _F32P, ctypes.c_void_p, ctypes.c_void_p, _F32P, ctypes.c_void_p,
+                       _F32P, ctypes.c_int, _F32P, ctypes.c_void_p, _F32P, _I64P,
+                       ctypes.c_int64] + [_F64P] * 9 + [ctypes.c_int]
         g = self.lib.oracle_state_update
         g.restype = ctypes.c_int
         g.argtypes = [ctypes.c_int64] * 3 + [ctypes.c_int, _F64P, ctypes.c_void_p,
@@ -149,6 +157,71 @@ class Oracle:
             h_last = h_last.reshape(batch, dim, N)
         return y, h_last
 
+    # -- the scan's gradients ----------------------------------------------
+    def selective_scan_bwd(self, x, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
+                           softplus=True, h0=None, dh_last=None, io="f32", channels=None,
+                           nthreads=1):
+        """Gradients of the loss sum(dy * y) + sum(dh_last * h_last) with
+        respect to every input of ``selective_scan`` (same arguments, plus the
+        upstream ``dy`` in the io type and ``dh_last`` fp32 or None).
+
+        Returns a dict of fp64 arrays: ``dx, ddelta, dz`` (batch, L, dim) —
+        ``dz`` None without z — ``dh0`` (batch, dim, N), and ``dA`` (dim, N),
+        ``dB, dC`` (batch, L, N), ``dD, ddelta_bias`` (dim). ``ddelta`` is the
+        gradient with respect to the raw delta (before bias and softplus).
+        With ``channels`` (a list of (b, d) pairs) the per-channel outputs are
+        (nchan, L) / (nchan, N) and the summed ones cover the listed channels
+        only."""
+        x = np.asarray(x)
+        batch, L, dim = x.shape
+        N = np.asarray(A).shape[1]
+        x = self._io_array(x, io, (batch, L, dim), "x")
+        delta = self._io_array(delta, io, (batch, L, dim), "delta")
+        B = self._io_array(B, io, (batch, L, N), "B")
+        C = self._io_array(C, io, (batch, L, N), "C")
+        z = self._io_array(z, io, (batch, L, dim), "z", optional=True)
+        dy = self._io_array(dy, io, (batch, L, dim), "dy")
+        A = self._f32_array(A, (dim, N), "A", optional=False)
+        D = self._f32_array(D, (dim,), "D")
+        delta_bias = self._f32_array(delta_bias, (dim,), "delta_bias")
+        h0 = self._f32_array(h0, (batch, dim, N), "h0")
+        dh_last = self._f32_array(dh_last, (batch, dim, N), "dh_last")
+        full = channels is None
+        if full:
+            bb, dd = np.meshgrid(np.arange(batch), np.arange(dim), indexing="ij")
+            chans = np.stack([bb.ravel(), dd.ravel()], axis=1).astype(np.int64)
+        else:
+            chans = np.ascontiguousarray(np.asarray(channels, dtype=np.int64).reshape(-1, 2))
+        nchan = chans.shape[0]
+        out = {k: np.empty((nchan, L), dtype=np.float64) for k in ("dx", "ddelta", "dz")}
+        out["dh0"] = np.empty((nchan, N), dtype=np.float64)
+        out["dA"] = np.empty((dim, N), dtype=np.float64)
+        out["dB"] = np.empty((batch, L, N), dtype=np.float64)
+        out["dC"] = np.empty((batch, L, N), dtype=np.float64)
+        out["dD"] = np.empty((dim,), dtype=np.float64)
+        out["ddelta_bias"] = np.empty((dim,), dtype=np.float64)
+        f64 = lambda k: self._ptr(out[k], ctypes.c_double)  # noqa: E731
+        rc = self.lib.oracle_selective_scan_bwd(
+            batch, L, dim, N, 1 if io == "bf16" else 0, self._ptr(x), self._ptr(delta),
+            self._ptr(A, ctypes.c_float), self._ptr(B), self._ptr(C),
+            self._ptr(D, ctypes.c_float), self._ptr(z), self._ptr(delta_bias, ctypes.c_float),
+            1 if softplus else 0, self._ptr(h0, ctypes.c_float), self._ptr(dy),
+            self._ptr(dh_last, ctypes.c_float), self._ptr(chans, ctypes.c_int64), nchan,
+            f64("dx"), f64("ddelta"), f64("dz"), f64("dh0"), f64("dA"), f64("dB"), f64("dC"),
+            f64("dD"), f64("ddelta_bias"), int(nthreads))
+        if rc == -2:
+            raise MemoryError("oracle_selective_scan_bwd ran out of memory")
+        if rc != 0:
+            raise ValueError("oracle_selective_scan_bwd rejected its arguments")
+        if z is None:
+            out["dz"] = None
+        if full:
+            for k in ("dx", "ddelta", "dz"):
+                if out[k] is not None:
+                    out[k] = out[k].reshape(batch, dim, L).transpose(0, 2, 1).copy()
+            out["dh0"] = out["dh0"].reshape(batch, dim, N)
+        return out
+
     # -- decode ------------------------------------------------------------
     def state_update(self, state, x, delta, A, B, C, D=None, z=None, delta_bias=None,
                      softplus=True, io="f32"):
@@ -197,3 +270,7 @@ def selective_scan(*args, **kwargs):
 
 def state_update(*args, **kwargs):
     return get().state_update(*args, **kwargs)
+
+
+def selective_scan_bwd(*args, **kwargs):
+    return get().selective_scan_bwd(*args, **kwargs)

@@ -204,3 +204,222 @@ int oracle_state_update(int64_t batch, int64_t dim, int64_t dstate, int is_bf16,
   }
   return 0;
 }
+
+/* ------------------------------------------------------------------------
+ * Backward pass: the gradient of the scan above, by reverse-mode
+ * differentiation of its loop (the recomputation-based training of the
+ * §3.3 Hardware-Aware algorithm needs exactly these gradients; the pages give
+ * no formulas for them, so they are derived here from the forward loop by the
+ * chain rule). For the loss  sum dy[b,t,d] y[b,t,d] + sum dh_last[b,d,n]
+ * h_last[b,d,n], with per-step quantities of one channel (b, d):
+ *
+ *   v_t = delta_t + bias,  Dt_t = softplus(v_t) (or v_t),  a_tn = exp(Dt_t A_n)
+ *   h_tn = a_tn h_(t-1)n + Dt_t B_tn x_t,   s_t = sum_n C_tn h_tn + D x_t
+ *   y_t = s_t SiLU(z_t)  (or s_t)
+ *
+ * the adjoint of the state, lam_tn = dLoss/dh_tn, obeys
+ *   lam_(L-1)n = C_(L-1)n g_(L-1) + dh_last_n,
+ *   lam_tn     = C_tn g_t + a_(t+1)n lam_(t+1)n,   g_t = dy_t SiLU(z_t)
+ * and the input gradients are
+ *   dz_t     = dy_t s_t SiLU'(z_t),   SiLU'(z) = sig(z) (1 + z (1 - sig(z)))
+ *   dx_t     = D g_t + Dt_t sum_n lam_tn B_tn
+ *   dDt_t    = x_t sum_n lam_tn B_tn + sum_n lam_tn A_n a_tn h_(t-1)n
+ *   ddelta_t = dDt_t softplus'(v_t) = dDt_t sig(v_t)  (1 above the cutoff 20,
+ *              where the forward uses the identity; 1 without softplus)
+ *   dbias    = sum_(b,t) ddelta_t,  dD = sum_(b,t) g_t x_t
+ *   dA_n     = sum_(b,t) lam_tn Dt_t a_tn h_(t-1)n
+ *   dB_tn    = sum_d lam_tn Dt_t x_t,   dC_tn = sum_d g_t h_tn
+ *   dh0_n    = a_0n lam_0n.
+ * ------------------------------------------------------------------------ */
+
+typedef struct {
+  scan_job fwd;         /* inputs; fwd.y / fwd.h_last unused */
+  const void* dy;       /* (batch, seqlen, dim) io type */
+  const float* dh_last; /* (batch, dim, dstate) fp32 or NULL */
+  /* per listed channel k */
+  double* dx;           /* (nchan, seqlen) */
+  double* ddelta;       /* (nchan, seqlen) */
+  double* dz;           /* (nchan, seqlen) or NULL */
+  double* dh0;          /* (nchan, dstate) */
+} bwd_job;
+
+/* Per-thread accumulators of the gradients summed over channels. */
+typedef struct {
+  double* dA;    /* (dim, dstate) */
+  double* dB;    /* (batch, seqlen, dstate) */
+  double* dC;    /* (batch, seqlen, dstate) */
+  double* dD;    /* (dim) */
+  double* dbias; /* (dim) */
+} bwd_acc;
+
+static double sigmoid(double v) { return 1.0 / (1.0 + exp(-v)); }
+
+/* One channel: the forward loop again, keeping every state, then the adjoint
+ * loop backwards in t. `hist` holds (seqlen + 1) * dstate doubles. */
+static void bwd_one_channel(const bwd_job* j, const bwd_acc* acc, int64_t k, double* hist,
+                            double* s_hist) {
+  const scan_job* f = &j->fwd;
+  const int64_t b = f->chans[2 * k], d = f->chans[2 * k + 1];
+  const int64_t L = f->seqlen, Dm = f->dim, N = f->dstate;
+  const double bias = f->bias ? (double)f->bias[d] : 0.0;
+  const double Dd = f->D ? (double)f->D[d] : 0.0;
+  /* hist[0] = h_(-1), hist[t + 1] = h_t */
+  for (int64_t n = 0; n < N; ++n)
+    hist[n] = f->h0 ? (double)f->h0[(b * Dm + d) * N + n] : 0.0;
+  for (int64_t t = 0; t < L; ++t) {
+    const int64_t i_bld = (b * L + t) * Dm + d, i_bln = (b * L + t) * N;
+    const double xv = widen(f->x, i_bld, f->is_bf16);
+    const double v = widen(f->delta, i_bld, f->is_bf16) + bias;
+    const double dt = f->softplus ? softplus(v) : v;
+    double s = 0.0;
+    for (int64_t n = 0; n < N; ++n) {
+      const double a = exp(dt * (double)f->A[d * N + n]);
+      hist[(t + 1) * N + n] = a * hist[t * N + n] + dt * widen(f->B, i_bln + n, f->is_bf16) * xv;
+      s += widen(f->C, i_bln + n, f->is_bf16) * hist[(t + 1) * N + n];
+    }
+    s_hist[t] = s + Dd * xv;
+  }
+  double lam[ORACLE_MAX_N];
+  for (int64_t n = 0; n < N; ++n)
+    lam[n] = j->dh_last ? (double)j->dh_last[(b * Dm + d) * N + n] : 0.0;
+  for (int64_t t = L - 1; t >= 0; --t) {
+    const int64_t i_bld = (b * L + t) * Dm + d, i_bln = (b * L + t) * N;
+    const double xv = widen(f->x, i_bld, f->is_bf16);
+    const double v = widen(f->delta, i_bld, f->is_bf16) + bias;
+    const double dt = f->softplus ? softplus(v) : v;
+    const double dyv = widen(j->dy, i_bld, f->is_bf16);
+    double g = dyv;
+    if (f->z) {
+      const double zv = widen(f->z, i_bld, f->is_bf16);
+      const double sg = sigmoid(zv);
+      g = dyv * zv * sg;
+      if (j->dz) j->dz[k * L + t] = dyv * s_hist[t] * sg * (1.0 + zv * (1.0 - sg));
+    }
+    acc->dD[d] += g * xv;
+    double sum_lb = 0.0, sum_la = 0.0;
+    for (int64_t n = 0; n < N; ++n) {
+      const double An = (double)f->A[d * N + n];
+      const double a = exp(dt * An);
+      const double hprev = hist[t * N + n];
+      lam[n] += widen(f->C, i_bln + n, f->is_bf16) * g;
+      acc->dC[i_bln + n] += g * hist[(t + 1) * N + n];
+      acc->dB[i_bln + n] += lam[n] * dt * xv;
+      sum_lb += lam[n] * widen(f->B, i_bln + n, f->is_bf16);
+      sum_la += lam[n] * An * a * hprev;
+      acc->dA[d * N + n] += lam[n] * dt * a * hprev;
+      lam[n] *= a;
+    }
+    j->dx[k * L + t] = Dd * g + dt * sum_lb;
+    const double ddt = xv * sum_lb + sum_la;
+    const double dv = !f->softplus ? ddt : (v > 20.0 ? ddt : ddt * sigmoid(v));
+    j->ddelta[k * L + t] = dv;
+    acc->dbias[d] += dv;
+  }
+  for (int64_t n = 0; n < N; ++n) j->dh0[k * N + n] = lam[n];
+}
+
+typedef struct {
+  const bwd_job* job;
+  bwd_acc acc;
+  int64_t lo, hi;
+  int failed;
+} bwd_slice;
+
+static void* bwd_worker(void* arg) {
+  bwd_slice* s = (bwd_slice*)arg;
+  const scan_job* f = &s->job->fwd;
+  double* hist = (double*)malloc((size_t)(f->seqlen + 1) * (size_t)f->dstate * sizeof(double));
+  double* s_hist = (double*)malloc((size_t)(f->seqlen > 0 ? f->seqlen : 1) * sizeof(double));
+  if (!hist || !s_hist) {
+    s->failed = 1;
+  } else {
+    for (int64_t k = s->lo; k < s->hi; ++k) bwd_one_channel(s->job, &s->acc, k, hist, s_hist);
+  }
+  free(hist);
+  free(s_hist);
+  return NULL;
+}
+
+/*
+ * oracle_selective_scan_bwd -- gradients of the scan for the `nchan`
+ * channels listed in `chans` (pairs (b, d)), over `nthreads` threads.
+ * Per-channel outputs dx, ddelta, dz (NULL when z is NULL), dh0 are indexed
+ * by list position. dA, dB, dC, dD, dbias are sums over the listed channels
+ * (all of a row b's channels give dB, dC of row b; all rows b of channel d
+ * give dA[d], dD[d], dbias[d]); they are overwritten. Threads accumulate
+ * privately and the sums are added in thread order, so results do not depend
+ * on timing. Returns 0, -1 on bad arguments, -2 when memory runs out.
+ */
+int oracle_selective_scan_bwd(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
+                              int is_bf16, const void* x, const void* delta, const float* A,
+                              const void* B, const void* C, const float* D, const void* z,
+                              const float* bias, int softplus_on, const float* h0,
+                              const void* dy, const float* dh_last, const int64_t* chans,
+                              int64_t nchan, double* dx, double* ddelta, double* dz,
+                              double* dh0, double* dA, double* dB, double* dC, double* dD,
+                              double* dbias, int nthreads) {
+  if (batch < 0 || seqlen < 0 || dim < 0 || dstate <= 0 || dstate > ORACLE_MAX_N) return -1;
+  if (!x || !delta || !A || !B || !C || !dy || !chans || !dx || !ddelta || !dh0 || !dA ||
+      !dB || !dC || !dD || !dbias || (z && !dz))
+    return -1;
+  for (int64_t k = 0; k < nchan; ++k)
+    if (chans[2 * k] < 0 || chans[2 * k] >= batch || chans[2 * k + 1] < 0 ||
+        chans[2 * k + 1] >= dim)
+      return -1;
+  if (nthreads < 1) nthreads = 1;
+  if (nthreads > 64) nthreads = 64;
+  if (nchan < nthreads) nthreads = nchan > 0 ? (int)nchan : 1;
+  bwd_job job;
+  scan_job f = {batch, seqlen, dim, dstate, is_bf16, x, delta, A, B, C, D, z,
+                bias, softplus_on, h0, chans, nchan, NULL, NULL};
+  job.fwd = f;
+  job.dy = dy;
+  job.dh_last = dh_last;
+  job.dx = dx;
+  job.ddelta = ddelta;
+  job.dz = z ? dz : NULL;
+  job.dh0 = dh0;
+  const size_t nA = (size_t)dim * dstate, nBC = (size_t)batch * seqlen * dstate;
+  const size_t per = nA + 2 * nBC + 2 * (size_t)dim;
+  bwd_slice sl[64];
+  pthread_t tid[64];
+  int rc = 0;
+  for (int w = 0; w < nthreads; ++w) {
+    double* m = (double*)calloc(per > 0 ? per : 1, sizeof(double));
+    sl[w].job = &job;
+    sl[w].lo = nchan * w / nthreads;
+    sl[w].hi = nchan * (w + 1) / nthreads;
+    sl[w].failed = m == NULL;
+    sl[w].acc.dA = m;
+    sl[w].acc.dB = m ? m + nA : NULL;
+    sl[w].acc.dC = m ? m + nA + nBC : NULL;
+    sl[w].acc.dD = m ? m + nA + 2 * nBC : NULL;
+    sl[w].acc.dbias = m ? m + nA + 2 * nBC + dim : NULL;
+    tid[w] = 0;
+  }
+  for (int w = 0; w < nthreads; ++w) {
+    if (sl[w].failed) continue;
+    if (nthreads == 1 || pthread_create(&tid[w], NULL, bwd_worker, &sl[w]) != 0) {
+      tid[w] = 0;
+      bwd_worker(&sl[w]);
+    }
+  }
+  for (int w = 0; w < nthreads; ++w)
+    if (tid[w]) pthread_join(tid[w], NULL);
+  memset(dA, 0, nA * sizeof(double));
+  memset(dB, 0, nBC * sizeof(double));
+  memset(dC, 0, nBC * sizeof(double));
+  memset(dD, 0, (size_t)dim * sizeof(double));
+  memset(dbias, 0, (size_t)dim * sizeof(double));
+  for (int w = 0; w < nthreads; ++w) {
+    if (sl[w].failed) rc = -2;
+    if (!sl[w].acc.dA) continue;
+    for (size_t i = 0; i < nA; ++i) dA[i] += sl[w].acc.dA[i];
+    for (size_t i = 0; i < nBC; ++i) dB[i] += sl[w].acc.dB[i];
+    for (size_t i = 0; i < nBC; ++i) dC[i] += sl[w].acc.dC[i];
+    for (int64_t i = 0; i < dim; ++i) dD[i] += sl[w].acc.dD[i];
+    for (int64_t i = 0; i < dim; ++i) dbias[i] += sl[w].acc.dbias[i];
+    free(sl[w].acc.dA);
+  }
+  return rc;
+}

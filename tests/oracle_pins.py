@@ -311,6 +311,113 @@ def pin_decode_single_step_by_hand(o):
             _close(state[b, d], h, 1e-13, 1e-15, what="decode by hand h")
 
 
+# --------------------------------------------------------------------------
+# pins of the backward pass (gradients of the scan)
+_GRAD_OF = {"x": "dx", "delta": "ddelta", "z": "dz", "B": "dB", "C": "dC", "A": "dA",
+            "D": "dD", "delta_bias": "ddelta_bias", "h0": "dh0"}
+
+
+def _loss(o, c, dy, dh_last):
+    """sum dy * y + sum dh_last * h_last, in fp64, through the forward oracle."""
+    y, hl = o.selective_scan(c["x"], c["delta"], c["A"], c["B"], c["C"], D=c["D"], z=c["z"],
+                             delta_bias=c["delta_bias"], softplus=c["softplus"], h0=c["h0"])
+    return float(np.sum(dy.astype(np.float64) * y) + np.sum(dh_last.astype(np.float64) * hl))
+
+
+def _bwd(o, c, dy, dh_last):
+    return o.selective_scan_bwd(c["x"], c["delta"], c["A"], c["B"], c["C"], dy, D=c["D"],
+                                z=c["z"], delta_bias=c["delta_bias"], softplus=c["softplus"],
+                                h0=c["h0"], dh_last=dh_last)
+
+
+def _finite_differences(o, c, dy, dh_last, name):
+    """Central differences of the loss in every fp32 element of input `name`,
+    using the step the fp32 rounding actually takes."""
+    base = c[name]
+    fd = np.zeros(base.shape, dtype=np.float64)
+    for i in np.ndindex(base.shape):
+        v = float(base[i])
+        h = 2.0 ** -11 * max(2.0 ** -4, abs(v))
+        hi, lo = np.float32(v + h), np.float32(v - h)
+        cc = dict(c)
+        arr = base.copy()
+        arr[i] = hi
+        cc[name] = arr
+        f_hi = _loss(o, cc, dy, dh_last)
+        arr = base.copy()
+        arr[i] = lo
+        cc[name] = arr
+        f_lo = _loss(o, cc, dy, dh_last)
+        fd[i] = (f_hi - f_lo) / (float(hi) - float(lo))
+    return fd
+
+
+def _check_fd(o, c, seed, what):
+    r = _rng(seed)
+    dy = _f32(r.standard_normal(c["x"].shape))
+    dh_last = _f32(r.standard_normal((c["x"].shape[0], c["x"].shape[2], c["A"].shape[1])))
+    g = _bwd(o, c, dy, dh_last)
+    for name, gname in _GRAD_OF.items():
+        if c.get(name) is None:
+            if name == "z":
+                assert g["dz"] is None, f"{what}: dz without z"
+            continue
+        fd = _finite_differences(o, c, dy, dh_last, name)
+        scale = max(1.0, float(np.max(np.abs(fd))))
+        _close(g[gname], fd, 0.0, 2e-6 * scale, what=f"{what}: {gname} vs central differences")
+
+
+def pin_bwd_finite_differences(o):
+    """Every gradient of the backward pass equals central differences of the
+    (separately pinned) forward oracle: gate, skip, h0, bias and softplus on."""
+    c = random_case(101, batch=2, L=6, dim=3, N=4)
+    _check_fd(o, c, 102, "all terms")
+
+
+def pin_bwd_finite_differences_plain(o):
+    """The same without gate, skip, h0 or softplus, and with a bias so large
+    that softplus would sit above its cutoff of 20 (checked separately)."""
+    c = random_case(103, batch=2, L=5, dim=2, N=3, gate=False, skip=False, h0=False,
+                    softplus=False)
+    # without softplus keep Delta > 0, so the recurrence decays
+    c["delta"] = _f32(np.abs(c["delta"]))
+    c["delta_bias"] = _f32(np.abs(c["delta_bias"]))
+    _check_fd(o, c, 104, "plain")
+    c = random_case(105, batch=1, L=4, dim=2, N=2)
+    c["delta_bias"] = _f32([21.0, 0.3])  # channel 0 above the softplus cutoff
+    c["A"] = _f32([[-0.01, -0.02], [-1.0, -2.0]])
+    _check_fd(o, c, 106, "softplus cutoff")
+
+
+def pin_bwd_autograd(o):
+    """Reverse-mode autodiff (torch, fp64, CPU) of the §3.3 loop with the
+    §3.4 skip and gate, written here from the page, agrees with the
+    hand-derived adjoint loop of the oracle."""
+    import torch
+    c = random_case(107, batch=2, L=5, dim=3, N=4)
+    r = _rng(108)
+    dy = _f32(r.standard_normal(c["x"].shape))
+    dh_last = _f32(r.standard_normal((2, 3, 4)))
+    t = {k: torch.tensor(v.astype(np.float64), requires_grad=True)
+         for k, v in c.items() if isinstance(v, np.ndarray)}
+    dt = torch.nn.functional.softplus(t["delta"] + t["delta_bias"], threshold=20.0)
+    h = t["h0"]
+    ys = []
+    for s in range(c["x"].shape[1]):
+        dA = torch.exp(dt[:, s, :, None] * t["A"])
+        dBx = dt[:, s, :, None] * t["B"][:, s, None, :] * t["x"][:, s, :, None]
+        h = dA * h + dBx
+        yy = (h * t["C"][:, s, None, :]).sum(-1) + t["D"] * t["x"][:, s]
+        ys.append(yy * torch.nn.functional.silu(t["z"][:, s]))
+    y = torch.stack(ys, dim=1)
+    loss = (y * torch.tensor(dy.astype(np.float64))).sum() + \
+        (h * torch.tensor(dh_last.astype(np.float64))).sum()
+    loss.backward()
+    g = _bwd(o, c, dy, dh_last)
+    for name, gname in _GRAD_OF.items():
+        _close(g[gname], t[name].grad.numpy(), 1e-10, 1e-12, what=f"autograd {gname}")
+
+
 ALL_PINS = [
     pin_softplus_library,
     pin_silu_library,
@@ -325,4 +432,7 @@ ALL_PINS = [
     pin_golden_hand_worked,
     pin_decode_steps_equal_scan,
     pin_decode_single_step_by_hand,
+    pin_bwd_finite_differences,
+    pin_bwd_finite_differences_plain,
+    pin_bwd_autograd,
 ]

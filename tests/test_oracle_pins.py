@@ -72,6 +72,23 @@ MUTANTS = {
     "decode_drops_gate": ("      if (z) acc *= silu(widen(z, i_bd, is_bf16));\n", ""),
     "decode_state_not_kept": ("        h[n] = dA * h[n] + dB * xv;\n        acc +=",
                               "        const double hn = dA * h[n] + dB * xv;\n        acc += 0 * hn +"),
+    # backward pass
+    "bwd_drops_A_term_of_dDelta": ("const double ddt = xv * sum_lb + sum_la;",
+                                   "const double ddt = xv * sum_lb;"),
+    "bwd_dA_uses_new_state": ("acc->dA[d * N + n] += lam[n] * dt * a * hprev;",
+                              "acc->dA[d * N + n] += lam[n] * dt * hist[(t + 1) * N + n];"),
+    "bwd_adjoint_not_decayed": ("      lam[n] *= a;\n", "      lam[n] *= 1.0;\n"),
+    "bwd_silu_derivative_is_sigmoid": ("sg * (1.0 + zv * (1.0 - sg))", "sg"),
+    "bwd_softplus_derivative_dropped": ("(v > 20.0 ? ddt : ddt * sigmoid(v))", "ddt"),
+    "bwd_dB_without_delta": ("acc->dB[i_bln + n] += lam[n] * dt * xv;",
+                             "acc->dB[i_bln + n] += lam[n] * xv;"),
+    "bwd_dC_ignores_gate": ("acc->dC[i_bln + n] += g * hist[(t + 1) * N + n];",
+                            "acc->dC[i_bln + n] += dyv * hist[(t + 1) * N + n];"),
+    "bwd_dh_last_ignored": ("lam[n] = j->dh_last ? (double)j->dh_last[(b * Dm + d) * N + n] : 0.0;",
+                            "lam[n] = 0.0;"),
+    "bwd_dx_drops_skip": ("j->dx[k * L + t] = Dd * g + dt * sum_lb;",
+                          "j->dx[k * L + t] = dt * sum_lb;"),
+    "bwd_dh0_before_decay": ("      lam[n] *= a;\n", "      if (t > 0) lam[n] *= a;\n"),
 }
 
 
