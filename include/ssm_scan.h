@@ -174,6 +174,51 @@ int ssm_state_update(int64_t batch, int64_t dim, int64_t dstate, int io_dtype, f
                      int softplus, void* y, void* stream);
 
 /*
+ * ssm_scan_bwd_workspace_bytes -- bytes of device workspace ssm_scan_bwd
+ * needs for these sizes (0 for unsupported sizes or dtypes). It holds state
+ * checkpoints every 4 steps: about 4 * batch * seqlen * dim * dstate / 4
+ * bytes, plus per-segment carries and partial sums.
+ */
+size_t ssm_scan_bwd_workspace_bytes(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
+                                    int io_dtype);
+
+/*
+ * ssm_scan_bwd -- gradients of the selective scan (the backward pass that the
+ * §3.3 Hardware-Aware algorithm trains with: intermediate states are not
+ * stored by the forward but recomputed here from the inputs). For the loss
+ *
+ *   sum_{b,t,d} dy[b,t,d] * y[b,t,d]  +  sum_{b,d,n} dh_last[b,d,n] * h_last[b,d,n]
+ *
+ * with y, h_last as ssm_scan_fwd computes them from the same inputs, it
+ * writes (overwrites) the gradient with respect to every input:
+ *
+ *   dx, ddelta, dz : (batch, seqlen, dim)   io_dtype; ddelta is the gradient
+ *                    with respect to the raw delta (before bias and softplus);
+ *                    dz must be NULL exactly when z is NULL
+ *   dA             : (dim, dstate) fp32
+ *   dB, dC         : (batch, seqlen, dstate) fp32 (sums over channels)
+ *   dD, ddelta_bias: (dim) fp32, nullable (not written when NULL); dD is
+ *                    the gradient at the given D, or at D = 0 when D is NULL
+ *   dh0            : (batch, dim, dstate) fp32, nullable; the gradient with
+ *                    respect to the initial state (h0, or the zero state)
+ *
+ * Inputs x, delta, A, B, C, D, z, delta_bias, softplus, h0 are those of the
+ * forward call; dy is (batch, seqlen, dim) io_dtype and dh_last (batch, dim,
+ * dstate) fp32 or NULL (zero). dstate must be 2, 4, 8 or 16. No output may
+ * overlap an input or another output. workspace: device memory of at least
+ * ssm_scan_bwd_workspace_bytes(), 16-byte aligned, used as scratch only.
+ * Sums over channels, batch rows and segments are taken in a fixed order:
+ * results do not depend on scheduling. Returns SSM_OK or SSM_ERR_*.
+ */
+int ssm_scan_bwd(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate, int io_dtype,
+                 const void* x, const void* delta, const float* A, const void* B,
+                 const void* C, const float* D, const void* z, const float* delta_bias,
+                 int softplus, const float* h0, const void* dy, const float* dh_last,
+                 void* dx, void* ddelta, float* dA, float* dB, float* dC, float* dD, void* dz,
+                 float* ddelta_bias, float* dh0, void* workspace, size_t workspace_bytes,
+                 void* stream);
+
+/*
  * ssm_scan_status -- synchronise `stream`, then report whether every CTA of
  * the last ssm_scan_fwd call that used this workspace (with these sizes)
  * finished normally: SSM_OK, or SSM_ERR_TIMEOUT if a bounded wait inside a

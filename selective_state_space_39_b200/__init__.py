@@ -10,13 +10,16 @@ from ._binding import (  # noqa: F401
     ScanPlan,
     SsmError,
     lib,
+    scan_bwd_workspace_bytes,
     scan_plan,
     scan_workspace_bytes,
+    ssm_scan_bwd,
     ssm_scan_fwd,
     ssm_scan_fwd_noalloc,
     ssm_scan_status,
     ssm_state_update,
 )
 
-__all__ = ["ssm_scan_fwd", "ssm_scan_fwd_noalloc", "ssm_state_update", "ssm_scan_status", "scan_plan",
-           "scan_workspace_bytes", "SsmError", "SSM_DTYPE_F32", "SSM_DTYPE_BF16", "lib"]
+__all__ = ["ssm_scan_fwd", "ssm_scan_fwd_noalloc", "ssm_scan_bwd", "ssm_state_update",
+           "ssm_scan_status", "scan_plan", "scan_workspace_bytes", "scan_bwd_workspace_bytes",
+           "SsmError", "SSM_DTYPE_F32", "SSM_DTYPE_BF16", "lib"]

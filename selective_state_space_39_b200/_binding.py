@@ -75,6 +75,11 @@ def lib() -> ctypes.CDLL:
         L.ssm_scan_status.restype = ctypes.c_int
         L.ssm_scan_status.argtypes = [_VP, ctypes.c_size_t, _I64, _I64, _I64, _I64, ctypes.c_int,
                                       _VP]
+        L.ssm_scan_bwd_workspace_bytes.restype = ctypes.c_size_t
+        L.ssm_scan_bwd_workspace_bytes.argtypes = [_I64, _I64, _I64, _I64, ctypes.c_int]
+        L.ssm_scan_bwd.restype = ctypes.c_int
+        L.ssm_scan_bwd.argtypes = [_I64, _I64, _I64, _I64, ctypes.c_int] + [_VP] * 8 + \
+            [ctypes.c_int] + [_VP] * 13 + [ctypes.c_size_t, _VP]
         L.ssm_state_update.restype = ctypes.c_int
         L.ssm_state_update.argtypes = [_I64, _I64, _I64, ctypes.c_int, _VP, _VP, _VP, _VP, _VP,
                                        _VP, _VP, _VP, _VP, ctypes.c_int, _VP, _VP]
@@ -168,6 +173,63 @@ def ssm_scan_fwd(x, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=Tr
     if rc != 0:
         raise SsmError(rc, "ssm_scan_fwd")
     return y, h_last
+
+
+def scan_bwd_workspace_bytes(batch, seqlen, dim, dstate, dtype=torch.bfloat16) -> int:
+    return int(lib().ssm_scan_bwd_workspace_bytes(batch, seqlen, dim, dstate, _io_code(dtype)))
+
+
+def ssm_scan_bwd(x, delta, A, B, C, dy, D=None, z=None, delta_bias=None, softplus=True, h0=None,
+                 dh_last=None, workspace=None, want_dD=True, want_ddelta_bias=True, want_dh0=True,
+                 stream=None):
+    """Gradients of the selective scan through ssm_scan_bwd of libssmscan.so,
+    for the loss sum(dy * y) + sum(dh_last * h_last) (dh_last may be None).
+
+    Inputs as for ssm_scan_fwd, plus dy (batch, L, dim) in the io dtype and
+    dh_last (batch, dim, N) float32. Returns a dict: dx, ddelta, dz (io
+    dtype; dz None without z), dA (dim, N), dB, dC (batch, L, N), dD,
+    ddelta_bias (dim,), dh0 (batch, dim, N), all float32 except the first
+    three (a gradient not asked for is None)."""
+    if x.dim() != 3:
+        raise ValueError("x must be (batch, seqlen, dim)")
+    batch, L, dim = x.shape
+    if A.dim() != 2 or A.shape[0] != dim:
+        raise ValueError("A must be (dim, dstate)")
+    N = A.shape[1]
+    dev = x.device
+    io = _io_code(x.dtype)
+    bld, bln, bdn = (batch, L, dim), (batch, L, N), (batch, dim, N)
+    f32 = torch.float32
+    ins = [_ptr(x, "x", x.dtype, bld), _ptr(delta, "delta", x.dtype, bld, dev),
+           _ptr(A, "A", f32, (dim, N), dev), _ptr(B, "B", x.dtype, bln, dev),
+           _ptr(C, "C", x.dtype, bln, dev), _ptr(D, "D", f32, (dim,), dev),
+           _ptr(z, "z", x.dtype, bld, dev), _ptr(delta_bias, "delta_bias", f32, (dim,), dev)]
+    ph0 = _ptr(h0, "h0", f32, bdn, dev)
+    pdy = _ptr(dy, "dy", x.dtype, bld, dev)
+    pdh = _ptr(dh_last, "dh_last", f32, bdn, dev)
+    g = {"dx": torch.empty(bld, dtype=x.dtype, device=dev),
+         "ddelta": torch.empty(bld, dtype=x.dtype, device=dev),
+         "dz": torch.empty(bld, dtype=x.dtype, device=dev) if z is not None else None,
+         "dA": torch.empty((dim, N), dtype=f32, device=dev),
+         "dB": torch.empty(bln, dtype=f32, device=dev),
+         "dC": torch.empty(bln, dtype=f32, device=dev),
+         "dD": torch.empty((dim,), dtype=f32, device=dev) if want_dD else None,
+         "ddelta_bias": torch.empty((dim,), dtype=f32, device=dev) if want_ddelta_bias else None,
+         "dh0": torch.empty(bdn, dtype=f32, device=dev) if want_dh0 else None}
+    P = {k: (v.data_ptr() if v is not None else None) for k, v in g.items()}
+    with torch.cuda.device(dev):
+        need = scan_bwd_workspace_bytes(batch, L, dim, N, x.dtype)
+        if workspace is None:
+            workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+        pws = _ptr(workspace, "workspace", None, None, dev)
+        rc = lib().ssm_scan_bwd(batch, L, dim, N, io, *ins, 1 if softplus else 0, ph0, pdy, pdh,
+                                P["dx"], P["ddelta"], P["dA"], P["dB"], P["dC"], P["dD"],
+                                P["dz"], P["ddelta_bias"], P["dh0"], pws,
+                                workspace.numel() * workspace.element_size(),
+                                _stream_ptr(stream, dev))
+    if rc != 0:
+        raise SsmError(rc, "ssm_scan_bwd", with_detail=True)
+    return g
 
 
 def ssm_scan_fwd_noalloc(x, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,

@@ -102,6 +102,56 @@ ScanPlan make_plan(const Dims& d) {
   return pl;
 }
 
+// Split of the backward pass: enough (segment, channel block, batch row) CTAs
+// for about 16 resident carry-pass CTAs per SM, segments of at least 8 tiles
+// of 4 steps; the workspace layout follows BwdParams.
+int bwd_dims_status(const Dims& d) {
+  if (d.io != SSM_DTYPE_F32 && d.io != SSM_DTYPE_BF16) return SSM_ERR_UNSUPPORTED;
+  if (d.batch < 0 || d.seqlen < 0 || d.dim < 0 || d.dstate <= 0) return SSM_ERR_INVALID_ARG;
+  if (!scan_bwd_dstate_supported((int)std::min<int64_t>(d.dstate, 1 << 20)))
+    return SSM_ERR_UNSUPPORTED;
+  if (d.batch > 65535 || d.dim > (1 << 24) || d.seqlen > (1 << 30)) return SSM_ERR_UNSUPPORTED;
+  return SSM_OK;
+}
+
+BwdPlan make_bwd_plan(const Dims& d) {
+  BwdPlan pl{};
+  const int T = kBwdTileSteps;
+  pl.dblocks = (int)std::max<int64_t>(1, (d.dim + kBwdThreads - 1) / kBwdThreads);
+  const int64_t tiles = std::max<int64_t>(1, (d.seqlen + T - 1) / T);
+  pl.ntiles = (int)tiles;
+  const int64_t cols = std::max<int64_t>(1, d.batch * pl.dblocks);
+  int64_t nseg = std::max<int64_t>(1, ((int64_t)device_sms() * 16 + cols - 1) / cols);
+  nseg = std::min<int64_t>(nseg, std::max<int64_t>(1, tiles / 8));
+  const long forced = env_long("SSM_SCAN_BWD_SEGMENTS", 0);
+  if (forced > 0) nseg = forced;
+  nseg = std::min<int64_t>(std::min<int64_t>(nseg, tiles), 65535);
+  const int64_t tiles_per_seg = (tiles + nseg - 1) / nseg;
+  pl.seg_steps = (int)(tiles_per_seg * T);
+  pl.nseg = (int)((tiles + tiles_per_seg - 1) / tiles_per_seg);
+  const size_t B = (size_t)d.batch, N = (size_t)d.dstate, Dm = (size_t)d.dim;
+  const size_t S = (size_t)pl.nseg, L = (size_t)std::max<int64_t>(d.seqlen, 0);
+  size_t off = 0;
+  auto take = [&](size_t floats) {
+    const size_t at = off;
+    off = align_up(off + sizeof(float) * floats, 256);
+    return at;
+  };
+  pl.off_ck = take(B * tiles * N * Dm);
+  pl.off_qk = take(B * tiles * Dm);
+  pl.off_hloc = take(B * S * N * Dm);
+  pl.off_mloc = take(B * S * N * Dm);
+  pl.off_hin = take(B * S * N * Dm);
+  pl.off_muin = take(B * S * N * Dm);
+  pl.off_qseg = take(B * S * Dm);
+  pl.off_dbc = take(B * pl.dblocks * L * 2 * N);
+  pl.off_dA = take(B * S * N * Dm);
+  pl.off_dD = take(B * S * Dm);
+  pl.off_dbias = take(B * S * Dm);
+  pl.bytes = off;
+  return pl;
+}
+
 // --- TMA tensor maps --------------------------------------------------------
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -349,6 +399,106 @@ int ssm_state_update(int64_t batch, int64_t dim, int64_t dstate, int io_dtype, f
   return cuda_status(launch_decode(p, (int)dstate, io_dtype == SSM_DTYPE_BF16,
                                    static_cast<cudaStream_t>(stream)),
                      "decode launch");
+}
+
+size_t ssm_scan_bwd_workspace_bytes(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
+                                    int io_dtype) {
+  const Dims d{batch, seqlen, dim, dstate, io_dtype};
+  if (bwd_dims_status(d) != SSM_OK) return 0;
+  if (batch == 0 || dim == 0 || seqlen == 0) return 0;
+  return make_bwd_plan(d).bytes;
+}
+
+int ssm_scan_bwd(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate, int io_dtype,
+                 const void* x, const void* delta, const float* A, const void* B,
+                 const void* C, const float* D, const void* z, const float* delta_bias,
+                 int softplus, const float* h0, const void* dy, const float* dh_last,
+                 void* dx, void* ddelta, float* dA, float* dB, float* dC, float* dD, void* dz,
+                 float* ddelta_bias, float* dh0, void* workspace, size_t workspace_bytes,
+                 void* stream) {
+  const Dims d{batch, seqlen, dim, dstate, io_dtype};
+  int st = bwd_dims_status(d);
+  if (st != SSM_OK) return st;
+  if (batch == 0 || dim == 0) return SSM_OK;
+  if (!A || !dA || (!z) != (!dz)) return SSM_ERR_INVALID_ARG;
+  if (seqlen > 0 && (!x || !delta || !B || !C || !dy || !dx || !ddelta || !dB || !dC))
+    return SSM_ERR_INVALID_ARG;
+  const size_t es = io_bytes(io_dtype);
+  const void* io_ptrs[] = {x, delta, B, C, z, dy, dx, ddelta, dz};
+  for (const void* p : io_ptrs)
+    if (p && !aligned(p, es)) return SSM_ERR_INVALID_ARG;
+  const void* f32_ptrs[] = {A, D, delta_bias, h0, dh_last, dA, dB, dC, dD, ddelta_bias, dh0};
+  for (const void* p : f32_ptrs)
+    if (p && !aligned(p, 4)) return SSM_ERR_INVALID_ARG;
+  // no output may overlap an input or another output
+  const size_t n_bld = (size_t)batch * seqlen * dim, n_bln = (size_t)batch * seqlen * dstate;
+  const size_t n_bdn = (size_t)batch * dim * dstate, n_dn = (size_t)dim * dstate;
+  struct Span {
+    const void* p;
+    size_t bytes;
+  };
+  const Span ins[] = {{x, n_bld * es},      {delta, n_bld * es}, {z, n_bld * es},
+                      {dy, n_bld * es},     {B, n_bln * es},     {C, n_bln * es},
+                      {A, n_dn * 4},        {D, (size_t)dim * 4}, {delta_bias, (size_t)dim * 4},
+                      {h0, n_bdn * 4},      {dh_last, n_bdn * 4}};
+  const Span outs[] = {{dx, n_bld * es},  {ddelta, n_bld * es}, {dz, n_bld * es},
+                       {dA, n_dn * 4},    {dB, n_bln * 4},      {dC, n_bln * 4},
+                       {dD, (size_t)dim * 4}, {ddelta_bias, (size_t)dim * 4}, {dh0, n_bdn * 4}};
+  for (size_t i = 0; i < sizeof outs / sizeof outs[0]; ++i) {
+    for (const Span& in : ins)
+      if (overlap(outs[i].p, outs[i].bytes, in.p, in.bytes))
+        return fail(SSM_ERR_INVALID_ARG, "ssm_scan_bwd: an output overlaps an input");
+    for (size_t j = i + 1; j < sizeof outs / sizeof outs[0]; ++j)
+      if (overlap(outs[i].p, outs[i].bytes, outs[j].p, outs[j].bytes))
+        return fail(SSM_ERR_INVALID_ARG, "ssm_scan_bwd: two outputs overlap");
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (seqlen == 0) {
+    // no steps: h_last = h0, so dh0 = dh_last; every other gradient is zero
+    cudaError_t e = cudaMemsetAsync(dA, 0, n_dn * 4, s);
+    if (e == cudaSuccess && dD) e = cudaMemsetAsync(dD, 0, (size_t)dim * 4, s);
+    if (e == cudaSuccess && ddelta_bias) e = cudaMemsetAsync(ddelta_bias, 0, (size_t)dim * 4, s);
+    if (e == cudaSuccess && dh0)
+      e = dh_last ? cudaMemcpyAsync(dh0, dh_last, n_bdn * 4, cudaMemcpyDeviceToDevice, s)
+                  : cudaMemsetAsync(dh0, 0, n_bdn * 4, s);
+    return cuda_status(e, "ssm_scan_bwd: empty sequence");
+  }
+  const BwdPlan pl = make_bwd_plan(d);
+  if (!workspace || workspace_bytes < pl.bytes || !aligned(workspace, 16))
+    return fail(SSM_ERR_WORKSPACE, "ssm_scan_bwd: workspace missing, too small or unaligned");
+
+  BwdParams p{};
+  p.batch = (int)batch;
+  p.seqlen = (int)seqlen;
+  p.dim = (int)dim;
+  p.nseg = pl.nseg;
+  p.seg_steps = pl.seg_steps;
+  p.dblocks = pl.dblocks;
+  p.ntiles = pl.ntiles;
+  p.softplus = softplus ? 1 : 0;
+  p.scal_pairs = (io_dtype == SSM_DTYPE_BF16 && dim % 2 == 0 && aligned(x, 4) &&
+                  aligned(delta, 4) && aligned(dy, 4) && (!z || aligned(z, 4)))
+                     ? 1
+                     : 0;
+  p.x = x; p.delta = delta; p.z = z; p.B = B; p.C = C;
+  p.A = A; p.D = D; p.bias = delta_bias; p.h0 = h0;
+  p.dy = dy; p.dh_last = dh_last;
+  p.dx = dx; p.ddelta = ddelta; p.dz = dz;
+  p.dA = dA; p.dB = dB; p.dC = dC; p.dD = dD; p.dbias = ddelta_bias; p.dh0 = dh0;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  p.ws_ck = reinterpret_cast<float*>(ws + pl.off_ck);
+  p.ws_qk = reinterpret_cast<float*>(ws + pl.off_qk);
+  p.ws_hloc = reinterpret_cast<float*>(ws + pl.off_hloc);
+  p.ws_mloc = reinterpret_cast<float*>(ws + pl.off_mloc);
+  p.ws_hin = reinterpret_cast<float*>(ws + pl.off_hin);
+  p.ws_muin = reinterpret_cast<float*>(ws + pl.off_muin);
+  p.ws_qseg = reinterpret_cast<float*>(ws + pl.off_qseg);
+  p.ws_dbc = reinterpret_cast<float*>(ws + pl.off_dbc);
+  p.ws_dA = reinterpret_cast<float*>(ws + pl.off_dA);
+  p.ws_dD = reinterpret_cast<float*>(ws + pl.off_dD);
+  p.ws_dbias = reinterpret_cast<float*>(ws + pl.off_dbias);
+  return cuda_status(launch_scan_bwd(p, (int)dstate, io_dtype == SSM_DTYPE_BF16, s),
+                     "backward launch");
 }
 
 }  // extern "C"

@@ -36,6 +36,8 @@ _lib = None
 
 # stream ids, one per tensor role
 STREAM_X, STREAM_DELTA, STREAM_Z, STREAM_B, STREAM_C, STREAM_H0, STREAM_BIAS = 1, 2, 3, 4, 5, 6, 7
+# upstream gradients of the backward pass
+STREAM_DY, STREAM_DH_LAST = 8, 9
 KIND_NORMAL, KIND_UNIFORM = 0, 1
 OUT_F64, OUT_F32, OUT_BF16 = 0, 1, 2
 
@@ -235,6 +237,18 @@ def workload_inputs(w: ScanWorkload, nthreads=None, batch=None, batch_offset=0):
     return make_scan_inputs(w.batch if batch is None else batch, w.seqlen, w.dim, w.dstate,
                             w.io, w.seed, gate=w.gate, skip=w.skip, with_h0=w.with_h0,
                             nthreads=nthreads, batch_offset=batch_offset)
+
+
+def make_grad_inputs(batch, seqlen, dim, dstate, io, seed, *, with_dh_last=True, nthreads=None,
+                     batch_offset=0):
+    """Upstream gradients for the backward pass: dy (batch, L, dim) in the io
+    type and dh_last (batch, dim, dstate) fp32, both N(0, 1)."""
+    o_ld, o_dn = batch_offset * seqlen * dim, batch_offset * dim * dstate
+    return {
+        "dy": fill((batch, seqlen, dim), seed, STREAM_DY, out=io, offset=o_ld, nthreads=nthreads),
+        "dh_last": (fill((batch, dim, dstate), seed, STREAM_DH_LAST, out="f32", offset=o_dn,
+                         nthreads=nthreads) if with_dh_last else None),
+    }
 
 
 def make_decode_inputs(batch, dim, dstate, io, seed, step, nthreads=None):

@@ -137,6 +137,39 @@ def test_state_update_rejects_bad_arguments(L):
     assert upd(batch=0) == 0
 
 
+@no_gpu_only
+def test_scan_bwd_rejects_bad_arguments(L):
+    K = 1 << 16  # spacing of the fake buffers: none of them overlap
+
+    def bwd(**kw):
+        a = dict(batch=2, seqlen=32, dim=64, dstate=16, io=1, x=FAKE, delta=FAKE + K,
+                 A=FAKE + 2 * K, B=FAKE + 3 * K, C=FAKE + 4 * K, D=None, z=FAKE + 5 * K,
+                 bias=None, sp=1, h0=None, dy=FAKE + 6 * K, dh_last=None, dx=FAKE + 7 * K,
+                 ddelta=FAKE + 8 * K, dA=FAKE + 9 * K, dB=FAKE + 10 * K, dC=FAKE + 11 * K,
+                 dD=None, dz=FAKE + 12 * K, dbias=None, dh0=None, ws=None, ws_bytes=0)
+        a.update(kw)
+        return L.ssm_scan_bwd(a["batch"], a["seqlen"], a["dim"], a["dstate"], a["io"], a["x"],
+                              a["delta"], a["A"], a["B"], a["C"], a["D"], a["z"], a["bias"],
+                              a["sp"], a["h0"], a["dy"], a["dh_last"], a["dx"], a["ddelta"],
+                              a["dA"], a["dB"], a["dC"], a["dD"], a["dz"], a["dbias"], a["dh0"],
+                              a["ws"], a["ws_bytes"], None)
+    assert bwd(dz=None) == -1                 # z given without dz
+    assert bwd(z=None) == -1                  # dz given without z
+    assert bwd(dy=None) == -1
+    assert bwd(dA=None) == -1
+    assert bwd(dx=FAKE + 1) == -1             # misaligned bf16
+    assert bwd(dB=FAKE + 10 * K + 2) == -1    # misaligned fp32
+    assert bwd(dx=FAKE + 6 * K + 64) == -1    # dx overlaps dy
+    assert bwd(dC=FAKE + 10 * K + 64) == -1   # dC overlaps dB
+    assert bwd(dstate=32) == -2               # the backward supports dstate <= 16
+    assert bwd(io=3) == -2
+    assert bwd() == -3                        # no workspace
+    need = L.ssm_scan_bwd_workspace_bytes(2, 32, 64, 16, 1)
+    assert need > 0 and L.ssm_scan_bwd_workspace_bytes(2, 32, 64, 32, 1) == 0
+    assert bwd(ws=FAKE * 64, ws_bytes=need - 1) == -3
+    assert bwd(batch=0) == 0 and bwd(dim=0) == 0
+
+
 def test_binding_has_no_cpu_path():
     from selective_state_space_39_b200 import ssm_scan_fwd
     x = torch.zeros(1, 4, 8)
