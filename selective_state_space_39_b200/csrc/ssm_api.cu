@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "../../include/ssm_scan.h"
+#include "ssm_bwd_internal.h"
 #include "ssm_internal.h"
 
 namespace ssm {

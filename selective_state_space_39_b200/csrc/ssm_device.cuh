@@ -174,23 +174,6 @@ __device__ __forceinline__ void griddep_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-// --------------------------------------------------------------- cp.async --
-// 4-byte asynchronous copy global -> shared; `src_bytes` < 4 copies that many
-// bytes and zero-fills the rest (0: nothing is read, `src` is not touched).
-__device__ __forceinline__ void cp_async4(void* dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)), "l"(src),
-               "r"(src_bytes)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-// Wait until at most `Pending` of this thread's committed groups are in flight.
-template <int Pending>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(Pending) : "memory");
-}
-
 // -------------------------------------------------------------------- TMA --
 // 3-D tiled bulk tensor load global -> shared, completing on `bar`.
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
