@@ -9,6 +9,7 @@ of an N-times larger global batch (weak scaling, no data-path collective);
 the time is the max over ranks.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --pass bwd [--workload NAME]  # the backward pass (gradients)
   python bench.py --impl reference ...   # the fp64 CPU oracle on host cores
 """
 from __future__ import annotations
@@ -44,6 +45,8 @@ def parse_args():
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
                     choices=sorted(gen.SCAN_WORKLOADS) + sorted(gen.DECODE_WORKLOADS))
+    ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd"],
+                    help="bwd: time ssm_scan_bwd (the gradients) on the same workload")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
@@ -268,7 +271,9 @@ def decode_bench(args):
     #     the flush's dirty lines; (2) flushed by reading 256 MB (clean
     #     lines): the call's own DRAM traffic; (3) back to back: the 33.5 MB
     #     state stays in L2, as across consecutive decode steps.
-    cold_ms = timed(lambda i: flush.fill_(i & 0xFF))
+    sampler = ClockSampler(0)
+    with sampler:
+        cold_ms = timed(lambda i: flush.fill_(i & 0xFF))
     read_ms = timed(lambda i: flush.view(torch.int64).sum())
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
@@ -322,7 +327,145 @@ def decode_bench(args):
         "cuda_graph": {"calls": w.steps, "ms_per_step": graph_ms,
                        "value": nbd / (graph_ms * 1e-3),
                        "algorithmic_gbs": round(algo / (graph_ms * 1e-3) / 1e9, 1)},
-        "gpu_launches": 2 * K,
+        "gpu_launches": 2 * K, "clocks": sampler.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+BWD_METRIC = "selective-scan backward elements/s (B·L·D, all gradients)"
+
+
+def bwd_algorithmic_bytes(w, batch):
+    """Bytes the backward must move at least: x, delta, (z), dy read and dx,
+    ddelta, (dz) written once per element; B, C read and dB, dC (fp32)
+    written per (b, t, n); per-channel parameters and their gradients."""
+    es = 2 if w.io == "bf16" else 4
+    bld, bln = batch * w.seqlen * w.dim, batch * w.seqlen * w.dstate
+    per_elem = ((4 if w.gate else 3) + (3 if w.gate else 2)) * es
+    state = batch * w.dim * w.dstate * 4 * (3 if w.with_h0 else 2)  # dh_last, dh0 (+ h0)
+    params = 2 * (w.dim * w.dstate * 4 + w.dim * 4 * (2 if w.skip else 1))
+    return bld * per_elem + bln * (2 * es + 2 * 4) + state + params
+
+
+def bwd_alu_ops_per_element(w):
+    """FP32 operations of the adjoint loop in its plain form, per state: the
+    recomputed update (2), the adjoint (2: C g + mu, then a lam), the four
+    products and sums of dB, dC, dA and dDelta's A term (2 each: 8): 12N."""
+    return 12 * w.dstate
+
+
+def cpu_oracle_bwd_rate(w, inp, grads, target_s, rng_seed=0):
+    """Backward oracle throughput (elements/s) on a bounded channel sample."""
+    import oracle
+    threads = gen.default_threads()
+    batch = inp["x"].shape[0]
+    rng = np.random.default_rng(rng_seed)
+    all_ch = [(b, d) for b in range(batch) for d in range(w.dim)]
+
+    def run(n):
+        idx = rng.choice(len(all_ch), size=min(n, len(all_ch)), replace=False)
+        chans = [all_ch[i] for i in idx]
+        t0 = time.perf_counter()
+        oracle.selective_scan_bwd(inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"],
+                                  grads["dy"], D=inp["D"], z=inp["z"],
+                                  delta_bias=inp["delta_bias"], h0=inp["h0"],
+                                  dh_last=grads["dh_last"], io=w.io, channels=chans,
+                                  nthreads=threads)
+        return len(chans), time.perf_counter() - t0
+
+    n, dt = run(threads)
+    per_chan = dt / max(n, 1) * threads
+    n2 = int(max(threads, min(len(all_ch), target_s / max(per_chan, 1e-9) * threads)))
+    n2 = max(threads, n2 // threads * threads)
+    n, dt = run(n2)
+    return (n * w.seqlen / dt, threads,
+            f"{n} of {len(all_ch)} channels x {w.seqlen} steps (gradients of the listed "
+            f"channels), {dt:.1f} s")
+
+
+def backward_bench(args):
+    """--pass bwd: ssm_scan_bwd on the workload (one GPU), timed like the
+    forward: L2 flushed (256 MB write) before every call, CUDA events."""
+    import torch
+
+    from selective_state_space_39_b200 import scan_bwd_workspace_bytes, ssm_scan_bwd
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        raise SystemExit("--pass bwd runs on one GPU")
+    w = gen.SCAN_WORKLOADS[args.workload]
+    device = torch.device("cuda", 0)
+    dtype = torch.bfloat16 if w.io == "bf16" else torch.float32
+    inp = gen.workload_inputs(w)
+    grads = gen.make_grad_inputs(w.batch, w.seqlen, w.dim, w.dstate, w.io, w.seed)
+
+    def to_dev(a):
+        if a is None:
+            return None
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+    d = {k: to_dev(v) for k, v in inp.items()}
+    g = {k: to_dev(v) for k, v in grads.items()}
+    ws = torch.empty(max(1, scan_bwd_workspace_bytes(w.batch, w.seqlen, w.dim, w.dstate, dtype)),
+                     dtype=torch.uint8, device=device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    def step():
+        return ssm_scan_bwd(d["x"], d["delta"], d["A"], d["B"], d["C"], g["dy"], D=d["D"],
+                            z=d["z"], delta_bias=d["delta_bias"], h0=d["h0"],
+                            dh_last=g["dh_last"], workspace=ws)
+
+    for _ in range(max(3, args.warmup)):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    sampler = ClockSampler(0)
+    with sampler:
+        for i in range(K):
+            flush.fill_(i & 0xFF)
+            ev[i][0].record()
+            step()
+            ev[i][1].record()
+        torch.cuda.synchronize()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    ms = statistics.mean(step_ms)
+    elements = w.batch * w.seqlen * w.dim
+    clocks = sampler.summary()
+    sm_mhz = clocks.get("sm_mhz") or B200_MAX_SM_MHZ
+    alu_peak = B200_SMS * FP32_LANES_PER_SM * sm_mhz * 1e6 / 1e9
+    alu = bwd_alu_ops_per_element(w) * elements / (ms * 1e-3) / 1e9
+    peak, peak_kind = measured_hbm_peak()
+    algo = bwd_algorithmic_bytes(w, w.batch)
+    gbs = algo / (ms * 1e-3) / 1e9
+    kernel = "ssm_scan_bwd: carry, compose, main, reduce (4 launches)"
+    cpu = None
+    if not args.no_cpu_baseline:
+        v, cores, sample = cpu_oracle_bwd_rate(w, inp, grads, args.cpu_seconds)
+        cpu = {"value": v, "unit": "elements/s", "cores": cores, "kind": "oracle",
+               "sample": sample}
+    line = {
+        "metric": BWD_METRIC, "value": elements / (ms * 1e-3), "unit": "elements/s",
+        "n_gpus": 1, "steps": K, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if w.io == "bf16" else "f32",
+        "data": "synthetic (seeded Philox4x32-10, Mamba-shaped recipe; dy, dh_last N(0,1))",
+        "config": {"workload": w.name, "pass": "backward", "batch": w.batch, "seqlen": w.seqlen,
+                   "dim": w.dim, "dstate": w.dstate, "io": w.io,
+                   "l2": "flushed (256 MB write) before every timed step"},
+        "roofline": {"bound": "alu", "achieved": round(alu, 1), "peak": round(alu_peak, 1),
+                     "unit": "Gop/s", "frac": round(alu / alu_peak, 4), "traffic": None,
+                     "kernel": kernel, "ops_per_element": bwd_alu_ops_per_element(w),
+                     "peak_kind": f"derived: {B200_SMS} SMs x {FP32_LANES_PER_SM} FP32 lanes x "
+                                  f"{sm_mhz:.0f} MHz sampled SM clock"},
+        "hbm_roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak,
+                         "unit": "GB/s", "frac": round(gbs / peak, 4), "traffic": None,
+                         "kernel": kernel, "algorithmic_bytes_per_launch": algo,
+                         "peak_kind": peak_kind},
+        "cpu_baseline": cpu, "gpu_launches": 4 * K, "clocks": clocks,
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -334,6 +477,8 @@ def main():
         return reference_arm(args)
     if args.workload in gen.DECODE_WORKLOADS:
         return decode_bench(args)
+    if args.which == "bwd":
+        return backward_bench(args)
 
     import torch
 
