@@ -13,8 +13,8 @@ The backward pass (``selective_scan_bwd``) is the reverse-mode derivative
 of the same loop, written out in ``ssm_oracle.c``. What it computes follows
 the page "Mamba 논문 리뷰: Selective State Space Models로 Transformer를
 넘어서" (youngju.dev): §2.2 discretised recurrence,
-§3.1 softplus step size, §3.3 simplified ``selective_scan``, §3.4 block gate
-and D skip. Every function here is pinned by ``tests/test_oracle_pins.py``
+§3.1 softplus step size, §3.3 simplified ``selective_scan``, §3.4 block gate,
+D skip and the causal depthwise conv1d + SiLU (``conv1d_silu``). Every function here is pinned by ``tests/test_oracle_pins.py``
 against closed forms, brute force and invariants.
 
 bf16 arrays are passed as numpy ``uint16`` holding the raw bf16 bits with
@@ -75,6 +75,14 @@ class Oracle:
                        _F32P, ctypes.c_void_p, ctypes.c_void_p, _F32P, ctypes.c_void_p,
                        _F32P, ctypes.c_int, _F32P, ctypes.c_void_p, _F32P, _I64P,
                        ctypes.c_int64] + [_F64P] * 9 + [ctypes.c_int]
+        cf = self.lib.oracle_conv1d_silu
+        cf.restype = ctypes.c_int
+        cf.argtypes = [ctypes.c_int64] * 4 + [ctypes.c_int, ctypes.c_void_p, _F32P, _F32P,
+                                              ctypes.c_int, _F64P]
+        cb = self.lib.oracle_conv1d_silu_bwd
+        cb.restype = ctypes.c_int
+        cb.argtypes = [ctypes.c_int64] * 4 + [ctypes.c_int, ctypes.c_void_p, _F32P, _F32P,
+                                              ctypes.c_int, ctypes.c_void_p, _F64P, _F64P, _F64P]
         g = self.lib.oracle_state_update
         g.restype = ctypes.c_int
         g.argtypes = [ctypes.c_int64] * 3 + [ctypes.c_int, _F64P, ctypes.c_void_p,
@@ -222,6 +230,51 @@ class Oracle:
             out["dh0"] = out["dh0"].reshape(batch, dim, N)
         return out
 
+    # -- the block's causal depthwise conv1d + SiLU ---------------------------
+    def conv1d_silu(self, x, w, bias=None, silu=True, io="f32"):
+        """out[b,t,d] = SiLU(bias[d] + sum_k w[d,k] x[b, t-(width-1)+k, d]) with
+        zero padding before t = 0; x (batch, L, dim) in the io type, w (dim,
+        width) and bias (dim,) fp32. Returns out in fp64."""
+        x = np.asarray(x)
+        batch, L, dim = x.shape
+        width = np.asarray(w).shape[1]
+        x = self._io_array(x, io, (batch, L, dim), "x")
+        w = self._f32_array(w, (dim, width), "w", optional=False)
+        bias = self._f32_array(bias, (dim,), "bias")
+        out = np.empty((batch, L, dim), dtype=np.float64)
+        rc = self.lib.oracle_conv1d_silu(batch, L, dim, width, 1 if io == "bf16" else 0,
+                                         self._ptr(x), self._ptr(w, ctypes.c_float),
+                                         self._ptr(bias, ctypes.c_float), 1 if silu else 0,
+                                         self._ptr(out, ctypes.c_double))
+        if rc != 0:
+            raise ValueError("oracle_conv1d_silu rejected its arguments")
+        return out
+
+    def conv1d_silu_bwd(self, x, w, dout, bias=None, silu=True, io="f32"):
+        """Gradients of sum(dout * out) for conv1d_silu: returns (dx (batch, L,
+        dim), dw (dim, width), dbias (dim,)) in fp64."""
+        x = np.asarray(x)
+        batch, L, dim = x.shape
+        width = np.asarray(w).shape[1]
+        x = self._io_array(x, io, (batch, L, dim), "x")
+        dout = self._io_array(dout, io, (batch, L, dim), "dout")
+        w = self._f32_array(w, (dim, width), "w", optional=False)
+        bias = self._f32_array(bias, (dim,), "bias")
+        dx = np.empty((batch, L, dim), dtype=np.float64)
+        dw = np.empty((dim, width), dtype=np.float64)
+        db = np.empty((dim,), dtype=np.float64)
+        rc = self.lib.oracle_conv1d_silu_bwd(batch, L, dim, width, 1 if io == "bf16" else 0,
+                                             self._ptr(x), self._ptr(w, ctypes.c_float),
+                                             self._ptr(bias, ctypes.c_float), 1 if silu else 0,
+                                             self._ptr(dout), self._ptr(dx, ctypes.c_double),
+                                             self._ptr(dw, ctypes.c_double),
+                                             self._ptr(db, ctypes.c_double))
+        if rc == -2:
+            raise MemoryError("oracle_conv1d_silu_bwd ran out of memory")
+        if rc != 0:
+            raise ValueError("oracle_conv1d_silu_bwd rejected its arguments")
+        return dx, dw, db
+
     # -- decode ------------------------------------------------------------
     def state_update(self, state, x, delta, A, B, C, D=None, z=None, delta_bias=None,
                      softplus=True, io="f32"):
@@ -274,3 +327,11 @@ def state_update(*args, **kwargs):
 
 def selective_scan_bwd(*args, **kwargs):
     return get().selective_scan_bwd(*args, **kwargs)
+
+
+def conv1d_silu(*args, **kwargs):
+    return get().conv1d_silu(*args, **kwargs)
+
+
+def conv1d_silu_bwd(*args, **kwargs):
+    return get().conv1d_silu_bwd(*args, **kwargs)

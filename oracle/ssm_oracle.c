@@ -423,3 +423,88 @@ int oracle_selective_scan_bwd(int64_t batch, int64_t seqlen, int64_t dim, int64_
   }
   return rc;
 }
+
+/* ------------------------------------------------------------------------
+ * The block's causal depthwise convolution and SiLU (page "Mamba 논문 리뷰",
+ * §3.4 Mamba Block: conv1d = nn.Conv1d(d_inner, d_inner, d_conv,
+ * padding=d_conv-1, groups=d_inner), its output cut to the first L steps,
+ * then SiLU). Per batch row b, channel d and step t, with taps k < width:
+ *
+ *   u[b,t,d]   = bias[d] + sum_k w[d,k] * x[b, t - (width-1) + k, d]
+ *                (x at negative steps is the zero padding)
+ *   out[b,t,d] = SiLU(u[b,t,d])  (or u without SiLU)
+ *
+ * The backward, for the loss sum dout * out, is
+ *   du[t]    = dout[t] * SiLU'(u[t])  (or dout[t])
+ *   dx[s]    = sum_k w[d,k] * du[s + (width-1) - k]   (terms with t >= L are 0)
+ *   dw[d,k]  = sum_(b,t) du[b,t,d] * x[b, t - (width-1) + k, d]
+ *   dbias[d] = sum_(b,t) du[b,t,d]
+ * ------------------------------------------------------------------------ */
+
+static double conv_u(const void* x, const float* w, const float* bias, int is_bf16, int64_t b,
+                     int64_t t, int64_t d, int64_t L, int64_t Dm, int64_t width) {
+  double u = bias ? (double)bias[d] : 0.0;
+  for (int64_t k = 0; k < width; ++k) {
+    const int64_t s = t - (width - 1) + k;
+    if (s < 0) continue;
+    u += (double)w[d * width + k] * widen(x, (b * L + s) * Dm + d, is_bf16);
+  }
+  return u;
+}
+
+/* oracle_conv1d_silu -- out (batch, seqlen, dim) fp64. Returns 0 or -1. */
+int oracle_conv1d_silu(int64_t batch, int64_t seqlen, int64_t dim, int64_t width, int is_bf16,
+                       const void* x, const float* w, const float* bias, int silu_on,
+                       double* out) {
+  if (batch < 0 || seqlen < 0 || dim < 0 || width < 1 || !x || !w || !out) return -1;
+  for (int64_t b = 0; b < batch; ++b)
+    for (int64_t t = 0; t < seqlen; ++t)
+      for (int64_t d = 0; d < dim; ++d) {
+        const double u = conv_u(x, w, bias, is_bf16, b, t, d, seqlen, dim, width);
+        out[(b * seqlen + t) * dim + d] = silu_on ? silu(u) : u;
+      }
+  return 0;
+}
+
+/* oracle_conv1d_silu_bwd -- dx (batch, seqlen, dim), dw (dim, width), dbias
+ * (dim), fp64, overwritten. Returns 0, -1 on bad arguments, -2 without memory. */
+int oracle_conv1d_silu_bwd(int64_t batch, int64_t seqlen, int64_t dim, int64_t width,
+                           int is_bf16, const void* x, const float* w, const float* bias,
+                           int silu_on, const void* dout, double* dx, double* dw,
+                           double* dbias) {
+  if (batch < 0 || seqlen < 0 || dim < 0 || width < 1 || !x || !w || !dout || !dx || !dw ||
+      !dbias)
+    return -1;
+  double* du = (double*)malloc((size_t)(seqlen > 0 ? seqlen : 1) * sizeof(double));
+  if (!du) return -2;
+  memset(dw, 0, (size_t)dim * width * sizeof(double));
+  memset(dbias, 0, (size_t)dim * sizeof(double));
+  for (int64_t b = 0; b < batch; ++b)
+    for (int64_t d = 0; d < dim; ++d) {
+      for (int64_t t = 0; t < seqlen; ++t) {
+        const double g = widen(dout, (b * seqlen + t) * dim + d, is_bf16);
+        if (silu_on) {
+          const double u = conv_u(x, w, bias, is_bf16, b, t, d, seqlen, dim, width);
+          const double sg = sigmoid(u);
+          du[t] = g * sg * (1.0 + u * (1.0 - sg));
+        } else {
+          du[t] = g;
+        }
+        dbias[d] += du[t];
+        for (int64_t k = 0; k < width; ++k) {
+          const int64_t s = t - (width - 1) + k;
+          if (s >= 0) dw[d * width + k] += du[t] * widen(x, (b * seqlen + s) * dim + d, is_bf16);
+        }
+      }
+      for (int64_t s = 0; s < seqlen; ++s) {
+        double acc = 0.0;
+        for (int64_t k = 0; k < width; ++k) {
+          const int64_t t = s + (width - 1) - k;
+          if (t < seqlen) acc += (double)w[d * width + k] * du[t];
+        }
+        dx[(b * seqlen + s) * dim + d] = acc;
+      }
+    }
+  free(du);
+  return 0;
+}

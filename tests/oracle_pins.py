@@ -418,6 +418,85 @@ def pin_bwd_autograd(o):
         _close(g[gname], t[name].grad.numpy(), 1e-10, 1e-12, what=f"autograd {gname}")
 
 
+# --------------------------------------------------------------------------
+# pins of the block's causal depthwise conv1d + SiLU (§3.4 Mamba Block)
+def _conv_case(seed, batch=2, L=9, dim=3, width=4):
+    r = _rng(seed)
+    return (_f32(r.standard_normal((batch, L, dim))), _f32(0.5 * r.standard_normal((dim, width))),
+            _f32(r.uniform(-0.5, 0.5, dim)))
+
+
+def pin_conv_matches_torch_conv1d(o):
+    """The page's own formulation: nn.Conv1d(groups=dim, padding=width-1) (torch's
+    conv1d, fp64 CPU) cut to the first L outputs, then SiLU."""
+    import torch
+    for width in (2, 3, 4):
+        x, w, b = _conv_case(201 + width, width=width)
+        xt = torch.tensor(x.astype(np.float64)).transpose(1, 2)
+        u = torch.nn.functional.conv1d(xt, torch.tensor(w.astype(np.float64))[:, None, :],
+                                       torch.tensor(b.astype(np.float64)), padding=width - 1,
+                                       groups=x.shape[2])[:, :, :x.shape[1]].transpose(1, 2)
+        _close(o.conv1d_silu(x, w, b, silu=False), u.numpy(), 1e-13, 1e-14, what="conv, no SiLU")
+        _close(o.conv1d_silu(x, w, b, silu=True), torch.nn.functional.silu(u).numpy(), 1e-13,
+               1e-14, what="conv + SiLU")
+
+
+def pin_conv_by_hand(o):
+    """One channel, width 4, x = 1..5, w = (0.5, -1, 2, 0.25), bias 0.1:
+    u_t = 0.1 + sum_k w_k x_(t-3+k) written out term by term."""
+    x = _f32([1, 2, 3, 4, 5]).reshape(1, 5, 1)
+    w = _f32([[0.5, -1.0, 2.0, 0.25]])
+    b = _f32([0.1])
+    bias = float(np.float32(0.1))
+    want = [bias + 0.25 * 1,
+            bias + 2.0 * 1 + 0.25 * 2,
+            bias - 1.0 * 1 + 2.0 * 2 + 0.25 * 3,
+            bias + 0.5 * 1 - 1.0 * 2 + 2.0 * 3 + 0.25 * 4,
+            bias + 0.5 * 2 - 1.0 * 3 + 2.0 * 4 + 0.25 * 5]
+    _close(o.conv1d_silu(x, w, b, silu=False)[0, :, 0], want, 1e-15, 0, what="conv by hand")
+    _close(o.conv1d_silu(x, w, b, silu=True)[0, :, 0], [v / (1 + math.exp(-v)) for v in want],
+           1e-15, 0, what="conv + SiLU by hand")
+
+
+def pin_conv_is_causal(o):
+    """Changing x at step s changes the output at steps s .. s+width-1 only."""
+    x, w, b = _conv_case(207, L=12)
+    base = o.conv1d_silu(x, w, b)
+    s = 5
+    x2 = x.copy()
+    x2[:, s, :] += 1.0
+    diff = np.abs(o.conv1d_silu(x2, w, b) - base).max(axis=(0, 2))
+    assert np.all(diff[:s] == 0) and np.all(diff[s + 4:] == 0), "conv is not causal / too wide"
+    assert np.all(diff[s:s + 4] > 0), "conv ignores a tap"
+
+
+def pin_conv_bwd_finite_differences(o):
+    """dx, dw, dbias of the conv backward equal central differences of the
+    (separately pinned) forward, with and without SiLU."""
+    for silu in (True, False):
+        x, w, b = _conv_case(209, batch=2, L=7, dim=2)
+        dout = _f32(_rng(210).standard_normal(x.shape))
+        dx, dw, db = o.conv1d_silu_bwd(x, w, dout, b, silu=silu)
+        args = {"x": x, "w": w, "b": b}
+        for name, g in (("x", dx), ("w", dw), ("b", db)):
+            base = args[name]
+            fd = np.zeros(base.shape)
+            for i in np.ndindex(base.shape):
+                v = float(base[i])
+                h = 2.0 ** -11 * max(2.0 ** -4, abs(v))
+                vals = []
+                for vv in (np.float32(v + h), np.float32(v - h)):
+                    a = dict(args)
+                    arr = base.copy()
+                    arr[i] = vv
+                    a[name] = arr
+                    vals.append(float(np.sum(dout.astype(np.float64) *
+                                             o.conv1d_silu(a["x"], a["w"], a["b"], silu=silu))))
+                fd[i] = (vals[0] - vals[1]) / (float(np.float32(v + h)) - float(np.float32(v - h)))
+            scale = max(1.0, float(np.max(np.abs(fd))))
+            _close(g, fd, 0.0, 2e-6 * scale, what=f"conv d{name} vs central differences")
+
+
 ALL_PINS = [
     pin_softplus_library,
     pin_silu_library,
@@ -435,4 +514,8 @@ ALL_PINS = [
     pin_bwd_finite_differences,
     pin_bwd_finite_differences_plain,
     pin_bwd_autograd,
+    pin_conv_matches_torch_conv1d,
+    pin_conv_by_hand,
+    pin_conv_is_causal,
+    pin_conv_bwd_finite_differences,
 ]

@@ -89,6 +89,18 @@ MUTANTS = {
     "bwd_dx_drops_skip": ("j->dx[k * L + t] = Dd * g + dt * sum_lb;",
                           "j->dx[k * L + t] = dt * sum_lb;"),
     "bwd_dh0_before_decay": ("      lam[n] *= a;\n", "      if (t > 0) lam[n] *= a;\n"),
+    # causal conv1d + SiLU
+    "conv_taps_flipped": ("u += (double)w[d * width + k] * widen(x, (b * L + s) * Dm + d, is_bf16);",
+                          "u += (double)w[d * width + (width - 1 - k)] * widen(x, (b * L + s) * Dm + d, is_bf16);"),
+    "conv_off_by_one": ("    const int64_t s = t - (width - 1) + k;\n    if (s < 0) continue;",
+                        "    const int64_t s = t - width + k;\n    if (s < 0) continue;"),
+    "conv_bias_dropped": ("  double u = bias ? (double)bias[d] : 0.0;", "  double u = 0.0;"),
+    "conv_bwd_silu_derivative": ("du[t] = g * sg * (1.0 + u * (1.0 - sg));", "du[t] = g * sg;"),
+    "conv_bwd_dx_not_transposed": ("          const int64_t t = s + (width - 1) - k;",
+                                   "          const int64_t t = s - (width - 1) + k;"),
+    "conv_bwd_dw_wrong_step": ("if (s >= 0) dw[d * width + k] += du[t] * widen(x, (b * seqlen + s) * dim + d, is_bf16);",
+                               "if (s >= 0) dw[d * width + k] += du[t] * widen(x, (b * seqlen + t) * dim + d, is_bf16);"),
+    "conv_bwd_dbias_from_dout": ("        dbias[d] += du[t];", "        dbias[d] += g;"),
 }
 
 
