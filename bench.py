@@ -10,6 +10,7 @@ the time is the max over ranks.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
   python bench.py --pass bwd [--workload NAME]  # the backward pass (gradients)
+  python bench.py --op conv [--workload NAME]   # the block's causal conv1d + SiLU
   python bench.py --impl reference ...   # the fp64 CPU oracle on host cores
 """
 from __future__ import annotations
@@ -47,6 +48,9 @@ def parse_args():
                     choices=sorted(gen.SCAN_WORKLOADS) + sorted(gen.DECODE_WORKLOADS))
     ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd"],
                     help="bwd: time ssm_scan_bwd (the gradients) on the same workload")
+    ap.add_argument("--op", default="scan", choices=["scan", "conv"],
+                    help="conv: time the block's causal conv1d + SiLU (forward and backward) "
+                         "on the workload's (batch, seqlen, dim)")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
@@ -471,12 +475,100 @@ def backward_bench(args):
     return 0
 
 
+CONV_METRIC = "causal conv1d + SiLU elements/s (B·L·D) and achieved HBM GB/s"
+
+
+def conv_bench(args):
+    """--op conv: ssm_conv1d_silu_fwd and _bwd (width 4) on the workload's
+    (batch, seqlen, dim), one GPU, L2 flushed (256 MB write) before every call.
+    The line's value is the forward; the backward is reported beside it."""
+    import torch
+
+    from selective_state_space_39_b200 import (conv1d_silu_bwd_workspace_bytes,
+                                               ssm_conv1d_silu_bwd, ssm_conv1d_silu_fwd)
+    w = gen.SCAN_WORKLOADS[args.workload]
+    device = torch.device("cuda", 0)
+    dtype = torch.bfloat16 if w.io == "bf16" else torch.float32
+    width = 4
+    c = gen.make_conv_inputs(w.batch, w.seqlen, w.dim, width, w.io, w.seed)
+
+    def to_dev(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+    d = {k: to_dev(v) for k, v in c.items()}
+    out = torch.empty(d["x"].shape, dtype=dtype, device=device)
+    ws = torch.empty(max(1, conv1d_silu_bwd_workspace_bytes(w.batch, w.seqlen, w.dim, width,
+                                                            dtype)), dtype=torch.uint8,
+                     device=device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    def fwd():
+        ssm_conv1d_silu_fwd(d["x"], d["w"], d["bias"], out=out)
+
+    def bwd():
+        ssm_conv1d_silu_bwd(d["x"], d["w"], d["dout"], d["bias"], workspace=ws)
+
+    def timed(f, K):
+        for _ in range(max(3, args.warmup)):
+            flush.fill_(1)
+            f()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(K)]
+        for i in range(K):
+            flush.fill_(i & 0xFF)
+            ev[i][0].record()
+            f()
+            ev[i][1].record()
+        torch.cuda.synchronize()
+        return statistics.mean(a.elapsed_time(b) for a, b in ev)
+
+    K = args.steps
+    sampler = ClockSampler(0)
+    with sampler:
+        f_ms = timed(fwd, K)
+        b_ms = timed(bwd, K)
+    es = 2 if w.io == "bf16" else 4
+    n = w.batch * w.seqlen * w.dim
+    params = w.dim * (width + 1) * 4
+    f_bytes = 2 * n * es + params                # x read, out written
+    b_bytes = 3 * n * es + 3 * params            # x, dout read, dx written; w, dw, dbias
+    peak, peak_kind = measured_hbm_peak()
+    f_gbs = f_bytes / (f_ms * 1e-3) / 1e9
+    b_gbs = b_bytes / (b_ms * 1e-3) / 1e9
+    line = {
+        "metric": CONV_METRIC, "value": n / (f_ms * 1e-3), "unit": "elements/s", "n_gpus": 1,
+        "steps": K, "warmup": args.warmup, "ms_per_step": f_ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.io == "bf16" else "f32",
+        "data": "synthetic (seeded Philox4x32-10; x, dout N(0,1); taps, bias U[-0.5, 0.5])",
+        "config": {"workload": w.name, "op": "causal conv1d + SiLU, width 4", "batch": w.batch,
+                   "seqlen": w.seqlen, "dim": w.dim, "io": w.io,
+                   "l2": "flushed (256 MB write) before every timed call"},
+        "roofline": {"bound": "hbm", "achieved": round(f_gbs, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(f_gbs / peak, 4), "traffic": None,
+                     "kernel": "conv_fwd_kernel (1 launch)",
+                     "algorithmic_bytes_per_launch": f_bytes, "peak_kind": peak_kind},
+        "backward": {"ms_per_step": b_ms, "value": n / (b_ms * 1e-3), "unit": "elements/s",
+                     "roofline": {"bound": "hbm", "achieved": round(b_gbs, 1), "peak": peak,
+                                  "unit": "GB/s", "frac": round(b_gbs / peak, 4),
+                                  "kernel": "conv_bwd_kernel + conv_reduce_kernel (2 launches)",
+                                  "algorithmic_bytes_per_call": b_bytes}},
+        "gpu_launches": 3 * K, "clocks": sampler.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return reference_arm(args)
     if args.workload in gen.DECODE_WORKLOADS:
         return decode_bench(args)
+    if args.op == "conv":
+        return conv_bench(args)
     if args.which == "bwd":
         return backward_bench(args)
 

@@ -219,6 +219,45 @@ int ssm_scan_bwd(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate, int
                  void* stream);
 
 /*
+ * ssm_conv1d_silu_fwd -- the Mamba block's causal depthwise convolution and
+ * SiLU (§3.4 Mamba Block: nn.Conv1d(d_inner, d_inner, d_conv,
+ * padding=d_conv-1, groups=d_inner), output cut to the first L steps, then
+ * SiLU), the step that produces the scan's x:
+ *
+ *   out[b,t,d] = SiLU(bias[d] + sum_{k<width} w[d,k] * x[b, t-(width-1)+k, d])
+ *
+ * with x = 0 before t = 0 (silu = 0: the convolution alone).
+ *   x, out : (batch, seqlen, dim) io_dtype; out must not overlap x
+ *   w      : (dim, width) fp32, width 2, 3 or 4 (the block uses 4)
+ *   bias   : (dim) fp32, nullable (zero)
+ * dim a multiple of 4 (bf16) or 2 (fp32) with 8-byte aligned x and out takes
+ * 8-byte vector accesses; other shapes one element per thread.
+ * Returns SSM_OK or SSM_ERR_*.
+ */
+int ssm_conv1d_silu_fwd(int64_t batch, int64_t seqlen, int64_t dim, int64_t width, int io_dtype,
+                        const void* x, const float* w, const float* bias, int silu, void* out,
+                        void* stream);
+
+/* ssm_conv1d_silu_bwd_workspace_bytes -- workspace of ssm_conv1d_silu_bwd:
+ * per-(batch row, 128-step chunk) partial sums of dw and dbias. */
+size_t ssm_conv1d_silu_bwd_workspace_bytes(int64_t batch, int64_t seqlen, int64_t dim,
+                                           int64_t width, int io_dtype);
+
+/*
+ * ssm_conv1d_silu_bwd -- gradients of sum(dout * out) for
+ * ssm_conv1d_silu_fwd with the same x, w, bias, silu:
+ *   dx    : (batch, seqlen, dim) io_dtype (overwritten)
+ *   dw    : (dim, width) fp32, nullable; dbias : (dim) fp32, nullable
+ * dout is (batch, seqlen, dim) io_dtype. No output may overlap an input.
+ * Sums over batch rows and steps run in a fixed order. Returns SSM_OK or
+ * SSM_ERR_*.
+ */
+int ssm_conv1d_silu_bwd(int64_t batch, int64_t seqlen, int64_t dim, int64_t width, int io_dtype,
+                        const void* x, const float* w, const float* bias, int silu,
+                        const void* dout, void* dx, float* dw, float* dbias, void* workspace,
+                        size_t workspace_bytes, void* stream);
+
+/*
  * ssm_scan_status -- synchronise `stream`, then report whether every CTA of
  * the last ssm_scan_fwd call that used this workspace (with these sizes)
  * finished normally: SSM_OK, or SSM_ERR_TIMEOUT if a bounded wait inside a

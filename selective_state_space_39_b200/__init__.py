@@ -9,10 +9,13 @@ from ._binding import (  # noqa: F401
     SSM_DTYPE_F32,
     ScanPlan,
     SsmError,
+    conv1d_silu_bwd_workspace_bytes,
     lib,
     scan_bwd_workspace_bytes,
     scan_plan,
     scan_workspace_bytes,
+    ssm_conv1d_silu_bwd,
+    ssm_conv1d_silu_fwd,
     ssm_scan_bwd,
     ssm_scan_fwd,
     ssm_scan_fwd_noalloc,
@@ -22,4 +25,5 @@ from ._binding import (  # noqa: F401
 
 __all__ = ["ssm_scan_fwd", "ssm_scan_fwd_noalloc", "ssm_scan_bwd", "ssm_state_update",
            "ssm_scan_status", "scan_plan", "scan_workspace_bytes", "scan_bwd_workspace_bytes",
+           "ssm_conv1d_silu_fwd", "ssm_conv1d_silu_bwd", "conv1d_silu_bwd_workspace_bytes",
            "SsmError", "SSM_DTYPE_F32", "SSM_DTYPE_BF16", "lib"]

@@ -80,6 +80,15 @@ def lib() -> ctypes.CDLL:
         L.ssm_scan_bwd.restype = ctypes.c_int
         L.ssm_scan_bwd.argtypes = [_I64, _I64, _I64, _I64, ctypes.c_int] + [_VP] * 8 + \
             [ctypes.c_int] + [_VP] * 13 + [ctypes.c_size_t, _VP]
+        L.ssm_conv1d_silu_fwd.restype = ctypes.c_int
+        L.ssm_conv1d_silu_fwd.argtypes = [_I64, _I64, _I64, _I64, ctypes.c_int, _VP, _VP, _VP,
+                                          ctypes.c_int, _VP, _VP]
+        L.ssm_conv1d_silu_bwd_workspace_bytes.restype = ctypes.c_size_t
+        L.ssm_conv1d_silu_bwd_workspace_bytes.argtypes = [_I64, _I64, _I64, _I64, ctypes.c_int]
+        L.ssm_conv1d_silu_bwd.restype = ctypes.c_int
+        L.ssm_conv1d_silu_bwd.argtypes = [_I64, _I64, _I64, _I64, ctypes.c_int, _VP, _VP, _VP,
+                                          ctypes.c_int, _VP, _VP, _VP, _VP, _VP, ctypes.c_size_t,
+                                          _VP]
         L.ssm_state_update.restype = ctypes.c_int
         L.ssm_state_update.argtypes = [_I64, _I64, _I64, ctypes.c_int, _VP, _VP, _VP, _VP, _VP,
                                        _VP, _VP, _VP, _VP, ctypes.c_int, _VP, _VP]
@@ -229,6 +238,65 @@ def ssm_scan_bwd(x, delta, A, B, C, dy, D=None, z=None, delta_bias=None, softplu
                                 _stream_ptr(stream, dev))
     if rc != 0:
         raise SsmError(rc, "ssm_scan_bwd", with_detail=True)
+    return g
+
+
+def ssm_conv1d_silu_fwd(x, w, bias=None, silu=True, out=None, stream=None):
+    """The Mamba block's causal depthwise conv1d (+ SiLU) through
+    ssm_conv1d_silu_fwd of libssmscan.so. x: (batch, L, dim) float32 or
+    bfloat16; w: (dim, width) float32; bias: (dim,) float32. Returns out
+    (batch, L, dim) in x's dtype."""
+    if x.dim() != 3 or w.dim() != 2:
+        raise ValueError("x must be (batch, seqlen, dim) and w (dim, width)")
+    batch, L, dim = x.shape
+    width = w.shape[1]
+    dev = x.device
+    px = _ptr(x, "x", x.dtype, (batch, L, dim))
+    pw = _ptr(w, "w", torch.float32, (dim, width), dev)
+    pb = _ptr(bias, "bias", torch.float32, (dim,), dev)
+    if out is None:
+        out = torch.empty((batch, L, dim), dtype=x.dtype, device=dev)
+    po = _ptr(out, "out", x.dtype, (batch, L, dim), dev)
+    with torch.cuda.device(dev):
+        rc = lib().ssm_conv1d_silu_fwd(batch, L, dim, width, _io_code(x.dtype), px, pw, pb,
+                                       1 if silu else 0, po, _stream_ptr(stream, dev))
+    if rc != 0:
+        raise SsmError(rc, "ssm_conv1d_silu_fwd", with_detail=True)
+    return out
+
+
+def conv1d_silu_bwd_workspace_bytes(batch, seqlen, dim, width, dtype=torch.bfloat16) -> int:
+    return int(lib().ssm_conv1d_silu_bwd_workspace_bytes(batch, seqlen, dim, width,
+                                                         _io_code(dtype)))
+
+
+def ssm_conv1d_silu_bwd(x, w, dout, bias=None, silu=True, workspace=None, stream=None):
+    """Gradients of sum(dout * out) for ssm_conv1d_silu_fwd: returns a dict
+    dx (batch, L, dim) in x's dtype, dw (dim, width) and dbias (dim,) float32."""
+    if x.dim() != 3 or w.dim() != 2:
+        raise ValueError("x must be (batch, seqlen, dim) and w (dim, width)")
+    batch, L, dim = x.shape
+    width = w.shape[1]
+    dev = x.device
+    px = _ptr(x, "x", x.dtype, (batch, L, dim))
+    pw = _ptr(w, "w", torch.float32, (dim, width), dev)
+    pb = _ptr(bias, "bias", torch.float32, (dim,), dev)
+    pg = _ptr(dout, "dout", x.dtype, (batch, L, dim), dev)
+    g = {"dx": torch.empty((batch, L, dim), dtype=x.dtype, device=dev),
+         "dw": torch.empty((dim, width), dtype=torch.float32, device=dev),
+         "dbias": torch.empty((dim,), dtype=torch.float32, device=dev)}
+    with torch.cuda.device(dev):
+        need = conv1d_silu_bwd_workspace_bytes(batch, L, dim, width, x.dtype)
+        if workspace is None:
+            workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+        pws = _ptr(workspace, "workspace", None, None, dev)
+        rc = lib().ssm_conv1d_silu_bwd(batch, L, dim, width, _io_code(x.dtype), px, pw, pb,
+                                       1 if silu else 0, pg, g["dx"].data_ptr(),
+                                       g["dw"].data_ptr(), g["dbias"].data_ptr(), pws,
+                                       workspace.numel() * workspace.element_size(),
+                                       _stream_ptr(stream, dev))
+    if rc != 0:
+        raise SsmError(rc, "ssm_conv1d_silu_bwd", with_detail=True)
     return g
 
 

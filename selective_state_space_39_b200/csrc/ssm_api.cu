@@ -6,10 +6,12 @@
 #include <string.h>
 
 #include <algorithm>
+#include <initializer_list>
 #include <mutex>
 
 #include "../../include/ssm_scan.h"
 #include "ssm_bwd_internal.h"
+#include "ssm_conv_internal.h"
 #include "ssm_internal.h"
 
 namespace ssm {
@@ -500,6 +502,119 @@ int ssm_scan_bwd(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate, int
   p.ws_dbias = reinterpret_cast<float*>(ws + pl.off_dbias);
   return cuda_status(launch_scan_bwd(p, (int)dstate, io_dtype == SSM_DTYPE_BF16, s),
                      "backward launch");
+}
+
+// ---- causal depthwise conv1d + SiLU --------------------------------------
+
+static int conv_check(int64_t batch, int64_t seqlen, int64_t dim, int64_t width, int io_dtype) {
+  if (io_dtype != SSM_DTYPE_F32 && io_dtype != SSM_DTYPE_BF16) return SSM_ERR_UNSUPPORTED;
+  if (batch < 0 || seqlen < 0 || dim < 0 || width < 1) return SSM_ERR_INVALID_ARG;
+  if (!conv_width_supported((int)std::min<int64_t>(width, 1 << 20))) return SSM_ERR_UNSUPPORTED;
+  if (batch > 65535 || dim > (1 << 24) || seqlen > (1 << 30)) return SSM_ERR_UNSUPPORTED;
+  return SSM_OK;
+}
+
+static bool conv_vec(int64_t dim, int io_dtype, std::initializer_list<const void*> ptrs) {
+  const int64_t vec = io_dtype == SSM_DTYPE_BF16 ? 4 : 2;
+  if (dim % vec != 0) return false;
+  for (const void* p : ptrs)
+    if (p && !aligned(p, 8)) return false;
+  return true;
+}
+
+// Steps per CTA along the sequence (SSM_CONV_CHUNK overrides, 8 .. 4096).
+static int conv_chunk(bool backward) {
+  return (int)std::max(8L, std::min(4096L, env_long("SSM_CONV_CHUNK",
+                                                    backward ? kConvChunkBwd : kConvChunkFwd)));
+}
+
+static ConvParams conv_params(int64_t batch, int64_t seqlen, int64_t dim, int64_t width,
+                              int silu, bool backward) {
+  ConvParams p{};
+  p.batch = (int)batch;
+  p.seqlen = (int)seqlen;
+  p.dim = (int)dim;
+  p.width = (int)width;
+  p.chunk = conv_chunk(backward);
+  p.silu = silu ? 1 : 0;
+  p.w_vec = 0;
+  return p;
+}
+
+int ssm_conv1d_silu_fwd(int64_t batch, int64_t seqlen, int64_t dim, int64_t width, int io_dtype,
+                        const void* x, const float* w, const float* bias, int silu, void* out,
+                        void* stream) {
+  int st = conv_check(batch, seqlen, dim, width, io_dtype);
+  if (st != SSM_OK) return st;
+  if (batch == 0 || dim == 0 || seqlen == 0) return SSM_OK;
+  if (!x || !w || !out) return SSM_ERR_INVALID_ARG;
+  const size_t es = io_bytes(io_dtype), n = (size_t)batch * seqlen * dim;
+  if (!aligned(x, es) || !aligned(out, es) || !aligned(w, 4) || (bias && !aligned(bias, 4)))
+    return SSM_ERR_INVALID_ARG;
+  if (overlap(out, n * es, x, n * es) || overlap(out, n * es, w, (size_t)dim * width * 4) ||
+      overlap(out, n * es, bias, (size_t)dim * 4))
+    return fail(SSM_ERR_INVALID_ARG, "ssm_conv1d_silu_fwd: out overlaps an input");
+  ConvParams p = conv_params(batch, seqlen, dim, width, silu, false);
+  p.x = x; p.w = w; p.bias = bias; p.out = out;
+  p.w_vec = aligned(w, 16) ? 1 : 0;
+  return cuda_status(launch_conv(p, io_dtype == SSM_DTYPE_BF16, conv_vec(dim, io_dtype, {x, out}),
+                                 false, static_cast<cudaStream_t>(stream)),
+                     "conv1d forward launch");
+}
+
+size_t ssm_conv1d_silu_bwd_workspace_bytes(int64_t batch, int64_t seqlen, int64_t dim,
+                                           int64_t width, int io_dtype) {
+  if (conv_check(batch, seqlen, dim, width, io_dtype) != SSM_OK) return 0;
+  const int64_t ch = conv_chunk(true);
+  const size_t chunks = (size_t)((seqlen + ch - 1) / ch);
+  return align_up(sizeof(float) * (size_t)batch * chunks * dim * width, 256) +
+         sizeof(float) * (size_t)batch * chunks * dim;
+}
+
+int ssm_conv1d_silu_bwd(int64_t batch, int64_t seqlen, int64_t dim, int64_t width, int io_dtype,
+                        const void* x, const float* w, const float* bias, int silu,
+                        const void* dout, void* dx, float* dw, float* dbias, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  int st = conv_check(batch, seqlen, dim, width, io_dtype);
+  if (st != SSM_OK) return st;
+  if (batch == 0 || dim == 0) return SSM_OK;
+  if (!w) return SSM_ERR_INVALID_ARG;
+  if (seqlen > 0 && (!x || !dout || !dx)) return SSM_ERR_INVALID_ARG;
+  const size_t es = io_bytes(io_dtype), n = (size_t)batch * seqlen * dim;
+  const void* io_ptrs[] = {x, dout, dx};
+  for (const void* q : io_ptrs)
+    if (q && !aligned(q, es)) return SSM_ERR_INVALID_ARG;
+  const void* f_ptrs[] = {w, bias, dw, dbias};
+  for (const void* q : f_ptrs)
+    if (q && !aligned(q, 4)) return SSM_ERR_INVALID_ARG;
+  const size_t bw = (size_t)dim * width * 4, bd = (size_t)dim * 4;
+  if (overlap(dx, n * es, x, n * es) || overlap(dx, n * es, dout, n * es) ||
+      overlap(dx, n * es, w, bw) || overlap(dx, n * es, bias, bd) || overlap(dw, bw, w, bw) ||
+      overlap(dw, bw, bias, bd) || overlap(dbias, bd, w, bw) || overlap(dbias, bd, bias, bd) ||
+      overlap(dw, bw, dx, n * es) || overlap(dbias, bd, dx, n * es) || overlap(dw, bw, dbias, bd) ||
+      overlap(dw, bw, x, n * es) || overlap(dw, bw, dout, n * es) ||
+      overlap(dbias, bd, x, n * es) || overlap(dbias, bd, dout, n * es))
+    return fail(SSM_ERR_INVALID_ARG, "ssm_conv1d_silu_bwd: an output overlaps an input");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (seqlen == 0) {
+    cudaError_t e = dw ? cudaMemsetAsync(dw, 0, bw, s) : cudaSuccess;
+    if (e == cudaSuccess && dbias) e = cudaMemsetAsync(dbias, 0, bd, s);
+    return cuda_status(e, "ssm_conv1d_silu_bwd: empty sequence");
+  }
+  const size_t need = ssm_conv1d_silu_bwd_workspace_bytes(batch, seqlen, dim, width, io_dtype);
+  if (!workspace || workspace_bytes < need || !aligned(workspace, 16))
+    return fail(SSM_ERR_WORKSPACE, "ssm_conv1d_silu_bwd: workspace missing, too small or unaligned");
+  ConvParams p = conv_params(batch, seqlen, dim, width, silu, true);
+  p.x = x; p.w = w; p.bias = bias; p.dout = dout; p.dx = dx; p.dw = dw; p.dbias = dbias;
+  p.w_vec = aligned(w, 16) ? 1 : 0;
+  const size_t chunks = (size_t)((seqlen + p.chunk - 1) / p.chunk);
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  p.ws_dw = reinterpret_cast<float*>(ws);
+  p.ws_db = reinterpret_cast<float*>(
+      ws + align_up(sizeof(float) * (size_t)batch * chunks * dim * width, 256));
+  return cuda_status(launch_conv(p, io_dtype == SSM_DTYPE_BF16,
+                                 conv_vec(dim, io_dtype, {x, dout, dx}), true, s),
+                     "conv1d backward launch");
 }
 
 }  // extern "C"

@@ -38,6 +38,8 @@ _lib = None
 STREAM_X, STREAM_DELTA, STREAM_Z, STREAM_B, STREAM_C, STREAM_H0, STREAM_BIAS = 1, 2, 3, 4, 5, 6, 7
 # upstream gradients of the backward pass
 STREAM_DY, STREAM_DH_LAST = 8, 9
+# the block's causal conv1d: raw input, taps, bias, upstream gradient
+STREAM_CONV_X, STREAM_CONV_W, STREAM_CONV_BIAS, STREAM_CONV_DOUT = 10, 11, 12, 13
 KIND_NORMAL, KIND_UNIFORM = 0, 1
 OUT_F64, OUT_F32, OUT_BF16 = 0, 1, 2
 
@@ -248,6 +250,20 @@ def make_grad_inputs(batch, seqlen, dim, dstate, io, seed, *, with_dh_last=True,
         "dy": fill((batch, seqlen, dim), seed, STREAM_DY, out=io, offset=o_ld, nthreads=nthreads),
         "dh_last": (fill((batch, dim, dstate), seed, STREAM_DH_LAST, out="f32", offset=o_dn,
                          nthreads=nthreads) if with_dh_last else None),
+    }
+
+
+def make_conv_inputs(batch, seqlen, dim, width, io, seed, *, nthreads=None):
+    """Inputs of the block's causal depthwise conv1d: x (batch, L, dim) ~ N(0, 1)
+    in the io type, taps w (dim, width) and bias (dim,) ~ U[-0.5, 0.5] fp32
+    (the range of nn.Conv1d's default initialisation for groups = channels
+    and 4 taps), dout (batch, L, dim) ~ N(0, 1) in the io type."""
+    shape = (batch, seqlen, dim)
+    return {
+        "x": fill(shape, seed, STREAM_CONV_X, out=io, nthreads=nthreads),
+        "w": fill((dim, width), seed, STREAM_CONV_W, KIND_UNIFORM, -0.5, 0.5, out="f32"),
+        "bias": fill((dim,), seed, STREAM_CONV_BIAS, KIND_UNIFORM, -0.5, 0.5, out="f32"),
+        "dout": fill(shape, seed, STREAM_CONV_DOUT, out=io, nthreads=nthreads),
     }
 
 

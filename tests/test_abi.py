@@ -170,6 +170,38 @@ def test_scan_bwd_rejects_bad_arguments(L):
     assert bwd(batch=0) == 0 and bwd(dim=0) == 0
 
 
+@no_gpu_only
+def test_conv_rejects_bad_arguments(L):
+    K = 1 << 16
+
+    def fwd(**kw):
+        a = dict(batch=2, seqlen=32, dim=64, width=4, io=1, x=FAKE, w=FAKE + K, bias=None, silu=1,
+                 out=FAKE + 2 * K)
+        a.update(kw)
+        return L.ssm_conv1d_silu_fwd(a["batch"], a["seqlen"], a["dim"], a["width"], a["io"],
+                                     a["x"], a["w"], a["bias"], a["silu"], a["out"], None)
+
+    def bwd(**kw):
+        a = dict(batch=2, seqlen=32, dim=64, width=4, io=1, x=FAKE, w=FAKE + K, bias=None, silu=1,
+                 dout=FAKE + 2 * K, dx=FAKE + 3 * K, dw=FAKE + 4 * K, db=FAKE + 5 * K, ws=None,
+                 ws_bytes=0)
+        a.update(kw)
+        return L.ssm_conv1d_silu_bwd(a["batch"], a["seqlen"], a["dim"], a["width"], a["io"],
+                                     a["x"], a["w"], a["bias"], a["silu"], a["dout"], a["dx"],
+                                     a["dw"], a["db"], a["ws"], a["ws_bytes"], None)
+    assert fwd(x=None) == -1 and fwd(w=None) == -1 and fwd(out=None) == -1
+    assert fwd(width=5) == -2 and fwd(width=1) == -2 and fwd(io=2) == -2
+    assert fwd(out=FAKE + 64) == -1     # out overlaps x
+    assert fwd(out=FAKE + 2 * K + 1) == -1  # misaligned bf16
+    assert fwd(seqlen=0) == 0 and fwd(batch=0) == 0
+    assert bwd(dx=FAKE + 2 * K + 64) == -1  # dx overlaps dout
+    assert bwd(dw=FAKE + K) == -1       # dw overlaps w
+    assert bwd(dout=None) == -1
+    assert bwd() == -3                  # no workspace
+    need = L.ssm_conv1d_silu_bwd_workspace_bytes(2, 32, 64, 4, 1)
+    assert need > 0 and bwd(ws=FAKE * 64, ws_bytes=need - 1) == -3
+
+
 def test_binding_has_no_cpu_path():
     from selective_state_space_39_b200 import ssm_scan_fwd
     x = torch.zeros(1, 4, 8)
