@@ -224,12 +224,22 @@ __global__ void __launch_bounds__(kMaxThreads) conv_bwd_kernel(const ConvParams 
   // t runs over [t0, t1 + W - 1): du[t] for the chunk and the W-1 rows after
   // it (needed by dx of the chunk's last rows); dx[s] for s = t - (W-1) >= t0.
   const int tend = t1 + (W - 1);
+  const int tlim = min(L, tend);
+  // rows of the next group are loaded before the current group is computed
+  typename Vec<IOT, VEC>::Raw xn[kUnrollBwd], gn[kUnrollBwd];
+#pragma unroll
+  for (int j = 0; j < kUnrollBwd; ++j) {
+    xn[j] = load_raw<IOT, VEC>(x, t0 + j, tlim, dim, d0, row0);
+    gn[j] = load_raw<IOT, VEC>(dout, t0 + j, tlim, dim, d0, row0);
+  }
   for (int tb = t0; tb < tend; tb += kUnrollBwd) {
     typename Vec<IOT, VEC>::Raw xr[kUnrollBwd], gr[kUnrollBwd];
 #pragma unroll
     for (int j = 0; j < kUnrollBwd; ++j) {
-      xr[j] = load_raw<IOT, VEC>(x, tb + j, min(L, tend), dim, d0, row0);
-      gr[j] = load_raw<IOT, VEC>(dout, tb + j, min(L, tend), dim, d0, row0);
+      xr[j] = xn[j];
+      gr[j] = gn[j];
+      xn[j] = load_raw<IOT, VEC>(x, tb + kUnrollBwd + j, tlim, dim, d0, row0);
+      gn[j] = load_raw<IOT, VEC>(dout, tb + kUnrollBwd + j, tlim, dim, d0, row0);
     }
 #pragma unroll
     for (int j = 0; j < kUnrollBwd; ++j) {
