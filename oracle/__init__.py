@@ -69,6 +69,11 @@ class Oracle:
                       _F32P, ctypes.c_void_p, ctypes.c_void_p, _F32P, ctypes.c_void_p,
                       _F32P, ctypes.c_int, _F32P, _I64P, ctypes.c_int64, _F64P, _F64P,
                       ctypes.c_int]
+        fz = self.lib.oracle_selective_scan_zoh
+        fz.restype = ctypes.c_int
+        fz.argtypes = f.argtypes
+        gz = self.lib.oracle_state_update_zoh
+        gz.restype = ctypes.c_int
         fb = self.lib.oracle_selective_scan_bwd
         fb.restype = ctypes.c_int
         fb.argtypes = [ctypes.c_int64] * 4 + [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
@@ -88,6 +93,7 @@ class Oracle:
         g.argtypes = [ctypes.c_int64] * 3 + [ctypes.c_int, _F64P, ctypes.c_void_p,
                       ctypes.c_void_p, _F32P, ctypes.c_void_p, ctypes.c_void_p, _F32P,
                       ctypes.c_void_p, _F32P, ctypes.c_int, _F64P]
+        gz.argtypes = g.argtypes
 
     # -- helpers -----------------------------------------------------------
     @staticmethod
@@ -125,11 +131,12 @@ class Oracle:
 
     # -- the scan ----------------------------------------------------------
     def selective_scan(self, x, delta, A, B, C, D=None, z=None, delta_bias=None,
-                       softplus=True, h0=None, io="f32", channels=None, nthreads=1):
+                       softplus=True, h0=None, io="f32", channels=None, nthreads=1, zoh=False):
         """Selective scan over all channels, or over ``channels`` (a list of
         (b, d) pairs). Returns ``(y, h_last)`` in fp64: for all channels
         y is (batch, L, dim) and h_last (batch, dim, N); for a channel list
-        y is (nchan, L) and h_last (nchan, N)."""
+        y is (nchan, L) and h_last (nchan, N). ``zoh``: the exact zero-order
+        hold input term (exp(Delta A) - 1) / A * B instead of Delta * B."""
         x = np.asarray(x)
         batch, L, dim = x.shape
         N = np.asarray(A).shape[1]
@@ -151,7 +158,8 @@ class Oracle:
         nchan = chans.shape[0]
         y = np.empty((nchan, L), dtype=np.float64)
         h_last = np.empty((nchan, N), dtype=np.float64)
-        rc = self.lib.oracle_selective_scan(
+        fn = self.lib.oracle_selective_scan_zoh if zoh else self.lib.oracle_selective_scan
+        rc = fn(
             batch, L, dim, N, 1 if io == "bf16" else 0, self._ptr(x), self._ptr(delta),
             self._ptr(A, ctypes.c_float), self._ptr(B), self._ptr(C),
             self._ptr(D, ctypes.c_float), self._ptr(z), self._ptr(delta_bias, ctypes.c_float),
@@ -277,7 +285,7 @@ class Oracle:
 
     # -- decode ------------------------------------------------------------
     def state_update(self, state, x, delta, A, B, C, D=None, z=None, delta_bias=None,
-                     softplus=True, io="f32"):
+                     softplus=True, io="f32", zoh=False):
         """One decode step on the fp64 ``state`` (batch, dim, N), in place.
         Returns y (batch, dim) in fp64."""
         if state.dtype != np.float64 or not state.flags.c_contiguous:
@@ -292,7 +300,8 @@ class Oracle:
         D = self._f32_array(D, (dim,), "D")
         delta_bias = self._f32_array(delta_bias, (dim,), "delta_bias")
         y = np.empty((batch, dim), dtype=np.float64)
-        rc = self.lib.oracle_state_update(
+        fn = self.lib.oracle_state_update_zoh if zoh else self.lib.oracle_state_update
+        rc = fn(
             batch, dim, N, 1 if io == "bf16" else 0, self._ptr(state, ctypes.c_double),
             self._ptr(x), self._ptr(delta), self._ptr(A, ctypes.c_float), self._ptr(B),
             self._ptr(C), self._ptr(D, ctypes.c_float), self._ptr(z),

@@ -16,7 +16,9 @@
  *            + Delta * B[b,t,n] * x[b,t,d]           (discretised recurrence,
  *                                                    §2.2, with the simplified
  *                                                    deltaB = Delta*B of the
- *                                                    §3.3 selective_scan)
+ *                                                    §3.3 selective_scan; the
+ *                                                    _zoh entry points use the
+ *                                                    exact ZOH B-bar of §2.2)
  *   y      = sum_n C[b,t,n] * h[n] + D[d] * x[b,t,d] (readout, §2.2 y_t = C h_t,
  *                                                    plus the block's D skip)
  *   y     *= z / (1 + exp(-z))   if z is given       (block gate y * SiLU(z), §3.4)
@@ -65,6 +67,15 @@ static double softplus(double v) { return v > 20.0 ? v : log1p(exp(v)); }
 /* SiLU(z) = z * sigmoid(z) (§3.4 gate). */
 static double silu(double z) { return z / (1.0 + exp(-z)); }
 
+/* The factor that multiplies B[n] x in the state update: Delta (the
+ * simplified deltaB = Delta*B of the §3.3 selective_scan), or, for the exact
+ * zero-order hold of §2.2, B-bar = (Delta A)^-1 (exp(Delta A) - 1) Delta B,
+ * which for a diagonal A is (exp(Delta A_n) - 1) / A_n (Delta at A_n = 0). */
+static double input_coef(double dt, double An, int zoh) {
+  if (!zoh) return dt;
+  return An == 0.0 ? dt : expm1(dt * An) / An;
+}
+
 typedef struct {
   int64_t batch, seqlen, dim, dstate;
   int is_bf16;
@@ -82,6 +93,7 @@ typedef struct {
   int64_t nchan;
   double* y;           /* (nchan, seqlen)                 */
   double* h_last;      /* (nchan, dstate) or NULL         */
+  int zoh;             /* input term: 0 Delta*B (§3.3), 1 exact ZOH (§2.2) */
 } scan_job;
 
 /* One channel (b, d), sequentially in t: the loop of the §3.3 selective_scan
@@ -103,7 +115,8 @@ static void scan_one_channel(const scan_job* j, int64_t k) {
     double y = 0.0;
     for (int64_t n = 0; n < N; ++n) {
       const double dA = exp(dt * (double)j->A[d * N + n]);
-      const double dB = dt * widen(j->B, i_bln + n, j->is_bf16);
+      const double dB = input_coef(dt, (double)j->A[d * N + n], j->zoh) *
+                        widen(j->B, i_bln + n, j->is_bf16);
       h[n] = dA * h[n] + dB * xv;
       y += widen(j->C, i_bln + n, j->is_bf16) * h[n];
     }
@@ -131,12 +144,39 @@ static void* scan_worker(void* arg) {
  * (b, d) pairs in `chans`, splitting the channels over `nthreads` threads
  * (each channel stays sequential in t). Returns 0, or -1 on bad arguments.
  */
+static int scan_impl(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate, int is_bf16,
+                     const void* x, const void* delta, const float* A, const void* B,
+                     const void* C, const float* D, const void* z, const float* bias,
+                     int softplus_on, const float* h0, const int64_t* chans, int64_t nchan,
+                     double* y, double* h_last, int nthreads, int zoh);
+
 int oracle_selective_scan(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
                           int is_bf16, const void* x, const void* delta, const float* A,
                           const void* B, const void* C, const float* D, const void* z,
                           const float* bias, int softplus_on, const float* h0,
                           const int64_t* chans, int64_t nchan, double* y, double* h_last,
                           int nthreads) {
+  return scan_impl(batch, seqlen, dim, dstate, is_bf16, x, delta, A, B, C, D, z, bias,
+                   softplus_on, h0, chans, nchan, y, h_last, nthreads, 0);
+}
+
+/* oracle_selective_scan_zoh -- the same scan with the exact zero-order-hold
+ * input term of §2.2 (B-bar = (exp(Delta A) - 1) / A * B per state). */
+int oracle_selective_scan_zoh(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
+                              int is_bf16, const void* x, const void* delta, const float* A,
+                              const void* B, const void* C, const float* D, const void* z,
+                              const float* bias, int softplus_on, const float* h0,
+                              const int64_t* chans, int64_t nchan, double* y, double* h_last,
+                              int nthreads) {
+  return scan_impl(batch, seqlen, dim, dstate, is_bf16, x, delta, A, B, C, D, z, bias,
+                   softplus_on, h0, chans, nchan, y, h_last, nthreads, 1);
+}
+
+static int scan_impl(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate, int is_bf16,
+                     const void* x, const void* delta, const float* A, const void* B,
+                     const void* C, const float* D, const void* z, const float* bias,
+                     int softplus_on, const float* h0, const int64_t* chans, int64_t nchan,
+                     double* y, double* h_last, int nthreads, int zoh) {
   if (batch < 0 || seqlen < 0 || dim < 0 || dstate <= 0 || dstate > ORACLE_MAX_N) return -1;
   if (!x || !delta || !A || !B || !C || !chans || !y) return -1;
   for (int64_t k = 0; k < nchan; ++k)
@@ -144,7 +184,7 @@ int oracle_selective_scan(int64_t batch, int64_t seqlen, int64_t dim, int64_t ds
         chans[2 * k + 1] >= dim)
       return -1;
   scan_job job = {batch, seqlen, dim, dstate, is_bf16, x, delta, A, B, C, D, z,
-                  bias, softplus_on, h0, chans, nchan, y, h_last};
+                  bias, softplus_on, h0, chans, nchan, y, h_last, zoh};
   if (nthreads < 1) nthreads = 1;
   if (nthreads > 256) nthreads = 256;
   if (nthreads == 1 || nchan < 2) {
@@ -177,10 +217,32 @@ int oracle_selective_scan(int64_t batch, int64_t seqlen, int64_t dim, int64_t ds
  * oracle's own fp64 (batch, dim, dstate) state, updated in place; y is
  * (batch, dim). x, delta, z are (batch, dim); B, C are (batch, dstate).
  */
+static int state_update_impl(int64_t batch, int64_t dim, int64_t dstate, int is_bf16,
+                             double* state, const void* x, const void* delta, const float* A,
+                             const void* B, const void* C, const float* D, const void* z,
+                             const float* bias, int softplus_on, double* y, int zoh);
+
 int oracle_state_update(int64_t batch, int64_t dim, int64_t dstate, int is_bf16,
                         double* state, const void* x, const void* delta, const float* A,
                         const void* B, const void* C, const float* D, const void* z,
                         const float* bias, int softplus_on, double* y) {
+  return state_update_impl(batch, dim, dstate, is_bf16, state, x, delta, A, B, C, D, z, bias,
+                           softplus_on, y, 0);
+}
+
+/* oracle_state_update_zoh -- one decode step with the exact ZOH input term. */
+int oracle_state_update_zoh(int64_t batch, int64_t dim, int64_t dstate, int is_bf16,
+                            double* state, const void* x, const void* delta, const float* A,
+                            const void* B, const void* C, const float* D, const void* z,
+                            const float* bias, int softplus_on, double* y) {
+  return state_update_impl(batch, dim, dstate, is_bf16, state, x, delta, A, B, C, D, z, bias,
+                           softplus_on, y, 1);
+}
+
+static int state_update_impl(int64_t batch, int64_t dim, int64_t dstate, int is_bf16,
+                             double* state, const void* x, const void* delta, const float* A,
+                             const void* B, const void* C, const float* D, const void* z,
+                             const float* bias, int softplus_on, double* y, int zoh) {
   if (batch < 0 || dim < 0 || dstate <= 0 || !state || !x || !delta || !A || !B || !C || !y)
     return -1;
   for (int64_t b = 0; b < batch; ++b) {
@@ -193,7 +255,8 @@ int oracle_state_update(int64_t batch, int64_t dim, int64_t dstate, int is_bf16,
       double acc = 0.0;
       for (int64_t n = 0; n < dstate; ++n) {
         const double dA = exp(dt * (double)A[d * dstate + n]);
-        const double dB = dt * widen(B, b * dstate + n, is_bf16);
+        const double dB = input_coef(dt, (double)A[d * dstate + n], zoh) *
+                          widen(B, b * dstate + n, is_bf16);
         h[n] = dA * h[n] + dB * xv;
         acc += widen(C, b * dstate + n, is_bf16) * h[n];
       }
@@ -371,7 +434,7 @@ int oracle_selective_scan_bwd(int64_t batch, int64_t seqlen, int64_t dim, int64_
   if (nchan < nthreads) nthreads = nchan > 0 ? (int)nchan : 1;
   bwd_job job;
   scan_job f = {batch, seqlen, dim, dstate, is_bf16, x, delta, A, B, C, D, z,
-                bias, softplus_on, h0, chans, nchan, NULL, NULL};
+                bias, softplus_on, h0, chans, nchan, NULL, NULL, 0};
   job.fwd = f;
   job.dy = dy;
   job.dh_last = dh_last;

@@ -497,6 +497,60 @@ def pin_conv_bwd_finite_differences(o):
             _close(g, fd, 0.0, 2e-6 * scale, what=f"conv d{name} vs central differences")
 
 
+# --------------------------------------------------------------------------
+# pins of the exact zero-order-hold input term (§2.2)
+def pin_zoh_matches_scipy_cont2discrete(o):
+    """Per step, the ZOH discretisation of dh/dt = diag(A_d) h + B_t x_t
+    computed by scipy.signal.cont2discrete(method='zoh') (a matrix exponential
+    of the augmented system), chained over the steps, equals the oracle's
+    ZOH scan."""
+    from scipy.signal import cont2discrete
+    c = random_case(301, batch=1, L=6, dim=2, N=3)
+    y, hl = o.selective_scan(c["x"], c["delta"], c["A"], c["B"], c["C"], D=c["D"], z=c["z"],
+                             delta_bias=c["delta_bias"], softplus=True, h0=c["h0"], zoh=True)
+    dt = _delta_f64(c)
+    for d in range(2):
+        A = np.diag(c["A"][d].astype(np.float64))
+        h = c["h0"][0, d].astype(np.float64)
+        for t in range(6):
+            Bcol = c["B"][0, t].astype(np.float64).reshape(3, 1)
+            Ad, Bd, _, _, _ = cont2discrete((A, Bcol, np.zeros((1, 3)), np.zeros((1, 1))),
+                                            float(dt[0, t, d]), method="zoh")
+            h = Ad @ h + Bd[:, 0] * float(c["x"][0, t, d])
+            yy = float(c["C"][0, t].astype(np.float64) @ h) + float(c["D"][d]) * float(c["x"][0, t, d])
+            zz = float(c["z"][0, t, d])
+            yy *= zz / (1 + math.exp(-zz))
+            _close(y[0, t, d], yy, 1e-10, 1e-12, what="zoh vs cont2discrete y")
+        _close(hl[0, d], h, 1e-10, 1e-12, what="zoh vs cont2discrete h_last")
+
+
+def pin_zoh_small_step_is_euler(o):
+    """For Delta |A| -> 0 the ZOH input term (exp(Delta A) - 1) / A tends to
+    Delta: with Delta ~ 1e-7 the two discretisations agree to ~1e-7 relative."""
+    c = random_case(303, gate=False, softplus=False)
+    c["delta"] = _f32(np.full(c["delta"].shape, 1e-7))
+    c["delta_bias"] = None
+    kw = dict(D=c["D"], softplus=False, h0=c["h0"])
+    ye, he = o.selective_scan(c["x"], c["delta"], c["A"], c["B"], c["C"], **kw)
+    yz, hz = o.selective_scan(c["x"], c["delta"], c["A"], c["B"], c["C"], zoh=True, **kw)
+    assert not np.array_equal(yz, ye), "zoh flag ignored"
+    _close(yz, ye, 1e-6, 1e-12, what="zoh small-step limit")
+
+
+def pin_zoh_decode_steps_equal_scan(o):
+    """L ZOH decode steps reproduce one ZOH scan."""
+    c = random_case(305, batch=2, L=5, dim=3, N=4)
+    y, hl = o.selective_scan(c["x"], c["delta"], c["A"], c["B"], c["C"], D=c["D"], z=c["z"],
+                             delta_bias=c["delta_bias"], softplus=True, h0=c["h0"], zoh=True)
+    state = c["h0"].astype(np.float64).copy()
+    for t in range(5):
+        yt = o.state_update(state, c["x"][:, t], c["delta"][:, t], c["A"], c["B"][:, t],
+                            c["C"][:, t], D=c["D"], z=c["z"][:, t], delta_bias=c["delta_bias"],
+                            softplus=True, zoh=True)
+        _close(yt, y[:, t], 1e-13, 1e-14, what="zoh decode step")
+    _close(state, hl, 1e-13, 1e-14, what="zoh decode state")
+
+
 ALL_PINS = [
     pin_softplus_library,
     pin_silu_library,
@@ -518,4 +572,7 @@ ALL_PINS = [
     pin_conv_by_hand,
     pin_conv_is_causal,
     pin_conv_bwd_finite_differences,
+    pin_zoh_matches_scipy_cont2discrete,
+    pin_zoh_small_step_is_euler,
+    pin_zoh_decode_steps_equal_scan,
 ]

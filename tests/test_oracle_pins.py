@@ -58,8 +58,8 @@ MUTANTS = {
     "readout_before_update": (
         "      h[n] = dA * h[n] + dB * xv;\n      y += widen(j->C, i_bln + n, j->is_bf16) * h[n];",
         "      y += widen(j->C, i_bln + n, j->is_bf16) * h[n];\n      h[n] = dA * h[n] + dB * xv;"),
-    "B_C_swapped": ("const double dB = dt * widen(j->B, i_bln + n, j->is_bf16);\n      h[n] = dA * h[n] + dB * xv;\n      y += widen(j->C,",
-                    "const double dB = dt * widen(j->C, i_bln + n, j->is_bf16);\n      h[n] = dA * h[n] + dB * xv;\n      y += widen(j->B,"),
+    "B_C_swapped": ("                        widen(j->B, i_bln + n, j->is_bf16);\n      h[n] = dA * h[n] + dB * xv;\n      y += widen(j->C,",
+                    "                        widen(j->C, i_bln + n, j->is_bf16);\n      h[n] = dA * h[n] + dB * xv;\n      y += widen(j->B,"),
     "bias_dropped": ("widen(j->delta, i_bld, j->is_bf16) + bias;", "widen(j->delta, i_bld, j->is_bf16);"),
     "softplus_as_exp": ("return v > 20.0 ? v : log1p(exp(v));", "return v > 20.0 ? v : exp(v);"),
     "sigmoid_not_silu": ("return z / (1.0 + exp(-z));", "return 1.0 / (1.0 + exp(-z));"),
@@ -67,8 +67,8 @@ MUTANTS = {
     "A_transposed": ("exp(dt * (double)j->A[d * N + n])", "exp(dt * (double)j->A[(n * Dm + d) % (Dm * N)])"),
     "x_index_wrong": ("const double xv = widen(j->x, i_bld, j->is_bf16);",
                       "const double xv = widen(j->x, (i_bld + 1) % (j->batch * L * Dm), j->is_bf16);"),
-    "dB_without_delta": ("const double dB = dt * widen(j->B, i_bln + n, j->is_bf16);",
-                         "const double dB = widen(j->B, i_bln + n, j->is_bf16);"),
+    "dB_without_delta": ("      const double dB = input_coef(dt, (double)j->A[d * N + n], j->zoh) *\n",
+                         "      const double dB = 1.0 *\n"),
     "decode_drops_gate": ("      if (z) acc *= silu(widen(z, i_bd, is_bf16));\n", ""),
     "decode_state_not_kept": ("        h[n] = dA * h[n] + dB * xv;\n        acc +=",
                               "        const double hn = dA * h[n] + dB * xv;\n        acc += 0 * hn +"),
@@ -101,6 +101,12 @@ MUTANTS = {
     "conv_bwd_dw_wrong_step": ("if (s >= 0) dw[d * width + k] += du[t] * widen(x, (b * seqlen + s) * dim + d, is_bf16);",
                                "if (s >= 0) dw[d * width + k] += du[t] * widen(x, (b * seqlen + t) * dim + d, is_bf16);"),
     "conv_bwd_dbias_from_dout": ("        dbias[d] += du[t];", "        dbias[d] += g;"),
+    # exact zero-order hold
+    "zoh_is_euler": ("  return An == 0.0 ? dt : expm1(dt * An) / An;", "  return dt;"),
+    "zoh_no_division_by_A": ("  return An == 0.0 ? dt : expm1(dt * An) / An;",
+                             "  return An == 0.0 ? dt : expm1(dt * An);"),
+    "zoh_sign_flipped": ("  return An == 0.0 ? dt : expm1(dt * An) / An;",
+                         "  return An == 0.0 ? dt : -expm1(dt * An) / An;"),
 }
 
 
