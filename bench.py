@@ -48,6 +48,8 @@ def parse_args():
                     choices=sorted(gen.SCAN_WORKLOADS) + sorted(gen.DECODE_WORKLOADS))
     ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd"],
                     help="bwd: time ssm_scan_bwd (the gradients) on the same workload")
+    ap.add_argument("--zoh", action="store_true",
+                    help="scan with the exact zero-order-hold input term (ssm_scan_fwd_zoh)")
     ap.add_argument("--op", default="scan", choices=["scan", "conv"],
                     help="conv: time the block's causal conv1d + SiLU (forward and backward) "
                          "on the workload's (batch, seqlen, dim)")
@@ -69,11 +71,13 @@ def algorithmic_bytes(w, batch):
     return bld * per_elem + 2 * bln * es + state + params
 
 
-def alu_ops_per_element(w):
+def alu_ops_per_element(w, zoh=False):
     """FP32 operations the recurrence needs per element in its plain form:
     per state one multiply for the decay power, one for Delta x B, one FMA for
-    the state and one for the readout (4N), as counted for the roofline."""
-    return 4 * w.dstate
+    the state and one for the readout (4N), as counted for the roofline. The
+    exact ZOH input term adds one operation per state (the power
+    exp(Delta A_n) - 1 next to the decay): 5N."""
+    return (5 if zoh else 4) * w.dstate
 
 
 def measured_traffic(workload):
@@ -159,7 +163,7 @@ class ClockSampler:
                 "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
 
 
-def cpu_oracle_rate(w, inp, target_s, rng_seed=0):
+def cpu_oracle_rate(w, inp, target_s, rng_seed=0, zoh=False):
     """Oracle throughput (elements/s) on a bounded sample of the workload's
     channels, all host threads. Returns (value, cores, sample text)."""
     import oracle
@@ -174,7 +178,7 @@ def cpu_oracle_rate(w, inp, target_s, rng_seed=0):
         t0 = time.perf_counter()
         oracle.selective_scan(inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], D=inp["D"],
                               z=inp["z"], delta_bias=inp["delta_bias"], h0=inp["h0"], io=w.io,
-                              channels=chans, nthreads=threads)
+                              channels=chans, nthreads=threads, zoh=zoh)
         return len(chans), time.perf_counter() - t0
 
     n, dt = run(threads)  # calibration
@@ -607,7 +611,8 @@ def main():
 
     def step():
         ssm_scan_fwd(d["x"], d["delta"], d["A"], d["B"], d["C"], D=d["D"], z=d["z"],
-                     delta_bias=d["delta_bias"], h0=d["h0"], y=y, h_last=h_last, workspace=ws)
+                     delta_bias=d["delta_bias"], h0=d["h0"], y=y, h_last=h_last, workspace=ws,
+                     zoh=args.zoh)
 
     for _ in range(max(3, args.warmup)):
         flush.fill_(1)
@@ -641,12 +646,14 @@ def main():
     sm_mhz = clocks.get("sm_mhz") or B200_MAX_SM_MHZ
     alu_peak = B200_SMS * FP32_LANES_PER_SM * sm_mhz * 1e6 / 1e9  # Gop/s
     mean_s = statistics.mean(step_ms) * 1e-3
-    alu_achieved = alu_ops_per_element(w) * nb * w.seqlen * w.dim / mean_s / 1e9
-    traffic = measured_traffic(w.name) if world == 1 or nb == w.batch else None
-    kernel = "ssm_scan_fwd: carry pass + main pass (%d launches)" % plan.kernels
+    alu_achieved = alu_ops_per_element(w, args.zoh) * nb * w.seqlen * w.dim / mean_s / 1e9
+    traffic = (measured_traffic(w.name) if (world == 1 or nb == w.batch) and not args.zoh
+               else None)
+    kernel = "%s: carry pass + main pass (%d launches)" % (
+        "ssm_scan_fwd_zoh" if args.zoh else "ssm_scan_fwd", plan.kernels)
     roofline = {"bound": "alu", "achieved": round(alu_achieved, 1), "peak": round(alu_peak, 1),
                 "unit": "Gop/s", "frac": round(alu_achieved / alu_peak, 4), "traffic": traffic,
-                "kernel": kernel, "ops_per_element": alu_ops_per_element(w),
+                "kernel": kernel, "ops_per_element": alu_ops_per_element(w, args.zoh),
                 "peak_kind": f"derived: {B200_SMS} SMs x {FP32_LANES_PER_SM} FP32 lanes x "
                              f"{sm_mhz:.0f} MHz sampled SM clock"}
     peak, peak_kind = measured_hbm_peak()
@@ -686,7 +693,7 @@ def main():
 
     cpu = None
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
-        v, cores, sample = cpu_oracle_rate(w, inp, args.cpu_seconds)
+        v, cores, sample = cpu_oracle_rate(w, inp, args.cpu_seconds, zoh=args.zoh)
         cpu = {"value": v, "unit": "elements/s", "cores": cores, "kind": "oracle",
                "sample": sample}
 
@@ -701,6 +708,7 @@ def main():
                        "seqlen": w.seqlen, "dim": w.dim, "dstate": w.dstate, "io": w.io,
                        "gate": w.gate, "skip": w.skip, "h0": w.with_h0,
                        "segments": plan.segments, "segment_steps": plan.segment_steps,
+                       "input_term": "exact ZOH" if args.zoh else "Delta B",
                        "l2": "flushed (256 MB write) before every timed step",
                        "parallelism": f"dp{world} (batch shards, no data-path collective)"},
             "hbm_gbs": round(achieved, 1), "hbm_frac_of_peak": round(achieved / peak, 4),

@@ -127,6 +127,22 @@ int ssm_scan_fwd(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate, int
                  size_t workspace_bytes, void* stream);
 
 /*
+ * ssm_scan_fwd_zoh -- ssm_scan_fwd with the exact zero-order-hold input term
+ * of §2.2 instead of the simplified Delta * B of the §3.3 listing:
+ *
+ *   h[n] = exp(Delta A[d,n]) h[n] + B-bar[n] x[b,t,d],
+ *   B-bar[n] = (Delta A)^-1 (exp(Delta A) - 1) Delta B = (exp(Delta A[d,n]) - 1) / A[d,n] * B[b,t,n]
+ *
+ * (Delta B where A[d,n] = 0). Same arguments, layouts, workspace and errors as
+ * ssm_scan_fwd (the workspace size is the same).
+ */
+int ssm_scan_fwd_zoh(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate, int io_dtype,
+                     const void* x, const void* delta, const float* A, const void* B,
+                     const void* C, const float* D, const void* z, const float* delta_bias,
+                     int softplus, const float* h0, void* y, float* h_last, void* workspace,
+                     size_t workspace_bytes, void* stream);
+
+/*
  * ssm_scan_fwd_noalloc -- ssm_scan_fwd for callers that cannot allocate
  * device memory. The Mamba pages have no counterpart to this call; it exists
  * for callers that only get their input and output buffers and may not call
@@ -256,6 +272,13 @@ int ssm_conv1d_silu_bwd(int64_t batch, int64_t seqlen, int64_t dim, int64_t widt
                         const void* x, const float* w, const float* bias, int silu,
                         const void* dout, void* dx, float* dw, float* dbias, void* workspace,
                         size_t workspace_bytes, void* stream);
+
+/* ssm_state_update_zoh -- ssm_state_update with the exact zero-order-hold
+ * input term (see ssm_scan_fwd_zoh). Same arguments and errors. */
+int ssm_state_update_zoh(int64_t batch, int64_t dim, int64_t dstate, int io_dtype, float* state,
+                         const void* x, const void* delta, const float* A, const void* B,
+                         const void* C, const float* D, const void* z, const float* delta_bias,
+                         int softplus, void* y, void* stream);
 
 /*
  * ssm_scan_status -- synchronise `stream`, then report whether every CTA of

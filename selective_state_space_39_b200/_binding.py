@@ -68,6 +68,8 @@ def lib() -> ctypes.CDLL:
         L.ssm_scan_fwd.argtypes = [_I64, _I64, _I64, _I64, ctypes.c_int, _VP, _VP, _VP, _VP, _VP,
                                    _VP, _VP, _VP, ctypes.c_int, _VP, _VP, _VP, _VP,
                                    ctypes.c_size_t, _VP]
+        L.ssm_scan_fwd_zoh.restype = ctypes.c_int
+        L.ssm_scan_fwd_zoh.argtypes = L.ssm_scan_fwd.argtypes
         L.ssm_scan_fwd_noalloc.restype = ctypes.c_int
         L.ssm_scan_fwd_noalloc.argtypes = [_I64, _I64, _I64, _I64, ctypes.c_int, _VP, _VP, _VP,
                                            _VP, _VP, _VP, _VP, _VP, ctypes.c_int, _VP, _VP, _VP,
@@ -92,6 +94,8 @@ def lib() -> ctypes.CDLL:
         L.ssm_state_update.restype = ctypes.c_int
         L.ssm_state_update.argtypes = [_I64, _I64, _I64, ctypes.c_int, _VP, _VP, _VP, _VP, _VP,
                                        _VP, _VP, _VP, _VP, ctypes.c_int, _VP, _VP]
+        L.ssm_state_update_zoh.restype = ctypes.c_int
+        L.ssm_state_update_zoh.argtypes = L.ssm_state_update.argtypes
         _lib = L
     return _lib
 
@@ -141,8 +145,10 @@ def scan_workspace_bytes(batch, seqlen, dim, dstate, dtype=torch.bfloat16) -> in
 
 
 def ssm_scan_fwd(x, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True, h0=None,
-                 y=None, h_last=None, workspace=None, return_last_state=True, stream=None):
-    """Selective scan through ssm_scan_fwd of libssmscan.so.
+                 y=None, h_last=None, workspace=None, return_last_state=True, stream=None,
+                 zoh=False):
+    """Selective scan through ssm_scan_fwd of libssmscan.so (ssm_scan_fwd_zoh
+    with ``zoh=True``: the exact zero-order-hold input term).
 
     x, delta, z: (batch, L, dim); B, C: (batch, L, N) -- all float32 or all
     bfloat16. A: (dim, N), D and delta_bias: (dim,), h0: (batch, dim, N),
@@ -175,12 +181,12 @@ def ssm_scan_fwd(x, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=Tr
         if workspace is None:
             workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
         pws = _ptr(workspace, "workspace", None, None, dev)
-        rc = lib().ssm_scan_fwd(batch, L, dim, N, io, args_io[0], args_io[1], pA, pB, pC, pD, pz,
-                                pbias, 1 if softplus else 0, ph0, py, ph, pws,
-                                workspace.numel() * workspace.element_size(),
-                                _stream_ptr(stream, dev))
+        fn = lib().ssm_scan_fwd_zoh if zoh else lib().ssm_scan_fwd
+        rc = fn(batch, L, dim, N, io, args_io[0], args_io[1], pA, pB, pC, pD, pz,
+                pbias, 1 if softplus else 0, ph0, py, ph, pws,
+                workspace.numel() * workspace.element_size(), _stream_ptr(stream, dev))
     if rc != 0:
-        raise SsmError(rc, "ssm_scan_fwd")
+        raise SsmError(rc, "ssm_scan_fwd_zoh" if zoh else "ssm_scan_fwd")
     return y, h_last
 
 
@@ -354,9 +360,10 @@ def ssm_scan_status(workspace, batch, seqlen, dim, dstate, dtype=torch.bfloat16,
 
 
 def ssm_state_update(state, x, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
-                     y=None, stream=None):
-    """One decode step through ssm_state_update of libssmscan.so; updates the
-    float32 state (batch, dim, N) in place and returns y (batch, dim)."""
+                     y=None, stream=None, zoh=False):
+    """One decode step through ssm_state_update of libssmscan.so
+    (ssm_state_update_zoh with ``zoh=True``); updates the float32 state
+    (batch, dim, N) in place and returns y (batch, dim)."""
     if state.dim() != 3:
         raise ValueError("state must be (batch, dim, dstate)")
     batch, dim, N = state.shape
@@ -376,8 +383,9 @@ def ssm_state_update(state, x, delta, A, B, C, D=None, z=None, delta_bias=None, 
         y = torch.empty(bd, dtype=x.dtype, device=dev)
     py = _ptr(y, "y", x.dtype, bd, dev)
     with torch.cuda.device(dev):
-        rc = lib().ssm_state_update(batch, dim, N, io, ps, px, pdl, pA, pB, pC, pD, pz, pbias,
-                                    1 if softplus else 0, py, _stream_ptr(stream, dev))
+        fn = lib().ssm_state_update_zoh if zoh else lib().ssm_state_update
+        rc = fn(batch, dim, N, io, ps, px, pdl, pA, pB, pC, pD, pz, pbias,
+                1 if softplus else 0, py, _stream_ptr(stream, dev))
     if rc != 0:
-        raise SsmError(rc, "ssm_state_update")
+        raise SsmError(rc, "ssm_state_update_zoh" if zoh else "ssm_state_update")
     return y

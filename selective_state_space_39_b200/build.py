@@ -34,14 +34,34 @@ def up_to_date() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile every source to an object in parallel, then link the shared
+    library (same flags as one nvcc call over all sources)."""
     if not force and up_to_date():
         return LIB_PATH
-    tmp = LIB_PATH + ".tmp.%d" % os.getpid()
-    cmd = [nvcc()] + ARCH + FLAGS + ["-o", tmp] + SOURCES
+    from concurrent.futures import ThreadPoolExecutor
+    obj_dir = os.path.join(HERE, "_build")
+    os.makedirs(obj_dir, exist_ok=True)
+    compile_flags = [f for f in FLAGS if f != "-shared"]
+    tag = "%d" % os.getpid()
+    objs = [os.path.join(obj_dir, os.path.basename(src) + "." + tag + ".o") for src in SOURCES]
+
+    def compile_one(pair):
+        src, obj = pair
+        cmd = [nvcc()] + ARCH + compile_flags + ["-c", src, "-o", obj]
+        if verbose:
+            print(" ".join(cmd), file=sys.stderr)
+        subprocess.run(cmd, check=True)
+
+    with ThreadPoolExecutor(max_workers=len(SOURCES)) as ex:
+        list(ex.map(compile_one, zip(SOURCES, objs)))
+    tmp = LIB_PATH + ".tmp." + tag
+    cmd = [nvcc()] + ARCH + ["-shared", "-Xcompiler", "-fPIC", "-o", tmp] + objs
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.run(cmd, check=True)
     os.replace(tmp, LIB_PATH)
+    for o in objs:
+        os.remove(o)
     return LIB_PATH
 
 

@@ -273,11 +273,37 @@ size_t ssm_scan_workspace_bytes(int64_t batch, int64_t seqlen, int64_t dim, int6
   return make_plan(d).bytes;
 }
 
+static int scan_fwd_impl(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
+                         int io_dtype, const void* x, const void* delta, const float* A,
+                         const void* B, const void* C, const float* D, const void* z,
+                         const float* delta_bias, int softplus, const float* h0, void* y,
+                         float* h_last, void* workspace, size_t workspace_bytes, void* stream,
+                         bool zoh);
+
 int ssm_scan_fwd(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate, int io_dtype,
                  const void* x, const void* delta, const float* A, const void* B,
                  const void* C, const float* D, const void* z, const float* delta_bias,
                  int softplus, const float* h0, void* y, float* h_last, void* workspace,
                  size_t workspace_bytes, void* stream) {
+  return scan_fwd_impl(batch, seqlen, dim, dstate, io_dtype, x, delta, A, B, C, D, z, delta_bias,
+                       softplus, h0, y, h_last, workspace, workspace_bytes, stream, false);
+}
+
+int ssm_scan_fwd_zoh(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate, int io_dtype,
+                     const void* x, const void* delta, const float* A, const void* B,
+                     const void* C, const float* D, const void* z, const float* delta_bias,
+                     int softplus, const float* h0, void* y, float* h_last, void* workspace,
+                     size_t workspace_bytes, void* stream) {
+  return scan_fwd_impl(batch, seqlen, dim, dstate, io_dtype, x, delta, A, B, C, D, z, delta_bias,
+                       softplus, h0, y, h_last, workspace, workspace_bytes, stream, true);
+}
+
+static int scan_fwd_impl(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
+                         int io_dtype, const void* x, const void* delta, const float* A,
+                         const void* B, const void* C, const float* D, const void* z,
+                         const float* delta_bias, int softplus, const float* h0, void* y,
+                         float* h_last, void* workspace, size_t workspace_bytes, void* stream,
+                         bool zoh) {
   const Dims d{batch, seqlen, dim, dstate, io_dtype};
   int st = dims_status(d);
   if (st != SSM_OK) return st;
@@ -336,7 +362,7 @@ int ssm_scan_fwd(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate, int
     if (!ok) return SSM_ERR_CUDA;
   }
   st = cuda_status(launch_scan(pl, p, use_tma ? &maps : nullptr, use_tma, (int)dstate,
-                               io_dtype == SSM_DTYPE_BF16, static_cast<cudaStream_t>(stream)),
+                               io_dtype == SSM_DTYPE_BF16, zoh, static_cast<cudaStream_t>(stream)),
                    use_tma ? "scan launch (TMA path)" : "scan launch (plain-load path)");
   return st;
 }
@@ -365,10 +391,33 @@ int ssm_scan_status(const void* workspace, size_t workspace_bytes, int64_t batch
   return SSM_OK;
 }
 
+static int state_update_impl(int64_t batch, int64_t dim, int64_t dstate, int io_dtype,
+                             float* state, const void* x, const void* delta, const float* A,
+                             const void* B, const void* C, const float* D, const void* z,
+                             const float* delta_bias, int softplus, void* y, void* stream,
+                             bool zoh);
+
 int ssm_state_update(int64_t batch, int64_t dim, int64_t dstate, int io_dtype, float* state,
                      const void* x, const void* delta, const float* A, const void* B,
                      const void* C, const float* D, const void* z, const float* delta_bias,
                      int softplus, void* y, void* stream) {
+  return state_update_impl(batch, dim, dstate, io_dtype, state, x, delta, A, B, C, D, z,
+                           delta_bias, softplus, y, stream, false);
+}
+
+int ssm_state_update_zoh(int64_t batch, int64_t dim, int64_t dstate, int io_dtype, float* state,
+                         const void* x, const void* delta, const float* A, const void* B,
+                         const void* C, const float* D, const void* z, const float* delta_bias,
+                         int softplus, void* y, void* stream) {
+  return state_update_impl(batch, dim, dstate, io_dtype, state, x, delta, A, B, C, D, z,
+                           delta_bias, softplus, y, stream, true);
+}
+
+static int state_update_impl(int64_t batch, int64_t dim, int64_t dstate, int io_dtype,
+                             float* state, const void* x, const void* delta, const float* A,
+                             const void* B, const void* C, const float* D, const void* z,
+                             const float* delta_bias, int softplus, void* y, void* stream,
+                             bool zoh) {
   const Dims d{batch, 1, dim, dstate, io_dtype};
   int st = dims_status(d);
   if (st != SSM_OK) return st;
@@ -399,7 +448,7 @@ int ssm_state_update(int64_t batch, int64_t dim, int64_t dstate, int io_dtype, f
   p.state = state;
   p.x = x; p.delta = delta; p.z = z; p.B = B; p.C = C;
   p.A = A; p.D = D; p.bias = delta_bias; p.y = y;
-  return cuda_status(launch_decode(p, (int)dstate, io_dtype == SSM_DTYPE_BF16,
+  return cuda_status(launch_decode(p, (int)dstate, io_dtype == SSM_DTYPE_BF16, zoh,
                                    static_cast<cudaStream_t>(stream)),
                      "decode launch");
 }

@@ -88,9 +88,11 @@ struct DecodeParams {
 };
 
 // Kernel launchers (ssm_scan_kernels.cu). Return a cudaError_t.
+// zoh: the exact zero-order-hold input term instead of Delta B.
 cudaError_t launch_scan(const ScanPlan& plan, const ScanParams& p, const ScanMaps* maps,
-                        bool use_tma, int dstate, bool bf16, cudaStream_t stream);
-cudaError_t launch_decode(const DecodeParams& p, int dstate, bool bf16, cudaStream_t stream);
+                        bool use_tma, int dstate, bool bf16, bool zoh, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeParams& p, int dstate, bool bf16, bool zoh,
+                          cudaStream_t stream);
 bool scan_dstate_supported(int dstate);
 // Resident CTAs per SM of the main-pass kernel on the current device (0 if
 // the query fails).

@@ -106,11 +106,22 @@ struct StepScalars {
   float rr;      // r^2, the step of the alpha chain over state pairs
   float rho;     // s_{t-1} / s_t (generic A)
   float q;       // Delta (precise) or Delta log2(e) (fast)
-  float s;       // the state scale s_t ~ Delta x
+  float s;       // the state scale s_t ~ Delta x (ZOH: x / A_0, or x)
+  float m0, m1;  // ZOH, structured A: exp(Delta A_n) - 1 for states 0 and 1
+  float e2;      // ZOH, structured A: the step of that chain over state pairs
 };
 
 // Step size, decay base and state scale for one channel and step.
-template <bool kFast>
+//
+// Input term (kZoh = false, the simplified deltaB of the selective_scan
+// listing): Delta x B_n, with s = Delta x (fast: times log2 e, matched by B
+// pre-scaled by ln 2). Exact zero-order hold (kZoh, §2.2 B-bar):
+// x B_n (exp(Delta A_n) - 1) / A_n. With structured A (kS) that is
+// s B_n / (n+1) m_n with s = x / A_0 and m_n = r^(n+1) - 1 (B
+// pre-scaled by 1/(n+1)); m_n is built without cancellation from
+// m_0 = expm1(Delta A_0): m_(n+2) = m_n r^2 + m_0 (1 + r), every term of one
+// sign. Generic A under ZOH uses s = x and forms each state's factor itself.
+template <bool kFast, bool kZoh = false, bool kS = true>
 __device__ __forceinline__ StepScalars step_scalars(float xv, float dv, const Chan& ch,
                                                     int softplus, float& s_prev) {
   StepScalars o;
@@ -124,10 +135,19 @@ __device__ __forceinline__ StepScalars step_scalars(float xv, float dv, const Ch
     q = softplus ? (v > kSoftplusCut ? v : log1pf(expf(v))) : v;
     r = expf(q * ch.A0);
   }
-  // s = Delta x in the path's units (fast: times log2 e, matched by B
-  // pre-scaled by ln 2), kept away from zero.
-  float s = q * xv;
-  s = s + copysignf(kScaleFloor, s);
+  float s;
+  if constexpr (!kZoh) {
+    s = q * xv;
+  } else if constexpr (kS) {
+    s = kFast ? xv * rcp_approx(ch.A0) : xv / ch.A0;
+    const float em1 = kFast ? r - 1.f : expm1f(q * ch.A0);  // exp(Delta A_0) - 1
+    o.m0 = em1;
+    o.m1 = fmaf(em1, r, em1);
+    o.e2 = em1 * (1.f + r);
+  } else {
+    s = xv;
+  }
+  s = s + copysignf(kScaleFloor, s);  // kept away from zero
   const float rho = kFast ? s_prev * rcp_approx(s) : s_prev / s;
   s_prev = s;
   o.q = q;
@@ -143,7 +163,8 @@ __device__ __forceinline__ StepScalars step_scalars(float xv, float dv, const Ch
 // The scan kernel. kAgg = carry pass (segments 0..nseg-2: end state and
 // sum of Delta, no output); !kAgg = main pass (all segments, y and h_last).
 // Grid: (dtiles, segments, batch). Block: NT threads, CPT channels each.
-template <typename IOT, int N, int CPT, int NT, int T, int STAGES, bool kAgg, bool kTma>
+template <typename IOT, int N, int CPT, int NT, int T, int STAGES, bool kAgg, bool kTma,
+          bool kZoh>
 __global__ void __launch_bounds__(NT, SSM_MIN_CTAS) scan_kernel(const ScanParams p,
                                                   const __grid_constant__ ScanMaps maps) {
   using IO = Io<IOT>;
@@ -218,6 +239,8 @@ __global__ void __launch_bounds__(NT, SSM_MIN_CTAS) scan_kernel(const ScanParams
       ch[c].A0 = Ar[0];
 #pragma unroll
       for (int n = 1; n < N; ++n) structured = structured && (Ar[n] == (float)(n + 1) * Ar[0]);
+      // the ZOH chain divides by A_0: A = 0 takes the per-state path
+      if constexpr (kZoh) structured = structured && Ar[0] != 0.f;
       const float bias = p.bias ? p.bias[d] : 0.f;
       ch[c].bias = kFast ? bias * kLog2e : bias;
       ch[c].Dd = p.D ? p.D[d] : 0.f;
@@ -397,11 +420,26 @@ __global__ void __launch_bounds__(NT, SSM_MIN_CTAS) scan_kernel(const ScanParams
         // alpha_n = rho r^(n+1), two states at a time: (a0, a1) * (r^2)^k
         float2 a = make_float2(sc[c].a0, sc[c].a1);
         const float2 rr = make_float2(sc[c].rr, sc[c].rr);
+        if constexpr (kZoh) {
+          // input B_n / (n+1) m_n, m pairs stepped by m <- m r^2 + m_0 (1 + r)
+          float2 m = make_float2(sc[c].m0, sc[c].m1);
+          const float2 e2 = make_float2(sc[c].e2, sc[c].e2);
 #pragma unroll
-        for (int k = 0; k < NP; ++k) {
-          g[c][k] = fma2(a, g[c][k], B2[k]);
-          if (k + 1 < NP) a = mul2(a, rr);
-          if constexpr (!kAgg) acc[c] = fma2(C2[k], g[c][k], acc[c]);
+          for (int k = 0; k < NP; ++k) {
+            g[c][k] = fma2(a, g[c][k], mul2(B2[k], m));
+            if (k + 1 < NP) {
+              a = mul2(a, rr);
+              m = fma2(m, rr, e2);
+            }
+            if constexpr (!kAgg) acc[c] = fma2(C2[k], g[c][k], acc[c]);
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < NP; ++k) {
+            g[c][k] = fma2(a, g[c][k], B2[k]);
+            if (k + 1 < NP) a = mul2(a, rr);
+            if constexpr (!kAgg) acc[c] = fma2(C2[k], g[c][k], acc[c]);
+          }
         }
 #endif
       }
@@ -416,14 +454,22 @@ __global__ void __launch_bounds__(NT, SSM_MIN_CTAS) scan_kernel(const ScanParams
 #pragma unroll
         for (int k = 0; k < NP; ++k) {
           float2 a;
-          if constexpr (kFast) {
-            a = make_float2(rho * ex2_approx(q * __ldg(Ar + 2 * k)),
-                            rho * ex2_approx(q * __ldg(Ar + 2 * k + 1)));
+          const float A_lo = __ldg(Ar + 2 * k), A_hi = __ldg(Ar + 2 * k + 1);
+          const float e_lo = kFast ? ex2_approx(q * A_lo) : expf(q * A_lo);
+          const float e_hi = kFast ? ex2_approx(q * A_hi) : expf(q * A_hi);
+          a = make_float2(rho * e_lo, rho * e_hi);
+          if constexpr (kZoh) {
+            // input B_n (exp(Delta A_n) - 1) / A_n (Delta where A_n = 0), s = x
+            const float dt = kFast ? q * kLn2 : q;
+            auto coef = [&](float An, float e) {
+              if (An == 0.f) return dt;
+              return kFast ? (e - 1.f) * rcp_approx(An) : expm1f(dt * An) / An;
+            };
+            const float2 in2 = make_float2(B2[k].x * coef(A_lo, e_lo), B2[k].y * coef(A_hi, e_hi));
+            g[c][k] = fma2(a, g[c][k], in2);
           } else {
-            a = make_float2(rho * expf(q * __ldg(Ar + 2 * k)),
-                            rho * expf(q * __ldg(Ar + 2 * k + 1)));
+            g[c][k] = fma2(a, g[c][k], B2[k]);
           }
-          g[c][k] = fma2(a, g[c][k], B2[k]);
           if constexpr (!kAgg) acc[c] = fma2(C2[k], g[c][k], acc[c]);
         }
       }
@@ -512,8 +558,11 @@ __global__ void __launch_bounds__(NT, SSM_MIN_CTAS) scan_kernel(const ScanParams
         const IOT* sc = reinterpret_cast<const IOT*>(st + L::kOffC);
         float* fb = bcf + (buf * 2 + 0) * T * N;
         float* fc = bcf + (buf * 2 + 1) * T * N;
-        const float bscale = kFast ? kLn2 : 1.f;
         for (int i = tid; i < T * N; i += NT) {
+          // Delta B (fast: ln 2, see step_scalars); ZOH: 1/(n+1) (structured) or 1
+          float bscale;
+          if constexpr (kZoh) bscale = cta_structured ? 1.f / (float)(i % N + 1) : 1.f;
+          else bscale = kFast ? kLn2 : 1.f;
           fb[i] = IO::load(sb + i) * bscale;
           if (!kAgg) fc[i] = IO::load(sc + i);
         }
@@ -540,7 +589,8 @@ __global__ void __launch_bounds__(NT, SSM_MIN_CTAS) scan_kernel(const ScanParams
         StepScalars sc_next[CPT];
 #pragma unroll
         for (int c = 0; c < CPT; ++c)
-          sc_next[c] = step_scalars<kFast>(in_next.x[c], in_next.d[c], ch[c], softplus, s_prev[c]);
+          sc_next[c] = step_scalars<kFast, kZoh, decltype(kStructTag)::value>(
+              in_next.x[c], in_next.d[c], ch[c], softplus, s_prev[c]);
         float s_last[CPT];
 #pragma unroll(kFull ? kTileUnroll : 1)
         for (int row = 0; row < nst; ++row) {
@@ -556,7 +606,8 @@ __global__ void __launch_bounds__(NT, SSM_MIN_CTAS) scan_kernel(const ScanParams
 #pragma unroll
           for (int c = 0; c < CPT; ++c) {
             float sp = sc[c].s;
-            sc_next[c] = step_scalars<kFast>(in_next.x[c], in_next.d[c], ch[c], softplus, sp);
+            sc_next[c] = step_scalars<kFast, kZoh, decltype(kStructTag)::value>(
+                in_next.x[c], in_next.d[c], ch[c], softplus, sp);
           }
           state_step(kStructTag, in, sc, fb + row * N, fc + row * N, t0 + row);
         }
@@ -617,7 +668,7 @@ __global__ void __launch_bounds__(NT, SSM_MIN_CTAS) scan_kernel(const ScanParams
 // across the LPC lanes by shuffles. Every load of a thread is issued before
 // any arithmetic, so each thread makes a single round trip to memory: the
 // kernel is otherwise bound by the latency of its waves, not by bandwidth.
-template <typename IOT, int N>
+template <typename IOT, int N, bool kZoh>
 __global__ void __launch_bounds__(256) decode_kernel(const DecodeParams p) {
   using IO = Io<IOT>;
   constexpr bool kFast = std::is_same<IOT, uint16_t>::value;
@@ -676,7 +727,15 @@ __global__ void __launch_bounds__(256) decode_kernel(const DecodeParams p) {
 #pragma unroll
   for (int k = 0; k < SPT; ++k) {
     const float e = kFast ? ex2_approx(dtl * a[k]) : expf(dtl * a[k]);
-    h[k] = fmaf(e, h[k], dx * bb[k]);
+    if constexpr (kZoh) {
+      // exact ZOH input: x B_n (exp(Delta A_n) - 1) / A_n (Delta where A_n = 0)
+      const float coef = a[k] == 0.f ? dt
+                         : kFast     ? (e - 1.f) * rcp_approx(a[k])
+                                     : expm1f(dt * a[k]) / a[k];
+      h[k] = fmaf(e, h[k], xv * coef * bb[k]);
+    } else {
+      h[k] = fmaf(e, h[k], dx * bb[k]);
+    }
     acc = fmaf(cv[k], h[k], acc);
   }
 #pragma unroll
@@ -716,7 +775,7 @@ cudaError_t ensure_smem_attr(const void* kernel, int smem) {
   return e;
 }
 
-template <typename IOT, int N, int CPT>
+template <typename IOT, int N, int CPT, bool kZoh>
 cudaError_t launch_scan_t(const ScanPlan& plan, const ScanParams& p, const ScanMaps* maps,
                           bool use_tma, cudaStream_t stream) {
   constexpr int NT = scan_threads(CPT), T = kScanTileSteps, S = kScanStages;
@@ -748,20 +807,20 @@ cudaError_t launch_scan_t(const ScanPlan& plan, const ScanParams& p, const ScanM
   if (use_tma) {
     constexpr int smem = scan_smem_bytes<IOT, N, CPT, NT, T, S>();
     if (plan.nseg > 1) {
-      err = run(scan_kernel<IOT, N, CPT, NT, T, S, true, true>, smem,
+      err = run(scan_kernel<IOT, N, CPT, NT, T, S, true, true, kZoh>, smem,
                 dim3(plan.dtiles, plan.nseg - 1, p.batch));
       if (err != cudaSuccess) return err;
     }
-    return run(scan_kernel<IOT, N, CPT, NT, T, S, false, true>, smem,
+    return run(scan_kernel<IOT, N, CPT, NT, T, S, false, true, kZoh>, smem,
                dim3(plan.dtiles, plan.nseg, p.batch), plan.nseg > 1);
   }
   constexpr int smem = scan_smem_bytes<IOT, N, CPT, NT, T, 1>();
   if (plan.nseg > 1) {
-    err = run(scan_kernel<IOT, N, CPT, NT, T, 1, true, false>, smem,
+    err = run(scan_kernel<IOT, N, CPT, NT, T, 1, true, false, kZoh>, smem,
               dim3(plan.dtiles, plan.nseg - 1, p.batch));
     if (err != cudaSuccess) return err;
   }
-  return run(scan_kernel<IOT, N, CPT, NT, T, 1, false, false>, smem,
+  return run(scan_kernel<IOT, N, CPT, NT, T, 1, false, false, kZoh>, smem,
              dim3(plan.dtiles, plan.nseg, p.batch), plan.nseg > 1);
 }
 
@@ -769,7 +828,7 @@ template <typename IOT, int N, int CPT>
 int ctas_per_sm_t() {
   constexpr int NT = scan_threads(CPT), T = kScanTileSteps, S = kScanStages;
   int n = 0;
-  auto kernel = scan_kernel<IOT, N, CPT, NT, T, S, false, true>;
+  auto kernel = scan_kernel<IOT, N, CPT, NT, T, S, false, true, false>;
   constexpr int smem = scan_smem_bytes<IOT, N, CPT, NT, T, S>();
   if (ensure_smem_attr(reinterpret_cast<const void*>(kernel), smem) != cudaSuccess ||
       cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, NT, smem) != cudaSuccess) {
@@ -792,21 +851,21 @@ int ctas_per_sm_io(int dstate) {
   }
 }
 
-template <typename IOT>
+template <typename IOT, bool kZoh>
 cudaError_t launch_scan_io(const ScanPlan& plan, const ScanParams& p, const ScanMaps* maps,
                            bool use_tma, int dstate, cudaStream_t stream) {
   switch (dstate) {
-    case 2: return launch_scan_t<IOT, 2, 2>(plan, p, maps, use_tma, stream);
-    case 4: return launch_scan_t<IOT, 4, 2>(plan, p, maps, use_tma, stream);
-    case 8: return launch_scan_t<IOT, 8, 2>(plan, p, maps, use_tma, stream);
-    case 16: return launch_scan_t<IOT, 16, SSM_CPT16>(plan, p, maps, use_tma, stream);
-    case 32: return launch_scan_t<IOT, 32, 1>(plan, p, maps, use_tma, stream);
-    case 64: return launch_scan_t<IOT, 64, 1>(plan, p, maps, use_tma, stream);
+    case 2: return launch_scan_t<IOT, 2, 2, kZoh>(plan, p, maps, use_tma, stream);
+    case 4: return launch_scan_t<IOT, 4, 2, kZoh>(plan, p, maps, use_tma, stream);
+    case 8: return launch_scan_t<IOT, 8, 2, kZoh>(plan, p, maps, use_tma, stream);
+    case 16: return launch_scan_t<IOT, 16, SSM_CPT16, kZoh>(plan, p, maps, use_tma, stream);
+    case 32: return launch_scan_t<IOT, 32, 1, kZoh>(plan, p, maps, use_tma, stream);
+    case 64: return launch_scan_t<IOT, 64, 1, kZoh>(plan, p, maps, use_tma, stream);
     default: return cudaErrorInvalidValue;
   }
 }
 
-template <typename IOT>
+template <typename IOT, bool kZoh>
 cudaError_t launch_decode_io(const DecodeParams& p, int dstate, cudaStream_t stream) {
   const size_t chans = (size_t)p.batch * p.dim;
   auto go = [&](auto kernel, int lpc) -> cudaError_t {
@@ -816,12 +875,12 @@ cudaError_t launch_decode_io(const DecodeParams& p, int dstate, cudaStream_t str
     return cudaGetLastError();
   };
   switch (dstate) {
-    case 2: return go(decode_kernel<IOT, 2>, 1);
-    case 4: return go(decode_kernel<IOT, 4>, 1);
-    case 8: return go(decode_kernel<IOT, 8>, 2);
-    case 16: return go(decode_kernel<IOT, 16>, 4);
-    case 32: return go(decode_kernel<IOT, 32>, 8);
-    case 64: return go(decode_kernel<IOT, 64>, 16);
+    case 2: return go(decode_kernel<IOT, 2, kZoh>, 1);
+    case 4: return go(decode_kernel<IOT, 4, kZoh>, 1);
+    case 8: return go(decode_kernel<IOT, 8, kZoh>, 2);
+    case 16: return go(decode_kernel<IOT, 16, kZoh>, 4);
+    case 32: return go(decode_kernel<IOT, 32, kZoh>, 8);
+    case 64: return go(decode_kernel<IOT, 64, kZoh>, 16);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -840,14 +899,21 @@ int scan_ctas_per_sm(int dstate, bool bf16) {
 }
 
 cudaError_t launch_scan(const ScanPlan& plan, const ScanParams& p, const ScanMaps* maps,
-                        bool use_tma, int dstate, bool bf16, cudaStream_t stream) {
-  return bf16 ? launch_scan_io<uint16_t>(plan, p, maps, use_tma, dstate, stream)
-              : launch_scan_io<float>(plan, p, maps, use_tma, dstate, stream);
+                        bool use_tma, int dstate, bool bf16, bool zoh, cudaStream_t stream) {
+  if (zoh)
+    return bf16 ? launch_scan_io<uint16_t, true>(plan, p, maps, use_tma, dstate, stream)
+                : launch_scan_io<float, true>(plan, p, maps, use_tma, dstate, stream);
+  return bf16 ? launch_scan_io<uint16_t, false>(plan, p, maps, use_tma, dstate, stream)
+              : launch_scan_io<float, false>(plan, p, maps, use_tma, dstate, stream);
 }
 
-cudaError_t launch_decode(const DecodeParams& p, int dstate, bool bf16, cudaStream_t stream) {
-  return bf16 ? launch_decode_io<uint16_t>(p, dstate, stream)
-              : launch_decode_io<float>(p, dstate, stream);
+cudaError_t launch_decode(const DecodeParams& p, int dstate, bool bf16, bool zoh,
+                          cudaStream_t stream) {
+  if (zoh)
+    return bf16 ? launch_decode_io<uint16_t, true>(p, dstate, stream)
+                : launch_decode_io<float, true>(p, dstate, stream);
+  return bf16 ? launch_decode_io<uint16_t, false>(p, dstate, stream)
+              : launch_decode_io<float, false>(p, dstate, stream);
 }
 
 }  // namespace ssm
