@@ -116,7 +116,8 @@ int ssm_scan_plan(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate, in
  *                    bytes (may be NULL when that is 0); contents on entry
  *                    are ignored; it must not be used by concurrent calls.
  *
- * y must not overlap any input. h_last may alias h0 (in-place resume).
+ * y must not overlap any input. y may be NULL when h_last is given (only the
+ * final state is wanted). h_last may alias h0 (in-place resume).
  * seqlen == 0 writes only h_last (= h0 or zero). batch or dim == 0 is a
  * no-op. Returns SSM_OK or SSM_ERR_*.
  */
@@ -279,6 +280,36 @@ int ssm_state_update_zoh(int64_t batch, int64_t dim, int64_t dstate, int io_dtyp
                          const void* x, const void* delta, const float* A, const void* B,
                          const void* C, const float* D, const void* z, const float* delta_bias,
                          int softplus, void* y, void* stream);
+
+/*
+ * Splitting one sequence across ranks (devices). A chunk of steps acts on the
+ * state as the affine map h -> P h + e with P_n = exp(A[d,n] * sum_t Delta_t)
+ * and e the chunk's end state from a zero start (§2.2 recurrence; the maps
+ * compose associatively, which is the parallel scan of the allinfo.ai.kr
+ * page). With the sequence cut into chunks 0..R-1 in order, rank r:
+ *   1. ssm_scan_fwd(h0 = NULL, y = NULL, h_last = e_r) on its chunk, and
+ *      ssm_delta_sum(...) -> S_r;
+ *   2. gathers (e, S) of every rank (e.g. an all-gather);
+ *   3. ssm_compose_carries(r, ...) -> its true entering state;
+ *   4. ssm_scan_fwd(h0 = that state) on its chunk -> its y, and on the last
+ *      rank the sequence's h_last.
+ * (ssm_scan_fwd accepts y = NULL when h_last is given: state only.)
+ */
+
+/* ssm_delta_sum -- dsum[b,d] = sum_t Delta[b,t,d], Delta = softplus(delta +
+ * delta_bias) (or delta + delta_bias), fp32 (batch, dim). delta is
+ * (batch, seqlen, dim) io_dtype; delta_bias (dim) fp32, nullable. */
+int ssm_delta_sum(int64_t batch, int64_t seqlen, int64_t dim, int io_dtype, const void* delta,
+                  const float* delta_bias, int softplus, float* dsum, void* stream);
+
+/* ssm_compose_carries -- h_in = the state entering chunk `rank`: starting from
+ * h0 (nullable: zero), apply h <- exp(A[d,n] dsum_all[r,b,d]) h + hend_all[r,b,d,n]
+ * for r = 0 .. rank-1. A (dim, dstate); h0, h_in (batch, dim, dstate);
+ * hend_all (ranks, batch, dim, dstate); dsum_all (ranks, batch, dim); fp32.
+ * h_in must not overlap an input. */
+int ssm_compose_carries(int64_t rank, int64_t batch, int64_t dim, int64_t dstate, const float* A,
+                        const float* h0, const float* hend_all, const float* dsum_all,
+                        float* h_in, void* stream);
 
 /*
  * ssm_scan_status -- synchronise `stream`, then report whether every CTA of

@@ -94,6 +94,11 @@ def lib() -> ctypes.CDLL:
         L.ssm_state_update.restype = ctypes.c_int
         L.ssm_state_update.argtypes = [_I64, _I64, _I64, ctypes.c_int, _VP, _VP, _VP, _VP, _VP,
                                        _VP, _VP, _VP, _VP, ctypes.c_int, _VP, _VP]
+        L.ssm_delta_sum.restype = ctypes.c_int
+        L.ssm_delta_sum.argtypes = [_I64, _I64, _I64, ctypes.c_int, _VP, _VP, ctypes.c_int, _VP,
+                                    _VP]
+        L.ssm_compose_carries.restype = ctypes.c_int
+        L.ssm_compose_carries.argtypes = [_I64, _I64, _I64, _I64, _VP, _VP, _VP, _VP, _VP, _VP]
         L.ssm_state_update_zoh.restype = ctypes.c_int
         L.ssm_state_update_zoh.argtypes = L.ssm_state_update.argtypes
         _lib = L
@@ -146,13 +151,14 @@ def scan_workspace_bytes(batch, seqlen, dim, dstate, dtype=torch.bfloat16) -> in
 
 def ssm_scan_fwd(x, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True, h0=None,
                  y=None, h_last=None, workspace=None, return_last_state=True, stream=None,
-                 zoh=False):
+                 zoh=False, return_y=True):
     """Selective scan through ssm_scan_fwd of libssmscan.so (ssm_scan_fwd_zoh
     with ``zoh=True``: the exact zero-order-hold input term).
 
     x, delta, z: (batch, L, dim); B, C: (batch, L, N) -- all float32 or all
     bfloat16. A: (dim, N), D and delta_bias: (dim,), h0: (batch, dim, N),
-    float32. Returns (y, h_last); h_last is None when not requested."""
+    float32. Returns (y, h_last); h_last is None when not requested, y is None
+    with ``return_y=False`` (the final state only: no y is written)."""
     if x.dim() != 3:
         raise ValueError("x must be (batch, seqlen, dim)")
     batch, L, dim = x.shape
@@ -170,10 +176,10 @@ def ssm_scan_fwd(x, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=Tr
     pz = _ptr(z, "z", x.dtype, bld, dev)
     pbias = _ptr(delta_bias, "delta_bias", torch.float32, (dim,), dev)
     ph0 = _ptr(h0, "h0", torch.float32, (batch, dim, N), dev)
-    if y is None:
+    if y is None and return_y:
         y = torch.empty(bld, dtype=x.dtype, device=dev)
     py = _ptr(y, "y", x.dtype, bld, dev)
-    if h_last is None and return_last_state:
+    if h_last is None and (return_last_state or not return_y):
         h_last = torch.empty((batch, dim, N), dtype=torch.float32, device=dev)
     ph = _ptr(h_last, "h_last", torch.float32, (batch, dim, N), dev)
     with torch.cuda.device(dev):
@@ -304,6 +310,50 @@ def ssm_conv1d_silu_bwd(x, w, dout, bias=None, silu=True, workspace=None, stream
     if rc != 0:
         raise SsmError(rc, "ssm_conv1d_silu_bwd", with_detail=True)
     return g
+
+
+def ssm_delta_sum(delta, delta_bias=None, softplus=True, out=None, stream=None):
+    """dsum (batch, dim) float32 = sum over the sequence of Delta =
+    softplus(delta + delta_bias), through ssm_delta_sum of libssmscan.so."""
+    if delta.dim() != 3:
+        raise ValueError("delta must be (batch, seqlen, dim)")
+    batch, L, dim = delta.shape
+    dev = delta.device
+    pd = _ptr(delta, "delta", delta.dtype, (batch, L, dim))
+    pb = _ptr(delta_bias, "delta_bias", torch.float32, (dim,), dev)
+    if out is None:
+        out = torch.empty((batch, dim), dtype=torch.float32, device=dev)
+    po = _ptr(out, "out", torch.float32, (batch, dim), dev)
+    with torch.cuda.device(dev):
+        rc = lib().ssm_delta_sum(batch, L, dim, _io_code(delta.dtype), pd, pb, 1 if softplus else 0,
+                                 po, _stream_ptr(stream, dev))
+    if rc != 0:
+        raise SsmError(rc, "ssm_delta_sum")
+    return out
+
+
+def ssm_compose_carries(rank, A, hend_all, dsum_all, h0=None, out=None, stream=None):
+    """The state entering chunk `rank` of a sequence cut into chunks: h0 (or
+    zero) carried through chunks 0..rank-1, each given by its end state from
+    zero (hend_all[r], (batch, dim, N)) and its sum of Delta (dsum_all[r],
+    (batch, dim)), through ssm_compose_carries of libssmscan.so."""
+    R, batch, dim, N = hend_all.shape
+    dev = hend_all.device
+    pA = _ptr(A, "A", torch.float32, (dim, N), dev)
+    ph = _ptr(hend_all, "hend_all", torch.float32, (R, batch, dim, N), dev)
+    pd = _ptr(dsum_all, "dsum_all", torch.float32, (R, batch, dim), dev)
+    p0 = _ptr(h0, "h0", torch.float32, (batch, dim, N), dev)
+    if not 0 <= rank <= R:
+        raise ValueError("rank out of range")
+    if out is None:
+        out = torch.empty((batch, dim, N), dtype=torch.float32, device=dev)
+    po = _ptr(out, "out", torch.float32, (batch, dim, N), dev)
+    with torch.cuda.device(dev):
+        rc = lib().ssm_compose_carries(rank, batch, dim, N, pA, p0, ph, pd, po,
+                                       _stream_ptr(stream, dev))
+    if rc != 0:
+        raise SsmError(rc, "ssm_compose_carries")
+    return out
 
 
 def ssm_scan_fwd_noalloc(x, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,

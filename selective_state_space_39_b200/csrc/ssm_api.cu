@@ -12,6 +12,7 @@
 #include "../../include/ssm_scan.h"
 #include "ssm_bwd_internal.h"
 #include "ssm_conv_internal.h"
+#include "ssm_seqpar_internal.h"
 #include "ssm_internal.h"
 
 namespace ssm {
@@ -312,7 +313,8 @@ static int scan_fwd_impl(int64_t batch, int64_t seqlen, int64_t dim, int64_t dst
   const size_t n_bld = (size_t)batch * seqlen * dim, n_bln = (size_t)batch * seqlen * dstate;
   // required pointers and element alignment
   if (!A) return SSM_ERR_INVALID_ARG;
-  if (seqlen > 0 && (!x || !delta || !B || !C || !y)) return SSM_ERR_INVALID_ARG;
+  // y may be NULL when h_last is wanted alone (the state after the sequence)
+  if (seqlen > 0 && (!x || !delta || !B || !C || (!y && !h_last))) return SSM_ERR_INVALID_ARG;
   const void* io_ptrs[] = {x, delta, B, C, z, y};
   for (const void* p : io_ptrs)
     if (p && !aligned(p, es)) return SSM_ERR_INVALID_ARG;
@@ -664,6 +666,59 @@ int ssm_conv1d_silu_bwd(int64_t batch, int64_t seqlen, int64_t dim, int64_t widt
   return cuda_status(launch_conv(p, io_dtype == SSM_DTYPE_BF16,
                                  conv_vec(dim, io_dtype, {x, dout, dx}), true, s),
                      "conv1d backward launch");
+}
+
+// ---- one sequence split across ranks ----------------------------------------
+
+int ssm_delta_sum(int64_t batch, int64_t seqlen, int64_t dim, int io_dtype, const void* delta,
+                  const float* delta_bias, int softplus, float* dsum, void* stream) {
+  if (io_dtype != SSM_DTYPE_F32 && io_dtype != SSM_DTYPE_BF16) return SSM_ERR_UNSUPPORTED;
+  if (batch < 0 || seqlen < 0 || dim < 0) return SSM_ERR_INVALID_ARG;
+  if (batch == 0 || dim == 0) return SSM_OK;
+  if (!dsum || (seqlen > 0 && !delta)) return SSM_ERR_INVALID_ARG;
+  const size_t es = io_bytes(io_dtype);
+  if ((delta && !aligned(delta, es)) || !aligned(dsum, 4) || (delta_bias && !aligned(delta_bias, 4)))
+    return SSM_ERR_INVALID_ARG;
+  if (overlap(dsum, (size_t)batch * dim * 4, delta, (size_t)batch * seqlen * dim * es))
+    return SSM_ERR_INVALID_ARG;
+  SeqParParams p{};
+  p.batch = (int)batch;
+  p.seqlen = (int)seqlen;
+  p.dim = (int)dim;
+  p.softplus = softplus ? 1 : 0;
+  p.delta = delta;
+  p.bias = delta_bias;
+  p.dsum = dsum;
+  return cuda_status(launch_delta_sum(p, io_dtype == SSM_DTYPE_BF16,
+                                      static_cast<cudaStream_t>(stream)),
+                     "delta-sum launch");
+}
+
+int ssm_compose_carries(int64_t rank, int64_t batch, int64_t dim, int64_t dstate, const float* A,
+                        const float* h0, const float* hend_all, const float* dsum_all,
+                        float* h_in, void* stream) {
+  if (rank < 0 || batch < 0 || dim < 0 || dstate <= 0) return SSM_ERR_INVALID_ARG;
+  if (batch == 0 || dim == 0) return SSM_OK;
+  if (!A || !h_in || (rank > 0 && (!hend_all || !dsum_all))) return SSM_ERR_INVALID_ARG;
+  const void* f[] = {A, h0, hend_all, dsum_all, h_in};
+  for (const void* q : f)
+    if (q && !aligned(q, 4)) return SSM_ERR_INVALID_ARG;
+  const size_t state = (size_t)batch * dim * dstate * 4;
+  if (overlap(h_in, state, hend_all, (size_t)rank * state) ||
+      overlap(h_in, state, dsum_all, (size_t)rank * batch * dim * 4) ||
+      overlap(h_in, state, A, (size_t)dim * dstate * 4))
+    return SSM_ERR_INVALID_ARG;
+  SeqParParams p{};
+  p.batch = (int)batch;
+  p.dim = (int)dim;
+  p.dstate = (int)dstate;
+  p.rank = (int)rank;
+  p.A = A;
+  p.h0 = h0;
+  p.hend_all = hend_all;
+  p.dsum_all = dsum_all;
+  p.h_in = h_in;
+  return cuda_status(launch_compose(p, static_cast<cudaStream_t>(stream)), "compose launch");
 }
 
 }  // extern "C"

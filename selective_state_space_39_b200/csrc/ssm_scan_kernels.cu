@@ -490,7 +490,9 @@ __global__ void __launch_bounds__(NT, SSM_MIN_CTAS) scan_kernel(const ScanParams
         yv[c] = yy;
       }
       IOT* yrow = reinterpret_cast<IOT*>(p.y) + ((size_t)b * L_ + t_abs) * dim + d_first;
-      if (vec_store) {
+      if (!p.y) {
+        // state only (y not wanted)
+      } else if (vec_store) {
         if constexpr (CPT == 4)
           IO::store4(yrow, yv[0], yv[1], yv[2], yv[3]);
         else

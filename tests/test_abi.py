@@ -202,6 +202,22 @@ def test_conv_rejects_bad_arguments(L):
     assert need > 0 and bwd(ws=FAKE * 64, ws_bytes=need - 1) == -3
 
 
+@no_gpu_only
+def test_sequence_split_helpers_reject_bad_arguments(L):
+    K = 1 << 16
+    assert L.ssm_delta_sum(2, 32, 64, 1, None, None, 1, FAKE, None) == -1  # delta missing
+    assert L.ssm_delta_sum(2, 32, 64, 1, FAKE, None, 1, FAKE + 64, None) == -1  # overlap
+    assert L.ssm_delta_sum(2, 32, 64, 7, FAKE, None, 1, FAKE + K, None) == -2
+    assert L.ssm_delta_sum(0, 32, 64, 1, FAKE, None, 1, FAKE + K, None) == 0
+    assert L.ssm_compose_carries(2, 2, 64, 16, FAKE, None, None, None, FAKE + K, None) == -1
+    assert L.ssm_compose_carries(-1, 2, 64, 16, FAKE, None, FAKE + 2 * K, FAKE + 3 * K,
+                                 FAKE + K, None) == -1
+    assert L.ssm_compose_carries(1, 2, 64, 16, FAKE, None, FAKE + 2 * K, FAKE + 3 * K,
+                                 FAKE + 2 * K + 64, None) == -1  # h_in overlaps hend_all
+    assert L.ssm_compose_carries(1, 0, 64, 16, FAKE, None, FAKE + 2 * K, FAKE + 3 * K,
+                                 FAKE + K, None) == 0
+
+
 def test_binding_has_no_cpu_path():
     from selective_state_space_39_b200 import ssm_scan_fwd
     x = torch.zeros(1, 4, 8)
