@@ -48,6 +48,9 @@ def parse_args():
                     choices=sorted(gen.SCAN_WORKLOADS) + sorted(gen.DECODE_WORKLOADS))
     ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd"],
                     help="bwd: time ssm_scan_bwd (the gradients) on the same workload")
+    ap.add_argument("--learned-a", action="store_true",
+                    help="A with no (n+1) A[d,0] structure (as after training): the "
+                         "one-exp-per-state path")
     ap.add_argument("--zoh", action="store_true",
                     help="scan with the exact zero-order-hold input term (ssm_scan_fwd_zoh)")
     ap.add_argument("--op", default="scan", choices=["scan", "conv"],
@@ -404,6 +407,8 @@ def backward_bench(args):
     device = torch.device("cuda", 0)
     dtype = torch.bfloat16 if w.io == "bf16" else torch.float32
     inp = gen.workload_inputs(w)
+    if args.learned_a:
+        inp["A"] = gen.a_matrix_learned(w.dim, w.dstate, w.seed)
     grads = gen.make_grad_inputs(w.batch, w.seqlen, w.dim, w.dstate, w.io, w.seed)
 
     def to_dev(a):
@@ -463,6 +468,7 @@ def backward_bench(args):
         "data": "synthetic (seeded Philox4x32-10, Mamba-shaped recipe; dy, dh_last N(0,1))",
         "config": {"workload": w.name, "pass": "backward", "batch": w.batch, "seqlen": w.seqlen,
                    "dim": w.dim, "dstate": w.dstate, "io": w.io,
+                   "A": "learned-like (unstructured)" if args.learned_a else "(n+1) A[d,0]",
                    "l2": "flushed (256 MB write) before every timed step"},
         "roofline": {"bound": "alu", "achieved": round(alu, 1), "peak": round(alu_peak, 1),
                      "unit": "Gop/s", "frac": round(alu / alu_peak, 4), "traffic": None,
@@ -592,6 +598,8 @@ def main():
     # weak scaling: global batch = world * w.batch; this rank's shard
     b0, nb = sdist.batch_shard(world * w.batch, world, rank)
     inp = gen.workload_inputs(w, batch=nb, batch_offset=b0)
+    if args.learned_a:
+        inp["A"] = gen.a_matrix_learned(w.dim, w.dstate, w.seed)
     dtype = torch.bfloat16 if w.io == "bf16" else torch.float32
 
     def to_dev(a):
@@ -647,8 +655,8 @@ def main():
     alu_peak = B200_SMS * FP32_LANES_PER_SM * sm_mhz * 1e6 / 1e9  # Gop/s
     mean_s = statistics.mean(step_ms) * 1e-3
     alu_achieved = alu_ops_per_element(w, args.zoh) * nb * w.seqlen * w.dim / mean_s / 1e9
-    traffic = (measured_traffic(w.name) if (world == 1 or nb == w.batch) and not args.zoh
-               else None)
+    traffic = (measured_traffic(w.name)
+               if (world == 1 or nb == w.batch) and not args.zoh and not args.learned_a else None)
     kernel = "%s: carry pass + main pass (%d launches)" % (
         "ssm_scan_fwd_zoh" if args.zoh else "ssm_scan_fwd", plan.kernels)
     roofline = {"bound": "alu", "achieved": round(alu_achieved, 1), "peak": round(alu_peak, 1),
@@ -709,6 +717,7 @@ def main():
                        "gate": w.gate, "skip": w.skip, "h0": w.with_h0,
                        "segments": plan.segments, "segment_steps": plan.segment_steps,
                        "input_term": "exact ZOH" if args.zoh else "Delta B",
+                       "A": "learned-like (unstructured)" if args.learned_a else "(n+1) A[d,0]",
                        "l2": "flushed (256 MB write) before every timed step",
                        "parallelism": f"dp{world} (batch shards, no data-path collective)"},
             "hbm_gbs": round(achieved, 1), "hbm_frac_of_peak": round(achieved / peak, 4),

@@ -30,8 +30,8 @@
  *     the caller's next synchronisation.
  *   - Return value: SSM_OK, or a negative SSM_ERR_* code. Argument errors
  *     are detected on the host before anything is enqueued.
- *   - Pointers must be aligned to their element size (h0 / h_last to 8
- *     bytes; for ssm_state_update the state and A to 16 bytes when
+ *   - Pointers must be aligned to their element size (h0 / h_last and A
+ *     of the scan and its backward to 8 bytes; for ssm_state_update the state and A to 16 bytes when
  *     dstate % 4 == 0, else 8, and B, C to four elements when dstate % 4 == 0,
  *     else two). The fast
  *     path also wants 16-byte aligned bases and rows (dim and dstate

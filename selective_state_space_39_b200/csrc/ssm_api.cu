@@ -322,6 +322,7 @@ static int scan_fwd_impl(int64_t batch, int64_t seqlen, int64_t dim, int64_t dst
   for (const void* p : f32_ptrs)
     if (p && !aligned(p, 4)) return SSM_ERR_INVALID_ARG;
   if ((h0 && !aligned(h0, 8)) || (h_last && !aligned(h_last, 8))) return SSM_ERR_INVALID_ARG;
+  if (!aligned(A, 8)) return SSM_ERR_INVALID_ARG;  // rows of A are read as pairs
   // y must not overlap an input
   const size_t by = n_bld * es;
   if (overlap(y, by, x, n_bld * es) || overlap(y, by, delta, n_bld * es) ||
@@ -484,6 +485,7 @@ int ssm_scan_bwd(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate, int
   const void* f32_ptrs[] = {A, D, delta_bias, h0, dh_last, dA, dB, dC, dD, ddelta_bias, dh0};
   for (const void* p : f32_ptrs)
     if (p && !aligned(p, 4)) return SSM_ERR_INVALID_ARG;
+  if (!aligned(A, 8)) return SSM_ERR_INVALID_ARG;  // rows of A are read as pairs
   // no output may overlap an input or another output
   const size_t n_bld = (size_t)batch * seqlen * dim, n_bln = (size_t)batch * seqlen * dstate;
   const size_t n_bdn = (size_t)batch * dim * dstate, n_dn = (size_t)dim * dstate;

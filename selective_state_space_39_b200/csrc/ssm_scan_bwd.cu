@@ -157,9 +157,9 @@ __device__ __forceinline__ float sigmoid_f(float z) {
 
 // Decays a_n = exp(Delta A_n) of one step as pairs (a_2k, a_2k+1):
 // structured A by a multiply chain from r = exp(Delta A_0), else one exp per
-// state (A row read through L1).
+// state (Ap: the row of A as pairs, in registers).
 template <int N, bool kFast, bool kStruct>
-__device__ __forceinline__ void decays2(float q, float A0, const float* Arow,
+__device__ __forceinline__ void decays2(float q, float A0, const float2 (&Ap)[N / 2],
                                         float2 (&a)[N / 2]) {
   if constexpr (kStruct) {
     const float r = exp_u<kFast>(q * A0);
@@ -171,17 +171,8 @@ __device__ __forceinline__ void decays2(float q, float A0, const float* Arow,
   } else {
 #pragma unroll
     for (int k = 0; k < N / 2; ++k)
-      a[k] = make_float2(exp_u<kFast>(q * __ldg(Arow + 2 * k)),
-                         exp_u<kFast>(q * __ldg(Arow + 2 * k + 1)));
+      a[k] = make_float2(exp_u<kFast>(q * Ap[k].x), exp_u<kFast>(q * Ap[k].y));
   }
-}
-
-// (A_2k, A_2k+1) for the dDelta sum: (2k+1, 2k+2) when structured (times
-// A_0 after the sum).
-template <bool kStruct>
-__device__ __forceinline__ float2 a_coef2(int k, const float* Arow) {
-  if constexpr (kStruct) return make_float2((float)(2 * k + 1), (float)(2 * k + 2));
-  else return make_float2(__ldg(Arow + 2 * k), __ldg(Arow + 2 * k + 1));
 }
 
 // Structured-A test over the CTA (A[d,n] == (n+1) A[d,0] for all its channels).
@@ -312,6 +303,10 @@ __device__ __forceinline__ void carry_body(const BwdParams& p, unsigned char* sm
   //   P_n   prod_{u <= t} a_n(u) from the segment start,
   //   m_n   sum_t P_n(t) C_n(t) g_t: the segment's outgoing adjoint from a
   //         zero end, a(t0) lam(t0), accumulated forwards.
+  float2 Ap[NP];  // row of A as pairs (the one-exp-per-state path reads it)
+#pragma unroll
+  for (int k = 0; k < NP; ++k)
+    Ap[k] = kStruct ? make_float2(0.f, 0.f) : __ldg(reinterpret_cast<const float2*>(Arow) + k);
   float2 h[NP], P[NP], m[NP];
 #pragma unroll
   for (int k = 0; k < NP; ++k) {
@@ -353,7 +348,7 @@ __device__ __forceinline__ void carry_body(const BwdParams& p, unsigned char* sm
       if (j < nt) {
         const StepIn s = step_in<IOT, kFast>(sS, j, tid, bias, p.softplus, has_z);
         float2 a[NP];
-        decays2<N, kFast, kStruct>(s.q, A0, Arow, a);
+        decays2<N, kFast, kStruct>(s.q, A0, Ap, a);
         const float2 dtx = make_float2(s.dt * s.x, s.dt * s.x);
         const float2 g2 = make_float2(s.g, s.g);
 #pragma unroll
@@ -479,9 +474,10 @@ __device__ __forceinline__ void issue_main_tile(const BwdParams& p, unsigned cha
 }
 
 // Decays of this thread's state pairs q0 .. q0+NQ-1: (r^(2q+1), r^(2q+2)),
-// or one exp per state for generic A.
+// or one exp per state for generic A (Ap: this thread's pairs of A).
 template <int N, bool kFast, bool kStruct>
-__device__ __forceinline__ void decays_own(float qs, float A0, const float* Arow, int q0,
+__device__ __forceinline__ void decays_own(float qs, float A0,
+                                           const float2 (&Ap)[MainShape<N>::NQ], int q0,
                                            float2 (&a)[MainShape<N>::NQ]) {
   constexpr int NQ = MainShape<N>::NQ;
   if constexpr (kStruct) {
@@ -502,8 +498,8 @@ __device__ __forceinline__ void decays_own(float qs, float A0, const float* Arow
   } else {
 #pragma unroll
     for (int i = 0; i < NQ; ++i)
-      a[i] = make_float2(exp_u<kFast>(qs * __ldg(Arow + 2 * (q0 + i))),
-                         exp_u<kFast>(qs * __ldg(Arow + 2 * (q0 + i) + 1)));
+      a[i] = make_float2(exp_u<kFast>(qs * Ap[i].x), exp_u<kFast>(qs * Ap[i].y));
+    (void)q0;
   }
 }
 
@@ -579,7 +575,7 @@ __device__ __forceinline__ void main_body(const BwdParams& p, unsigned char* sme
     float2 he[NQ];
     {
       float2 P[NQ];
-      decays_own<N, kFast, kStruct>(sCk[N * kNT + c], A0, Arow, q0, P);
+      decays_own<N, kFast, kStruct>(sCk[N * kNT + c], A0, coef, q0, P);
 #pragma unroll
       for (int i = 0; i < NQ; ++i) {
         const int n = 2 * (q0 + i);
@@ -593,7 +589,7 @@ __device__ __forceinline__ void main_body(const BwdParams& p, unsigned char* sme
     for (int j = 0; j < kBT; ++j) {
       const StepIn s = step_in<IOT, kFast>(sScal, j, c, bias, p.softplus, has_z);
       float2 a[NQ];
-      decays_own<N, kFast, kStruct>(s.q, A0, Arow, q0, a);
+      decays_own<N, kFast, kStruct>(s.q, A0, coef, q0, a);
       const float2 dtx = make_float2(s.dt * s.x, s.dt * s.x);
 #pragma unroll
       for (int i = 0; i < NQ; ++i)
@@ -605,7 +601,7 @@ __device__ __forceinline__ void main_body(const BwdParams& p, unsigned char* sme
       if (j < nt) {
         const StepIn s = step_in<IOT, kFast>(sScal, j, c, bias, p.softplus, has_z);
         float2 a[NQ];
-        decays_own<N, kFast, kStruct>(s.q, A0, Arow, q0, a);
+        decays_own<N, kFast, kStruct>(s.q, A0, coef, q0, a);
         const float2 g2 = make_float2(s.g, s.g);
         const float2 dt2 = make_float2(s.dt, s.dt);
         const float2 dtx2 = make_float2(s.dt * s.x, s.dt * s.x);

@@ -369,6 +369,10 @@ __global__ void __launch_bounds__(NT, SSM_MIN_CTAS) scan_kernel(const ScanParams
     return in;
   };
 
+  // Rows of A for the one-exp-per-state path, held in registers (loaded by
+  // run_tiles for that path only).
+  float2 Areg[CPT][NP];
+
   // State update (and readout) of one step, given its precomputed scalars.
   auto state_step = [&](auto kStructTag, const StepIn& in, const StepScalars* sc, const float* Bt,
                         const float* Ct, int t_abs) {
@@ -446,7 +450,6 @@ __global__ void __launch_bounds__(NT, SSM_MIN_CTAS) scan_kernel(const ScanParams
     } else {
 #pragma unroll
       for (int c = 0; c < CPT; ++c) {
-        const float* Ar = p.A + (size_t)(ch[c].valid ? d_first + c : 0) * N;
         const float2* B2 = reinterpret_cast<const float2*>(Bt);
         const float2* C2 = reinterpret_cast<const float2*>(Ct);
         (void)C2;
@@ -454,7 +457,7 @@ __global__ void __launch_bounds__(NT, SSM_MIN_CTAS) scan_kernel(const ScanParams
 #pragma unroll
         for (int k = 0; k < NP; ++k) {
           float2 a;
-          const float A_lo = __ldg(Ar + 2 * k), A_hi = __ldg(Ar + 2 * k + 1);
+          const float A_lo = Areg[c][k].x, A_hi = Areg[c][k].y;
           const float e_lo = kFast ? ex2_approx(q * A_lo) : expf(q * A_lo);
           const float e_hi = kFast ? ex2_approx(q * A_hi) : expf(q * A_hi);
           a = make_float2(rho * e_lo, rho * e_hi);
@@ -507,6 +510,15 @@ __global__ void __launch_bounds__(NT, SSM_MIN_CTAS) scan_kernel(const ScanParams
 
   // ---- tile loop ----------------------------------------------------------
   auto run_tiles = [&](auto kStructTag) {
+    if constexpr (!decltype(kStructTag)::value) {
+#pragma unroll
+      for (int c = 0; c < CPT; ++c) {
+        const float2* Ar =
+            reinterpret_cast<const float2*>(p.A + (size_t)(ch[c].valid ? d_first + c : 0) * N);
+#pragma unroll
+        for (int k = 0; k < NP; ++k) Areg[c][k] = __ldg(Ar + k);
+      }
+    }
     for (int it = 0; it < ntiles; ++it) {
       const int buf = it & 1;
       unsigned char* st;

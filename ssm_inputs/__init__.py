@@ -40,6 +40,8 @@ STREAM_X, STREAM_DELTA, STREAM_Z, STREAM_B, STREAM_C, STREAM_H0, STREAM_BIAS = 1
 STREAM_DY, STREAM_DH_LAST = 8, 9
 # the block's causal conv1d: raw input, taps, bias, upstream gradient
 STREAM_CONV_X, STREAM_CONV_W, STREAM_CONV_BIAS, STREAM_CONV_DOUT = 10, 11, 12, 13
+# a learned-looking A (no (n + 1) A[d, 0] structure)
+STREAM_A_LEARNED = 14
 KIND_NORMAL, KIND_UNIFORM = 0, 1
 OUT_F64, OUT_F32, OUT_BF16 = 0, 1, 2
 
@@ -204,6 +206,15 @@ DECODE_WORKLOADS = {
 def a_matrix(dim, dstate):
     """A[d, n] = -(n + 1) for every channel, as fp32."""
     return np.tile(-np.arange(1, dstate + 1, dtype=np.float32), (dim, 1))
+
+
+def a_matrix_learned(dim, dstate, seed):
+    """A[d, n] = -exp(A_log[d, n]) with A_log = log(n + 1) + U[-0.5, 0.5]: the
+    initial values perturbed per (d, n) as training moves them, so that A has
+    no (n + 1) A[d, 0] structure (fp32)."""
+    jitter = fill((dim, dstate), seed, STREAM_A_LEARNED, KIND_UNIFORM, -0.5, 0.5, out="f64")
+    a_log = np.log(np.arange(1, dstate + 1, dtype=np.float64))[None, :] + jitter
+    return (-np.exp(a_log)).astype(np.float32)
 
 
 def delta_bias(dim, seed, nthreads=None):

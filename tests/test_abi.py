@@ -106,6 +106,7 @@ def test_scan_rejects_bad_arguments(L):
     assert scan(L, x=FAKE + 1) == -1            # misaligned bf16
     assert scan(L, io=0, B=FAKE + 12290) == -1  # misaligned fp32
     assert scan(L, h0=FAKE + 4) == -1           # h0 needs 8-byte alignment
+    assert scan(L, A=FAKE + 8192 + 4) == -1     # rows of A are read as pairs
     assert scan(L, y=FAKE + 2) == -1            # y overlaps x
     assert scan(L, dstate=5) == -2
     assert scan(L, seqlen=-3) == -1
