@@ -223,3 +223,31 @@ def test_repeated_calls_are_deterministic():
     y1, h1 = gpu_scan(inp)
     y2, h2 = gpu_scan(inp)
     assert torch.equal(y1, y2) and torch.equal(h1, h2)
+
+
+# ------------------------------------------------------ A without structure
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("N", [2, 8, 16, 32, 64])
+def test_learned_A_one_exp_per_state(monkeypatch, io, N):
+    """A with no (n+1) A[d,0] structure (as after training) takes the
+    one-exp-per-state path, part of whose exps run on the FMA pipe; segments
+    3, so the carry composition of that path is covered too."""
+    monkeypatch.setenv("SSM_SCAN_SEGMENTS", "3")
+    inp = gen.make_scan_inputs(2, 90, 200, N, io, 41, with_h0=True)
+    inp["A"] = gen.a_matrix_learned(200, N, 41)
+    y, hl = gpu_scan(inp)
+    yr, hr = oracle_scan(inp, io)
+    _check(host(y), host(hl), yr, hr, io, f"learned A {io} N={N}")
+
+
+def test_learned_A_mamba130m_layer_sampled():
+    w = gen.SCAN_WORKLOADS["mamba130m_layer_b8_l2048_d1536"]
+    inp = gen.workload_inputs(w)
+    inp["A"] = gen.a_matrix_learned(w.dim, w.dstate, w.seed)
+    y, hl = gpu_scan(inp)
+    chans = sample_channels(w.batch, w.dim, 12)
+    yr, hr = oracle_scan(inp, w.io, channels=chans)
+    yg, hg = host(y), host(hl)
+    ys = np.stack([yg[b, :, d] for b, d in chans])
+    hs = np.stack([hg[b, d] for b, d in chans])
+    _check(ys, hs, yr, hr, w.io, "learned A 8x2048x1536")
