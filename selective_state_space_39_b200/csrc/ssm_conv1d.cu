@@ -37,7 +37,7 @@ namespace {
 
 constexpr int kMaxThreads = 192;  // CTA size cap: two or more CTAs per SM
 constexpr int kUnroll = 8;     // forward: steps whose loads are in flight together
-constexpr int kUnrollBwd = 8;  // backward: the same (two tensors per step)
+constexpr int kUnrollBwd = 4;  // backward: the same (two tensors per step)
 
 template <bool kFast>
 __device__ __forceinline__ float sigmoid_c(float u) {
