@@ -88,6 +88,10 @@ class Oracle:
         cb.restype = ctypes.c_int
         cb.argtypes = [ctypes.c_int64] * 4 + [ctypes.c_int, ctypes.c_void_p, _F32P, _F32P,
                                               ctypes.c_int, ctypes.c_void_p, _F64P, _F64P, _F64P]
+        cu = self.lib.oracle_conv1d_silu_update
+        cu.restype = ctypes.c_int
+        cu.argtypes = [ctypes.c_int64] * 3 + [ctypes.c_int, _F64P, ctypes.c_void_p, _F32P, _F32P,
+                                              ctypes.c_int, _F64P]
         g = self.lib.oracle_state_update
         g.restype = ctypes.c_int
         g.argtypes = [ctypes.c_int64] * 3 + [ctypes.c_int, _F64P, ctypes.c_void_p,
@@ -282,6 +286,27 @@ class Oracle:
         if rc != 0:
             raise ValueError("oracle_conv1d_silu_bwd rejected its arguments")
         return dx, dw, db
+
+    def conv1d_silu_update(self, state, x, w, bias=None, silu=True, io="f32"):
+        """One decode step of the causal conv on the fp64 ``state`` (batch,
+        dim, width-1; oldest input first), in place. x is (batch, dim).
+        Returns out (batch, dim) in fp64."""
+        if state.dtype != np.float64 or not state.flags.c_contiguous:
+            raise TypeError("state must be a C-contiguous float64 array")
+        batch, dim, S = state.shape
+        width = S + 1
+        x = self._io_array(x, io, (batch, dim), "x")
+        w = self._f32_array(w, (dim, width), "w", optional=False)
+        bias = self._f32_array(bias, (dim,), "bias")
+        out = np.empty((batch, dim), dtype=np.float64)
+        rc = self.lib.oracle_conv1d_silu_update(batch, dim, width, 1 if io == "bf16" else 0,
+                                                self._ptr(state, ctypes.c_double), self._ptr(x),
+                                                self._ptr(w, ctypes.c_float),
+                                                self._ptr(bias, ctypes.c_float), 1 if silu else 0,
+                                                self._ptr(out, ctypes.c_double))
+        if rc != 0:
+            raise ValueError("oracle_conv1d_silu_update rejected its arguments")
+        return out
 
     # -- decode ------------------------------------------------------------
     def state_update(self, state, x, delta, A, B, C, D=None, z=None, delta_bias=None,

@@ -571,3 +571,28 @@ int oracle_conv1d_silu_bwd(int64_t batch, int64_t seqlen, int64_t dim, int64_t w
   free(du);
   return 0;
 }
+
+/* oracle_conv1d_silu_update -- one decode step of the block's causal conv:
+ * state (batch, dim, width-1) holds the last width-1 inputs of each channel,
+ * oldest first (zero at the start of a sequence); x (batch, dim) is the new
+ * input. out = SiLU(bias + sum_(k < width-1) w[d,k] state[k] + w[d,width-1] x)
+ * (or without SiLU), then the state drops its oldest input and appends x.
+ * The state is the oracle's own fp64 copy. Returns 0 or -1. */
+int oracle_conv1d_silu_update(int64_t batch, int64_t dim, int64_t width, int is_bf16,
+                              double* state, const void* x, const float* w, const float* bias,
+                              int silu_on, double* out) {
+  if (batch < 0 || dim < 0 || width < 1 || !state || !x || !w || !out) return -1;
+  const int64_t S = width - 1;
+  for (int64_t b = 0; b < batch; ++b)
+    for (int64_t d = 0; d < dim; ++d) {
+      double* st = state + (b * dim + d) * S;
+      const double xv = widen(x, b * dim + d, is_bf16);
+      double u = bias ? (double)bias[d] : 0.0;
+      for (int64_t k = 0; k < S; ++k) u += (double)w[d * width + k] * st[k];
+      u += (double)w[d * width + S] * xv;
+      out[b * dim + d] = silu_on ? silu(u) : u;
+      for (int64_t k = 0; k + 1 < S; ++k) st[k] = st[k + 1];
+      if (S > 0) st[S - 1] = xv;
+    }
+  return 0;
+}

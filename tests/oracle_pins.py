@@ -551,6 +551,18 @@ def pin_zoh_decode_steps_equal_scan(o):
     _close(state, hl, 1e-13, 1e-14, what="zoh decode state")
 
 
+def pin_conv_update_steps_equal_conv(o):
+    """L conv decode steps from a zero state reproduce the (separately pinned)
+    causal conv over the sequence, for widths 2, 3, 4."""
+    for width in (2, 3, 4):
+        x, w, b = _conv_case(211 + width, batch=2, L=7, dim=3, width=width)
+        full = o.conv1d_silu(x, w, b)
+        state = np.zeros((2, 3, width - 1))
+        for t in range(7):
+            out = o.conv1d_silu_update(state, np.ascontiguousarray(x[:, t]), w, b)
+            _close(out, full[:, t], 1e-14, 1e-15, what=f"conv step {t} width {width}")
+
+
 ALL_PINS = [
     pin_softplus_library,
     pin_silu_library,
@@ -572,6 +584,7 @@ ALL_PINS = [
     pin_conv_by_hand,
     pin_conv_is_causal,
     pin_conv_bwd_finite_differences,
+    pin_conv_update_steps_equal_conv,
     pin_zoh_matches_scipy_cont2discrete,
     pin_zoh_small_step_is_euler,
     pin_zoh_decode_steps_equal_scan,

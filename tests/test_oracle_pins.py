@@ -101,6 +101,7 @@ MUTANTS = {
     "conv_bwd_dw_wrong_step": ("if (s >= 0) dw[d * width + k] += du[t] * widen(x, (b * seqlen + s) * dim + d, is_bf16);",
                                "if (s >= 0) dw[d * width + k] += du[t] * widen(x, (b * seqlen + t) * dim + d, is_bf16);"),
     "conv_bwd_dbias_from_dout": ("        dbias[d] += du[t];", "        dbias[d] += g;"),
+    "conv_update_state_not_shifted": ("      for (int64_t k = 0; k + 1 < S; ++k) st[k] = st[k + 1];\n", ""),
     # exact zero-order hold
     "zoh_is_euler": ("  return An == 0.0 ? dt : expm1(dt * An) / An;", "  return dt;"),
     "zoh_no_division_by_A": ("  return An == 0.0 ? dt : expm1(dt * An) / An;",
