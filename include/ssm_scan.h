@@ -255,6 +255,20 @@ int ssm_conv1d_silu_fwd(int64_t batch, int64_t seqlen, int64_t dim, int64_t widt
                         const void* x, const float* w, const float* bias, int silu, void* out,
                         void* stream);
 
+/*
+ * ssm_conv1d_silu_update -- one decode step of the same convolution (the
+ * step form for single-token decode, beside ssm_state_update):
+ *   conv_state : (batch, dim, width-1) io_dtype, the channel's last width-1
+ *                inputs, oldest first (zero at the start of a sequence);
+ *                read and updated in place (drops the oldest, appends x)
+ *   x, out     : (batch, dim) io_dtype
+ *   out[b,d]   = SiLU(bias[d] + sum_(k<width-1) w[d,k] state[k] + w[d,width-1] x[b,d])
+ * width 2, 3 or 4. No buffer may overlap another. Returns SSM_OK or SSM_ERR_*.
+ */
+int ssm_conv1d_silu_update(int64_t batch, int64_t dim, int64_t width, int io_dtype,
+                           void* conv_state, const void* x, const float* w, const float* bias,
+                           int silu, void* out, void* stream);
+
 /* ssm_conv1d_silu_bwd_workspace_bytes -- workspace of ssm_conv1d_silu_bwd:
  * per-(batch row, 128-step chunk) partial sums of dw and dbias. */
 size_t ssm_conv1d_silu_bwd_workspace_bytes(int64_t batch, int64_t seqlen, int64_t dim,

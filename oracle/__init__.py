@@ -369,3 +369,7 @@ def conv1d_silu(*args, **kwargs):
 
 def conv1d_silu_bwd(*args, **kwargs):
     return get().conv1d_silu_bwd(*args, **kwargs)
+
+
+def conv1d_silu_update(*args, **kwargs):
+    return get().conv1d_silu_update(*args, **kwargs)

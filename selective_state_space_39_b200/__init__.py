@@ -17,6 +17,7 @@ from ._binding import (  # noqa: F401
     ssm_compose_carries,
     ssm_conv1d_silu_bwd,
     ssm_conv1d_silu_fwd,
+    ssm_conv1d_silu_update,
     ssm_delta_sum,
     ssm_scan_bwd,
     ssm_scan_fwd,
@@ -27,6 +28,7 @@ from ._binding import (  # noqa: F401
 
 __all__ = ["ssm_scan_fwd", "ssm_scan_fwd_noalloc", "ssm_scan_bwd", "ssm_state_update",
            "ssm_scan_status", "scan_plan", "scan_workspace_bytes", "scan_bwd_workspace_bytes",
-           "ssm_conv1d_silu_fwd", "ssm_conv1d_silu_bwd", "conv1d_silu_bwd_workspace_bytes",
+           "ssm_conv1d_silu_fwd", "ssm_conv1d_silu_bwd", "ssm_conv1d_silu_update",
+           "conv1d_silu_bwd_workspace_bytes",
            "ssm_delta_sum", "ssm_compose_carries",
            "SsmError", "SSM_DTYPE_F32", "SSM_DTYPE_BF16", "lib"]

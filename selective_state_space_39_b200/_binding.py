@@ -85,6 +85,9 @@ def lib() -> ctypes.CDLL:
         L.ssm_conv1d_silu_fwd.restype = ctypes.c_int
         L.ssm_conv1d_silu_fwd.argtypes = [_I64, _I64, _I64, _I64, ctypes.c_int, _VP, _VP, _VP,
                                           ctypes.c_int, _VP, _VP]
+        L.ssm_conv1d_silu_update.restype = ctypes.c_int
+        L.ssm_conv1d_silu_update.argtypes = [_I64, _I64, _I64, ctypes.c_int, _VP, _VP, _VP, _VP,
+                                             ctypes.c_int, _VP, _VP]
         L.ssm_conv1d_silu_bwd_workspace_bytes.restype = ctypes.c_size_t
         L.ssm_conv1d_silu_bwd_workspace_bytes.argtypes = [_I64, _I64, _I64, _I64, ctypes.c_int]
         L.ssm_conv1d_silu_bwd.restype = ctypes.c_int
@@ -274,6 +277,30 @@ def ssm_conv1d_silu_fwd(x, w, bias=None, silu=True, out=None, stream=None):
                                        1 if silu else 0, po, _stream_ptr(stream, dev))
     if rc != 0:
         raise SsmError(rc, "ssm_conv1d_silu_fwd", with_detail=True)
+    return out
+
+
+def ssm_conv1d_silu_update(conv_state, x, w, bias=None, silu=True, out=None, stream=None):
+    """One decode step of the causal conv through ssm_conv1d_silu_update of
+    libssmscan.so: conv_state (batch, dim, width-1) in x's dtype (the last
+    inputs, oldest first) is updated in place; returns out (batch, dim)."""
+    if x.dim() != 2 or conv_state.dim() != 3:
+        raise ValueError("x must be (batch, dim) and conv_state (batch, dim, width-1)")
+    batch, dim = x.shape
+    width = conv_state.shape[2] + 1
+    dev = x.device
+    ps = _ptr(conv_state, "conv_state", x.dtype, (batch, dim, width - 1), dev)
+    px = _ptr(x, "x", x.dtype, (batch, dim))
+    pw = _ptr(w, "w", torch.float32, (dim, width), dev)
+    pb = _ptr(bias, "bias", torch.float32, (dim,), dev)
+    if out is None:
+        out = torch.empty((batch, dim), dtype=x.dtype, device=dev)
+    po = _ptr(out, "out", x.dtype, (batch, dim), dev)
+    with torch.cuda.device(dev):
+        rc = lib().ssm_conv1d_silu_update(batch, dim, width, _io_code(x.dtype), ps, px, pw, pb,
+                                          1 if silu else 0, po, _stream_ptr(stream, dev))
+    if rc != 0:
+        raise SsmError(rc, "ssm_conv1d_silu_update", with_detail=True)
     return out
 
 

@@ -615,6 +615,29 @@ int ssm_conv1d_silu_fwd(int64_t batch, int64_t seqlen, int64_t dim, int64_t widt
                      "conv1d forward launch");
 }
 
+int ssm_conv1d_silu_update(int64_t batch, int64_t dim, int64_t width, int io_dtype,
+                           void* conv_state, const void* x, const float* w, const float* bias,
+                           int silu, void* out, void* stream) {
+  int st = conv_check(batch, 1, dim, width, io_dtype);
+  if (st != SSM_OK) return st;
+  if (batch == 0 || dim == 0) return SSM_OK;
+  if (!conv_state || !x || !w || !out) return SSM_ERR_INVALID_ARG;
+  const size_t es = io_bytes(io_dtype), n = (size_t)batch * dim;
+  if (!aligned(conv_state, es) || !aligned(x, es) || !aligned(out, es) || !aligned(w, 4) ||
+      (bias && !aligned(bias, 4)))
+    return SSM_ERR_INVALID_ARG;
+  const size_t bs = n * (size_t)(width - 1) * es;
+  if (overlap(out, n * es, conv_state, bs) || overlap(out, n * es, x, n * es) ||
+      overlap(conv_state, bs, x, n * es) || overlap(out, n * es, w, (size_t)dim * width * 4) ||
+      overlap(conv_state, bs, w, (size_t)dim * width * 4))
+    return fail(SSM_ERR_INVALID_ARG, "ssm_conv1d_silu_update: buffers overlap");
+  ConvParams p = conv_params(batch, 1, dim, width, silu, false);
+  p.x = x; p.w = w; p.bias = bias; p.out = conv_state; p.dx = out;
+  return cuda_status(launch_conv_update(p, io_dtype == SSM_DTYPE_BF16,
+                                        static_cast<cudaStream_t>(stream)),
+                     "conv1d update launch");
+}
+
 size_t ssm_conv1d_silu_bwd_workspace_bytes(int64_t batch, int64_t seqlen, int64_t dim,
                                            int64_t width, int io_dtype) {
   if (conv_check(batch, seqlen, dim, width, io_dtype) != SSM_OK) return 0;

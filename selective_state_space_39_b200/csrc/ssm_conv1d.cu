@@ -325,6 +325,31 @@ __global__ void __launch_bounds__(256) conv_reduce_kernel(const ConvParams p, in
   }
 }
 
+// One decode step per (b, d): out = SiLU(bias + sum_k w_k state_k + w_(W-1) x),
+// then the rolling state (the last W-1 inputs, oldest first, in the io type)
+// drops its oldest entry and appends x.
+template <typename IOT, int W>
+__global__ void __launch_bounds__(256) conv_update_kernel(const ConvParams p) {
+  using IO = Io<IOT>;
+  constexpr bool kFast = std::is_same<IOT, uint16_t>::value;
+  const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (size_t)p.batch * p.dim) return;
+  const int d = (int)(i % p.dim);
+  IOT* st = reinterpret_cast<IOT*>(p.out) + i * (W - 1);  // the state (in/out)
+  float sv[W - 1];
+#pragma unroll
+  for (int k = 0; k < W - 1; ++k) sv[k] = IO::load(st + k);
+  const float xv = IO::load(reinterpret_cast<const IOT*>(p.x) + i);
+  float u = p.bias ? __ldg(p.bias + d) : 0.f;
+#pragma unroll
+  for (int k = 0; k < W - 1; ++k) u = fmaf(__ldg(p.w + (size_t)d * W + k), sv[k], u);
+  u = fmaf(__ldg(p.w + (size_t)d * W + W - 1), xv, u);
+  IO::store(reinterpret_cast<IOT*>(p.dx) + i, p.silu ? u * sigmoid_c<kFast>(u) : u);
+#pragma unroll
+  for (int k = 0; k + 1 < W - 1; ++k) IO::store(st + k, sv[k + 1]);
+  IO::store(st + (W - 2), xv);
+}
+
 int sm_count() {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -376,7 +401,24 @@ cudaError_t launch_w(const ConvParams& p, bool backward, cudaStream_t stream) {
   }
 }
 
+template <typename IOT>
+cudaError_t launch_update_io(const ConvParams& p, cudaStream_t stream) {
+  const size_t n = (size_t)p.batch * p.dim;
+  const unsigned blocks = (unsigned)((n + 255) / 256);
+  switch (p.width) {
+    case 2: conv_update_kernel<IOT, 2><<<blocks, 256, 0, stream>>>(p); break;
+    case 3: conv_update_kernel<IOT, 3><<<blocks, 256, 0, stream>>>(p); break;
+    case 4: conv_update_kernel<IOT, 4><<<blocks, 256, 0, stream>>>(p); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
 }  // namespace
+
+cudaError_t launch_conv_update(const ConvParams& p, bool bf16, cudaStream_t stream) {
+  return bf16 ? launch_update_io<uint16_t>(p, stream) : launch_update_io<float>(p, stream);
+}
 
 bool conv_width_supported(int width) { return width >= 2 && width <= 4; }
 

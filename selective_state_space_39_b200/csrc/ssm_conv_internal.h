@@ -31,6 +31,9 @@ struct ConvParams {
 };
 
 bool conv_width_supported(int width);
+// Decode step: p.out is the rolling state (batch, dim, width-1) io, p.x the
+// new input (batch, dim), p.dx the output (batch, dim).
+cudaError_t launch_conv_update(const ConvParams& p, bool bf16, cudaStream_t stream);
 // vec: 8-byte vector path (dim a multiple of 4 for bf16 / 2 for fp32, 8-byte
 // aligned tensors); otherwise one element per thread.
 cudaError_t launch_conv(const ConvParams& p, bool bf16, bool vec, bool backward,

@@ -201,6 +201,13 @@ def test_conv_rejects_bad_arguments(L):
     assert bwd() == -3                  # no workspace
     need = L.ssm_conv1d_silu_bwd_workspace_bytes(2, 32, 64, 4, 1)
     assert need > 0 and bwd(ws=FAKE * 64, ws_bytes=need - 1) == -3
+    # decode step: state (2, 64, 3) bf16 = 768 bytes
+    upd = lambda **kw: L.ssm_conv1d_silu_update(  # noqa: E731
+        kw.get("batch", 2), 64, kw.get("width", 4), 1, kw.get("state", FAKE), kw.get("x", FAKE + K),
+        FAKE + 2 * K, None, 1, kw.get("out", FAKE + 3 * K), None)
+    assert upd(state=None) == -1 and upd(x=None) == -1
+    assert upd(out=FAKE + 64) == -1     # out overlaps the state
+    assert upd(width=6) == -2 and upd(batch=0) == 0
 
 
 @no_gpu_only

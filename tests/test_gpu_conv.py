@@ -96,3 +96,22 @@ def test_conv_bwd_deterministic():
     g1, g2 = run_bwd(c), run_bwd(c)
     for k in ("dx", "dw", "dbias"):
         assert torch.equal(g1[k], g2[k]), k
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("width", [2, 3, 4])
+def test_conv_update_steps_match_oracle(io, width):
+    """Decode steps of the conv (rolling state) against the oracle's steps,
+    and against the GPU's own conv over the same tokens."""
+    import oracle
+    from selective_state_space_39_b200 import ssm_conv1d_silu_fwd, ssm_conv1d_silu_update
+    c = gen.make_conv_inputs(3, 9, 130, width, io, 13)
+    st = torch.zeros((3, 130, width - 1), dtype=dev(c["x"]).dtype, device="cuda")
+    ref = np.zeros((3, 130, width - 1))
+    full = host(ssm_conv1d_silu_fwd(dev(c["x"]), dev(c["w"]), dev(c["bias"])))
+    for t in range(9):
+        xt = np.ascontiguousarray(c["x"][:, t])
+        out = host(ssm_conv1d_silu_update(st, dev(xt), dev(c["w"]), dev(c["bias"])))
+        want = oracle.conv1d_silu_update(ref, xt, c["w"], c["bias"], io=io)
+        assert rel_err(out, want) <= TOL[io], f"step {t}"
+        assert rel_err(out, full[:, t]) <= TOL[io], f"step {t} vs the conv"
