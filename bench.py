@@ -132,7 +132,7 @@ class ClockSampler:
                 idx = int(vis.split(",")[device_index])
             self.h = pynvml.nvmlDeviceGetHandleByIndex(idx)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
-        except Exception as e:  # pragma: no cover - depends on the box
+        except Exception as e:  # pragma: no cover - depends on the machine
             self.nvml, self.error = None, f"nvml unavailable: {e}"
         self.t = threading.Thread(target=self._run, daemon=True)
 

@@ -56,13 +56,13 @@ enum {
 enum {
   SSM_OK = 0,
   SSM_ERR_INVALID_ARG = -1, /* null required pointer, bad size, misaligned, aliasing */
-  SSM_ERR_UNSUPPORTED = -2, /* dstate or io_dtype this build does not support       */
+  SSM_ERR_UNSUPPORTED = -2, /* dstate or io_dtype this library does not support     */
   SSM_ERR_WORKSPACE = -3,   /* workspace missing or smaller than required           */
   SSM_ERR_CUDA = -4,        /* a CUDA runtime call or kernel launch failed          */
   SSM_ERR_TIMEOUT = -5,     /* a bounded wait inside a kernel gave up (ssm_scan_status) */
 };
 
-/* dstate (N) values this build supports: 2, 4, 8, 16, 32, 64. */
+/* dstate (N) values this library supports: 2, 4, 8, 16, 32, 64. */
 #define SSM_MAX_DSTATE 64
 
 /*

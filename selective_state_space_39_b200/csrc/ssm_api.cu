@@ -47,7 +47,7 @@ int dims_status(const Dims& d) {
   if (d.batch < 0 || d.seqlen < 0 || d.dim < 0) return SSM_ERR_INVALID_ARG;
   if (d.dstate <= 0) return SSM_ERR_INVALID_ARG;
   if (!scan_dstate_supported((int)std::min<int64_t>(d.dstate, 1 << 20))) return SSM_ERR_UNSUPPORTED;
-  // grid and index limits of this build
+  // grid and index limits of this library
   if (d.batch > 65535 || d.dim > (1 << 24) || d.seqlen > (1 << 30)) return SSM_ERR_UNSUPPORTED;
   return SSM_OK;
 }
