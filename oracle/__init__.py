@@ -14,7 +14,9 @@ of the same loop, written out in ``ssm_oracle.c``. What it computes follows
 the page "Mamba 논문 리뷰: Selective State Space Models로 Transformer를
 넘어서" (youngju.dev): §2.2 discretised recurrence,
 §3.1 softplus step size, §3.3 simplified ``selective_scan``, §3.4 block gate,
-D skip and the causal depthwise conv1d + SiLU (``conv1d_silu``). Every function here is pinned by ``tests/test_oracle_pins.py``
+D skip and the causal depthwise conv1d + SiLU (``conv1d_silu``), §4.1 the
+multi-head SSD form (``ssd_scan``). Every function here is pinned by
+``tests/test_oracle_pins.py``
 against closed forms, brute force and invariants.
 
 bf16 arrays are passed as numpy ``uint16`` holding the raw bf16 bits with
@@ -98,6 +100,12 @@ class Oracle:
                       ctypes.c_void_p, _F32P, ctypes.c_void_p, ctypes.c_void_p, _F32P,
                       ctypes.c_void_p, _F32P, ctypes.c_int, _F64P]
         gz.argtypes = g.argtypes
+        sd = self.lib.oracle_ssd_scan
+        sd.restype = ctypes.c_int
+        sd.argtypes = [ctypes.c_int64] * 5 + [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+                                              _F32P, ctypes.c_void_p, ctypes.c_void_p, _F32P,
+                                              _F32P, ctypes.c_int, _F32P, _I64P, ctypes.c_int64,
+                                              _F64P, _F64P]
 
     # -- helpers -----------------------------------------------------------
     @staticmethod
@@ -337,6 +345,52 @@ class Oracle:
         return y
 
 
+    # -- Mamba-2 SSD ---------------------------------------------------------
+    def ssd_scan(self, x, dt, A, B, C, D=None, dt_bias=None, softplus=True, h0=None, io="f32",
+                 pairs=None):
+        """The multi-head SSD scan (scalar A per head, B and C shared by the
+        heads). x (batch, L, heads, headdim), dt (batch, L, heads), A (heads,),
+        B, C (batch, L, dstate), D, dt_bias (heads,) or None, h0 (batch, heads,
+        headdim, dstate) or None. Returns y (batch, L, heads, headdim) and
+        h_last (batch, heads, headdim, dstate) in fp64; with ``pairs`` (a list
+        of (b, h)) y is (npairs, L, headdim) and h_last (npairs, headdim,
+        dstate)."""
+        x = np.asarray(x)
+        batch, L, H, P = x.shape
+        N = np.asarray(B).shape[-1]
+        x = self._io_array(x, io, (batch, L, H, P), "x")
+        dt = self._io_array(dt, io, (batch, L, H), "dt")
+        B = self._io_array(B, io, (batch, L, N), "B")
+        C = self._io_array(C, io, (batch, L, N), "C")
+        A = self._f32_array(A, (H,), "A", optional=False)
+        D = self._f32_array(D, (H,), "D")
+        dt_bias = self._f32_array(dt_bias, (H,), "dt_bias")
+        h0 = self._f32_array(h0, (batch, H, P, N), "h0")
+        full = pairs is None
+        if full:
+            bb, hh = np.meshgrid(np.arange(batch), np.arange(H), indexing="ij")
+            pr = np.stack([bb.ravel(), hh.ravel()], axis=1).astype(np.int64)
+        else:
+            pr = np.ascontiguousarray(np.asarray(pairs, dtype=np.int64).reshape(-1, 2))
+        npairs = pr.shape[0]
+        y = np.empty((npairs, L, P), dtype=np.float64)
+        h_last = np.empty((npairs, P, N), dtype=np.float64)
+        rc = self.lib.oracle_ssd_scan(
+            batch, L, H, P, N, 1 if io == "bf16" else 0, self._ptr(x), self._ptr(dt),
+            self._ptr(A, ctypes.c_float), self._ptr(B), self._ptr(C),
+            self._ptr(D, ctypes.c_float), self._ptr(dt_bias, ctypes.c_float),
+            1 if softplus else 0, self._ptr(h0, ctypes.c_float), self._ptr(pr, ctypes.c_int64),
+            npairs, self._ptr(y, ctypes.c_double), self._ptr(h_last, ctypes.c_double))
+        if rc == -2:
+            raise MemoryError("oracle_ssd_scan ran out of memory")
+        if rc != 0:
+            raise ValueError("oracle_ssd_scan rejected its arguments")
+        if full:
+            y = y.reshape(batch, H, L, P).transpose(0, 2, 1, 3).copy()
+            h_last = h_last.reshape(batch, H, P, N)
+        return y, h_last
+
+
 _default = None
 
 
@@ -373,3 +427,7 @@ def conv1d_silu_bwd(*args, **kwargs):
 
 def conv1d_silu_update(*args, **kwargs):
     return get().conv1d_silu_update(*args, **kwargs)
+
+
+def ssd_scan(*args, **kwargs):
+    return get().ssd_scan(*args, **kwargs)

@@ -596,3 +596,65 @@ int oracle_conv1d_silu_update(int64_t batch, int64_t dim, int64_t width, int is_
     }
   return 0;
 }
+
+/* ---------------------------------------------------------------------------
+ * Mamba-2 SSD scan (page "Mamba 논문 리뷰", §4.1 State Space Duality and
+ * §4.2: multi-head, larger state). Head h of width P (headdim) has one scalar
+ * A[h] and one step Delta[b,t,h]; B and C (N wide) are shared by every head.
+ * The state of a head is an N x P matrix, held here as S[p][n]:
+ *
+ *   Delta      = softplus(dt[b,t,h] + dt_bias[h])   (or without softplus)
+ *   S[p][n]    = exp(Delta A[h]) S[p][n] + Delta B[b,t,n] x[b,t,h,p]
+ *   y[b,t,h,p] = sum_n C[b,t,n] S[p][n] + D[h] x[b,t,h,p]
+ *
+ * i.e. §4.1's h_t = A_t h_{t-1} + B_t x_t, y_t = C_t h_t with the scalar
+ * A_t = exp(Delta_t A[h]) and the input term Delta_t B_t of §3.3, per head.
+ * Layouts: x, y (batch, seqlen, nheads, headdim); dt (batch, seqlen, nheads);
+ * B, C (batch, seqlen, dstate); A, D, dt_bias (nheads); h0, h_last
+ * (batch, nheads, headdim, dstate). pairs (npairs x 2 int64: b, h) selects
+ * the heads computed; y_out is (npairs, seqlen, headdim) and h_last_out
+ * (npairs, headdim, dstate), fp64.
+ * Returns 0, -1 on bad arguments, -2 without memory.
+ */
+int oracle_ssd_scan(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim,
+                    int64_t dstate, int is_bf16, const void* x, const void* dt, const float* A,
+                    const void* Bm, const void* Cm, const float* D, const float* dt_bias,
+                    int softplus_on, const float* h0, const int64_t* pairs, int64_t npairs,
+                    double* y_out, double* h_last_out) {
+  if (batch < 0 || seqlen < 0 || nheads < 0 || headdim < 1 || dstate < 1 || npairs < 0 ||
+      !x || !dt || !A || !Bm || !Cm || !pairs || !y_out || !h_last_out)
+    return -1;
+  const int64_t P = headdim, N = dstate, H = nheads, L = seqlen;
+  double* S = (double*)malloc((size_t)(P * N) * sizeof(double));
+  if (!S) return -2;
+  for (int64_t k = 0; k < npairs; ++k) {
+    const int64_t b = pairs[2 * k], h = pairs[2 * k + 1];
+    if (b < 0 || b >= batch || h < 0 || h >= H) {
+      free(S);
+      return -1;
+    }
+    for (int64_t p = 0; p < P; ++p)
+      for (int64_t n = 0; n < N; ++n)
+        S[p * N + n] = h0 ? (double)h0[((b * H + h) * P + p) * N + n] : 0.0;
+    const double bias = dt_bias ? (double)dt_bias[h] : 0.0;
+    const double Dh = D ? (double)D[h] : 0.0;
+    for (int64_t t = 0; t < L; ++t) {
+      const double v = widen(dt, (b * L + t) * H + h, is_bf16) + bias;
+      const double delta = softplus_on ? softplus(v) : v;
+      const double a = exp(delta * (double)A[h]);
+      for (int64_t p = 0; p < P; ++p) {
+        const double xv = widen(x, ((b * L + t) * H + h) * P + p, is_bf16);
+        double acc = 0.0;
+        for (int64_t n = 0; n < N; ++n) {
+          const double bn = widen(Bm, (b * L + t) * N + n, is_bf16);
+          S[p * N + n] = a * S[p * N + n] + delta * bn * xv;
+          acc += widen(Cm, (b * L + t) * N + n, is_bf16) * S[p * N + n];
+        }
+        y_out[(k * L + t) * P + p] = acc + Dh * xv;
+      }
+    }
+    memcpy(h_last_out + k * P * N, S, (size_t)(P * N) * sizeof(double));
+  }
+  free(S);
+  return 0;
+}

@@ -563,6 +563,107 @@ def pin_conv_update_steps_equal_conv(o):
             _close(out, full[:, t], 1e-14, 1e-15, what=f"conv step {t} width {width}")
 
 
+def _ssd_case(seed, batch=2, L=10, H=3, P=4, N=5, h0=True):
+    r = _rng(seed)
+    return dict(
+        x=_f32(r.standard_normal((batch, L, H, P))),
+        dt=_f32(0.5 * r.standard_normal((batch, L, H))),
+        A=_f32(-r.uniform(0.5, 4.0, H)),
+        B=_f32(r.standard_normal((batch, L, N))),
+        C=_f32(r.standard_normal((batch, L, N))),
+        D=_f32(r.standard_normal(H)),
+        dt_bias=_f32(np.log(np.expm1(r.uniform(0.05, 0.5, H)))),
+        h0=_f32(r.standard_normal((batch, H, P, N))) if h0 else None,
+    )
+
+
+def _ssd(o, c, **kw):
+    return o.ssd_scan(c["x"], c["dt"], c["A"], c["B"], c["C"], D=c["D"], dt_bias=c["dt_bias"],
+                      h0=c["h0"], **kw)
+
+
+def pin_ssd_dual_matrix_form(o):
+    """The SSD output against §4.1's dual form, brute force: per head,
+    Y = (T . M) X with T the causal mask and the semi-separable
+    M_ts = (C_t . B_s) [prod_{s<r<=t} exp(Delta_r A)] Delta_s, plus the
+    initial state's term C_t (prod_{r<=t} exp(Delta_r A)) h0 and D x_t."""
+    c = _ssd_case(301)
+    y, _ = _ssd(o, c)
+    batch, L, H, P = c["x"].shape
+    dt = _softplus_lib(c["dt"].astype(np.float64) + c["dt_bias"].astype(np.float64))
+    want = np.zeros((batch, L, H, P))
+    for b in range(batch):
+        for h in range(H):
+            a = np.exp(dt[b, :, h] * float(c["A"][h]))
+            M = np.zeros((L, L))
+            for t in range(L):
+                for s in range(t + 1):
+                    decay = 1.0
+                    for r in range(s + 1, t + 1):
+                        decay *= a[r]
+                    M[t, s] = float(np.dot(c["C"][b, t].astype(np.float64),
+                                           c["B"][b, s].astype(np.float64))) * decay * dt[b, s, h]
+            X = c["x"][b, :, h].astype(np.float64)
+            Y = M @ X
+            for t in range(L):
+                decay = np.prod(a[: t + 1])
+                Y[t] += decay * (c["h0"][b, h].astype(np.float64) @ c["C"][b, t].astype(np.float64))
+            want[b, :, h] = Y + float(c["D"][h]) * X
+    _close(y, want, 1e-11, 1e-12, what="ssd dual form")
+
+
+def pin_ssd_is_tied_selective_scan(o):
+    """An SSD head is the selective scan over its headdim channels with A
+    tied across states (A[d,n] = A[h]) and Delta, D, bias tied across the
+    head's channels: the multi-head form against the separately pinned
+    per-channel scan."""
+    c = _ssd_case(303, batch=2, L=11, H=3, P=4, N=5)
+    y, hl = _ssd(o, c)
+    batch, L, H, P = c["x"].shape
+    N = c["B"].shape[-1]
+    dim = H * P
+    tie = lambda v: np.repeat(v, P, axis=-1)  # noqa: E731  head value -> its channels
+    ys, hs = o.selective_scan(c["x"].reshape(batch, L, dim), tie(c["dt"]),
+                              np.repeat(tie(c["A"])[:, None], N, axis=1), c["B"], c["C"],
+                              D=tie(c["D"]), delta_bias=tie(c["dt_bias"]),
+                              h0=c["h0"].reshape(batch, dim, N))
+    _close(y, ys.reshape(batch, L, H, P), 1e-13, 1e-13, what="ssd vs tied scan y")
+    _close(hl, hs.reshape(batch, H, P, N), 1e-13, 1e-13, what="ssd vs tied scan h")
+
+
+def pin_ssd_A_zero_is_cumulative_outer_product(o):
+    """A = 0, Delta = 1 (no softplus): the state is the running sum of the
+    outer products x_s B_s^T (linear attention), y_t = S_t C_t; computed with
+    the library cumulative sum."""
+    c = _ssd_case(305, h0=False)
+    batch, L, H, P = c["x"].shape
+    y, hl = o.ssd_scan(c["x"], np.ones((batch, L, H), np.float32), np.zeros(H, np.float32),
+                       c["B"], c["C"], softplus=False)
+    outer = np.einsum("blhp,bln->blhpn", c["x"].astype(np.float64), c["B"].astype(np.float64))
+    S = np.cumsum(outer, axis=1)
+    _close(y, np.einsum("blhpn,bln->blhp", S, c["C"].astype(np.float64)), 1e-12, 1e-12,
+           what="ssd A=0 y")
+    _close(hl, S[:, -1], 1e-12, 1e-12, what="ssd A=0 h")
+
+
+def pin_ssd_split_invariance(o):
+    """Running the first k steps, then the rest from the state reached,
+    equals one run (the state carries everything)."""
+    c = _ssd_case(307, L=13)
+    y, hl = _ssd(o, c)
+    k = 6
+    first = {key: (v[:, :k] if key in ("x", "dt", "B", "C") else v) for key, v in c.items()}
+    y1, h1 = _ssd(o, first)
+    second = {key: (np.ascontiguousarray(v[:, k:]) if key in ("x", "dt", "B", "C") else v)
+              for key, v in c.items()}
+    second["h0"] = h1.astype(np.float32)
+    y2, h2 = _ssd(o, second)
+    _close(y1, y[:, :k], 1e-14, 1e-15, what="ssd first part")
+    # the carried state is rounded to fp32 for the second run
+    _close(y2, y[:, k:], 1e-6, 1e-6, what="ssd second part")
+    _close(h2, hl, 1e-6, 1e-6, what="ssd end state")
+
+
 ALL_PINS = [
     pin_softplus_library,
     pin_silu_library,
@@ -588,4 +689,8 @@ ALL_PINS = [
     pin_zoh_matches_scipy_cont2discrete,
     pin_zoh_small_step_is_euler,
     pin_zoh_decode_steps_equal_scan,
+    pin_ssd_dual_matrix_form,
+    pin_ssd_is_tied_selective_scan,
+    pin_ssd_A_zero_is_cumulative_outer_product,
+    pin_ssd_split_invariance,
 ]

@@ -79,3 +79,25 @@ def test_decode_steps_equal_the_scan():
                               delta_bias=dev(inp["delta_bias"]))
         assert rel_err(host(yt), host(y)[:, t]) <= 1e-5
     assert rel_err(host(state), host(hl)) <= 1e-5
+
+
+@pytest.mark.parametrize("N,batch,dim", [(8, 80, 4001), (64, 11, 3791)])
+def test_decode_large_ragged(N, batch, dim):
+    """Large grids (over 600k threads) with a ragged last block: every output
+    and state element against the oracle."""
+    from selective_state_space_39_b200 import ssm_state_update
+    seed = 40 + N
+    const = gen.decode_constants(dim, N, seed)
+    rng = np.random.default_rng(seed)
+    A = (-rng.uniform(0.2, 3.0, (dim, N))).astype(np.float32)
+    state = torch.from_numpy(rng.standard_normal((batch, dim, N)).astype(np.float32)).cuda()
+    ref = host(state).copy()
+    for step in range(3):
+        inp = gen.make_decode_inputs(batch, dim, N, "bf16", seed, step)
+        kw = dict(D=const["D"], z=inp["z"], delta_bias=const["delta_bias"])
+        y = ssm_state_update(state, dev(inp["x"]), dev(inp["delta"]), dev(A), dev(inp["B"]),
+                             dev(inp["C"]), **{k: dev(v) for k, v in kw.items()})
+        yr = oracle.state_update(ref, inp["x"], inp["delta"], A, inp["B"], inp["C"], io="bf16",
+                                 **kw)
+        assert rel_err(host(y), yr) <= TOL["bf16"], f"step {step}"
+    assert rel_err(host(state), ref) <= TOL["bf16"]

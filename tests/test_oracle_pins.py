@@ -106,6 +106,24 @@ MUTANTS = {
     "zoh_is_euler": ("  return An == 0.0 ? dt : expm1(dt * An) / An;", "  return dt;"),
     "zoh_no_division_by_A": ("  return An == 0.0 ? dt : expm1(dt * An) / An;",
                              "  return An == 0.0 ? dt : expm1(dt * An);"),
+    # Mamba-2 SSD
+    "ssd_readout_before_update": (
+        "          S[p * N + n] = a * S[p * N + n] + delta * bn * xv;\n          acc += widen(Cm, (b * L + t) * N + n, is_bf16) * S[p * N + n];",
+        "          acc += widen(Cm, (b * L + t) * N + n, is_bf16) * S[p * N + n];\n          S[p * N + n] = a * S[p * N + n] + delta * bn * xv;"),
+    "ssd_B_C_swapped": ("const double bn = widen(Bm, (b * L + t) * N + n, is_bf16);",
+                        "const double bn = widen(Cm, (b * L + t) * N + n, is_bf16);"),
+    "ssd_bias_dropped": ("const double v = widen(dt, (b * L + t) * H + h, is_bf16) + bias;",
+                         "const double v = widen(dt, (b * L + t) * H + h, is_bf16);"),
+    "ssd_skip_dropped": ("y_out[(k * L + t) * P + p] = acc + Dh * xv;",
+                         "y_out[(k * L + t) * P + p] = acc;"),
+    "ssd_h0_ignored": ("S[p * N + n] = h0 ? (double)h0[((b * H + h) * P + p) * N + n] : 0.0;",
+                       "S[p * N + n] = 0.0;"),
+    "ssd_input_without_delta": ("S[p * N + n] = a * S[p * N + n] + delta * bn * xv;",
+                                "S[p * N + n] = a * S[p * N + n] + bn * xv;"),
+    "ssd_sign_of_A": ("const double a = exp(delta * (double)A[h]);",
+                      "const double a = exp(-delta * (double)A[h]);"),
+    "ssd_x_of_head_zero": ("const double xv = widen(x, ((b * L + t) * H + h) * P + p, is_bf16);",
+                           "const double xv = widen(x, ((b * L + t) * H + 0) * P + p, is_bf16);"),
     "zoh_sign_flipped": ("  return An == 0.0 ? dt : expm1(dt * An) / An;",
                          "  return An == 0.0 ? dt : -expm1(dt * An) / An;"),
 }
