@@ -11,6 +11,7 @@ the time is the max over ranks.
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
   python bench.py --pass bwd [--workload NAME]  # the backward pass (gradients)
   python bench.py --op conv [--workload NAME]   # the block's causal conv1d + SiLU
+  python bench.py --op ssd [--workload NAME]    # the multi-head SSD scan (Mamba-2)
   python bench.py --impl reference ...   # the fp64 CPU oracle on host cores
 """
 from __future__ import annotations
@@ -45,7 +46,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
-                    choices=sorted(gen.SCAN_WORKLOADS) + sorted(gen.DECODE_WORKLOADS))
+                    choices=sorted(gen.SCAN_WORKLOADS) + sorted(gen.DECODE_WORKLOADS) +
+                    sorted(gen.SSD_WORKLOADS))
     ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd"],
                     help="bwd: time ssm_scan_bwd (the gradients) on the same workload")
     ap.add_argument("--learned-a", action="store_true",
@@ -53,9 +55,10 @@ def parse_args():
                          "one-exp-per-state path")
     ap.add_argument("--zoh", action="store_true",
                     help="scan with the exact zero-order-hold input term (ssm_scan_fwd_zoh)")
-    ap.add_argument("--op", default="scan", choices=["scan", "conv"],
+    ap.add_argument("--op", default="scan", choices=["scan", "conv", "ssd"],
                     help="conv: time the block's causal conv1d + SiLU (forward and backward) "
-                         "on the workload's (batch, seqlen, dim)")
+                         "on the workload's (batch, seqlen, dim); ssd: the multi-head SSD scan "
+                         "(default workload " + "ssd_mamba2_b4_l4096_h64_p64_n128)")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
@@ -99,6 +102,18 @@ def measured_traffic(workload):
         return t["workloads"].get(workload, {}).get("per_call")
     except Exception:
         return None
+
+
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def measured_bf16_peak():
+    """Dense bf16 tensor peak: the burst figure (a kernel timed alone)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
 
 
 def measured_hbm_peak():
@@ -571,10 +586,198 @@ def conv_bench(args):
     return 0
 
 
+SSD_METRIC = "SSD scan elements/s (B·L·H·P) with tensor-core TFLOP/s and HBM GB/s"
+DEFAULT_SSD_WORKLOAD = "ssd_mamba2_b4_l4096_h64_p64_n128"
+
+
+def ssd_cost(w):
+    """Algorithmic bytes and FLOPs of one SSD call. Bytes: x read and y written
+    (bf16), B, C, dt read, h0 read and h_last written (fp32). FLOPs: the
+    chunked dual form's products per (batch, head, chunk of Q): G X over the
+    causal half (Q^2 P), C H and the state's (w X)^T B (2 Q N P each), and
+    C B^T over the causal half (Q^2 N), once per chunk (B and C are shared by
+    the heads)."""
+    Q, P, N = 32, w.headdim, w.dstate
+    tok = w.batch * w.seqlen
+    nbytes = 2 * 2 * tok * w.nheads * P + 2 * 2 * tok * N + 2 * tok * w.nheads + \
+        4 * w.batch * w.nheads * P * N * (2 if w.with_h0 else 1)
+    flops = tok * w.nheads * (Q * P + 4 * N * P) + tok * Q * N
+    return nbytes, flops
+
+
+def cpu_oracle_ssd_rate(w, inp, target_s, rng_seed=0):
+    """Oracle throughput (elements/s) on a bounded sample of (batch, head)
+    pairs (single host thread). Returns (value, cores, sample text)."""
+    import oracle
+    rng = np.random.default_rng(rng_seed)
+    pairs_all = [(b, h) for b in range(w.batch) for h in range(w.nheads)]
+
+    def run(n):
+        idx = rng.choice(len(pairs_all), size=min(n, len(pairs_all)), replace=False)
+        t0 = time.perf_counter()
+        oracle.ssd_scan(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], D=inp["D"],
+                        dt_bias=inp["dt_bias"], h0=inp["h0"], io=w.io,
+                        pairs=[pairs_all[i] for i in idx])
+        return len(idx), time.perf_counter() - t0
+
+    n, dt = run(1)
+    n2 = int(max(1, min(len(pairs_all), target_s / max(dt, 1e-9))))
+    n, dt = run(n2)
+    return (n * w.seqlen * w.headdim / dt, 1,
+            f"{n} of {len(pairs_all)} (batch, head) pairs x {w.seqlen} steps, {dt:.1f} s")
+
+
+def ssd_bench(args):
+    """--op ssd / --workload ssd_*: the multi-head SSD scan (ssm_ssd_scan_fwd,
+    one launch per step), one GPU, L2 flushed (256 MB write) before every
+    timed call. e2e: pinned host inputs copied in, y and h_last copied out,
+    every step, through the Python entry point."""
+    import torch
+
+    from selective_state_space_39_b200 import ssm_ssd_scan_fwd
+    w = gen.SSD_WORKLOADS[args.workload]
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    inp = gen.ssd_workload_inputs(w)
+
+    def to_host(a):
+        if a is None:
+            return None
+        t = torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16) \
+            if a.dtype == np.uint16 else torch.from_numpy(np.ascontiguousarray(a))
+        return t.pin_memory()
+
+    h = {k: to_host(v) for k, v in inp.items()}
+    d = {k: (v.to(device) if v is not None else None) for k, v in h.items()}
+    P, N = w.headdim, w.dstate
+    y = torch.empty((w.batch, w.seqlen, w.nheads, P), dtype=torch.bfloat16, device=device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    def call():
+        return ssm_ssd_scan_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], D=d["D"],
+                                dt_bias=d["dt_bias"], h0=d["h0"], return_last_state=True, y=y)
+
+    for _ in range(max(3, args.warmup)):
+        flush.fill_(1)
+        call()
+    torch.cuda.synchronize()
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    sampler = ClockSampler(0)
+    with sampler:
+        for i in range(K):
+            flush.fill_(i & 0xFF)
+            ev[i][0].record()
+            call()
+            ev[i][1].record()
+        torch.cuda.synchronize()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+
+    # end to end: host -> device inputs, the call, device -> host outputs
+    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    hl_host = torch.empty((w.batch, w.nheads, P, N), dtype=torch.float32).pin_memory()
+    keys = [k for k in ("x", "dt", "B", "C", "h0") if h[k] is not None]
+    h2d = sum(h[k].numel() * h[k].element_size() for k in keys)
+    d2h = y_host.numel() * 2 + hl_host.numel() * 4
+    E = max(3, args.e2e_steps)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(E):
+        for k in keys:
+            d[k].copy_(h[k], non_blocking=True)
+        _, hl = call()
+        y_host.copy_(y, non_blocking=True)
+        hl_host.copy_(hl, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / E
+
+    elems = w.elements
+    nbytes, flops = ssd_cost(w)
+    hbm_peak, hbm_kind = measured_hbm_peak()
+    tc_peak, tc_kind = measured_bf16_peak()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    tfs = flops / (ms * 1e-3) / 1e12
+    # the roofline bound is the larger of the two floors
+    t_hbm, t_tc = nbytes / (hbm_peak * 1e9), flops / (tc_peak * 1e12)
+    if t_hbm >= t_tc:
+        roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                "frac": round(gbs / hbm_peak, 4), "peak_kind": hbm_kind}
+    else:
+        roof = {"bound": "tensor", "achieved": round(tfs, 1), "peak": tc_peak,
+                "unit": "TFLOP/s", "frac": round(tfs / tc_peak, 4), "peak_kind": tc_kind}
+    roof.update({"traffic": None, "kernel": f"ssd_fwd_kernel<{N}> (1 launch)",
+                 "algorithmic_bytes_per_launch": nbytes, "algorithmic_flops_per_launch": flops,
+                 "tensor": {"achieved_tflops": round(tfs, 1), "peak": tc_peak,
+                            "frac": round(tfs / tc_peak, 4), "peak_kind": tc_kind},
+                 "hbm": {"achieved_gbs": round(gbs, 1), "peak": hbm_peak,
+                         "frac": round(gbs / hbm_peak, 4), "peak_kind": hbm_kind}})
+    line = {
+        "metric": SSD_METRIC, "value": elems / (ms * 1e-3), "unit": "elements/s", "n_gpus": 1,
+        "steps": K, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded Philox4x32-10; x, B, C N(0,1), dt N(0,0.25), A -U[1,16])",
+        "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen,
+                   "nheads": w.nheads, "headdim": P, "dstate": N, "io": w.io,
+                   "h0": w.with_h0, "l2": "flushed (256 MB write) before every timed call"},
+        "roofline": roof,
+        "e2e": {"value": elems / (e2e_ms * 1e-3), "unit": "elements/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": K, "clocks": sampler.summary(),
+    }
+    if not args.no_cpu_baseline:
+        v, cores, sample = cpu_oracle_ssd_rate(w, inp, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": v, "unit": "elements/s", "cores": cores,
+                                "kind": "oracle", "sample": sample}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def ssd_reference_arm(args):
+    """--impl reference on an SSD workload: the fp64 oracle, one (batch, head)
+    pair per step, on the host (rank 0 only)."""
+    import oracle
+    w = gen.SSD_WORKLOADS[args.workload]
+    inp = gen.ssd_workload_inputs(w)
+    rng = np.random.default_rng(1)
+    times = []
+    for i in range(args.warmup + args.steps):
+        pair = (int(rng.integers(w.batch)), int(rng.integers(w.nheads)))
+        t0 = time.perf_counter()
+        oracle.ssd_scan(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], D=inp["D"],
+                        dt_bias=inp["dt_bias"], h0=inp["h0"], io=w.io, pairs=[pair])
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = args.steps * w.seqlen * w.headdim / total
+    sample = f"1 random (batch, head) pair x {w.seqlen} steps per step"
+    line = {
+        "impl": "reference", "metric": SSD_METRIC, "value": value, "unit": "elements/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen,
+                   "nheads": w.nheads, "headdim": w.headdim, "dstate": w.dstate, "io": w.io},
+        "cpu_baseline": {"value": value, "unit": "elements/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "elements/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
+    if args.op == "ssd" and args.workload not in gen.SSD_WORKLOADS:
+        args.workload = DEFAULT_SSD_WORKLOAD
     if args.impl == "reference":
+        if args.workload in gen.SSD_WORKLOADS:
+            return ssd_reference_arm(args) if int(os.environ.get("RANK", 0)) == 0 else 0
         return reference_arm(args)
+    if args.workload in gen.SSD_WORKLOADS:
+        return ssd_bench(args)
     if args.workload in gen.DECODE_WORKLOADS:
         return decode_bench(args)
     if args.op == "conv":

@@ -326,6 +326,35 @@ int ssm_compose_carries(int64_t rank, int64_t batch, int64_t dim, int64_t dstate
                         float* h_in, void* stream);
 
 /*
+ * ssm_ssd_scan_fwd -- the multi-head SSD scan of Mamba-2 (same page, §4.1
+ * State Space Duality: the SSM as a semi-separable matrix, and §4.2:
+ * multi-head, state 64 to 256). Head h (width headdim) has one scalar A[h]
+ * and one step per token; B and C are shared by every head. Per batch b,
+ * head h, with the head's state S (headdim x dstate, fp32):
+ *
+ *   Delta        = softplus(dt[b,t,h] + dt_bias[h])   (or no softplus)
+ *   S[p][n]      = exp(Delta * A[h]) * S[p][n] + Delta * B[b,t,n] * x[b,t,h,p]
+ *   y[b,t,h,p]   = sum_n C[b,t,n] * S[p][n] + D[h] * x[b,t,h,p]
+ *
+ * starting from h0[b,h] (or zero) and ending in h_last[b,h]. Computed chunk
+ * by chunk on the tensor cores (bf16 operands, fp32 accumulation and state).
+ *   x, y     : (batch, seqlen, nheads, headdim) bf16 (io_dtype must be
+ *              SSM_DTYPE_BF16); y must not overlap an input
+ *   dt       : (batch, seqlen, nheads) bf16
+ *   B, C     : (batch, seqlen, dstate) bf16
+ *   A        : (nheads) fp32;  D, dt_bias : (nheads) fp32, nullable
+ *   h0       : (batch, nheads, headdim, dstate) fp32, nullable (zero)
+ *   h_last   : (batch, nheads, headdim, dstate) fp32, nullable (not written)
+ * headdim must be 64 and dstate 64, 128 or 256 (else SSM_ERR_UNSUPPORTED).
+ * x, B, C and y 16-byte aligned, h0 / h_last 8-byte aligned.
+ * Returns SSM_OK or SSM_ERR_*.
+ */
+int ssm_ssd_scan_fwd(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim,
+                     int64_t dstate, int io_dtype, const void* x, const void* dt, const float* A,
+                     const void* B, const void* C, const float* D, const float* dt_bias,
+                     int softplus, const float* h0, void* y, float* h_last, void* stream);
+
+/*
  * ssm_scan_status -- synchronise `stream`, then report whether every CTA of
  * the last ssm_scan_fwd call that used this workspace (with these sizes)
  * finished normally: SSM_OK, or SSM_ERR_TIMEOUT if a bounded wait inside a

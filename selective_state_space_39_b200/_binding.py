@@ -104,6 +104,9 @@ def lib() -> ctypes.CDLL:
         L.ssm_compose_carries.argtypes = [_I64, _I64, _I64, _I64, _VP, _VP, _VP, _VP, _VP, _VP]
         L.ssm_state_update_zoh.restype = ctypes.c_int
         L.ssm_state_update_zoh.argtypes = L.ssm_state_update.argtypes
+        L.ssm_ssd_scan_fwd.restype = ctypes.c_int
+        L.ssm_ssd_scan_fwd.argtypes = [_I64] * 5 + [ctypes.c_int] + [_VP] * 7 + \
+            [ctypes.c_int, _VP, _VP, _VP, _VP]
         _lib = L
     return _lib
 
@@ -466,3 +469,39 @@ def ssm_state_update(state, x, delta, A, B, C, D=None, z=None, delta_bias=None, 
     if rc != 0:
         raise SsmError(rc, "ssm_state_update_zoh" if zoh else "ssm_state_update")
     return y
+
+
+def ssm_ssd_scan_fwd(x, dt, A, B, C, D=None, dt_bias=None, softplus=True, h0=None,
+                     return_last_state=False, y=None, stream=None):
+    """The multi-head SSD scan through ssm_ssd_scan_fwd of libssmscan.so:
+    x (batch, L, heads, headdim) bf16, dt (batch, L, heads) bf16, A (heads,)
+    fp32, B, C (batch, L, dstate) bf16, D and dt_bias (heads,) fp32 or None,
+    h0 (batch, heads, headdim, dstate) fp32 or None. Returns y (and h_last
+    with ``return_last_state``)."""
+    if x.dim() != 4:
+        raise ValueError("x must be (batch, seqlen, heads, headdim)")
+    batch, L, H, P = x.shape
+    N = B.shape[-1]
+    dev = x.device
+    io = _io_code(x.dtype)
+    px = _ptr(x, "x", x.dtype)
+    pdt = _ptr(dt, "dt", x.dtype, (batch, L, H), dev)
+    pA = _ptr(A, "A", torch.float32, (H,), dev)
+    pB = _ptr(B, "B", x.dtype, (batch, L, N), dev)
+    pC = _ptr(C, "C", x.dtype, (batch, L, N), dev)
+    pD = _ptr(D, "D", torch.float32, (H,), dev)
+    pbias = _ptr(dt_bias, "dt_bias", torch.float32, (H,), dev)
+    ph0 = _ptr(h0, "h0", torch.float32, (batch, H, P, N), dev)
+    if y is None:
+        y = torch.empty((batch, L, H, P), dtype=x.dtype, device=dev)
+    py = _ptr(y, "y", x.dtype, (batch, L, H, P), dev)
+    h_last = (torch.empty((batch, H, P, N), dtype=torch.float32, device=dev)
+              if return_last_state else None)
+    ph = _ptr(h_last, "h_last")
+    with torch.cuda.device(dev):
+        rc = lib().ssm_ssd_scan_fwd(batch, L, H, P, N, io, px, pdt, pA, pB, pC, pD, pbias,
+                                    1 if softplus else 0, ph0, py, ph, _stream_ptr(stream, dev))
+    if rc != 0:
+        raise SsmError(rc, "ssm_ssd_scan_fwd", with_detail=True)
+    return (y, h_last) if return_last_state else y
+

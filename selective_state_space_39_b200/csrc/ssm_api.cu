@@ -13,6 +13,7 @@
 #include "ssm_bwd_internal.h"
 #include "ssm_conv_internal.h"
 #include "ssm_seqpar_internal.h"
+#include "ssm_ssd_internal.h"
 #include "ssm_internal.h"
 
 namespace ssm {
@@ -636,6 +637,54 @@ int ssm_conv1d_silu_update(int64_t batch, int64_t dim, int64_t width, int io_dty
   return cuda_status(launch_conv_update(p, io_dtype == SSM_DTYPE_BF16,
                                         static_cast<cudaStream_t>(stream)),
                      "conv1d update launch");
+}
+
+int ssm_ssd_scan_fwd(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim,
+                     int64_t dstate, int io_dtype, const void* x, const void* dt, const float* A,
+                     const void* B, const void* C, const float* D, const float* dt_bias,
+                     int softplus, const float* h0, void* y, float* h_last, void* stream) {
+  if (io_dtype != SSM_DTYPE_F32 && io_dtype != SSM_DTYPE_BF16) return SSM_ERR_INVALID_ARG;
+  if (batch < 0 || seqlen < 0 || nheads < 0 || headdim <= 0 || dstate <= 0)
+    return SSM_ERR_INVALID_ARG;
+  if (io_dtype != SSM_DTYPE_BF16 || headdim != kSsdHeadDim ||
+      !ssd_dstate_supported((int)std::min<int64_t>(dstate, 1 << 20)))
+    return fail(SSM_ERR_UNSUPPORTED, "ssm_ssd_scan_fwd: bf16 io, headdim 64 and dstate 64, "
+                                     "128 or 256 only");
+  if (batch > 65535 || nheads > (1 << 20) || seqlen > (1 << 30)) return SSM_ERR_UNSUPPORTED;
+  if (batch == 0 || nheads == 0) return SSM_OK;
+  if (!A) return SSM_ERR_INVALID_ARG;
+  if (seqlen > 0 && (!x || !dt || !B || !C || !y)) return SSM_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(y, 16) ||
+      !aligned(dt, 2) || !aligned(A, 4) || (D && !aligned(D, 4)) ||
+      (dt_bias && !aligned(dt_bias, 4)) || (h0 && !aligned(h0, 8)) ||
+      (h_last && !aligned(h_last, 8)))
+    return fail(SSM_ERR_INVALID_ARG, "ssm_ssd_scan_fwd: misaligned pointer");
+  const size_t nx = (size_t)batch * seqlen * nheads * headdim * 2;
+  const size_t nbc = (size_t)batch * seqlen * dstate * 2;
+  const size_t ndt = (size_t)batch * seqlen * nheads * 2;
+  const size_t nh = (size_t)batch * nheads * headdim * dstate * 4;
+  if (overlap(y, nx, x, nx) || overlap(y, nx, dt, ndt) || overlap(y, nx, B, nbc) ||
+      overlap(y, nx, C, nbc) || overlap(y, nx, h_last, nh) || overlap(h_last, nh, x, nx) ||
+      overlap(h_last, nh, B, nbc) || overlap(h_last, nh, C, nbc) ||
+      (h_last != h0 && overlap(h_last, nh, h0, nh)))
+    return fail(SSM_ERR_INVALID_ARG, "ssm_ssd_scan_fwd: buffers overlap");
+  SsdParams p{};
+  p.batch = (int)batch;
+  p.nheads = (int)nheads;
+  p.dstate = (int)dstate;
+  p.seqlen = seqlen;
+  p.softplus = softplus ? 1 : 0;
+  p.x = static_cast<const uint16_t*>(x);
+  p.dt = static_cast<const uint16_t*>(dt);
+  p.B = static_cast<const uint16_t*>(B);
+  p.C = static_cast<const uint16_t*>(C);
+  p.A = A;
+  p.D = D;
+  p.dt_bias = dt_bias;
+  p.h0 = h0;
+  p.y = static_cast<uint16_t*>(y);
+  p.h_last = h_last;
+  return cuda_status(launch_ssd_fwd(p, static_cast<cudaStream_t>(stream)), "ssd scan launch");
 }
 
 size_t ssm_conv1d_silu_bwd_workspace_bytes(int64_t batch, int64_t seqlen, int64_t dim,

@@ -1,0 +1,377 @@
+// ssm_ssd.cu -- sm_100a kernel of the multi-head SSD scan (Mamba-2).
+//
+// Page "Mamba 논문 리뷰: Selective State Space Models로 Transformer를 넘어서"
+// (youngju.dev), §4.1 State Space Duality and §4.2 (multi-head, larger
+// state). A head h of width P = 64 has one scalar A[h] and one step
+// Delta_t = softplus(dt[b,t,h] + dt_bias[h]) per token; B_t and C_t (N wide)
+// are shared by the heads. With a_t = exp(Delta_t A[h]) the head's output is
+// the semi-separable matrix of §4.1 acting on its inputs,
+//   y_t = sum_{s<=t} (C_t . B_s) [prod_{s<r<=t} a_r] Delta_s x_s + D[h] x_t,
+// which the kernel evaluates chunk by chunk (Q = 32 steps), walking the
+// chunks of one (batch, head) in order and carrying the N x P state H in fp32
+// registers. With cum_t = sum_{r<=t} Delta_r A[h] inside the chunk:
+//   G[t][s] = (C_t . B_s) e^{cum_t - cum_s} Delta_s   (s <= t, else 0)
+//   Y       = G X + diag(e^{cum}) C H + D X
+//   H      <- e^{cum_end} H + (w X)^T B,   w_s = e^{cum_end - cum_s} Delta_s
+// The four products (C B^T, G X, C H, (w X)^T B) are bf16 tensor-core MMAs
+// (mma.sync m16n8k16, fp32 accumulation) fed from shared memory by ldmatrix;
+// x, B and C chunks are double-buffered with cp.async (zero-filled past the
+// end of the sequence, where Delta is taken as 0 so that the padded steps
+// change nothing).
+#include <mutex>
+#include <set>
+#include <utility>
+
+#include "ssm_device.cuh"
+#include "ssm_ssd_internal.h"
+
+namespace ssm {
+
+namespace {
+
+constexpr int kQ = kSsdChunk;    // steps per chunk
+constexpr int kP = kSsdHeadDim;  // head width
+constexpr int kThreads = 256;    // 8 warps
+constexpr int kPadX = kP + 8;    // shared row of an x chunk (elements; 16-byte skew)
+constexpr int kPadG = kQ + 8;    // shared row of G
+
+static_assert(kQ == 32, "the in-chunk cumulative sum is one warp's scan");
+
+template <int N>
+struct SsdLayout {
+  static constexpr int kPadN = N + 8;
+  static constexpr int x_elems = 2 * kQ * kPadX;   // two buffers
+  static constexpr int bc_elems = 2 * kQ * kPadN;  // two buffers each for B and C
+  static constexpr int g_elems = kQ * kPadG;
+  static constexpr int h_elems = kP * kPadN;
+  static constexpr int bf16_bytes = 2 * (x_elems + 2 * bc_elems + g_elems + h_elems);
+  static constexpr int bytes = bf16_bytes + 4 * (4 * kQ + 4);
+  static_assert(bf16_bytes % 16 == 0, "float arrays start 16-byte aligned");
+};
+
+// ------------------------------------------------------------ PTX wrappers --
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1,
+                                          uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+// d += a (16x16, row) * b (16x8, col), bf16 operands, fp32 accumulators.
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// 16-byte asynchronous copy; with valid == false nothing is read and the
+// destination is zero-filled.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(valid ? 16 : 0));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;"); }
+__device__ __forceinline__ void cp_async_wait_prev() {
+  asm volatile("cp.async.wait_group 1;" ::: "memory");
+}
+// Both halves of a bf16 pair times their own weight, repacked.
+__device__ __forceinline__ uint32_t scale_bf16x2(uint32_t v, float lo, float hi) {
+  return pack_bf16x2(bf16_lo(v) * lo, bf16_hi(v) * hi);
+}
+
+// One CTA per (head, batch row). Warp w owns: rows 16*(w/4).. of S, G and Y;
+// columns 8*(w%4).. of S and G, 16*(w%4).. of Y; rows 16*(w%4).. (p) and
+// columns (w/4)*N/2.. (n) of the state.
+template <int N>
+__global__ void __launch_bounds__(kThreads, (N <= 128) ? 2 : 1) ssd_fwd_kernel(const SsdParams p) {
+  using Lay = SsdLayout<N>;
+  constexpr int kPadN = Lay::kPadN;
+  constexpr int kNW = N / 2;   // state columns per warp
+  constexpr int kNT = kNW / 8; // n8 tiles per warp
+  static_assert(kNT % 2 == 0, "state tiles come in pairs from one ldmatrix.x4");
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  uint16_t* Xs = reinterpret_cast<uint16_t*>(smem_raw);
+  uint16_t* Bs = Xs + Lay::x_elems;
+  uint16_t* Cs = Bs + Lay::bc_elems;
+  uint16_t* Gs = Cs + Lay::bc_elems;
+  uint16_t* Hs = Gs + Lay::g_elems;
+  float* s_dt = reinterpret_cast<float*>(smem_raw + Lay::bf16_bytes);  // Delta_s
+  float* s_cum = s_dt + kQ;                                            // cum_t
+  float* s_ecum = s_cum + kQ;                                          // e^{cum_t}
+  float* s_w = s_ecum + kQ;                                            // w_s
+  float* s_decay = s_w + kQ;                                           // e^{cum_end}
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, tig = lane & 3;
+  const int h = blockIdx.x, b = blockIdx.y;
+  const int H = p.nheads;
+  const int64_t L = p.seqlen;
+  const float Ah = p.A[h];
+  const float bias = p.dt_bias ? p.dt_bias[h] : 0.f;
+  const float Dh = p.D ? p.D[h] : 0.f;
+  const int nchunks = (int)((L + kQ - 1) / kQ);
+  const size_t row_x = (size_t)H * kP;  // elements between steps of x and y
+  const uint16_t* xg = p.x + ((size_t)b * L * H + h) * kP;
+  const uint16_t* Bg = p.B + (size_t)b * L * N;
+  const uint16_t* Cg = p.C + (size_t)b * L * N;
+  const uint16_t* dtg = p.dt + (size_t)b * L * H + h;
+  uint16_t* yg = p.y + ((size_t)b * L * H + h) * kP;
+
+  // ---- state tile in registers: hacc[j] = rows p0, p0 + 8; columns n_j, n_j + 1
+  const int pt = warp & 3, ng = warp >> 2;
+  const int p0 = 16 * pt + g;
+  float hacc[kNT][4];
+#pragma unroll
+  for (int j = 0; j < kNT; ++j) {
+    const int n = ng * kNW + 8 * j + 2 * tig;
+    if (p.h0) {
+      const float* src = p.h0 + (((size_t)b * H + h) * kP + p0) * N + n;
+      const float2 u = *reinterpret_cast<const float2*>(src);
+      const float2 v = *reinterpret_cast<const float2*>(src + 8 * N);
+      hacc[j][0] = u.x; hacc[j][1] = u.y; hacc[j][2] = v.x; hacc[j][3] = v.y;
+    } else {
+      hacc[j][0] = hacc[j][1] = hacc[j][2] = hacc[j][3] = 0.f;
+    }
+  }
+  auto store_state_bf16 = [&]() {
+#pragma unroll
+    for (int j = 0; j < kNT; ++j) {
+      const int n = ng * kNW + 8 * j + 2 * tig;
+      *reinterpret_cast<uint32_t*>(Hs + p0 * kPadN + n) = pack_bf16x2(hacc[j][0], hacc[j][1]);
+      *reinterpret_cast<uint32_t*>(Hs + (p0 + 8) * kPadN + n) =
+          pack_bf16x2(hacc[j][2], hacc[j][3]);
+    }
+  };
+  store_state_bf16();
+
+  // ---- chunk loader (x: kQ rows of 128 B; B, C: kQ rows of 2N B)
+  auto load_chunk = [&](int c, int buf) {
+    const int64_t t0 = (int64_t)c * kQ;
+    constexpr int kXPieces = kQ * kP / 8;
+    constexpr int kBPieces = kQ * N / 8;
+#pragma unroll
+    for (int i = tid; i < kXPieces; i += kThreads) {
+      const int r = i / (kP / 8), q = i % (kP / 8);
+      const bool ok = t0 + r < L;
+      const uint16_t* src = ok ? xg + (size_t)(t0 + r) * row_x + q * 8 : xg;
+      cp_async16(smem_u32(Xs + (buf * kQ + r) * kPadX + q * 8), src, ok);
+    }
+#pragma unroll
+    for (int i = tid; i < kBPieces; i += kThreads) {
+      const int r = i / (N / 8), q = i % (N / 8);
+      const bool ok = t0 + r < L;
+      const size_t off = ok ? (size_t)(t0 + r) * N + q * 8 : 0;
+      cp_async16(smem_u32(Bs + (buf * kQ + r) * kPadN + q * 8), Bg + off, ok);
+      cp_async16(smem_u32(Cs + (buf * kQ + r) * kPadN + q * 8), Cg + off, ok);
+    }
+  };
+
+  float dt_raw = 0.f;  // warp 0: raw step of the chunk about to run (lane = step)
+  if (nchunks > 0) {
+    load_chunk(0, 0);
+    cp_async_commit();
+    if (warp == 0 && lane < L) dt_raw = bf16_to_f32(dtg[(size_t)lane * H]);
+  }
+
+  for (int c = 0; c < nchunks; ++c) {
+    const int buf = c & 1;
+    const int64_t t0 = (int64_t)c * kQ;
+    if (c + 1 < nchunks) load_chunk(c + 1, buf ^ 1);
+    cp_async_commit();
+
+    // ---- steps, their in-chunk cumulative sum and the weights (warp 0)
+    if (warp == 0) {
+      float d = 0.f;
+      if (t0 + lane < L) {
+        const float v = dt_raw + bias;
+        d = p.softplus ? (v > kSoftplusCut ? v : log1pf(__expf(v))) : v;
+      }
+      const int64_t tn = t0 + kQ + lane;
+      dt_raw = tn < L ? bf16_to_f32(dtg[(size_t)tn * H]) : 0.f;
+      float cum = d * Ah;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float u = __shfl_up_sync(0xffffffffu, cum, o);
+        if (lane >= o) cum += u;
+      }
+      const float cend = __shfl_sync(0xffffffffu, cum, 31);
+      s_dt[lane] = d;
+      s_cum[lane] = cum;
+      s_ecum[lane] = __expf(cum);
+      s_w[lane] = __expf(cend - cum) * d;
+      if (lane == 0) s_decay[0] = __expf(cend);
+    }
+    cp_async_wait_prev();
+    __syncthreads();
+
+    const uint16_t* Xb = Xs + buf * kQ * kPadX;
+    const uint16_t* Bb = Bs + buf * kQ * kPadN;
+    const uint16_t* Cb = Cs + buf * kQ * kPadN;
+    const int rt = warp >> 2;  // row tile of S, G, Y
+    const int cq = warp & 3;   // column quarter
+
+    // ---- S = C B^T on this warp's 16 x 8 tile, then G (bf16) into shared
+    {
+      float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+      if (8 * cq <= 16 * rt + 15) {  // the tile holds entries with s <= t
+#pragma unroll
+        for (int k0 = 0; k0 < N; k0 += 32) {
+          uint32_t b0, b1, b2, b3, a0, a1, a2, a3;
+          ldsm_x4(smem_u32(Bb + (8 * cq + (lane & 7)) * kPadN + k0 + (lane >> 3) * 8), b0, b1,
+                  b2, b3);
+          ldsm_x4(smem_u32(Cb + (16 * rt + (lane & 15)) * kPadN + k0 + (lane >> 4) * 8), a0, a1,
+                  a2, a3);
+          mma_bf16(sacc, a0, a1, a2, a3, b0, b1);
+          ldsm_x4(smem_u32(Cb + (16 * rt + (lane & 15)) * kPadN + k0 + 16 + (lane >> 4) * 8), a0,
+                  a1, a2, a3);
+          mma_bf16(sacc, a0, a1, a2, a3, b2, b3);
+        }
+      }
+      const int ta = 16 * rt + g, tb = ta + 8, s0 = 8 * cq + 2 * tig;
+      const float cuma = s_cum[ta], cumb = s_cum[tb];
+      const float cs0 = s_cum[s0], cs1 = s_cum[s0 + 1];
+      const float d0 = s_dt[s0], d1 = s_dt[s0 + 1];
+      const float g0 = s0 <= ta ? sacc[0] * __expf(cuma - cs0) * d0 : 0.f;
+      const float g1 = s0 + 1 <= ta ? sacc[1] * __expf(cuma - cs1) * d1 : 0.f;
+      const float g2 = s0 <= tb ? sacc[2] * __expf(cumb - cs0) * d0 : 0.f;
+      const float g3 = s0 + 1 <= tb ? sacc[3] * __expf(cumb - cs1) * d1 : 0.f;
+      *reinterpret_cast<uint32_t*>(Gs + ta * kPadG + s0) = pack_bf16x2(g0, g1);
+      *reinterpret_cast<uint32_t*>(Gs + tb * kPadG + s0) = pack_bf16x2(g2, g3);
+    }
+    __syncthreads();
+
+    // ---- Y = G X + diag(e^cum) C H + D x on rows 16 rt.., columns 16 cq..
+    {
+      float y1[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      float y2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+      for (int k0 = 0; k0 < kQ; k0 += 16) {
+        if (k0 <= 16 * rt) {
+          uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
+          ldsm_x4(smem_u32(Gs + (16 * rt + (lane & 15)) * kPadG + k0 + (lane >> 4) * 8), a0, a1,
+                  a2, a3);
+          ldsm_x4_t(smem_u32(Xb + (k0 + (lane & 7) + ((lane >> 3) & 1) * 8) * kPadX + 16 * cq +
+                             (lane >> 4) * 8),
+                    b0, b1, b2, b3);
+          mma_bf16(y1[0], a0, a1, a2, a3, b0, b1);
+          mma_bf16(y1[1], a0, a1, a2, a3, b2, b3);
+        }
+      }
+#pragma unroll
+      for (int k0 = 0; k0 < N; k0 += 16) {
+        uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
+        ldsm_x4(smem_u32(Cb + (16 * rt + (lane & 15)) * kPadN + k0 + (lane >> 4) * 8), a0, a1,
+                a2, a3);
+        ldsm_x4(smem_u32(Hs + (16 * cq + (lane & 7) + (lane >> 4) * 8) * kPadN + k0 +
+                         ((lane >> 3) & 1) * 8),
+                b0, b1, b2, b3);
+        mma_bf16(y2[0], a0, a1, a2, a3, b0, b1);
+        mma_bf16(y2[1], a0, a1, a2, a3, b2, b3);
+      }
+      const int ta = 16 * rt + g, tb = ta + 8;
+      const float ea = s_ecum[ta], eb = s_ecum[tb];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int pc = 16 * cq + 8 * j + 2 * tig;
+        const uint32_t xa = *reinterpret_cast<const uint32_t*>(Xb + ta * kPadX + pc);
+        const uint32_t xb = *reinterpret_cast<const uint32_t*>(Xb + tb * kPadX + pc);
+        if (t0 + ta < L)
+          *reinterpret_cast<uint32_t*>(yg + (size_t)(t0 + ta) * row_x + pc) =
+              pack_bf16x2(fmaf(Dh, bf16_lo(xa), fmaf(ea, y2[j][0], y1[j][0])),
+                          fmaf(Dh, bf16_hi(xa), fmaf(ea, y2[j][1], y1[j][1])));
+        if (t0 + tb < L)
+          *reinterpret_cast<uint32_t*>(yg + (size_t)(t0 + tb) * row_x + pc) =
+              pack_bf16x2(fmaf(Dh, bf16_lo(xb), fmaf(eb, y2[j][2], y1[j][2])),
+                          fmaf(Dh, bf16_hi(xb), fmaf(eb, y2[j][3], y1[j][3])));
+      }
+    }
+
+    // ---- H <- e^{cum_end} H + (w X)^T B on rows 16 pt.. (p), columns ng N/2.. (n)
+    {
+      const float decay = s_decay[0];
+#pragma unroll
+      for (int j = 0; j < kNT; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) hacc[j][e] *= decay;
+#pragma unroll
+      for (int k0 = 0; k0 < kQ; k0 += 16) {
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4_t(smem_u32(Xb + (k0 + (lane & 7) + (lane >> 4) * 8) * kPadX + 16 * pt +
+                           ((lane >> 3) & 1) * 8),
+                  a0, a1, a2, a3);
+        const int s = k0 + 2 * tig;
+        const float w0 = s_w[s], w1 = s_w[s + 1], w8 = s_w[s + 8], w9 = s_w[s + 9];
+        a0 = scale_bf16x2(a0, w0, w1);
+        a1 = scale_bf16x2(a1, w0, w1);
+        a2 = scale_bf16x2(a2, w8, w9);
+        a3 = scale_bf16x2(a3, w8, w9);
+#pragma unroll
+        for (int j = 0; j < kNT; j += 2) {
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_t(smem_u32(Bb + (k0 + (lane & 7) + ((lane >> 3) & 1) * 8) * kPadN + ng * kNW +
+                             8 * j + (lane >> 4) * 8),
+                    b0, b1, b2, b3);
+          mma_bf16(hacc[j], a0, a1, a2, a3, b0, b1);
+          mma_bf16(hacc[j + 1], a0, a1, a2, a3, b2, b3);
+        }
+      }
+    }
+    __syncthreads();
+    store_state_bf16();
+  }
+
+  if (p.h_last) {
+#pragma unroll
+    for (int j = 0; j < kNT; ++j) {
+      const int n = ng * kNW + 8 * j + 2 * tig;
+      float* dst = p.h_last + (((size_t)b * H + h) * kP + p0) * N + n;
+      *reinterpret_cast<float2*>(dst) = make_float2(hacc[j][0], hacc[j][1]);
+      *reinterpret_cast<float2*>(dst + 8 * N) = make_float2(hacc[j][2], hacc[j][3]);
+    }
+  }
+}
+
+cudaError_t set_smem_once(const void* kernel, int smem) {
+  static std::mutex mu;
+  static std::set<std::pair<const void*, int>> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  if (done.count({kernel, dev})) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess) done.insert({kernel, dev});
+  return e;
+}
+
+template <int N>
+cudaError_t launch_n(const SsdParams& p, cudaStream_t stream) {
+  constexpr int smem = SsdLayout<N>::bytes;
+  cudaError_t e = set_smem_once(reinterpret_cast<const void*>(ssd_fwd_kernel<N>), smem);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((unsigned)p.nheads, (unsigned)p.batch);
+  ssd_fwd_kernel<N><<<grid, kThreads, smem, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool ssd_dstate_supported(int dstate) { return dstate == 64 || dstate == 128 || dstate == 256; }
+
+cudaError_t launch_ssd_fwd(const SsdParams& p, cudaStream_t stream) {
+  switch (p.dstate) {
+    case 64: return launch_n<64>(p, stream);
+    case 128: return launch_n<128>(p, stream);
+    case 256: return launch_n<256>(p, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace ssm

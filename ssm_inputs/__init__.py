@@ -42,6 +42,8 @@ STREAM_DY, STREAM_DH_LAST = 8, 9
 STREAM_CONV_X, STREAM_CONV_W, STREAM_CONV_BIAS, STREAM_CONV_DOUT = 10, 11, 12, 13
 # a learned-looking A (no (n + 1) A[d, 0] structure)
 STREAM_A_LEARNED = 14
+# Mamba-2 SSD: per-head A and step bias
+STREAM_SSD_A, STREAM_SSD_BIAS = 15, 16
 KIND_NORMAL, KIND_UNIFORM = 0, 1
 OUT_F64, OUT_F32, OUT_BF16 = 0, 1, 2
 
@@ -198,6 +200,33 @@ SCAN_WORKLOADS = {
         "pythia1b_layer_b4_l4096_d4096_h0", 4, 4096, 4096, 16, "bf16", 2, with_h0=True),
     "long_b1_l262144_d1536": ScanWorkload("long_b1_l262144_d1536", 1, 262144, 1536, 16, "bf16", 3),
 }
+@dataclass(frozen=True)
+class SsdWorkload:
+    name: str
+    batch: int
+    seqlen: int
+    nheads: int
+    headdim: int
+    dstate: int
+    io: str
+    seed: int
+    with_h0: bool = False
+
+    @property
+    def elements(self) -> int:
+        return self.batch * self.seqlen * self.nheads * self.headdim
+
+
+# The Mamba-2 layer of d_model 2048 (expand 2: 4096 channels = 64 heads of 64,
+# d_state 128): the pages' example input (1 x 1024) and the 4 x 4096 batch of
+# the 1B-scale scan.
+SSD_WORKLOADS = {
+    "ssd_mamba2_b1_l1024_h64_p64_n128": SsdWorkload(
+        "ssd_mamba2_b1_l1024_h64_p64_n128", 1, 1024, 64, 64, 128, "bf16", 5),
+    "ssd_mamba2_b4_l4096_h64_p64_n128": SsdWorkload(
+        "ssd_mamba2_b4_l4096_h64_p64_n128", 4, 4096, 64, 64, 128, "bf16", 6, with_h0=True),
+}
+
 DECODE_WORKLOADS = {
     "decode_b128_d4096_x1000": DecodeWorkload("decode_b128_d4096_x1000", 128, 4096, 16, "bf16", 4, 1000),
 }
@@ -276,6 +305,32 @@ def make_conv_inputs(batch, seqlen, dim, width, io, seed, *, nthreads=None):
         "bias": fill((dim,), seed, STREAM_CONV_BIAS, KIND_UNIFORM, -0.5, 0.5, out="f32"),
         "dout": fill(shape, seed, STREAM_CONV_DOUT, out=io, nthreads=nthreads),
     }
+
+
+def make_ssd_inputs(batch, seqlen, nheads, headdim, dstate, io, seed, *, with_h0=False,
+                    nthreads=None):
+    """Inputs of one multi-head SSD scan: x (batch, L, heads, headdim) ~ N(0, 1),
+    dt (batch, L, heads) ~ N(0, 0.5^2), B, C (batch, L, dstate) ~ N(0, 1), all
+    in the io type; per head A ~ -U[1, 16], dt_bias = log(expm1(U[0.001, 0.1])),
+    D = 1 (fp32); h0 (batch, heads, headdim, dstate) ~ N(0, 1) fp32 or None."""
+    return {
+        "x": fill((batch, seqlen, nheads, headdim), seed, STREAM_X, out=io, nthreads=nthreads),
+        "dt": fill((batch, seqlen, nheads), seed, STREAM_DELTA, b=0.5, out=io, nthreads=nthreads),
+        "B": fill((batch, seqlen, dstate), seed, STREAM_B, out=io, nthreads=nthreads),
+        "C": fill((batch, seqlen, dstate), seed, STREAM_C, out=io, nthreads=nthreads),
+        "A": (-fill((nheads,), seed, STREAM_SSD_A, KIND_UNIFORM, 1.0, 16.0, out="f64")).astype(
+            np.float32),
+        "D": np.ones(nheads, dtype=np.float32),
+        "dt_bias": np.log(np.expm1(fill((nheads,), seed, STREAM_SSD_BIAS, KIND_UNIFORM, 0.001,
+                                        0.1, out="f64"))).astype(np.float32),
+        "h0": (fill((batch, nheads, headdim, dstate), seed, STREAM_H0, out="f32",
+                    nthreads=nthreads) if with_h0 else None),
+    }
+
+
+def ssd_workload_inputs(w: SsdWorkload, nthreads=None):
+    return make_ssd_inputs(w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.io, w.seed,
+                           with_h0=w.with_h0, nthreads=nthreads)
 
 
 def make_decode_inputs(batch, dim, dstate, io, seed, step, nthreads=None):

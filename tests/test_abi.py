@@ -226,6 +226,35 @@ def test_sequence_split_helpers_reject_bad_arguments(L):
                                  FAKE + K, None) == 0
 
 
+def test_ssd_rejects_bad_arguments(L):
+    K = 1 << 18  # spacing of the fake buffers: none of them overlap
+
+    def ssd(**kw):
+        a = dict(batch=2, seqlen=64, nheads=2, headdim=64, dstate=128, io=1, x=FAKE, dt=FAKE + K,
+                 A=FAKE + 2 * K, B=FAKE + 3 * K, C=FAKE + 4 * K, D=None, bias=None, sp=1, h0=None,
+                 y=FAKE + 5 * K, h_last=None)
+        a.update(kw)
+        return L.ssm_ssd_scan_fwd(a["batch"], a["seqlen"], a["nheads"], a["headdim"],
+                                  a["dstate"], a["io"], a["x"], a["dt"], a["A"], a["B"], a["C"],
+                                  a["D"], a["bias"], a["sp"], a["h0"], a["y"], a["h_last"], None)
+    assert ssd(io=0) == -2            # fp32 io: the tensor-core path is bf16
+    assert ssd(io=7) == -1
+    assert ssd(headdim=32) == -2
+    assert ssd(dstate=16) == -2
+    assert ssd(dstate=0) == -1
+    assert ssd(batch=-1) == -1
+    assert ssd(x=None) == -1
+    assert ssd(A=None) == -1
+    assert ssd(y=None) == -1
+    assert ssd(x=FAKE + 8) == -1       # x needs 16-byte alignment
+    assert ssd(B=FAKE + 3 * K + 2) == -1
+    assert ssd(h0=FAKE + 6 * K + 4) == -1  # h0 needs 8-byte alignment
+    assert ssd(y=FAKE + 16) == -1      # y overlaps x
+    assert ssd(h_last=FAKE + 3 * K) == -1  # h_last overlaps B
+    assert ssd(batch=0) == 0
+    assert ssd(nheads=0) == 0
+
+
 def test_binding_has_no_cpu_path():
     from selective_state_space_39_b200 import ssm_scan_fwd
     x = torch.zeros(1, 4, 8)
