@@ -15,7 +15,7 @@
 //   H      <- e^{cum_end} H + (w X)^T B,   w_s = e^{cum_end - cum_s} Delta_s
 // The four products (C B^T, G X, C H, (w X)^T B) are bf16 tensor-core MMAs
 // (mma.sync m16n8k16, fp32 accumulation) fed from shared memory by ldmatrix;
-// x, B and C chunks are double-buffered with cp.async (zero-filled past the
+// x, B and C chunks arrive by cp.async two chunks ahead (zero-filled past the
 // end of the sequence, where Delta is taken as 0 so that the padded steps
 // change nothing).
 #include <mutex>
@@ -36,16 +36,23 @@ constexpr int kPadX = kP + 8;    // shared row of an x chunk (elements; 16-byte 
 constexpr int kPadG = kQ + 8;    // shared row of G
 
 static_assert(kQ == 32, "the in-chunk cumulative sum is one warp's scan");
+// The warp that computes the steps (Delta, cumulative sums, weights): warp 2
+// holds an S tile above the diagonal (row tile 0, columns 16..23) and so has
+// no S product to take.
+constexpr int kStepWarp = 2;
 
 template <int N>
 struct SsdLayout {
   static constexpr int kPadN = N + 8;
-  static constexpr int x_elems = 2 * kQ * kPadX;   // two buffers
-  static constexpr int bc_elems = 2 * kQ * kPadN;  // two buffers each for B and C
-  static constexpr int g_elems = kQ * kPadG;
-  static constexpr int h_elems = kP * kPadN;
-  static constexpr int bf16_bytes = 2 * (x_elems + 2 * bc_elems + g_elems + h_elems);
-  static constexpr int bytes = bf16_bytes + 4 * (4 * kQ + 4);
+  static constexpr int kStages = 3;               // x, B, C chunk buffers
+  static constexpr int x_elems = kQ * kPadX;      // one buffer
+  static constexpr int bc_elems = kQ * kPadN;     // one buffer of B (or C)
+  static constexpr int g_elems = kQ * kPadG;      // one buffer of G (two)
+  static constexpr int h_elems = kP * kPadN;      // one bf16 state copy (two)
+  static constexpr int bf16_bytes =
+      2 * (kStages * (x_elems + 2 * bc_elems) + 2 * g_elems + 2 * h_elems);
+  static constexpr int step_floats = 4 * kQ + 4;  // Delta, cum, e^cum, w, e^cum_end
+  static constexpr int bytes = bf16_bytes + 4 * kStages * step_floats;
   static_assert(bf16_bytes % 16 == 0, "float arrays start 16-byte aligned");
 };
 
@@ -63,9 +70,10 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t&
                : "r"(addr));
 }
 // d += a (16x16, row) * b (16x8, col), bf16 operands, fp32 accumulators.
+// Registers only (not volatile): independent MMAs may be interleaved.
 __device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
       "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
@@ -78,35 +86,87 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool v
                "r"(valid ? 16 : 0));
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;"); }
-__device__ __forceinline__ void cp_async_wait_prev() {
-  asm volatile("cp.async.wait_group 1;" ::: "memory");
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 // Both halves of a bf16 pair times their own weight, repacked.
 __device__ __forceinline__ uint32_t scale_bf16x2(uint32_t v, float lo, float hi) {
   return pack_bf16x2(bf16_lo(v) * lo, bf16_hi(v) * hi);
 }
 
-// One CTA per (head, batch row). Warp w owns: rows 16*(w/4).. of S, G and Y;
-// columns 8*(w%4).. of S and G, 16*(w%4).. of Y; rows 16*(w%4).. (p) and
-// columns (w/4)*N/2.. (n) of the state.
+// Per-chunk step quantities (one of three rotating buffers).
+struct StepBuf {
+  float* dt;    // Delta_s
+  float* cum;   // cum_t
+  float* ecum;  // e^{cum_t}
+  float* w;     // e^{cum_end - cum_s} Delta_s
+  float* decay; // [0] = e^{cum_end}
+};
+
+// S = C B^T on warp (rt, cq)'s 16 x 8 tile, then G = S e^{cum_t - cum_s}
+// Delta_s (s <= t, else 0) as bf16 into Gd.
+template <int N>
+__device__ __forceinline__ void chunk_g(const uint16_t* Bb, const uint16_t* Cb, uint16_t* Gd,
+                                        const StepBuf& st, int rt, int cq, int lane) {
+  constexpr int kPadN = N + 8;
+  const int g = lane >> 2, tig = lane & 3;
+  float sacc[4] = {0.f, 0.f, 0.f, 0.f}, sodd[4] = {0.f, 0.f, 0.f, 0.f};
+  if (8 * cq <= 16 * rt + 15) {  // the tile holds entries with s <= t
+#pragma unroll
+    for (int k0 = 0; k0 < N; k0 += 32) {
+      uint32_t b0, b1, b2, b3, a0, a1, a2, a3, c0, c1, c2, c3;
+      ldsm_x4(smem_u32(Bb + (8 * cq + (lane & 7)) * kPadN + k0 + (lane >> 3) * 8), b0, b1, b2,
+              b3);
+      ldsm_x4(smem_u32(Cb + (16 * rt + (lane & 15)) * kPadN + k0 + (lane >> 4) * 8), a0, a1, a2,
+              a3);
+      ldsm_x4(smem_u32(Cb + (16 * rt + (lane & 15)) * kPadN + k0 + 16 + (lane >> 4) * 8), c0, c1,
+              c2, c3);
+      mma_bf16(sacc, a0, a1, a2, a3, b0, b1);  // two chains: even and odd k-steps
+      mma_bf16(sodd, c0, c1, c2, c3, b2, b3);
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 4; ++e) sacc[e] += sodd[e];
+  const int ta = 16 * rt + g, tb = ta + 8, s0 = 8 * cq + 2 * tig;
+  const float cuma = st.cum[ta], cumb = st.cum[tb];
+  const float cs0 = st.cum[s0], cs1 = st.cum[s0 + 1];
+  const float d0 = st.dt[s0], d1 = st.dt[s0 + 1];
+  const float g0 = s0 <= ta ? sacc[0] * __expf(cuma - cs0) * d0 : 0.f;
+  const float g1 = s0 + 1 <= ta ? sacc[1] * __expf(cuma - cs1) * d1 : 0.f;
+  const float g2 = s0 <= tb ? sacc[2] * __expf(cumb - cs0) * d0 : 0.f;
+  const float g3 = s0 + 1 <= tb ? sacc[3] * __expf(cumb - cs1) * d1 : 0.f;
+  *reinterpret_cast<uint32_t*>(Gd + ta * kPadG + s0) = pack_bf16x2(g0, g1);
+  *reinterpret_cast<uint32_t*>(Gd + tb * kPadG + s0) = pack_bf16x2(g2, g3);
+}
+
+// One CTA per (head, batch row); 8 warps. Warp w owns rows 16*(w/4).. of
+// S, G and Y; columns 8*(w%4).. of S and G, 16*(w%4).. of Y; and the state
+// tile rows 16*(w%4).. (p) x columns (w/4)*N/2.. (n).
+//
+// Software pipeline, one CTA barrier per chunk: iteration c computes G of
+// chunk c+1, Y and the state update of chunk c, the step quantities of chunk
+// c+2 (warp kStepWarp), and has the x/B/C copy of chunk c+2 in flight. x, B, C and
+// the step quantities rotate through three buffers; G and the bf16 state
+// copy through two.
 template <int N>
 __global__ void __launch_bounds__(kThreads, (N <= 128) ? 2 : 1) ssd_fwd_kernel(const SsdParams p) {
   using Lay = SsdLayout<N>;
   constexpr int kPadN = Lay::kPadN;
+  constexpr int kS = Lay::kStages;
   constexpr int kNW = N / 2;   // state columns per warp
   constexpr int kNT = kNW / 8; // n8 tiles per warp
   static_assert(kNT % 2 == 0, "state tiles come in pairs from one ldmatrix.x4");
   extern __shared__ __align__(16) unsigned char smem_raw[];
   uint16_t* Xs = reinterpret_cast<uint16_t*>(smem_raw);
-  uint16_t* Bs = Xs + Lay::x_elems;
-  uint16_t* Cs = Bs + Lay::bc_elems;
-  uint16_t* Gs = Cs + Lay::bc_elems;
-  uint16_t* Hs = Gs + Lay::g_elems;
-  float* s_dt = reinterpret_cast<float*>(smem_raw + Lay::bf16_bytes);  // Delta_s
-  float* s_cum = s_dt + kQ;                                            // cum_t
-  float* s_ecum = s_cum + kQ;                                          // e^{cum_t}
-  float* s_w = s_ecum + kQ;                                            // w_s
-  float* s_decay = s_w + kQ;                                           // e^{cum_end}
+  uint16_t* Bs = Xs + kS * Lay::x_elems;
+  uint16_t* Cs = Bs + kS * Lay::bc_elems;
+  uint16_t* Gs = Cs + kS * Lay::bc_elems;
+  uint16_t* Hs = Gs + 2 * Lay::g_elems;
+  float* fbase = reinterpret_cast<float*>(smem_raw + Lay::bf16_bytes);
+  auto step_buf = [&](int i) {
+    float* f = fbase + i * Lay::step_floats;
+    return StepBuf{f, f + kQ, f + 2 * kQ, f + 3 * kQ, f + 4 * kQ};
+  };
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, tig = lane & 3;
@@ -123,6 +183,8 @@ __global__ void __launch_bounds__(kThreads, (N <= 128) ? 2 : 1) ssd_fwd_kernel(c
   const uint16_t* Cg = p.C + (size_t)b * L * N;
   const uint16_t* dtg = p.dt + (size_t)b * L * H + h;
   uint16_t* yg = p.y + ((size_t)b * L * H + h) * kP;
+  const int rt = warp >> 2;  // row tile of S, G, Y
+  const int cq = warp & 3;   // column quarter of S, G, Y
 
   // ---- state tile in registers: hacc[j] = rows p0, p0 + 8; columns n_j, n_j + 1
   const int pt = warp & 3, ng = warp >> 2;
@@ -140,19 +202,19 @@ __global__ void __launch_bounds__(kThreads, (N <= 128) ? 2 : 1) ssd_fwd_kernel(c
       hacc[j][0] = hacc[j][1] = hacc[j][2] = hacc[j][3] = 0.f;
     }
   }
-  auto store_state_bf16 = [&]() {
+  auto store_state_bf16 = [&](uint16_t* Hd) {
 #pragma unroll
     for (int j = 0; j < kNT; ++j) {
       const int n = ng * kNW + 8 * j + 2 * tig;
-      *reinterpret_cast<uint32_t*>(Hs + p0 * kPadN + n) = pack_bf16x2(hacc[j][0], hacc[j][1]);
-      *reinterpret_cast<uint32_t*>(Hs + (p0 + 8) * kPadN + n) =
+      *reinterpret_cast<uint32_t*>(Hd + p0 * kPadN + n) = pack_bf16x2(hacc[j][0], hacc[j][1]);
+      *reinterpret_cast<uint32_t*>(Hd + (p0 + 8) * kPadN + n) =
           pack_bf16x2(hacc[j][2], hacc[j][3]);
     }
   };
-  store_state_bf16();
 
   // ---- chunk loader (x: kQ rows of 128 B; B, C: kQ rows of 2N B)
-  auto load_chunk = [&](int c, int buf) {
+  auto load_chunk = [&](int c) {
+    const int buf = c % kS;
     const int64_t t0 = (int64_t)c * kQ;
     constexpr int kXPieces = kQ * kP / 8;
     constexpr int kBPieces = kQ * N / 8;
@@ -161,170 +223,169 @@ __global__ void __launch_bounds__(kThreads, (N <= 128) ? 2 : 1) ssd_fwd_kernel(c
       const int r = i / (kP / 8), q = i % (kP / 8);
       const bool ok = t0 + r < L;
       const uint16_t* src = ok ? xg + (size_t)(t0 + r) * row_x + q * 8 : xg;
-      cp_async16(smem_u32(Xs + (buf * kQ + r) * kPadX + q * 8), src, ok);
+      cp_async16(smem_u32(Xs + buf * Lay::x_elems + r * kPadX + q * 8), src, ok);
     }
 #pragma unroll
     for (int i = tid; i < kBPieces; i += kThreads) {
       const int r = i / (N / 8), q = i % (N / 8);
       const bool ok = t0 + r < L;
       const size_t off = ok ? (size_t)(t0 + r) * N + q * 8 : 0;
-      cp_async16(smem_u32(Bs + (buf * kQ + r) * kPadN + q * 8), Bg + off, ok);
-      cp_async16(smem_u32(Cs + (buf * kQ + r) * kPadN + q * 8), Cg + off, ok);
+      cp_async16(smem_u32(Bs + buf * Lay::bc_elems + r * kPadN + q * 8), Bg + off, ok);
+      cp_async16(smem_u32(Cs + buf * Lay::bc_elems + r * kPadN + q * 8), Cg + off, ok);
     }
   };
-
-  float dt_raw = 0.f;  // warp 0: raw step of the chunk about to run (lane = step)
-  if (nchunks > 0) {
-    load_chunk(0, 0);
-    cp_async_commit();
-    if (warp == 0 && lane < L) dt_raw = bf16_to_f32(dtg[(size_t)lane * H]);
-  }
-
-  for (int c = 0; c < nchunks; ++c) {
-    const int buf = c & 1;
-    const int64_t t0 = (int64_t)c * kQ;
-    if (c + 1 < nchunks) load_chunk(c + 1, buf ^ 1);
-    cp_async_commit();
-
-    // ---- steps, their in-chunk cumulative sum and the weights (warp 0)
-    if (warp == 0) {
-      float d = 0.f;
-      if (t0 + lane < L) {
-        const float v = dt_raw + bias;
-        d = p.softplus ? (v > kSoftplusCut ? v : log1pf(__expf(v))) : v;
-      }
-      const int64_t tn = t0 + kQ + lane;
-      dt_raw = tn < L ? bf16_to_f32(dtg[(size_t)tn * H]) : 0.f;
-      float cum = d * Ah;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const float u = __shfl_up_sync(0xffffffffu, cum, o);
-        if (lane >= o) cum += u;
-      }
-      const float cend = __shfl_sync(0xffffffffu, cum, 31);
-      s_dt[lane] = d;
-      s_cum[lane] = cum;
-      s_ecum[lane] = __expf(cum);
-      s_w[lane] = __expf(cend - cum) * d;
-      if (lane == 0) s_decay[0] = __expf(cend);
+  // raw step of chunk c (lane = step in the chunk), 0 past the end
+  auto load_dt = [&](int c) {
+    const int64_t t = (int64_t)c * kQ + lane;
+    return t < L ? bf16_to_f32(dtg[(size_t)t * H]) : 0.f;
+  };
+  // kStepWarp: Delta, its in-chunk cumulative sum and the weights of chunk c
+  auto chunk_steps = [&](int c, float raw) {
+    const StepBuf st = step_buf(c % kS);
+    float d = 0.f;
+    if ((int64_t)c * kQ + lane < L) {
+      const float v = raw + bias;
+      d = p.softplus ? (v > kSoftplusCut ? v : log1pf(__expf(v))) : v;
     }
-    cp_async_wait_prev();
+    float cum = d * Ah;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float u = __shfl_up_sync(0xffffffffu, cum, o);
+      if (lane >= o) cum += u;
+    }
+    const float cend = __shfl_sync(0xffffffffu, cum, 31);
+    st.dt[lane] = d;
+    st.cum[lane] = cum;
+    st.ecum[lane] = __expf(cum);
+    st.w[lane] = __expf(cend - cum) * d;
+    if (lane == 0) st.decay[0] = __expf(cend);
+  };
+
+  if (nchunks > 0) {
+    // ---- prologue: chunks 0 and 1 in shared memory, their steps, G of chunk 0
+    load_chunk(0);
+    if (nchunks > 1) load_chunk(1);
+    cp_async_commit();
+    float dt_raw = 0.f;  // kStepWarp: raw steps two chunks ahead
+    if (warp == kStepWarp) {
+      chunk_steps(0, load_dt(0));
+      if (nchunks > 1) chunk_steps(1, load_dt(1));
+      dt_raw = load_dt(2);
+    }
+    store_state_bf16(Hs);
+    cp_async_wait_all();
+    __syncthreads();
+    chunk_g<N>(Bs, Cs, Gs, step_buf(0), rt, cq, lane);
     __syncthreads();
 
-    const uint16_t* Xb = Xs + buf * kQ * kPadX;
-    const uint16_t* Bb = Bs + buf * kQ * kPadN;
-    const uint16_t* Cb = Cs + buf * kQ * kPadN;
-    const int rt = warp >> 2;  // row tile of S, G, Y
-    const int cq = warp & 3;   // column quarter
+    for (int c = 0; c < nchunks; ++c) {
+      const int buf = c % kS;
+      const int64_t t0 = (int64_t)c * kQ;
+      if (c + 2 < nchunks) load_chunk(c + 2);
+      cp_async_commit();
+      if (warp == kStepWarp && c + 2 < nchunks) {
+        chunk_steps(c + 2, dt_raw);
+        dt_raw = load_dt(c + 3);
+      }
+      // ---- G of the next chunk
+      if (c + 1 < nchunks) {
+        const int nb = (c + 1) % kS;
+        chunk_g<N>(Bs + nb * Lay::bc_elems, Cs + nb * Lay::bc_elems,
+                   Gs + ((c + 1) & 1) * Lay::g_elems, step_buf(nb), rt, cq, lane);
+      }
+      const StepBuf st = step_buf(buf);
+      const uint16_t* Xb = Xs + buf * Lay::x_elems;
+      const uint16_t* Bb = Bs + buf * Lay::bc_elems;
+      const uint16_t* Cb = Cs + buf * Lay::bc_elems;
+      const uint16_t* Gb = Gs + (c & 1) * Lay::g_elems;
+      const uint16_t* Hb = Hs + (c & 1) * Lay::h_elems;
 
-    // ---- S = C B^T on this warp's 16 x 8 tile, then G (bf16) into shared
-    {
-      float sacc[4] = {0.f, 0.f, 0.f, 0.f};
-      if (8 * cq <= 16 * rt + 15) {  // the tile holds entries with s <= t
+      // ---- Y = G X + diag(e^cum) C H + D x on rows 16 rt.., columns 16 cq..
+      {
+        float y1[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        float y2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        float y3[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};  // odd k-steps of C H
 #pragma unroll
-        for (int k0 = 0; k0 < N; k0 += 32) {
-          uint32_t b0, b1, b2, b3, a0, a1, a2, a3;
-          ldsm_x4(smem_u32(Bb + (8 * cq + (lane & 7)) * kPadN + k0 + (lane >> 3) * 8), b0, b1,
-                  b2, b3);
+        for (int k0 = 0; k0 < kQ; k0 += 16) {
+          if (k0 <= 16 * rt) {
+            uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
+            ldsm_x4(smem_u32(Gb + (16 * rt + (lane & 15)) * kPadG + k0 + (lane >> 4) * 8), a0,
+                    a1, a2, a3);
+            ldsm_x4_t(smem_u32(Xb + (k0 + (lane & 7) + ((lane >> 3) & 1) * 8) * kPadX +
+                               16 * cq + (lane >> 4) * 8),
+                      b0, b1, b2, b3);
+            mma_bf16(y1[0], a0, a1, a2, a3, b0, b1);
+            mma_bf16(y1[1], a0, a1, a2, a3, b2, b3);
+          }
+        }
+#pragma unroll
+        for (int k0 = 0; k0 < N; k0 += 16) {
+          uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
           ldsm_x4(smem_u32(Cb + (16 * rt + (lane & 15)) * kPadN + k0 + (lane >> 4) * 8), a0, a1,
                   a2, a3);
-          mma_bf16(sacc, a0, a1, a2, a3, b0, b1);
-          ldsm_x4(smem_u32(Cb + (16 * rt + (lane & 15)) * kPadN + k0 + 16 + (lane >> 4) * 8), a0,
-                  a1, a2, a3);
-          mma_bf16(sacc, a0, a1, a2, a3, b2, b3);
-        }
-      }
-      const int ta = 16 * rt + g, tb = ta + 8, s0 = 8 * cq + 2 * tig;
-      const float cuma = s_cum[ta], cumb = s_cum[tb];
-      const float cs0 = s_cum[s0], cs1 = s_cum[s0 + 1];
-      const float d0 = s_dt[s0], d1 = s_dt[s0 + 1];
-      const float g0 = s0 <= ta ? sacc[0] * __expf(cuma - cs0) * d0 : 0.f;
-      const float g1 = s0 + 1 <= ta ? sacc[1] * __expf(cuma - cs1) * d1 : 0.f;
-      const float g2 = s0 <= tb ? sacc[2] * __expf(cumb - cs0) * d0 : 0.f;
-      const float g3 = s0 + 1 <= tb ? sacc[3] * __expf(cumb - cs1) * d1 : 0.f;
-      *reinterpret_cast<uint32_t*>(Gs + ta * kPadG + s0) = pack_bf16x2(g0, g1);
-      *reinterpret_cast<uint32_t*>(Gs + tb * kPadG + s0) = pack_bf16x2(g2, g3);
-    }
-    __syncthreads();
-
-    // ---- Y = G X + diag(e^cum) C H + D x on rows 16 rt.., columns 16 cq..
-    {
-      float y1[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-      float y2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-      for (int k0 = 0; k0 < kQ; k0 += 16) {
-        if (k0 <= 16 * rt) {
-          uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
-          ldsm_x4(smem_u32(Gs + (16 * rt + (lane & 15)) * kPadG + k0 + (lane >> 4) * 8), a0, a1,
-                  a2, a3);
-          ldsm_x4_t(smem_u32(Xb + (k0 + (lane & 7) + ((lane >> 3) & 1) * 8) * kPadX + 16 * cq +
-                             (lane >> 4) * 8),
-                    b0, b1, b2, b3);
-          mma_bf16(y1[0], a0, a1, a2, a3, b0, b1);
-          mma_bf16(y1[1], a0, a1, a2, a3, b2, b3);
-        }
-      }
-#pragma unroll
-      for (int k0 = 0; k0 < N; k0 += 16) {
-        uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
-        ldsm_x4(smem_u32(Cb + (16 * rt + (lane & 15)) * kPadN + k0 + (lane >> 4) * 8), a0, a1,
-                a2, a3);
-        ldsm_x4(smem_u32(Hs + (16 * cq + (lane & 7) + (lane >> 4) * 8) * kPadN + k0 +
-                         ((lane >> 3) & 1) * 8),
-                b0, b1, b2, b3);
-        mma_bf16(y2[0], a0, a1, a2, a3, b0, b1);
-        mma_bf16(y2[1], a0, a1, a2, a3, b2, b3);
-      }
-      const int ta = 16 * rt + g, tb = ta + 8;
-      const float ea = s_ecum[ta], eb = s_ecum[tb];
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const int pc = 16 * cq + 8 * j + 2 * tig;
-        const uint32_t xa = *reinterpret_cast<const uint32_t*>(Xb + ta * kPadX + pc);
-        const uint32_t xb = *reinterpret_cast<const uint32_t*>(Xb + tb * kPadX + pc);
-        if (t0 + ta < L)
-          *reinterpret_cast<uint32_t*>(yg + (size_t)(t0 + ta) * row_x + pc) =
-              pack_bf16x2(fmaf(Dh, bf16_lo(xa), fmaf(ea, y2[j][0], y1[j][0])),
-                          fmaf(Dh, bf16_hi(xa), fmaf(ea, y2[j][1], y1[j][1])));
-        if (t0 + tb < L)
-          *reinterpret_cast<uint32_t*>(yg + (size_t)(t0 + tb) * row_x + pc) =
-              pack_bf16x2(fmaf(Dh, bf16_lo(xb), fmaf(eb, y2[j][2], y1[j][2])),
-                          fmaf(Dh, bf16_hi(xb), fmaf(eb, y2[j][3], y1[j][3])));
-      }
-    }
-
-    // ---- H <- e^{cum_end} H + (w X)^T B on rows 16 pt.. (p), columns ng N/2.. (n)
-    {
-      const float decay = s_decay[0];
-#pragma unroll
-      for (int j = 0; j < kNT; ++j)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) hacc[j][e] *= decay;
-#pragma unroll
-      for (int k0 = 0; k0 < kQ; k0 += 16) {
-        uint32_t a0, a1, a2, a3;
-        ldsm_x4_t(smem_u32(Xb + (k0 + (lane & 7) + (lane >> 4) * 8) * kPadX + 16 * pt +
+          ldsm_x4(smem_u32(Hb + (16 * cq + (lane & 7) + (lane >> 4) * 8) * kPadN + k0 +
                            ((lane >> 3) & 1) * 8),
-                  a0, a1, a2, a3);
-        const int s = k0 + 2 * tig;
-        const float w0 = s_w[s], w1 = s_w[s + 1], w8 = s_w[s + 8], w9 = s_w[s + 9];
-        a0 = scale_bf16x2(a0, w0, w1);
-        a1 = scale_bf16x2(a1, w0, w1);
-        a2 = scale_bf16x2(a2, w8, w9);
-        a3 = scale_bf16x2(a3, w8, w9);
+                  b0, b1, b2, b3);
+          float (&ya)[2][4] = (k0 & 16) ? y3 : y2;
+          mma_bf16(ya[0], a0, a1, a2, a3, b0, b1);
+          mma_bf16(ya[1], a0, a1, a2, a3, b2, b3);
+        }
 #pragma unroll
-        for (int j = 0; j < kNT; j += 2) {
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4_t(smem_u32(Bb + (k0 + (lane & 7) + ((lane >> 3) & 1) * 8) * kPadN + ng * kNW +
-                             8 * j + (lane >> 4) * 8),
-                    b0, b1, b2, b3);
-          mma_bf16(hacc[j], a0, a1, a2, a3, b0, b1);
-          mma_bf16(hacc[j + 1], a0, a1, a2, a3, b2, b3);
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) y2[j][e] += y3[j][e];
+        const int ta = 16 * rt + g, tb = ta + 8;
+        const float ea = st.ecum[ta], eb = st.ecum[tb];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int pc = 16 * cq + 8 * j + 2 * tig;
+          const uint32_t xa = *reinterpret_cast<const uint32_t*>(Xb + ta * kPadX + pc);
+          const uint32_t xb = *reinterpret_cast<const uint32_t*>(Xb + tb * kPadX + pc);
+          if (t0 + ta < L)
+            *reinterpret_cast<uint32_t*>(yg + (size_t)(t0 + ta) * row_x + pc) =
+                pack_bf16x2(fmaf(Dh, bf16_lo(xa), fmaf(ea, y2[j][0], y1[j][0])),
+                            fmaf(Dh, bf16_hi(xa), fmaf(ea, y2[j][1], y1[j][1])));
+          if (t0 + tb < L)
+            *reinterpret_cast<uint32_t*>(yg + (size_t)(t0 + tb) * row_x + pc) =
+                pack_bf16x2(fmaf(Dh, bf16_lo(xb), fmaf(eb, y2[j][2], y1[j][2])),
+                            fmaf(Dh, bf16_hi(xb), fmaf(eb, y2[j][3], y1[j][3])));
         }
       }
+
+      // ---- H <- e^{cum_end} H + (w X)^T B on rows 16 pt.. (p), columns ng N/2.. (n)
+      {
+        const float decay = st.decay[0];
+#pragma unroll
+        for (int j = 0; j < kNT; ++j)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) hacc[j][e] *= decay;
+#pragma unroll
+        for (int k0 = 0; k0 < kQ; k0 += 16) {
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4_t(smem_u32(Xb + (k0 + (lane & 7) + (lane >> 4) * 8) * kPadX + 16 * pt +
+                             ((lane >> 3) & 1) * 8),
+                    a0, a1, a2, a3);
+          const int s = k0 + 2 * tig;
+          const float w0 = st.w[s], w1 = st.w[s + 1], w8 = st.w[s + 8], w9 = st.w[s + 9];
+          a0 = scale_bf16x2(a0, w0, w1);
+          a1 = scale_bf16x2(a1, w0, w1);
+          a2 = scale_bf16x2(a2, w8, w9);
+          a3 = scale_bf16x2(a3, w8, w9);
+#pragma unroll
+          for (int j = 0; j < kNT; j += 2) {
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4_t(smem_u32(Bb + (k0 + (lane & 7) + ((lane >> 3) & 1) * 8) * kPadN +
+                               ng * kNW + 8 * j + (lane >> 4) * 8),
+                      b0, b1, b2, b3);
+            mma_bf16(hacc[j], a0, a1, a2, a3, b0, b1);
+            mma_bf16(hacc[j + 1], a0, a1, a2, a3, b2, b3);
+          }
+        }
+        store_state_bf16(Hs + ((c + 1) & 1) * Lay::h_elems);
+      }
+      cp_async_wait_all();
+      __syncthreads();
     }
-    __syncthreads();
-    store_state_bf16();
   }
 
   if (p.h_last) {
