@@ -86,12 +86,13 @@ def alu_ops_per_element(w, zoh=False):
     return (5 if zoh else 4) * w.dstate
 
 
-def measured_traffic(workload):
-    """DRAM bytes per call from the committed ncu capture, or None when the
-    kernel sources changed since that capture (or none was taken)."""
+def measured_traffic(workload, record="traffic.json"):
+    """DRAM bytes per call from the committed ncu capture (profiles/<record>),
+    or None when the kernel sources changed since that capture (or none was
+    taken)."""
     import hashlib
     try:
-        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+        with open(os.path.join(ROOT, "profiles", record)) as f:
             t = json.load(f)
         h = hashlib.sha256()
         for src in t["kernel_sources"]:
@@ -707,7 +708,8 @@ def ssd_bench(args):
     else:
         roof = {"bound": "tensor", "achieved": round(tfs, 1), "peak": tc_peak,
                 "unit": "TFLOP/s", "frac": round(tfs / tc_peak, 4), "peak_kind": tc_kind}
-    roof.update({"traffic": None, "kernel": f"ssd_fwd_kernel<{N}> (1 launch)",
+    roof.update({"traffic": measured_traffic(w.name, "ssd_traffic.json"),
+                 "kernel": f"ssd_fwd_kernel<{N}> (1 launch)",
                  "algorithmic_bytes_per_launch": nbytes, "algorithmic_flops_per_launch": flops,
                  "tensor": {"achieved_tflops": round(tfs, 1), "peak": tc_peak,
                             "frac": round(tfs / tc_peak, 4), "peak_kind": tc_kind},
