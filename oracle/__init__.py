@@ -15,7 +15,8 @@ the page "Mamba 논문 리뷰: Selective State Space Models로 Transformer를
 넘어서" (youngju.dev): §2.2 discretised recurrence,
 §3.1 softplus step size, §3.3 simplified ``selective_scan``, §3.4 block gate,
 D skip and the causal depthwise conv1d + SiLU (``conv1d_silu``), §4.1 the
-multi-head SSD form (``ssd_scan``). Every function here is pinned by
+multi-head SSD form (``ssd_scan``) and its recurrent decode step
+(``ssd_state_update``). Every function here is pinned by
 ``tests/test_oracle_pins.py``
 against closed forms, brute force and invariants.
 
@@ -100,6 +101,11 @@ class Oracle:
                       ctypes.c_void_p, _F32P, ctypes.c_void_p, ctypes.c_void_p, _F32P,
                       ctypes.c_void_p, _F32P, ctypes.c_int, _F64P]
         gz.argtypes = g.argtypes
+        su = self.lib.oracle_ssd_state_update
+        su.restype = ctypes.c_int
+        su.argtypes = [ctypes.c_int64] * 4 + [ctypes.c_int, _F64P, ctypes.c_void_p,
+                                              ctypes.c_void_p, _F32P, ctypes.c_void_p,
+                                              ctypes.c_void_p, _F32P, _F32P, ctypes.c_int, _F64P]
         sd = self.lib.oracle_ssd_scan
         sd.restype = ctypes.c_int
         sd.argtypes = [ctypes.c_int64] * 5 + [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
@@ -391,6 +397,32 @@ class Oracle:
         return y, h_last
 
 
+    def ssd_state_update(self, state, x, dt, A, B, C, D=None, dt_bias=None, softplus=True,
+                         io="f32"):
+        """One SSD decode step on the fp64 ``state`` (batch, heads, headdim,
+        dstate), in place. x (batch, heads, headdim), dt (batch, heads), B, C
+        (batch, dstate). Returns y (batch, heads, headdim) in fp64."""
+        if state.dtype != np.float64 or not state.flags.c_contiguous:
+            raise TypeError("state must be a C-contiguous float64 array")
+        batch, H, P, N = state.shape
+        x = self._io_array(x, io, (batch, H, P), "x")
+        dt = self._io_array(dt, io, (batch, H), "dt")
+        B = self._io_array(B, io, (batch, N), "B")
+        C = self._io_array(C, io, (batch, N), "C")
+        A = self._f32_array(A, (H,), "A", optional=False)
+        D = self._f32_array(D, (H,), "D")
+        dt_bias = self._f32_array(dt_bias, (H,), "dt_bias")
+        y = np.empty((batch, H, P), dtype=np.float64)
+        rc = self.lib.oracle_ssd_state_update(
+            batch, H, P, N, 1 if io == "bf16" else 0, self._ptr(state, ctypes.c_double),
+            self._ptr(x), self._ptr(dt), self._ptr(A, ctypes.c_float), self._ptr(B),
+            self._ptr(C), self._ptr(D, ctypes.c_float), self._ptr(dt_bias, ctypes.c_float),
+            1 if softplus else 0, self._ptr(y, ctypes.c_double))
+        if rc != 0:
+            raise ValueError("oracle_ssd_state_update rejected its arguments")
+        return y
+
+
 _default = None
 
 
@@ -431,3 +463,8 @@ def conv1d_silu_update(*args, **kwargs):
 
 def ssd_scan(*args, **kwargs):
     return get().ssd_scan(*args, **kwargs)
+
+
+def ssd_state_update(*args, **kwargs):
+    return get().ssd_state_update(*args, **kwargs)
+

@@ -658,3 +658,37 @@ int oracle_ssd_scan(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headd
   free(S);
   return 0;
 }
+
+/* oracle_ssd_state_update -- one decode step of the multi-head SSD: the
+ * recurrent side of §4.1's duality (state update, O(1) per token), on the
+ * oracle's own fp64 state (batch, nheads, headdim, dstate), in place.
+ * x (batch, nheads, headdim), dt (batch, nheads), B, C (batch, dstate) in the
+ * io type; A, D, dt_bias (nheads) fp32 (D, dt_bias nullable); y (batch,
+ * nheads, headdim) fp64. Same arithmetic as one step of oracle_ssd_scan.
+ * Returns 0 or -1. */
+int oracle_ssd_state_update(int64_t batch, int64_t nheads, int64_t headdim, int64_t dstate,
+                            int is_bf16, double* state, const void* x, const void* dt,
+                            const float* A, const void* Bm, const void* Cm, const float* D,
+                            const float* dt_bias, int softplus_on, double* y) {
+  if (batch < 0 || nheads < 0 || headdim < 1 || dstate < 1 || !state || !x || !dt || !A ||
+      !Bm || !Cm || !y)
+    return -1;
+  const int64_t H = nheads, P = headdim, N = dstate;
+  for (int64_t b = 0; b < batch; ++b)
+    for (int64_t h = 0; h < H; ++h) {
+      const double v = widen(dt, b * H + h, is_bf16) + (dt_bias ? (double)dt_bias[h] : 0.0);
+      const double delta = softplus_on ? softplus(v) : v;
+      const double a = exp(delta * (double)A[h]);
+      for (int64_t p = 0; p < P; ++p) {
+        const double xv = widen(x, (b * H + h) * P + p, is_bf16);
+        double* S = state + ((b * H + h) * P + p) * N;
+        double acc = 0.0;
+        for (int64_t n = 0; n < N; ++n) {
+          S[n] = a * S[n] + delta * widen(Bm, b * N + n, is_bf16) * xv;
+          acc += widen(Cm, b * N + n, is_bf16) * S[n];
+        }
+        y[(b * H + h) * P + p] = acc + (D ? (double)D[h] : 0.0) * xv;
+      }
+    }
+  return 0;
+}

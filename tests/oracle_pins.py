@@ -664,6 +664,43 @@ def pin_ssd_split_invariance(o):
     _close(h2, hl, 1e-6, 1e-6, what="ssd end state")
 
 
+def pin_ssd_decode_steps_equal_scan(o):
+    """L SSD decode steps from h0 reproduce the (separately pinned) SSD scan:
+    every y_t and the end state."""
+    c = _ssd_case(311, batch=2, L=7, H=3, P=4, N=5)
+    y, hl = _ssd(o, c)
+    state = c["h0"].astype(np.float64).copy()
+    for t in range(7):
+        yt = o.ssd_state_update(state, np.ascontiguousarray(c["x"][:, t]),
+                                np.ascontiguousarray(c["dt"][:, t]), c["A"],
+                                np.ascontiguousarray(c["B"][:, t]),
+                                np.ascontiguousarray(c["C"][:, t]), D=c["D"],
+                                dt_bias=c["dt_bias"])
+        _close(yt, y[:, t], 1e-13, 1e-14, what=f"ssd decode step {t}")
+    _close(state, hl, 1e-13, 1e-14, what="ssd decode state")
+
+
+def pin_ssd_decode_single_step_by_hand(o):
+    """One SSD decode step written out element by element."""
+    c = _ssd_case(313, batch=1, L=1, H=2, P=3, N=4)
+    state = c["h0"].astype(np.float64).copy()
+    before = state.copy()
+    y = o.ssd_state_update(state, c["x"][:, 0], c["dt"][:, 0], c["A"], c["B"][:, 0],
+                           c["C"][:, 0], D=c["D"], dt_bias=c["dt_bias"])
+    for h in range(2):
+        v = float(c["dt"][0, 0, h]) + float(c["dt_bias"][h])
+        delta = math.log1p(math.exp(v))
+        a = math.exp(delta * float(c["A"][h]))
+        for p in range(3):
+            xv = float(c["x"][0, 0, h, p])
+            acc = 0.0
+            for n in range(4):
+                hn = a * before[0, h, p, n] + delta * float(c["B"][0, 0, n]) * xv
+                _close(state[0, h, p, n], hn, 1e-14, 1e-15, what="ssd step state")
+                acc += float(c["C"][0, 0, n]) * hn
+            _close(y[0, h, p], acc + float(c["D"][h]) * xv, 1e-13, 1e-15, what="ssd step y")
+
+
 ALL_PINS = [
     pin_softplus_library,
     pin_silu_library,
@@ -693,4 +730,6 @@ ALL_PINS = [
     pin_ssd_is_tied_selective_scan,
     pin_ssd_A_zero_is_cumulative_outer_product,
     pin_ssd_split_invariance,
+    pin_ssd_decode_steps_equal_scan,
+    pin_ssd_decode_single_step_by_hand,
 ]

@@ -124,6 +124,14 @@ MUTANTS = {
                       "const double a = exp(-delta * (double)A[h]);"),
     "ssd_x_of_head_zero": ("const double xv = widen(x, ((b * L + t) * H + h) * P + p, is_bf16);",
                            "const double xv = widen(x, ((b * L + t) * H + 0) * P + p, is_bf16);"),
+    "ssd_decode_state_not_kept": (
+        "          S[n] = a * S[n] + delta * widen(Bm, b * N + n, is_bf16) * xv;\n          acc += widen(Cm, b * N + n, is_bf16) * S[n];",
+        "          const double sn = a * S[n] + delta * widen(Bm, b * N + n, is_bf16) * xv;\n          acc += widen(Cm, b * N + n, is_bf16) * sn;"),
+    "ssd_decode_skip_dropped": ("        y[(b * H + h) * P + p] = acc + (D ? (double)D[h] : 0.0) * xv;",
+                                "        y[(b * H + h) * P + p] = acc;"),
+    "ssd_decode_bias_dropped": (
+        "const double v = widen(dt, b * H + h, is_bf16) + (dt_bias ? (double)dt_bias[h] : 0.0);",
+        "const double v = widen(dt, b * H + h, is_bf16);"),
     "zoh_sign_flipped": ("  return An == 0.0 ? dt : expm1(dt * An) / An;",
                          "  return An == 0.0 ? dt : -expm1(dt * An) / An;"),
 }
