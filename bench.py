@@ -47,7 +47,7 @@ def parse_args():
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
                     choices=sorted(gen.SCAN_WORKLOADS) + sorted(gen.DECODE_WORKLOADS) +
-                    sorted(gen.SSD_WORKLOADS))
+                    sorted(gen.SSD_WORKLOADS) + sorted(gen.SSD_DECODE_WORKLOADS))
     ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd"],
                     help="bwd: time ssm_scan_bwd (the gradients) on the same workload")
     ap.add_argument("--learned-a", action="store_true",
@@ -736,6 +736,94 @@ def ssd_bench(args):
     return 0
 
 
+def ssd_decode_bench(args):
+    """--workload ssd_decode_*: ssm_ssd_state_update calls on a resident fp32
+    state (one step = one call over every sequence, head and row). Timed with
+    L2 flushed before every call (by a write, and by a read) and back to back."""
+    import torch
+
+    from selective_state_space_39_b200 import ssm_ssd_state_update
+    w = gen.SSD_DECODE_WORKLOADS[args.workload]
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    const = gen.ssd_constants(w.nheads, w.seed)
+
+    def to_dev(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16).copy()).view(torch.bfloat16).to(device)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+    steps_in = [{k: to_dev(v) for k, v in gen.make_ssd_decode_inputs(
+        w.batch, w.nheads, w.headdim, w.dstate, w.io, w.seed, i).items()} for i in range(8)]
+    A, D, bias = (to_dev(const[k]) for k in ("A", "D", "dt_bias"))
+    state = torch.zeros((w.batch, w.nheads, w.headdim, w.dstate), dtype=torch.float32,
+                        device=device)
+    dtype = torch.bfloat16 if w.io == "bf16" else torch.float32
+    y = torch.empty((w.batch, w.nheads, w.headdim), dtype=dtype, device=device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    def call(i):
+        s_ = steps_in[i % len(steps_in)]
+        ssm_ssd_state_update(state, s_["x"], s_["dt"], A, s_["B"], s_["C"], D=D, dt_bias=bias,
+                             y=y)
+
+    for i in range(max(3, args.warmup)):
+        call(i)
+    torch.cuda.synchronize()
+    K = args.steps
+
+    def timed(prep):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(K)]
+        for i in range(K):
+            prep(i)
+            ev[i][0].record()
+            call(i)
+            ev[i][1].record()
+        torch.cuda.synchronize()
+        return statistics.mean(a.elapsed_time(b) for a, b in ev)
+
+    sampler = ClockSampler(0)
+    with sampler:
+        cold_ms = timed(lambda i: flush.fill_(i & 0xFF))
+    read_ms = timed(lambda i: flush.view(torch.int64).sum())
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(K):
+        call(i)
+    e1.record()
+    torch.cuda.synchronize()
+    warm_ms = e0.elapsed_time(e1) / K
+    es = 2 if w.io == "bf16" else 4
+    rows = w.batch * w.nheads * w.headdim
+    algo = rows * w.dstate * 4 * 2 + rows * es * 2 + w.batch * w.nheads * es + \
+        2 * w.batch * w.dstate * es + 3 * w.nheads * 4
+    peak, peak_kind = measured_hbm_peak()
+    gbs = algo / (cold_ms * 1e-3) / 1e9
+    line = {
+        "metric": "SSD decode state-update rows/s (B·H·P per step) and HBM GB/s",
+        "value": rows / (cold_ms * 1e-3), "unit": "rows/s", "n_gpus": 1, "steps": K,
+        "warmup": args.warmup, "ms_per_step": cold_ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.io,
+        "data": "synthetic (seeded Philox4x32-10, the SSD recipe)",
+        "config": {"workload": w.name, "batch": w.batch, "nheads": w.nheads,
+                   "headdim": w.headdim, "dstate": w.dstate,
+                   "l2": "flushed (256 MB write) before every timed call"},
+        "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(gbs / peak, 4), "traffic": None,
+                     "kernel": f"ssd_decode_kernel<{w.dstate}> (1 launch)",
+                     "algorithmic_bytes_per_launch": algo, "peak_kind": peak_kind},
+        "read_flushed_l2": {"ms_per_step": read_ms,
+                            "algorithmic_gbs": round(algo / (read_ms * 1e-3) / 1e9, 1),
+                            "frac": round(algo / (read_ms * 1e-3) / 1e9 / peak, 4)},
+        "back_to_back": {"ms_per_step": warm_ms,
+                         "algorithmic_gbs": round(algo / (warm_ms * 1e-3) / 1e9, 1)},
+        "gpu_launches": 2 * K, "clocks": sampler.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def ssd_reference_arm(args):
     """--impl reference on an SSD workload: the fp64 oracle, one (batch, head)
     pair per step, on the host (rank 0 only)."""
@@ -780,6 +868,8 @@ def main():
         return reference_arm(args)
     if args.workload in gen.SSD_WORKLOADS:
         return ssd_bench(args)
+    if args.workload in gen.SSD_DECODE_WORKLOADS:
+        return ssd_decode_bench(args)
     if args.workload in gen.DECODE_WORKLOADS:
         return decode_bench(args)
     if args.op == "conv":

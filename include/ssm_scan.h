@@ -355,6 +355,29 @@ int ssm_ssd_scan_fwd(int64_t batch, int64_t seqlen, int64_t nheads, int64_t head
                      int softplus, const float* h0, void* y, float* h_last, void* stream);
 
 /*
+ * ssm_ssd_state_update -- one decode step of the multi-head SSD (same page,
+ * §4.1: the recurrent side of the duality, O(1) work per generated token),
+ * on a carried fp32 state updated in place. Per batch b, head h, row p:
+ *
+ *   Delta    = softplus(dt[b,h] + dt_bias[h])   (or no softplus)
+ *   S[n]     = exp(Delta * A[h]) * S[n] + Delta * B[b,n] * x[b,h,p]
+ *   y[b,h,p] = sum_n C[b,n] * S[n] + D[h] * x[b,h,p]
+ *
+ *   state    : (batch, nheads, headdim, dstate) fp32, read and written
+ *   x, y     : (batch, nheads, headdim) io_dtype
+ *   dt       : (batch, nheads) io_dtype
+ *   B, C     : (batch, dstate) io_dtype
+ *   A        : (nheads) fp32;  D, dt_bias : (nheads) fp32, nullable
+ * dstate 32, 64, 128 or 256 (else SSM_ERR_UNSUPPORTED); any headdim. state,
+ * B and C 16-byte aligned. No output may overlap an input.
+ * Returns SSM_OK or SSM_ERR_*.
+ */
+int ssm_ssd_state_update(int64_t batch, int64_t nheads, int64_t headdim, int64_t dstate,
+                         int io_dtype, float* state, const void* x, const void* dt,
+                         const float* A, const void* B, const void* C, const float* D,
+                         const float* dt_bias, int softplus, void* y, void* stream);
+
+/*
  * ssm_scan_status -- synchronise `stream`, then report whether every CTA of
  * the last ssm_scan_fwd call that used this workspace (with these sizes)
  * finished normally: SSM_OK, or SSM_ERR_TIMEOUT if a bounded wait inside a

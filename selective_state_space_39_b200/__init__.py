@@ -24,6 +24,7 @@ from ._binding import (  # noqa: F401
     ssm_scan_fwd_noalloc,
     ssm_scan_status,
     ssm_ssd_scan_fwd,
+    ssm_ssd_state_update,
     ssm_state_update,
 )
 
@@ -32,4 +33,5 @@ __all__ = ["ssm_scan_fwd", "ssm_scan_fwd_noalloc", "ssm_scan_bwd", "ssm_state_up
            "ssm_conv1d_silu_fwd", "ssm_conv1d_silu_bwd", "ssm_conv1d_silu_update",
            "conv1d_silu_bwd_workspace_bytes",
            "ssm_delta_sum", "ssm_compose_carries", "ssm_ssd_scan_fwd",
+           "ssm_ssd_state_update",
            "SsmError", "SSM_DTYPE_F32", "SSM_DTYPE_BF16", "lib"]

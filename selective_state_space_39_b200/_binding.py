@@ -104,6 +104,9 @@ def lib() -> ctypes.CDLL:
         L.ssm_compose_carries.argtypes = [_I64, _I64, _I64, _I64, _VP, _VP, _VP, _VP, _VP, _VP]
         L.ssm_state_update_zoh.restype = ctypes.c_int
         L.ssm_state_update_zoh.argtypes = L.ssm_state_update.argtypes
+        L.ssm_ssd_state_update.restype = ctypes.c_int
+        L.ssm_ssd_state_update.argtypes = [_I64] * 4 + [ctypes.c_int] + [_VP] * 8 + \
+            [ctypes.c_int, _VP, _VP]
         L.ssm_ssd_scan_fwd.restype = ctypes.c_int
         L.ssm_ssd_scan_fwd.argtypes = [_I64] * 5 + [ctypes.c_int] + [_VP] * 7 + \
             [ctypes.c_int, _VP, _VP, _VP, _VP]
@@ -504,4 +507,33 @@ def ssm_ssd_scan_fwd(x, dt, A, B, C, D=None, dt_bias=None, softplus=True, h0=Non
     if rc != 0:
         raise SsmError(rc, "ssm_ssd_scan_fwd", with_detail=True)
     return (y, h_last) if return_last_state else y
+
+
+def ssm_ssd_state_update(state, x, dt, A, B, C, D=None, dt_bias=None, softplus=True, y=None,
+                         stream=None):
+    """One SSD decode step through ssm_ssd_state_update of libssmscan.so:
+    updates the float32 state (batch, heads, headdim, dstate) in place and
+    returns y (batch, heads, headdim) in x's dtype."""
+    if state.dim() != 4:
+        raise ValueError("state must be (batch, heads, headdim, dstate)")
+    batch, H, P, N = state.shape
+    dev = state.device
+    io = _io_code(x.dtype)
+    ps = _ptr(state, "state", torch.float32)
+    px = _ptr(x, "x", x.dtype, (batch, H, P), dev)
+    pdt = _ptr(dt, "dt", x.dtype, (batch, H), dev)
+    pA = _ptr(A, "A", torch.float32, (H,), dev)
+    pB = _ptr(B, "B", x.dtype, (batch, N), dev)
+    pC = _ptr(C, "C", x.dtype, (batch, N), dev)
+    pD = _ptr(D, "D", torch.float32, (H,), dev)
+    pbias = _ptr(dt_bias, "dt_bias", torch.float32, (H,), dev)
+    if y is None:
+        y = torch.empty((batch, H, P), dtype=x.dtype, device=dev)
+    py = _ptr(y, "y", x.dtype, (batch, H, P), dev)
+    with torch.cuda.device(dev):
+        rc = lib().ssm_ssd_state_update(batch, H, P, N, io, ps, px, pdt, pA, pB, pC, pD, pbias,
+                                        1 if softplus else 0, py, _stream_ptr(stream, dev))
+    if rc != 0:
+        raise SsmError(rc, "ssm_ssd_state_update", with_detail=True)
+    return y
 

@@ -13,6 +13,7 @@
 #include "ssm_bwd_internal.h"
 #include "ssm_conv_internal.h"
 #include "ssm_seqpar_internal.h"
+#include "ssm_ssd_decode_internal.h"
 #include "ssm_ssd_internal.h"
 #include "ssm_internal.h"
 
@@ -685,6 +686,52 @@ int ssm_ssd_scan_fwd(int64_t batch, int64_t seqlen, int64_t nheads, int64_t head
   p.y = static_cast<uint16_t*>(y);
   p.h_last = h_last;
   return cuda_status(launch_ssd_fwd(p, static_cast<cudaStream_t>(stream)), "ssd scan launch");
+}
+
+int ssm_ssd_state_update(int64_t batch, int64_t nheads, int64_t headdim, int64_t dstate,
+                         int io_dtype, float* state, const void* x, const void* dt,
+                         const float* A, const void* B, const void* C, const float* D,
+                         const float* dt_bias, int softplus, void* y, void* stream) {
+  if (io_dtype != SSM_DTYPE_F32 && io_dtype != SSM_DTYPE_BF16) return SSM_ERR_INVALID_ARG;
+  if (batch < 0 || nheads < 0 || headdim < 0 || dstate <= 0) return SSM_ERR_INVALID_ARG;
+  if (!ssd_decode_dstate_supported((int)std::min<int64_t>(dstate, 1 << 20)))
+    return fail(SSM_ERR_UNSUPPORTED, "ssm_ssd_state_update: dstate 32, 64, 128 or 256 only");
+  if (batch > (1 << 24) || nheads > (1 << 20) || headdim > (1 << 20) ||
+      batch * nheads * headdim > ((int64_t)1 << 26))
+    return SSM_ERR_UNSUPPORTED;
+  if (batch == 0 || nheads == 0 || headdim == 0) return SSM_OK;
+  if (!state || !x || !dt || !A || !B || !C || !y) return SSM_ERR_INVALID_ARG;
+  const size_t es = io_bytes(io_dtype);
+  if (!aligned(state, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(x, es) ||
+      !aligned(dt, es) || !aligned(y, es) || !aligned(A, 4) || (D && !aligned(D, 4)) ||
+      (dt_bias && !aligned(dt_bias, 4)))
+    return fail(SSM_ERR_INVALID_ARG, "ssm_ssd_state_update: misaligned pointer");
+  const size_t rows = (size_t)batch * nheads * headdim;
+  const size_t ns = rows * dstate * 4, nx = rows * es, ndt = (size_t)batch * nheads * es,
+               nbc = (size_t)batch * dstate * es;
+  if (overlap(y, nx, state, ns) || overlap(y, nx, x, nx) || overlap(y, nx, dt, ndt) ||
+      overlap(y, nx, B, nbc) || overlap(y, nx, C, nbc) || overlap(state, ns, x, nx) ||
+      overlap(state, ns, dt, ndt) || overlap(state, ns, B, nbc) || overlap(state, ns, C, nbc) ||
+      overlap(state, ns, A, (size_t)nheads * 4))
+    return fail(SSM_ERR_INVALID_ARG, "ssm_ssd_state_update: buffers overlap");
+  SsdDecodeParams p{};
+  p.batch = (int)batch;
+  p.nheads = (int)nheads;
+  p.headdim = (int)headdim;
+  p.dstate = (int)dstate;
+  p.softplus = softplus ? 1 : 0;
+  p.state = state;
+  p.x = x;
+  p.dt = dt;
+  p.B = B;
+  p.C = C;
+  p.A = A;
+  p.D = D;
+  p.dt_bias = dt_bias;
+  p.y = y;
+  return cuda_status(launch_ssd_decode(p, io_dtype == SSM_DTYPE_BF16,
+                                       static_cast<cudaStream_t>(stream)),
+                     "ssd decode launch");
 }
 
 size_t ssm_conv1d_silu_bwd_workspace_bytes(int64_t batch, int64_t seqlen, int64_t dim,

@@ -227,6 +227,25 @@ SSD_WORKLOADS = {
         "ssd_mamba2_b4_l4096_h64_p64_n128", 4, 4096, 64, 64, 128, "bf16", 6, with_h0=True),
 }
 
+@dataclass(frozen=True)
+class SsdDecodeWorkload:
+    name: str
+    batch: int
+    nheads: int
+    headdim: int
+    dstate: int
+    io: str
+    seed: int
+    steps: int
+
+
+# Decode on the same Mamba-2 layer: 64 sequences, 64 heads of 64, d_state 128
+# (a 134 MB fp32 state, larger than L2), 1000 generated tokens.
+SSD_DECODE_WORKLOADS = {
+    "ssd_decode_b64_h64_p64_n128_x1000": SsdDecodeWorkload(
+        "ssd_decode_b64_h64_p64_n128_x1000", 64, 64, 64, 128, "bf16", 7, 1000),
+}
+
 DECODE_WORKLOADS = {
     "decode_b128_d4096_x1000": DecodeWorkload("decode_b128_d4096_x1000", 128, 4096, 16, "bf16", 4, 1000),
 }
@@ -318,13 +337,36 @@ def make_ssd_inputs(batch, seqlen, nheads, headdim, dstate, io, seed, *, with_h0
         "dt": fill((batch, seqlen, nheads), seed, STREAM_DELTA, b=0.5, out=io, nthreads=nthreads),
         "B": fill((batch, seqlen, dstate), seed, STREAM_B, out=io, nthreads=nthreads),
         "C": fill((batch, seqlen, dstate), seed, STREAM_C, out=io, nthreads=nthreads),
+        **ssd_constants(nheads, seed),
+        "h0": (fill((batch, nheads, headdim, dstate), seed, STREAM_H0, out="f32",
+                    nthreads=nthreads) if with_h0 else None),
+    }
+
+
+def ssd_constants(nheads, seed):
+    """Per-head parameters of the SSD recipe: A ~ -U[1, 16], dt_bias =
+    log(expm1(U[0.001, 0.1])), D = 1 (fp32)."""
+    return {
         "A": (-fill((nheads,), seed, STREAM_SSD_A, KIND_UNIFORM, 1.0, 16.0, out="f64")).astype(
             np.float32),
         "D": np.ones(nheads, dtype=np.float32),
         "dt_bias": np.log(np.expm1(fill((nheads,), seed, STREAM_SSD_BIAS, KIND_UNIFORM, 0.001,
                                         0.1, out="f64"))).astype(np.float32),
-        "h0": (fill((batch, nheads, headdim, dstate), seed, STREAM_H0, out="f32",
-                    nthreads=nthreads) if with_h0 else None),
+    }
+
+
+def make_ssd_decode_inputs(batch, nheads, headdim, dstate, io, seed, step, nthreads=None):
+    """Inputs of SSD decode step `step`: the step's slice of a (steps, ...)
+    stream (x (batch, heads, headdim), dt (batch, heads), B, C (batch,
+    dstate)), so step k's values do not depend on how many steps are drawn."""
+    nx, nd, nn = batch * nheads * headdim, batch * nheads, batch * dstate
+    return {
+        "x": fill((batch, nheads, headdim), seed, STREAM_X, out=io, offset=step * nx,
+                  nthreads=nthreads),
+        "dt": fill((batch, nheads), seed, STREAM_DELTA, b=0.5, out=io, offset=step * nd,
+                   nthreads=nthreads),
+        "B": fill((batch, dstate), seed, STREAM_B, out=io, offset=step * nn, nthreads=nthreads),
+        "C": fill((batch, dstate), seed, STREAM_C, out=io, offset=step * nn, nthreads=nthreads),
     }
 
 

@@ -255,6 +255,33 @@ def test_ssd_rejects_bad_arguments(L):
     assert ssd(nheads=0) == 0
 
 
+def test_ssd_state_update_rejects_bad_arguments(L):
+    K = 1 << 20
+
+    def upd(**kw):
+        a = dict(batch=2, nheads=4, headdim=64, dstate=128, io=1, state=FAKE, x=FAKE + K,
+                 dt=FAKE + 2 * K, A=FAKE + 3 * K, B=FAKE + 4 * K, C=FAKE + 5 * K, D=None,
+                 bias=None, sp=1, y=FAKE + 6 * K)
+        a.update(kw)
+        return L.ssm_ssd_state_update(a["batch"], a["nheads"], a["headdim"], a["dstate"],
+                                      a["io"], a["state"], a["x"], a["dt"], a["A"], a["B"],
+                                      a["C"], a["D"], a["bias"], a["sp"], a["y"], None)
+    assert upd(dstate=16) == -2
+    assert upd(dstate=0) == -1
+    assert upd(io=5) == -1
+    assert upd(batch=-1) == -1
+    assert upd(state=None) == -1
+    assert upd(A=None) == -1
+    assert upd(y=None) == -1
+    assert upd(state=FAKE + 8) == -1         # the state needs 16-byte alignment
+    assert upd(C=FAKE + 5 * K + 4) == -1
+    assert upd(x=FAKE + K + 1) == -1         # bf16 x misaligned
+    assert upd(y=FAKE + 1024) == -1          # y inside the state
+    assert upd(x=FAKE + 4096) == -1          # x inside the state
+    assert upd(batch=0) == 0
+    assert upd(headdim=0) == 0
+
+
 def test_binding_has_no_cpu_path():
     from selective_state_space_39_b200 import ssm_scan_fwd
     x = torch.zeros(1, 4, 8)

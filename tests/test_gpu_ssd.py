@@ -1,5 +1,6 @@
 """GPU parity of the multi-head SSD scan (Mamba-2, tensor-core chunked form,
-through the C ABI) against the fp64 oracle's sequential per-head loop.
+through the C ABI) and of its decode step against the fp64 oracle's
+sequential per-head loop.
 
 Bound: max|g - g_ref| / max|g_ref| <= 1e-2 for y and h_last: bf16 io, with
 the chunk's products taken on bf16 tensor-core operands (the decay-weighted
@@ -116,3 +117,87 @@ def test_ssd_split_sequence_carries_the_state():
                               cut(d["B"], 96, 200), cut(d["C"], 96, 200), D=d["D"],
                               dt_bias=d["dt_bias"], h0=h1, return_last_state=True)
     assert torch.equal(torch.cat([y1, y2], dim=1), y) and torch.equal(h2, hl)
+
+
+# ---- decode step (fp32 state in HBM; fp32 arithmetic: 1e-5 for fp32 io, 1e-2 bf16)
+DTOL = {"f32": 1e-5, "bf16": 1e-2}
+
+
+def decode_inputs(batch, H, P, N, io, seed, step):
+    return gen.make_ssd_decode_inputs(batch, H, P, N, io, seed, step)
+
+
+@pytest.mark.parametrize("N", [32, 64, 128, 256])
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("optional", [True, False])
+def test_ssd_decode_shapes(N, io, optional):
+    """Odd head counts and widths (3 x 5 heads of 7), 10 carried steps."""
+    from selective_state_space_39_b200 import ssm_ssd_state_update
+    batch, H, P = 3, 5, 7
+    seed = N + (3 if optional else 0)
+    const = gen.ssd_constants(H, seed)
+    rng = np.random.default_rng(seed)
+    state = torch.from_numpy(rng.standard_normal((batch, H, P, N)).astype(np.float32)).cuda()
+    ref = host(state).copy()
+    kw = dict(D=const["D"], dt_bias=const["dt_bias"]) if optional else {}
+    for step in range(10):
+        inp = decode_inputs(batch, H, P, N, io, seed, step)
+        y = ssm_ssd_state_update(state, dev(inp["x"]), dev(inp["dt"]), dev(const["A"]),
+                                 dev(inp["B"]), dev(inp["C"]),
+                                 **{k: dev(v) for k, v in kw.items()})
+        yr = oracle.ssd_state_update(ref, inp["x"], inp["dt"], const["A"], inp["B"], inp["C"],
+                                     io=io, **kw)
+        assert rel_err(host(y), yr) <= DTOL[io], f"step {step}"
+    assert rel_err(host(state), ref) <= DTOL[io]
+
+
+def test_ssd_decode_workload_sampled():
+    """64 sequences x 64 heads x 64, d_state 128, bf16, 1000 carried steps; the
+    oracle runs the same steps on sampled sequences and heads."""
+    from selective_state_space_39_b200 import ssm_ssd_state_update
+    w = gen.SSD_DECODE_WORKLOADS["ssd_decode_b64_h64_p64_n128_x1000"]
+    const = gen.ssd_constants(w.nheads, w.seed)
+    A, D, bias = dev(const["A"]), dev(const["D"]), dev(const["dt_bias"])
+    state = torch.zeros((w.batch, w.nheads, w.headdim, w.dstate), dtype=torch.float32,
+                        device="cuda")
+    bs, hs = np.array([0, 1, 31, 63]), np.array([0, 5, 32, 63])
+    ref = np.zeros((len(bs), len(hs), w.headdim, w.dstate))
+    sub = lambda a: np.ascontiguousarray(a[bs][:, hs])  # noqa: E731
+    ys, yrs = [], []
+    for step in range(w.steps):
+        inp = decode_inputs(w.batch, w.nheads, w.headdim, w.dstate, w.io, w.seed, step)
+        y = ssm_ssd_state_update(state, dev(inp["x"]), dev(inp["dt"]), A, dev(inp["B"]),
+                                 dev(inp["C"]), D=D, dt_bias=bias)
+        if step % 50 == 49 or step < 3:
+            ys.append(host(y)[bs][:, hs])
+        yr = oracle.ssd_state_update(ref, sub(inp["x"]), sub(inp["dt"]),
+                                     np.ascontiguousarray(const["A"][hs]),
+                                     np.ascontiguousarray(inp["B"][bs]),
+                                     np.ascontiguousarray(inp["C"][bs]), D=const["D"][hs],
+                                     dt_bias=const["dt_bias"][hs], io=w.io)
+        if step % 50 == 49 or step < 3:
+            yrs.append(yr)
+    ey = rel_err(np.stack(ys), np.stack(yrs))
+    eh = rel_err(host(state)[bs][:, hs], ref)
+    print(f"ssd decode 1000 steps: rel err y {ey:.3e} state {eh:.3e}")
+    assert torch.isfinite(state).all()
+    assert ey <= DTOL["bf16"] and eh <= DTOL["bf16"]
+
+
+def test_ssd_decode_steps_equal_the_scan():
+    """L decode steps on the GPU match the GPU's chunked SSD scan over the same
+    tokens (bf16; the scan's tensor-core operands set the bound)."""
+    from selective_state_space_39_b200 import ssm_ssd_scan_fwd, ssm_ssd_state_update
+    inp = gen.make_ssd_inputs(2, 70, 3, 64, 128, "bf16", 23, with_h0=True)
+    d = {k: dev(v) for k, v in inp.items()}
+    y, hl = ssm_ssd_scan_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], D=d["D"],
+                             dt_bias=d["dt_bias"], h0=d["h0"], return_last_state=True)
+    state = d["h0"].clone()
+    yd = []
+    for t in range(70):
+        col = lambda k: dev(np.ascontiguousarray(inp[k][:, t]))  # noqa: E731
+        yd.append(ssm_ssd_state_update(state, col("x"), col("dt"), d["A"], col("B"), col("C"),
+                                       D=d["D"], dt_bias=d["dt_bias"]))
+    assert rel_err(host(torch.stack(yd, dim=1)), host(y)) <= TOL
+    assert rel_err(host(state), host(hl)) <= TOL
+
