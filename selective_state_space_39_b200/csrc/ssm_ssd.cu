@@ -48,11 +48,12 @@ struct SsdLayout {
   static constexpr int x_elems = kQ * kPadX;      // one buffer
   static constexpr int bc_elems = kQ * kPadN;     // one buffer of B (or C)
   static constexpr int g_elems = kQ * kPadG;      // one buffer of G (two)
-  static constexpr int h_elems = kP * kPadN;      // one bf16 state copy (two)
-  static constexpr int bf16_bytes =
-      2 * (kStages * (x_elems + 2 * bc_elems) + 2 * g_elems + 2 * h_elems);
+  static constexpr int bf16_bytes = 2 * (kStages * (x_elems + 2 * bc_elems) + 2 * g_elems);
   static constexpr int step_floats = 4 * kQ + 4;  // Delta, cum, e^cum, w, e^cum_end
-  static constexpr int bytes = bf16_bytes + 4 * kStages * step_floats;
+  // half of C H from the warps holding the upper state columns: per state
+  // row tile, 16 floats per lane
+  static constexpr int part_floats = 4 * 32 * 16;
+  static constexpr int bytes = bf16_bytes + 4 * kStages * step_floats + 4 * part_floats;
   static_assert(bf16_bytes % 16 == 0, "float arrays start 16-byte aligned");
 };
 
@@ -88,6 +89,27 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool v
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;"); }
 __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+// Named barriers between the two warps that share state rows: the producer
+// arrives (its shared-memory writes become visible to the consumer), the
+// consumer waits. Both warps pass one of each per chunk, unconditionally.
+// Barrier ids 1..4 (one per pair, id 0 is __syncthreads), 64 threads each;
+// immediate ids so that the kernel reserves five barriers, not sixteen.
+__device__ __forceinline__ void named_arrive(int pair) {
+  switch (pair) {
+    case 0: asm volatile("bar.arrive 1, 64;" ::: "memory"); break;
+    case 1: asm volatile("bar.arrive 2, 64;" ::: "memory"); break;
+    case 2: asm volatile("bar.arrive 3, 64;" ::: "memory"); break;
+    default: asm volatile("bar.arrive 4, 64;" ::: "memory"); break;
+  }
+}
+__device__ __forceinline__ void named_sync(int pair) {
+  switch (pair) {
+    case 0: asm volatile("bar.sync 1, 64;" ::: "memory"); break;
+    case 1: asm volatile("bar.sync 2, 64;" ::: "memory"); break;
+    case 2: asm volatile("bar.sync 3, 64;" ::: "memory"); break;
+    default: asm volatile("bar.sync 4, 64;" ::: "memory"); break;
+  }
 }
 // Both halves of a bf16 pair times their own weight, repacked.
 __device__ __forceinline__ uint32_t scale_bf16x2(uint32_t v, float lo, float hi) {
@@ -139,15 +161,17 @@ __device__ __forceinline__ void chunk_g(const uint16_t* Bb, const uint16_t* Cb, 
   *reinterpret_cast<uint32_t*>(Gd + tb * kPadG + s0) = pack_bf16x2(g2, g3);
 }
 
-// One CTA per (head, batch row); 8 warps. Warp w owns rows 16*(w/4).. of
-// S, G and Y; columns 8*(w%4).. of S and G, 16*(w%4).. of Y; and the state
-// tile rows 16*(w%4).. (p) x columns (w/4)*N/2.. (n).
+// One CTA per (head, batch row); 8 warps. Warp w owns the S / G tile rows
+// 16*(w/4).., columns 8*(w%4)..; and the state tile rows p in 16*(w%4)..,
+// state columns (w/4)*N/2... The readout C H is taken from the state
+// accumulators themselves: each warp forms it over its half of the states for
+// its 16 rows p and all 32 steps, the warp holding the upper half hands its
+// sum over (named barrier per pair), and the other finishes Y for those rows.
 //
 // Software pipeline, one CTA barrier per chunk: iteration c computes G of
 // chunk c+1, Y and the state update of chunk c, the step quantities of chunk
 // c+2 (warp kStepWarp), and has the x/B/C copy of chunk c+2 in flight. x, B, C and
-// the step quantities rotate through three buffers; G and the bf16 state
-// copy through two.
+// the step quantities rotate through three buffers; G through two.
 template <int N>
 __global__ void __launch_bounds__(kThreads, (N <= 128) ? 2 : 1) ssd_fwd_kernel(const SsdParams p) {
   using Lay = SsdLayout<N>;
@@ -161,8 +185,8 @@ __global__ void __launch_bounds__(kThreads, (N <= 128) ? 2 : 1) ssd_fwd_kernel(c
   uint16_t* Bs = Xs + kS * Lay::x_elems;
   uint16_t* Cs = Bs + kS * Lay::bc_elems;
   uint16_t* Gs = Cs + kS * Lay::bc_elems;
-  uint16_t* Hs = Gs + 2 * Lay::g_elems;
   float* fbase = reinterpret_cast<float*>(smem_raw + Lay::bf16_bytes);
+  float4* part = reinterpret_cast<float4*>(fbase + kS * Lay::step_floats);
   auto step_buf = [&](int i) {
     float* f = fbase + i * Lay::step_floats;
     return StepBuf{f, f + kQ, f + 2 * kQ, f + 3 * kQ, f + 4 * kQ};
@@ -202,15 +226,7 @@ __global__ void __launch_bounds__(kThreads, (N <= 128) ? 2 : 1) ssd_fwd_kernel(c
       hacc[j][0] = hacc[j][1] = hacc[j][2] = hacc[j][3] = 0.f;
     }
   }
-  auto store_state_bf16 = [&](uint16_t* Hd) {
-#pragma unroll
-    for (int j = 0; j < kNT; ++j) {
-      const int n = ng * kNW + 8 * j + 2 * tig;
-      *reinterpret_cast<uint32_t*>(Hd + p0 * kPadN + n) = pack_bf16x2(hacc[j][0], hacc[j][1]);
-      *reinterpret_cast<uint32_t*>(Hd + (p0 + 8) * kPadN + n) =
-          pack_bf16x2(hacc[j][2], hacc[j][3]);
-    }
-  };
+
 
   // ---- chunk loader (x: kQ rows of 128 B; B, C: kQ rows of 2N B)
   auto load_chunk = [&](int c) {
@@ -272,7 +288,6 @@ __global__ void __launch_bounds__(kThreads, (N <= 128) ? 2 : 1) ssd_fwd_kernel(c
       if (nchunks > 1) chunk_steps(1, load_dt(1));
       dt_raw = load_dt(2);
     }
-    store_state_bf16(Hs);
     cp_async_wait_all();
     __syncthreads();
     chunk_g<N>(Bs, Cs, Gs, step_buf(0), rt, cq, lane);
@@ -298,58 +313,41 @@ __global__ void __launch_bounds__(kThreads, (N <= 128) ? 2 : 1) ssd_fwd_kernel(c
       const uint16_t* Bb = Bs + buf * Lay::bc_elems;
       const uint16_t* Cb = Cs + buf * Lay::bc_elems;
       const uint16_t* Gb = Gs + (c & 1) * Lay::g_elems;
-      const uint16_t* Hb = Hs + (c & 1) * Lay::h_elems;
 
-      // ---- Y = G X + diag(e^cum) C H + D x on rows 16 rt.., columns 16 cq..
-      {
-        float y1[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-        float y2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-        float y3[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};  // odd k-steps of C H
+      // ---- C H for rows t (both row tiles) x this warp's 16 state rows p, over
+      // its half of the states: the fp32 state accumulators, packed to bf16,
+      // are the B operand as they stand (rows p, state pairs 2 tig, 2 tig + 1).
+      float yc[2][2][4];
 #pragma unroll
-        for (int k0 = 0; k0 < kQ; k0 += 16) {
-          if (k0 <= 16 * rt) {
-            uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
-            ldsm_x4(smem_u32(Gb + (16 * rt + (lane & 15)) * kPadG + k0 + (lane >> 4) * 8), a0,
-                    a1, a2, a3);
-            ldsm_x4_t(smem_u32(Xb + (k0 + (lane & 7) + ((lane >> 3) & 1) * 8) * kPadX +
-                               16 * cq + (lane >> 4) * 8),
-                      b0, b1, b2, b3);
-            mma_bf16(y1[0], a0, a1, a2, a3, b0, b1);
-            mma_bf16(y1[1], a0, a1, a2, a3, b2, b3);
-          }
+      for (int r = 0; r < 2; ++r)
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) yc[r][q][e] = 0.f;
+#pragma unroll
+      for (int i = 0; i < kNT / 2; ++i) {
+        const uint32_t b00 = pack_bf16x2(hacc[2 * i][0], hacc[2 * i][1]);
+        const uint32_t b01 = pack_bf16x2(hacc[2 * i + 1][0], hacc[2 * i + 1][1]);
+        const uint32_t b10 = pack_bf16x2(hacc[2 * i][2], hacc[2 * i][3]);
+        const uint32_t b11 = pack_bf16x2(hacc[2 * i + 1][2], hacc[2 * i + 1][3]);
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(smem_u32(Cb + (16 * r + (lane & 15)) * kPadN + ng * kNW + 16 * i +
+                           (lane >> 4) * 8),
+                  a0, a1, a2, a3);
+          mma_bf16(yc[r][0], a0, a1, a2, a3, b00, b01);
+          mma_bf16(yc[r][1], a0, a1, a2, a3, b10, b11);
         }
+      }
+      if (ng == 1) {  // hand the upper half to the warp with the same rows p
 #pragma unroll
-        for (int k0 = 0; k0 < N; k0 += 16) {
-          uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
-          ldsm_x4(smem_u32(Cb + (16 * rt + (lane & 15)) * kPadN + k0 + (lane >> 4) * 8), a0, a1,
-                  a2, a3);
-          ldsm_x4(smem_u32(Hb + (16 * cq + (lane & 7) + (lane >> 4) * 8) * kPadN + k0 +
-                           ((lane >> 3) & 1) * 8),
-                  b0, b1, b2, b3);
-          float (&ya)[2][4] = (k0 & 16) ? y3 : y2;
-          mma_bf16(ya[0], a0, a1, a2, a3, b0, b1);
-          mma_bf16(ya[1], a0, a1, a2, a3, b2, b3);
-        }
+        for (int r = 0; r < 2; ++r)
 #pragma unroll
-        for (int j = 0; j < 2; ++j)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) y2[j][e] += y3[j][e];
-        const int ta = 16 * rt + g, tb = ta + 8;
-        const float ea = st.ecum[ta], eb = st.ecum[tb];
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const int pc = 16 * cq + 8 * j + 2 * tig;
-          const uint32_t xa = *reinterpret_cast<const uint32_t*>(Xb + ta * kPadX + pc);
-          const uint32_t xb = *reinterpret_cast<const uint32_t*>(Xb + tb * kPadX + pc);
-          if (t0 + ta < L)
-            *reinterpret_cast<uint32_t*>(yg + (size_t)(t0 + ta) * row_x + pc) =
-                pack_bf16x2(fmaf(Dh, bf16_lo(xa), fmaf(ea, y2[j][0], y1[j][0])),
-                            fmaf(Dh, bf16_hi(xa), fmaf(ea, y2[j][1], y1[j][1])));
-          if (t0 + tb < L)
-            *reinterpret_cast<uint32_t*>(yg + (size_t)(t0 + tb) * row_x + pc) =
-                pack_bf16x2(fmaf(Dh, bf16_lo(xb), fmaf(eb, y2[j][2], y1[j][2])),
-                            fmaf(Dh, bf16_hi(xb), fmaf(eb, y2[j][3], y1[j][3])));
-        }
+          for (int q = 0; q < 2; ++q)
+            part[(pt * 4 + r * 2 + q) * 32 + lane] =
+                make_float4(yc[r][q][0], yc[r][q][1], yc[r][q][2], yc[r][q][3]);
+        named_arrive(pt);
       }
 
       // ---- H <- e^{cum_end} H + (w X)^T B on rows 16 pt.. (p), columns ng N/2.. (n)
@@ -381,7 +379,60 @@ __global__ void __launch_bounds__(kThreads, (N <= 128) ? 2 : 1) ssd_fwd_kernel(c
             mma_bf16(hacc[j + 1], a0, a1, a2, a3, b2, b3);
           }
         }
-        store_state_bf16(Hs + ((c + 1) & 1) * Lay::h_elems);
+      }
+
+      // ---- Y = G X + diag(e^cum) C H + D x on rows t (both tiles), columns 16 pt..
+      if (ng == 0) {
+        float y1[2][2][4];
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+#pragma unroll
+          for (int q = 0; q < 2; ++q)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) y1[r][q][e] = 0.f;
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+#pragma unroll
+          for (int k0 = 0; k0 <= 16 * r; k0 += 16) {
+            uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
+            ldsm_x4(smem_u32(Gb + (16 * r + (lane & 15)) * kPadG + k0 + (lane >> 4) * 8), a0,
+                    a1, a2, a3);
+            ldsm_x4_t(smem_u32(Xb + (k0 + (lane & 7) + ((lane >> 3) & 1) * 8) * kPadX +
+                               16 * pt + (lane >> 4) * 8),
+                      b0, b1, b2, b3);
+            mma_bf16(y1[r][0], a0, a1, a2, a3, b0, b1);
+            mma_bf16(y1[r][1], a0, a1, a2, a3, b2, b3);
+          }
+        named_sync(pt);
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const float4 o = part[(pt * 4 + r * 2 + q) * 32 + lane];
+            yc[r][q][0] += o.x;
+            yc[r][q][1] += o.y;
+            yc[r][q][2] += o.z;
+            yc[r][q][3] += o.w;
+          }
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const int ta = 16 * r + g, tb = ta + 8;
+          const float ea = st.ecum[ta], eb = st.ecum[tb];
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const int pc = 16 * pt + 8 * q + 2 * tig;
+            const uint32_t xa = *reinterpret_cast<const uint32_t*>(Xb + ta * kPadX + pc);
+            const uint32_t xb = *reinterpret_cast<const uint32_t*>(Xb + tb * kPadX + pc);
+            if (t0 + ta < L)
+              *reinterpret_cast<uint32_t*>(yg + (size_t)(t0 + ta) * row_x + pc) =
+                  pack_bf16x2(fmaf(Dh, bf16_lo(xa), fmaf(ea, yc[r][q][0], y1[r][q][0])),
+                              fmaf(Dh, bf16_hi(xa), fmaf(ea, yc[r][q][1], y1[r][q][1])));
+            if (t0 + tb < L)
+              *reinterpret_cast<uint32_t*>(yg + (size_t)(t0 + tb) * row_x + pc) =
+                  pack_bf16x2(fmaf(Dh, bf16_lo(xb), fmaf(eb, yc[r][q][2], y1[r][q][2])),
+                              fmaf(Dh, bf16_hi(xb), fmaf(eb, yc[r][q][3], y1[r][q][3])));
+          }
+        }
       }
       cp_async_wait_all();
       __syncthreads();
