@@ -10,9 +10,9 @@
 namespace ssm {
 
 // Steps per CTA chunk along the sequence (measured best on the 8 x 2048 x
-// 1536 bf16 layer among 32, 64, 128): forward 32, backward 128.
+// 1536 bf16 layer among 32 .. 256): forward 32, backward 256.
 constexpr int kConvChunkFwd = 32;
-constexpr int kConvChunkBwd = 128;
+constexpr int kConvChunkBwd = 256;
 
 struct ConvParams {
   int batch, seqlen, dim, width, chunk;
