@@ -824,6 +824,55 @@ def ssd_decode_bench(args):
     return 0
 
 
+def decode_reference_arm(args):
+    """--impl reference on a decode workload: the fp64 oracle's decode step over
+    every batch row and channel (or head row) of the workload, one call per
+    step, on the host (rank 0 only)."""
+    import oracle
+    ssd = args.workload in gen.SSD_DECODE_WORKLOADS
+    w = (gen.SSD_DECODE_WORKLOADS if ssd else gen.DECODE_WORKLOADS)[args.workload]
+    if ssd:
+        const = gen.ssd_constants(w.nheads, w.seed)
+        state = np.zeros((w.batch, w.nheads, w.headdim, w.dstate))
+        rows = w.batch * w.nheads * w.headdim
+    else:
+        const = gen.decode_constants(w.dim, w.dstate, w.seed)
+        state = np.zeros((w.batch, w.dim, w.dstate))
+        rows = w.batch * w.dim
+    times = []
+    for i in range(args.warmup + args.steps):
+        if ssd:
+            d = gen.make_ssd_decode_inputs(w.batch, w.nheads, w.headdim, w.dstate, w.io, w.seed,
+                                           i)
+            t0 = time.perf_counter()
+            oracle.ssd_state_update(state, d["x"], d["dt"], const["A"], d["B"], d["C"],
+                                    D=const["D"], dt_bias=const["dt_bias"], io=w.io)
+        else:
+            d = gen.make_decode_inputs(w.batch, w.dim, w.dstate, w.io, w.seed, i)
+            t0 = time.perf_counter()
+            oracle.state_update(state, d["x"], d["delta"], const["A"], d["B"], d["C"],
+                                D=const["D"], z=d["z"], delta_bias=const["delta_bias"], io=w.io)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = args.steps * rows / total
+    unit = "rows/s" if ssd else "elements/s"
+    line = {
+        "impl": "reference",
+        "metric": ("SSD decode state-update rows/s (B·H·P per step) and HBM GB/s" if ssd else
+                   "decode state-update elements/s (B·D per step) and HBM GB/s"),
+        "value": value, "unit": unit, "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": w.name},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": 1, "kind": "oracle",
+                         "sample": "every row of the workload, one decode step per step"},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def ssd_reference_arm(args):
     """--impl reference on an SSD workload: the fp64 oracle, one (batch, head)
     pair per step, on the host (rank 0 only)."""
@@ -863,8 +912,12 @@ def main():
     if args.op == "ssd" and args.workload not in gen.SSD_WORKLOADS:
         args.workload = DEFAULT_SSD_WORKLOAD
     if args.impl == "reference":
+        if int(os.environ.get("RANK", 0)) != 0:
+            return 0
         if args.workload in gen.SSD_WORKLOADS:
-            return ssd_reference_arm(args) if int(os.environ.get("RANK", 0)) == 0 else 0
+            return ssd_reference_arm(args)
+        if args.workload in gen.DECODE_WORKLOADS or args.workload in gen.SSD_DECODE_WORKLOADS:
+            return decode_reference_arm(args)
         return reference_arm(args)
     if args.workload in gen.SSD_WORKLOADS:
         return ssd_bench(args)
