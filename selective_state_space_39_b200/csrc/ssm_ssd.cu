@@ -90,19 +90,11 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
-// Named barriers between the two warps that share state rows: the producer
-// arrives (its shared-memory writes become visible to the consumer), the
-// consumer waits. Both warps pass one of each per chunk, unconditionally.
-// Barrier ids 1..4 (one per pair, id 0 is __syncthreads), 64 threads each;
-// immediate ids so that the kernel reserves five barriers, not sixteen.
-__device__ __forceinline__ void named_arrive(int pair) {
-  switch (pair) {
-    case 0: asm volatile("bar.arrive 1, 64;" ::: "memory"); break;
-    case 1: asm volatile("bar.arrive 2, 64;" ::: "memory"); break;
-    case 2: asm volatile("bar.arrive 3, 64;" ::: "memory"); break;
-    default: asm volatile("bar.arrive 4, 64;" ::: "memory"); break;
-  }
-}
+// Named barrier of the two warps that share state rows (ids 1..4, one per
+// pair; id 0 is __syncthreads), 64 threads: both warps write their hand-over
+// to shared memory, pass the barrier (which makes the writes visible to the
+// partner), then read the partner's. Both pass it once per chunk,
+// unconditionally. Immediate ids: the kernel reserves five barriers.
 __device__ __forceinline__ void named_sync(int pair) {
   switch (pair) {
     case 0: asm volatile("bar.sync 1, 64;" ::: "memory"); break;
@@ -165,8 +157,9 @@ __device__ __forceinline__ void chunk_g(const uint16_t* Bb, const uint16_t* Cb, 
 // 16*(w/4).., columns 8*(w%4)..; and the state tile rows p in 16*(w%4)..,
 // state columns (w/4)*N/2... The readout C H is taken from the state
 // accumulators themselves: each warp forms it over its half of the states for
-// its 16 rows p and all 32 steps, the warp holding the upper half hands its
-// sum over (named barrier per pair), and the other finishes Y for those rows.
+// its 16 rows p and all 32 steps; the two warps of a pair exchange halves
+// through shared memory (a named barrier per pair) and each finishes Y for
+// one row tile of those rows.
 //
 // Software pipeline, one CTA barrier per chunk: iteration c computes G of
 // chunk c+1, Y and the state update of chunk c, the step quantities of chunk
@@ -340,14 +333,14 @@ __global__ void __launch_bounds__(kThreads, (N <= 128) ? 2 : 1) ssd_fwd_kernel(c
           mma_bf16(yc[r][1], a0, a1, a2, a3, b10, b11);
         }
       }
-      if (ng == 1) {  // hand the upper half to the warp with the same rows p
+      // Each warp of a pair finishes one row tile of Y (ng = 0: steps 0..15,
+      // ng = 1: steps 16..31) and hands its half-state sum for the other
+      // tile to its partner.
 #pragma unroll
-        for (int r = 0; r < 2; ++r)
-#pragma unroll
-          for (int q = 0; q < 2; ++q)
-            part[(pt * 4 + r * 2 + q) * 32 + lane] =
-                make_float4(yc[r][q][0], yc[r][q][1], yc[r][q][2], yc[r][q][3]);
-        named_arrive(pt);
+      for (int q = 0; q < 2; ++q) {  // static indices: yc stays in registers
+        const float4 v0 = make_float4(yc[0][q][0], yc[0][q][1], yc[0][q][2], yc[0][q][3]);
+        const float4 v1 = make_float4(yc[1][q][0], yc[1][q][1], yc[1][q][2], yc[1][q][3]);
+        part[((pt * 2 + ng) * 2 + q) * 32 + lane] = ng ? v0 : v1;  // the partner's tile
       }
 
       // ---- H <- e^{cum_end} H + (w X)^T B on rows 16 pt.. (p), columns ng N/2.. (n)
@@ -381,57 +374,48 @@ __global__ void __launch_bounds__(kThreads, (N <= 128) ? 2 : 1) ssd_fwd_kernel(c
         }
       }
 
-      // ---- Y = G X + diag(e^cum) C H + D x on rows t (both tiles), columns 16 pt..
-      if (ng == 0) {
-        float y1[2][2][4];
+      // ---- Y = G X + diag(e^cum) C H + D x on row tile r = ng, columns 16 pt..
+      {
+        const int r = ng;
+        float y1[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-        for (int r = 0; r < 2; ++r)
-#pragma unroll
-          for (int q = 0; q < 2; ++q)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) y1[r][q][e] = 0.f;
-#pragma unroll
-        for (int r = 0; r < 2; ++r)
-#pragma unroll
-          for (int k0 = 0; k0 <= 16 * r; k0 += 16) {
+        for (int k0 = 0; k0 < kQ; k0 += 16) {
+          if (k0 <= 16 * r) {
             uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
             ldsm_x4(smem_u32(Gb + (16 * r + (lane & 15)) * kPadG + k0 + (lane >> 4) * 8), a0,
                     a1, a2, a3);
             ldsm_x4_t(smem_u32(Xb + (k0 + (lane & 7) + ((lane >> 3) & 1) * 8) * kPadX +
                                16 * pt + (lane >> 4) * 8),
                       b0, b1, b2, b3);
-            mma_bf16(y1[r][0], a0, a1, a2, a3, b0, b1);
-            mma_bf16(y1[r][1], a0, a1, a2, a3, b2, b3);
+            mma_bf16(y1[0], a0, a1, a2, a3, b0, b1);
+            mma_bf16(y1[1], a0, a1, a2, a3, b2, b3);
           }
-        named_sync(pt);
+        }
+        named_sync(pt);  // both warps of the pair have written their hand-over
+        float ysum[2][4];
 #pragma unroll
-        for (int r = 0; r < 2; ++r)
+        for (int q = 0; q < 2; ++q) {
+          const float4 o = part[((pt * 2 + (1 - ng)) * 2 + q) * 32 + lane];
+          ysum[q][0] = (ng ? yc[1][q][0] : yc[0][q][0]) + o.x;
+          ysum[q][1] = (ng ? yc[1][q][1] : yc[0][q][1]) + o.y;
+          ysum[q][2] = (ng ? yc[1][q][2] : yc[0][q][2]) + o.z;
+          ysum[q][3] = (ng ? yc[1][q][3] : yc[0][q][3]) + o.w;
+        }
+        const int ta = 16 * r + g, tb = ta + 8;
+        const float ea = st.ecum[ta], eb = st.ecum[tb];
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            const float4 o = part[(pt * 4 + r * 2 + q) * 32 + lane];
-            yc[r][q][0] += o.x;
-            yc[r][q][1] += o.y;
-            yc[r][q][2] += o.z;
-            yc[r][q][3] += o.w;
-          }
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          const int ta = 16 * r + g, tb = ta + 8;
-          const float ea = st.ecum[ta], eb = st.ecum[tb];
-#pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            const int pc = 16 * pt + 8 * q + 2 * tig;
-            const uint32_t xa = *reinterpret_cast<const uint32_t*>(Xb + ta * kPadX + pc);
-            const uint32_t xb = *reinterpret_cast<const uint32_t*>(Xb + tb * kPadX + pc);
-            if (t0 + ta < L)
-              *reinterpret_cast<uint32_t*>(yg + (size_t)(t0 + ta) * row_x + pc) =
-                  pack_bf16x2(fmaf(Dh, bf16_lo(xa), fmaf(ea, yc[r][q][0], y1[r][q][0])),
-                              fmaf(Dh, bf16_hi(xa), fmaf(ea, yc[r][q][1], y1[r][q][1])));
-            if (t0 + tb < L)
-              *reinterpret_cast<uint32_t*>(yg + (size_t)(t0 + tb) * row_x + pc) =
-                  pack_bf16x2(fmaf(Dh, bf16_lo(xb), fmaf(eb, yc[r][q][2], y1[r][q][2])),
-                              fmaf(Dh, bf16_hi(xb), fmaf(eb, yc[r][q][3], y1[r][q][3])));
-          }
+        for (int q = 0; q < 2; ++q) {
+          const int pc = 16 * pt + 8 * q + 2 * tig;
+          const uint32_t xa = *reinterpret_cast<const uint32_t*>(Xb + ta * kPadX + pc);
+          const uint32_t xb = *reinterpret_cast<const uint32_t*>(Xb + tb * kPadX + pc);
+          if (t0 + ta < L)
+            *reinterpret_cast<uint32_t*>(yg + (size_t)(t0 + ta) * row_x + pc) =
+                pack_bf16x2(fmaf(Dh, bf16_lo(xa), fmaf(ea, ysum[q][0], y1[q][0])),
+                            fmaf(Dh, bf16_hi(xa), fmaf(ea, ysum[q][1], y1[q][1])));
+          if (t0 + tb < L)
+            *reinterpret_cast<uint32_t*>(yg + (size_t)(t0 + tb) * row_x + pc) =
+                pack_bf16x2(fmaf(Dh, bf16_lo(xb), fmaf(eb, ysum[q][2], y1[q][2])),
+                            fmaf(Dh, bf16_hi(xb), fmaf(eb, ysum[q][3], y1[q][3])));
         }
       }
       cp_async_wait_all();
