@@ -14,10 +14,11 @@
 //   Y       = G X + diag(e^{cum}) C H + D X
 //   H      <- e^{cum_end} H + (w X)^T B,   w_s = e^{cum_end - cum_s} Delta_s
 // The four products (C B^T, G X, C H, (w X)^T B) are bf16 tensor-core MMAs
-// (mma.sync m16n8k16, fp32 accumulation) fed from shared memory by ldmatrix;
-// x, B and C chunks arrive by cp.async two chunks ahead (zero-filled past the
-// end of the sequence, where Delta is taken as 0 so that the padded steps
-// change nothing).
+// (mma.sync m16n8k16, fp32 accumulation) fed from shared memory by ldmatrix,
+// except that C H reads the state from the accumulators it lives in; x, B and
+// C chunks arrive by cp.async two chunks ahead (zero-filled past the end of
+// the sequence, where Delta is taken as 0 so that the padded steps change
+// nothing).
 #include <mutex>
 #include <set>
 #include <utility>
@@ -50,9 +51,9 @@ struct SsdLayout {
   static constexpr int g_elems = kQ * kPadG;      // one buffer of G (two)
   static constexpr int bf16_bytes = 2 * (kStages * (x_elems + 2 * bc_elems) + 2 * g_elems);
   static constexpr int step_floats = 4 * kQ + 4;  // Delta, cum, e^cum, w, e^cum_end
-  // half of C H from the warps holding the upper state columns: per state
-  // row tile, 16 floats per lane
-  static constexpr int part_floats = 4 * 32 * 16;
+  // the C H halves the two warps of a state-row pair hand each other: per
+  // pair and direction, one row tile of 16 x 16 fp32 (8 floats per lane)
+  static constexpr int part_floats = 4 * 2 * 32 * 8;
   static constexpr int bytes = bf16_bytes + 4 * kStages * step_floats + 4 * part_floats;
   static_assert(bf16_bytes % 16 == 0, "float arrays start 16-byte aligned");
 };
@@ -163,8 +164,8 @@ __device__ __forceinline__ void chunk_g(const uint16_t* Bb, const uint16_t* Cb, 
 //
 // Software pipeline, one CTA barrier per chunk: iteration c computes G of
 // chunk c+1, Y and the state update of chunk c, the step quantities of chunk
-// c+2 (warp kStepWarp), and has the x/B/C copy of chunk c+2 in flight. x, B, C and
-// the step quantities rotate through three buffers; G through two.
+// c+2 (warp kStepWarp), and has the x/B/C copy of chunk c+2 in flight. x, B,
+// C and the step quantities rotate through three buffers; G through two.
 template <int N>
 __global__ void __launch_bounds__(kThreads, (N <= 128) ? 2 : 1) ssd_fwd_kernel(const SsdParams p) {
   using Lay = SsdLayout<N>;
