@@ -153,3 +153,46 @@ def test_pins_catch_planted_mistake(name, tmp_path):
         except (AssertionError, ValueError, FloatingPointError):
             failed.append(pin.__name__)
     assert failed, f"no pin caught the planted mistake {name}"
+
+
+# ---- property checks over random small shapes (CPU) ----------------------
+from hypothesis import given, settings  # noqa: E402
+from hypothesis import strategies as st  # noqa: E402
+
+
+@settings(max_examples=25, deadline=None)
+@given(batch=st.integers(1, 2), L=st.integers(1, 9), H=st.integers(1, 3), P=st.integers(1, 4),
+       N=st.integers(1, 5), seed=st.integers(0, 2**31 - 1), h0=st.booleans())
+def test_ssd_equals_tied_scan_any_shape(o, batch, L, H, P, N, seed, h0):
+    """For any small shape, an SSD head equals the per-channel scan with A tied
+    across states and Delta, D, bias tied across the head's channels."""
+    c = pins._ssd_case(seed, batch=batch, L=L, H=H, P=P, N=N, h0=h0)
+    y, hl = pins._ssd(o, c)
+    dim = H * P
+    tie = lambda v: np.repeat(v, P, axis=-1)  # noqa: E731
+    h0v = None if c["h0"] is None else c["h0"].reshape(batch, dim, N)
+    ys, hs = o.selective_scan(c["x"].reshape(batch, L, dim), tie(c["dt"]),
+                              np.repeat(tie(c["A"])[:, None], N, axis=1), c["B"], c["C"],
+                              D=tie(c["D"]), delta_bias=tie(c["dt_bias"]), h0=h0v)
+    assert np.allclose(y, ys.reshape(batch, L, H, P), rtol=1e-12, atol=1e-12)
+    assert np.allclose(hl, hs.reshape(batch, H, P, N), rtol=1e-12, atol=1e-12)
+
+
+@settings(max_examples=25, deadline=None)
+@given(L=st.integers(1, 12), split=st.integers(0, 12), seed=st.integers(0, 2**31 - 1))
+def test_scan_split_anywhere(o, L, split, seed):
+    """Scanning [0, k) and then [k, L) from the state reached equals one scan,
+    for every k (the state carries everything; fp32 hand-over of the state)."""
+    k = min(split, L)
+    c = pins.random_case(seed, batch=1, L=L, dim=2, N=3, gate=False)
+    kw = dict(D=c["D"], delta_bias=c["delta_bias"])
+    y, hl = o.selective_scan(c["x"], c["delta"], c["A"], c["B"], c["C"], h0=c["h0"], **kw)
+    part = lambda a, s: np.ascontiguousarray(a[:, s])  # noqa: E731
+    y1, h1 = o.selective_scan(part(c["x"], slice(0, k)), part(c["delta"], slice(0, k)), c["A"],
+                              part(c["B"], slice(0, k)), part(c["C"], slice(0, k)),
+                              h0=c["h0"], **kw)
+    y2, h2 = o.selective_scan(part(c["x"], slice(k, L)), part(c["delta"], slice(k, L)), c["A"],
+                              part(c["B"], slice(k, L)), part(c["C"], slice(k, L)),
+                              h0=h1.astype(np.float32), **kw)
+    assert np.allclose(np.concatenate([y1, y2], axis=1), y, rtol=1e-6, atol=1e-6)
+    assert np.allclose(h2, hl, rtol=1e-6, atol=1e-6)
