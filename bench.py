@@ -919,6 +919,10 @@ def main():
         if args.workload in gen.DECODE_WORKLOADS or args.workload in gen.SSD_DECODE_WORKLOADS:
             return decode_reference_arm(args)
         return reference_arm(args)
+    single = (args.op == "conv" or args.workload in gen.SSD_WORKLOADS or
+              args.workload in gen.DECODE_WORKLOADS or args.workload in gen.SSD_DECODE_WORKLOADS)
+    if single and int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        raise SystemExit("this mode runs on one GPU (the batch-sharded scan runs on N)")
     if args.workload in gen.SSD_WORKLOADS:
         return ssd_bench(args)
     if args.workload in gen.SSD_DECODE_WORKLOADS:
