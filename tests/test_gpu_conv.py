@@ -115,3 +115,15 @@ def test_conv_update_steps_match_oracle(io, width):
         want = oracle.conv1d_silu_update(ref, xt, c["w"], c["bias"], io=io)
         assert rel_err(out, want) <= TOL[io], f"step {t}"
         assert rel_err(out, full[:, t]) <= TOL[io], f"step {t} vs the conv"
+
+
+def test_conv_empty_sequence():
+    """L = 0: the forward writes nothing, the backward returns zero dw and
+    dbias (sums over no steps)."""
+    from selective_state_space_39_b200 import ssm_conv1d_silu_bwd, ssm_conv1d_silu_fwd
+    c = gen.make_conv_inputs(2, 0, 64, 4, "bf16", 21)
+    out = ssm_conv1d_silu_fwd(dev(c["x"]), dev(c["w"]), dev(c["bias"]))
+    assert out.shape == (2, 0, 64)
+    g = ssm_conv1d_silu_bwd(dev(c["x"]), dev(c["w"]), dev(c["dout"]), dev(c["bias"]))
+    assert g["dx"].shape == (2, 0, 64)
+    assert torch.count_nonzero(g["dw"]) == 0 and torch.count_nonzero(g["dbias"]) == 0

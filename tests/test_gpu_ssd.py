@@ -201,3 +201,18 @@ def test_ssd_decode_steps_equal_the_scan():
     assert rel_err(host(torch.stack(yd, dim=1)), host(y)) <= TOL
     assert rel_err(host(state), host(hl)) <= TOL
 
+
+
+def test_ssd_empty_batch_and_heads():
+    """batch = 0 or heads = 0: nothing to compute, the calls succeed."""
+    from selective_state_space_39_b200 import ssm_ssd_scan_fwd, ssm_ssd_state_update
+    for batch, H in ((0, 3), (2, 0)):
+        inp = gen.make_ssd_inputs(batch, 16, H, 64, 64, "bf16", 3)
+        y = ssm_ssd_scan_fwd(dev(inp["x"]), dev(inp["dt"]), dev(inp["A"]), dev(inp["B"]),
+                             dev(inp["C"]))
+        assert y.shape == (batch, 16, H, 64)
+        d = gen.make_ssd_decode_inputs(batch, H, 64, 64, "bf16", 3, 0)
+        state = torch.zeros((batch, H, 64, 64), dtype=torch.float32, device="cuda")
+        yd = ssm_ssd_state_update(state, dev(d["x"]), dev(d["dt"]), dev(inp["A"]), dev(d["B"]),
+                                  dev(d["C"]))
+        assert yd.shape == (batch, H, 64)
