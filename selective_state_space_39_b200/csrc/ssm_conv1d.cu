@@ -16,8 +16,8 @@
 //
 // Design (B200): both directions are HBM-bound elementwise streams (a few
 // FLOPs per element), so the kernels are built for bandwidth: each thread owns
-// VEC adjacent channels (8-byte vector loads and stores: 4 bf16 or 2 fp32)
-// and a chunk of T steps, keeps the W-1 previous rows in registers (a sliding
+// VEC adjacent channels (vector loads and stores: 4 bf16 or 2 fp32 channels in
+// 8 bytes; 2 bf16 in 4 bytes in the bf16 backward) and a chunk of T steps, keeps the W-1 previous rows in registers (a sliding
 // window: every input element is read once, plus a W-1 row halo per chunk),
 // and issues the loads of several steps before using them. Warps cover
 // contiguous channel runs of a row, so every access is coalesced. The weight
@@ -440,8 +440,9 @@ bool conv_width_supported(int width) { return width >= 2 && width <= 4; }
 
 cudaError_t launch_conv(const ConvParams& p, bool bf16, bool vec, bool backward,
                         cudaStream_t stream) {
-  // 8-byte vectors (4 bf16 or 2 fp32 channels per thread): enough threads to
-  // fill every SM with the registers a thread needs
+  // Vector paths: 8-byte vectors (4 bf16 or 2 fp32 channels per thread), and
+  // for the bf16 backward 4-byte vectors (2 channels), whose 64 registers let
+  // five CTAs share an SM
   if (bf16) {
     if (!vec) return launch_w<uint16_t, 1>(p, backward, stream);
     return backward ? launch_w<uint16_t, kConvBwdVecBf16>(p, true, stream)
