@@ -93,3 +93,27 @@ def test_decode_steps_are_stream_slices():
     s3 = gen.make_decode_inputs(4, 8, 16, "bf16", 4, step=3)
     full = gen.fill((5, 4, 8), 4, gen.STREAM_X, out="bf16")
     assert np.array_equal(s3["x"], full[3])
+
+
+def test_ssd_recipe():
+    w = gen.SSD_WORKLOADS["ssd_mamba2_b4_l4096_h64_p64_n128"]
+    assert (w.batch, w.seqlen, w.nheads, w.headdim, w.dstate) == (4, 4096, 64, 64, 128)
+    assert w.with_h0 and w.elements == 4 * 4096 * 64 * 64
+    inp = gen.make_ssd_inputs(2, 9, 5, 64, 32, "bf16", 6, with_h0=True)
+    assert inp["x"].shape == (2, 9, 5, 64) and inp["x"].dtype == np.uint16
+    assert inp["dt"].shape == (2, 9, 5) and inp["B"].shape == (2, 9, 32)
+    assert inp["h0"].shape == (2, 5, 64, 32) and inp["h0"].dtype == np.float32
+    c = gen.ssd_constants(64, 6)
+    assert np.all((c["A"] <= -1.0) & (c["A"] >= -16.0)) and np.all(c["D"] == 1.0)
+    u = np.log1p(np.exp(c["dt_bias"].astype(np.float64)))
+    assert np.all((u > 0.00099) & (u < 0.1001))
+    # the scan's inputs carry the same per-head constants
+    assert np.array_equal(gen.make_ssd_inputs(1, 2, 64, 64, 32, "bf16", 6)["A"], c["A"])
+
+
+def test_ssd_decode_steps_are_stream_slices():
+    s3 = gen.make_ssd_decode_inputs(2, 3, 4, 32, "bf16", 7, step=3)
+    full = gen.fill((5, 2, 3, 4), 7, gen.STREAM_X, out="bf16")
+    assert np.array_equal(s3["x"], full[3])
+    full_b = gen.fill((5, 2, 32), 7, gen.STREAM_B, out="bf16")
+    assert np.array_equal(s3["B"], full_b[3])
