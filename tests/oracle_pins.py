@@ -664,6 +664,34 @@ def pin_ssd_split_invariance(o):
     _close(h2, hl, 1e-6, 1e-6, what="ssd end state")
 
 
+def pin_ssd_zero_step_keeps_state(o):
+    """Delta = 0 (no softplus, dt = 0, no bias): the state stays h0 and
+    y_t = C_t . h0 + D x_t, for every step."""
+    c = _ssd_case(315, L=6)
+    zero = np.zeros_like(c["dt"])
+    y, hl = o.ssd_scan(c["x"], zero, c["A"], c["B"], c["C"], D=c["D"], softplus=False,
+                       h0=c["h0"])
+    _close(hl, c["h0"], 0.0, 0.0, what="ssd zero step state")
+    want = (np.einsum("bhpn,btn->bthp", c["h0"].astype(np.float64), c["C"].astype(np.float64))
+            + c["D"].astype(np.float64)[None, None, :, None] * c["x"])
+    _close(y, want, 1e-13, 1e-13, what="ssd zero step y")
+
+
+def pin_ssd_large_step_is_memoryless(o):
+    """Delta = 2000 with A <= -0.5: exp(Delta A) <= e^-1000 underflows to an
+    exact zero in fp64, so the state after each step is Delta B_t x_t alone
+    (no softplus, no skip)."""
+    c = _ssd_case(317, L=5)
+    big = np.full_like(c["dt"], 2000.0)
+    y, hl = o.ssd_scan(c["x"], big, c["A"], c["B"], c["C"], softplus=False, h0=c["h0"])
+    S = 2000.0 * np.einsum("bhp,bn->bhpn", c["x"][:, -1].astype(np.float64),
+                           c["B"][:, -1].astype(np.float64))
+    _close(hl, S, 1e-14, 0.0, what="ssd memoryless state")
+    yt = 2000.0 * np.einsum("bthp,btn,btn->bthp", c["x"].astype(np.float64),
+                            c["B"].astype(np.float64), c["C"].astype(np.float64))
+    _close(y, yt, 1e-12, 1e-9, what="ssd memoryless y")
+
+
 def pin_ssd_decode_steps_equal_scan(o):
     """L SSD decode steps from h0 reproduce the (separately pinned) SSD scan:
     every y_t and the end state."""
@@ -730,6 +758,8 @@ ALL_PINS = [
     pin_ssd_is_tied_selective_scan,
     pin_ssd_A_zero_is_cumulative_outer_product,
     pin_ssd_split_invariance,
+    pin_ssd_zero_step_keeps_state,
+    pin_ssd_large_step_is_memoryless,
     pin_ssd_decode_steps_equal_scan,
     pin_ssd_decode_single_step_by_hand,
 ]
