@@ -1,8 +1,5 @@
 """The oracle against its pins (CPU only), and mutation checks: copies of the
 oracle source with one plausible mistake planted each must fail a pin."""
-import os
-import shutil
-
 import numpy as np
 import pytest
 
