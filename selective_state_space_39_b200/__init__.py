@@ -34,4 +34,4 @@ __all__ = ["ssm_scan_fwd", "ssm_scan_fwd_noalloc", "ssm_scan_bwd", "ssm_state_up
            "conv1d_silu_bwd_workspace_bytes",
            "ssm_delta_sum", "ssm_compose_carries", "ssm_ssd_scan_fwd",
            "ssm_ssd_state_update",
-           "SsmError", "SSM_DTYPE_F32", "SSM_DTYPE_BF16", "lib"]
+           "SsmError", "ScanPlan", "SSM_DTYPE_F32", "SSM_DTYPE_BF16", "lib"]

@@ -4,7 +4,6 @@ Bound (max|y - y_ref| / max|y_ref|, same for h_last): 1e-5 for fp32 io,
 1e-2 for bf16 io with fp32 state. Full-size workloads are checked on sampled
 channels (every step of each sampled channel), plus properties that hold at
 any size (no NaN/Inf, TMA path == plain-load path bit for bit)."""
-import os
 
 import numpy as np
 import pytest

@@ -3,9 +3,6 @@ device memory (it takes its scratch from an array the library reserves on
 each GPU). Checked through the C ABI against ssm_scan_fwd, which uses a
 caller-provided workspace, on two calls in a row that share the reserved
 scratch. This file is collected last on purpose."""
-import os
-
-import numpy as np
 import pytest
 import torch
 
