@@ -38,6 +38,16 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// Tensors past 2^40 elements are rejected: no GPU holds one, and every byte
+// count and index computed for an accepted call then stays far from 64-bit
+// overflow. The product is taken in double, which cannot overflow here.
+constexpr double kMaxElements = 1099511627776.0;
+bool too_large(std::initializer_list<int64_t> dims) {
+  double n = 1.0;
+  for (int64_t d : dims) n *= (double)d;
+  return n > kMaxElements;
+}
+
 bool overlap(const void* a, size_t na, const void* b, size_t nb) {
   if (!a || !b || na == 0 || nb == 0) return false;
   const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
@@ -51,6 +61,9 @@ int dims_status(const Dims& d) {
   if (!scan_dstate_supported((int)std::min<int64_t>(d.dstate, 1 << 20))) return SSM_ERR_UNSUPPORTED;
   // grid and index limits of this library
   if (d.batch > 65535 || d.dim > (1 << 24) || d.seqlen > (1 << 30)) return SSM_ERR_UNSUPPORTED;
+  if (too_large({d.batch, d.seqlen, d.dim}) || too_large({d.batch, d.seqlen, d.dstate}) ||
+      too_large({d.batch, d.dim, d.dstate}))
+    return SSM_ERR_UNSUPPORTED;
   return SSM_OK;
 }
 
@@ -117,6 +130,9 @@ int bwd_dims_status(const Dims& d) {
   if (!scan_bwd_dstate_supported((int)std::min<int64_t>(d.dstate, 1 << 20)))
     return SSM_ERR_UNSUPPORTED;
   if (d.batch > 65535 || d.dim > (1 << 24) || d.seqlen > (1 << 30)) return SSM_ERR_UNSUPPORTED;
+  if (too_large({d.batch, d.seqlen, d.dim}) || too_large({d.batch, d.seqlen, d.dstate}) ||
+      too_large({d.batch, d.dim, d.dstate}))
+    return SSM_ERR_UNSUPPORTED;
   return SSM_OK;
 }
 
@@ -566,6 +582,7 @@ static int conv_check(int64_t batch, int64_t seqlen, int64_t dim, int64_t width,
   if (batch < 0 || seqlen < 0 || dim < 0 || width < 1) return SSM_ERR_INVALID_ARG;
   if (!conv_width_supported((int)std::min<int64_t>(width, 1 << 20))) return SSM_ERR_UNSUPPORTED;
   if (batch > 65535 || dim > (1 << 24) || seqlen > (1 << 30)) return SSM_ERR_UNSUPPORTED;
+  if (too_large({batch, seqlen, dim})) return SSM_ERR_UNSUPPORTED;
   return SSM_OK;
 }
 
@@ -652,6 +669,9 @@ int ssm_ssd_scan_fwd(int64_t batch, int64_t seqlen, int64_t nheads, int64_t head
     return fail(SSM_ERR_UNSUPPORTED, "ssm_ssd_scan_fwd: bf16 io, headdim 64 and dstate 64, "
                                      "128 or 256 only");
   if (batch > 65535 || nheads > (1 << 20) || seqlen > (1 << 30)) return SSM_ERR_UNSUPPORTED;
+  if (too_large({batch, seqlen, nheads, headdim}) || too_large({batch, seqlen, dstate}) ||
+      too_large({batch, nheads, headdim, dstate}))
+    return SSM_ERR_UNSUPPORTED;
   if (batch == 0 || nheads == 0) return SSM_OK;
   if (!A) return SSM_ERR_INVALID_ARG;
   if (seqlen > 0 && (!x || !dt || !B || !C || !y)) return SSM_ERR_INVALID_ARG;
@@ -697,7 +717,7 @@ int ssm_ssd_state_update(int64_t batch, int64_t nheads, int64_t headdim, int64_t
   if (!ssd_decode_dstate_supported((int)std::min<int64_t>(dstate, 1 << 20)))
     return fail(SSM_ERR_UNSUPPORTED, "ssm_ssd_state_update: dstate 32, 64, 128 or 256 only");
   if (batch > (1 << 24) || nheads > (1 << 20) || headdim > (1 << 20) ||
-      batch * nheads * headdim > ((int64_t)1 << 26))
+      too_large({batch, nheads, headdim, (int64_t)1 << 14}))  // at most 2^26 state rows
     return SSM_ERR_UNSUPPORTED;
   if (batch == 0 || nheads == 0 || headdim == 0) return SSM_OK;
   if (!state || !x || !dt || !A || !B || !C || !y) return SSM_ERR_INVALID_ARG;
@@ -795,6 +815,7 @@ int ssm_delta_sum(int64_t batch, int64_t seqlen, int64_t dim, int io_dtype, cons
                   const float* delta_bias, int softplus, float* dsum, void* stream) {
   if (io_dtype != SSM_DTYPE_F32 && io_dtype != SSM_DTYPE_BF16) return SSM_ERR_UNSUPPORTED;
   if (batch < 0 || seqlen < 0 || dim < 0) return SSM_ERR_INVALID_ARG;
+  if (too_large({batch, seqlen, dim})) return SSM_ERR_UNSUPPORTED;
   if (batch == 0 || dim == 0) return SSM_OK;
   if (!dsum || (seqlen > 0 && !delta)) return SSM_ERR_INVALID_ARG;
   const size_t es = io_bytes(io_dtype);
@@ -819,6 +840,7 @@ int ssm_compose_carries(int64_t rank, int64_t batch, int64_t dim, int64_t dstate
                         const float* h0, const float* hend_all, const float* dsum_all,
                         float* h_in, void* stream) {
   if (rank < 0 || batch < 0 || dim < 0 || dstate <= 0) return SSM_ERR_INVALID_ARG;
+  if (too_large({rank + 1, batch, dim, dstate})) return SSM_ERR_UNSUPPORTED;
   if (batch == 0 || dim == 0) return SSM_OK;
   if (!A || !h_in || (rank > 0 && (!hend_all || !dsum_all))) return SSM_ERR_INVALID_ARG;
   const void* f[] = {A, h0, hend_all, dsum_all, h_in};

@@ -226,6 +226,7 @@ def test_sequence_split_helpers_reject_bad_arguments(L):
                                  FAKE + K, None) == 0
 
 
+@no_gpu_only
 def test_ssd_rejects_bad_arguments(L):
     K = 1 << 18  # spacing of the fake buffers: none of them overlap
 
@@ -255,6 +256,7 @@ def test_ssd_rejects_bad_arguments(L):
     assert ssd(nheads=0) == 0
 
 
+@no_gpu_only
 def test_ssd_state_update_rejects_bad_arguments(L):
     K = 1 << 20
 
@@ -298,3 +300,22 @@ def test_product_never_imports_the_oracle():
                 text = open(os.path.join(dirpath, f)).read()
                 assert not re.search(r"^\s*(import|from)\s+oracle\b", text, re.M), f
                 assert "ssm_oracle" not in text and "liboracle" not in text, f
+
+
+@no_gpu_only
+def test_oversized_problems_are_rejected(L):
+    """Element counts past 2^40 are refused on the host (before any byte
+    count could overflow), whatever the pointers."""
+    p = bnd.ScanPlan()
+    assert L.ssm_scan_plan(65535, 1 << 30, 1 << 24, 16, 1, ctypes.byref(p)) == -2
+    assert L.ssm_scan_workspace_bytes(65535, 1 << 30, 1 << 24, 16, 1) == 0
+    assert scan(L, batch=65535, seqlen=1 << 30, dim=1 << 20) == -2
+    assert L.ssm_conv1d_silu_fwd(65535, 1 << 30, 1 << 20, 4, 1, FAKE, FAKE, None, 1, FAKE,
+                                 None) == -2
+    assert L.ssm_ssd_scan_fwd(65535, 1 << 30, 64, 64, 128, 1, FAKE, FAKE, FAKE, FAKE, FAKE,
+                              None, None, 1, None, FAKE, None, None) == -2
+    assert L.ssm_ssd_state_update(1 << 24, 1 << 20, 64, 128, 1, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                  FAKE, None, None, 1, FAKE, None) == -2
+    assert L.ssm_delta_sum(65535, 1 << 30, 1 << 20, 1, FAKE, None, 1, FAKE, None) == -2
+    assert L.ssm_compose_carries(1 << 20, 65535, 1 << 20, 16, FAKE, None, FAKE, FAKE, FAKE,
+                                 None) == -2
