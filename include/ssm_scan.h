@@ -56,7 +56,9 @@ enum {
 enum {
   SSM_OK = 0,
   SSM_ERR_INVALID_ARG = -1, /* null required pointer, bad size, misaligned, aliasing */
-  SSM_ERR_UNSUPPORTED = -2, /* dstate or io_dtype this library does not support     */
+  SSM_ERR_UNSUPPORTED = -2, /* dstate, io_dtype or size this library does not support
+                               (sizes: batch <= 65535, seqlen <= 2^30, dim <= 2^24, and
+                               no tensor above 2^40 elements)                          */
   SSM_ERR_WORKSPACE = -3,   /* workspace missing or smaller than required           */
   SSM_ERR_CUDA = -4,        /* a CUDA runtime call or kernel launch failed          */
   SSM_ERR_TIMEOUT = -5,     /* a bounded wait inside a kernel gave up (ssm_scan_status) */
