@@ -61,6 +61,8 @@ def parse_args():
                          "(default workload " + "ssd_mamba2_b4_l4096_h64_p64_n128)")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", dest="per_config", action="store_false",
+                    help="skip timing the other scan workloads and the decode workload")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU time of the oracle baseline sample")
     return ap.parse_args()
@@ -209,6 +211,228 @@ def cpu_oracle_rate(w, inp, target_s, rng_seed=0, zoh=False):
     return value, threads, f"{n} of {len(all_ch)} channels x {w.seqlen} steps, {dt:.1f} s"
 
 
+# Workloads reported beside the bench workload in `per_config` (one GPU).
+PER_CONFIG_SCANS = ("mamba130m_layer_b8_l2048_d1536", "pythia1b_layer_b4_l4096_d4096_h0",
+                    "long_b1_l262144_d1536")
+PER_CONFIG_DECODE = "decode_b128_d4096_x1000"
+
+
+def time_scan(w, nb, b0, device, K, warmup, zoh=False, learned_a=False, sync=None,
+              sample_clocks=False):
+    """K timed ssm_scan_fwd calls of workload `w` (batch rows b0 .. b0+nb of its
+    global batch) on `device`: inputs resident in HBM, the L2 flushed (256 MB
+    write) before every call, each call between CUDA events on the launching
+    stream. Returns the per-call times and what the caller needs to reuse the
+    call (inputs on the host and device, outputs, the plan, the call)."""
+    import torch
+
+    from selective_state_space_39_b200 import scan_plan, scan_workspace_bytes, ssm_scan_fwd
+
+    inp = gen.workload_inputs(w, batch=nb, batch_offset=b0)
+    if learned_a:
+        inp["A"] = gen.a_matrix_learned(w.dim, w.dstate, w.seed)
+    dtype = torch.bfloat16 if w.io == "bf16" else torch.float32
+
+    def to_dev(a):
+        if a is None:
+            return None
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+    d = {k: to_dev(v) for k, v in inp.items()}
+    y = torch.empty((nb, w.seqlen, w.dim), dtype=dtype, device=device)
+    h_last = torch.empty((nb, w.dim, w.dstate), dtype=torch.float32, device=device)
+    ws = torch.empty(max(1, scan_workspace_bytes(nb, w.seqlen, w.dim, w.dstate, dtype)),
+                     dtype=torch.uint8, device=device)
+    plan = scan_plan(nb, w.seqlen, w.dim, w.dstate, dtype)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    def step():
+        ssm_scan_fwd(d["x"], d["delta"], d["A"], d["B"], d["C"], D=d["D"], z=d["z"],
+                     delta_bias=d["delta_bias"], h0=d["h0"], y=y, h_last=h_last, workspace=ws,
+                     zoh=zoh)
+
+    for _ in range(max(3, warmup)):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    sampler = ClockSampler(device.index) if sample_clocks else None
+    if sync:
+        sync()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.__enter__()
+    for i in range(K):
+        flush.fill_(i & 0xFF)
+        starts[i].record()
+        step()
+        ends[i].record()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.__exit__(None, None, None)
+    if sync:
+        sync()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    return {"step_ms": step_ms, "plan": plan, "inp": inp, "d": d, "y": y, "h_last": h_last,
+            "step": step, "clocks": sampler.summary() if sampler else None}
+
+
+def scan_rooflines(w, nb, mean_s, clocks, zoh, plan, traffic):
+    """The call's HBM roofline (the workload metric: algorithmic bytes of the
+    call over its mean time, against the measured copy bandwidth) and its FP32
+    ALU figure (4N operations per element against 148 SMs x 128 lanes at the
+    sampled SM clock)."""
+    kernel = "%s: carry pass + main pass (%d launches)" % (
+        "ssm_scan_fwd_zoh" if zoh else "ssm_scan_fwd", plan.kernels)
+    peak, peak_kind = measured_hbm_peak()
+    algo = algorithmic_bytes(w, nb)
+    achieved = algo / mean_s / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": traffic, "kernel": kernel,
+                "algorithmic_bytes_per_launch": algo, "peak_kind": peak_kind}
+    sm_mhz = (clocks or {}).get("sm_mhz") or B200_MAX_SM_MHZ
+    alu_peak = B200_SMS * FP32_LANES_PER_SM * sm_mhz * 1e6 / 1e9  # Gop/s
+    alu = alu_ops_per_element(w, zoh) * nb * w.seqlen * w.dim / mean_s / 1e9
+    alu_roofline = {"bound": "alu", "achieved": round(alu, 1), "peak": round(alu_peak, 1),
+                    "unit": "Gop/s", "frac": round(alu / alu_peak, 4),
+                    "ops_per_element": alu_ops_per_element(w, zoh),
+                    "peak_kind": f"derived: {B200_SMS} SMs x {FP32_LANES_PER_SM} FP32 lanes x "
+                                 f"{sm_mhz:.0f} MHz sampled SM clock"}
+    return roofline, alu_roofline
+
+
+def scan_summary(w, run, traffic):
+    """One `per_config` entry for a scan workload."""
+    mean_s = statistics.mean(run["step_ms"]) * 1e-3
+    roof, alu = scan_rooflines(w, w.batch, mean_s, run["clocks"], False, run["plan"], traffic)
+    return {"metric": METRIC, "value": w.batch * w.seqlen * w.dim / mean_s,
+            "unit": "elements/s", "ms_per_step": mean_s * 1e3, "steps": len(run["step_ms"]),
+            "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "dim": w.dim,
+                       "dstate": w.dstate, "io": w.io, "h0": w.with_h0,
+                       "segments": run["plan"].segments,
+                       "l2": "flushed (256 MB write) before every timed step"},
+            "roofline": roof, "alu_roofline": alu, "clocks": run["clocks"]}
+
+
+def time_decode(w, device, K, warmup):
+    """ssm_state_update calls of decode workload `w` on a resident fp32 state
+    (one step = one call over all batch rows and channels), timed four ways:
+    L2 flushed by a 256 MB write before every call, flushed by a 256 MB read,
+    back to back, and the workload's whole run of w.steps calls captured in
+    one CUDA graph. Returns the per-call times in ms and the clock record."""
+    import torch
+
+    from selective_state_space_39_b200 import ssm_state_update
+    dtype = torch.bfloat16 if w.io == "bf16" else torch.float32
+    const = gen.decode_constants(w.dim, w.dstate, w.seed)
+
+    def to_dev(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16).copy()).view(torch.bfloat16).to(device)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+    steps_in = [{k: to_dev(v) for k, v in gen.make_decode_inputs(
+        w.batch, w.dim, w.dstate, w.io, w.seed, i).items()} for i in range(8)]
+    A, D, bias = (to_dev(const[k]) for k in ("A", "D", "delta_bias"))
+    state = torch.zeros((w.batch, w.dim, w.dstate), dtype=torch.float32, device=device)
+    y = torch.empty((w.batch, w.dim), dtype=dtype, device=device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    def call(i):
+        s = steps_in[i % len(steps_in)]
+        ssm_state_update(state, s["x"], s["delta"], A, s["B"], s["C"], D=D, z=s["z"],
+                         delta_bias=bias, y=y)
+
+    for i in range(max(3, warmup)):
+        call(i)
+    torch.cuda.synchronize()
+
+    def timed(prep):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(K)]
+        for i in range(K):
+            prep(i)
+            ev[i][0].record()
+            call(i)
+            ev[i][1].record()
+        torch.cuda.synchronize()
+        return statistics.mean(a.elapsed_time(b) for a, b in ev)
+
+    # (1) write-flushed: the call also pays for writing back the flush's dirty
+    #     lines; (2) read-flushed (clean lines): the call's own DRAM traffic;
+    #     (3) back to back: the 33.5 MB state stays in L2, as across
+    #     consecutive decode steps; (4) one CUDA graph of w.steps calls.
+    sampler = ClockSampler(device.index)
+    with sampler:
+        cold_ms = timed(lambda i: flush.fill_(i & 0xFF))
+    read_ms = timed(lambda i: flush.view(torch.int64).sum())
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(K):
+        call(i)
+    e1.record()
+    torch.cuda.synchronize()
+    warm_ms = e0.elapsed_time(e1) / K
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        call(0)  # first call outside capture (library state, attributes)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g):
+        for i in range(w.steps):
+            call(i)
+    g.replay()  # warm the graph
+    torch.cuda.synchronize()
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g0.record()
+    g.replay()
+    g1.record()
+    torch.cuda.synchronize()
+    graph_ms = g0.elapsed_time(g1) / w.steps
+    del g
+    return {"w": w, "K": K, "cold_ms": cold_ms, "read_ms": read_ms, "warm_ms": warm_ms,
+            "graph_ms": graph_ms, "clocks": sampler.summary()}
+
+
+def decode_algorithmic_bytes(w):
+    es = 2 if w.io == "bf16" else 4
+    nbd = w.batch * w.dim
+    return (nbd * w.dstate * 4 * 2 + nbd * es * 4 + 2 * w.batch * w.dstate * es +
+            w.dim * w.dstate * 4 + 2 * w.dim * 4)
+
+
+def decode_summary(r):
+    """The decode step's figures: the read-flushed call is the headline (the
+    call's own DRAM traffic); the others beside it."""
+    w = r["w"]
+    nbd = w.batch * w.dim
+    algo = decode_algorithmic_bytes(w)
+    peak, peak_kind = measured_hbm_peak()
+
+    def fig(ms):
+        gbs = algo / (ms * 1e-3) / 1e9
+        return {"ms_per_step": ms, "value": nbd / (ms * 1e-3), "algorithmic_gbs": round(gbs, 1),
+                "frac": round(gbs / peak, 4)}
+
+    read_gbs = algo / (r["read_ms"] * 1e-3) / 1e9
+    return {"metric": "decode state-update elements/s (B·D per step) and HBM GB/s",
+            "value": nbd / (r["read_ms"] * 1e-3), "unit": "elements/s",
+            "ms_per_step": r["read_ms"], "steps": r["K"],
+            "config": {"workload": w.name, "batch": w.batch, "dim": w.dim, "dstate": w.dstate,
+                       "io": w.io, "l2": "flushed (256 MB read) before every timed call"},
+            "roofline": {"bound": "hbm", "achieved": round(read_gbs, 1), "peak": peak,
+                         "unit": "GB/s", "frac": round(read_gbs / peak, 4),
+                         "algorithmic_bytes_per_launch": algo, "peak_kind": peak_kind},
+            "write_flushed_l2": fig(r["cold_ms"]), "warm_l2": fig(r["warm_ms"]),
+            "cuda_graph": dict(fig(r["graph_ms"]), calls=w.steps), "clocks": r["clocks"]}
+
+
+
 def reference_arm(args):
     """--impl reference: the fp64 oracle on the host cores, rank 0 only."""
     rank = int(os.environ.get("RANK", 0))
@@ -251,110 +475,22 @@ def reference_arm(args):
 
 def decode_bench(args):
     """--workload decode_*: ssm_state_update calls on a resident fp32 state
-    (one step = one call over all batch rows and channels). Timed twice: L2
-    flushed before every call, and back to back (the state fits in L2)."""
+    (one step = one call over all batch rows and channels), timed with the L2
+    flushed before every call (write and read flush), back to back (the state
+    fits in L2) and in one CUDA graph."""
     import torch
-
-    from selective_state_space_39_b200 import ssm_state_update
     w = gen.DECODE_WORKLOADS[args.workload]
-    device = torch.device("cuda", 0)
-    dtype = torch.bfloat16 if w.io == "bf16" else torch.float32
-    const = gen.decode_constants(w.dim, w.dstate, w.seed)
-
-    def to_dev(a):
-        if a.dtype == np.uint16:
-            return torch.from_numpy(a.view(np.int16).copy()).view(torch.bfloat16).to(device)
-        return torch.from_numpy(np.ascontiguousarray(a)).to(device)
-
-    steps_in = [{k: to_dev(v) for k, v in gen.make_decode_inputs(
-        w.batch, w.dim, w.dstate, w.io, w.seed, i).items()} for i in range(8)]
-    A, D, bias = (to_dev(const[k]) for k in ("A", "D", "delta_bias"))
-    state = torch.zeros((w.batch, w.dim, w.dstate), dtype=torch.float32, device=device)
-    y = torch.empty((w.batch, w.dim), dtype=dtype, device=device)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
-
-    def call(i):
-        s = steps_in[i % len(steps_in)]
-        ssm_state_update(state, s["x"], s["delta"], A, s["B"], s["C"], D=D, z=s["z"],
-                         delta_bias=bias, y=y)
-
-    for i in range(max(3, args.warmup)):
-        call(i)
-    torch.cuda.synchronize()
-    K = args.steps
-
-    def timed(prep):
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(K)]
-        for i in range(K):
-            prep(i)
-            ev[i][0].record()
-            call(i)
-            ev[i][1].record()
-        torch.cuda.synchronize()
-        return statistics.mean(a.elapsed_time(b) for a, b in ev)
-
-    # (1) L2 flushed by writing 256 MB: the call also pays for writing back
-    #     the flush's dirty lines; (2) flushed by reading 256 MB (clean
-    #     lines): the call's own DRAM traffic; (3) back to back: the 33.5 MB
-    #     state stays in L2, as across consecutive decode steps.
-    sampler = ClockSampler(0)
-    with sampler:
-        cold_ms = timed(lambda i: flush.fill_(i & 0xFF))
-    read_ms = timed(lambda i: flush.view(torch.int64).sum())
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for i in range(K):
-        call(i)
-    e1.record()
-    torch.cuda.synchronize()
-    warm_ms = e0.elapsed_time(e1) / K
-    # (4) the workload's whole decode run (w.steps consecutive calls) captured
-    #     in one CUDA graph and replayed: no per-call launch overhead.
-    g = torch.cuda.CUDAGraph()
-    side = torch.cuda.Stream()
-    side.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(side):
-        call(0)  # first call outside capture (library state, attributes)
-    torch.cuda.current_stream().wait_stream(side)
-    torch.cuda.synchronize()
-    with torch.cuda.graph(g):
-        for i in range(w.steps):
-            call(i)
-    g.replay()  # warm the graph
-    torch.cuda.synchronize()
-    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    g0.record()
-    g.replay()
-    g1.record()
-    torch.cuda.synchronize()
-    graph_ms = g0.elapsed_time(g1) / w.steps
-    del g
-    es = 2 if w.io == "bf16" else 4
-    nbd = w.batch * w.dim
-    algo = nbd * w.dstate * 4 * 2 + nbd * es * 4 + 2 * w.batch * w.dstate * es + \
-        w.dim * w.dstate * 4 + 2 * w.dim * 4
-    peak, peak_kind = measured_hbm_peak()
-    gbs = algo / (cold_ms * 1e-3) / 1e9
+    r = time_decode(w, torch.device("cuda", 0), args.steps, args.warmup)
+    s = decode_summary(r)
     line = {
-        "metric": "decode state-update elements/s (B·D per step) and HBM GB/s",
-        "value": nbd / (cold_ms * 1e-3), "unit": "elements/s", "n_gpus": 1, "steps": K,
-        "warmup": args.warmup, "ms_per_step": cold_ms, "higher_is_better": True,
-        "dtype": w.io, "data": "synthetic (seeded Philox4x32-10, Mamba-shaped recipe)",
-        "config": {"workload": w.name, "batch": w.batch, "dim": w.dim, "dstate": w.dstate,
-                   "l2": "flushed (256 MB write) before every timed call"},
-        "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(gbs / peak, 4), "algorithmic_bytes_per_launch": algo,
-                     "peak_kind": peak_kind},
-        "read_flushed_l2": {"ms_per_step": read_ms, "value": nbd / (read_ms * 1e-3),
-                            "algorithmic_gbs": round(algo / (read_ms * 1e-3) / 1e9, 1),
-                            "frac": round(algo / (read_ms * 1e-3) / 1e9 / peak, 4)},
-        "warm_l2": {"ms_per_step": warm_ms, "value": nbd / (warm_ms * 1e-3),
-                    "algorithmic_gbs": round(algo / (warm_ms * 1e-3) / 1e9, 1)},
-        "cuda_graph": {"calls": w.steps, "ms_per_step": graph_ms,
-                       "value": nbd / (graph_ms * 1e-3),
-                       "algorithmic_gbs": round(algo / (graph_ms * 1e-3) / 1e9, 1)},
-        "gpu_launches": 2 * K, "clocks": sampler.summary(),
+        "metric": s["metric"], "value": s["value"], "unit": "elements/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": s["ms_per_step"],
+        "higher_is_better": True, "dtype": w.io,
+        "data": "synthetic (seeded Philox4x32-10, Mamba-shaped recipe)",
+        "config": s["config"], "roofline": s["roofline"],
+        "write_flushed_l2": s["write_flushed_l2"], "warm_l2": s["warm_l2"],
+        "cuda_graph": s["cuda_graph"], "gpu_launches": 3 * args.steps + w.steps,
+        "clocks": s["clocks"],
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -937,7 +1073,6 @@ def main():
     import torch
 
     from selective_state_space_39_b200 import dist as sdist
-    from selective_state_space_39_b200 import scan_plan, scan_workspace_bytes, ssm_scan_fwd
 
     rank, local_rank, world = sdist.env_world()
     if not torch.cuda.is_available():
@@ -949,79 +1084,23 @@ def main():
     w = gen.SCAN_WORKLOADS[args.workload]
     # weak scaling: global batch = world * w.batch; this rank's shard
     b0, nb = sdist.batch_shard(world * w.batch, world, rank)
-    inp = gen.workload_inputs(w, batch=nb, batch_offset=b0)
-    if args.learned_a:
-        inp["A"] = gen.a_matrix_learned(w.dim, w.dstate, w.seed)
-    dtype = torch.bfloat16 if w.io == "bf16" else torch.float32
-
-    def to_dev(a):
-        if a is None:
-            return None
-        if a.dtype == np.uint16:
-            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
-        return torch.from_numpy(np.ascontiguousarray(a)).to(device)
-
-    d = {k: to_dev(v) for k, v in inp.items()}
-    y = torch.empty((nb, w.seqlen, w.dim), dtype=dtype, device=device)
-    h_last = torch.empty((nb, w.dim, w.dstate), dtype=torch.float32, device=device)
-    ws = torch.empty(max(1, scan_workspace_bytes(nb, w.seqlen, w.dim, w.dstate, dtype)),
-                     dtype=torch.uint8, device=device)
-    plan = scan_plan(nb, w.seqlen, w.dim, w.dstate, dtype)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
-
-    def step():
-        ssm_scan_fwd(d["x"], d["delta"], d["A"], d["B"], d["C"], D=d["D"], z=d["z"],
-                     delta_bias=d["delta_bias"], h0=d["h0"], y=y, h_last=h_last, workspace=ws,
-                     zoh=args.zoh)
-
-    for _ in range(max(3, args.warmup)):
-        flush.fill_(1)
-        step()
-    torch.cuda.synchronize()
-
+    run = time_scan(w, nb, b0, device, args.steps, args.warmup, zoh=args.zoh,
+                    learned_a=args.learned_a, sync=lambda: sdist.barrier(device),
+                    sample_clocks=True)
+    step_ms, plan, inp, d, y, h_last, step = (run[k] for k in (
+        "step_ms", "plan", "inp", "d", "y", "h_last", "step"))
+    dtype = y.dtype
     K = args.steps
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    sampler = ClockSampler(device.index)
-    sdist.barrier(device)
-    torch.cuda.synchronize()
-    with sampler:
-        for i in range(K):
-            flush.fill_(i & 0xFF)
-            starts[i].record()
-            step()
-            ends[i].record()
-        torch.cuda.synchronize()
-    sdist.barrier(device)
-    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     local_ms = sum(step_ms)
     total_ms = sdist.max_over_ranks(local_ms, device)
     ms_per_step = total_ms / K
     elements = world * w.batch * w.seqlen * w.dim
     value = elements * K / (total_ms * 1e-3)
-
-    # Rooflines of the call (carry pass + main pass). The binding one is the
-    # FP32 ALU: the path does ~4N FP32 operations per 8 bytes moved.
-    clocks = sampler.summary()
-    sm_mhz = clocks.get("sm_mhz") or B200_MAX_SM_MHZ
-    alu_peak = B200_SMS * FP32_LANES_PER_SM * sm_mhz * 1e6 / 1e9  # Gop/s
+    clocks = run["clocks"]
     mean_s = statistics.mean(step_ms) * 1e-3
-    alu_achieved = alu_ops_per_element(w, args.zoh) * nb * w.seqlen * w.dim / mean_s / 1e9
-    traffic = (measured_traffic(w.name)
-               if (world == 1 or nb == w.batch) and not args.zoh and not args.learned_a else None)
-    kernel = "%s: carry pass + main pass (%d launches)" % (
-        "ssm_scan_fwd_zoh" if args.zoh else "ssm_scan_fwd", plan.kernels)
-    roofline = {"bound": "alu", "achieved": round(alu_achieved, 1), "peak": round(alu_peak, 1),
-                "unit": "Gop/s", "frac": round(alu_achieved / alu_peak, 4), "traffic": traffic,
-                "kernel": kernel, "ops_per_element": alu_ops_per_element(w, args.zoh),
-                "peak_kind": f"derived: {B200_SMS} SMs x {FP32_LANES_PER_SM} FP32 lanes x "
-                             f"{sm_mhz:.0f} MHz sampled SM clock"}
-    peak, peak_kind = measured_hbm_peak()
-    algo = algorithmic_bytes(w, nb)
-    achieved = algo / mean_s / 1e9
-    hbm_roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                    "frac": round(achieved / peak, 4), "traffic": traffic, "kernel": kernel,
-                    "algorithmic_bytes_per_launch": algo, "peak_kind": peak_kind}
+    use_traffic = (world == 1 or nb == w.batch) and not args.zoh and not args.learned_a
+    roofline, alu_roofline = scan_rooflines(w, nb, mean_s, clocks, args.zoh, plan,
+                                            measured_traffic(w.name) if use_traffic else None)
 
     # end to end through the public call: pinned host inputs -> device -> scan -> host
     e2e = None
@@ -1050,12 +1129,32 @@ def main():
         e2e_ms = sdist.max_over_ranks(statistics.mean(e_ms), device)
         e2e = {"value": elements / (e2e_ms * 1e-3), "unit": "elements/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+    del run, d, y, h_last, step
 
     cpu = None
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         v, cores, sample = cpu_oracle_rate(w, inp, args.cpu_seconds, zoh=args.zoh)
         cpu = {"value": v, "unit": "elements/s", "cores": cores, "kind": "oracle",
                "sample": sample}
+    del inp
+
+    # The other workloads of the scan (and the decode workload), timed the same
+    # way in this run on one GPU; they are reported, not part of `value`.
+    per_config = None
+    if world == 1 and not args.zoh and not args.learned_a and args.per_config:
+        per_config = {}
+        for name in PER_CONFIG_SCANS:
+            if name == w.name:
+                continue
+            wc = gen.SCAN_WORKLOADS[name]
+            rc = time_scan(wc, wc.batch, 0, device, args.steps, args.warmup,
+                           sample_clocks=True)
+            per_config[name] = scan_summary(wc, rc, measured_traffic(wc.name))
+            del rc
+            torch.cuda.empty_cache()
+        per_config[PER_CONFIG_DECODE] = decode_summary(
+            time_decode(gen.DECODE_WORKLOADS[PER_CONFIG_DECODE], device, args.steps,
+                        args.warmup))
 
     if rank == 0:
         line = {
@@ -1072,10 +1171,12 @@ def main():
                        "A": "learned-like (unstructured)" if args.learned_a else "(n+1) A[d,0]",
                        "l2": "flushed (256 MB write) before every timed step",
                        "parallelism": f"dp{world} (batch shards, no data-path collective)"},
-            "hbm_gbs": round(achieved, 1), "hbm_frac_of_peak": round(achieved / peak, 4),
-            "roofline": roofline, "hbm_roofline": hbm_roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": K * plan.kernels, "clocks": clocks,
+            "hbm_gbs": roofline["achieved"], "hbm_frac_of_peak": roofline["frac"],
+            "roofline": roofline, "alu_roofline": alu_roofline, "cpu_baseline": cpu,
+            "e2e": e2e, "gpu_launches": K * plan.kernels, "clocks": clocks,
         }
+        if per_config is not None:
+            line["per_config"] = per_config
         print(json.dumps(line), flush=True)
     sdist.finish()
     return 0

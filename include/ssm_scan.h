@@ -19,7 +19,11 @@
  * Conventions for every entry point:
  *   - All tensor pointers are DEVICE pointers owned by the caller, dense and
  *     row-major (C order) in the layouts given below. The library never
- *     allocates, frees or synchronises, and keeps no mutable global state.
+ *     allocates, frees or synchronises. Apart from small caches of its own
+ *     (kernel attributes set once, driver entry points), its one piece of
+ *     mutable global state is the fixed scratch array of the no-alloc entry
+ *     (ssm_scan_fwd_noalloc below), shared by every call of that entry on a
+ *     device; all other entry points keep their state in caller memory.
  *   - io_dtype selects the storage type of x, delta, z, B, C and y:
  *     SSM_DTYPE_F32 (IEEE binary32) or SSM_DTYPE_BF16 (bfloat16). A, D,
  *     delta_bias, h0, h_last and the decode state are always fp32.
@@ -70,9 +74,11 @@ enum {
 /*
  * How ssm_scan_fwd splits a problem (see ssm_scan_plan). The sequence is cut
  * into `segments` of `segment_steps` steps; with more than one segment a
- * carry pass computes each segment's end state and the main pass composes
- * them (the recurrence of §2.2 is an associative composition of affine
- * maps h -> a*h + b, which the pages' parallel associative scan relies on).
+ * carry pass computes each segment's end state, a small kernel (with three or
+ * more segments) composes them into every segment's start state, and the
+ * main pass runs each segment from its start (the recurrence of §2.2 is an
+ * associative composition of affine maps h -> a*h + b, which the pages'
+ * parallel associative scan relies on).
  */
 typedef struct {
   int32_t segments;
@@ -154,9 +160,9 @@ int ssm_scan_fwd_zoh(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
  * a host framework). Same arguments, layouts and results as ssm_scan_fwd,
  * without the workspace.
  *
- * Scratch: a fixed 8 MiB array reserved in device memory by the library on
+ * Scratch: a fixed 16 MiB array reserved in device memory by the library on
  * every GPU that loads it, kept until the process exits. Problems whose
- * ssm_scan_workspace_bytes(...) exceeds 8 MiB are rejected with
+ * ssm_scan_workspace_bytes(...) exceeds 16 MiB are rejected with
  * SSM_ERR_WORKSPACE (ssm_last_error_detail says how much they need); use
  * ssm_scan_fwd for those.
  *   - The first call on each device looks up the scratch's device address
@@ -167,6 +173,12 @@ int ssm_scan_fwd_zoh(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
  *     writes every scratch word it reads). Calls that can run at the same
  *     time on the GPU (different streams or host threads, without ordering
  *     between them) race on the scratch and must be serialised by the caller.
+ *   - The scratch's address is cached per device together with the context
+ *     it was looked up in; after cudaDeviceReset the next call (made before
+ *     any stream capture, as above) looks it up again.
+ *   - A bounded wait inside the kernels that times out records it in the
+ *     scratch; ssm_scan_status_noalloc (below) reads it, as ssm_scan_status
+ *     does for ssm_scan_fwd.
  *   - Allocates and frees nothing. Returns SSM_OK or SSM_ERR_*.
  */
 int ssm_scan_fwd_noalloc(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
@@ -174,6 +186,19 @@ int ssm_scan_fwd_noalloc(int64_t batch, int64_t seqlen, int64_t dim, int64_t dst
                          const void* B, const void* C, const float* D, const void* z,
                          const float* delta_bias, int softplus, const float* h0, void* y,
                          float* h_last, void* stream);
+
+/*
+ * ssm_scan_status_noalloc -- ssm_scan_status for the no-alloc entry (no
+ * counterpart on the pages either): synchronise `stream`, then report from
+ * the reserved scratch whether every CTA of the last ssm_scan_fwd_noalloc
+ * call on this device with these sizes finished normally: SSM_OK, or
+ * SSM_ERR_TIMEOUT if a bounded wait gave up (y and h_last are then
+ * incomplete). The status words belong to the last no-alloc call on the
+ * device, whatever its sizes; pass the sizes of that call. Returns
+ * SSM_ERR_WORKSPACE for sizes the scratch cannot hold, like the entry itself.
+ */
+int ssm_scan_status_noalloc(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
+                            int io_dtype, void* stream);
 
 /*
  * ssm_state_update -- one decode step: the recurrent, O(1)-per-token form of
@@ -339,7 +364,10 @@ int ssm_compose_carries(int64_t rank, int64_t batch, int64_t dim, int64_t dstate
  *   y[b,t,h,p]   = sum_n C[b,t,n] * S[p][n] + D[h] * x[b,t,h,p]
  *
  * starting from h0[b,h] (or zero) and ending in h_last[b,h]. Computed chunk
- * by chunk on the tensor cores (bf16 operands, fp32 accumulation and state).
+ * by chunk on the tensor cores (bf16 operands, fp32 accumulation and state):
+ * with dstate 64 or 128, an even nheads and 16-byte aligned h0 / h_last on
+ * the fifth-generation (tcgen05) path, the state held in tensor memory;
+ * otherwise (or with SSM_SSD_LEGACY=1) on the warp-level MMA path.
  *   x, y     : (batch, seqlen, nheads, headdim) bf16 (io_dtype must be
  *              SSM_DTYPE_BF16); y must not overlap an input
  *   dt       : (batch, seqlen, nheads) bf16
@@ -355,6 +383,17 @@ int ssm_ssd_scan_fwd(int64_t batch, int64_t seqlen, int64_t nheads, int64_t head
                      int64_t dstate, int io_dtype, const void* x, const void* dt, const float* A,
                      const void* B, const void* C, const float* D, const float* dt_bias,
                      int softplus, const float* h0, void* y, float* h_last, void* stream);
+
+/*
+ * ssm_ssd_scan_status -- synchronise `stream`, then report whether a CTA of
+ * an ssm_ssd_scan_fwd call on the current device gave up a bounded wait
+ * (2 s, or SSM_SCAN_WAIT_LIMIT_NS nanoseconds) since the last call of this
+ * function: SSM_OK, or SSM_ERR_TIMEOUT (that call's y and h_last are then
+ * incomplete). The flag is per device and cleared by this call. For testing
+ * this path, SSM_SSD_TEST_STALL=1 makes the first CTA wait for data that
+ * never arrives.
+ */
+int ssm_ssd_scan_status(void* stream);
 
 /*
  * ssm_ssd_state_update -- one decode step of the multi-head SSD (same page,

@@ -77,6 +77,8 @@ def lib() -> ctypes.CDLL:
         L.ssm_scan_status.restype = ctypes.c_int
         L.ssm_scan_status.argtypes = [_VP, ctypes.c_size_t, _I64, _I64, _I64, _I64, ctypes.c_int,
                                       _VP]
+        L.ssm_scan_status_noalloc.restype = ctypes.c_int
+        L.ssm_scan_status_noalloc.argtypes = [_I64, _I64, _I64, _I64, ctypes.c_int, _VP]
         L.ssm_scan_bwd_workspace_bytes.restype = ctypes.c_size_t
         L.ssm_scan_bwd_workspace_bytes.argtypes = [_I64, _I64, _I64, _I64, ctypes.c_int]
         L.ssm_scan_bwd.restype = ctypes.c_int
@@ -107,6 +109,8 @@ def lib() -> ctypes.CDLL:
         L.ssm_ssd_state_update.restype = ctypes.c_int
         L.ssm_ssd_state_update.argtypes = [_I64] * 4 + [ctypes.c_int] + [_VP] * 8 + \
             [ctypes.c_int, _VP, _VP]
+        L.ssm_ssd_scan_status.restype = ctypes.c_int
+        L.ssm_ssd_scan_status.argtypes = [_VP]
         L.ssm_ssd_scan_fwd.restype = ctypes.c_int
         L.ssm_ssd_scan_fwd.argtypes = [_I64] * 5 + [ctypes.c_int] + [_VP] * 7 + \
             [ctypes.c_int, _VP, _VP, _VP, _VP]
@@ -394,7 +398,7 @@ def ssm_scan_fwd_noalloc(x, delta, A, B, C, D=None, z=None, delta_bias=None, sof
     """The selective scan through ssm_scan_fwd_noalloc of libssmscan.so.
 
     For callers that cannot allocate device memory around the call: the
-    library takes its scratch from an 8 MiB array it reserves on each GPU, so
+    library takes its scratch from a 16 MiB array it reserves on each GPU, so
     apart from the outputs (allocated here only when not passed in) nothing
     is allocated. Problems needing more scratch raise SsmError (-3). Calls
     that may overlap on the GPU share that scratch and must be ordered by the
@@ -442,6 +446,26 @@ def ssm_scan_status(workspace, batch, seqlen, dim, dstate, dtype=torch.bfloat16,
                                          _stream_ptr(stream, dev)))
 
 
+def ssm_scan_status_noalloc(batch, seqlen, dim, dstate, dtype=torch.bfloat16, device=None,
+                            stream=None):
+    """Synchronise the stream and return the status code of the last
+    ssm_scan_fwd_noalloc call on the device (0 = every CTA finished; -5 = a
+    bounded wait timed out), read from the library's reserved scratch."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    with torch.cuda.device(dev):
+        return int(lib().ssm_scan_status_noalloc(batch, seqlen, dim, dstate, _io_code(dtype),
+                                                 _stream_ptr(stream, dev)))
+
+
+def ssm_ssd_scan_status(device=None, stream=None):
+    """Synchronise the stream and return 0, or -5 if a CTA of an SSD scan on
+    the device gave up a bounded wait since the last call (the flag is then
+    cleared)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    with torch.cuda.device(dev):
+        return int(lib().ssm_ssd_scan_status(_stream_ptr(stream, dev)))
+
+
 def ssm_state_update(state, x, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
                      y=None, stream=None, zoh=False):
     """One decode step through ssm_state_update of libssmscan.so
@@ -475,12 +499,12 @@ def ssm_state_update(state, x, delta, A, B, C, D=None, z=None, delta_bias=None, 
 
 
 def ssm_ssd_scan_fwd(x, dt, A, B, C, D=None, dt_bias=None, softplus=True, h0=None,
-                     return_last_state=False, y=None, stream=None):
+                     return_last_state=False, y=None, stream=None, h_last=None):
     """The multi-head SSD scan through ssm_ssd_scan_fwd of libssmscan.so:
     x (batch, L, heads, headdim) bf16, dt (batch, L, heads) bf16, A (heads,)
     fp32, B, C (batch, L, dstate) bf16, D and dt_bias (heads,) fp32 or None,
     h0 (batch, heads, headdim, dstate) fp32 or None. Returns y (and h_last
-    with ``return_last_state``)."""
+    with ``return_last_state``; ``h_last`` may be given, and may be h0)."""
     if x.dim() != 4:
         raise ValueError("x must be (batch, seqlen, heads, headdim)")
     batch, L, H, P = x.shape
@@ -498,9 +522,9 @@ def ssm_ssd_scan_fwd(x, dt, A, B, C, D=None, dt_bias=None, softplus=True, h0=Non
     if y is None:
         y = torch.empty((batch, L, H, P), dtype=x.dtype, device=dev)
     py = _ptr(y, "y", x.dtype, (batch, L, H, P), dev)
-    h_last = (torch.empty((batch, H, P, N), dtype=torch.float32, device=dev)
-              if return_last_state else None)
-    ph = _ptr(h_last, "h_last")
+    if h_last is None and return_last_state:
+        h_last = torch.empty((batch, H, P, N), dtype=torch.float32, device=dev)
+    ph = _ptr(h_last, "h_last", torch.float32, (batch, H, P, N), dev)
     with torch.cuda.device(dev):
         rc = lib().ssm_ssd_scan_fwd(batch, L, H, P, N, io, px, pdt, pA, pB, pC, pD, pbias,
                                     1 if softplus else 0, ph0, py, ph, _stream_ptr(stream, dev))

@@ -10,11 +10,11 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 SOURCES = [os.path.join(CSRC, f) for f in ("ssm_scan_kernels.cu", "ssm_scan_bwd.cu",
                                            "ssm_conv1d.cu", "ssm_seqpar.cu", "ssm_ssd.cu",
-                                           "ssm_ssd_decode.cu",
+                                           "ssm_ssd_tc.cu", "ssm_ssd_decode.cu",
                                            "ssm_api.cu")]
 HEADERS = [os.path.join(CSRC, f) for f in ("ssm_device.cuh", "ssm_internal.h",
                                             "ssm_bwd_internal.h", "ssm_conv_internal.h",
-                                            "ssm_seqpar_internal.h", "ssm_ssd_internal.h",
+                                            "ssm_seqpar_internal.h", "ssm_ssd_internal.h", "ssm_tc.cuh",
                                             "ssm_ssd_decode_internal.h")] + [
     os.path.join(os.path.dirname(HERE), "include", "ssm_scan.h")]
 LIB_PATH = os.path.join(HERE, "libssmscan.so")

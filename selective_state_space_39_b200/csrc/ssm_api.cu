@@ -218,6 +218,23 @@ bool encode_3d(CUtensorMap* map, const void* base, int io, int64_t batch, int64_
   return r == CUDA_SUCCESS;
 }
 
+// Tiled map of a bf16 tensor with the 128-byte swizzle (rank dims, innermost
+// first; strides in bytes of dims 1..rank-1); box rows of 64 elements.
+bool encode_sw128_bf16(CUtensorMap* map, const void* base, int rank, const cuuint64_t* gdim,
+                       const cuuint64_t* gstride, const cuuint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint32_t estride[5] = {1, 1, 1, 1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank,
+                        const_cast<void*>(base), gdim, gstride, box, estride,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    snprintf(g_detail, sizeof g_detail, "cuTensorMapEncodeTiled (128-byte swizzle) failed: %d",
+             (int)r);
+  return r == CUDA_SUCCESS;
+}
+
 // TMA needs 16-byte aligned bases and 16-byte multiples for row strides.
 bool tma_eligible(const Dims& d, const void* x, const void* delta, const void* z, const void* B,
                   const void* C) {
@@ -280,7 +297,7 @@ int ssm_scan_plan(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate, in
   out->channels_per_cta = pl.dtile;
   out->ctas_carry = pl.ctas_agg;
   out->ctas_main = pl.ctas_main;
-  out->kernels = (batch > 0 && dim > 0) ? (pl.nseg > 1 ? 2 : 1) : 0;
+  out->kernels = (batch > 0 && dim > 0) ? (pl.nseg > 2 ? 3 : pl.nseg > 1 ? 2 : 1) : 0;
   out->workspace_bytes = (int64_t)pl.bytes;
   return SSM_OK;
 }
@@ -705,7 +722,40 @@ int ssm_ssd_scan_fwd(int64_t batch, int64_t seqlen, int64_t nheads, int64_t head
   p.h0 = h0;
   p.y = static_cast<uint16_t*>(y);
   p.h_last = h_last;
+  p.wait_limit_ns = (uint64_t)std::max(1L, env_long("SSM_SCAN_WAIT_LIMIT_NS",
+                                                    (long)kDefaultWaitLimitNs));
+  p.test_stall = env_long("SSM_SSD_TEST_STALL", 0) != 0 ? 1 : 0;
+  // The tcgen05 kernel: dstate 64 or 128, an even head count, 16-byte aligned
+  // state buffers; SSM_SSD_LEGACY=1 keeps the mma.sync kernel.
+  const bool tc = seqlen > 0 && ssd_tc_supported((int)dstate, (int)nheads) &&
+                  env_long("SSM_SSD_LEGACY", 0) == 0 && (!h0 || aligned(h0, 16)) &&
+                  (!h_last || aligned(h_last, 16)) && encode_fn() != nullptr;
+  if (tc) {
+    SsdTcMaps maps;
+    memset(&maps, 0, sizeof maps);
+    const cuuint64_t xd[4] = {(cuuint64_t)headdim, (cuuint64_t)nheads, (cuuint64_t)seqlen,
+                              (cuuint64_t)batch};
+    const cuuint64_t xs[3] = {(cuuint64_t)(headdim * 2), (cuuint64_t)(nheads * headdim * 2),
+                              (cuuint64_t)(seqlen * nheads * headdim * 2)};
+    const cuuint32_t xb[4] = {64, 1, 128, 1};
+    const cuuint64_t bd[3] = {(cuuint64_t)dstate, (cuuint64_t)seqlen, (cuuint64_t)batch};
+    const cuuint64_t bs[2] = {(cuuint64_t)(dstate * 2), (cuuint64_t)(seqlen * dstate * 2)};
+    const cuuint32_t bb[3] = {64, 128, 1};
+    if (!encode_sw128_bf16(&maps.x, x, 4, xd, xs, xb) ||
+        !encode_sw128_bf16(&maps.B, B, 3, bd, bs, bb) ||
+        !encode_sw128_bf16(&maps.C, C, 3, bd, bs, bb))
+      return SSM_ERR_CUDA;
+    return cuda_status(launch_ssd_tc(p, maps, static_cast<cudaStream_t>(stream)),
+                       "ssd scan launch (tcgen05)");
+  }
   return cuda_status(launch_ssd_fwd(p, static_cast<cudaStream_t>(stream)), "ssd scan launch");
+}
+
+int ssm_ssd_scan_status(void* stream) {
+  int v = 0;
+  const cudaError_t e = ssd_tc_status(static_cast<cudaStream_t>(stream), &v);
+  if (e != cudaSuccess) return fail(SSM_ERR_CUDA, "ssm_ssd_scan_status", e);
+  return v ? fail(SSM_ERR_TIMEOUT, "a CTA of the SSD scan gave up a bounded wait") : SSM_OK;
 }
 
 int ssm_ssd_state_update(int64_t batch, int64_t nheads, int64_t headdim, int64_t dstate,
@@ -880,7 +930,7 @@ int ssm_compose_carries(int64_t rank, int64_t batch, int64_t dim, int64_t dstate
 // workspace. It allocates nothing.
 namespace {
 
-constexpr size_t kNoallocScratchBytes = size_t(8) << 20;  // 8 MiB per GPU
+constexpr size_t kNoallocScratchBytes = size_t(16) << 20;  // 16 MiB per GPU
 constexpr int kNoallocMaxDevices = 64;
 
 // The reserved scratch. In host code this name is only a stand-in for the
@@ -889,25 +939,72 @@ constexpr int kNoallocMaxDevices = 64;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
 
 std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kNoallocMaxDevices] = {};
+// Address of the scratch per device, with the context it was looked up in:
+// a context that was torn down and created again (cudaDeviceReset) loads the
+// module again, and the address is then looked up again.
+struct NoallocEntry {
+  CUcontext ctx;
+  void* ptr;
+};
+NoallocEntry g_noalloc[kNoallocMaxDevices] = {};
 
-// Device address of the scratch on the current device, looked up the first
-// time this device is seen (with the device current).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+CtxGetCurrentFn ctx_get_current_fn() {
+  static CtxGetCurrentFn fn = []() -> CtxGetCurrentFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    return reinterpret_cast<CtxGetCurrentFn>(p);
+  }();
+  return fn;
+}
+
+// Device address of the scratch on the current device, looked up (with the
+// device current) the first time this device's context is seen.
 int noalloc_scratch(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return fail(SSM_ERR_CUDA, "ssm_scan_fwd_noalloc: cudaGetDevice", e);
   if (dev < 0 || dev >= kNoallocMaxDevices)
     return fail(SSM_ERR_UNSUPPORTED, "ssm_scan_fwd_noalloc: device index above 63");
+  CtxGetCurrentFn ctx_fn = ctx_get_current_fn();
+  if (!ctx_fn) return fail(SSM_ERR_CUDA, "ssm_scan_fwd_noalloc: cuCtxGetCurrent unavailable");
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  CUcontext ctx = nullptr;
+  if (ctx_fn(&ctx) != CUDA_SUCCESS) ctx = nullptr;
+  if (!ctx || g_noalloc[dev].ctx != ctx || !g_noalloc[dev].ptr) {
     void* p = nullptr;
+    // also makes the device's primary context current when none was
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess || !p)
       return fail(SSM_ERR_CUDA, "ssm_scan_fwd_noalloc: cudaGetSymbolAddress of the scratch", e);
-    g_noalloc_ptr[dev] = p;
+    if (ctx_fn(&ctx) != CUDA_SUCCESS || !ctx)
+      return fail(SSM_ERR_CUDA, "ssm_scan_fwd_noalloc: no current context");
+    g_noalloc[dev].ctx = ctx;
+    g_noalloc[dev].ptr = p;
   }
-  *out = g_noalloc_ptr[dev];
+  *out = g_noalloc[dev].ptr;
+  return SSM_OK;
+}
+
+// Scratch bytes a problem needs, or an error code when it is invalid or does
+// not fit the reserved array.
+int noalloc_need(const Dims& d, size_t* need) {
+  const int st = dims_status(d);
+  if (st != SSM_OK) return st;
+  *need = make_plan(d).bytes;
+  if (*need > kNoallocScratchBytes) {
+    snprintf(g_detail, sizeof g_detail,
+             "ssm_scan_fwd_noalloc: this problem needs %zu bytes of scratch but the built-in "
+             "scratch holds %zu; call ssm_scan_fwd with a workspace instead",
+             *need, kNoallocScratchBytes);
+    return SSM_ERR_WORKSPACE;
+  }
   return SSM_OK;
 }
 
@@ -923,17 +1020,31 @@ extern "C" int ssm_scan_fwd_noalloc(int64_t batch, int64_t seqlen, int64_t dim, 
   const int st = dims_status(d);
   if (st != SSM_OK) return st;
   if (batch == 0 || dim == 0) return SSM_OK;
-  const size_t need = make_plan(d).bytes;
-  if (need > kNoallocScratchBytes) {
-    snprintf(g_detail, sizeof g_detail,
-             "ssm_scan_fwd_noalloc: this problem needs %zu bytes of scratch but the built-in "
-             "scratch holds %zu; call ssm_scan_fwd with a workspace instead",
-             need, kNoallocScratchBytes);
-    return SSM_ERR_WORKSPACE;
-  }
+  size_t need = 0;
+  int rc = noalloc_need(d, &need);
+  if (rc != SSM_OK) return rc;
   void* scratch = nullptr;
-  const int rc = noalloc_scratch(&scratch);
+  rc = noalloc_scratch(&scratch);
   if (rc != SSM_OK) return rc;
   return ssm_scan_fwd(batch, seqlen, dim, dstate, io_dtype, x, delta, A, B, C, D, z, delta_bias,
                       softplus, h0, y, h_last, scratch, kNoallocScratchBytes, stream);
+}
+
+// The per-CTA status words of a no-alloc call live in the reserved scratch,
+// which its callers cannot name: this reads them there (as ssm_scan_status
+// does from a caller's workspace).
+extern "C" int ssm_scan_status_noalloc(int64_t batch, int64_t seqlen, int64_t dim,
+                                       int64_t dstate, int io_dtype, void* stream) {
+  const Dims d{batch, seqlen, dim, dstate, io_dtype};
+  const int st = dims_status(d);
+  if (st != SSM_OK) return st;
+  if (batch == 0 || dim == 0) return SSM_OK;
+  size_t need = 0;
+  int rc = noalloc_need(d, &need);
+  if (rc != SSM_OK) return rc;
+  void* scratch = nullptr;
+  rc = noalloc_scratch(&scratch);
+  if (rc != SSM_OK) return rc;
+  return ssm_scan_status(scratch, kNoallocScratchBytes, batch, seqlen, dim, dstate, io_dtype,
+                         stream);
 }

@@ -14,8 +14,9 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 // softplus(v) is taken as v itself above this cut (natural-log units).
 constexpr float kSoftplusCut = 20.0f;
-// Smallest magnitude of the per-step rescaling factor of the state (2^-64);
-// see the scaled recurrence in ssm_scan_kernels.cu.
+// Input multipliers below this magnitude (2^-64) do not become the state's
+// scale; such a step takes the exact slow path of the scaled recurrence in
+// ssm_scan_kernels.cu.
 constexpr float kScaleFloor = 5.42101086242752217e-20f;
 
 // ---------------------------------------------------------------- MUFU ----
@@ -58,6 +59,13 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
   return __fmul2_rn(a, b);
 #else
   return make_float2(a.x * b.x, a.y * b.y);
+#endif
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+#if SSM_PACKED_FP32
+  return __fadd2_rn(a, b);
+#else
+  return make_float2(a.x + b.x, a.y + b.y);
 #endif
 }
 
@@ -163,6 +171,21 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     if (mbar_try_wait(bar, parity)) return true;
     if (global_timer_ns() - t0 > limit_ns) return false;
   }
+}
+
+// ------------------------------------------------------------- cp.async --
+// 16-byte asynchronous copy global -> shared (L1 bypassed).
+__device__ __forceinline__ void cp_async_16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit_group() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+// Wait until at most `n` committed groups of this thread are still in flight.
+template <int n>
+__device__ __forceinline__ void cp_async_wait_group() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(n) : "memory");
 }
 
 // ------------------------------------------- programmatic dependent launch --

@@ -3,6 +3,7 @@
 // public ABI.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -26,9 +27,24 @@ struct SsdParams {
   const float* h0;     // (batch, nheads, headdim, dstate) or null
   uint16_t* y;         // (batch, seqlen, nheads, headdim) bf16
   float* h_last;       // (batch, nheads, headdim, dstate) or null
+  uint64_t wait_limit_ns;  // bound on every wait of the tensor-core kernel
+  int test_stall;          // test hook: its first CTA waits for 16 bytes that never arrive
+};
+
+// TMA maps of the tensor-core kernel (128-byte swizzle): x as (headdim, nheads,
+// seqlen, batch) with a 64 x 1 x 128 x 1 box; B and C as (dstate, seqlen,
+// batch) with a 64 x 128 x 1 box.
+struct alignas(64) SsdTcMaps {
+  CUtensorMap x, B, C;
 };
 
 bool ssd_dstate_supported(int dstate);
 cudaError_t launch_ssd_fwd(const SsdParams& p, cudaStream_t stream);
+// The tensor-core (tcgen05) kernel: dstate 64 or 128, an even head count.
+bool ssd_tc_supported(int dstate, int nheads);
+cudaError_t launch_ssd_tc(const SsdParams& p, const SsdTcMaps& maps, cudaStream_t stream);
+// Synchronise `stream`; *out = 1 (and the flag cleared) if a CTA of the
+// tensor-core kernel gave up a wait since the last call, else 0.
+cudaError_t ssd_tc_status(cudaStream_t stream, int* out);
 
 }  // namespace ssm

@@ -53,7 +53,7 @@ def test_plan_splits_long_sequences(L):
     assert L.ssm_scan_plan(1, 262144, 1536, 16, 1, ctypes.byref(p)) == 0
     assert p.segments > 1 and p.segment_steps % 16 == 0
     assert (p.segments - 1) * p.segment_steps < 262144 <= p.segments * p.segment_steps
-    assert p.kernels == 2 and p.channels_per_cta == 256 and p.channel_tiles == 6
+    assert p.kernels == 3 and p.channels_per_cta == 256 and p.channel_tiles == 6
     assert p.ctas_main == p.segments * 6 and p.ctas_carry == (p.segments - 1) * 6
     assert p.workspace_bytes == L.ssm_scan_workspace_bytes(1, 262144, 1536, 16, 1)
     q = bnd.ScanPlan()
@@ -319,3 +319,17 @@ def test_oversized_problems_are_rejected(L):
     assert L.ssm_delta_sum(65535, 1 << 30, 1 << 20, 1, FAKE, None, 1, FAKE, None) == -2
     assert L.ssm_compose_carries(1 << 20, 65535, 1 << 20, 16, FAKE, None, FAKE, FAKE, FAKE,
                                  None) == -2
+
+
+def test_noalloc_status_rejects_on_the_host(L):
+    """ssm_scan_status_noalloc checks its sizes before it looks at any GPU:
+    bad dtype or dstate, and problems the reserved scratch cannot hold."""
+    assert L.ssm_scan_status_noalloc(1, 16, 64, 16, 7, None) == -2      # dtype
+    assert L.ssm_scan_status_noalloc(1, 16, 64, 3, 1, None) == -2       # dstate
+    assert L.ssm_scan_status_noalloc(-1, 16, 64, 16, 1, None) == -1     # size
+    assert L.ssm_scan_status_noalloc(0, 16, 64, 16, 1, None) == 0       # empty: nothing ran
+    os.environ["SSM_SCAN_SEGMENTS"] = "64"
+    try:
+        assert L.ssm_scan_status_noalloc(8, 4096, 2048, 16, 1, None) == -3
+    finally:
+        del os.environ["SSM_SCAN_SEGMENTS"]

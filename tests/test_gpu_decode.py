@@ -101,3 +101,39 @@ def test_decode_large_ragged(N, batch, dim):
                                  **kw)
         assert rel_err(host(y), yr) <= TOL["bf16"], f"step {step}"
     assert rel_err(host(state), ref) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("N,io,optional,batch,dim", [
+    (16, "f32", True, 8, 768), (16, "bf16", True, 8, 768), (16, "bf16", False, 8, 768),
+    (16, "f32", False, 8, 768), (32, "f32", True, 4, 384), (32, "bf16", False, 12, 384),
+    (64, "bf16", True, 4, 192), (64, "f32", False, 8, 192),
+    (16, "bf16", True, 96, 4096),  # 1536 tiles: several per CTA
+])
+def test_pipelined_decode_shapes(monkeypatch, N, io, optional, batch, dim):
+    """Shapes the pipelined decode kernel takes (batch a multiple of 4, whole
+    tiles of 1024 / N channels, 16-byte aligned rows): against the oracle step
+    by step, and bit for bit against the one-shot kernel
+    (SSM_DECODE_ONE_SHOT=1), which does the same arithmetic."""
+    from selective_state_space_39_b200 import ssm_state_update
+    steps = 6 if batch < 96 else 3
+    seed = 100 + N + (7 if optional else 0)
+    const = gen.decode_constants(dim, N, seed)
+    rng = np.random.default_rng(seed)
+    A = (-rng.uniform(0.2, 3.0, (dim, N))).astype(np.float32) if N != 16 else const["A"]
+    h0 = rng.standard_normal((batch, dim, N)).astype(np.float32)
+    ref = h0.astype(np.float64)
+    s2, s1 = dev(h0).clone(), dev(h0).clone()
+    for step in range(steps):
+        inp = gen.make_decode_inputs(batch, dim, N, io, seed, step)
+        kw = dict(D=const["D"], z=inp["z"], delta_bias=const["delta_bias"]) if optional else {}
+        args = (dev(inp["x"]), dev(inp["delta"]), dev(A), dev(inp["B"]), dev(inp["C"]))
+        dkw = {k: dev(v) for k, v in kw.items()}
+        monkeypatch.delenv("SSM_DECODE_ONE_SHOT", raising=False)
+        y2 = ssm_state_update(s2, *args, **dkw)
+        monkeypatch.setenv("SSM_DECODE_ONE_SHOT", "1")
+        y1 = ssm_state_update(s1, *args, **dkw)
+        monkeypatch.delenv("SSM_DECODE_ONE_SHOT")
+        yr = oracle.state_update(ref, inp["x"], inp["delta"], A, inp["B"], inp["C"], io=io, **kw)
+        assert rel_err(host(y2), yr) <= TOL[io], f"step {step}"
+        assert torch.equal(y1, y2) and torch.equal(s1, s2), f"step {step}"
+    assert rel_err(host(s2), ref) <= TOL[io]

@@ -216,3 +216,62 @@ def test_ssd_empty_batch_and_heads():
         yd = ssm_ssd_state_update(state, dev(d["x"]), dev(d["dt"]), dev(inp["A"]), dev(d["B"]),
                                   dev(d["C"]))
         assert yd.shape == (batch, H, 64)
+
+
+# ------------------------------------------- the tcgen05 path (state in TMEM)
+@pytest.mark.parametrize("N", [64, 128])
+@pytest.mark.parametrize("L", [1, 127, 128, 129, 300])
+def test_ssd_tcgen05_matches_oracle_and_legacy(monkeypatch, N, L):
+    """Even head counts with dstate 64 / 128 take the tcgen05 kernel (128-step
+    chunks, state in tensor memory); SSM_SSD_LEGACY=1 the warp-level MMA one.
+    Lengths around the chunk size: one step, a ragged single chunk, exactly
+    one chunk, one step past it, and two chunks plus a ragged one."""
+    inp = gen.make_ssd_inputs(2, L, 4, 64, N, "bf16", 300 + N + L, with_h0=True)
+    yr, hr = reference(inp)
+    monkeypatch.delenv("SSM_SSD_LEGACY", raising=False)
+    y, hl = run(inp)
+    monkeypatch.setenv("SSM_SSD_LEGACY", "1")
+    y2, hl2 = run(inp)
+    for what, (a, b) in {"tcgen05": (y, hl), "legacy": (y2, hl2)}.items():
+        ey, eh = rel_err(host(a), yr), rel_err(host(b), hr)
+        print(f"{what} N={N} L={L}: y {ey:.3e} h_last {eh:.3e}")
+        assert torch.isfinite(a.float()).all() and torch.isfinite(b).all()
+        assert ey <= TOL and eh <= TOL, f"{what} N={N} L={L}"
+
+
+def test_ssd_tcgen05_in_place_state_and_no_h_last(monkeypatch):
+    """h_last may be h0 itself (each CTA reads its heads' state before it
+    writes them); without h_last only y is written."""
+    monkeypatch.delenv("SSM_SSD_LEGACY", raising=False)
+    from selective_state_space_39_b200 import ssm_ssd_scan_fwd
+    inp = gen.make_ssd_inputs(2, 200, 6, 64, 128, "bf16", 311, with_h0=True)
+    yr, hr = reference(inp)
+    h = dev(inp["h0"]).clone()
+    y, hl = ssm_ssd_scan_fwd(dev(inp["x"]), dev(inp["dt"]), dev(inp["A"]), dev(inp["B"]),
+                             dev(inp["C"]), D=dev(inp["D"]), dt_bias=dev(inp["dt_bias"]), h0=h,
+                             h_last=h, return_last_state=True)
+    assert hl.data_ptr() == h.data_ptr()
+    assert rel_err(host(y), yr) <= TOL and rel_err(host(hl), hr) <= TOL
+    y3 = run(inp, last=False)
+    assert rel_err(host(y3), yr) <= TOL
+
+
+def test_ssd_tcgen05_timeout_is_reported(monkeypatch):
+    """One CTA waits for 16 bytes that no copy delivers (test hook): its
+    bounded wait runs out, it frees its tensor memory, ssm_ssd_scan_status
+    reports the timeout once, and the next call is correct."""
+    from selective_state_space_39_b200 import ssm_ssd_scan_status
+    monkeypatch.delenv("SSM_SSD_LEGACY", raising=False)
+    inp = gen.make_ssd_inputs(1, 256, 4, 64, 128, "bf16", 313, with_h0=True)
+    assert ssm_ssd_scan_status() == 0
+    monkeypatch.setenv("SSM_SSD_TEST_STALL", "1")
+    monkeypatch.setenv("SSM_SCAN_WAIT_LIMIT_NS", "20000000")  # 20 ms
+    run(inp)
+    assert ssm_ssd_scan_status() == -5
+    assert ssm_ssd_scan_status() == 0  # the flag is cleared
+    monkeypatch.delenv("SSM_SSD_TEST_STALL")
+    monkeypatch.delenv("SSM_SCAN_WAIT_LIMIT_NS")
+    y, hl = run(inp)
+    assert ssm_ssd_scan_status() == 0
+    yr, hr = reference(inp)
+    assert rel_err(host(y), yr) <= TOL and rel_err(host(hl), hr) <= TOL
