@@ -101,22 +101,37 @@ def test_ssd_deterministic():
     assert torch.equal(y1, y2) and torch.equal(h1, h2)
 
 
-def test_ssd_split_sequence_carries_the_state():
-    """Two calls (first 96 steps, then the rest from the returned state) match
-    one call over the whole sequence."""
+@pytest.mark.parametrize("legacy", [False, True])
+def test_ssd_split_sequence_carries_the_state(monkeypatch, legacy):
+    """Two calls (the first steps, then the rest from the returned state)
+    against one call over the whole sequence. Split at a multiple of the
+    kernels' chunk lengths (128 steps for the tcgen05 kernel, 32 for the
+    warp-level one) the chunks and their arithmetic are the same, so the
+    results are bit for bit equal; split anywhere else (96) the chunks group
+    the steps differently, and both calls together still match the oracle's
+    sequential loop within the bound."""
     from selective_state_space_39_b200 import ssm_ssd_scan_fwd
-    inp = gen.make_ssd_inputs(1, 200, 2, 64, 128, "bf16", 21, with_h0=True)
+    if legacy:
+        monkeypatch.setenv("SSM_SSD_LEGACY", "1")
+    else:
+        monkeypatch.delenv("SSM_SSD_LEGACY", raising=False)
+    inp = gen.make_ssd_inputs(1, 300, 2, 64, 128, "bf16", 21, with_h0=True)
     d = {k: dev(v) for k, v in inp.items()}
     y, hl = ssm_ssd_scan_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], D=d["D"],
                              dt_bias=d["dt_bias"], h0=d["h0"], return_last_state=True)
+    yr, hr = reference(inp)
     cut = lambda t, a, b: t[:, a:b].contiguous()  # noqa: E731
-    y1, h1 = ssm_ssd_scan_fwd(cut(d["x"], 0, 96), cut(d["dt"], 0, 96), d["A"],
-                              cut(d["B"], 0, 96), cut(d["C"], 0, 96), D=d["D"],
-                              dt_bias=d["dt_bias"], h0=d["h0"], return_last_state=True)
-    y2, h2 = ssm_ssd_scan_fwd(cut(d["x"], 96, 200), cut(d["dt"], 96, 200), d["A"],
-                              cut(d["B"], 96, 200), cut(d["C"], 96, 200), D=d["D"],
-                              dt_bias=d["dt_bias"], h0=h1, return_last_state=True)
-    assert torch.equal(torch.cat([y1, y2], dim=1), y) and torch.equal(h2, hl)
+    for k in (128, 96):
+        y1, h1 = ssm_ssd_scan_fwd(cut(d["x"], 0, k), cut(d["dt"], 0, k), d["A"],
+                                  cut(d["B"], 0, k), cut(d["C"], 0, k), D=d["D"],
+                                  dt_bias=d["dt_bias"], h0=d["h0"], return_last_state=True)
+        y2, h2 = ssm_ssd_scan_fwd(cut(d["x"], k, 300), cut(d["dt"], k, 300), d["A"],
+                                  cut(d["B"], k, 300), cut(d["C"], k, 300), D=d["D"],
+                                  dt_bias=d["dt_bias"], h0=h1, return_last_state=True)
+        ys = torch.cat([y1, y2], dim=1)
+        if k == 128 or legacy:
+            assert torch.equal(ys, y) and torch.equal(h2, hl), f"split at {k}"
+        assert rel_err(host(ys), yr) <= TOL and rel_err(host(h2), hr) <= TOL, f"split at {k}"
 
 
 # ---- decode step (fp32 state in HBM; fp32 arithmetic: 1e-5 for fp32 io, 1e-2 bf16)
