@@ -136,7 +136,7 @@ class ClockSampler:
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
                0x100: "display_clock_setting"}
 
-    def __init__(self, device_index, interval_s=0.002):
+    def __init__(self, device_index, interval_s=0.0002):
         self.samples, self.reasons, self.max_mhz, self.error = [], 0, None, None
         self.interval = interval_s
         self._stop = threading.Event()

@@ -74,9 +74,10 @@ enum {
 /*
  * How ssm_scan_fwd splits a problem (see ssm_scan_plan). The sequence is cut
  * into `segments` of `segment_steps` steps; with more than one segment a
- * carry pass computes each segment's end state, a small kernel (with three or
- * more segments) composes them into every segment's start state, and the
- * main pass runs each segment from its start (the recurrence of §2.2 is an
+ * carry pass computes each segment's end state, the carries are composed into
+ * every segment's start state (by the main pass itself up to 9 segments, by a
+ * small kernel between the passes above that), and the main pass runs each
+ * segment from its start (the recurrence of §2.2 is an
  * associative composition of affine maps h -> a*h + b, which the pages'
  * parallel associative scan relies on).
  */

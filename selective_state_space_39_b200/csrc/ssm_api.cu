@@ -297,7 +297,7 @@ int ssm_scan_plan(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate, in
   out->channels_per_cta = pl.dtile;
   out->ctas_carry = pl.ctas_agg;
   out->ctas_main = pl.ctas_main;
-  out->kernels = (batch > 0 && dim > 0) ? (pl.nseg > 2 ? 3 : pl.nseg > 1 ? 2 : 1) : 0;
+  out->kernels = (batch > 0 && dim > 0) ? (pl.nseg > kScanPrologueCompose ? 3 : pl.nseg > 1 ? 2 : 1) : 0;
   out->workspace_bytes = (int64_t)pl.bytes;
   return SSM_OK;
 }

@@ -25,6 +25,9 @@ constexpr int kScanThreads = SSM_CTA_THREADS;  // threads per CTA with 1 or 2 ch
 constexpr int scan_threads(int cpt) { return cpt == 4 ? kScanThreads / 2 : kScanThreads; }
 constexpr int kScanTileSteps = SSM_TILE_STEPS;
 constexpr int kScanStages = SSM_STAGES;
+// Segment counts up to which the main pass composes the segment carries in
+// its prologue (above it a separate kernel does, between the two passes).
+constexpr int kScanPrologueCompose = 9;
 // Per-CTA status codes written to the workspace status area.
 constexpr int kCtaOk = 0;
 constexpr int kCtaTimeout = 1;

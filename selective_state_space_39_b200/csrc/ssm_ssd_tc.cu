@@ -71,8 +71,8 @@ struct TcLayout {
   static constexpr int kOffG = kOffC + kBC;
   static constexpr int kOffHb = kOffG + kG;
   static constexpr int kOffSteps = kOffHb + kHb;
-  // per head: Delta[Q], cum[Q], w[Q]; warp sums [2][4]; decay [2]; error flag
-  static constexpr int kStepFloats = kTHeads * 3 * kTQ + kTHeads * 4 + kTHeads + 2;
+  // per head: Delta[Q], cum[Q], w[Q], E[Q]; warp sums [2][4]; decay [2]
+  static constexpr int kStepFloats = kTHeads * 4 * kTQ + kTHeads * 4 + kTHeads + 2;
   static constexpr int kOffBar = round_up(kOffSteps + kStepFloats * 4, 8);
   static constexpr int kNumBars = 6;  // B/C, x (two buffers), S, first MMAs, second MMAs
   static constexpr int kOffSlot = kOffBar + kNumBars * 8;
@@ -109,7 +109,8 @@ __global__ void __launch_bounds__(kTThreads, 1)
   float* f_delta = reinterpret_cast<float*>(sm + Ly::kOffSteps);  // [2][Q]
   float* f_cum = f_delta + kTHeads * kTQ;                          // [2][Q]
   float* f_w = f_cum + kTHeads * kTQ;                              // [2][Q]
-  float* f_wsum = f_w + kTHeads * kTQ;                             // [2][4]
+  float* f_e = f_w + kTHeads * kTQ;                                // [2][Q]
+  float* f_wsum = f_e + kTHeads * kTQ;                             // [2][4]
   float* f_decay = f_wsum + kTHeads * 4;                           // [2]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Ly::kOffBar);
   uint64_t* bar_bc = bars + 0;
@@ -119,7 +120,8 @@ __global__ void __launch_bounds__(kTThreads, 1)
   uint64_t* bar_m2 = bars + 5;
   (void)bar_m2;
   uint32_t* slot = reinterpret_cast<uint32_t*>(sm + Ly::kOffSlot);
-  unsigned char* xbuf[2] = {sm + Ly::kOffX0, sm + Ly::kOffX1};
+  unsigned char* const xbuf0 = sm + Ly::kOffX0;
+  unsigned char* const xbuf1 = sm + Ly::kOffX1;
   unsigned char* sB = sm + Ly::kOffB;
   unsigned char* sC = sm + Ly::kOffC;
   unsigned char* sG = sm + Ly::kOffG;
@@ -178,33 +180,34 @@ __global__ void __launch_bounds__(kTThreads, 1)
     }
   };
   auto issue_x = [&](int c, int i) {
-    mbar_arrive_expect_tx(&bar_x[i], (uint32_t)(kTHeads * Ly::kBlk) + ((stall && c == 0) ? 16u : 0u));
+    uint64_t* bar = i ? &bar_x[1] : &bar_x[0];
+    unsigned char* dst = i ? xbuf1 : xbuf0;
+    mbar_arrive_expect_tx(bar, (uint32_t)(kTHeads * Ly::kBlk) + ((stall && c == 0) ? 16u : 0u));
 #pragma unroll
     for (int hh = 0; hh < kTHeads; ++hh)
-      tc::tma_load_4d(xbuf[i] + hh * Ly::kBlk, &maps.x, &bar_x[i], 0, h0 + hh, c * kTQ, b);
+      tc::tma_load_4d(dst + hh * Ly::kBlk, &maps.x, bar, 0, h0 + hh, c * kTQ, b);
   };
-  // Phases armed and phases waited per barrier (thread 0 keeps the count; the
-  // error path drains what is still in flight before TMEM and shared memory
-  // are released).
-  int armed[Ly::kNumBars] = {0, 0, 0, 0, 0, 0}, waited[Ly::kNumBars] = {0, 0, 0, 0, 0, 0};
+  // Each barrier completes once per chunk (an x buffer every other chunk), in
+  // order, so the phase to wait for follows from the chunk index; on the
+  // error path thread 0 waits (bounded) for the completions still owed.
+  // armed_*: phases armed so far by thread 0 (B/C, x0, x1, S, MMA1, MMA2).
+  int armed_bc = 0, armed_x0 = 0, armed_x1 = 0, armed_s = 0, armed_m1 = 0, armed_m2 = 0;
+  // phases waited (every thread)
+  int waited_bc = 0, waited_x0 = 0, waited_x1 = 0, waited_s = 0, waited_m1 = 0, waited_m2 = 0;
   if (tid == 0 && nchunks > 0) {
     issue_bc(0);
     issue_x(0, 0);
-    armed[0] = 1;
-    armed[1] = 1;
+    armed_bc = 1;
+    armed_x0 = 1;
   }
-  // bars: 0 = B/C, 1 + i = x buffer i, 3 = S, 4 = first MMAs, 5 = second MMAs
-  auto wait_bar = [&](int i) {
-    const bool r = cta_wait(&bars[i], (uint32_t)(waited[i] & 1), p.wait_limit_ns);
-    if (r) ++waited[i];
-    return r;
-  };
-  // raw dt of this thread's step in chunk c, both heads
+  // raw dt of this thread's step in chunk c, both heads (one 4-byte load:
+  // h0 and H are even)
   auto load_dt = [&](int c, float (&r)[kTHeads]) {
     const int64_t t = (int64_t)c * kTQ + tid;
-#pragma unroll
-    for (int hh = 0; hh < kTHeads; ++hh)
-      r[hh] = t < L ? bf16_to_f32(p.dt[((size_t)b * L + t) * H + h0 + hh]) : 0.f;
+    const uint32_t w = t < L ? *reinterpret_cast<const uint32_t*>(p.dt + ((size_t)b * L + t) * H + h0)
+                             : 0u;
+    r[0] = bf16_lo(w);
+    r[1] = bf16_hi(w);
   };
   float dt_next[kTHeads];
   if (nchunks > 0) load_dt(0, dt_next);
@@ -252,11 +255,14 @@ __global__ void __launch_bounds__(kTThreads, 1)
     for (int hh = 0; hh < kTHeads; ++hh) {
       const float cend = f_cum[hh * kTQ + kTQ - 1];
       f_w[hh * kTQ + tid] = expf(cend - cum[hh]) * dl[hh];
+      // factor of column s of G below the diagonal 32 x 32 blocks (<= Delta_s)
+      f_e[hh * kTQ + tid] = expf(f_cum[hh * kTQ + (tid | 31)] - cum[hh]) * dl[hh];
       if (tid == 0) f_decay[hh] = expf(cend);
     }
     // ---- 2. S = C B^T once this chunk's B and C have landed
-    ok = wait_bar(0);
+    ok = cta_wait(bar_bc, (uint32_t)(c & 1), p.wait_limit_ns);
     if (!ok) break;
+    ++waited_bc;
     if (tid == 0) {
       tc::fence_after_sync();
       constexpr uint32_t id = tc::idesc_bf16(128, 128, 0, 0);
@@ -267,22 +273,25 @@ __global__ void __launch_bounds__(kTThreads, 1)
                      tc::sdesc(smem_u32(sB) + o, 16, 1024), id, ks > 0);
       }
       tc::commit(bar_s);
-      ++armed[3];
+      ++armed_s;
     }
     // ---- 3. this chunk's x: w-scaled copy into the other buffer (row s =
     //      thread); the state: bf16 copy for the readout, then scaled by
     //      e^{cum_end} in place for the update (row hp = thread)
-    ok = wait_bar(1 + xi);
+    ok = cta_wait(xi ? &bar_x[1] : &bar_x[0], (uint32_t)((c >> 1) & 1), p.wait_limit_ns);
     if (!ok) break;
+    if (xi) ++waited_x1; else ++waited_x0;
+    unsigned char* const xcur = xi ? xbuf1 : xbuf0;  // x of this chunk
+    unsigned char* const xoth = xi ? xbuf0 : xbuf1;  // its w-scaled copy
     {
-      const unsigned char* src = xbuf[xi];
-      unsigned char* dst = xbuf[xi ^ 1];
+      const unsigned char* src = xcur;
+      unsigned char* dst = xoth;
 #pragma unroll
       for (int hh = 0; hh < kTHeads; ++hh) {
         const float w = f_w[hh * kTQ + tid];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          const uint32_t o = hh * Ly::kBlk + tid * 128 + j * 16;
+          const uint32_t o = hh * Ly::kBlk + tid * 128 + ((j + tid) & 7) * 16;
           const uint4 q = *reinterpret_cast<const uint4*>(src + o);
           const float v[8] = {bf16_lo(q.x) * w, bf16_hi(q.x) * w, bf16_lo(q.y) * w,
                               bf16_hi(q.y) * w, bf16_lo(q.z) * w, bf16_hi(q.z) * w,
@@ -292,53 +301,73 @@ __global__ void __launch_bounds__(kTThreads, 1)
       }
       const float decay = f_decay[tid / kTP];
 #pragma unroll
-      for (int c0 = 0; c0 < N; c0 += 32) {
-        float v[32];
+      for (int c0 = 0; c0 < N; c0 += 64) {
+        float v[32], u[32];
         tc::ld32(tH + c0, v);
+        tc::ld32(tH + c0 + 32, u);
         tc::wait_ld();
 #pragma unroll
         for (int j = 0; j < 32; j += 8) {
-          const int col = c0 + j;
-          *reinterpret_cast<uint4*>(sHb + (col / 64) * Ly::kBlk + tc::sw128(tid, col % 64)) =
-              pack8(v + j);
+          *reinterpret_cast<uint4*>(sHb + (c0 / 64) * Ly::kBlk + tc::sw128(tid, j)) = pack8(v + j);
+          *reinterpret_cast<uint4*>(sHb + (c0 / 64) * Ly::kBlk + tc::sw128(tid, 32 + j)) =
+              pack8(u + j);
         }
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] *= decay;
+        for (int j = 0; j < 32; ++j) {
+          v[j] *= decay;
+          u[j] *= decay;
+        }
         tc::st32(tH + c0, v);
+        tc::st32(tH + c0 + 32, u);
       }
       tc::wait_st();
     }
     tc::fence_proxy_async_smem();
     tc::fence_before_sync();
     // ---- 4. G of head 0 from S (row t = thread)
-    ok = wait_bar(3);
+    ok = cta_wait(bar_s, (uint32_t)(c & 1), p.wait_limit_ns);
     if (!ok) break;
+    ++waited_s;
     tc::fence_after_sync();
+    // G row t (= thread) of head hh from S, in 32-column blocks j: below the
+    // diagonal block (32 j + 31 < t's block) e^{cum_t - cum_s} Delta_s =
+    // F_j E_s with F_j = e^{cum_t - cum_{32 j + 31}} (both factors <= 1, one
+    // exp per block); the diagonal block takes one exp per entry; above it G
+    // is zero.
     auto make_g = [&](int hh) {
       const float ct = f_cum[hh * kTQ + tid];
+      const int tb = tid >> 5;  // this row's diagonal block
 #pragma unroll
-      for (int c0 = 0; c0 < kTQ; c0 += 32) {
-        float v[32];
-        tc::ld32(tS + c0, v);
+      for (int c0 = 0; c0 < kTQ; c0 += 64) {
+        float v[2][32];
+        tc::ld32(tS + c0, v[0]);
+        tc::ld32(tS + c0 + 32, v[1]);
         tc::wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; j += 8) {
-          float g[8];
-          const int s0 = c0 + j;
-          if (s0 <= tid) {
+        for (int hb = 0; hb < 2; ++hb) {
+          const int j = (c0 >> 5) + hb;  // column block
+          const int s0 = 32 * j;
+          float g[32];
+          if (j < tb) {
+            const float F = expf(ct - f_cum[hh * kTQ + s0 + 31]);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const int s = s0 + e;
-              g[e] = s <= tid ? v[j + e] * ex2_approx((ct - f_cum[hh * kTQ + s]) * kLog2e) *
-                                    f_delta[hh * kTQ + s]
-                              : 0.f;
+            for (int e = 0; e < 32; ++e) g[e] = v[hb][e] * F * f_e[hh * kTQ + s0 + e];
+          } else if (j == tb) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const int sidx = s0 + e;
+              g[e] = sidx <= tid ? v[hb][e] * ex2_approx((ct - f_cum[hh * kTQ + sidx]) * kLog2e) *
+                                       f_delta[hh * kTQ + sidx]
+                                 : 0.f;
             }
           } else {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) g[e] = 0.f;
+            for (int e = 0; e < 32; ++e) g[e] = 0.f;
           }
-          *reinterpret_cast<uint4*>(sG + (s0 / 64) * Ly::kBlk + tc::sw128(tid, s0 % 64)) =
-              pack8(g);
+#pragma unroll
+          for (int e = 0; e < 32; e += 8)
+            *reinterpret_cast<uint4*>(sG + (s0 / 64) * Ly::kBlk + tc::sw128(tid, (s0 + e) % 64)) =
+                pack8(g + e);
         }
       }
     };
@@ -363,7 +392,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
 #pragma unroll
         for (int ks = 0; ks < kTQ / 16; ++ks) {
           const uint32_t o = ks * 2048;
-          tc::mma_bf16(tm + kColH, tc::sdesc(smem_u32(xbuf[xi ^ 1]) + o, Ly::kBlk, 1024),
+          tc::mma_bf16(tm + kColH, tc::sdesc(smem_u32(xoth) + o, Ly::kBlk, 1024),
                        tc::sdesc(smem_u32(sB) + o, Ly::kBlk, 1024), id, 1u);
         }
       }
@@ -373,22 +402,23 @@ __global__ void __launch_bounds__(kTThreads, 1)
         for (int ks = 0; ks < kTQ / 16; ++ks) {
           const uint32_t oa = (ks / 4) * Ly::kBlk + (ks % 4) * 32;
           tc::mma_bf16(tm + kColYd, tc::sdesc(smem_u32(sG) + oa, 16, 1024),
-                       tc::sdesc(smem_u32(xbuf[xi]) + ks * 2048, Ly::kBlk, 1024), id, ks > 0);
+                       tc::sdesc(smem_u32(xcur) + ks * 2048, Ly::kBlk, 1024), id, ks > 0);
         }
       }
       tc::commit(bar_m1);
-      ++armed[4];
+      ++armed_m1;
     }
     // ---- 6. the buffers of B, C and the scaled x are free: next chunk's
     //      loads; G of head 1 (G's buffer is free too), then its G X
-    ok = wait_bar(4);
+    ok = cta_wait(bar_m1, (uint32_t)(c & 1), p.wait_limit_ns);
     if (!ok) break;
+    ++waited_m1;
     tc::fence_after_sync();
     if (tid == 0 && c + 1 < nchunks) {
       issue_bc(c + 1);
       issue_x(c + 1, xi ^ 1);
-      ++armed[0];
-      ++armed[1 + (xi ^ 1)];
+      ++armed_bc;
+      if (xi) ++armed_x0; else ++armed_x1;
     }
     make_g(1);
     tc::fence_proxy_async_smem();
@@ -401,15 +431,16 @@ __global__ void __launch_bounds__(kTThreads, 1)
       for (int ks = 0; ks < kTQ / 16; ++ks) {
         const uint32_t oa = (ks / 4) * Ly::kBlk + (ks % 4) * 32;
         tc::mma_bf16(tm + kColYd + kTP, tc::sdesc(smem_u32(sG) + oa, 16, 1024),
-                     tc::sdesc(smem_u32(xbuf[xi]) + Ly::kBlk + ks * 2048, Ly::kBlk, 1024), id,
+                     tc::sdesc(smem_u32(xcur) + Ly::kBlk + ks * 2048, Ly::kBlk, 1024), id,
                      ks > 0);
       }
       tc::commit(bar_m2);
-      ++armed[5];
+      ++armed_m2;
     }
     // ---- 7. y_t = Yd + e^{cum_t} Yo + D x_t (row t = thread)
-    ok = wait_bar(5);
+    ok = cta_wait(bar_m2, (uint32_t)(c & 1), p.wait_limit_ns);
     if (!ok) break;
+    ++waited_m2;
     tc::fence_after_sync();
     {
       const int64_t t = t0 + tid;
@@ -426,7 +457,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
 #pragma unroll
           for (int j = 0; j < 32; j += 8) {
             const int pc = c0 + j;
-            const uint4 q = *reinterpret_cast<const uint4*>(xbuf[xi] + hh * Ly::kBlk +
+            const uint4 q = *reinterpret_cast<const uint4*>(xcur + hh * Ly::kBlk +
                                                             tc::sw128(tid, pc));
             const float xv[8] = {bf16_lo(q.x), bf16_hi(q.x), bf16_lo(q.y), bf16_hi(q.y),
                                  bf16_lo(q.z), bf16_hi(q.z), bf16_lo(q.w), bf16_hi(q.w)};
@@ -459,9 +490,15 @@ __global__ void __launch_bounds__(kTThreads, 1)
   } else if (tid == 0) {
     // A wait ran out: let this CTA's own copies and MMAs in flight land
     // (bounded) before its shared and tensor memory are released.
-    for (int i = 0; i < Ly::kNumBars; ++i)
-      for (int k = waited[i]; k < armed[i]; ++k)
-        (void)mbar_wait_bounded(&bars[i], (uint32_t)(k & 1), 1000000ull);
+    auto drain = [&](uint64_t* bar, int done, int armed) {
+      for (int k = done; k < armed; ++k) (void)mbar_wait_bounded(bar, (uint32_t)(k & 1), 1000000ull);
+    };
+    drain(bar_bc, waited_bc, armed_bc);
+    drain(&bar_x[0], waited_x0, armed_x0);
+    drain(&bar_x[1], waited_x1, armed_x1);
+    drain(bar_s, waited_s, armed_s);
+    drain(bar_m1, waited_m1, armed_m1);
+    drain(bar_m2, waited_m2, armed_m2);
     atomicExch(&g_ssd_status, 1);
   }
   tc::fence_before_sync();

@@ -53,7 +53,8 @@ def test_plan_splits_long_sequences(L):
     assert L.ssm_scan_plan(1, 262144, 1536, 16, 1, ctypes.byref(p)) == 0
     assert p.segments > 1 and p.segment_steps % 16 == 0
     assert (p.segments - 1) * p.segment_steps < 262144 <= p.segments * p.segment_steps
-    assert p.kernels == 3 and p.channels_per_cta == 256 and p.channel_tiles == 6
+    assert p.kernels == (3 if p.segments > 9 else 2)
+    assert p.channels_per_cta == 256 and p.channel_tiles == 6
     assert p.ctas_main == p.segments * 6 and p.ctas_carry == (p.segments - 1) * 6
     assert p.workspace_bytes == L.ssm_scan_workspace_bytes(1, 262144, 1536, 16, 1)
     q = bnd.ScanPlan()
