@@ -14,22 +14,27 @@
 //   y_t     = sum_s G[t][s] x_s + e^{cum_t} C_t H + D x_t
 //   H      <- e^{cum_end} H + sum_s w_s x_s B_s^T,   w_s = e^{cum_end - cum_s} Delta_s
 //
-// Design (B200). One CTA (128 threads, one per TMEM lane) per batch row and
-// pair of heads walks the chunks in order. Every product is one tcgen05 MMA
-// of M = 128 (bf16 operands from shared memory, fp32 accumulators in TMEM):
-// S (t x s, K = N), the readout C H^T (t x (2 heads x p), K = N), the
-// state update (2 heads x p) x n with K = s, and G X per head (t x p, K = s).
-// The state (2 x 64 rows, N columns) never leaves TMEM: each chunk one pass
-// of the threads reads it, keeps a bf16 copy in shared memory for the
-// readout, and writes it back scaled by e^{cum_end} before the update MMA
-// accumulates onto it. x, B and C chunks arrive by TMA with the 128-byte
-// swizzle the MMA descriptors describe (no multicast); the next chunk's B, C
-// and x are loaded as soon as the current chunk's MMAs have released their
-// buffers (two x buffers alternate between the raw x and the w-scaled x).
-// Steps past the sequence end read zeros and take Delta = 0, so they change
-// nothing. Every wait is bounded; a wait that runs out stops the CTA (after
-// its copies and MMAs in flight land, bounded too), frees its TMEM and sets
-// the status word that ssm_ssd_scan_status reports.
+// Design (B200). One CTA of eight warps per batch row and pair of heads walks
+// the chunks in order; warps w and w + 4 share TMEM lanes 32 (w % 4) .. and
+// split each row's columns (or the two heads) between them. Every product
+// is a tcgen05 MMA of M = 128 with fp32 accumulators in TMEM:
+//   S = C B^T (t x s, K = N; both operands from shared memory),
+//   the readout C H^T (t x (2 heads x p), K = N; H as a bf16 copy in shared
+//   memory),
+//   the state update (2 heads x p) x n, K = s (w-scaled x and B from shared
+//   memory, accumulating onto the state in TMEM),
+//   G X per head (t x p, K = s; G from TMEM, where it is written over S).
+// The state (2 x 64 rows, N columns) never leaves TMEM: each chunk the
+// threads read it, keep the bf16 copy for the readout and write it back
+// scaled by e^{cum_end} before the update MMA accumulates onto it. x, B and
+// C arrive by TMA with the 128-byte swizzle the MMA descriptors describe (no
+// multicast); the next chunk's copies start as soon as the chunk's MMAs have
+// released their buffers (two x buffers alternate between the raw x and the
+// w-scaled x), and the next chunk's step quantities are computed while the
+// chunk's MMAs run. Steps past the sequence end read zeros and take Delta =
+// 0, so they change nothing. Every wait is bounded; a wait that runs out
+// stops the CTA (after its copies and MMAs in flight land, bounded too),
+// frees its TMEM and sets the flag that ssm_ssd_scan_status reports.
 #include <stdlib.h>
 
 #include <mutex>
@@ -50,31 +55,32 @@ namespace {
 constexpr int kTQ = 128;        // steps per chunk
 constexpr int kTP = 64;         // head width
 constexpr int kTHeads = 2;      // heads per CTA
-constexpr int kTThreads = 128;  // one thread per TMEM lane
+constexpr int kTThreads = 256;  // eight warps, two per TMEM lane quadrant
 constexpr uint32_t kTmemCols = 512;
+// TMEM columns: the state, S (then G of both heads, bf16 pairs), G X, C H^T
 constexpr uint32_t kColH = 0, kColS = 128, kColYd = 256, kColYo = 384;
 
 constexpr int round_up(int v, int m) { return (v + m - 1) / m * m; }
 
 template <int N>
 struct TcLayout {
-  static constexpr int kNB = N / 64;                     // 64-wide blocks of the state
-  static constexpr int kBlk = kTQ * 128;                 // one [128 rows][64] bf16 tile
-  static constexpr int kXBuf = kTHeads * kBlk;           // [head][t][64 p]
-  static constexpr int kBC = kNB * kBlk;                 // [n block][t][64 n]
-  static constexpr int kG = 2 * kBlk;                    // [s block][t][64 s]
-  static constexpr int kHb = kNB * kBlk;                 // [n block][2 x 64 rows hp][64 n]
+  static constexpr int kNB = N / 64;               // 64-wide blocks of the state
+  static constexpr int kBlk = kTQ * 128;           // one [128 rows][64] bf16 tile
+  static constexpr int kXBuf = kTHeads * kBlk;     // [head][t][64 p]
+  static constexpr int kBC = kNB * kBlk;           // [n block][t][64 n]
+  static constexpr int kHb = kNB * kBlk;           // [n block][2 x 64 rows hp][64 n]
   static constexpr int kOffX0 = 0;
   static constexpr int kOffX1 = kXBuf;
   static constexpr int kOffB = 2 * kXBuf;
   static constexpr int kOffC = kOffB + kBC;
-  static constexpr int kOffG = kOffC + kBC;
-  static constexpr int kOffHb = kOffG + kG;
+  static constexpr int kOffHb = kOffC + kBC;
   static constexpr int kOffSteps = kOffHb + kHb;
-  // per head: Delta[Q], cum[Q], w[Q], E[Q]; warp sums [2][4]; decay [2]
-  static constexpr int kStepFloats = kTHeads * 4 * kTQ + kTHeads * 4 + kTHeads + 2;
+  // step quantities, two buffers (this chunk, the next): per head Delta[Q],
+  // cum[Q], w[Q], E[Q]
+  static constexpr int kStepBuf = kTHeads * 4 * kTQ;
+  static constexpr int kStepFloats = 2 * kStepBuf + kTHeads * 4 + 2 * kTHeads;
   static constexpr int kOffBar = round_up(kOffSteps + kStepFloats * 4, 8);
-  static constexpr int kNumBars = 6;  // B/C, x (two buffers), S, first MMAs, second MMAs
+  static constexpr int kNumBars = 5;  // B/C, x (two buffers), S, the chunk's MMAs
   static constexpr int kOffSlot = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffSlot + 16 + 1024;  // + room to align the base to 1024
   static_assert(N == 64 || N == 128, "state width 64 or 128");
@@ -87,10 +93,21 @@ __device__ __forceinline__ bool cta_wait(uint64_t* bar, uint32_t parity, uint64_
   return __syncthreads_and(ok) != 0;
 }
 
-// Eight fp32 values scaled and packed as eight bf16 (one 16-byte chunk).
+// Eight fp32 values packed as eight bf16 (one 16-byte chunk).
 __device__ __forceinline__ uint4 pack8(const float* v) {
   return make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
                     pack_bf16x2(v[6], v[7]));
+}
+
+// D (TMEM) = A B (+ D): A (M x 16, bf16 pairs) from TMEM, B from a
+// shared-memory descriptor; one K = 16 step, issued by one thread.
+__device__ __forceinline__ void mma_bf16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
+                                                uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
 }
 
 template <int N>
@@ -98,42 +115,44 @@ __global__ void __launch_bounds__(kTThreads, 1)
     ssd_tc_kernel(const SsdParams p, const __grid_constant__ SsdTcMaps maps) {
   using Ly = TcLayout<N>;
   constexpr int kNB = Ly::kNB;
+  constexpr int kHalfN = N / 2;  // state columns per warp of a lane quadrant
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int quad = warp & 3, half = warp >> 2;
+  const int row = 32 * quad + lane;  // this thread's TMEM lane: a step t or a state row
   const int h0 = blockIdx.x * kTHeads, b = blockIdx.y;
   const int H = p.nheads;
   const int64_t L = p.seqlen;
   const int nchunks = (int)((L + kTQ - 1) / kTQ);
 
-  float* f_delta = reinterpret_cast<float*>(sm + Ly::kOffSteps);  // [2][Q]
-  float* f_cum = f_delta + kTHeads * kTQ;                          // [2][Q]
-  float* f_w = f_cum + kTHeads * kTQ;                              // [2][Q]
-  float* f_e = f_w + kTHeads * kTQ;                                // [2][Q]
-  float* f_wsum = f_e + kTHeads * kTQ;                             // [2][4]
-  float* f_decay = f_wsum + kTHeads * 4;                           // [2]
+  float* steps = reinterpret_cast<float*>(sm + Ly::kOffSteps);
+  float* f_wsum = steps + 2 * Ly::kStepBuf;  // [head][quadrant]
+  float* f_decay = f_wsum + kTHeads * 4;     // [buffer][head]
+  // step arrays of buffer i: Delta, cum, w, E, each [head][Q]
+  auto sdelta = [&](int i) { return steps + i * Ly::kStepBuf; };
+  auto scum = [&](int i) { return steps + i * Ly::kStepBuf + kTHeads * kTQ; };
+  auto sw = [&](int i) { return steps + i * Ly::kStepBuf + 2 * kTHeads * kTQ; };
+  auto se = [&](int i) { return steps + i * Ly::kStepBuf + 3 * kTHeads * kTQ; };
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Ly::kOffBar);
   uint64_t* bar_bc = bars + 0;
-  uint64_t* bar_x = bars + 1;  // [2]
+  uint64_t* bar_x0 = bars + 1;
+  uint64_t* bar_x1 = bars + 2;
   uint64_t* bar_s = bars + 3;
-  uint64_t* bar_m1 = bars + 4;
-  uint64_t* bar_m2 = bars + 5;
-  (void)bar_m2;
+  uint64_t* bar_m = bars + 4;
   uint32_t* slot = reinterpret_cast<uint32_t*>(sm + Ly::kOffSlot);
   unsigned char* const xbuf0 = sm + Ly::kOffX0;
   unsigned char* const xbuf1 = sm + Ly::kOffX1;
   unsigned char* sB = sm + Ly::kOffB;
   unsigned char* sC = sm + Ly::kOffC;
-  unsigned char* sG = sm + Ly::kOffG;
   unsigned char* sHb = sm + Ly::kOffHb;
 
-  float Ah[kTHeads], bias[kTHeads], Dh[kTHeads];
-#pragma unroll
-  for (int i = 0; i < kTHeads; ++i) {
-    Ah[i] = p.A[h0 + i];
-    bias[i] = p.dt_bias ? p.dt_bias[h0 + i] : 0.f;
-    Dh[i] = p.D ? p.D[h0 + i] : 0.f;
-  }
+  // per-head constants of the head this thread computes steps for (s_hh) and
+  // writes outputs for (half)
+  const int s_hh = tid >> 7;
+  const float A_s = p.A[h0 + s_hh];
+  const float bias_s = p.dt_bias ? p.dt_bias[h0 + s_hh] : 0.f;
+  const float D_o = p.D ? p.D[h0 + half] : 0.f;
 
   if (tid == 0) {
     for (int i = 0; i < Ly::kNumBars; ++i) mbar_init(&bars[i], 1);
@@ -147,16 +166,17 @@ __global__ void __launch_bounds__(kTThreads, 1)
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tm = *slot;
-  const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+  const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
   const uint32_t tH = tm + lane_base + kColH, tS = tm + lane_base + kColS;
   const uint32_t tYd = tm + lane_base + kColYd, tYo = tm + lane_base + kColYo;
 
-  // ---- initial state: thread = TMEM lane = state row (head h0 + tid / 64, p)
+  // ---- initial state: TMEM lane = state row (head h0 + row / 64, p); the
+  //      two warps of a quadrant write one half of the N columns each
   {
-    const float* src = p.h0 ? p.h0 + (((size_t)b * H + h0 + tid / kTP) * kTP + tid % kTP) * N
+    const float* src = p.h0 ? p.h0 + (((size_t)b * H + h0 + row / kTP) * kTP + row % kTP) * N
                             : nullptr;
 #pragma unroll
-    for (int c0 = 0; c0 < N; c0 += 32) {
+    for (int c0 = half * kHalfN; c0 < (half + 1) * kHalfN; c0 += 32) {
       float v[32];
 #pragma unroll
       for (int j = 0; j < 32; j += 4) {
@@ -180,86 +200,71 @@ __global__ void __launch_bounds__(kTThreads, 1)
     }
   };
   auto issue_x = [&](int c, int i) {
-    uint64_t* bar = i ? &bar_x[1] : &bar_x[0];
+    uint64_t* bar = i ? bar_x1 : bar_x0;
     unsigned char* dst = i ? xbuf1 : xbuf0;
     mbar_arrive_expect_tx(bar, (uint32_t)(kTHeads * Ly::kBlk) + ((stall && c == 0) ? 16u : 0u));
 #pragma unroll
     for (int hh = 0; hh < kTHeads; ++hh)
       tc::tma_load_4d(dst + hh * Ly::kBlk, &maps.x, bar, 0, h0 + hh, c * kTQ, b);
   };
-  // Each barrier completes once per chunk (an x buffer every other chunk), in
-  // order, so the phase to wait for follows from the chunk index; on the
+  // Phases armed (thread 0) and waited (every thread) per barrier; on the
   // error path thread 0 waits (bounded) for the completions still owed.
-  // armed_*: phases armed so far by thread 0 (B/C, x0, x1, S, MMA1, MMA2).
-  int armed_bc = 0, armed_x0 = 0, armed_x1 = 0, armed_s = 0, armed_m1 = 0, armed_m2 = 0;
-  // phases waited (every thread)
-  int waited_bc = 0, waited_x0 = 0, waited_x1 = 0, waited_s = 0, waited_m1 = 0, waited_m2 = 0;
-  if (tid == 0 && nchunks > 0) {
-    issue_bc(0);
-    issue_x(0, 0);
-    armed_bc = 1;
-    armed_x0 = 1;
-  }
-  // raw dt of this thread's step in chunk c, both heads (one 4-byte load:
-  // h0 and H are even)
-  auto load_dt = [&](int c, float (&r)[kTHeads]) {
-    const int64_t t = (int64_t)c * kTQ + tid;
-    const uint32_t w = t < L ? *reinterpret_cast<const uint32_t*>(p.dt + ((size_t)b * L + t) * H + h0)
-                             : 0u;
-    r[0] = bf16_lo(w);
-    r[1] = bf16_hi(w);
+  int armed_bc = 0, armed_x0 = 0, armed_x1 = 0, armed_s = 0, armed_m = 0;
+  int waited_bc = 0, waited_x0 = 0, waited_x1 = 0, waited_s = 0, waited_m = 0;
+
+  // Step quantities of chunk c into buffer c & 1: thread = (head tid / 128,
+  // step tid % 128); Delta, the in-chunk cumulative sum of Delta A (a scan
+  // over the four warps of the head), w_s, E_s = e^{cum_{end of s's 32-step
+  // block} - cum_s} Delta_s and e^{cum_end}. Every thread calls it.
+  const int s_t = tid & 127, s_q = (tid >> 5) & 3;
+  auto load_dt = [&](int c) {
+    const int64_t t = (int64_t)c * kTQ + s_t;
+    return t < L ? bf16_to_f32(p.dt[((size_t)b * L + t) * H + h0 + s_hh]) : 0.f;
   };
-  float dt_next[kTHeads];
-  if (nchunks > 0) load_dt(0, dt_next);
+  auto compute_steps = [&](int c, float raw) {
+    const int i = c & 1;
+    float d = 0.f;
+    if ((int64_t)c * kTQ + s_t < L) {
+      const float v = raw + bias_s;
+      // softplus(v) = ln 2 * log2(1 + 2^(v log2 e)), v above the cut
+      d = p.softplus ? (v > kSoftplusCut ? v : kLn2 * lg2_approx(1.f + ex2_approx(v * kLog2e))) : v;
+    }
+    float a = d * A_s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float u = __shfl_up_sync(0xffffffffu, a, o);
+      if (lane >= o) a += u;
+    }
+    if (lane == 31) f_wsum[s_hh * 4 + s_q] = a;
+    __syncthreads();
+    for (int w = 0; w < s_q; ++w) a += f_wsum[s_hh * 4 + w];
+    sdelta(i)[s_hh * kTQ + s_t] = d;
+    scum(i)[s_hh * kTQ + s_t] = a;
+    __syncthreads();
+    const float cend = scum(i)[s_hh * kTQ + kTQ - 1];
+    sw(i)[s_hh * kTQ + s_t] = ex2_approx((cend - a) * kLog2e) * d;
+    se(i)[s_hh * kTQ + s_t] = ex2_approx((scum(i)[s_hh * kTQ + (s_t | 31)] - a) * kLog2e) * d;
+    if (s_t == 0) f_decay[i * kTHeads + s_hh] = ex2_approx(cend * kLog2e);
+  };
+
+  if (nchunks > 0) {
+    if (tid == 0) {
+      issue_bc(0);
+      issue_x(0, 0);
+      armed_bc = 1;
+      armed_x0 = 1;
+    }
+    compute_steps(0, load_dt(0));
+  }
+  __syncthreads();
 
   bool ok = true;
   int c = 0;
   for (; c < nchunks; ++c) {
-    const int xi = c & 1;
+    const int xi = c & 1, sb = c & 1;
     const int64_t t0 = (int64_t)c * kTQ;
-    // ---- 1. steps of the chunk: Delta, the in-chunk cumulative sum of
-    //      Delta A (block scan over the 128 threads), the weights w
-    float dtr[kTHeads];
-#pragma unroll
-    for (int hh = 0; hh < kTHeads; ++hh) dtr[hh] = dt_next[hh];
-    if (c + 1 < nchunks) load_dt(c + 1, dt_next);
-    float dl[kTHeads], cum[kTHeads];
-#pragma unroll
-    for (int hh = 0; hh < kTHeads; ++hh) {
-      float d = 0.f;
-      if (t0 + tid < L) {
-        const float v = dtr[hh] + bias[hh];
-        d = p.softplus ? (v > kSoftplusCut ? v : log1pf(expf(v))) : v;
-      }
-      dl[hh] = d;
-      float a = d * Ah[hh];
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const float u = __shfl_up_sync(0xffffffffu, a, o);
-        if (lane >= o) a += u;
-      }
-      cum[hh] = a;
-      if (lane == 31) f_wsum[hh * 4 + warp] = a;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int hh = 0; hh < kTHeads; ++hh) {
-      float off = 0.f;
-      for (int w = 0; w < warp; ++w) off += f_wsum[hh * 4 + w];
-      cum[hh] += off;
-      f_delta[hh * kTQ + tid] = dl[hh];
-      f_cum[hh * kTQ + tid] = cum[hh];
-    }
-    __syncthreads();
-#pragma unroll
-    for (int hh = 0; hh < kTHeads; ++hh) {
-      const float cend = f_cum[hh * kTQ + kTQ - 1];
-      f_w[hh * kTQ + tid] = expf(cend - cum[hh]) * dl[hh];
-      // factor of column s of G below the diagonal 32 x 32 blocks (<= Delta_s)
-      f_e[hh * kTQ + tid] = expf(f_cum[hh * kTQ + (tid | 31)] - cum[hh]) * dl[hh];
-      if (tid == 0) f_decay[hh] = expf(cend);
-    }
-    // ---- 2. S = C B^T once this chunk's B and C have landed
+    const float dt_next = c + 1 < nchunks ? load_dt(c + 1) : 0.f;
+    // ---- S = C B^T once this chunk's B and C have landed
     ok = cta_wait(bar_bc, (uint32_t)(c & 1), p.wait_limit_ns);
     if (!ok) break;
     ++waited_bc;
@@ -275,107 +280,108 @@ __global__ void __launch_bounds__(kTThreads, 1)
       tc::commit(bar_s);
       ++armed_s;
     }
-    // ---- 3. this chunk's x: w-scaled copy into the other buffer (row s =
-    //      thread); the state: bf16 copy for the readout, then scaled by
-    //      e^{cum_end} in place for the update (row hp = thread)
-    ok = cta_wait(xi ? &bar_x[1] : &bar_x[0], (uint32_t)((c >> 1) & 1), p.wait_limit_ns);
+    // ---- this chunk's x: its w-scaled copy into the other buffer (thread =
+    //      (head, step)); the state: bf16 copy for the readout, then scaled
+    //      by e^{cum_end} for the update (thread = state row, half the columns)
+    ok = cta_wait(xi ? bar_x1 : bar_x0, (uint32_t)((c >> 1) & 1), p.wait_limit_ns);
     if (!ok) break;
     if (xi) ++waited_x1; else ++waited_x0;
     unsigned char* const xcur = xi ? xbuf1 : xbuf0;  // x of this chunk
     unsigned char* const xoth = xi ? xbuf0 : xbuf1;  // its w-scaled copy
     {
-      const unsigned char* src = xcur;
-      unsigned char* dst = xoth;
+      const float w = sw(sb)[s_hh * kTQ + s_t];
 #pragma unroll
-      for (int hh = 0; hh < kTHeads; ++hh) {
-        const float w = f_w[hh * kTQ + tid];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const uint32_t o = hh * Ly::kBlk + tid * 128 + ((j + tid) & 7) * 16;
-          const uint4 q = *reinterpret_cast<const uint4*>(src + o);
-          const float v[8] = {bf16_lo(q.x) * w, bf16_hi(q.x) * w, bf16_lo(q.y) * w,
-                              bf16_hi(q.y) * w, bf16_lo(q.z) * w, bf16_hi(q.z) * w,
-                              bf16_lo(q.w) * w, bf16_hi(q.w) * w};
-          *reinterpret_cast<uint4*>(dst + o) = pack8(v);
-        }
+      for (int j = 0; j < 8; ++j) {
+        // a rotated chunk order keeps the 16-byte accesses of a warp on
+        // distinct banks
+        const uint32_t o = s_hh * Ly::kBlk + s_t * 128 + ((j + s_t) & 7) * 16;
+        const uint4 q = *reinterpret_cast<const uint4*>(xcur + o);
+        const float v[8] = {bf16_lo(q.x) * w, bf16_hi(q.x) * w, bf16_lo(q.y) * w,
+                            bf16_hi(q.y) * w, bf16_lo(q.z) * w, bf16_hi(q.z) * w,
+                            bf16_lo(q.w) * w, bf16_hi(q.w) * w};
+        *reinterpret_cast<uint4*>(xoth + o) = pack8(v);
       }
-      const float decay = f_decay[tid / kTP];
+      const float decay = f_decay[sb * kTHeads + row / kTP];
 #pragma unroll
-      for (int c0 = 0; c0 < N; c0 += 64) {
-        float v[32], u[32];
+      for (int c0 = half * kHalfN; c0 < (half + 1) * kHalfN; c0 += 32) {
+        float v[32];
         tc::ld32(tH + c0, v);
-        tc::ld32(tH + c0 + 32, u);
         tc::wait_ld();
 #pragma unroll
         for (int j = 0; j < 32; j += 8) {
-          *reinterpret_cast<uint4*>(sHb + (c0 / 64) * Ly::kBlk + tc::sw128(tid, j)) = pack8(v + j);
-          *reinterpret_cast<uint4*>(sHb + (c0 / 64) * Ly::kBlk + tc::sw128(tid, 32 + j)) =
-              pack8(u + j);
+          const int col = c0 + j;
+          *reinterpret_cast<uint4*>(sHb + (col / 64) * Ly::kBlk + tc::sw128(row, col % 64)) =
+              pack8(v + j);
         }
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          v[j] *= decay;
-          u[j] *= decay;
-        }
+        for (int j = 0; j < 32; ++j) v[j] *= decay;
         tc::st32(tH + c0, v);
-        tc::st32(tH + c0 + 32, u);
       }
       tc::wait_st();
     }
     tc::fence_proxy_async_smem();
     tc::fence_before_sync();
-    // ---- 4. G of head 0 from S (row t = thread)
+    // ---- G of both heads from S (thread = step t, half the columns), written
+    //      over S as bf16 pairs: G of head hh at columns kColS + 64 hh + s / 2.
+    //      32-column blocks j below the diagonal block: e^{cum_t - cum_s}
+    //      Delta_s = F_j E_s with F_j = e^{cum_t - cum_{32 j + 31}} (both
+    //      factors <= 1, one exp per block); the diagonal block one exp per
+    //      entry; above it zero.
     ok = cta_wait(bar_s, (uint32_t)(c & 1), p.wait_limit_ns);
     if (!ok) break;
     ++waited_s;
     tc::fence_after_sync();
-    // G row t (= thread) of head hh from S, in 32-column blocks j: below the
-    // diagonal block (32 j + 31 < t's block) e^{cum_t - cum_s} Delta_s =
-    // F_j E_s with F_j = e^{cum_t - cum_{32 j + 31}} (both factors <= 1, one
-    // exp per block); the diagonal block takes one exp per entry; above it G
-    // is zero.
-    auto make_g = [&](int hh) {
-      const float ct = f_cum[hh * kTQ + tid];
-      const int tb = tid >> 5;  // this row's diagonal block
+    {
+      float v[2][32];
+      tc::ld32(tS + 64 * half, v[0]);
+      tc::ld32(tS + 64 * half + 32, v[1]);
+      tc::wait_ld();
+      uint32_t gp[kTHeads][32];
+      const int t = row, tb = t >> 5;
 #pragma unroll
-      for (int c0 = 0; c0 < kTQ; c0 += 64) {
-        float v[2][32];
-        tc::ld32(tS + c0, v[0]);
-        tc::ld32(tS + c0 + 32, v[1]);
-        tc::wait_ld();
+      for (int hh = 0; hh < kTHeads; ++hh) {
+        const float* cum = scum(sb) + hh * kTQ;
+        const float* del = sdelta(sb) + hh * kTQ;
+        const float* E = se(sb) + hh * kTQ;
+        const float ct = cum[t];
 #pragma unroll
-        for (int hb = 0; hb < 2; ++hb) {
-          const int j = (c0 >> 5) + hb;  // column block
-          const int s0 = 32 * j;
+        for (int jj = 0; jj < 2; ++jj) {
+          const int j = 2 * half + jj, s0 = 32 * j;
           float g[32];
           if (j < tb) {
-            const float F = expf(ct - f_cum[hh * kTQ + s0 + 31]);
+            const float F = ex2_approx((ct - cum[s0 + 31]) * kLog2e);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) g[e] = v[hb][e] * F * f_e[hh * kTQ + s0 + e];
+            for (int e = 0; e < 32; ++e) g[e] = v[jj][e] * F * E[s0 + e];
           } else if (j == tb) {
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
               const int sidx = s0 + e;
-              g[e] = sidx <= tid ? v[hb][e] * ex2_approx((ct - f_cum[hh * kTQ + sidx]) * kLog2e) *
-                                       f_delta[hh * kTQ + sidx]
-                                 : 0.f;
+              g[e] = sidx <= t ? v[jj][e] * ex2_approx((ct - cum[sidx]) * kLog2e) * del[sidx] : 0.f;
             }
           } else {
 #pragma unroll
             for (int e = 0; e < 32; ++e) g[e] = 0.f;
           }
 #pragma unroll
-          for (int e = 0; e < 32; e += 8)
-            *reinterpret_cast<uint4*>(sG + (s0 / 64) * Ly::kBlk + tc::sw128(tid, (s0 + e) % 64)) =
-                pack8(g + e);
+          for (int e = 0; e < 32; e += 2) gp[hh][jj * 16 + e / 2] = pack_bf16x2(g[e], g[e + 1]);
         }
       }
-    };
-    make_g(0);
-    tc::fence_proxy_async_smem();
+      // every warp has read its columns of S before any is overwritten
+      tc::fence_before_sync();
+      __syncthreads();
+      tc::fence_after_sync();
+#pragma unroll
+      for (int hh = 0; hh < kTHeads; ++hh) {
+        float f[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(gp[hh][e]);
+        tc::st32(tS + 64 * hh + 32 * half, f);
+      }
+      tc::wait_st();
+    }
     tc::fence_before_sync();
     __syncthreads();
-    // ---- 5. the readout C H^T, the state update, G X of head 0
+    // ---- the chunk's products: C H^T, the state update, G X of both heads
     if (tid == 0) {
       tc::fence_after_sync();
       {  // Yo (t x 2P) = C (t x N) . Hb^T, both K-major over n
@@ -396,23 +402,26 @@ __global__ void __launch_bounds__(kTThreads, 1)
                        tc::sdesc(smem_u32(sB) + o, Ly::kBlk, 1024), id, 1u);
         }
       }
-      {  // Yd[:, head 0] (t x P) = G (t x s, K-major) . x_0 (s x P, MN-major)
+      {  // Yd[:, head hh] (t x P) = G_hh (TMEM, t x s) . x_hh (s x P, MN-major)
         constexpr uint32_t id = tc::idesc_bf16(128, kTP, 0, 1);
 #pragma unroll
-        for (int ks = 0; ks < kTQ / 16; ++ks) {
-          const uint32_t oa = (ks / 4) * Ly::kBlk + (ks % 4) * 32;
-          tc::mma_bf16(tm + kColYd, tc::sdesc(smem_u32(sG) + oa, 16, 1024),
-                       tc::sdesc(smem_u32(xcur) + ks * 2048, Ly::kBlk, 1024), id, ks > 0);
-        }
+        for (int hh = 0; hh < kTHeads; ++hh)
+#pragma unroll
+          for (int ks = 0; ks < kTQ / 16; ++ks)
+            mma_bf16_tmem_a(tm + kColYd + kTP * hh, tm + kColS + 64 * hh + ks * 8,
+                            tc::sdesc(smem_u32(xcur) + hh * Ly::kBlk + ks * 2048, Ly::kBlk, 1024),
+                            id, ks > 0);
       }
-      tc::commit(bar_m1);
-      ++armed_m1;
+      tc::commit(bar_m);
+      ++armed_m;
     }
-    // ---- 6. the buffers of B, C and the scaled x are free: next chunk's
-    //      loads; G of head 1 (G's buffer is free too), then its G X
-    ok = cta_wait(bar_m1, (uint32_t)(c & 1), p.wait_limit_ns);
+    // ---- the next chunk's step quantities while the products run
+    if (c + 1 < nchunks) compute_steps(c + 1, dt_next);
+    // ---- the buffers of B, C and the scaled x are free: next chunk's loads;
+    //      y_t = Yd + e^{cum_t} Yo + D x_t (thread = (head, step t))
+    ok = cta_wait(bar_m, (uint32_t)(c & 1), p.wait_limit_ns);
     if (!ok) break;
-    ++waited_m1;
+    ++waited_m;
     tc::fence_after_sync();
     if (tid == 0 && c + 1 < nchunks) {
       issue_bc(c + 1);
@@ -420,52 +429,27 @@ __global__ void __launch_bounds__(kTThreads, 1)
       ++armed_bc;
       if (xi) ++armed_x0; else ++armed_x1;
     }
-    make_g(1);
-    tc::fence_proxy_async_smem();
-    tc::fence_before_sync();
-    __syncthreads();
-    if (tid == 0) {
-      tc::fence_after_sync();
-      constexpr uint32_t id = tc::idesc_bf16(128, kTP, 0, 1);
-#pragma unroll
-      for (int ks = 0; ks < kTQ / 16; ++ks) {
-        const uint32_t oa = (ks / 4) * Ly::kBlk + (ks % 4) * 32;
-        tc::mma_bf16(tm + kColYd + kTP, tc::sdesc(smem_u32(sG) + oa, 16, 1024),
-                     tc::sdesc(smem_u32(xcur) + Ly::kBlk + ks * 2048, Ly::kBlk, 1024), id,
-                     ks > 0);
-      }
-      tc::commit(bar_m2);
-      ++armed_m2;
-    }
-    // ---- 7. y_t = Yd + e^{cum_t} Yo + D x_t (row t = thread)
-    ok = cta_wait(bar_m2, (uint32_t)(c & 1), p.wait_limit_ns);
-    if (!ok) break;
-    ++waited_m2;
-    tc::fence_after_sync();
     {
-      const int64_t t = t0 + tid;
+      const int t = row, hh = half;  // TMEM lane t; warps 4-7 take head 1
+      const int64_t tg = t0 + t;
+      const float ec = ex2_approx(scum(sb)[hh * kTQ + t] * kLog2e);
+      uint16_t* yrow = p.y + (((size_t)b * L + (tg < L ? tg : 0)) * H + h0 + hh) * kTP;
 #pragma unroll
-      for (int hh = 0; hh < kTHeads; ++hh) {
-        const float ec = expf(f_cum[hh * kTQ + tid]);
-        uint16_t* yrow = p.y + (((size_t)b * L + (t < L ? t : 0)) * H + h0 + hh) * kTP;
+      for (int c0 = 0; c0 < kTP; c0 += 32) {
+        float yd[32], yo[32];
+        tc::ld32(tYd + hh * kTP + c0, yd);
+        tc::ld32(tYo + hh * kTP + c0, yo);
+        tc::wait_ld();
 #pragma unroll
-        for (int c0 = 0; c0 < kTP; c0 += 32) {
-          float yd[32], yo[32];
-          tc::ld32(tYd + hh * kTP + c0, yd);
-          tc::ld32(tYo + hh * kTP + c0, yo);
-          tc::wait_ld();
+        for (int j = 0; j < 32; j += 8) {
+          const int pc = c0 + j;
+          const uint4 q = *reinterpret_cast<const uint4*>(xcur + hh * Ly::kBlk + tc::sw128(t, pc));
+          const float xv[8] = {bf16_lo(q.x), bf16_hi(q.x), bf16_lo(q.y), bf16_hi(q.y),
+                               bf16_lo(q.z), bf16_hi(q.z), bf16_lo(q.w), bf16_hi(q.w)};
+          float o[8];
 #pragma unroll
-          for (int j = 0; j < 32; j += 8) {
-            const int pc = c0 + j;
-            const uint4 q = *reinterpret_cast<const uint4*>(xcur + hh * Ly::kBlk +
-                                                            tc::sw128(tid, pc));
-            const float xv[8] = {bf16_lo(q.x), bf16_hi(q.x), bf16_lo(q.y), bf16_hi(q.y),
-                                 bf16_lo(q.z), bf16_hi(q.z), bf16_lo(q.w), bf16_hi(q.w)};
-            float o[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) o[e] = fmaf(Dh[hh], xv[e], fmaf(ec, yo[j + e], yd[j + e]));
-            if (t < L) *reinterpret_cast<uint4*>(yrow + pc) = pack8(o);
-          }
+          for (int e = 0; e < 8; ++e) o[e] = fmaf(D_o, xv[e], fmaf(ec, yo[j + e], yd[j + e]));
+          if (tg < L) *reinterpret_cast<uint4*>(yrow + pc) = pack8(o);
         }
       }
     }
@@ -476,9 +460,9 @@ __global__ void __launch_bounds__(kTThreads, 1)
   if (ok) {
     if (p.h_last) {
       tc::fence_after_sync();
-      float* dst = p.h_last + (((size_t)b * H + h0 + tid / kTP) * kTP + tid % kTP) * N;
+      float* dst = p.h_last + (((size_t)b * H + h0 + row / kTP) * kTP + row % kTP) * N;
 #pragma unroll
-      for (int c0 = 0; c0 < N; c0 += 32) {
+      for (int c0 = half * kHalfN; c0 < (half + 1) * kHalfN; c0 += 32) {
         float v[32];
         tc::ld32(tH + c0, v);
         tc::wait_ld();
@@ -494,11 +478,10 @@ __global__ void __launch_bounds__(kTThreads, 1)
       for (int k = done; k < armed; ++k) (void)mbar_wait_bounded(bar, (uint32_t)(k & 1), 1000000ull);
     };
     drain(bar_bc, waited_bc, armed_bc);
-    drain(&bar_x[0], waited_x0, armed_x0);
-    drain(&bar_x[1], waited_x1, armed_x1);
+    drain(bar_x0, waited_x0, armed_x0);
+    drain(bar_x1, waited_x1, armed_x1);
     drain(bar_s, waited_s, armed_s);
-    drain(bar_m1, waited_m1, armed_m1);
-    drain(bar_m2, waited_m2, armed_m2);
+    drain(bar_m, waited_m, armed_m);
     atomicExch(&g_ssd_status, 1);
   }
   tc::fence_before_sync();
