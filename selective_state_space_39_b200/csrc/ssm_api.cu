@@ -743,7 +743,8 @@ int ssm_ssd_scan_fwd(int64_t batch, int64_t seqlen, int64_t nheads, int64_t head
     const cuuint32_t bb[3] = {64, 128, 1};
     if (!encode_sw128_bf16(&maps.x, x, 4, xd, xs, xb) ||
         !encode_sw128_bf16(&maps.B, B, 3, bd, bs, bb) ||
-        !encode_sw128_bf16(&maps.C, C, 3, bd, bs, bb))
+        !encode_sw128_bf16(&maps.C, C, 3, bd, bs, bb) ||
+        !encode_sw128_bf16(&maps.y, y, 4, xd, xs, xb))
       return SSM_ERR_CUDA;
     return cuda_status(launch_ssd_tc(p, maps, static_cast<cudaStream_t>(stream)),
                        "ssd scan launch (tcgen05)");

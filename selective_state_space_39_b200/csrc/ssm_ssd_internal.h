@@ -35,7 +35,7 @@ struct SsdParams {
 // seqlen, batch) with a 64 x 1 x 128 x 1 box; B and C as (dstate, seqlen,
 // batch) with a 64 x 128 x 1 box.
 struct alignas(64) SsdTcMaps {
-  CUtensorMap x, B, C;
+  CUtensorMap x, B, C, y;  // y: the same geometry as x
 };
 
 bool ssd_dstate_supported(int dstate);

@@ -14,9 +14,13 @@
 //   y_t     = sum_s G[t][s] x_s + e^{cum_t} C_t H + D x_t
 //   H      <- e^{cum_end} H + sum_s w_s x_s B_s^T,   w_s = e^{cum_end - cum_s} Delta_s
 //
-// Design (B200). One CTA of eight warps per batch row and pair of heads walks
-// the chunks in order; warps w and w + 4 share TMEM lanes 32 (w % 4) .. and
-// split each row's columns (or the two heads) between them. Every product
+// Design (B200). One CTA per batch row and pair of heads walks the chunks in
+// order: one warp issues the TMA copies and the MMAs, eight compute warps do
+// the rest (warps w and w + 4 share TMEM lanes 32 (w % 4) .. and split each
+// row's columns, or the two heads, between them); they meet at mbarriers,
+// so the MMAs of a chunk run while the compute warps prepare the next
+// chunk's step quantities, and the next chunk's S while they write this
+// chunk's outputs. Every product
 // is a tcgen05 MMA of M = 128 with fp32 accumulators in TMEM:
 //   S = C B^T (t x s, K = N; both operands from shared memory),
 //   the readout C H^T (t x (2 heads x p), K = N; H as a bf16 copy in shared
@@ -31,7 +35,8 @@
 // multicast); the next chunk's copies start as soon as the chunk's MMAs have
 // released their buffers (two x buffers alternate between the raw x and the
 // w-scaled x), and the next chunk's step quantities are computed while the
-// chunk's MMAs run. Steps past the sequence end read zeros and take Delta =
+// chunk's MMAs run (its tiles are prefetched into L2 a chunk ahead). Steps
+// past the sequence end read zeros and take Delta =
 // 0, so they change nothing. Every wait is bounded; a wait that runs out
 // stops the CTA (after its copies and MMAs in flight land, bounded too),
 // frees its TMEM and sets the flag that ssm_ssd_scan_status reports.
@@ -55,7 +60,8 @@ namespace {
 constexpr int kTQ = 128;        // steps per chunk
 constexpr int kTP = 64;         // head width
 constexpr int kTHeads = 2;      // heads per CTA
-constexpr int kTThreads = 256;  // eight warps, two per TMEM lane quadrant
+constexpr int kTWork = 256;     // eight compute warps, two per TMEM lane quadrant
+constexpr int kTThreads = kTWork + 32;  // and one warp that issues copies and MMAs
 constexpr uint32_t kTmemCols = 512;
 // TMEM columns: the state, S (then G of both heads, bf16 pairs), G X, C H^T
 constexpr uint32_t kColH = 0, kColS = 128, kColYd = 256, kColYo = 384;
@@ -69,29 +75,26 @@ struct TcLayout {
   static constexpr int kXBuf = kTHeads * kBlk;     // [head][t][64 p]
   static constexpr int kBC = kNB * kBlk;           // [n block][t][64 n]
   static constexpr int kHb = kNB * kBlk;           // [n block][2 x 64 rows hp][64 n]
+  // two buffers of raw x (a chunk's y is staged over its x), the w-scaled x
   static constexpr int kOffX0 = 0;
   static constexpr int kOffX1 = kXBuf;
-  static constexpr int kOffB = 2 * kXBuf;
+  static constexpr int kOffXs = 2 * kXBuf;
+  static constexpr int kOffB = 3 * kXBuf;
   static constexpr int kOffC = kOffB + kBC;
   static constexpr int kOffHb = kOffC + kBC;
   static constexpr int kOffSteps = kOffHb + kHb;
   // step quantities, two buffers (this chunk, the next): per head Delta[Q],
   // cum[Q], w[Q], E[Q]
   static constexpr int kStepBuf = kTHeads * 4 * kTQ;
-  static constexpr int kStepFloats = 2 * kStepBuf + kTHeads * 4 + 2 * kTHeads;
+  static constexpr int kStepFloats = 2 * kStepBuf + kTHeads * 4 + 2 * kTHeads + 2;
   static constexpr int kOffBar = round_up(kOffSteps + kStepFloats * 4, 8);
-  static constexpr int kNumBars = 5;  // B/C, x (two buffers), S, the chunk's MMAs
+  // B/C, x (two buffers), S, readout + update, G X, operands, x buffer free
+  static constexpr int kNumBars = 8;
   static constexpr int kOffSlot = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffSlot + 16 + 1024;  // + room to align the base to 1024
   static_assert(N == 64 || N == 128, "state width 64 or 128");
+  static_assert(kBytes <= 227 * 1024, "shared memory of one CTA");
 };
-
-// Wait for phase `parity` of `bar`, every thread of the CTA; false everywhere
-// if any thread's wait ran out.
-__device__ __forceinline__ bool cta_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
-  const bool ok = mbar_wait_bounded(bar, parity, limit_ns);
-  return __syncthreads_and(ok) != 0;
-}
 
 // Eight fp32 values packed as eight bf16 (one 16-byte chunk).
 __device__ __forceinline__ uint4 pack8(const float* v) {
@@ -110,17 +113,42 @@ __device__ __forceinline__ void mma_bf16_tmem_a(uint32_t d_tmem, uint32_t a_tmem
       : "memory");
 }
 
+// Named barrier of the compute warps (id 1, 256 threads) with an AND vote:
+// every compute thread gets the same answer, so all leave a loop together.
+__device__ __forceinline__ bool work_vote(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred q, p;\n\tsetp.ne.u32 q, %1, 0;\n\t"
+      "barrier.cta.red.and.pred p, 1, %2, q;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "n"(kTWork)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void work_sync() {
+  asm volatile("barrier.cta.sync 1, %0;" ::"n"(kTWork) : "memory");
+}
+// A value the compiler cannot treat as loop-invariant: the issuing warp
+// derives its descriptors from it each chunk instead of keeping dozens live.
+__device__ __forceinline__ uint32_t opaque(uint32_t v) {
+  asm volatile("mov.b32 %0, %0;" : "+r"(v));
+  return v;
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
 template <int N>
 __global__ void __launch_bounds__(kTThreads, 1)
     ssd_tc_kernel(const SsdParams p, const __grid_constant__ SsdTcMaps maps) {
   using Ly = TcLayout<N>;
   constexpr int kNB = Ly::kNB;
-  constexpr int kHalfN = N / 2;  // state columns per warp of a lane quadrant
+  constexpr int kHalfN = N / 2;  // state columns per compute warp of a lane quadrant
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int quad = warp & 3, half = warp >> 2;
-  const int row = 32 * quad + lane;  // this thread's TMEM lane: a step t or a state row
+  const bool issuer = warp == kTWork / 32;  // the ninth warp issues copies and MMAs
+  const int quad = warp & 3, half = (warp >> 2) & 1;
+  const int row = 32 * quad + lane;  // a compute thread's TMEM lane: a step t or a state row
   const int h0 = blockIdx.x * kTHeads, b = blockIdx.y;
   const int H = p.nheads;
   const int64_t L = p.seqlen;
@@ -129,179 +157,236 @@ __global__ void __launch_bounds__(kTThreads, 1)
   float* steps = reinterpret_cast<float*>(sm + Ly::kOffSteps);
   float* f_wsum = steps + 2 * Ly::kStepBuf;  // [head][quadrant]
   float* f_decay = f_wsum + kTHeads * 4;     // [buffer][head]
-  // step arrays of buffer i: Delta, cum, w, E, each [head][Q]
+  // step arrays of buffer i, each [head][Q]: Delta, cum (in units of log2,
+  // i.e. log2 e times the sum of Delta A), w, E
   auto sdelta = [&](int i) { return steps + i * Ly::kStepBuf; };
   auto scum = [&](int i) { return steps + i * Ly::kStepBuf + kTHeads * kTQ; };
   auto sw = [&](int i) { return steps + i * Ly::kStepBuf + 2 * kTHeads * kTQ; };
   auto se = [&](int i) { return steps + i * Ly::kStepBuf + 3 * kTHeads * kTQ; };
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Ly::kOffBar);
-  uint64_t* bar_bc = bars + 0;
-  uint64_t* bar_x0 = bars + 1;
+  uint64_t* bar_bc = bars + 0;     // B and C of a chunk landed (TMA)
+  uint64_t* bar_x0 = bars + 1;     // x landed in buffer 0 / 1 (TMA)
   uint64_t* bar_x1 = bars + 2;
-  uint64_t* bar_s = bars + 3;
-  uint64_t* bar_m = bars + 4;
+  uint64_t* bar_s = bars + 3;      // S = C B^T done (MMA commit)
+  uint64_t* bar_h = bars + 4;      // readout C H^T and state update done (MMA commit)
+  uint64_t* bar_m = bars + 5;      // G X done: every product of the chunk (MMA commit)
+  uint64_t* bar_work = bars + 6;   // the compute warps' operands are written (256 arrivals)
+  uint64_t* bar_xfree = bars + 7;  // a chunk's y has left its x buffer (bulk store read)
   uint32_t* slot = reinterpret_cast<uint32_t*>(sm + Ly::kOffSlot);
   unsigned char* const xbuf0 = sm + Ly::kOffX0;
   unsigned char* const xbuf1 = sm + Ly::kOffX1;
+  unsigned char* const sXs = sm + Ly::kOffXs;
   unsigned char* sB = sm + Ly::kOffB;
   unsigned char* sC = sm + Ly::kOffC;
   unsigned char* sHb = sm + Ly::kOffHb;
-
-  // per-head constants of the head this thread computes steps for (s_hh) and
-  // writes outputs for (half)
-  const int s_hh = tid >> 7;
-  const float A_s = p.A[h0 + s_hh];
-  const float bias_s = p.dt_bias ? p.dt_bias[h0 + s_hh] : 0.f;
-  const float D_o = p.D ? p.D[h0 + half] : 0.f;
+  int* f_fail = reinterpret_cast<int*>(f_decay + 2 * kTHeads);
 
   if (tid == 0) {
-    for (int i = 0; i < Ly::kNumBars; ++i) mbar_init(&bars[i], 1);
+    for (int i = 0; i < Ly::kNumBars; ++i) mbar_init(&bars[i], i == 6 ? kTWork : 1);
+    *f_fail = 0;
     fence_mbar_init();
     prefetch_tensormap(&maps.x);
     prefetch_tensormap(&maps.B);
     prefetch_tensormap(&maps.C);
+    prefetch_tensormap(&maps.y);
   }
   if (warp == 0) tc::tmem_alloc(slot, kTmemCols);
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tm = *slot;
-  const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
-  const uint32_t tH = tm + lane_base + kColH, tS = tm + lane_base + kColS;
-  const uint32_t tYd = tm + lane_base + kColYd, tYo = tm + lane_base + kColYo;
-
-  // ---- initial state: TMEM lane = state row (head h0 + row / 64, p); the
-  //      two warps of a quadrant write one half of the N columns each
-  {
-    const float* src = p.h0 ? p.h0 + (((size_t)b * H + h0 + row / kTP) * kTP + row % kTP) * N
-                            : nullptr;
-#pragma unroll
-    for (int c0 = half * kHalfN; c0 < (half + 1) * kHalfN; c0 += 32) {
-      float v[32];
-#pragma unroll
-      for (int j = 0; j < 32; j += 4) {
-        const float4 q = src ? *reinterpret_cast<const float4*>(src + c0 + j)
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
-        v[j] = q.x; v[j + 1] = q.y; v[j + 2] = q.z; v[j + 3] = q.w;
-      }
-      tc::st32(tH + c0, v);
-    }
-    tc::wait_st();
-  }
-
-  // TMA issue (thread 0): B and C of chunk c; x of chunk c into buffer i.
   const bool stall = p.test_stall && blockIdx.x == 0 && blockIdx.y == 0;
-  auto issue_bc = [&](int c) {
-    mbar_arrive_expect_tx(bar_bc, (uint32_t)(2 * kNB * Ly::kBlk));
-#pragma unroll
-    for (int nb = 0; nb < kNB; ++nb) {
-      tma_load_3d(sB + nb * Ly::kBlk, &maps.B, bar_bc, nb * 64, c * kTQ, b);
-      tma_load_3d(sC + nb * Ly::kBlk, &maps.C, bar_bc, nb * 64, c * kTQ, b);
-    }
-  };
-  auto issue_x = [&](int c, int i) {
-    uint64_t* bar = i ? bar_x1 : bar_x0;
-    unsigned char* dst = i ? xbuf1 : xbuf0;
-    mbar_arrive_expect_tx(bar, (uint32_t)(kTHeads * Ly::kBlk) + ((stall && c == 0) ? 16u : 0u));
-#pragma unroll
-    for (int hh = 0; hh < kTHeads; ++hh)
-      tc::tma_load_4d(dst + hh * Ly::kBlk, &maps.x, bar, 0, h0 + hh, c * kTQ, b);
-  };
-  // Phases armed (thread 0) and waited (every thread) per barrier; on the
-  // error path thread 0 waits (bounded) for the completions still owed.
-  int armed_bc = 0, armed_x0 = 0, armed_x1 = 0, armed_s = 0, armed_m = 0;
-  int waited_bc = 0, waited_x0 = 0, waited_x1 = 0, waited_s = 0, waited_m = 0;
 
-  // Step quantities of chunk c into buffer c & 1: thread = (head tid / 128,
-  // step tid % 128); Delta, the in-chunk cumulative sum of Delta A (a scan
-  // over the four warps of the head), w_s, E_s = e^{cum_{end of s's 32-step
-  // block} - cum_s} Delta_s and e^{cum_end}. Every thread calls it.
-  const int s_t = tid & 127, s_q = (tid >> 5) & 3;
-  auto load_dt = [&](int c) {
-    const int64_t t = (int64_t)c * kTQ + s_t;
-    return t < L ? bf16_to_f32(p.dt[((size_t)b * L + t) * H + h0 + s_hh]) : 0.f;
-  };
-  auto compute_steps = [&](int c, float raw) {
-    const int i = c & 1;
-    float d = 0.f;
-    if ((int64_t)c * kTQ + s_t < L) {
-      const float v = raw + bias_s;
-      // softplus(v) = ln 2 * log2(1 + 2^(v log2 e)), v above the cut
-      d = p.softplus ? (v > kSoftplusCut ? v : kLn2 * lg2_approx(1.f + ex2_approx(v * kLog2e))) : v;
-    }
-    float a = d * A_s;
+  if (issuer) {
+    // ------------------------------------------------------ issuing warp --
+    if (lane == 0 && nchunks > 0) {
+      auto issue_bc = [&](int c) {
+        mbar_arrive_expect_tx(bar_bc, (uint32_t)(2 * kNB * Ly::kBlk));
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const float u = __shfl_up_sync(0xffffffffu, a, o);
-      if (lane >= o) a += u;
-    }
-    if (lane == 31) f_wsum[s_hh * 4 + s_q] = a;
-    __syncthreads();
-    for (int w = 0; w < s_q; ++w) a += f_wsum[s_hh * 4 + w];
-    sdelta(i)[s_hh * kTQ + s_t] = d;
-    scum(i)[s_hh * kTQ + s_t] = a;
-    __syncthreads();
-    const float cend = scum(i)[s_hh * kTQ + kTQ - 1];
-    sw(i)[s_hh * kTQ + s_t] = ex2_approx((cend - a) * kLog2e) * d;
-    se(i)[s_hh * kTQ + s_t] = ex2_approx((scum(i)[s_hh * kTQ + (s_t | 31)] - a) * kLog2e) * d;
-    if (s_t == 0) f_decay[i * kTHeads + s_hh] = ex2_approx(cend * kLog2e);
-  };
-
-  if (nchunks > 0) {
-    if (tid == 0) {
+        for (int nb = 0; nb < kNB; ++nb) {
+          tma_load_3d(sB + nb * Ly::kBlk, &maps.B, bar_bc, nb * 64, c * kTQ, b);
+          tma_load_3d(sC + nb * Ly::kBlk, &maps.C, bar_bc, nb * 64, c * kTQ, b);
+        }
+      };
+      auto issue_x = [&](int c, int i) {
+        uint64_t* bar = i ? bar_x1 : bar_x0;
+        unsigned char* dst = i ? xbuf1 : xbuf0;
+        mbar_arrive_expect_tx(bar,
+                              (uint32_t)(kTHeads * Ly::kBlk) + ((stall && c == 0) ? 16u : 0u));
+#pragma unroll
+        for (int hh = 0; hh < kTHeads; ++hh)
+          tc::tma_load_4d(dst + hh * Ly::kBlk, &maps.x, bar, 0, h0 + hh, c * kTQ, b);
+      };
+      // last phase armed per barrier (-1: none): on the error path each is
+      // waited for (bounded); earlier phases complete first
+      int last_bc = 0, last_x0 = 0, last_x1 = -1, last_s = -1, last_h = -1, last_m = -1;
       issue_bc(0);
       issue_x(0, 0);
-      armed_bc = 1;
-      armed_x0 = 1;
+      bool ok = true;
+      for (int c = 0; c < nchunks; ++c) {
+        const int xi = c & 1;
+        const uint32_t uB = opaque(smem_u32(sB)), uC = opaque(smem_u32(sC));
+        const uint32_t uHb = opaque(smem_u32(sHb)), uXs = opaque(smem_u32(sXs));
+        const uint32_t uxcur = opaque(smem_u32(xi ? xbuf1 : xbuf0));
+        const uint32_t tmo = opaque(tm);
+        // S = C B^T once this chunk's B and C have landed and the previous
+        // chunk's G X no longer reads the S columns
+        ok = mbar_wait_bounded(bar_bc, (uint32_t)(c & 1), p.wait_limit_ns);
+        if (ok && c > 0) ok = mbar_wait_bounded(bar_m, (uint32_t)((c - 1) & 1), p.wait_limit_ns);
+        if (!ok) break;
+        tc::fence_after_sync();
+        {
+          constexpr uint32_t id = tc::idesc_bf16(128, 128, 0, 0);
+#pragma unroll
+          for (int ks = 0; ks < N / 16; ++ks) {
+            const uint32_t o = (ks / 4) * Ly::kBlk + (ks % 4) * 32;
+            tc::mma_bf16(tmo + kColS, tc::sdesc(uC + o, 16, 1024), tc::sdesc(uB + o, 16, 1024), id,
+                         ks > 0);
+          }
+          tc::commit(bar_s);
+          last_s = c;
+        }
+        // the next chunk's x, into the buffer the previous chunk's y has left
+        if (c + 1 < nchunks) {
+          if (c > 0) {
+            ok = mbar_wait_bounded(bar_xfree, (uint32_t)((c - 1) & 1), p.wait_limit_ns);
+            if (!ok) break;
+          }
+          issue_x(c + 1, xi ^ 1);
+          if (xi) last_x0 = c + 1; else last_x1 = c + 1;
+        }
+        // the compute warps have written G (over S), the scaled x, the bf16
+        // copy of the state and the scaled state
+        ok = mbar_wait_bounded(bar_work, (uint32_t)(c & 1), p.wait_limit_ns);
+        if (!ok) break;
+        tc::fence_after_sync();
+        {  // Yo (t x 2P) = C (t x N) . Hb^T, both K-major over n
+          constexpr uint32_t id = tc::idesc_bf16(128, 128, 0, 0);
+#pragma unroll
+          for (int ks = 0; ks < N / 16; ++ks) {
+            const uint32_t o = (ks / 4) * Ly::kBlk + (ks % 4) * 32;
+            tc::mma_bf16(tmo + kColYo, tc::sdesc(uC + o, 16, 1024), tc::sdesc(uHb + o, 16, 1024),
+                         id, ks > 0);
+          }
+        }
+        {  // H (2P x N) += Xs^T (2P x s) . B (s x N), both MN-major over s
+          constexpr uint32_t id = tc::idesc_bf16(128, N, 1, 1);
+#pragma unroll
+          for (int ks = 0; ks < kTQ / 16; ++ks) {
+            const uint32_t o = ks * 2048;
+            tc::mma_bf16(tmo + kColH, tc::sdesc(uXs + o, Ly::kBlk, 1024),
+                         tc::sdesc(uB + o, Ly::kBlk, 1024), id, 1u);
+          }
+        }
+        tc::commit(bar_h);
+        last_h = c;
+        {  // Yd[:, head hh] (t x P) = G_hh (TMEM, t x s) . x_hh (s x P, MN-major)
+          constexpr uint32_t id = tc::idesc_bf16(128, kTP, 0, 1);
+#pragma unroll
+          for (int hh = 0; hh < kTHeads; ++hh)
+#pragma unroll
+            for (int ks = 0; ks < kTQ / 16; ++ks)
+              mma_bf16_tmem_a(tmo + kColYd + kTP * hh,
+                              tmo + kColS + 64 * (ks / 4) + 32 * hh + 8 * (ks % 4),
+                              tc::sdesc(uxcur + hh * Ly::kBlk + ks * 2048, Ly::kBlk, 1024), id,
+                              ks > 0);
+        }
+        tc::commit(bar_m);
+        last_m = c;
+        // B and C are free once the readout and the state update are done
+        if (c + 1 < nchunks) {
+          ok = mbar_wait_bounded(bar_h, (uint32_t)(c & 1), p.wait_limit_ns);
+          if (!ok) break;
+          issue_bc(c + 1);
+          last_bc = c + 1;
+        }
+      }
+      if (!ok) {
+        // let this CTA's own copies and MMAs in flight land (bounded) before
+        // its shared and tensor memory are released
+        auto drain = [&](uint64_t* bar, int k) {
+          if (k >= 0) (void)mbar_wait_bounded(bar, (uint32_t)(k & 1), 1000000ull);
+        };
+        drain(bar_bc, last_bc);
+        drain(bar_x0, last_x0 >= 0 ? last_x0 / 2 : -1);
+        drain(bar_x1, last_x1 >= 0 ? last_x1 / 2 : -1);
+        drain(bar_s, last_s);
+        drain(bar_h, last_h);
+        drain(bar_m, last_m);
+        *f_fail = 1;
+      }
     }
-    compute_steps(0, load_dt(0));
-  }
-  __syncthreads();
+    __syncwarp();
+  } else {
+    // ----------------------------------------------------- compute warps --
+    const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
+    const uint32_t tH = tm + lane_base + kColH, tS = tm + lane_base + kColS;
+    const uint32_t tYd = tm + lane_base + kColYd, tYo = tm + lane_base + kColYo;
+    // per-head constants of the head this thread computes steps for (s_hh)
+    // and writes outputs for (half)
+    const int s_hh = tid >> 7, s_t = tid & 127, s_q = (tid >> 5) & 3;
+    const float A2 = p.A[h0 + s_hh] * kLog2e;
+    const float bias_s = p.dt_bias ? p.dt_bias[h0 + s_hh] : 0.f;
+    const float D_o = p.D ? p.D[h0 + half] : 0.f;
 
-  bool ok = true;
-  int c = 0;
-  for (; c < nchunks; ++c) {
-    const int xi = c & 1, sb = c & 1;
-    const int64_t t0 = (int64_t)c * kTQ;
-    const float dt_next = c + 1 < nchunks ? load_dt(c + 1) : 0.f;
-    // ---- S = C B^T once this chunk's B and C have landed
-    ok = cta_wait(bar_bc, (uint32_t)(c & 1), p.wait_limit_ns);
-    if (!ok) break;
-    ++waited_bc;
-    if (tid == 0) {
-      tc::fence_after_sync();
-      constexpr uint32_t id = tc::idesc_bf16(128, 128, 0, 0);
-#pragma unroll
-      for (int ks = 0; ks < N / 16; ++ks) {
-        const uint32_t o = (ks / 4) * Ly::kBlk + (ks % 4) * 32;
-        tc::mma_bf16(tm + kColS, tc::sdesc(smem_u32(sC) + o, 16, 1024),
-                     tc::sdesc(smem_u32(sB) + o, 16, 1024), id, ks > 0);
-      }
-      tc::commit(bar_s);
-      ++armed_s;
-    }
-    // ---- this chunk's x: its w-scaled copy into the other buffer (thread =
-    //      (head, step)); the state: bf16 copy for the readout, then scaled
-    //      by e^{cum_end} for the update (thread = state row, half the columns)
-    ok = cta_wait(xi ? bar_x1 : bar_x0, (uint32_t)((c >> 1) & 1), p.wait_limit_ns);
-    if (!ok) break;
-    if (xi) ++waited_x1; else ++waited_x0;
-    unsigned char* const xcur = xi ? xbuf1 : xbuf0;  // x of this chunk
-    unsigned char* const xoth = xi ? xbuf0 : xbuf1;  // its w-scaled copy
+    // initial state: TMEM lane = state row (head h0 + row / 64, p); the two
+    // warps of a quadrant write one half of the N columns each
     {
-      const float w = sw(sb)[s_hh * kTQ + s_t];
+      const float* src = p.h0 ? p.h0 + (((size_t)b * H + h0 + row / kTP) * kTP + row % kTP) * N
+                              : nullptr;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        // a rotated chunk order keeps the 16-byte accesses of a warp on
-        // distinct banks
-        const uint32_t o = s_hh * Ly::kBlk + s_t * 128 + ((j + s_t) & 7) * 16;
-        const uint4 q = *reinterpret_cast<const uint4*>(xcur + o);
-        const float v[8] = {bf16_lo(q.x) * w, bf16_hi(q.x) * w, bf16_lo(q.y) * w,
-                            bf16_hi(q.y) * w, bf16_lo(q.z) * w, bf16_hi(q.z) * w,
-                            bf16_lo(q.w) * w, bf16_hi(q.w) * w};
-        *reinterpret_cast<uint4*>(xoth + o) = pack8(v);
+      for (int c0 = half * kHalfN; c0 < (half + 1) * kHalfN; c0 += 32) {
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+          const float4 q = src ? *reinterpret_cast<const float4*>(src + c0 + j)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+          v[j] = q.x; v[j + 1] = q.y; v[j + 2] = q.z; v[j + 3] = q.w;
+        }
+        tc::st32(tH + c0, v);
       }
-      const float decay = f_decay[sb * kTHeads + row / kTP];
+      tc::wait_st();
+    }
+
+    // Step quantities of chunk c into buffer c & 1: thread = (head s_hh,
+    // step s_t); Delta, the in-chunk cumulative sum of Delta A (a scan over
+    // the four warps of the head), w_s, E_s = e^{cum_{end of s's 32-step
+    // block} - cum_s} Delta_s and e^{cum_end}. Every compute thread calls it.
+    auto load_dt = [&](int c) {
+      const int64_t t = (int64_t)c * kTQ + s_t;
+      return t < L ? bf16_to_f32(p.dt[((size_t)b * L + t) * H + h0 + s_hh]) : 0.f;
+    };
+    auto compute_steps = [&](int c, float raw) {
+      const int i = c & 1;
+      float d = 0.f;
+      if ((int64_t)c * kTQ + s_t < L) {
+        const float v = raw + bias_s;
+        // softplus(v) = ln 2 log2(1 + 2^(v log2 e)); v above the cut
+        d = p.softplus ? (v > kSoftplusCut ? v : kLn2 * lg2_approx(1.f + ex2_approx(v * kLog2e)))
+                       : v;
+      }
+      float a = d * A2;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float u = __shfl_up_sync(0xffffffffu, a, o);
+        if (lane >= o) a += u;
+      }
+      if (lane == 31) f_wsum[s_hh * 4 + s_q] = a;
+      work_sync();
+      for (int w = 0; w < s_q; ++w) a += f_wsum[s_hh * 4 + w];
+      sdelta(i)[s_hh * kTQ + s_t] = d;
+      scum(i)[s_hh * kTQ + s_t] = a;
+      work_sync();
+      const float cend = scum(i)[s_hh * kTQ + kTQ - 1];
+      sw(i)[s_hh * kTQ + s_t] = ex2_approx(cend - a) * d;
+      se(i)[s_hh * kTQ + s_t] = ex2_approx(scum(i)[s_hh * kTQ + (s_t | 31)] - a) * d;
+      if (s_t == 0) f_decay[i * kTHeads + s_hh] = ex2_approx(cend);
+    };
+    // The state entering a chunk (thread = state row, half the columns): a
+    // bf16 copy for the readout, then scaled by e^{cum_end} in TMEM so that
+    // the update MMA accumulates onto it.
+    auto prep_state = [&](int i) {
+      const float decay = f_decay[i * kTHeads + row / kTP];
 #pragma unroll
       for (int c0 = half * kHalfN; c0 < (half + 1) * kHalfN; c0 += 32) {
         float v[32];
@@ -318,147 +403,149 @@ __global__ void __launch_bounds__(kTThreads, 1)
         tc::st32(tH + c0, v);
       }
       tc::wait_st();
+    };
+    if (nchunks > 0) {
+      compute_steps(0, load_dt(0));
+      work_sync();
+      prep_state(0);
     }
-    tc::fence_proxy_async_smem();
-    tc::fence_before_sync();
-    // ---- G of both heads from S (thread = step t, half the columns), written
-    //      over S as bf16 pairs: G of head hh at columns kColS + 64 hh + s / 2.
-    //      32-column blocks j below the diagonal block: e^{cum_t - cum_s}
-    //      Delta_s = F_j E_s with F_j = e^{cum_t - cum_{32 j + 31}} (both
-    //      factors <= 1, one exp per block); the diagonal block one exp per
-    //      entry; above it zero.
-    ok = cta_wait(bar_s, (uint32_t)(c & 1), p.wait_limit_ns);
-    if (!ok) break;
-    ++waited_s;
-    tc::fence_after_sync();
-    {
-      float v[2][32];
-      tc::ld32(tS + 64 * half, v[0]);
-      tc::ld32(tS + 64 * half + 32, v[1]);
-      tc::wait_ld();
-      uint32_t gp[kTHeads][32];
-      const int t = row, tb = t >> 5;
+
+    bool ok = true;
+    for (int c = 0; c < nchunks; ++c) {
+      const int xi = c & 1, sb = c & 1;
+      const int64_t t0 = (int64_t)c * kTQ;
+      const float dt_next = c + 1 < nchunks ? load_dt(c + 1) : 0.f;
+      unsigned char* const xcur = xi ? xbuf1 : xbuf0;  // x of this chunk, then its y
+      // ---- the w-scaled copy of x (thread = (head, step))
+      ok = work_vote(mbar_wait_bounded(xi ? bar_x1 : bar_x0, (uint32_t)((c >> 1) & 1),
+                                       p.wait_limit_ns));
+      if (!ok) break;
+      {
+        const float w = sw(sb)[s_hh * kTQ + s_t];
 #pragma unroll
-      for (int hh = 0; hh < kTHeads; ++hh) {
-        const float* cum = scum(sb) + hh * kTQ;
-        const float* del = sdelta(sb) + hh * kTQ;
-        const float* E = se(sb) + hh * kTQ;
-        const float ct = cum[t];
+        for (int j = 0; j < 8; ++j) {
+          // a rotated chunk order keeps a warp's 16-byte accesses on distinct banks
+          const uint32_t o = s_hh * Ly::kBlk + s_t * 128 + ((j + s_t) & 7) * 16;
+          const uint4 q = *reinterpret_cast<const uint4*>(xcur + o);
+          const float v[8] = {bf16_lo(q.x) * w, bf16_hi(q.x) * w, bf16_lo(q.y) * w,
+                              bf16_hi(q.y) * w, bf16_lo(q.z) * w, bf16_hi(q.z) * w,
+                              bf16_lo(q.w) * w, bf16_hi(q.w) * w};
+          *reinterpret_cast<uint4*>(sXs + o) = pack8(v);
+        }
+      }
+      // the previous chunk's y store has read its buffer: the issuing warp
+      // may load the next x there
+      if (c > 0 && tid == 0) {
+        tc::bulk_wait_read_all();
+        mbar_arrive(bar_xfree);
+      }
+      // ---- G of both heads from S (thread = step t, the 64 steps s of its
+      //      half), written as bf16 pairs over the S columns the thread read:
+      //      G_hh(t, s) at column kColS + 64 (s / 64) + 32 hh + (s % 64) / 2, so
+      //      no other warp's columns are touched. 32-column blocks j below the
+      //      diagonal block: e^{cum_t - cum_s} Delta_s = F_j E_s with F_j =
+      //      e^{cum_t - cum_{32 j + 31}} (both factors <= 1, one exp per block);
+      //      the diagonal block one exp per entry; above it zero.
+      ok = work_vote(mbar_wait_bounded(bar_s, (uint32_t)(c & 1), p.wait_limit_ns));
+      if (!ok) break;
+      tc::fence_after_sync();
+      {
+        float v[2][32];
+        tc::ld32(tS + 64 * half, v[0]);
+        tc::ld32(tS + 64 * half + 32, v[1]);
+        tc::wait_ld();
+        const int t = row, tb = t >> 5;
 #pragma unroll
-        for (int jj = 0; jj < 2; ++jj) {
-          const int j = 2 * half + jj, s0 = 32 * j;
-          float g[32];
-          if (j < tb) {
-            const float F = ex2_approx((ct - cum[s0 + 31]) * kLog2e);
+        for (int hh = 0; hh < kTHeads; ++hh) {
+          const float* cum = scum(sb) + hh * kTQ;
+          const float* del = sdelta(sb) + hh * kTQ;
+          const float* E = se(sb) + hh * kTQ;
+          const float ct = cum[t];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) g[e] = v[jj][e] * F * E[s0 + e];
-          } else if (j == tb) {
+          for (int jj = 0; jj < 2; ++jj) {
+            const int j = 2 * half + jj, s0 = 32 * j;
+            uint32_t gp[16];
+            if (j < tb) {
+              const float F = ex2_approx(ct - cum[s0 + 31]);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const int sidx = s0 + e;
-              g[e] = sidx <= t ? v[jj][e] * ex2_approx((ct - cum[sidx]) * kLog2e) * del[sidx] : 0.f;
+              for (int e = 0; e < 32; e += 4) {
+                const float4 E4 = *reinterpret_cast<const float4*>(E + s0 + e);
+                gp[e / 2] = pack_bf16x2(v[jj][e] * F * E4.x, v[jj][e + 1] * F * E4.y);
+                gp[e / 2 + 1] = pack_bf16x2(v[jj][e + 2] * F * E4.z, v[jj][e + 3] * F * E4.w);
+              }
+            } else if (j == tb) {
+#pragma unroll
+              for (int e = 0; e < 32; e += 4) {
+                const float4 c4 = *reinterpret_cast<const float4*>(cum + s0 + e);
+                const float4 d4 = *reinterpret_cast<const float4*>(del + s0 + e);
+                const float cc[4] = {c4.x, c4.y, c4.z, c4.w}, dd[4] = {d4.x, d4.y, d4.z, d4.w};
+                float g[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                  g[u] = s0 + e + u <= t ? v[jj][e + u] * ex2_approx(ct - cc[u]) * dd[u] : 0.f;
+                gp[e / 2] = pack_bf16x2(g[0], g[1]);
+                gp[e / 2 + 1] = pack_bf16x2(g[2], g[3]);
+              }
+            } else {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) gp[e] = 0u;
             }
-          } else {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) g[e] = 0.f;
+            tc::st16(tS + 64 * half + 32 * hh + 16 * jj, gp);
           }
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) gp[hh][jj * 16 + e / 2] = pack_bf16x2(g[e], g[e + 1]);
         }
+        tc::wait_st();
       }
-      // every warp has read its columns of S before any is overwritten
+      // operands ready: shared-memory writes visible to the tensor core, the
+      // TMEM writes ordered before the MMAs the issuing warp starts next
+      tc::fence_proxy_async_smem();
       tc::fence_before_sync();
-      __syncthreads();
+      mbar_arrive(bar_work);
+      // ---- the next chunk's step quantities while the products run
+      if (c + 1 < nchunks) compute_steps(c + 1, dt_next);
+      // ---- the state entering the next chunk, once this chunk's update is in
+      ok = work_vote(mbar_wait_bounded(bar_h, (uint32_t)(c & 1), p.wait_limit_ns));
+      if (!ok) break;
       tc::fence_after_sync();
-#pragma unroll
-      for (int hh = 0; hh < kTHeads; ++hh) {
-        float f[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(gp[hh][e]);
-        tc::st32(tS + 64 * hh + 32 * half, f);
-      }
-      tc::wait_st();
-    }
-    tc::fence_before_sync();
-    __syncthreads();
-    // ---- the chunk's products: C H^T, the state update, G X of both heads
-    if (tid == 0) {
+      if (c + 1 < nchunks) prep_state((c + 1) & 1);
+      // ---- y_t = Yd + e^{cum_t} Yo + D x_t (thread = (head `half`, step t)),
+      //      written over x_t in shared memory, then stored by TMA
+      ok = work_vote(mbar_wait_bounded(bar_m, (uint32_t)(c & 1), p.wait_limit_ns));
+      if (!ok) break;
       tc::fence_after_sync();
-      {  // Yo (t x 2P) = C (t x N) . Hb^T, both K-major over n
-        constexpr uint32_t id = tc::idesc_bf16(128, 128, 0, 0);
+      {
+        const int t = row, hh = half;
+        const float ec = ex2_approx(scum(sb)[hh * kTQ + t]);
+        unsigned char* const xrow = xcur + hh * Ly::kBlk;
 #pragma unroll
-        for (int ks = 0; ks < N / 16; ++ks) {
-          const uint32_t o = (ks / 4) * Ly::kBlk + (ks % 4) * 32;
-          tc::mma_bf16(tm + kColYo, tc::sdesc(smem_u32(sC) + o, 16, 1024),
-                       tc::sdesc(smem_u32(sHb) + o, 16, 1024), id, ks > 0);
+        for (int c0 = 0; c0 < kTP; c0 += 32) {
+          float yd[32], yo[32];
+          tc::ld32(tYd + hh * kTP + c0, yd);
+          tc::ld32(tYo + hh * kTP + c0, yo);
+          tc::wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; j += 8) {
+            uint4* const px = reinterpret_cast<uint4*>(xrow + tc::sw128(t, c0 + j));
+            const uint4 q = *px;
+            const float xv[8] = {bf16_lo(q.x), bf16_hi(q.x), bf16_lo(q.y), bf16_hi(q.y),
+                                 bf16_lo(q.z), bf16_hi(q.z), bf16_lo(q.w), bf16_hi(q.w)};
+            float o[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) o[e] = fmaf(D_o, xv[e], fmaf(ec, yo[j + e], yd[j + e]));
+            *px = pack8(o);
+          }
         }
       }
-      {  // H (2P x N) += Xt^T (2P x s) . B (s x N), both MN-major over s
-        constexpr uint32_t id = tc::idesc_bf16(128, N, 1, 1);
-#pragma unroll
-        for (int ks = 0; ks < kTQ / 16; ++ks) {
-          const uint32_t o = ks * 2048;
-          tc::mma_bf16(tm + kColH, tc::sdesc(smem_u32(xoth) + o, Ly::kBlk, 1024),
-                       tc::sdesc(smem_u32(sB) + o, Ly::kBlk, 1024), id, 1u);
-        }
-      }
-      {  // Yd[:, head hh] (t x P) = G_hh (TMEM, t x s) . x_hh (s x P, MN-major)
-        constexpr uint32_t id = tc::idesc_bf16(128, kTP, 0, 1);
+      tc::fence_proxy_async_smem();
+      work_sync();
+      if (tid == 0) {  // rows past the sequence end are not written
 #pragma unroll
         for (int hh = 0; hh < kTHeads; ++hh)
-#pragma unroll
-          for (int ks = 0; ks < kTQ / 16; ++ks)
-            mma_bf16_tmem_a(tm + kColYd + kTP * hh, tm + kColS + 64 * hh + ks * 8,
-                            tc::sdesc(smem_u32(xcur) + hh * Ly::kBlk + ks * 2048, Ly::kBlk, 1024),
-                            id, ks > 0);
-      }
-      tc::commit(bar_m);
-      ++armed_m;
-    }
-    // ---- the next chunk's step quantities while the products run
-    if (c + 1 < nchunks) compute_steps(c + 1, dt_next);
-    // ---- the buffers of B, C and the scaled x are free: next chunk's loads;
-    //      y_t = Yd + e^{cum_t} Yo + D x_t (thread = (head, step t))
-    ok = cta_wait(bar_m, (uint32_t)(c & 1), p.wait_limit_ns);
-    if (!ok) break;
-    ++waited_m;
-    tc::fence_after_sync();
-    if (tid == 0 && c + 1 < nchunks) {
-      issue_bc(c + 1);
-      issue_x(c + 1, xi ^ 1);
-      ++armed_bc;
-      if (xi) ++armed_x0; else ++armed_x1;
-    }
-    {
-      const int t = row, hh = half;  // TMEM lane t; warps 4-7 take head 1
-      const int64_t tg = t0 + t;
-      const float ec = ex2_approx(scum(sb)[hh * kTQ + t] * kLog2e);
-      uint16_t* yrow = p.y + (((size_t)b * L + (tg < L ? tg : 0)) * H + h0 + hh) * kTP;
-#pragma unroll
-      for (int c0 = 0; c0 < kTP; c0 += 32) {
-        float yd[32], yo[32];
-        tc::ld32(tYd + hh * kTP + c0, yd);
-        tc::ld32(tYo + hh * kTP + c0, yo);
-        tc::wait_ld();
-#pragma unroll
-        for (int j = 0; j < 32; j += 8) {
-          const int pc = c0 + j;
-          const uint4 q = *reinterpret_cast<const uint4*>(xcur + hh * Ly::kBlk + tc::sw128(t, pc));
-          const float xv[8] = {bf16_lo(q.x), bf16_hi(q.x), bf16_lo(q.y), bf16_hi(q.y),
-                               bf16_lo(q.z), bf16_hi(q.z), bf16_lo(q.w), bf16_hi(q.w)};
-          float o[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) o[e] = fmaf(D_o, xv[e], fmaf(ec, yo[j + e], yd[j + e]));
-          if (tg < L) *reinterpret_cast<uint4*>(yrow + pc) = pack8(o);
-        }
+          tc::tma_store_4d(&maps.y, xcur + hh * Ly::kBlk, 0, h0 + hh, (int)t0, b);
+        tc::bulk_commit();
       }
     }
-    tc::fence_before_sync();
-    __syncthreads();
-  }
-
-  if (ok) {
-    if (p.h_last) {
+    if (tid == 0) tc::bulk_wait_all();
+    if (ok && p.h_last) {
       tc::fence_after_sync();
       float* dst = p.h_last + (((size_t)b * H + h0 + row / kTP) * kTP + row % kTP) * N;
 #pragma unroll
@@ -471,21 +558,11 @@ __global__ void __launch_bounds__(kTThreads, 1)
           *reinterpret_cast<float4*>(dst + c0 + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
       }
     }
-  } else if (tid == 0) {
-    // A wait ran out: let this CTA's own copies and MMAs in flight land
-    // (bounded) before its shared and tensor memory are released.
-    auto drain = [&](uint64_t* bar, int done, int armed) {
-      for (int k = done; k < armed; ++k) (void)mbar_wait_bounded(bar, (uint32_t)(k & 1), 1000000ull);
-    };
-    drain(bar_bc, waited_bc, armed_bc);
-    drain(bar_x0, waited_x0, armed_x0);
-    drain(bar_x1, waited_x1, armed_x1);
-    drain(bar_s, waited_s, armed_s);
-    drain(bar_m, waited_m, armed_m);
-    atomicExch(&g_ssd_status, 1);
+    if (!ok && tid == 0) *f_fail = 1;
   }
   tc::fence_before_sync();
   __syncthreads();
+  if (tid == 0 && *f_fail) atomicExch(&g_ssd_status, 1);
   if (warp == 0) tc::tmem_dealloc(tm, kTmemCols);
 }
 
