@@ -726,9 +726,9 @@ int ssm_ssd_scan_fwd(int64_t batch, int64_t seqlen, int64_t nheads, int64_t head
                                                     (long)kDefaultWaitLimitNs));
   p.test_stall = env_long("SSM_SSD_TEST_STALL", 0) != 0 ? 1 : 0;
   // The tcgen05 kernel: dstate 64 or 128, an even head count, 16-byte aligned
-  // state buffers; SSM_SSD_LEGACY=1 keeps the mma.sync kernel.
+  // state buffers, 4-byte aligned dt; SSM_SSD_LEGACY=1 keeps the mma.sync kernel.
   const bool tc = seqlen > 0 && ssd_tc_supported((int)dstate, (int)nheads) &&
-                  env_long("SSM_SSD_LEGACY", 0) == 0 && (!h0 || aligned(h0, 16)) &&
+                  env_long("SSM_SSD_LEGACY", 0) == 0 && aligned(dt, 4) && (!h0 || aligned(h0, 16)) &&
                   (!h_last || aligned(h_last, 16)) && encode_fn() != nullptr;
   if (tc) {
     SsdTcMaps maps;

@@ -87,9 +87,12 @@ struct TcLayout {
   // cum[Q], w[Q], E[Q]
   static constexpr int kStepBuf = kTHeads * 4 * kTQ;
   static constexpr int kStepFloats = 2 * kStepBuf + kTHeads * 4 + 2 * kTHeads + 2;
-  static constexpr int kOffBar = round_up(kOffSteps + kStepFloats * 4, 8);
-  // B/C, x (two buffers), S, readout + update, G X, operands, x buffer free
-  static constexpr int kNumBars = 8;
+  // raw Delta of three chunks in flight: [chunk % 3][head][Q] pairs (h0, h0 + 1)
+  static constexpr int kOffDt = round_up(kOffSteps + kStepFloats * 4, 16);
+  static constexpr int kOffBar = kOffDt + 3 * kTHeads * kTQ * 4;
+  // B/C, x (two buffers), S, readout + update, G X, operands, x buffer free,
+  // scaled x and state written
+  static constexpr int kNumBars = 9;
   static constexpr int kOffSlot = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffSlot + 16 + 1024;  // + room to align the base to 1024
   static_assert(N == 64 || N == 128, "state width 64 or 128");
@@ -127,6 +130,11 @@ __device__ __forceinline__ bool work_vote(bool v) {
 }
 __device__ __forceinline__ void work_sync() {
   asm volatile("barrier.cta.sync 1, %0;" ::"n"(kTWork) : "memory");
+}
+// 4-byte asynchronous copy global -> shared.
+__device__ __forceinline__ void cp_async_4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src)
+               : "memory");
 }
 // A value the compiler cannot treat as loop-invariant: the issuing warp
 // derives its descriptors from it each chunk instead of keeping dozens live.
@@ -172,6 +180,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
   uint64_t* bar_m = bars + 5;      // G X done: every product of the chunk (MMA commit)
   uint64_t* bar_work = bars + 6;   // the compute warps' operands are written (256 arrivals)
   uint64_t* bar_xfree = bars + 7;  // a chunk's y has left its x buffer (bulk store read)
+  uint64_t* bar_xs = bars + 8;     // the scaled x and the prepared state are written (256)
   uint32_t* slot = reinterpret_cast<uint32_t*>(sm + Ly::kOffSlot);
   unsigned char* const xbuf0 = sm + Ly::kOffX0;
   unsigned char* const xbuf1 = sm + Ly::kOffX1;
@@ -182,7 +191,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
   int* f_fail = reinterpret_cast<int*>(f_decay + 2 * kTHeads);
 
   if (tid == 0) {
-    for (int i = 0; i < Ly::kNumBars; ++i) mbar_init(&bars[i], i == 6 ? kTWork : 1);
+    for (int i = 0; i < Ly::kNumBars; ++i) mbar_init(&bars[i], (i == 6 || i == 8) ? kTWork : 1);
     *f_fail = 0;
     fence_mbar_init();
     prefetch_tensormap(&maps.x);
@@ -255,9 +264,9 @@ __global__ void __launch_bounds__(kTThreads, 1)
           issue_x(c + 1, xi ^ 1);
           if (xi) last_x0 = c + 1; else last_x1 = c + 1;
         }
-        // the compute warps have written G (over S), the scaled x, the bf16
-        // copy of the state and the scaled state
-        ok = mbar_wait_bounded(bar_work, (uint32_t)(c & 1), p.wait_limit_ns);
+        // the compute warps have written the scaled x, the bf16 copy of the
+        // state and the scaled state
+        ok = mbar_wait_bounded(bar_xs, (uint32_t)(c & 1), p.wait_limit_ns);
         if (!ok) break;
         tc::fence_after_sync();
         {  // Yo (t x 2P) = C (t x N) . Hb^T, both K-major over n
@@ -280,6 +289,10 @@ __global__ void __launch_bounds__(kTThreads, 1)
         }
         tc::commit(bar_h);
         last_h = c;
+        // ... and G (over S)
+        ok = mbar_wait_bounded(bar_work, (uint32_t)(c & 1), p.wait_limit_ns);
+        if (!ok) break;
+        tc::fence_after_sync();
         {  // Yd[:, head hh] (t x P) = G_hh (TMEM, t x s) . x_hh (s x P, MN-major)
           constexpr uint32_t id = tc::idesc_bf16(128, kTP, 0, 1);
 #pragma unroll
@@ -352,15 +365,24 @@ __global__ void __launch_bounds__(kTThreads, 1)
     // step s_t); Delta, the in-chunk cumulative sum of Delta A (a scan over
     // the four warps of the head), w_s, E_s = e^{cum_{end of s's 32-step
     // block} - cum_s} Delta_s and e^{cum_end}. Every compute thread calls it.
-    auto load_dt = [&](int c) {
+    // Raw Delta of chunk c, two chunks ahead by an asynchronous copy into this
+    // thread's own slot (the pair of heads; the thread keeps its head's half),
+    // so that no thread waits on a global load at a barrier. One commit group
+    // per call, empty past the end.
+    uint32_t* const sdt = reinterpret_cast<uint32_t*>(sm + Ly::kOffDt);
+    auto fetch_dt = [&](int c) {
       const int64_t t = (int64_t)c * kTQ + s_t;
-      return t < L ? bf16_to_f32(p.dt[((size_t)b * L + t) * H + h0 + s_hh]) : 0.f;
+      if (c < nchunks && t < L)
+        cp_async_4(&sdt[((c % 3) * kTHeads + s_hh) * kTQ + s_t],
+                   p.dt + ((size_t)b * L + t) * H + h0);
+      cp_async_commit_group();
     };
-    auto compute_steps = [&](int c, float raw) {
+    auto compute_steps = [&](int c) {
       const int i = c & 1;
       float d = 0.f;
       if ((int64_t)c * kTQ + s_t < L) {
-        const float v = raw + bias_s;
+        const uint32_t pr = sdt[((c % 3) * kTHeads + s_hh) * kTQ + s_t];
+        const float v = (s_hh ? bf16_hi(pr) : bf16_lo(pr)) + bias_s;
         // softplus(v) = ln 2 log2(1 + 2^(v log2 e)); v above the cut
         d = p.softplus ? (v > kSoftplusCut ? v : kLn2 * lg2_approx(1.f + ex2_approx(v * kLog2e)))
                        : v;
@@ -404,8 +426,11 @@ __global__ void __launch_bounds__(kTThreads, 1)
       }
       tc::wait_st();
     };
+    fetch_dt(0);
+    fetch_dt(1);
     if (nchunks > 0) {
-      compute_steps(0, load_dt(0));
+      cp_async_wait_group<1>();
+      compute_steps(0);
       work_sync();
       prep_state(0);
     }
@@ -414,7 +439,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
     for (int c = 0; c < nchunks; ++c) {
       const int xi = c & 1, sb = c & 1;
       const int64_t t0 = (int64_t)c * kTQ;
-      const float dt_next = c + 1 < nchunks ? load_dt(c + 1) : 0.f;
+      fetch_dt(c + 2);
       unsigned char* const xcur = xi ? xbuf1 : xbuf0;  // x of this chunk, then its y
       // ---- the w-scaled copy of x (thread = (head, step))
       ok = work_vote(mbar_wait_bounded(xi ? bar_x1 : bar_x0, (uint32_t)((c >> 1) & 1),
@@ -433,6 +458,11 @@ __global__ void __launch_bounds__(kTThreads, 1)
           *reinterpret_cast<uint4*>(sXs + o) = pack8(v);
         }
       }
+      // the scaled x (and the state prepared in the previous iteration) are
+      // ready for the readout and update MMAs
+      tc::fence_proxy_async_smem();
+      tc::fence_before_sync();
+      mbar_arrive(bar_xs);
       // the previous chunk's y store has read its buffer: the issuing warp
       // may load the next x there
       if (c > 0 && tid == 0) {
@@ -501,8 +531,12 @@ __global__ void __launch_bounds__(kTThreads, 1)
       tc::fence_before_sync();
       mbar_arrive(bar_work);
       // ---- the next chunk's step quantities while the products run
-      if (c + 1 < nchunks) compute_steps(c + 1, dt_next);
-      // ---- the state entering the next chunk, once this chunk's update is in
+      if (c + 1 < nchunks) {
+        cp_async_wait_group<1>();  // chunk c + 1's copy has landed (c + 2's may not)
+        compute_steps(c + 1);
+      }
+      // ---- the state entering the next chunk, once this chunk's readout and
+      //      update are in
       ok = work_vote(mbar_wait_bounded(bar_h, (uint32_t)(c & 1), p.wait_limit_ns));
       if (!ok) break;
       tc::fence_after_sync();
