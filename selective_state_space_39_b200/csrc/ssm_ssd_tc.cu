@@ -61,7 +61,8 @@ constexpr int kTQ = 128;        // steps per chunk
 constexpr int kTP = 64;         // head width
 constexpr int kTHeads = 2;      // heads per CTA
 constexpr int kTWork = 256;     // eight compute warps, two per TMEM lane quadrant
-constexpr int kTThreads = kTWork + 32;  // and one warp that issues copies and MMAs
+// and two warps: one issues the copies and MMAs, one computes the step quantities
+constexpr int kTThreads = kTWork + 64;
 constexpr uint32_t kTmemCols = 512;
 // TMEM columns: the state, S (then G of both heads, bf16 pairs), G X, C H^T
 constexpr uint32_t kColH = 0, kColS = 128, kColYd = 256, kColYo = 384;
@@ -83,16 +84,14 @@ struct TcLayout {
   static constexpr int kOffC = kOffB + kBC;
   static constexpr int kOffHb = kOffC + kBC;
   static constexpr int kOffSteps = kOffHb + kHb;
-  // step quantities, two buffers (this chunk, the next): per head Delta[Q],
-  // cum[Q], w[Q], E[Q]
+  // step quantities, per head Delta[Q], cum[Q], w[Q], E[Q]
   static constexpr int kStepBuf = kTHeads * 4 * kTQ;
-  static constexpr int kStepFloats = 2 * kStepBuf + kTHeads * 4 + 2 * kTHeads + 2;
-  // raw Delta of three chunks in flight: [chunk % 3][head][Q] pairs (h0, h0 + 1)
-  static constexpr int kOffDt = round_up(kOffSteps + kStepFloats * 4, 16);
-  static constexpr int kOffBar = kOffDt + 3 * kTHeads * kTQ * 4;
+  // three buffers (chunk % 3), then e^{cum_end} per buffer and head, a flag
+  static constexpr int kStepFloats = 3 * kStepBuf + 3 * kTHeads + 2;
+  static constexpr int kOffBar = round_up(kOffSteps + kStepFloats * 4, 8);
   // B/C, x (two buffers), S, readout + update, G X, operands, x buffer free,
-  // scaled x and state written
-  static constexpr int kNumBars = 9;
+  // scaled x and state written, step buffer written (3), step buffer read (3)
+  static constexpr int kNumBars = 15;
   static constexpr int kOffSlot = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffSlot + 16 + 1024;  // + room to align the base to 1024
   static_assert(N == 64 || N == 128, "state width 64 or 128");
@@ -131,11 +130,6 @@ __device__ __forceinline__ bool work_vote(bool v) {
 __device__ __forceinline__ void work_sync() {
   asm volatile("barrier.cta.sync 1, %0;" ::"n"(kTWork) : "memory");
 }
-// 4-byte asynchronous copy global -> shared.
-__device__ __forceinline__ void cp_async_4(void* dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src)
-               : "memory");
-}
 // A value the compiler cannot treat as loop-invariant: the issuing warp
 // derives its descriptors from it each chunk instead of keeping dozens live.
 __device__ __forceinline__ uint32_t opaque(uint32_t v) {
@@ -154,7 +148,8 @@ __global__ void __launch_bounds__(kTThreads, 1)
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bool issuer = warp == kTWork / 32;  // the ninth warp issues copies and MMAs
+  const bool issuer = warp == kTWork / 32;       // the ninth warp issues copies and MMAs
+  const bool stepper = warp == kTWork / 32 + 1;  // the tenth computes step quantities
   const int quad = warp & 3, half = (warp >> 2) & 1;
   const int row = 32 * quad + lane;  // a compute thread's TMEM lane: a step t or a state row
   const int h0 = blockIdx.x * kTHeads, b = blockIdx.y;
@@ -163,8 +158,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
   const int nchunks = (int)((L + kTQ - 1) / kTQ);
 
   float* steps = reinterpret_cast<float*>(sm + Ly::kOffSteps);
-  float* f_wsum = steps + 2 * Ly::kStepBuf;  // [head][quadrant]
-  float* f_decay = f_wsum + kTHeads * 4;     // [buffer][head]
+  float* f_decay = steps + 3 * Ly::kStepBuf;  // [buffer][head]
   // step arrays of buffer i, each [head][Q]: Delta, cum (in units of log2,
   // i.e. log2 e times the sum of Delta A), w, E
   auto sdelta = [&](int i) { return steps + i * Ly::kStepBuf; };
@@ -181,6 +175,8 @@ __global__ void __launch_bounds__(kTThreads, 1)
   uint64_t* bar_work = bars + 6;   // the compute warps' operands are written (256 arrivals)
   uint64_t* bar_xfree = bars + 7;  // a chunk's y has left its x buffer (bulk store read)
   uint64_t* bar_xs = bars + 8;     // the scaled x and the prepared state are written (256)
+  uint64_t* bar_sready = bars + 9;  // [3] step buffer written (32 arrivals)
+  uint64_t* bar_sfree = bars + 12;  // [3] step buffer read for the last time
   uint32_t* slot = reinterpret_cast<uint32_t*>(sm + Ly::kOffSlot);
   unsigned char* const xbuf0 = sm + Ly::kOffX0;
   unsigned char* const xbuf1 = sm + Ly::kOffX1;
@@ -188,10 +184,11 @@ __global__ void __launch_bounds__(kTThreads, 1)
   unsigned char* sB = sm + Ly::kOffB;
   unsigned char* sC = sm + Ly::kOffC;
   unsigned char* sHb = sm + Ly::kOffHb;
-  int* f_fail = reinterpret_cast<int*>(f_decay + 2 * kTHeads);
+  int* f_fail = reinterpret_cast<int*>(f_decay + 3 * kTHeads);
 
   if (tid == 0) {
-    for (int i = 0; i < Ly::kNumBars; ++i) mbar_init(&bars[i], (i == 6 || i == 8) ? kTWork : 1);
+    for (int i = 0; i < Ly::kNumBars; ++i)
+      mbar_init(&bars[i], (i == 6 || i == 8) ? kTWork : (i >= 9 && i < 12) ? 32 : 1);
     *f_fail = 0;
     fence_mbar_init();
     prefetch_tensormap(&maps.x);
@@ -330,6 +327,79 @@ __global__ void __launch_bounds__(kTThreads, 1)
       }
     }
     __syncwarp();
+  } else if (stepper) {
+    // ------------------------------------------------------- steps warp --
+    // Step quantities of chunk k into buffer k % 3, up to three chunks ahead
+    // of the compute warps; lane = the four steps t = 4 lane + u of both
+    // heads: Delta, cum (the in-chunk inclusive sum of Delta A, in log2
+    // units), w_s = e^{cum_end - cum_s} Delta_s, E_s = e^{cum_{end of s's
+    // 32-step block} - cum_s} Delta_s, and e^{cum_end} per head.
+    float A2[kTHeads], bias[kTHeads];
+#pragma unroll
+    for (int hh = 0; hh < kTHeads; ++hh) {
+      A2[hh] = p.A[h0 + hh] * kLog2e;
+      bias[hh] = p.dt_bias ? p.dt_bias[h0 + hh] : 0.f;
+    }
+    bool ok = true;
+    for (int k = 0; k < nchunks; ++k) {
+      const int i = k % 3;
+      const int64_t tb = (int64_t)k * kTQ + 4 * lane;
+      uint32_t raw[4];  // dt of heads h0, h0 + 1 (4-byte aligned pairs)
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        raw[u] = tb + u < L ? *reinterpret_cast<const uint32_t*>(
+                                  p.dt + ((size_t)b * L + tb + u) * H + h0)
+                            : 0u;
+      // the buffer's previous chunk has been read for the last time
+      if (k >= 3) {
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bar_sfree[i], (uint32_t)(((k - 3) / 3) & 1),
+                                                        p.wait_limit_ns));
+        if (!ok) break;
+      }
+#pragma unroll
+      for (int hh = 0; hh < kTHeads; ++hh) {
+        float d[4], a[4];
+        float run = 0.f;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float v = (hh ? bf16_hi(raw[u]) : bf16_lo(raw[u])) + bias[hh];
+          // softplus(v) = ln 2 log2(1 + 2^(v log2 e)); v above the cut
+          const float dv =
+              tb + u >= L ? 0.f
+              : p.softplus
+                  ? (v > kSoftplusCut ? v : kLn2 * lg2_approx(1.f + ex2_approx(v * kLog2e)))
+                  : v;
+          d[u] = dv;
+          run = fmaf(dv, A2[hh], run);
+          a[u] = run;
+        }
+        float incl = run;  // scan of the lanes' sums
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const float q = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += q;
+        }
+        const float excl = incl - run;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) a[u] += excl;
+        const float cend = __shfl_sync(0xffffffffu, a[3], 31);
+        const float cblk = __shfl_sync(0xffffffffu, a[3], lane | 7);  // t = 32 (t / 32) + 31
+        float w[4], e[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          w[u] = ex2_approx(cend - a[u]) * d[u];
+          e[u] = ex2_approx(cblk - a[u]) * d[u];
+        }
+        const int o = hh * kTQ + 4 * lane;
+        *reinterpret_cast<float4*>(sdelta(i) + o) = make_float4(d[0], d[1], d[2], d[3]);
+        *reinterpret_cast<float4*>(scum(i) + o) = make_float4(a[0], a[1], a[2], a[3]);
+        *reinterpret_cast<float4*>(sw(i) + o) = make_float4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<float4*>(se(i) + o) = make_float4(e[0], e[1], e[2], e[3]);
+        if (lane == 0) f_decay[i * kTHeads + hh] = ex2_approx(cend);
+      }
+      mbar_arrive(&bar_sready[i]);
+    }
+    if (!ok && lane == 0) *f_fail = 1;
   } else {
     // ----------------------------------------------------- compute warps --
     const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
@@ -337,9 +407,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
     const uint32_t tYd = tm + lane_base + kColYd, tYo = tm + lane_base + kColYo;
     // per-head constants of the head this thread computes steps for (s_hh)
     // and writes outputs for (half)
-    const int s_hh = tid >> 7, s_t = tid & 127, s_q = (tid >> 5) & 3;
-    const float A2 = p.A[h0 + s_hh] * kLog2e;
-    const float bias_s = p.dt_bias ? p.dt_bias[h0 + s_hh] : 0.f;
+    const int s_hh = tid >> 7, s_t = tid & 127;
     const float D_o = p.D ? p.D[h0 + half] : 0.f;
 
     // initial state: TMEM lane = state row (head h0 + row / 64, p); the two
@@ -361,49 +429,6 @@ __global__ void __launch_bounds__(kTThreads, 1)
       tc::wait_st();
     }
 
-    // Step quantities of chunk c into buffer c & 1: thread = (head s_hh,
-    // step s_t); Delta, the in-chunk cumulative sum of Delta A (a scan over
-    // the four warps of the head), w_s, E_s = e^{cum_{end of s's 32-step
-    // block} - cum_s} Delta_s and e^{cum_end}. Every compute thread calls it.
-    // Raw Delta of chunk c, two chunks ahead by an asynchronous copy into this
-    // thread's own slot (the pair of heads; the thread keeps its head's half),
-    // so that no thread waits on a global load at a barrier. One commit group
-    // per call, empty past the end.
-    uint32_t* const sdt = reinterpret_cast<uint32_t*>(sm + Ly::kOffDt);
-    auto fetch_dt = [&](int c) {
-      const int64_t t = (int64_t)c * kTQ + s_t;
-      if (c < nchunks && t < L)
-        cp_async_4(&sdt[((c % 3) * kTHeads + s_hh) * kTQ + s_t],
-                   p.dt + ((size_t)b * L + t) * H + h0);
-      cp_async_commit_group();
-    };
-    auto compute_steps = [&](int c) {
-      const int i = c & 1;
-      float d = 0.f;
-      if ((int64_t)c * kTQ + s_t < L) {
-        const uint32_t pr = sdt[((c % 3) * kTHeads + s_hh) * kTQ + s_t];
-        const float v = (s_hh ? bf16_hi(pr) : bf16_lo(pr)) + bias_s;
-        // softplus(v) = ln 2 log2(1 + 2^(v log2 e)); v above the cut
-        d = p.softplus ? (v > kSoftplusCut ? v : kLn2 * lg2_approx(1.f + ex2_approx(v * kLog2e)))
-                       : v;
-      }
-      float a = d * A2;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const float u = __shfl_up_sync(0xffffffffu, a, o);
-        if (lane >= o) a += u;
-      }
-      if (lane == 31) f_wsum[s_hh * 4 + s_q] = a;
-      work_sync();
-      for (int w = 0; w < s_q; ++w) a += f_wsum[s_hh * 4 + w];
-      sdelta(i)[s_hh * kTQ + s_t] = d;
-      scum(i)[s_hh * kTQ + s_t] = a;
-      work_sync();
-      const float cend = scum(i)[s_hh * kTQ + kTQ - 1];
-      sw(i)[s_hh * kTQ + s_t] = ex2_approx(cend - a) * d;
-      se(i)[s_hh * kTQ + s_t] = ex2_approx(scum(i)[s_hh * kTQ + (s_t | 31)] - a) * d;
-      if (s_t == 0) f_decay[i * kTHeads + s_hh] = ex2_approx(cend);
-    };
     // The state entering a chunk (thread = state row, half the columns): a
     // bf16 copy for the readout, then scaled by e^{cum_end} in TMEM so that
     // the update MMA accumulates onto it.
@@ -421,25 +446,23 @@ __global__ void __launch_bounds__(kTThreads, 1)
               pack8(v + j);
         }
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] *= decay;
+        for (int j = 0; j < 32; j += 2) {
+          const float2 q2 = mul2(make_float2(v[j], v[j + 1]), make_float2(decay, decay));
+          v[j] = q2.x;
+          v[j + 1] = q2.y;
+        }
         tc::st32(tH + c0, v);
       }
       tc::wait_st();
     };
-    fetch_dt(0);
-    fetch_dt(1);
-    if (nchunks > 0) {
-      cp_async_wait_group<1>();
-      compute_steps(0);
-      work_sync();
-      prep_state(0);
-    }
-
     bool ok = true;
-    for (int c = 0; c < nchunks; ++c) {
-      const int xi = c & 1, sb = c & 1;
+    if (nchunks > 0) {
+      ok = work_vote(mbar_wait_bounded(&bar_sready[0], 0u, p.wait_limit_ns));
+      if (ok) prep_state(0);
+    }
+    for (int c = 0; c < nchunks && ok; ++c) {
+      const int xi = c & 1, sb = c % 3;
       const int64_t t0 = (int64_t)c * kTQ;
-      fetch_dt(c + 2);
       unsigned char* const xcur = xi ? xbuf1 : xbuf0;  // x of this chunk, then its y
       // ---- the w-scaled copy of x (thread = (head, step))
       ok = work_vote(mbar_wait_bounded(xi ? bar_x1 : bar_x0, (uint32_t)((c >> 1) & 1),
@@ -452,10 +475,14 @@ __global__ void __launch_bounds__(kTThreads, 1)
           // a rotated chunk order keeps a warp's 16-byte accesses on distinct banks
           const uint32_t o = s_hh * Ly::kBlk + s_t * 128 + ((j + s_t) & 7) * 16;
           const uint4 q = *reinterpret_cast<const uint4*>(xcur + o);
-          const float v[8] = {bf16_lo(q.x) * w, bf16_hi(q.x) * w, bf16_lo(q.y) * w,
-                              bf16_hi(q.y) * w, bf16_lo(q.z) * w, bf16_hi(q.z) * w,
-                              bf16_lo(q.w) * w, bf16_hi(q.w) * w};
-          *reinterpret_cast<uint4*>(sXs + o) = pack8(v);
+          const float2 w2 = make_float2(w, w);
+          const float2 a0 = mul2(make_float2(bf16_lo(q.x), bf16_hi(q.x)), w2);
+          const float2 a1 = mul2(make_float2(bf16_lo(q.y), bf16_hi(q.y)), w2);
+          const float2 a2 = mul2(make_float2(bf16_lo(q.z), bf16_hi(q.z)), w2);
+          const float2 a3 = mul2(make_float2(bf16_lo(q.w), bf16_hi(q.w)), w2);
+          *reinterpret_cast<uint4*>(sXs + o) =
+              make_uint4(pack_bf16x2(a0.x, a0.y), pack_bf16x2(a1.x, a1.y), pack_bf16x2(a2.x, a2.y),
+                         pack_bf16x2(a3.x, a3.y));
         }
       }
       // the scaled x (and the state prepared in the previous iteration) are
@@ -497,11 +524,16 @@ __global__ void __launch_bounds__(kTThreads, 1)
             uint32_t gp[16];
             if (j < tb) {
               const float F = ex2_approx(ct - cum[s0 + 31]);
+              const float2 F2 = make_float2(F, F);
 #pragma unroll
               for (int e = 0; e < 32; e += 4) {
                 const float4 E4 = *reinterpret_cast<const float4*>(E + s0 + e);
-                gp[e / 2] = pack_bf16x2(v[jj][e] * F * E4.x, v[jj][e + 1] * F * E4.y);
-                gp[e / 2 + 1] = pack_bf16x2(v[jj][e + 2] * F * E4.z, v[jj][e + 3] * F * E4.w);
+                const float2 g0 = mul2(mul2(make_float2(v[jj][e], v[jj][e + 1]), F2),
+                                       make_float2(E4.x, E4.y));
+                const float2 g1 = mul2(mul2(make_float2(v[jj][e + 2], v[jj][e + 3]), F2),
+                                       make_float2(E4.z, E4.w));
+                gp[e / 2] = pack_bf16x2(g0.x, g0.y);
+                gp[e / 2 + 1] = pack_bf16x2(g1.x, g1.y);
               }
             } else if (j == tb) {
 #pragma unroll
@@ -509,12 +541,20 @@ __global__ void __launch_bounds__(kTThreads, 1)
                 const float4 c4 = *reinterpret_cast<const float4*>(cum + s0 + e);
                 const float4 d4 = *reinterpret_cast<const float4*>(del + s0 + e);
                 const float cc[4] = {c4.x, c4.y, c4.z, c4.w}, dd[4] = {d4.x, d4.y, d4.z, d4.w};
-                float g[4];
+                float ex[4];
 #pragma unroll
-                for (int u = 0; u < 4; ++u)
-                  g[u] = s0 + e + u <= t ? v[jj][e + u] * ex2_approx(ct - cc[u]) * dd[u] : 0.f;
-                gp[e / 2] = pack_bf16x2(g[0], g[1]);
-                gp[e / 2 + 1] = pack_bf16x2(g[2], g[3]);
+                for (int u = 0; u < 4; ++u) ex[u] = ex2_approx(ct - cc[u]);
+                float2 g0 = mul2(mul2(make_float2(v[jj][e], v[jj][e + 1]), make_float2(ex[0], ex[1])),
+                                 make_float2(dd[0], dd[1]));
+                float2 g1 = mul2(mul2(make_float2(v[jj][e + 2], v[jj][e + 3]), make_float2(ex[2], ex[3])),
+                                 make_float2(dd[2], dd[3]));
+                const int sb0 = s0 + e;  // steps s > t are above the diagonal
+                if (sb0 > t) g0.x = 0.f;
+                if (sb0 + 1 > t) g0.y = 0.f;
+                if (sb0 + 2 > t) g1.x = 0.f;
+                if (sb0 + 3 > t) g1.y = 0.f;
+                gp[e / 2] = pack_bf16x2(g0.x, g0.y);
+                gp[e / 2 + 1] = pack_bf16x2(g1.x, g1.y);
               }
             } else {
 #pragma unroll
@@ -530,17 +570,18 @@ __global__ void __launch_bounds__(kTThreads, 1)
       tc::fence_proxy_async_smem();
       tc::fence_before_sync();
       mbar_arrive(bar_work);
-      // ---- the next chunk's step quantities while the products run
-      if (c + 1 < nchunks) {
-        cp_async_wait_group<1>();  // chunk c + 1's copy has landed (c + 2's may not)
-        compute_steps(c + 1);
-      }
       // ---- the state entering the next chunk, once this chunk's readout and
-      //      update are in
-      ok = work_vote(mbar_wait_bounded(bar_h, (uint32_t)(c & 1), p.wait_limit_ns));
+      //      update are in and the next chunk's step quantities are written
+      {
+        bool w = mbar_wait_bounded(bar_h, (uint32_t)(c & 1), p.wait_limit_ns);
+        if (w && c + 1 < nchunks)
+          w = mbar_wait_bounded(&bar_sready[(c + 1) % 3], (uint32_t)(((c + 1) / 3) & 1),
+                                p.wait_limit_ns);
+        ok = work_vote(w);
+      }
       if (!ok) break;
       tc::fence_after_sync();
-      if (c + 1 < nchunks) prep_state((c + 1) & 1);
+      if (c + 1 < nchunks) prep_state((c + 1) % 3);
       // ---- y_t = Yd + e^{cum_t} Yo + D x_t (thread = (head `half`, step t)),
       //      written over x_t in shared memory, then stored by TMA
       ok = work_vote(mbar_wait_bounded(bar_m, (uint32_t)(c & 1), p.wait_limit_ns));
@@ -564,7 +605,13 @@ __global__ void __launch_bounds__(kTThreads, 1)
                                  bf16_lo(q.z), bf16_hi(q.z), bf16_lo(q.w), bf16_hi(q.w)};
             float o[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) o[e] = fmaf(D_o, xv[e], fmaf(ec, yo[j + e], yd[j + e]));
+            for (int e = 0; e < 8; e += 2) {
+              const float2 r = fma2(make_float2(ec, ec), make_float2(yo[j + e], yo[j + e + 1]),
+                                    make_float2(yd[j + e], yd[j + e + 1]));
+              const float2 q2 = fma2(make_float2(D_o, D_o), make_float2(xv[e], xv[e + 1]), r);
+              o[e] = q2.x;
+              o[e + 1] = q2.y;
+            }
             *px = pack8(o);
           }
         }
@@ -576,6 +623,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
         for (int hh = 0; hh < kTHeads; ++hh)
           tc::tma_store_4d(&maps.y, xcur + hh * Ly::kBlk, 0, h0 + hh, (int)t0, b);
         tc::bulk_commit();
+        mbar_arrive(&bar_sfree[sb]);  // the chunk's step buffer is free
       }
     }
     if (tid == 0) tc::bulk_wait_all();
