@@ -90,8 +90,9 @@ struct TcLayout {
   static constexpr int kStepFloats = 3 * kStepBuf + 3 * kTHeads + 2;
   static constexpr int kOffBar = round_up(kOffSteps + kStepFloats * 4, 8);
   // B/C, x (two buffers), S, readout + update, G X, operands, x buffer free,
-  // scaled x and state written, step buffer written (3), step buffer read (3)
-  static constexpr int kNumBars = 15;
+  // scaled x and state written, step buffer written (3), step buffer read (3),
+  // the second head's G written
+  static constexpr int kNumBars = 16;
   static constexpr int kOffSlot = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffSlot + 16 + 1024;  // + room to align the base to 1024
   static_assert(N == 64 || N == 128, "state width 64 or 128");
@@ -129,6 +130,17 @@ __device__ __forceinline__ bool work_vote(bool v) {
 }
 __device__ __forceinline__ void work_sync() {
   asm volatile("barrier.cta.sync 1, %0;" ::"n"(kTWork) : "memory");
+}
+// Non-blocking test of phase `parity` of `bar`.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return r != 0;
 }
 // A value the compiler cannot treat as loop-invariant: the issuing warp
 // derives its descriptors from it each chunk instead of keeping dozens live.
@@ -172,11 +184,12 @@ __global__ void __launch_bounds__(kTThreads, 1)
   uint64_t* bar_s = bars + 3;      // S = C B^T done (MMA commit)
   uint64_t* bar_h = bars + 4;      // readout C H^T and state update done (MMA commit)
   uint64_t* bar_m = bars + 5;      // G X done: every product of the chunk (MMA commit)
-  uint64_t* bar_work = bars + 6;   // the compute warps' operands are written (256 arrivals)
+  uint64_t* bar_work = bars + 6;   // G of the first head is written (256 arrivals)
   uint64_t* bar_xfree = bars + 7;  // a chunk's y has left its x buffer (bulk store read)
   uint64_t* bar_xs = bars + 8;     // the scaled x and the prepared state are written (256)
   uint64_t* bar_sready = bars + 9;  // [3] step buffer written (32 arrivals)
   uint64_t* bar_sfree = bars + 12;  // [3] step buffer read for the last time
+  uint64_t* bar_work1 = bars + 15;  // G of the second head is written (256 arrivals)
   uint32_t* slot = reinterpret_cast<uint32_t*>(sm + Ly::kOffSlot);
   unsigned char* const xbuf0 = sm + Ly::kOffX0;
   unsigned char* const xbuf1 = sm + Ly::kOffX1;
@@ -188,7 +201,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
 
   if (tid == 0) {
     for (int i = 0; i < Ly::kNumBars; ++i)
-      mbar_init(&bars[i], (i == 6 || i == 8) ? kTWork : (i >= 9 && i < 12) ? 32 : 1);
+      mbar_init(&bars[i], (i == 6 || i == 8 || i == 15) ? kTWork : (i >= 9 && i < 12) ? 32 : 1);
     *f_fail = 0;
     fence_mbar_init();
     prefetch_tensormap(&maps.x);
@@ -286,25 +299,32 @@ __global__ void __launch_bounds__(kTThreads, 1)
         }
         tc::commit(bar_h);
         last_h = c;
-        // ... and G (over S)
-        ok = mbar_wait_bounded(bar_work, (uint32_t)(c & 1), p.wait_limit_ns);
-        if (!ok) break;
-        tc::fence_after_sync();
-        {  // Yd[:, head hh] (t x P) = G_hh (TMEM, t x s) . x_hh (s x P, MN-major)
+        // ... and G (over S), head by head: Yd[:, head hh] (t x P) =
+        // G_hh (TMEM, t x s) . x_hh (s x P, MN-major). B and C of the next
+        // chunk go out once the readout and the state update are done.
+        bool bc_out = c + 1 >= nchunks;
+#pragma unroll
+        for (int hh = 0; hh < kTHeads; ++hh) {
+          ok = mbar_wait_bounded(hh ? bar_work1 : bar_work, (uint32_t)(c & 1), p.wait_limit_ns);
+          if (!ok) break;
+          tc::fence_after_sync();
           constexpr uint32_t id = tc::idesc_bf16(128, kTP, 0, 1);
 #pragma unroll
-          for (int hh = 0; hh < kTHeads; ++hh)
-#pragma unroll
-            for (int ks = 0; ks < kTQ / 16; ++ks)
-              mma_bf16_tmem_a(tmo + kColYd + kTP * hh,
-                              tmo + kColS + 64 * (ks / 4) + 32 * hh + 8 * (ks % 4),
-                              tc::sdesc(uxcur + hh * Ly::kBlk + ks * 2048, Ly::kBlk, 1024), id,
-                              ks > 0);
+          for (int ks = 0; ks < kTQ / 16; ++ks)
+            mma_bf16_tmem_a(tmo + kColYd + kTP * hh,
+                            tmo + kColS + 64 * (ks / 4) + 32 * hh + 8 * (ks % 4),
+                            tc::sdesc(uxcur + hh * Ly::kBlk + ks * 2048, Ly::kBlk, 1024), id,
+                            ks > 0);
+          if (hh == 0 && !bc_out && mbar_test_wait(bar_h, (uint32_t)(c & 1))) {
+            issue_bc(c + 1);
+            last_bc = c + 1;
+            bc_out = true;
+          }
         }
+        if (!ok) break;
         tc::commit(bar_m);
         last_m = c;
-        // B and C are free once the readout and the state update are done
-        if (c + 1 < nchunks) {
+        if (!bc_out) {
           ok = mbar_wait_bounded(bar_h, (uint32_t)(c & 1), p.wait_limit_ns);
           if (!ok) break;
           issue_bc(c + 1);
@@ -322,7 +342,10 @@ __global__ void __launch_bounds__(kTThreads, 1)
         drain(bar_x1, last_x1 >= 0 ? last_x1 / 2 : -1);
         drain(bar_s, last_s);
         drain(bar_h, last_h);
-        drain(bar_m, last_m);
+        // MMAs issued after the last commit (a chunk's first G X) complete
+        // with one more phase of bar_m
+        tc::commit(bar_m);
+        drain(bar_m, last_m + 1);
         *f_fail = 1;
       }
     }
@@ -562,14 +585,12 @@ __global__ void __launch_bounds__(kTThreads, 1)
             }
             tc::st16(tS + 64 * half + 32 * hh + 16 * jj, gp);
           }
+          // this head's G is written: its G X may start
+          tc::wait_st();
+          tc::fence_before_sync();
+          mbar_arrive(hh ? bar_work1 : bar_work);
         }
-        tc::wait_st();
       }
-      // operands ready: shared-memory writes visible to the tensor core, the
-      // TMEM writes ordered before the MMAs the issuing warp starts next
-      tc::fence_proxy_async_smem();
-      tc::fence_before_sync();
-      mbar_arrive(bar_work);
       // ---- the state entering the next chunk, once this chunk's readout and
       //      update are in and the next chunk's step quantities are written
       {
