@@ -844,8 +844,11 @@ def ssd_bench(args):
     else:
         roof = {"bound": "tensor", "achieved": round(tfs, 1), "peak": tc_peak,
                 "unit": "TFLOP/s", "frac": round(tfs / tc_peak, 4), "peak_kind": tc_kind}
-    roof.update({"traffic": measured_traffic(w.name, "ssd_traffic.json"),
-                 "kernel": f"ssd_fwd_kernel<{N}> (1 launch)",
+    # the tensor-core kernel serves dstate 64 / 128 with an even head count
+    tc = N in (64, 128) and w.nheads % 2 == 0 and os.environ.get("SSM_SSD_LEGACY", "0") == "0"
+    roof.update({"traffic": measured_traffic(w.name, "ssd_tc_traffic.json" if tc
+                                             else "ssd_traffic.json"),
+                 "kernel": f"{'ssd_tc_kernel' if tc else 'ssd_fwd_kernel'}<{N}> (1 launch)",
                  "algorithmic_bytes_per_launch": nbytes, "algorithmic_flops_per_launch": flops,
                  "tensor": {"achieved_tflops": round(tfs, 1), "peak": tc_peak,
                             "frac": round(tfs / tc_peak, 4), "peak_kind": tc_kind},
