@@ -727,14 +727,15 @@ SSD_METRIC = "SSD scan elements/s (B·L·H·P) with tensor-core TFLOP/s and HBM 
 DEFAULT_SSD_WORKLOAD = "ssd_mamba2_b4_l4096_h64_p64_n128"
 
 
-def ssd_cost(w):
+def ssd_cost(w, Q=32):
     """Algorithmic bytes and FLOPs of one SSD call. Bytes: x read and y written
     (bf16), B, C, dt read, h0 read and h_last written (fp32). FLOPs: the
-    chunked dual form's products per (batch, head, chunk of Q): G X over the
-    causal half (Q^2 P), C H and the state's (w X)^T B (2 Q N P each), and
+    chunked dual form's products per (batch, head, chunk of Q steps): G X over
+    the causal half (Q^2 P), C H and the state's (w X)^T B (2 Q N P each), and
     C B^T over the causal half (Q^2 N), once per chunk (B and C are shared by
-    the heads)."""
-    Q, P, N = 32, w.headdim, w.dstate
+    the heads). Q is the chunk length of the kernel that runs (128 for the
+    tensor-core kernel, 32 for the mma.sync one)."""
+    P, N = w.headdim, w.dstate
     tok = w.batch * w.seqlen
     nbytes = 2 * 2 * tok * w.nheads * P + 2 * 2 * tok * N + 2 * tok * w.nheads + \
         4 * w.batch * w.nheads * P * N * (2 if w.with_h0 else 1)
@@ -831,7 +832,9 @@ def ssd_bench(args):
     e2e_ms = e0.elapsed_time(e1) / E
 
     elems = w.elements
-    nbytes, flops = ssd_cost(w)
+    # the tensor-core kernel serves dstate 64 / 128 with an even head count
+    tc = N in (64, 128) and w.nheads % 2 == 0 and os.environ.get("SSM_SSD_LEGACY", "0") == "0"
+    nbytes, flops = ssd_cost(w, Q=128 if tc else 32)
     hbm_peak, hbm_kind = measured_hbm_peak()
     tc_peak, tc_kind = measured_bf16_peak()
     gbs = nbytes / (ms * 1e-3) / 1e9
@@ -844,8 +847,6 @@ def ssd_bench(args):
     else:
         roof = {"bound": "tensor", "achieved": round(tfs, 1), "peak": tc_peak,
                 "unit": "TFLOP/s", "frac": round(tfs / tc_peak, 4), "peak_kind": tc_kind}
-    # the tensor-core kernel serves dstate 64 / 128 with an even head count
-    tc = N in (64, 128) and w.nheads % 2 == 0 and os.environ.get("SSM_SSD_LEGACY", "0") == "0"
     roof.update({"traffic": measured_traffic(w.name, "ssd_tc_traffic.json" if tc
                                              else "ssd_traffic.json"),
                  "kernel": f"{'ssd_tc_kernel' if tc else 'ssd_fwd_kernel'}<{N}> (1 launch)",
