@@ -15,13 +15,15 @@
 //   H      <- e^{cum_end} H + sum_s w_s x_s B_s^T,   w_s = e^{cum_end - cum_s} Delta_s
 //
 // Design (B200). One CTA per batch row and pair of heads walks the chunks in
-// order: one warp issues the TMA copies and the MMAs, eight compute warps do
-// the rest (warps w and w + 4 share TMEM lanes 32 (w % 4) .. and split each
-// row's columns, or the two heads, between them); they meet at mbarriers,
-// so the MMAs of a chunk run while the compute warps prepare the next
-// chunk's step quantities, and the next chunk's S while they write this
-// chunk's outputs. Every product
-// is a tcgen05 MMA of M = 128 with fp32 accumulators in TMEM:
+// order. Warp roles: one warp issues every TMA copy and MMA, one computes the
+// step quantities (Delta, cum, w, E, e^{cum_end}) up to three chunks ahead,
+// sixteen compute warps do the rest (warps w, w + 4, w + 8, w + 12 share TMEM
+// lanes 32 (w % 4) .. and take a quarter of each row's columns, or a head and
+// half its columns, each). They meet at mbarriers: the readout and the state
+// update run while the compute warps form G, G X of the first head while they
+// form the second head's G, the next chunk's S while they write this chunk's
+// outputs. Every product is a tcgen05 MMA of M = 128 with fp32 accumulators
+// in TMEM:
 //   S = C B^T (t x s, K = N; both operands from shared memory),
 //   the readout C H^T (t x (2 heads x p), K = N; H as a bf16 copy in shared
 //   memory),
@@ -32,13 +34,11 @@
 // threads read it, keep the bf16 copy for the readout and write it back
 // scaled by e^{cum_end} before the update MMA accumulates onto it. x, B and
 // C arrive by TMA with the 128-byte swizzle the MMA descriptors describe (no
-// multicast); the next chunk's copies start as soon as the chunk's MMAs have
-// released their buffers (two x buffers alternate between the raw x and the
-// w-scaled x), and the next chunk's step quantities are computed while the
-// chunk's MMAs run (its tiles are prefetched into L2 a chunk ahead). Steps
-// past the sequence end read zeros and take Delta =
-// 0, so they change nothing. Every wait is bounded; a wait that runs out
-// stops the CTA (after its copies and MMAs in flight land, bounded too),
+// multicast): x a chunk ahead into two buffers, B and C once the readout and
+// the update have released them. y is written over the chunk's x in shared
+// memory and stored by TMA. Steps past the sequence end read zeros and take
+// Delta = 0, so they change nothing. Every wait is bounded; a wait that runs
+// out stops the CTA (after its copies and MMAs in flight land, bounded too),
 // frees its TMEM and sets the flag that ssm_ssd_scan_status reports.
 #include <stdlib.h>
 
@@ -60,7 +60,7 @@ namespace {
 constexpr int kTQ = 128;        // steps per chunk
 constexpr int kTP = 64;         // head width
 constexpr int kTHeads = 2;      // heads per CTA
-constexpr int kTWork = 256;     // eight compute warps, two per TMEM lane quadrant
+constexpr int kTWork = 512;     // sixteen compute warps, four per TMEM lane quadrant
 // and two warps: one issues the copies and MMAs, one computes the step quantities
 constexpr int kTThreads = kTWork + 64;
 constexpr uint32_t kTmemCols = 512;
@@ -156,13 +156,14 @@ __global__ void __launch_bounds__(kTThreads, 1)
     ssd_tc_kernel(const SsdParams p, const __grid_constant__ SsdTcMaps maps) {
   using Ly = TcLayout<N>;
   constexpr int kNB = Ly::kNB;
-  constexpr int kHalfN = N / 2;  // state columns per compute warp of a lane quadrant
+  constexpr int kQN = N / 4;  // state columns per compute warp of a lane quadrant
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bool issuer = warp == kTWork / 32;       // the ninth warp issues copies and MMAs
-  const bool stepper = warp == kTWork / 32 + 1;  // the tenth computes step quantities
-  const int quad = warp & 3, half = (warp >> 2) & 1;
+  const bool issuer = warp == kTWork / 32;       // warp 16 issues copies and MMAs
+  const bool stepper = warp == kTWork / 32 + 1;  // warp 17 computes step quantities
+  // a compute warp's TMEM lane quadrant and its quarter of the quadrant's work
+  const int quad = warp & 3, grp = (warp >> 2) & 3;
   const int row = 32 * quad + lane;  // a compute thread's TMEM lane: a step t or a state row
   const int h0 = blockIdx.x * kTHeads, b = blockIdx.y;
   const int H = p.nheads;
@@ -312,7 +313,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
 #pragma unroll
           for (int ks = 0; ks < kTQ / 16; ++ks)
             mma_bf16_tmem_a(tmo + kColYd + kTP * hh,
-                            tmo + kColS + 64 * (ks / 4) + 32 * hh + 8 * (ks % 4),
+                            tmo + kColS + 32 * (ks / 2) + 16 * hh + 8 * (ks % 2),
                             tc::sdesc(uxcur + hh * Ly::kBlk + ks * 2048, Ly::kBlk, 1024), id,
                             ks > 0);
           if (hh == 0 && !bc_out && mbar_test_wait(bar_h, (uint32_t)(c & 1))) {
@@ -428,54 +429,64 @@ __global__ void __launch_bounds__(kTThreads, 1)
     const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
     const uint32_t tH = tm + lane_base + kColH, tS = tm + lane_base + kColS;
     const uint32_t tYd = tm + lane_base + kColYd, tYo = tm + lane_base + kColYo;
-    // per-head constants of the head this thread computes steps for (s_hh)
-    // and writes outputs for (half)
-    const int s_hh = tid >> 7, s_t = tid & 127;
-    const float D_o = p.D ? p.D[h0 + half] : 0.f;
+    // the scaled copy of x: thread = (half of a row's 16-byte chunks, head, step)
+    const int s_t = tid & 127, s_hh = (tid >> 7) & 1, s_ch = tid >> 8;
+    // the epilogue: thread = (head, half of the head's 64 columns, step)
+    const int e_hh = grp >> 1, e_ph = grp & 1;
+    const float D_o = p.D ? p.D[h0 + e_hh] : 0.f;
+    // this warp's N / 4 columns of the state (TMEM lane = state row)
+    auto ldq = [&](uint32_t a, float (&v)[kQN]) {
+      if constexpr (kQN == 32) tc::ld32(a, v);
+      else tc::ld16(a, v);
+    };
+    auto stq = [&](uint32_t a, const float (&v)[kQN]) {
+      if constexpr (kQN == 32) {
+        tc::st32(a, v);
+      } else {
+        uint32_t r[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(v[i]);
+        tc::st16(a, r);
+      }
+    };
+    const int q0 = grp * kQN;  // first state column of this warp
 
-    // initial state: TMEM lane = state row (head h0 + row / 64, p); the two
-    // warps of a quadrant write one half of the N columns each
+    // initial state: TMEM lane = state row (head h0 + row / 64, p)
     {
       const float* src = p.h0 ? p.h0 + (((size_t)b * H + h0 + row / kTP) * kTP + row % kTP) * N
                               : nullptr;
+      float v[kQN];
 #pragma unroll
-      for (int c0 = half * kHalfN; c0 < (half + 1) * kHalfN; c0 += 32) {
-        float v[32];
-#pragma unroll
-        for (int j = 0; j < 32; j += 4) {
-          const float4 q = src ? *reinterpret_cast<const float4*>(src + c0 + j)
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
-          v[j] = q.x; v[j + 1] = q.y; v[j + 2] = q.z; v[j + 3] = q.w;
-        }
-        tc::st32(tH + c0, v);
+      for (int j = 0; j < kQN; j += 4) {
+        const float4 q = src ? *reinterpret_cast<const float4*>(src + q0 + j)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+        v[j] = q.x; v[j + 1] = q.y; v[j + 2] = q.z; v[j + 3] = q.w;
       }
+      stq(tH + q0, v);
       tc::wait_st();
     }
 
-    // The state entering a chunk (thread = state row, half the columns): a
-    // bf16 copy for the readout, then scaled by e^{cum_end} in TMEM so that
-    // the update MMA accumulates onto it.
+    // The state entering a chunk (thread = state row, N / 4 columns): a bf16
+    // copy for the readout, then scaled by e^{cum_end} in TMEM so that the
+    // update MMA accumulates onto it.
     auto prep_state = [&](int i) {
       const float decay = f_decay[i * kTHeads + row / kTP];
+      float v[kQN];
+      ldq(tH + q0, v);
+      tc::wait_ld();
 #pragma unroll
-      for (int c0 = half * kHalfN; c0 < (half + 1) * kHalfN; c0 += 32) {
-        float v[32];
-        tc::ld32(tH + c0, v);
-        tc::wait_ld();
-#pragma unroll
-        for (int j = 0; j < 32; j += 8) {
-          const int col = c0 + j;
-          *reinterpret_cast<uint4*>(sHb + (col / 64) * Ly::kBlk + tc::sw128(row, col % 64)) =
-              pack8(v + j);
-        }
-#pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          const float2 q2 = mul2(make_float2(v[j], v[j + 1]), make_float2(decay, decay));
-          v[j] = q2.x;
-          v[j + 1] = q2.y;
-        }
-        tc::st32(tH + c0, v);
+      for (int j = 0; j < kQN; j += 8) {
+        const int col = q0 + j;
+        *reinterpret_cast<uint4*>(sHb + (col / 64) * Ly::kBlk + tc::sw128(row, col % 64)) =
+            pack8(v + j);
       }
+#pragma unroll
+      for (int j = 0; j < kQN; j += 2) {
+        const float2 q2 = mul2(make_float2(v[j], v[j + 1]), make_float2(decay, decay));
+        v[j] = q2.x;
+        v[j + 1] = q2.y;
+      }
+      stq(tH + q0, v);
       tc::wait_st();
     };
     bool ok = true;
@@ -487,15 +498,16 @@ __global__ void __launch_bounds__(kTThreads, 1)
       const int xi = c & 1, sb = c % 3;
       const int64_t t0 = (int64_t)c * kTQ;
       unsigned char* const xcur = xi ? xbuf1 : xbuf0;  // x of this chunk, then its y
-      // ---- the w-scaled copy of x (thread = (head, step))
+      // ---- the w-scaled copy of x (thread = (head, step, half the chunks))
       ok = work_vote(mbar_wait_bounded(xi ? bar_x1 : bar_x0, (uint32_t)((c >> 1) & 1),
                                        p.wait_limit_ns));
       if (!ok) break;
       {
         const float w = sw(sb)[s_hh * kTQ + s_t];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int jj = 0; jj < 4; ++jj) {
           // a rotated chunk order keeps a warp's 16-byte accesses on distinct banks
+          const int j = 4 * s_ch + jj;
           const uint32_t o = s_hh * Ly::kBlk + s_t * 128 + ((j + s_t) & 7) * 16;
           const uint4 q = *reinterpret_cast<const uint4*>(xcur + o);
           const float2 w2 = make_float2(w, w);
@@ -519,72 +531,65 @@ __global__ void __launch_bounds__(kTThreads, 1)
         tc::bulk_wait_read_all();
         mbar_arrive(bar_xfree);
       }
-      // ---- G of both heads from S (thread = step t, the 64 steps s of its
-      //      half), written as bf16 pairs over the S columns the thread read:
-      //      G_hh(t, s) at column kColS + 64 (s / 64) + 32 hh + (s % 64) / 2, so
-      //      no other warp's columns are touched. 32-column blocks j below the
-      //      diagonal block: e^{cum_t - cum_s} Delta_s = F_j E_s with F_j =
+      // ---- G of both heads from S (thread = step t, the 32 steps s of block
+      //      j = this warp's quarter), written as bf16 pairs over the S columns
+      //      the thread read: G_hh(t, s) at column kColS + 32 (s / 32) + 16 hh
+      //      + (s % 32) / 2, so no other warp's columns are touched. Blocks
+      //      below the diagonal: e^{cum_t - cum_s} Delta_s = F_j E_s with F_j =
       //      e^{cum_t - cum_{32 j + 31}} (both factors <= 1, one exp per block);
       //      the diagonal block one exp per entry; above it zero.
       ok = work_vote(mbar_wait_bounded(bar_s, (uint32_t)(c & 1), p.wait_limit_ns));
       if (!ok) break;
       tc::fence_after_sync();
       {
-        float v[2][32];
-        tc::ld32(tS + 64 * half, v[0]);
-        tc::ld32(tS + 64 * half + 32, v[1]);
+        float v[32];
+        tc::ld32(tS + 32 * grp, v);
         tc::wait_ld();
-        const int t = row, tb = t >> 5;
+        const int t = row, tb = t >> 5, j = grp, s0 = 32 * j;
 #pragma unroll
         for (int hh = 0; hh < kTHeads; ++hh) {
           const float* cum = scum(sb) + hh * kTQ;
           const float* del = sdelta(sb) + hh * kTQ;
           const float* E = se(sb) + hh * kTQ;
           const float ct = cum[t];
+          uint32_t gp[16];
+          if (j < tb) {
+            const float F = ex2_approx(ct - cum[s0 + 31]);
+            const float2 F2 = make_float2(F, F);
 #pragma unroll
-          for (int jj = 0; jj < 2; ++jj) {
-            const int j = 2 * half + jj, s0 = 32 * j;
-            uint32_t gp[16];
-            if (j < tb) {
-              const float F = ex2_approx(ct - cum[s0 + 31]);
-              const float2 F2 = make_float2(F, F);
-#pragma unroll
-              for (int e = 0; e < 32; e += 4) {
-                const float4 E4 = *reinterpret_cast<const float4*>(E + s0 + e);
-                const float2 g0 = mul2(mul2(make_float2(v[jj][e], v[jj][e + 1]), F2),
-                                       make_float2(E4.x, E4.y));
-                const float2 g1 = mul2(mul2(make_float2(v[jj][e + 2], v[jj][e + 3]), F2),
-                                       make_float2(E4.z, E4.w));
-                gp[e / 2] = pack_bf16x2(g0.x, g0.y);
-                gp[e / 2 + 1] = pack_bf16x2(g1.x, g1.y);
-              }
-            } else if (j == tb) {
-#pragma unroll
-              for (int e = 0; e < 32; e += 4) {
-                const float4 c4 = *reinterpret_cast<const float4*>(cum + s0 + e);
-                const float4 d4 = *reinterpret_cast<const float4*>(del + s0 + e);
-                const float cc[4] = {c4.x, c4.y, c4.z, c4.w}, dd[4] = {d4.x, d4.y, d4.z, d4.w};
-                float ex[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) ex[u] = ex2_approx(ct - cc[u]);
-                float2 g0 = mul2(mul2(make_float2(v[jj][e], v[jj][e + 1]), make_float2(ex[0], ex[1])),
-                                 make_float2(dd[0], dd[1]));
-                float2 g1 = mul2(mul2(make_float2(v[jj][e + 2], v[jj][e + 3]), make_float2(ex[2], ex[3])),
-                                 make_float2(dd[2], dd[3]));
-                const int sb0 = s0 + e;  // steps s > t are above the diagonal
-                if (sb0 > t) g0.x = 0.f;
-                if (sb0 + 1 > t) g0.y = 0.f;
-                if (sb0 + 2 > t) g1.x = 0.f;
-                if (sb0 + 3 > t) g1.y = 0.f;
-                gp[e / 2] = pack_bf16x2(g0.x, g0.y);
-                gp[e / 2 + 1] = pack_bf16x2(g1.x, g1.y);
-              }
-            } else {
-#pragma unroll
-              for (int e = 0; e < 16; ++e) gp[e] = 0u;
+            for (int e = 0; e < 32; e += 4) {
+              const float4 E4 = *reinterpret_cast<const float4*>(E + s0 + e);
+              const float2 g0 =
+                  mul2(mul2(make_float2(v[e], v[e + 1]), F2), make_float2(E4.x, E4.y));
+              const float2 g1 =
+                  mul2(mul2(make_float2(v[e + 2], v[e + 3]), F2), make_float2(E4.z, E4.w));
+              gp[e / 2] = pack_bf16x2(g0.x, g0.y);
+              gp[e / 2 + 1] = pack_bf16x2(g1.x, g1.y);
             }
-            tc::st16(tS + 64 * half + 32 * hh + 16 * jj, gp);
+          } else if (j == tb) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+              const float4 c4 = *reinterpret_cast<const float4*>(cum + s0 + e);
+              const float4 d4 = *reinterpret_cast<const float4*>(del + s0 + e);
+              const float ex0 = ex2_approx(ct - c4.x), ex1 = ex2_approx(ct - c4.y);
+              const float ex2v = ex2_approx(ct - c4.z), ex3 = ex2_approx(ct - c4.w);
+              float2 g0 = mul2(mul2(make_float2(v[e], v[e + 1]), make_float2(ex0, ex1)),
+                               make_float2(d4.x, d4.y));
+              float2 g1 = mul2(mul2(make_float2(v[e + 2], v[e + 3]), make_float2(ex2v, ex3)),
+                               make_float2(d4.z, d4.w));
+              const int sb0 = s0 + e;  // steps s > t are above the diagonal
+              if (sb0 > t) g0.x = 0.f;
+              if (sb0 + 1 > t) g0.y = 0.f;
+              if (sb0 + 2 > t) g1.x = 0.f;
+              if (sb0 + 3 > t) g1.y = 0.f;
+              gp[e / 2] = pack_bf16x2(g0.x, g0.y);
+              gp[e / 2 + 1] = pack_bf16x2(g1.x, g1.y);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) gp[e] = 0u;
           }
+          tc::st16(tS + 32 * j + 16 * hh, gp);
           // this head's G is written: its G X may start
           tc::wait_st();
           tc::fence_before_sync();
@@ -603,17 +608,17 @@ __global__ void __launch_bounds__(kTThreads, 1)
       if (!ok) break;
       tc::fence_after_sync();
       if (c + 1 < nchunks) prep_state((c + 1) % 3);
-      // ---- y_t = Yd + e^{cum_t} Yo + D x_t (thread = (head `half`, step t)),
-      //      written over x_t in shared memory, then stored by TMA
+      // ---- y_t = Yd + e^{cum_t} Yo + D x_t (thread = (head, 32 of its columns,
+      //      step t)), written over x_t in shared memory, then stored by TMA
       ok = work_vote(mbar_wait_bounded(bar_m, (uint32_t)(c & 1), p.wait_limit_ns));
       if (!ok) break;
       tc::fence_after_sync();
       {
-        const int t = row, hh = half;
+        const int t = row, hh = e_hh;
         const float ec = ex2_approx(scum(sb)[hh * kTQ + t]);
         unsigned char* const xrow = xcur + hh * Ly::kBlk;
-#pragma unroll
-        for (int c0 = 0; c0 < kTP; c0 += 32) {
+        {
+          const int c0 = 32 * e_ph;
           float yd[32], yo[32];
           tc::ld32(tYd + hh * kTP + c0, yd);
           tc::ld32(tYo + hh * kTP + c0, yo);
@@ -650,16 +655,13 @@ __global__ void __launch_bounds__(kTThreads, 1)
     if (tid == 0) tc::bulk_wait_all();
     if (ok && p.h_last) {
       tc::fence_after_sync();
-      float* dst = p.h_last + (((size_t)b * H + h0 + row / kTP) * kTP + row % kTP) * N;
+      float* dst = p.h_last + (((size_t)b * H + h0 + row / kTP) * kTP + row % kTP) * N + q0;
+      float v[kQN];
+      ldq(tH + q0, v);
+      tc::wait_ld();
 #pragma unroll
-      for (int c0 = half * kHalfN; c0 < (half + 1) * kHalfN; c0 += 32) {
-        float v[32];
-        tc::ld32(tH + c0, v);
-        tc::wait_ld();
-#pragma unroll
-        for (int j = 0; j < 32; j += 4)
-          *reinterpret_cast<float4*>(dst + c0 + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-      }
+      for (int j = 0; j < kQN; j += 4)
+        *reinterpret_cast<float4*>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
     }
     if (!ok && tid == 0) *f_fail = 1;
   }
