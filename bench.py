@@ -167,6 +167,10 @@ class ClockSampler:
             time.sleep(self.interval)
 
     def __enter__(self):
+        # the main thread holds the GIL while it enqueues launches; a short
+        # switch interval lets this thread take a sample every interval
+        self._switch = sys.getswitchinterval()
+        sys.setswitchinterval(min(self._switch, self.interval / 2))
         if self.nvml:
             self.t.start()
         return self
@@ -175,6 +179,7 @@ class ClockSampler:
         self._stop.set()
         if self.nvml:
             self.t.join()
+        sys.setswitchinterval(self._switch)
 
     def summary(self):
         if not self.nvml:
@@ -350,11 +355,19 @@ def time_decode(w, device, K, warmup):
         call(i)
     torch.cuda.synchronize()
 
+    # A decode call is short on the GPU and longer than that on the host
+    # (Python, argument checks, the launch), so before each timed call the
+    # stream is held by a GPU-side delay (outside the events): the call is
+    # enqueued before the stream reaches it, and the events time the device.
+    def hold(n=1):
+        torch.cuda._sleep(200_000 * n)
+
     def timed(prep):
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(K)]
         for i in range(K):
             prep(i)
+            hold()
             ev[i][0].record()
             call(i)
             ev[i][1].record()
@@ -370,6 +383,7 @@ def time_decode(w, device, K, warmup):
         cold_ms = timed(lambda i: flush.fill_(i & 0xFF))
     read_ms = timed(lambda i: flush.view(torch.int64).sum())
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    hold(K)  # every call is enqueued before the stream reaches e0
     e0.record()
     for i in range(K):
         call(i)
@@ -912,11 +926,19 @@ def ssd_decode_bench(args):
     torch.cuda.synchronize()
     K = args.steps
 
+    # A decode call is short on the GPU and longer than that on the host
+    # (Python, argument checks, the launch), so before each timed call the
+    # stream is held by a GPU-side delay (outside the events): the call is
+    # enqueued before the stream reaches it, and the events time the device.
+    def hold(n=1):
+        torch.cuda._sleep(200_000 * n)
+
     def timed(prep):
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(K)]
         for i in range(K):
             prep(i)
+            hold()
             ev[i][0].record()
             call(i)
             ev[i][1].record()
@@ -928,6 +950,7 @@ def ssd_decode_bench(args):
         cold_ms = timed(lambda i: flush.fill_(i & 0xFF))
     read_ms = timed(lambda i: flush.view(torch.int64).sum())
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    hold(K)  # every call is enqueued before the stream reaches e0
     e0.record()
     for i in range(K):
         call(i)

@@ -918,100 +918,154 @@ __global__ void __launch_bounds__(256) scan_compose_kernel(const ScanParams p, i
 // across the LPC lanes by shuffles. Every load of a thread is issued before
 // any arithmetic, so each thread makes a single round trip to memory: the
 // kernel is otherwise bound by the latency of its waves, not by bandwidth.
+// States per thread of the one-shot decode kernel (8: two groups of four,
+// where N allows) and batch rows per thread (the row of A is loaded once for
+// them: with the state it is most of a thread's bytes in flight).
+#ifndef SSM_DEC_SPT8
+#define SSM_DEC_SPT8 1
+#endif
+#ifndef SSM_DEC_RB
+#define SSM_DEC_RB 2
+#endif
+template <int N>
+struct DecShape {
+  static constexpr int SPT = (SSM_DEC_SPT8 && N >= 8) ? 8 : (N % 4 == 0 ? 4 : 2);
+  static constexpr int GS = SPT >= 4 ? 4 : SPT;  // states per partial sum of y
+  static constexpr int NG = SPT / GS;            // partial sums per thread and row
+  static constexpr int LPC = N / SPT;            // lanes per channel
+  static constexpr int RB = SSM_DEC_RB;          // batch rows per thread
+  static_assert(LPC <= 32 && (LPC & (LPC - 1)) == 0, "lanes per channel must divide a warp");
+};
+
 template <typename IOT, int N, bool kZoh>
 __global__ void __launch_bounds__(256) decode_kernel(const DecodeParams p) {
   using IO = Io<IOT>;
+  using S = DecShape<N>;
   constexpr bool kFast = std::is_same<IOT, uint16_t>::value;
-  constexpr int SPT = (N % 4 == 0) ? 4 : 2;
-  constexpr int LPC = N / SPT;
-  static_assert(LPC <= 32 && (LPC & (LPC - 1)) == 0, "lanes per channel must divide a warp");
-  const size_t gtid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const size_t chan = gtid / LPC;  // b * dim + d
-  const int lane_in = (int)(gtid % LPC);
-  const size_t nchan = (size_t)p.batch * p.dim;
-  const bool valid = chan < nchan;
-  const size_t cc = valid ? chan : 0;
-  const int b = (int)(cc / p.dim), d = (int)(cc % p.dim);
+  constexpr int SPT = S::SPT, GS = S::GS, NG = S::NG, LPC = S::LPC, RB = S::RB;
+  // grid: x covers one batch row's channels (LPC lanes each), y groups of RB
+  // batch rows; no division by the run-time dim
+  const int tl = blockIdx.x * blockDim.x + threadIdx.x;
+  const int lane_in = tl % LPC;
+  const bool valid = tl / LPC < p.dim;
+  const int d = valid ? tl / LPC : p.dim - 1;
+  const int b0 = blockIdx.y * RB;
 
   // ---- all loads first ----
-  float* hp = p.state + cc * N + lane_in * SPT;
   const float* Ar = p.A + (size_t)d * N + lane_in * SPT;
-  const IOT* Bp = reinterpret_cast<const IOT*>(p.B) + (size_t)b * N + lane_in * SPT;
-  const IOT* Cp = reinterpret_cast<const IOT*>(p.C) + (size_t)b * N + lane_in * SPT;
-  float h[SPT], a[SPT], bb[SPT], cv[SPT];
-  if constexpr (SPT == 4) {
-    const float4 t4 = *reinterpret_cast<const float4*>(hp);
-    h[0] = t4.x; h[1] = t4.y; h[2] = t4.z; h[3] = t4.w;
-    const float4 a4 = __ldg(reinterpret_cast<const float4*>(Ar));
-    a[0] = a4.x; a[1] = a4.y; a[2] = a4.z; a[3] = a4.w;
-    const float4 b4 = IO::load4(Bp), c4 = IO::load4(Cp);
-    bb[0] = b4.x; bb[1] = b4.y; bb[2] = b4.z; bb[3] = b4.w;
-    cv[0] = c4.x; cv[1] = c4.y; cv[2] = c4.z; cv[3] = c4.w;
+  float a[SPT], h[RB][SPT], bb[RB][SPT], cv[RB][SPT], xv[RB], draw[RB], zz[RB];
+  if constexpr (SPT % 4 == 0) {
+#pragma unroll
+    for (int v = 0; v < SPT; v += 4) {
+      const float4 a4 = __ldg(reinterpret_cast<const float4*>(Ar + v));
+      a[v] = a4.x; a[v + 1] = a4.y; a[v + 2] = a4.z; a[v + 3] = a4.w;
+    }
   } else {
-    const float2 t2 = *reinterpret_cast<const float2*>(hp);
-    h[0] = t2.x; h[1] = t2.y;
     const float2 a2 = __ldg(reinterpret_cast<const float2*>(Ar));
     a[0] = a2.x; a[1] = a2.y;
-    const float2 b2 = IO::load2(Bp), c2 = IO::load2(Cp);
-    bb[0] = b2.x; bb[1] = b2.y; cv[0] = c2.x; cv[1] = c2.y;
   }
-  const float xv = IO::load(reinterpret_cast<const IOT*>(p.x) + cc);
-  const float draw = IO::load(reinterpret_cast<const IOT*>(p.delta) + cc);
+#pragma unroll
+  for (int r = 0; r < RB; ++r) {
+    const int b = min(b0 + r, p.batch - 1);  // rows past the end load row batch-1
+    const size_t cc = (size_t)b * p.dim + d;
+    const float* hp = p.state + cc * N + lane_in * SPT;
+    const IOT* Bp = reinterpret_cast<const IOT*>(p.B) + (size_t)b * N + lane_in * SPT;
+    const IOT* Cp = reinterpret_cast<const IOT*>(p.C) + (size_t)b * N + lane_in * SPT;
+    if constexpr (SPT % 4 == 0) {
+#pragma unroll
+      for (int v = 0; v < SPT; v += 4) {
+        const float4 t4 = *reinterpret_cast<const float4*>(hp + v);
+        h[r][v] = t4.x; h[r][v + 1] = t4.y; h[r][v + 2] = t4.z; h[r][v + 3] = t4.w;
+        const float4 b4 = IO::load4(Bp + v), c4 = IO::load4(Cp + v);
+        bb[r][v] = b4.x; bb[r][v + 1] = b4.y; bb[r][v + 2] = b4.z; bb[r][v + 3] = b4.w;
+        cv[r][v] = c4.x; cv[r][v + 1] = c4.y; cv[r][v + 2] = c4.z; cv[r][v + 3] = c4.w;
+      }
+    } else {
+      const float2 t2 = *reinterpret_cast<const float2*>(hp);
+      h[r][0] = t2.x; h[r][1] = t2.y;
+      const float2 b2 = IO::load2(Bp), c2 = IO::load2(Cp);
+      bb[r][0] = b2.x; bb[r][1] = b2.y; cv[r][0] = c2.x; cv[r][1] = c2.y;
+    }
+    xv[r] = IO::load(reinterpret_cast<const IOT*>(p.x) + cc);
+    draw[r] = IO::load(reinterpret_cast<const IOT*>(p.delta) + cc);
+    zz[r] = p.z ? IO::load(reinterpret_cast<const IOT*>(p.z) + cc) : 0.f;
+  }
   const float bias = p.bias ? p.bias[d] : 0.f;
   const float Dd = p.D ? p.D[d] : 0.f;
-  const float zz = p.z ? IO::load(reinterpret_cast<const IOT*>(p.z) + cc) : 0.f;
 
-  // ---- arithmetic ----
-  const float v = draw + bias;
-  float dt;
-  if (!p.softplus) {
-    dt = v;
-  } else if constexpr (kFast) {
-    dt = v > kSoftplusCut ? v : kLn2 * lg2_approx(1.f + ex2_approx(v * kLog2e));
-  } else {
-    dt = v > kSoftplusCut ? v : log1pf(expf(v));
-  }
-  const float dx = dt * xv;
-  const float dtl = kFast ? dt * kLog2e : dt;
-  float acc = 0.f;
+  // ---- arithmetic, row by row ----
 #pragma unroll
-  for (int k = 0; k < SPT; ++k) {
-    const float e = kFast ? ex2_approx(dtl * a[k]) : expf(dtl * a[k]);
-    if constexpr (kZoh) {
-      // exact ZOH input: x B_n (exp(Delta A_n) - 1) / A_n (Delta where A_n = 0)
-      const float coef = a[k] == 0.f ? dt
-                         : kFast     ? (e - 1.f) * rcp_approx(a[k])
-                                     : expm1f(dt * a[k]) / a[k];
-      h[k] = fmaf(e, h[k], xv * coef * bb[k]);
+  for (int r = 0; r < RB; ++r) {
+    const float v = draw[r] + bias;
+    float dt;
+    if (!p.softplus) {
+      dt = v;
+    } else if constexpr (kFast) {
+      dt = v > kSoftplusCut ? v : kLn2 * lg2_approx(1.f + ex2_approx(v * kLog2e));
     } else {
-      h[k] = fmaf(e, h[k], dx * bb[k]);
+      dt = v > kSoftplusCut ? v : log1pf(expf(v));
     }
-    acc = fmaf(cv[k], h[k], acc);
-  }
+    const float dx = dt * xv[r];
+    const float dtl = kFast ? dt * kLog2e : dt;
+    float part[NG];
 #pragma unroll
-  for (int off = LPC / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if (!valid) return;
-  if constexpr (SPT == 4) {
-    *reinterpret_cast<float4*>(hp) = make_float4(h[0], h[1], h[2], h[3]);
-  } else {
-    *reinterpret_cast<float2*>(hp) = make_float2(h[0], h[1]);
-  }
-  if (lane_in == 0) {
-    float yy = fmaf(Dd, xv, acc);
-    if (p.z) {
-      if constexpr (kFast) {
-        const float hz = 0.5f * zz;
-        yy *= fmaf(hz, tanh_approx(hz), hz);
-      } else {
-        yy *= zz / (1.f + expf(-zz));
+    for (int g = 0; g < NG; ++g) {
+      float acc = 0.f;
+#pragma unroll
+      for (int j = 0; j < GS; ++j) {
+        const int k = g * GS + j;
+        const float e = kFast ? ex2_approx(dtl * a[k]) : expf(dtl * a[k]);
+        if constexpr (kZoh) {
+          // exact ZOH input: x B_n (exp(Delta A_n) - 1) / A_n (Delta where A_n = 0)
+          const float coef = a[k] == 0.f ? dt
+                             : kFast     ? (e - 1.f) * rcp_approx(a[k])
+                                         : expm1f(dt * a[k]) / a[k];
+          h[r][k] = fmaf(e, h[r][k], xv[r] * coef * bb[r][k]);
+        } else {
+          h[r][k] = fmaf(e, h[r][k], dx * bb[r][k]);
+        }
+        acc = fmaf(cv[r][k], h[r][k], acc);
       }
+      part[g] = acc;
     }
-    IO::store(reinterpret_cast<IOT*>(p.y) + cc, yy);
+    // y: the partial sums of the channel's N / GS groups of GS states combined
+    // by the same pairing as an xor tree over one group per lane (group g with
+    // g ^ off, off = N / (2 GS) .. 1), so every kernel sums in the same order
+#pragma unroll
+    for (int off = N / GS / 2; off >= NG && off >= 1; off >>= 1)
+#pragma unroll
+      for (int g = 0; g < NG; ++g) part[g] += __shfl_xor_sync(0xffffffffu, part[g], off / NG);
+    float acc = part[0];
+    if constexpr (NG == 2) acc = part[0] + part[1];
+    const int b = b0 + r;
+    if (!valid || b >= p.batch) continue;
+    const size_t cc = (size_t)b * p.dim + d;
+    float* hp = p.state + cc * N + lane_in * SPT;
+#pragma unroll
+    for (int v = 0; v < SPT; v += (SPT % 4 == 0 ? 4 : 2)) {
+      if constexpr (SPT % 4 == 0)
+        *reinterpret_cast<float4*>(hp + v) =
+            make_float4(h[r][v], h[r][v + 1], h[r][v + 2], h[r][v + 3]);
+      else
+        *reinterpret_cast<float2*>(hp + v) = make_float2(h[r][v], h[r][v + 1]);
+    }
+    if (lane_in == 0) {
+      float yy = fmaf(Dd, xv[r], acc);
+      if (p.z) {
+        if constexpr (kFast) {
+          const float hz = 0.5f * zz[r];
+          yy *= fmaf(hz, tanh_approx(hz), hz);
+        } else {
+          yy *= zz[r] / (1.f + expf(-zz[r]));
+        }
+      }
+      IO::store(reinterpret_cast<IOT*>(p.y) + cc, yy);
+    }
   }
 }
 
 // -------------------------------------------------------------------------
-// Decode, pipelined: the same step as decode_kernel for the common aligned
+// Decode, pipelined (SSM_DECODE_PIPELINED=1): the same step as decode_kernel for the common aligned
 // shapes, but a CTA walks tiles of kDecTB batch rows x (1024 / N) channels
 // (16 KB of state) and brings the next tile's state, A rows and inputs into
 // shared memory by cp.async while it computes the current one. The state is
@@ -1183,11 +1237,13 @@ cudaError_t ensure_smem_attr(const void* kernel, int smem) {
   return e;
 }
 
-// SSM_DECODE_ONE_SHOT=1 in the environment keeps every decode step on the
-// one-shot kernel (the pipelined one is used where the shape allows).
+// SSM_DECODE_PIPELINED=1 in the environment runs the pipelined kernel where
+// the shape allows; by default every decode step takes the one-shot kernel,
+// which measured faster (it is issue-bound, and the pipelined kernel adds the
+// staging's instructions and barriers).
 bool decode2_enabled() {
-  const char* v = getenv("SSM_DECODE_ONE_SHOT");
-  return !(v && v[0] == '1');
+  const char* v = getenv("SSM_DECODE_PIPELINED");
+  return v && v[0] == '1';
 }
 
 template <typename IOT, int N, int CPT, bool kZoh>
@@ -1355,20 +1411,20 @@ cudaError_t launch_decode_io(const DecodeParams& p, int dstate, cudaStream_t str
     }
     if (e != cudaSuccess || used) return e;
   }
-  const size_t chans = (size_t)p.batch * p.dim;
   auto go = [&](auto kernel, int lpc) -> cudaError_t {
-    const size_t threads = chans * lpc;
-    const unsigned blocks = (unsigned)((threads + 255) / 256);
-    kernel<<<blocks, 256, 0, stream>>>(p);
+    constexpr int RB = SSM_DEC_RB;
+    const dim3 grid((unsigned)(((size_t)p.dim * lpc + 255) / 256),
+                    (unsigned)((p.batch + RB - 1) / RB));
+    kernel<<<grid, 256, 0, stream>>>(p);
     return cudaGetLastError();
   };
   switch (dstate) {
-    case 2: return go(decode_kernel<IOT, 2, kZoh>, 1);
-    case 4: return go(decode_kernel<IOT, 4, kZoh>, 1);
-    case 8: return go(decode_kernel<IOT, 8, kZoh>, 2);
-    case 16: return go(decode_kernel<IOT, 16, kZoh>, 4);
-    case 32: return go(decode_kernel<IOT, 32, kZoh>, 8);
-    case 64: return go(decode_kernel<IOT, 64, kZoh>, 16);
+    case 2: return go(decode_kernel<IOT, 2, kZoh>, DecShape<2>::LPC);
+    case 4: return go(decode_kernel<IOT, 4, kZoh>, DecShape<4>::LPC);
+    case 8: return go(decode_kernel<IOT, 8, kZoh>, DecShape<8>::LPC);
+    case 16: return go(decode_kernel<IOT, 16, kZoh>, DecShape<16>::LPC);
+    case 32: return go(decode_kernel<IOT, 32, kZoh>, DecShape<32>::LPC);
+    case 64: return go(decode_kernel<IOT, 64, kZoh>, DecShape<64>::LPC);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -113,7 +113,7 @@ def test_pipelined_decode_shapes(monkeypatch, N, io, optional, batch, dim):
     """Shapes the pipelined decode kernel takes (batch a multiple of 4, whole
     tiles of 1024 / N channels, 16-byte aligned rows): against the oracle step
     by step, and bit for bit against the one-shot kernel
-    (SSM_DECODE_ONE_SHOT=1), which does the same arithmetic."""
+    (the default), which does the same arithmetic."""
     from selective_state_space_39_b200 import ssm_state_update
     steps = 6 if batch < 96 else 3
     seed = 100 + N + (7 if optional else 0)
@@ -128,12 +128,36 @@ def test_pipelined_decode_shapes(monkeypatch, N, io, optional, batch, dim):
         kw = dict(D=const["D"], z=inp["z"], delta_bias=const["delta_bias"]) if optional else {}
         args = (dev(inp["x"]), dev(inp["delta"]), dev(A), dev(inp["B"]), dev(inp["C"]))
         dkw = {k: dev(v) for k, v in kw.items()}
-        monkeypatch.delenv("SSM_DECODE_ONE_SHOT", raising=False)
+        monkeypatch.setenv("SSM_DECODE_PIPELINED", "1")
         y2 = ssm_state_update(s2, *args, **dkw)
-        monkeypatch.setenv("SSM_DECODE_ONE_SHOT", "1")
+        monkeypatch.delenv("SSM_DECODE_PIPELINED")
         y1 = ssm_state_update(s1, *args, **dkw)
-        monkeypatch.delenv("SSM_DECODE_ONE_SHOT")
         yr = oracle.state_update(ref, inp["x"], inp["delta"], A, inp["B"], inp["C"], io=io, **kw)
         assert rel_err(host(y2), yr) <= TOL[io], f"step {step}"
         assert torch.equal(y1, y2) and torch.equal(s1, s2), f"step {step}"
     assert rel_err(host(s2), ref) <= TOL[io]
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("batch,dim,N,io", [(65535, 6, 4, "f32"), (3, 100, 16, "bf16")])
+def test_one_shot_decode_grid_edges(monkeypatch, batch, dim, N, io):
+    """The one-shot decode kernel's grid: the largest batch the library takes
+    (one grid row per batch row) and a partial last block of channels,
+    against the oracle step."""
+    from selective_state_space_39_b200 import ssm_state_update
+    monkeypatch.delenv("SSM_DECODE_PIPELINED", raising=False)
+    seed = 500 + N
+    rng = np.random.default_rng(seed)
+    A = (-rng.uniform(0.2, 3.0, (dim, N))).astype(np.float32)
+    const = gen.decode_constants(dim, N, seed)
+    h0 = rng.standard_normal((batch, dim, N)).astype(np.float32)
+    ref = h0.astype(np.float64)
+    s = dev(h0).clone()
+    for step in range(2):
+        inp = gen.make_decode_inputs(batch, dim, N, io, seed, step)
+        kw = dict(D=const["D"], z=inp["z"], delta_bias=const["delta_bias"])
+        y = ssm_state_update(s, dev(inp["x"]), dev(inp["delta"]), dev(A), dev(inp["B"]),
+                             dev(inp["C"]), **{k: dev(v) for k, v in kw.items()})
+        yr = oracle.state_update(ref, inp["x"], inp["delta"], A, inp["B"], inp["C"], io=io, **kw)
+        assert rel_err(host(y), yr) <= TOL[io], f"step {step}"
+    assert rel_err(host(s), ref) <= TOL[io]
