@@ -69,23 +69,28 @@ template <typename IOT, int N>
 __global__ void __launch_bounds__(256) ssd_decode_kernel(const SsdDecodeParams p) {
   using IO = Io<IOT>;
   constexpr int SPT = N / 32;
-  const size_t warp_id = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  // bf16 io takes the MUFU approximations (as the other kernels), fp32 io expf / log1pf
+  constexpr bool kFast = std::is_same<IOT, uint16_t>::value;
+  // row indices fit 32 bits (the entry point admits at most 2^26 rows): the
+  // (b, h) of a row comes from 32-bit divisions, far cheaper than 64-bit ones
+  const uint32_t warp_id = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  const size_t rows = (size_t)p.batch * p.nheads * p.headdim;
-  const size_t row0 = warp_id * kRows;
+  const uint32_t P = (uint32_t)p.headdim, H = (uint32_t)p.nheads;
+  const uint32_t rows = (uint32_t)p.batch * H * P;
+  const uint32_t row0 = warp_id * kRows;
   if (row0 >= rows) return;  // warp-uniform
 
   // ---- every load of every row first (rows past the end repeat the last one)
   float s[kRows][SPT], bb[kRows][SPT], cv[kRows][SPT], xv[kRows], raw[kRows], bias[kRows],
       Ah[kRows], Dh[kRows];
-  size_t rr[kRows];
+  uint32_t rr[kRows];
 #pragma unroll
   for (int r = 0; r < kRows; ++r) {
     rr[r] = row0 + r < rows ? row0 + r : rows - 1;
-    const size_t bh = rr[r] / p.headdim;
-    const int h = (int)(bh % p.nheads);
-    const size_t b = bh / p.nheads;
-    VecLoad<float, SPT>::run(p.state + rr[r] * N + lane * SPT, s[r]);
+    const uint32_t bh = rr[r] / P;
+    const int h = (int)(bh % H);
+    const size_t b = bh / H;
+    VecLoad<float, SPT>::run(p.state + (size_t)rr[r] * N + lane * SPT, s[r]);
     VecLoad<IOT, SPT>::run(static_cast<const IOT*>(p.B) + b * N + lane * SPT, bb[r]);
     VecLoad<IOT, SPT>::run(static_cast<const IOT*>(p.C) + b * N + lane * SPT, cv[r]);
     xv[r] = IO::load(static_cast<const IOT*>(p.x) + rr[r]);
@@ -99,8 +104,10 @@ __global__ void __launch_bounds__(256) ssd_decode_kernel(const SsdDecodeParams p
 #pragma unroll
   for (int r = 0; r < kRows; ++r) {
     const float v = raw[r] + bias[r];
-    const float d = p.softplus ? (v > kSoftplusCut ? v : log1pf(expf(v))) : v;
-    const float a = expf(d * Ah[r]);
+    float d = v;
+    if (p.softplus && v <= kSoftplusCut)
+      d = kFast ? kLn2 * lg2_approx(1.f + ex2_approx(v * kLog2e)) : log1pf(expf(v));
+    const float a = kFast ? ex2_approx(d * Ah[r] * kLog2e) : expf(d * Ah[r]);
     const float dx = d * xv[r];
     float acc = 0.f;
 #pragma unroll
@@ -111,7 +118,7 @@ __global__ void __launch_bounds__(256) ssd_decode_kernel(const SsdDecodeParams p
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
     if (row0 + r < rows) {
-      store_state<SPT>(p.state + rr[r] * N + lane * SPT, s[r]);
+      store_state<SPT>(p.state + (size_t)rr[r] * N + lane * SPT, s[r]);
       if (lane == 0) IO::store(static_cast<IOT*>(p.y) + rr[r], fmaf(Dh[r], xv[r], acc));
     }
   }
