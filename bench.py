@@ -150,6 +150,12 @@ class ClockSampler:
                 idx = int(vis.split(",")[device_index])
             self.h = pynvml.nvmlDeviceGetHandleByIndex(idx)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            # the first queries are slow (lazy set-up): made here, outside the
+            # timed region, so that sampling starts at once
+            get_reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                getattr(pynvml, "nvmlDeviceGetCurrentClocksThrottleReasons")
+            pynvml.nvmlDeviceGetClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            get_reasons(self.h)
         except Exception as e:  # pragma: no cover - depends on the machine
             self.nvml, self.error = None, f"nvml unavailable: {e}"
         self.t = threading.Thread(target=self._run, daemon=True)

@@ -348,9 +348,10 @@ template <typename IOT, int W>
 __global__ void __launch_bounds__(256) conv_update_kernel(const ConvParams p) {
   using IO = Io<IOT>;
   constexpr bool kFast = std::is_same<IOT, uint16_t>::value;
-  const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= (size_t)p.batch * p.dim) return;
-  const int d = (int)(i % p.dim);
+  // grid: x over the channels, y over the batch rows (no division per thread)
+  const int d = blockIdx.x * blockDim.x + threadIdx.x;
+  if (d >= p.dim) return;
+  const size_t i = (size_t)blockIdx.y * p.dim + d;
   IOT* st = reinterpret_cast<IOT*>(p.out) + i * (W - 1);  // the state (in/out)
   float sv[W - 1];
 #pragma unroll
@@ -419,8 +420,7 @@ cudaError_t launch_w(const ConvParams& p, bool backward, cudaStream_t stream) {
 
 template <typename IOT>
 cudaError_t launch_update_io(const ConvParams& p, cudaStream_t stream) {
-  const size_t n = (size_t)p.batch * p.dim;
-  const unsigned blocks = (unsigned)((n + 255) / 256);
+  const dim3 blocks((unsigned)((p.dim + 255) / 256), (unsigned)p.batch);
   switch (p.width) {
     case 2: conv_update_kernel<IOT, 2><<<blocks, 256, 0, stream>>>(p); break;
     case 3: conv_update_kernel<IOT, 3><<<blocks, 256, 0, stream>>>(p); break;
