@@ -17,7 +17,7 @@
 // Design (B200). Like the forward, the work is FP32-issue bound; memory is
 // used to avoid recomputation where it is cheaper than arithmetic:
 //
-//  * Four launches, none of which waits on another CTA:
+//  * Five launches, none of which waits on another CTA:
 //    1. carry: per (segment, channel block, batch row) one forward sweep from
 //       a zero state, storing the state at every 4-step tile start (and the
 //       summed decay exponent there) and the segment's end state; the same
@@ -31,9 +31,10 @@
 //       entry state is its checkpoint plus exp(A_n Q) times the segment's
 //       entering state; the tile's 4 steps are recomputed into a register
 //       history, then the adjoint runs backwards through them.
-//    4. reduce: dB and dC (sums over channels) from per-CTA partials, dA, dD,
-//       dbias (sums over batch rows and segments) from per-segment partials,
-//       in a fixed order, so results do not depend on scheduling.
+//    4. reduce (two launches): dB and dC (sums over channels) from per-CTA
+//       partials, dA, dD, dbias (sums over batch rows and segments) from
+//       per-segment partials, in a fixed order, so results do not depend on
+//       scheduling.
 //  * One channel per thread with its whole state in registers; the sums over
 //    n are in-thread. The sums over channels (dB, dC) go through shared
 //    memory: every thread writes its 2N values per step, then each thread
@@ -405,19 +406,47 @@ __global__ void __launch_bounds__(256) bwd_compose_kernel(const BwdParams p, int
     const int n = (int)((i / p.dim) % N);
     const int b = (int)(i / ((size_t)p.dim * N));
     const float An = p.A[(size_t)d * N + n];
+    // the loads of 8 segments are issued before their 8 dependent steps
+    constexpr int G = 8;
     float h = p.h0 ? p.h0[((size_t)b * p.dim + d) * N + n] : 0.f;
-    for (int s = 0; s < p.nseg; ++s) {
-      const size_t sb = (size_t)b * p.nseg + s;
-      const size_t at = (sb * N + n) * p.dim + d;
-      p.ws_hin[at] = h;
-      if (s < p.nseg - 1) h = fmaf(exp_u<kFast>(p.ws_qseg[sb * p.dim + d] * An), h, p.ws_hloc[at]);
+    for (int s0 = 0; s0 < p.nseg; s0 += G) {
+      float qv[G], lc[G];
+#pragma unroll
+      for (int j = 0; j < G; ++j) {
+        const int s = s0 + j;
+        const size_t sb = (size_t)b * p.nseg + s;
+        const bool step = s < p.nseg - 1;  // the last segment's carry is not needed
+        qv[j] = step ? p.ws_qseg[sb * p.dim + d] : 0.f;
+        lc[j] = step ? p.ws_hloc[(sb * N + n) * p.dim + d] : 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < G; ++j) {
+        const int s = s0 + j;
+        if (s >= p.nseg) break;
+        const size_t sb = (size_t)b * p.nseg + s;
+        p.ws_hin[(sb * N + n) * p.dim + d] = h;
+        if (s < p.nseg - 1) h = fmaf(exp_u<kFast>(qv[j] * An), h, lc[j]);
+      }
     }
     float mu = p.dh_last ? p.dh_last[((size_t)b * p.dim + d) * N + n] : 0.f;
-    for (int s = p.nseg - 1; s >= 0; --s) {
-      const size_t sb = (size_t)b * p.nseg + s;
-      const size_t at = (sb * N + n) * p.dim + d;
-      p.ws_muin[at] = mu;
-      if (s > 0) mu = fmaf(exp_u<kFast>(p.ws_qseg[sb * p.dim + d] * An), mu, p.ws_mloc[at]);
+    for (int s0 = p.nseg - 1; s0 >= 0; s0 -= G) {
+      float qv[G], lc[G];
+#pragma unroll
+      for (int j = 0; j < G; ++j) {
+        const int s = s0 - j;
+        const size_t sb = (size_t)b * p.nseg + (s > 0 ? s : 0);
+        const bool step = s > 0;  // the first segment's carry is not needed
+        qv[j] = step ? p.ws_qseg[sb * p.dim + d] : 0.f;
+        lc[j] = step ? p.ws_mloc[(sb * N + n) * p.dim + d] : 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < G; ++j) {
+        const int s = s0 - j;
+        if (s < 0) break;
+        const size_t sb = (size_t)b * p.nseg + s;
+        p.ws_muin[(sb * N + n) * p.dim + d] = mu;
+        if (s > 0) mu = fmaf(exp_u<kFast>(qv[j] * An), mu, lc[j]);
+      }
     }
   }
 }
@@ -714,41 +743,70 @@ __global__ void __launch_bounds__(MainShape<N>::NTHR, MainShape<N>::kMinBlocks)
 }
 
 // ---------------------------------------------------------------------------
-// 4. reduce: dB, dC over channel blocks; dA, dD, dbias over (batch, segment).
-__global__ void __launch_bounds__(256) bwd_reduce_kernel(const BwdParams p, int N) {
-  const int V = 2 * N;
-  const size_t n_bc = (size_t)p.batch * p.seqlen * V;
-  const size_t n_a = (size_t)p.dim * N;
-  const size_t total = n_bc + n_a + (size_t)p.dim;
-  const size_t bs = (size_t)p.batch * p.nseg;
-  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+// 4. reduce, two launches in a fixed order of summation (results do not
+// depend on scheduling). dB, dC: per (b, t, v) the sum over channel blocks,
+// one batch row per grid row (V = 2N a compile-time power of two: no
+// division by a run-time size).
+template <int N>
+__global__ void __launch_bounds__(256) bwd_reduce_bc_kernel(const BwdParams p) {
+  constexpr int V = 2 * N;
+  const int b = blockIdx.y;
+  const size_t per_row = (size_t)p.seqlen * V;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < per_row;
        i += (size_t)gridDim.x * blockDim.x) {
-    if (i < n_bc) {
-      const int v = (int)(i % V);
-      const size_t bt = i / V;  // b * L + t
-      const int t = (int)(bt % p.seqlen);
-      const int b = (int)(bt / p.seqlen);
-      float acc = 0.f;
-      for (int k = 0; k < p.dblocks; ++k)
-        acc += p.ws_dbc[(((size_t)b * p.dblocks + k) * p.seqlen + t) * V + v];
-      if (v < N) p.dB[bt * N + v] = acc;
-      else p.dC[bt * N + (v - N)] = acc;
-    } else if (i < n_bc + n_a) {
-      const size_t j = i - n_bc;  // d * N + n
-      const int n = (int)(j % N);
-      const int d = (int)(j / N);
-      float acc = 0.f;
-      for (size_t s = 0; s < bs; ++s) acc += p.ws_dA[(s * N + n) * p.dim + d];
-      p.dA[j] = acc;
+    const int v = (int)(i % V);
+    const size_t t = i / V;
+    float acc = 0.f;
+    for (int k = 0; k < p.dblocks; ++k)
+      acc += p.ws_dbc[(((size_t)b * p.dblocks + k) * p.seqlen + t) * V + v];
+    const size_t bt = (size_t)b * p.seqlen + t;
+    if (v < N) p.dB[bt * N + v] = acc;
+    else p.dC[bt * N + (v - N)] = acc;
+  }
+}
+
+// dA, dD, dbias: sums over the (batch, segment) partials. A CTA takes 32
+// consecutive channels (lanes: coalesced reads) and one state n (grid row n;
+// row N: dD and dbias); its 8 warps each sum every 8th partial, and the 8
+// slices are added in a fixed order (results do not depend on scheduling).
+template <int N>
+__global__ void __launch_bounds__(256) bwd_reduce_par_kernel(const BwdParams p) {
+  __shared__ float part[2][8][33];
+  const int lane = threadIdx.x & 31, slice = threadIdx.x >> 5;
+  const int d = blockIdx.x * 32 + lane;
+  const int n = blockIdx.y;
+  const bool valid = d < p.dim;
+  const size_t bs = (size_t)p.batch * p.nseg;
+  float a1 = 0.f, a2 = 0.f;
+  if (valid) {
+    if (n < N) {
+      const float* src = p.ws_dA + (size_t)n * p.dim + d;  // [s][N][dim]
+      const size_t stride = (size_t)N * p.dim;
+#pragma unroll 4
+      for (size_t s = slice; s < bs; s += 8) a1 += src[s * stride];
     } else {
-      const int d = (int)(i - n_bc - n_a);
-      float a1 = 0.f, a2 = 0.f;
-      for (size_t s = 0; s < bs; ++s) {
+#pragma unroll 4
+      for (size_t s = slice; s < bs; s += 8) {
         a1 += p.ws_dD[s * p.dim + d];
         a2 += p.ws_dbias[s * p.dim + d];
       }
-      if (p.dD) p.dD[d] = a1;
-      if (p.dbias) p.dbias[d] = a2;
+    }
+  }
+  part[0][slice][lane] = a1;
+  part[1][slice][lane] = a2;
+  __syncthreads();
+  if (slice == 0 && valid) {
+    float r1 = 0.f, r2 = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      r1 += part[0][k][lane];
+      r2 += part[1][k][lane];
+    }
+    if (n < N) {
+      p.dA[(size_t)d * N + n] = r1;
+    } else {
+      if (p.dD) p.dD[d] = r1;
+      if (p.dbias) p.dbias[d] = r2;
     }
   }
 }
@@ -786,8 +844,15 @@ cudaError_t launch_bwd_t(const BwdParams& p, cudaStream_t stream) {
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   bwd_main_kernel<IOT, N><<<grid, MainShape<N>::NTHR, main_bytes, stream>>>(p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const size_t red = (size_t)p.batch * p.seqlen * 2 * N + (size_t)p.dim * N + p.dim;
-  bwd_reduce_kernel<<<grid_for(red, 256), 256, 0, stream>>>(p, N);
+  {
+    const size_t per_row = (size_t)p.seqlen * 2 * N;
+    const int gx = std::max(1, std::min(grid_for(per_row, 256), 1 + 1184 / std::max(1, p.batch)));
+    bwd_reduce_bc_kernel<N><<<dim3((unsigned)gx, (unsigned)p.batch), 256, 0, stream>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  bwd_reduce_par_kernel<N><<<dim3((unsigned)((p.dim + 31) / 32), (unsigned)(N + 1)), 256, 0,
+                               stream>>>(p);
   return cudaGetLastError();
 }
 
