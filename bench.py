@@ -264,6 +264,13 @@ def time_scan(w, nb, b0, device, K, warmup, zoh=False, learned_a=False, sync=Non
                      delta_bias=d["delta_bias"], h0=d["h0"], y=y, h_last=h_last, workspace=ws,
                      zoh=zoh)
 
+    def step_rows(r0, r1):
+        """The same call on batch rows r0 .. r1 (rows are independent)."""
+        rows = lambda t: None if t is None else t[r0:r1]
+        ssm_scan_fwd(rows(d["x"]), rows(d["delta"]), d["A"], rows(d["B"]), rows(d["C"]),
+                     D=d["D"], z=rows(d["z"]), delta_bias=d["delta_bias"], h0=rows(d["h0"]),
+                     y=y[r0:r1], h_last=h_last[r0:r1], workspace=ws, zoh=zoh)
+
     for _ in range(max(3, warmup)):
         flush.fill_(1)
         step()
@@ -288,7 +295,8 @@ def time_scan(w, nb, b0, device, K, warmup, zoh=False, learned_a=False, sync=Non
         sync()
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     return {"step_ms": step_ms, "plan": plan, "inp": inp, "d": d, "y": y, "h_last": h_last,
-            "step": step, "clocks": sampler.summary() if sampler else None}
+            "step": step, "step_rows": step_rows,
+            "clocks": sampler.summary() if sampler else None}
 
 
 def scan_rooflines(w, nb, mean_s, clocks, zoh, plan, traffic):
@@ -1120,8 +1128,8 @@ def main():
     run = time_scan(w, nb, b0, device, args.steps, args.warmup, zoh=args.zoh,
                     learned_a=args.learned_a, sync=lambda: sdist.barrier(device),
                     sample_clocks=True)
-    step_ms, plan, inp, d, y, h_last, step = (run[k] for k in (
-        "step_ms", "plan", "inp", "d", "y", "h_last", "step"))
+    step_ms, plan, inp, d, y, h_last, step, step_rows = (run[k] for k in (
+        "step_ms", "plan", "inp", "d", "y", "h_last", "step", "step_rows"))
     dtype = y.dtype
     K = args.steps
     local_ms = sum(step_ms)
@@ -1145,24 +1153,51 @@ def main():
         h_host = torch.empty(h_last.shape, dtype=torch.float32).pin_memory()
         h2d = sum(t.numel() * t.element_size() for t in pinned.values() if t is not None)
         d2h = y_host.numel() * y_host.element_size() + h_host.numel() * h_host.element_size()
+        # The batch goes through in row chunks on three streams, so the copy of
+        # chunk j+1 in, the scan of chunk j and the copy of chunk j-1 out
+        # overlap (PCIe carries both directions at once); every byte of the
+        # step's inputs and results still crosses within the timed region.
+        batched = {"x", "delta", "z", "B", "C", "h0"}
+        nch = min(nb, 4)
+        bounds = [(nb * j // nch, nb * (j + 1) // nch) for j in range(nch)]
+        s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
         e_ms = []
         for i in range(args.e2e_steps + 2):
+            cur = torch.cuda.current_stream(device)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            for k, t in pinned.items():
-                if t is not None:
-                    d[k].copy_(t, non_blocking=True)
-            step()
-            y_host.copy_(y, non_blocking=True)
-            h_host.copy_(h_last, non_blocking=True)
-            e1.record()
+            e0.record(cur)
+            s_in.wait_stream(cur)
+            s_out.wait_stream(cur)
+            for j, (r0, r1) in enumerate(bounds):
+                with torch.cuda.stream(s_in):
+                    for k, t in pinned.items():
+                        if t is None:
+                            continue
+                        if k in batched:
+                            d[k][r0:r1].copy_(t[r0:r1], non_blocking=True)
+                        elif j == 0:
+                            d[k].copy_(t, non_blocking=True)
+                    ev_in = torch.cuda.Event()
+                    ev_in.record(s_in)
+                cur.wait_event(ev_in)
+                step_rows(r0, r1)
+                ev_c = torch.cuda.Event()
+                ev_c.record(cur)
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(ev_c)
+                    y_host[r0:r1].copy_(y[r0:r1], non_blocking=True)
+                    h_host[r0:r1].copy_(h_last[r0:r1], non_blocking=True)
+            cur.wait_stream(s_out)
+            e1.record(cur)
             e1.synchronize()
             if i >= 2:
                 e_ms.append(e0.elapsed_time(e1))
         e2e_ms = sdist.max_over_ranks(statistics.mean(e_ms), device)
         e2e = {"value": elements / (e2e_ms * 1e-3), "unit": "elements/s",
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
-    del run, d, y, h_last, step
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": e2e_ms,
+               "pipeline": f"{nch} batch-row chunks; copies in, scans and copies out overlap"}
+    del run, d, y, h_last, step, step_rows
 
     cpu = None
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
