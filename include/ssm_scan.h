@@ -366,9 +366,10 @@ int ssm_compose_carries(int64_t rank, int64_t batch, int64_t dim, int64_t dstate
  *
  * starting from h0[b,h] (or zero) and ending in h_last[b,h]. Computed chunk
  * by chunk on the tensor cores (bf16 operands, fp32 accumulation and state):
- * with dstate 64 or 128, an even nheads and 16-byte aligned h0 / h_last on
- * the fifth-generation (tcgen05) path, the state held in tensor memory;
- * otherwise (or with SSM_SSD_LEGACY=1) on the warp-level MMA path.
+ * with dstate 64 or 128, an even nheads, a 4-byte aligned dt and 16-byte
+ * aligned h0 / h_last on the fifth-generation (tcgen05) path, the state held
+ * in tensor memory; otherwise (or with SSM_SSD_LEGACY=1) on the warp-level
+ * MMA path.
  *   x, y     : (batch, seqlen, nheads, headdim) bf16 (io_dtype must be
  *              SSM_DTYPE_BF16); y must not overlap an input
  *   dt       : (batch, seqlen, nheads) bf16
