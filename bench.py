@@ -1246,9 +1246,10 @@ def main():
             per_config[name] = scan_summary(wc, rc, measured_traffic(wc.name))
             del rc
             torch.cuda.empty_cache()
+        # a decode call is ~20 us: at least 200 timed calls (a few ms in all)
         per_config[PER_CONFIG_DECODE] = decode_summary(
-            time_decode(gen.DECODE_WORKLOADS[PER_CONFIG_DECODE], device, args.steps,
-                        args.warmup))
+            time_decode(gen.DECODE_WORKLOADS[PER_CONFIG_DECODE], device, max(args.steps, 200),
+                        max(args.warmup, 10)))
 
     if rank == 0:
         line = {
