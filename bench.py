@@ -1183,8 +1183,10 @@ def main():
         # chunk j+1 in, the scan of chunk j and the copy of chunk j-1 out
         # overlap (PCIe carries both directions at once); every byte of the
         # step's inputs and results still crosses within the timed region.
+        # 4 chunks measured best on the 8 x 2048 x 1536 layer (3.39 ms a step,
+        # against 3.49 with 2 and 3.53 with 8; SSM_BENCH_E2E_CHUNKS sets it).
         batched = {"x", "delta", "z", "B", "C", "h0"}
-        nch = min(nb, 4)
+        nch = max(1, min(nb, int(os.environ.get("SSM_BENCH_E2E_CHUNKS", "4"))))
         bounds = [(nb * j // nch, nb * (j + 1) // nch) for j in range(nch)]
         s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
         e_ms = []
