@@ -37,6 +37,9 @@ def test_ssd_cost():
     tok = 4 * 4096
     assert nbytes == 2 * 2 * tok * 64 * 64 + 2 * 2 * tok * 128 + 2 * tok * 64 + 4 * 4 * 64 * 64 * 128 * 2
     assert flops == tok * 64 * (32 * 64 + 4 * 128 * 64) + tok * 32 * 128
+    # the tensor-core kernel's chunk of 128 steps
+    _, flops128 = bench.ssd_cost(w, Q=128)
+    assert flops128 == tok * 64 * (128 * 64 + 4 * 128 * 64) + tok * 128 * 128
 
 
 @pytest.mark.parametrize("workload", ["mamba130m_layer_b8_l2048_d1536",
