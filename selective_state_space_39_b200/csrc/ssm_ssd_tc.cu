@@ -433,7 +433,8 @@ __global__ void __launch_bounds__(kTThreads, 1)
     const int s_t = tid & 127, s_hh = (tid >> 7) & 1, s_ch = tid >> 8;
     // the epilogue: thread = (head, half of the head's 64 columns, step)
     const int e_hh = grp >> 1, e_ph = grp & 1;
-    const float D_o = p.D ? p.D[h0 + e_hh] : 0.f;
+    // the skip D x_t enters through G's diagonal: (G + diag(D)) X
+    const float D0 = p.D ? p.D[h0] : 0.f, D1 = p.D ? p.D[h0 + 1] : 0.f;
     // this warp's N / 4 columns of the state (TMEM lane = state row)
     auto ldq = [&](uint32_t a, float (&v)[kQN]) {
       if constexpr (kQN == 32) tc::ld32(a, v);
@@ -582,6 +583,11 @@ __global__ void __launch_bounds__(kTThreads, 1)
               if (sb0 + 1 > t) g0.y = 0.f;
               if (sb0 + 2 > t) g1.x = 0.f;
               if (sb0 + 3 > t) g1.y = 0.f;
+              const float Dh = hh ? D1 : D0;  // the diagonal entry s = t takes D
+              if (sb0 == t) g0.x += Dh;
+              if (sb0 + 1 == t) g0.y += Dh;
+              if (sb0 + 2 == t) g1.x += Dh;
+              if (sb0 + 3 == t) g1.y += Dh;
               gp[e / 2] = pack_bf16x2(g0.x, g0.y);
               gp[e / 2 + 1] = pack_bf16x2(g1.x, g1.y);
             }
@@ -608,8 +614,8 @@ __global__ void __launch_bounds__(kTThreads, 1)
       if (!ok) break;
       tc::fence_after_sync();
       if (c + 1 < nchunks) prep_state((c + 1) % 3);
-      // ---- y_t = Yd + e^{cum_t} Yo + D x_t (thread = (head, 32 of its columns,
-      //      step t)), written over x_t in shared memory, then stored by TMA
+      // ---- y_t = Yd + e^{cum_t} Yo (thread = (head, 32 of its columns, step t);
+      //      D x_t is in Yd), written over x_t in shared memory, then stored by TMA
       ok = work_vote(mbar_wait_bounded(bar_m, (uint32_t)(c & 1), p.wait_limit_ns));
       if (!ok) break;
       tc::fence_after_sync();
@@ -626,17 +632,13 @@ __global__ void __launch_bounds__(kTThreads, 1)
 #pragma unroll
           for (int j = 0; j < 32; j += 8) {
             uint4* const px = reinterpret_cast<uint4*>(xrow + tc::sw128(t, c0 + j));
-            const uint4 q = *px;
-            const float xv[8] = {bf16_lo(q.x), bf16_hi(q.x), bf16_lo(q.y), bf16_hi(q.y),
-                                 bf16_lo(q.z), bf16_hi(q.z), bf16_lo(q.w), bf16_hi(q.w)};
             float o[8];
 #pragma unroll
             for (int e = 0; e < 8; e += 2) {
               const float2 r = fma2(make_float2(ec, ec), make_float2(yo[j + e], yo[j + e + 1]),
                                     make_float2(yd[j + e], yd[j + e + 1]));
-              const float2 q2 = fma2(make_float2(D_o, D_o), make_float2(xv[e], xv[e + 1]), r);
-              o[e] = q2.x;
-              o[e + 1] = q2.y;
+              o[e] = r.x;
+              o[e + 1] = r.y;
             }
             *px = pack8(o);
           }
