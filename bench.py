@@ -228,6 +228,45 @@ PER_CONFIG_SCANS = ("mamba130m_layer_b8_l2048_d1536", "pythia1b_layer_b4_l4096_d
 PER_CONFIG_DECODE = "decode_b128_d4096_x1000"
 
 
+SCAN_BATCHED_INPUTS = ("x", "delta", "z", "B", "C", "h0")
+
+
+def pipelined_host_step(pinned, d, y, h_last, y_host, h_host, step_rows, nb, nch, streams):
+    """One end-to-end scan step from pinned host inputs to pinned host results,
+    enqueued on the current stream and two copy streams: the batch goes
+    through in `nch` row chunks, so the copy of chunk j+1 in, the scan of
+    chunk j and the copy of chunk j-1 out overlap (PCIe carries both
+    directions at once). Every byte of the step's inputs and results crosses.
+    Returns with the current stream waiting on the last copy out."""
+    import torch
+
+    s_in, s_out = streams
+    cur = torch.cuda.current_stream()
+    s_in.wait_stream(cur)
+    s_out.wait_stream(cur)
+    bounds = [(nb * j // nch, nb * (j + 1) // nch) for j in range(nch)]
+    for j, (r0, r1) in enumerate(bounds):
+        with torch.cuda.stream(s_in):
+            for k, t in pinned.items():
+                if t is None:
+                    continue
+                if k in SCAN_BATCHED_INPUTS:
+                    d[k][r0:r1].copy_(t[r0:r1], non_blocking=True)
+                elif j == 0:
+                    d[k].copy_(t, non_blocking=True)
+            ev_in = torch.cuda.Event()
+            ev_in.record(s_in)
+        cur.wait_event(ev_in)
+        step_rows(r0, r1)
+        ev_c = torch.cuda.Event()
+        ev_c.record(cur)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_c)
+            y_host[r0:r1].copy_(y[r0:r1], non_blocking=True)
+            h_host[r0:r1].copy_(h_last[r0:r1], non_blocking=True)
+    cur.wait_stream(s_out)
+
+
 def time_scan(w, nb, b0, device, K, warmup, zoh=False, learned_a=False, sync=None,
               sample_clocks=False):
     """K timed ssm_scan_fwd calls of workload `w` (batch rows b0 .. b0+nb of its
@@ -1179,43 +1218,17 @@ def main():
         h_host = torch.empty(h_last.shape, dtype=torch.float32).pin_memory()
         h2d = sum(t.numel() * t.element_size() for t in pinned.values() if t is not None)
         d2h = y_host.numel() * y_host.element_size() + h_host.numel() * h_host.element_size()
-        # The batch goes through in row chunks on three streams, so the copy of
-        # chunk j+1 in, the scan of chunk j and the copy of chunk j-1 out
-        # overlap (PCIe carries both directions at once); every byte of the
-        # step's inputs and results still crosses within the timed region.
         # 4 chunks measured best on the 8 x 2048 x 1536 layer (3.39 ms a step,
         # against 3.49 with 2 and 3.53 with 8; SSM_BENCH_E2E_CHUNKS sets it).
-        batched = {"x", "delta", "z", "B", "C", "h0"}
         nch = max(1, min(nb, int(os.environ.get("SSM_BENCH_E2E_CHUNKS", "4"))))
-        bounds = [(nb * j // nch, nb * (j + 1) // nch) for j in range(nch)]
-        s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+        streams = (torch.cuda.Stream(device), torch.cuda.Stream(device))
         e_ms = []
         for i in range(args.e2e_steps + 2):
             cur = torch.cuda.current_stream(device)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(cur)
-            s_in.wait_stream(cur)
-            s_out.wait_stream(cur)
-            for j, (r0, r1) in enumerate(bounds):
-                with torch.cuda.stream(s_in):
-                    for k, t in pinned.items():
-                        if t is None:
-                            continue
-                        if k in batched:
-                            d[k][r0:r1].copy_(t[r0:r1], non_blocking=True)
-                        elif j == 0:
-                            d[k].copy_(t, non_blocking=True)
-                    ev_in = torch.cuda.Event()
-                    ev_in.record(s_in)
-                cur.wait_event(ev_in)
-                step_rows(r0, r1)
-                ev_c = torch.cuda.Event()
-                ev_c.record(cur)
-                with torch.cuda.stream(s_out):
-                    s_out.wait_event(ev_c)
-                    y_host[r0:r1].copy_(y[r0:r1], non_blocking=True)
-                    h_host[r0:r1].copy_(h_last[r0:r1], non_blocking=True)
-            cur.wait_stream(s_out)
+            pipelined_host_step(pinned, d, y, h_last, y_host, h_host, step_rows, nb, nch,
+                                streams)
             e1.record(cur)
             e1.synchronize()
             if i >= 2:
