@@ -218,8 +218,16 @@ def cpu_oracle_rate(w, inp, target_s, rng_seed=0, zoh=False):
     n2 = int(max(threads, min(len(all_ch), target_s / max(per_chan, 1e-9) * threads)))
     n2 = max(threads, n2 // threads * threads)
     n, dt = run(n2)
-    value = n * w.seqlen / dt
-    return value, threads, f"{n} of {len(all_ch)} channels x {w.seqlen} steps, {dt:.1f} s"
+    # the whole workload in well under the target: time repeated passes of it
+    passes = 1
+    if n == len(all_ch) and dt < target_s / 2:
+        extra = min(99, int(np.ceil(target_s / max(dt, 1e-9))) - 1)
+        for _ in range(extra):
+            dt += run(n2)[1]
+        passes += extra
+    value = passes * n * w.seqlen / dt
+    rep = f", {passes} passes" if passes > 1 else ""
+    return value, threads, f"{n} of {len(all_ch)} channels x {w.seqlen} steps{rep}, {dt:.1f} s"
 
 
 # Workloads reported beside the bench workload in `per_config` (one GPU).
@@ -609,9 +617,16 @@ def cpu_oracle_bwd_rate(w, inp, grads, target_s, rng_seed=0):
     n2 = int(max(threads, min(len(all_ch), target_s / max(per_chan, 1e-9) * threads)))
     n2 = max(threads, n2 // threads * threads)
     n, dt = run(n2)
-    return (n * w.seqlen / dt, threads,
+    passes = 1
+    if n == len(all_ch) and dt < target_s / 2:
+        extra = min(99, int(np.ceil(target_s / max(dt, 1e-9))) - 1)
+        for _ in range(extra):
+            dt += run(n2)[1]
+        passes += extra
+    rep = f", {passes} passes" if passes > 1 else ""
+    return (passes * n * w.seqlen / dt, threads,
             f"{n} of {len(all_ch)} channels x {w.seqlen} steps (gradients of the listed "
-            f"channels), {dt:.1f} s")
+            f"channels){rep}, {dt:.1f} s")
 
 
 def backward_bench(args):
