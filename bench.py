@@ -423,14 +423,14 @@ def time_decode(w, device, K, warmup):
     def hold(n=1):
         torch.cuda._sleep(200_000 * n)
 
-    def timed(prep):
+    def timed(prep, fn=call):
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(K)]
         for i in range(K):
             prep(i)
             hold()
             ev[i][0].record()
-            call(i)
+            fn(i)
             ev[i][1].record()
         torch.cuda.synchronize()
         return statistics.mean(a.elapsed_time(b) for a, b in ev)
@@ -443,6 +443,12 @@ def time_decode(w, device, K, warmup):
     with sampler:
         cold_ms = timed(lambda i: flush.fill_(i & 0xFF))
     read_ms = timed(lambda i: flush.view(torch.int64).sum())
+    # the stream floor for the state's bytes: torch's device copy of the fp32
+    # state (read once, written once), timed the same way (a library kernel,
+    # outside the decode path)
+    state2 = torch.empty_like(state)
+    copy_ms = timed(lambda i: flush.view(torch.int64).sum(), fn=lambda i: state2.copy_(state))
+    del state2
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     hold(K)  # every call is enqueued before the stream reaches e0
     e0.record()
@@ -471,7 +477,8 @@ def time_decode(w, device, K, warmup):
     graph_ms = g0.elapsed_time(g1) / w.steps
     del g
     return {"w": w, "K": K, "cold_ms": cold_ms, "read_ms": read_ms, "warm_ms": warm_ms,
-            "graph_ms": graph_ms, "clocks": sampler.summary()}
+            "graph_ms": graph_ms, "copy_ms": copy_ms, "state_bytes": state.numel() * 4,
+            "clocks": sampler.summary()}
 
 
 def decode_algorithmic_bytes(w):
@@ -504,7 +511,13 @@ def decode_summary(r):
                          "unit": "GB/s", "frac": round(read_gbs / peak, 4),
                          "algorithmic_bytes_per_launch": algo, "peak_kind": peak_kind},
             "write_flushed_l2": fig(r["cold_ms"]), "warm_l2": fig(r["warm_ms"]),
-            "cuda_graph": dict(fig(r["graph_ms"]), calls=w.steps), "clocks": r["clocks"]}
+            "cuda_graph": dict(fig(r["graph_ms"]), calls=w.steps),
+            "state_copy_read_flushed": {
+                "ms": r["copy_ms"], "bytes": 2 * r["state_bytes"],
+                "gbs": round(2 * r["state_bytes"] / (r["copy_ms"] * 1e-3) / 1e9, 1),
+                "what": "torch device copy of the fp32 state (read and written once), L2 "
+                        "flushed by a 256 MB read: a stream of the state's bytes alone"},
+            "clocks": r["clocks"]}
 
 
 
@@ -564,8 +577,8 @@ def decode_bench(args):
         "data": "synthetic (seeded Philox4x32-10, Mamba-shaped recipe)",
         "config": s["config"], "roofline": s["roofline"],
         "write_flushed_l2": s["write_flushed_l2"], "warm_l2": s["warm_l2"],
-        "cuda_graph": s["cuda_graph"], "gpu_launches": 3 * args.steps + w.steps,
-        "clocks": s["clocks"],
+        "cuda_graph": s["cuda_graph"], "state_copy_read_flushed": s["state_copy_read_flushed"],
+        "gpu_launches": 3 * args.steps + w.steps, "clocks": s["clocks"],
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -1027,14 +1040,14 @@ def ssd_decode_bench(args):
     def hold(n=1):
         torch.cuda._sleep(200_000 * n)
 
-    def timed(prep):
+    def timed(prep, fn=call):
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(K)]
         for i in range(K):
             prep(i)
             hold()
             ev[i][0].record()
-            call(i)
+            fn(i)
             ev[i][1].record()
         torch.cuda.synchronize()
         return statistics.mean(a.elapsed_time(b) for a, b in ev)
@@ -1043,6 +1056,12 @@ def ssd_decode_bench(args):
     with sampler:
         cold_ms = timed(lambda i: flush.fill_(i & 0xFF))
     read_ms = timed(lambda i: flush.view(torch.int64).sum())
+    # the stream floor for the state's bytes: torch's device copy of the fp32
+    # state, timed the same way (a library kernel, outside the decode path)
+    state2 = torch.empty_like(state)
+    copy_cold_ms = timed(lambda i: flush.fill_(i & 0xFF), fn=lambda i: state2.copy_(state))
+    copy_read_ms = timed(lambda i: flush.view(torch.int64).sum(), fn=lambda i: state2.copy_(state))
+    del state2
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     hold(K)  # every call is enqueued before the stream reaches e0
     e0.record()
@@ -1075,7 +1094,12 @@ def ssd_decode_bench(args):
                             "frac": round(algo / (read_ms * 1e-3) / 1e9 / peak, 4)},
         "back_to_back": {"ms_per_step": warm_ms,
                          "algorithmic_gbs": round(algo / (warm_ms * 1e-3) / 1e9, 1)},
-        "gpu_launches": 2 * K, "clocks": sampler.summary(),
+        "state_copy": {
+            "bytes": 2 * state.numel() * 4, "write_flushed_ms": copy_cold_ms,
+            "read_flushed_ms": copy_read_ms,
+            "what": "torch device copy of the fp32 state (read and written once), L2 flushed "
+                    "the same two ways: a stream of the state's bytes alone"},
+        "gpu_launches": 3 * K, "clocks": sampler.summary(),
     }
     print(json.dumps(line), flush=True)
     return 0
