@@ -127,3 +127,25 @@ def test_conv_empty_sequence():
     g = ssm_conv1d_silu_bwd(dev(c["x"]), dev(c["w"]), dev(c["dout"]), dev(c["bias"]))
     assert g["dx"].shape == (2, 0, 64)
     assert torch.count_nonzero(g["dw"]) == 0 and torch.count_nonzero(g["dbias"]) == 0
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("L", [1, 2, 3])
+@pytest.mark.parametrize("dim", [256, 150])
+def test_conv_sequence_shorter_than_the_taps(io, L, dim):
+    """L < width (4): every output sees the zero left padding; the weight
+    gradient of the taps that never meet a token is zero. Vector and element
+    paths."""
+    c = gen.make_conv_inputs(2, L, dim, 4, io, 40 + L)
+    check(c, io, what=f"{io} L={L} dim={dim}")
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_conv_zero_input_run(io):
+    """x = 0 on a run of steps longer than the window (padding tokens): the
+    outputs there are SiLU(bias) exactly, and the gradients flow around it."""
+    c = gen.make_conv_inputs(2, 300, 256, 4, io, 47)
+    x = (gen.bf16_bits_to_f32(c["x"]) if io == "bf16" else c["x"]).copy()
+    x[:, 100:180] = 0.0
+    c["x"] = gen.f32_to_bf16_bits(x) if io == "bf16" else x.astype(np.float32)
+    check(c, io, what=f"{io} zero run")
