@@ -110,3 +110,27 @@ def test_zoh_decode_matches_oracle(io):
         e = rel_err(host(yt), yr)
         assert e <= TOL[io], f"zoh decode {io} step {t}: {e:.3e}"
     assert rel_err(host(state), ref) <= TOL[io]
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("segments", [None, "4"])
+def test_zoh_degenerate_inputs(monkeypatch, io, segments):
+    """The exact-ZOH scan on x = 0 runs across segments (the state only
+    decays), memoryless steps (delta + bias = 60: exp(Delta A) vanishes and the
+    input term is -B x / A), and |h0| ~ 1e3."""
+    if segments:
+        monkeypatch.setenv("SSM_SCAN_SEGMENTS", segments)
+    inp = gen.make_scan_inputs(2, 240, 264, 16, io, 31, with_h0=True)
+    f32 = (lambda a: gen.bf16_bits_to_f32(a)) if io == "bf16" else (lambda a: a)
+    back = (lambda a: gen.f32_to_bf16_bits(a)) if io == "bf16" else (lambda a: a)
+    x = f32(inp["x"]).astype(np.float32).copy()
+    x[:, 40:130, :] = 0.0
+    inp["x"] = back(x)
+    d = f32(inp["delta"]).astype(np.float32).copy()
+    d[:, 180:190, :] = 60.0
+    d[:, ::17, :] = 60.0
+    inp["delta"] = back(d)
+    inp["h0"] = (inp["h0"] * 1e3).astype(np.float32)
+    y, hl = gpu_zoh(inp)
+    yr, hr = oracle_zoh(inp, io)
+    check(host(y), host(hl), yr, hr, io, f"zoh degenerate {io} seg={segments}")
